@@ -1,0 +1,428 @@
+"""Plain CPU oracle for contextualized Learnable Token Eviction (LTE).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The GPU library never
+calls it and shares no code with it.
+
+Everything is computed in float64 with numpy, one (batch element, KV head) unit
+at a time, in the order the method is described.  Inputs given in bf16 or fp32
+are widened exactly to float64 by the caller (``np.asarray(x, np.float64)``).
+
+Sources (web pages; cited by title and figure/section):
+
+* [LTE] "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse
+  Attention and Contextualized Learnable Token Eviction" (He & Garner, 2025),
+  TL;DR, Abstract, and the captions of Figure 2 (eviction scheme: CNN
+  retention score r_{j,h}, attention sink s, sliding window w, decision taken
+  when a KV pair leaves the window, A-plus-column pattern) and Figure 3
+  (inference cache: circular SWA segment plus a capped out-of-window segment
+  holding sink and retained KVs; scoring batched and deferred).
+* [SWA-LA] "Sparse Linear Attention: Viewing SWA from the Perspective of
+  Linear Attention", section "Viewing SWA from the linear-state perspective"
+  (the window as a FIFO of slots, one slot overwritten per token).
+
+Readings taken where the pages are silent (each is restated where used):
+
+* window (t-w, t] holds w keys including the current token;
+* the cap C counts retained tokens only (sinks are extra); when more than C
+  tokens qualify, the C most recent are kept (FIFO ring);
+* retain iff r >= tau; the first s tokens are sinks and are never "retained";
+* CNN: conv1d over the channel concatenation [k; v] (k first), PyTorch
+  cross-correlation convention, per-layer zero padding outside [0, n), a
+  token is scorable only once its whole receptive field exists;
+* softmax scale is a parameter (1/sqrt(D) by default); KV head of query head
+  q is q // (Hq / Hkv).
+
+Parity pins: every function here is checked in ``tests/test_oracle_*.py``
+against something other than itself (library routines on special cases,
+closed forms, brute-force enumeration, an independent simulation).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def sigmoid(x):
+    """Logistic function 1 / (1 + exp(-x)) in float64."""
+    x = _f64(x)
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def silu(x):
+    """SiLU(x) = x * sigmoid(x) in float64."""
+    x = _f64(x)
+    return x * sigmoid(x)
+
+
+# ---------------------------------------------------------------------------
+# (1) retention scores: the per-KV-head CNN  [LTE, TL;DR; Abstract; Fig. 2]
+# ---------------------------------------------------------------------------
+
+@dataclass
+class CNN:
+    """Weights of one two-layer scoring CNN stack for ONE KV head.
+
+    w1 [C1, 2D, K1], b1 [C1], w2 [C1, K2], b2 scalar.  Layer l reads
+    ``past_l`` tokens before and ``K_l - 1 - past_l`` after the output token.
+    """
+    w1: np.ndarray
+    b1: np.ndarray
+    w2: np.ndarray
+    b2: float
+    past1: int
+    past2: int
+
+    @property
+    def future(self) -> int:
+        """F: how many tokens after j the score r_j depends on."""
+        return (self.w1.shape[2] - 1 - self.past1) + (self.w2.shape[1] - 1 - self.past2)
+
+    @property
+    def past(self) -> int:
+        """P: how many tokens before j the score r_j depends on."""
+        return self.past1 + self.past2
+
+
+def _shifted(x: np.ndarray, shift: int) -> np.ndarray:
+    """y[:, j] = x[:, j + shift] where 0 <= j + shift < n, else 0 (zero padding)."""
+    n = x.shape[1]
+    y = np.zeros_like(x)
+    lo, hi = max(0, -shift), min(n, n - shift)
+    if hi > lo:
+        y[:, lo:hi] = x[:, lo + shift:hi + shift]
+    return y
+
+
+def cnn_scores(k, v, cnn: CNN, n_avail: int | None = None) -> np.ndarray:
+    """Retention scores r_j of one (batch element, KV head) unit.
+
+    [LTE, Fig. 2]: a CNN stack reads short-range past and future context of
+    each KV pair and outputs a per-token, per-head retention score; the score
+    can be computed once the CNN receptive field is available.
+
+    Layer 1: u[c, j] = SiLU(b1[c] + sum_ch sum_kk w1[c, ch, kk] * x[ch, j+kk-past1])
+    Layer 2: r[j]    = sigmoid(b2 + sum_c sum_kk w2[c, kk] * u[c, j+kk-past2])
+    with x = [k; v] (channels 0..D-1 from k, D..2D-1 from v), and each layer's
+    input taken as 0 outside [0, n_avail).
+
+    k, v: [n, D] (any float dtype).  Returns r [n] float64; tokens whose
+    receptive field reaches past n_avail - 1 are not yet scorable and get NaN.
+    """
+    k = _f64(k)
+    v = _f64(v)
+    n = k.shape[0] if n_avail is None else int(n_avail)
+    x = np.concatenate([k[:n], v[:n]], axis=1).T            # [2D, n]
+    c1, two_d, k1 = cnn.w1.shape
+    assert two_d == x.shape[0]
+    u = np.zeros((c1, n))
+    for kk in range(k1):
+        u += _f64(cnn.w1[:, :, kk]) @ _shifted(x, kk - cnn.past1)
+    u = silu(u + _f64(cnn.b1)[:, None])
+    z = np.full(n, float(cnn.b2))
+    for kk in range(cnn.w2.shape[1]):
+        z += _f64(cnn.w2[:, kk]) @ _shifted(u, kk - cnn.past2)
+    r = sigmoid(z)
+    last = n - 1 - cnn.future                                 # last scorable token
+    r[max(0, last + 1):] = np.nan
+    return r
+
+
+# ---------------------------------------------------------------------------
+# (2) eviction decision and compaction  [LTE, Fig. 2 and Fig. 3]
+# ---------------------------------------------------------------------------
+
+def retention_mask(r, sink: int, tau: float) -> np.ndarray:
+    """m_j = (j >= s) and (r_j >= tau); unscored tokens (NaN) get 0.
+
+    [LTE, Fig. 2]: r_{j,h} decides whether the KV pair is evicted when it
+    moves out of the window; sinks are kept regardless, so they are never
+    counted as retained.
+    """
+    r = _f64(r)
+    m = np.zeros(r.shape[0], dtype=np.uint8)
+    for j in range(r.shape[0]):
+        if j >= sink and not math.isnan(r[j]) and r[j] >= tau:
+            m[j] = 1
+    return m
+
+
+def fed_mask(mask, sink: int) -> np.ndarray:
+    """A retention mask given directly (attention isolated from scoring), with
+    the sink positions forced to 0 because sinks are never 'retained'."""
+    m = np.asarray(mask, dtype=np.uint8).copy()
+    m[:sink] = 0
+    return m
+
+
+def compact(m) -> tuple[np.ndarray, int, np.ndarray]:
+    """Ascending list of retained positions, its length, and inclusive
+    prefix counts cnt[j] = #{i <= j : m_i = 1}.  Plain definition."""
+    m = np.asarray(m, dtype=np.int64)
+    idx = [j for j in range(m.shape[0]) if m[j]]
+    cnt = np.zeros(m.shape[0], dtype=np.int64)
+    running = 0
+    for j in range(m.shape[0]):
+        running += int(m[j])
+        cnt[j] = running
+    return np.array(idx, dtype=np.int64), len(idx), cnt
+
+
+# ---------------------------------------------------------------------------
+# (3) attended set and attention  [LTE, Fig. 2 right: A-plus-column pattern]
+# ---------------------------------------------------------------------------
+
+def attended_set(t: int, m, sink: int, window: int, cap: int) -> list[int]:
+    """Key positions query t attends to, for one KV head.
+
+    S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t,
+    Ret_t = the `cap` largest j in [s, t-w] with m_j = 1 (the C most recent
+    tokens that were kept when they left the window).
+    """
+    keys = set(range(0, min(sink, t + 1)))
+    keys |= set(range(max(0, t - window + 1), t + 1))
+    candidates = [j for j in range(sink, t - window + 1) if m[j]]
+    if cap > 0:
+        keys |= set(candidates[-cap:])
+    return sorted(keys)
+
+
+def attend(q_rows, K, V, scale: float):
+    """Softmax attention of the rows of q over keys K / values V (float64).
+
+    q_rows [G, D], K [n, D], V [n, Dv] -> (o [G, Dv], lse [G]) where
+    lse = log sum_j exp(scale * q . k_j).  Max-subtracted for range safety.
+    """
+    q_rows, K, V = _f64(q_rows), _f64(K), _f64(V)
+    logits = scale * (q_rows @ K.T)                           # [G, n]
+    mx = logits.max(axis=1, keepdims=True)
+    p = np.exp(logits - mx)
+    l = p.sum(axis=1, keepdims=True)
+    o = (p @ V) / l
+    lse = (mx + np.log(l))[:, 0]
+    return o, lse
+
+
+def prefill_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
+                 rows=None):
+    """Prefill of one (batch element, KV head) unit.
+
+    q [T, G, D] (the G query heads that share this KV head), k, v [T, D],
+    m [T] retention mask.  Returns o [T, G, D], lse [T, G] and the attended
+    count per row (rows not in `rows` are left as NaN / -1).
+    """
+    T, G, D = q.shape
+    o = np.full((T, G, v.shape[1]), np.nan)
+    lse = np.full((T, G), np.nan)
+    count = np.full(T, -1, dtype=np.int64)
+    k = _f64(k)
+    v = _f64(v)
+    for t in (range(T) if rows is None else rows):
+        S = attended_set(t, m, sink, window, cap)
+        o[t], lse[t] = attend(q[t], k[S], v[S], scale)
+        count[t] = len(S)
+    return o, lse, count
+
+
+def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | None = None):
+    """Prefill over a batch: q [B,T,Hq,D], k, v [B,T,Hkv,D], masks [B,Hkv,T].
+
+    GQA: query head qh uses KV head qh // (Hq // Hkv).  Returns o [B,T,Hq,D],
+    lse [B,Hq,T], count [B,Hkv,T].
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    o = np.zeros((B, T, Hq, v.shape[3]))
+    lse = np.zeros((B, Hq, T))
+    count = np.zeros((B, Hkv, T), dtype=np.int64)
+    for b in range(B):
+        for h in range(Hkv):
+            ou, lu, cu = prefill_unit(q[b, :, h * G:(h + 1) * G], k[b, :, h], v[b, :, h],
+                                      masks[b, h], sink, window, cap, scale)
+            o[b, :, h * G:(h + 1) * G] = ou
+            lse[b, h * G:(h + 1) * G] = lu.T
+            count[b, h] = cu
+    return o, lse, count
+
+
+# ---------------------------------------------------------------------------
+# (4) decode: the inference cache simulated slot by slot  [LTE, Fig. 3]
+#     window as a FIFO of w slots  [SWA-LA, "Viewing SWA from the
+#     linear-state perspective": one slot overwritten per token]
+# ---------------------------------------------------------------------------
+
+@dataclass
+class DecodeCache:
+    """Inference cache of one (batch element, KV head) unit, held literally.
+
+    * window ring: w slots, token j lives in slot j mod w while in (t-w, t];
+    * sink slots: s slots, token j < s moves to slot j when it leaves the window;
+    * retained ring: C slots, the i-th retained token (0-based) goes to slot
+      i mod C, overwriting the oldest one (the cap keeps the C most recent);
+    * r of window tokens, filled by deferred batched scoring.
+    """
+    D: int
+    sink: int
+    window: int
+    cap: int
+    tau: float
+    cnn: CNN | None
+    score_batch: int
+    win_k: np.ndarray = field(init=False)
+    win_v: np.ndarray = field(init=False)
+    win_pos: np.ndarray = field(init=False)
+    win_r: np.ndarray = field(init=False)
+    sink_k: np.ndarray = field(init=False)
+    sink_v: np.ndarray = field(init=False)
+    sink_pos: np.ndarray = field(init=False)
+    ret_k: np.ndarray = field(init=False)
+    ret_v: np.ndarray = field(init=False)
+    ret_pos: np.ndarray = field(init=False)
+    ret_total: int = 0
+    t: int = 0              # tokens received so far
+    n_scored: int = 0       # tokens [0, n_scored) have a score
+    fed: np.ndarray | None = None   # optional fed mask instead of the CNN
+
+    def __post_init__(self):
+        w, s, C, D = self.window, self.sink, self.cap, self.D
+        self.win_k = np.zeros((w, D)); self.win_v = np.zeros((w, D))
+        self.win_pos = np.full(w, -1, dtype=np.int64); self.win_r = np.full(w, np.nan)
+        self.sink_k = np.zeros((s, D)); self.sink_v = np.zeros((s, D))
+        self.sink_pos = np.full(s, -1, dtype=np.int64)
+        self.ret_k = np.zeros((C, D)); self.ret_v = np.zeros((C, D))
+        self.ret_pos = np.full(C, -1, dtype=np.int64)
+
+    # -- deferred scoring ---------------------------------------------------
+    def _score_from_window(self, j: int) -> float:
+        """r_j computed from the window ring alone; asserts that the whole
+        receptive field [j-P, j+F] (clipped at 0) is inside the window."""
+        if self.fed is not None:
+            return 1.0 if self.fed[j] else 0.0
+        P, F = self.cnn.past, self.cnn.future
+        lo = max(0, j - P)            # positions before 0 do not exist (padding)
+        n = j + F + 1 - lo
+        ks = np.zeros((n, self.D)); vs = np.zeros((n, self.D))
+        for i in range(lo, j + F + 1):
+            slot = i % self.window
+            assert self.win_pos[slot] == i, "receptive field left the window before scoring"
+            ks[i - lo] = self.win_k[slot]
+            vs[i - lo] = self.win_v[slot]
+        r = cnn_scores(ks, vs, self.cnn)
+        return float(r[j - lo])
+
+    def _maybe_score(self):
+        """Score the oldest `score_batch` scorable tokens once that many are
+        scorable (a token j is scorable when j + F < t)."""
+        F = 0 if self.cnn is None else self.cnn.future
+        last_scorable = self.t - 1 - F
+        while last_scorable - self.n_scored + 1 >= self.score_batch:
+            for j in range(self.n_scored, self.n_scored + self.score_batch):
+                self.win_r[j % self.window] = self._score_from_window(j)
+            self.n_scored += self.score_batch
+
+    # -- one token arrives ----------------------------------------------------
+    def append(self, k_t, v_t):
+        """Token t = self.t arrives: token t-w leaves the window first."""
+        t, w = self.t, self.window
+        leaving = t - w
+        if leaving >= 0:
+            slot = leaving % w
+            assert self.win_pos[slot] == leaving
+            if leaving < self.sink:
+                self.sink_k[leaving] = self.win_k[slot]
+                self.sink_v[leaving] = self.win_v[slot]
+                self.sink_pos[leaving] = leaving
+            else:
+                assert leaving < self.n_scored, "token left the window unscored"
+                r = self.win_r[slot]
+                if r >= self.tau and self.cap > 0:
+                    rs = self.ret_total % self.cap
+                    self.ret_k[rs] = self.win_k[slot]
+                    self.ret_v[rs] = self.win_v[slot]
+                    self.ret_pos[rs] = leaving
+                    self.ret_total += 1
+        slot = t % w
+        self.win_k[slot] = _f64(k_t); self.win_v[slot] = _f64(v_t)
+        self.win_pos[slot] = t; self.win_r[slot] = np.nan
+        self.t = t + 1
+        self._maybe_score()
+
+    def retained_positions(self) -> list[int]:
+        return sorted(int(p) for p in self.ret_pos if p >= 0)
+
+    def keys(self):
+        """All valid (position, k, v) of the cache, position-sorted."""
+        items = []
+        for i in range(self.window):
+            if self.win_pos[i] >= 0:
+                items.append((int(self.win_pos[i]), self.win_k[i], self.win_v[i]))
+        for i in range(self.sink):
+            if self.sink_pos[i] >= 0:
+                items.append((int(self.sink_pos[i]), self.sink_k[i], self.sink_v[i]))
+        for i in range(self.cap):
+            if self.ret_pos[i] >= 0:
+                items.append((int(self.ret_pos[i]), self.ret_k[i], self.ret_v[i]))
+        items.sort(key=lambda it: it[0])
+        return items
+
+    def attend(self, q_rows, scale: float):
+        """Attention of the newest token's G query rows over the cache."""
+        items = self.keys()
+        K = np.stack([it[1] for it in items])
+        V = np.stack([it[2] for it in items])
+        o, lse = attend(q_rows, K, V, scale)
+        return o, lse, [it[0] for it in items]
+
+
+def decode_unit(q, k, v, T0: int, sink: int, window: int, cap: int, tau: float,
+                cnn: CNN | None, score_batch: int, scale: float, fed=None):
+    """Feed tokens 0..T-1 of one unit through the cache; for every token
+    t >= T0 return its attention output, lse and attended positions.
+
+    q [T, G, D], k, v [T, D].  The prompt (t < T0) goes through the same
+    cache updates as decoding (no attention output is kept for it).
+    """
+    cache = DecodeCache(D=k.shape[1], sink=sink, window=window, cap=cap, tau=tau,
+                        cnn=cnn, score_batch=score_batch)
+    cache.fed = None if fed is None else np.asarray(fed)
+    outs, lses, sets, rets = [], [], [], []
+    for t in range(k.shape[0]):
+        cache.append(k[t], v[t])
+        if t >= T0:
+            o, lse, pos = cache.attend(q[t], scale)
+            outs.append(o); lses.append(lse); sets.append(pos)
+            rets.append(cache.retained_positions())
+    return np.array(outs), np.array(lses), sets, rets, cache
+
+
+def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int):
+    """The cache contents after a prompt of T0 tokens, read off the prefill
+    mask: window = positions (T0-1-w, T0-1], sinks = j < s with j <= T0-1-w,
+    retained = the C most recent j in [s, T0-1-w] with m_j = 1, with the
+    i-th retained token (0-based over all retained) in ring slot i mod C.
+
+    Returns dict of position arrays (-1 = empty) and ret_total.
+    """
+    last_out = T0 - 1 - window
+    win_pos = np.full(window, -1, dtype=np.int64)
+    for j in range(max(0, T0 - window), T0):
+        win_pos[j % window] = j
+    sink_pos = np.full(sink, -1, dtype=np.int64)
+    for j in range(min(sink, last_out + 1)):
+        sink_pos[j] = j
+    ret = [j for j in range(sink, last_out + 1) if m[j]]
+    ret_pos = np.full(cap, -1, dtype=np.int64)
+    for i, j in enumerate(ret):
+        if cap > 0:
+            ret_pos[i % cap] = j
+    return {"win_pos": win_pos, "sink_pos": sink_pos, "ret_pos": ret_pos,
+            "ret_total": len(ret)}

@@ -1,0 +1,100 @@
+"""Pins for the oracle's eviction, compaction and attended sets (no GPU).
+
+The oracle states S_t as a union of sink, window and the C most recent
+retained tokens.  Here it is checked against a differently phrased
+membership rule (a token j <= t-w survives iff fewer than C retained tokens
+left the window after it), against closed forms for the degenerate settings,
+and against numpy's cumsum for the prefix counts.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import lte_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def brute_member(j, t, m, s, w, C):
+    if j > t or j < 0:
+        return False
+    if j < s or j > t - w:
+        return True
+    if not m[j]:
+        return False
+    newer = sum(1 for i in range(j + 1, t - w + 1) if i >= s and m[i])
+    return newer < C
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_attended_set_vs_bruteforce(seed):
+    rng = np.random.default_rng(seed)
+    for _ in range(25):
+        T = int(rng.integers(1, 48))
+        s = int(rng.integers(0, 5))
+        w = int(rng.integers(1, 14))
+        C = int(rng.choice([0, 1, 2, 3, 8, 100]))
+        p = float(rng.choice([0.0, 0.3, 0.7, 1.0]))
+        m = O.fed_mask((rng.random(T) < p).astype(np.uint8), s)
+        for t in range(T):
+            S = O.attended_set(t, m, s, w, C)
+            ref = [j for j in range(T) if brute_member(j, t, m, s, w, C)]
+            assert S == ref, (T, s, w, C, t)
+
+
+def test_closed_forms():
+    rng = np.random.default_rng(11)
+    T, s, w = 200, 4, 16
+    m_rand = O.fed_mask((rng.random(T) < 0.4).astype(np.uint8), s)
+    zeros = np.zeros(T, np.uint8)
+    ones = O.fed_mask(np.ones(T, np.uint8), s)
+    for t in range(T):
+        # w >= T: full causal attention
+        assert len(O.attended_set(t, m_rand, s, T, 7)) == t + 1
+        # r == 0: sink + window
+        n0 = min(t + 1, w) + len([j for j in range(s) if j <= t - w])
+        assert len(O.attended_set(t, zeros, s, w, 50)) == n0
+        # C == 0: sink + window for any r
+        assert len(O.attended_set(t, m_rand, s, w, 0)) == n0
+        # r == 1 with C >= T: full causal attention
+        assert O.attended_set(t, ones, s, w, T) == list(range(t + 1))
+        # with the cap binding, exactly min(C, #retained) extra keys
+        nret = int(sum(ones[s:max(s, t - w + 1)]))
+        assert len(O.attended_set(t, ones, s, w, 10)) == n0 + min(10, nret)
+
+
+def test_compact_vs_cumsum():
+    rng = np.random.default_rng(2)
+    m = (rng.random(300) < 0.2).astype(np.uint8)
+    idx, n, cnt = O.compact(m)
+    assert n == int(m.sum())
+    np.testing.assert_array_equal(idx, np.flatnonzero(m))
+    np.testing.assert_array_equal(cnt, np.cumsum(m))
+
+
+def test_prefill_count_formula():
+    """Row count from the compaction arrays (the form a kernel uses):
+    |S_t| = min(t+1,w) + #sinks out of window + min(C, cnt[t-w])."""
+    rng = np.random.default_rng(4)
+    T, s, w, C = 300, 4, 32, 9
+    m = O.fed_mask((rng.random(T) < 0.3).astype(np.uint8), s)
+    _, _, cnt = O.compact(m)
+    for t in range(T):
+        n = cnt[t - w] if t - w >= 0 else 0
+        expect = min(t + 1, w) + len([j for j in range(s) if j <= t - w]) + min(C, n)
+        assert len(O.attended_set(t, m, s, w, C)) == expect
+
+
+def test_golden_fig2_setting():
+    """Fig. 2 of the LTE paper draws s=2, w=12; the fixture holds a mask and
+    the attended sets for that setting, written by tests/golden/make_golden.py
+    from the oracle and checked here against the brute-force rule too."""
+    with open(os.path.join(GOLDEN, "fig2_sets.json")) as f:
+        gold = json.load(f)
+    s, w, C = gold["sink"], gold["window"], gold["cap"]
+    m = np.array(gold["mask"], np.uint8)
+    for t, S in enumerate(gold["sets"]):
+        assert O.attended_set(t, m, s, w, C) == S
+        assert S == [j for j in range(len(m)) if brute_member(j, t, m, s, w, C)]
