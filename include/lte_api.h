@@ -1,0 +1,249 @@
+/*
+ * lte_api.h -- C ABI of the B200 (sm_100a) library for contextualized
+ * Learnable Token Eviction (LTE), the sparse-attention token mixer of the
+ * laLTE linear/sparse hybrid.
+ *
+ * Source of the method: "Alleviating Forgetfulness of Linear Attention by
+ * Hybrid Sparse Attention and Contextualized Learnable Token Eviction"
+ * (He & Garner, 2025): TL;DR and Abstract (a lightweight CNN over past and
+ * future neighbouring KVs predicts per-head retention; combined with an
+ * attention sink and sliding-window attention; constant time and space per
+ * step), Figure 2 caption (retention score r_{j,h} decides eviction when a
+ * KV pair leaves the window; the score can be computed once the CNN's
+ * receptive field is inside the window; per-head "A-plus-column" pattern),
+ * Figure 3 caption (inference cache = circular window segment + capped
+ * out-of-window segment holding sink and retained KVs; scoring batched and
+ * deferred).  The companion linear layer follows "Sparse Linear Attention:
+ * Viewing SWA from the Perspective of Linear Attention", section
+ * "Background: Linear attention" (state update equation).
+ *
+ * Conventions for every call
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the
+ *    library allocates no memory (scratch comes in `workspace`, sized by
+ *    lte_workspace_bytes) and synchronises nothing except
+ *    lte_read_device_error.  Every call enqueues its kernels on `stream`
+ *    (a cudaStream_t passed as void*; NULL = legacy default stream) and
+ *    returns immediately.
+ *  - Layouts are row-major.  Activations are [B, T, H, D] with the D
+ *    dimension contiguous; `lte_strides` gives the other three element
+ *    strides (NULL = contiguous).  Pointers must be 16-byte aligned and
+ *    strides multiples of 16 bytes.
+ *  - Notation: B batch, T tokens, Hq query heads, Hkv KV heads, G = Hq/Hkv,
+ *    D head dim, s sink, w window, C cap, tau threshold.  Query head q uses
+ *    KV head q / G.
+ *  - Errors: arguments are validated on the host before any launch; an
+ *    invalid call returns a non-zero lte_status and launches nothing.  A
+ *    failed launch returns LTE_ERR_CUDA.  Conditions only the device can see
+ *    (a bounded wait that ran out, an index out of range) are recorded in
+ *    the first 16 bytes of the workspace and read by lte_read_device_error.
+ *    Nothing aborts the process.
+ */
+#ifndef LTE_API_H
+#define LTE_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LTE_OK = 0,
+  LTE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or parameter */
+  LTE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. D not in {64,128}) */
+  LTE_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+  LTE_ERR_TIMEOUT = 4,       /* a device-side bounded wait ran out */
+  LTE_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required */
+  LTE_ERR_DEVICE = 6         /* a device-side check failed (see error word) */
+} lte_status;
+
+typedef enum { LTE_F32 = 0, LTE_BF16 = 1 } lte_dtype;
+
+/* Shapes and method parameters of one LTE layer.
+ * sink = s >= 0, window = w >= 1, cap = C >= 0 (retained tokens only; sinks
+ * are extra), tau = retention threshold (retain iff r >= tau), scale =
+ * softmax scale (1/sqrt(D) in the usual setting), dtype of q/k/v/o/caches. */
+typedef struct {
+  int32_t B, T, Hq, Hkv, D;
+  int32_t sink, window, cap;
+  float tau, scale;
+  int32_t dtype;
+} lte_dims;
+
+/* Element strides of a [B, T, H, D] tensor (D stride is 1). */
+typedef struct { int64_t b, t, h; } lte_strides;
+
+/* Weights of the per-KV-head scoring CNN (device pointers, fp32):
+ *   w1 [Hkv, c_hid, 2D, k1], b1 [Hkv, c_hid], w2 [Hkv, c_hid, k2], b2 [Hkv].
+ * Layer l reads past_l tokens before and (k_l - 1 - past_l) after the output
+ * token (PyTorch conv1d cross-correlation, zero padding outside the
+ * sequence); input channels are [k; v] (k first).  r_j depends on tokens
+ * [j - P, j + F] with P = past1 + past2, F = (k1-1-past1) + (k2-1-past2).
+ * Supported: c_hid <= 64, k1 <= 9, k2 <= 9. */
+typedef struct {
+  int32_t c_hid, k1, past1, k2, past2;
+  const float *w1, *b1, *w2, *b2;
+} lte_cnn;
+
+/* ---------------------------------------------------------------------------
+ * lte_score -- retention scores r_{j,h} of tokens j in [j_begin, j_end).
+ * [LTE paper, Fig. 2 caption: CNN stack over short-range past and future
+ * context; TL;DR: per-head retention scores.]
+ *   layer 1: u[c,j] = SiLU(b1[c] + sum_{ch<2D, kk<k1} w1[c,ch,kk] x[ch, j+kk-past1])
+ *   layer 2: r[j]   = sigmoid(b2 + sum_{c, kk<k2} w2[c,kk] u[c, j+kk-past2])
+ * k, v: [B,T,Hkv,D] (dtype), kv_strides may be NULL.  Requires
+ * 0 <= j_begin <= j_end <= T - F (the receptive field must be complete).
+ * r: fp32 [B, Hkv, T]; mask (nullable): uint8 [B, Hkv, T], written as
+ * (j >= sink) && (r >= tau).  Only positions [j_begin, j_end) are written.
+ * Arithmetic: fp32 accumulation in a fixed per-output order (results do not
+ * depend on j_begin/j_end or on the launch).
+ * ------------------------------------------------------------------------- */
+lte_status lte_score(const lte_dims* d, const lte_cnn* cnn,
+                     const void* k, const void* v, const lte_strides* kv_strides,
+                     int32_t j_begin, int32_t j_end,
+                     float* r, uint8_t* mask, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lte_evict_compact -- eviction decision and compaction of retained tokens.
+ * [LTE paper, Fig. 2 caption: a KV pair is kept or evicted when it moves out
+ * of the window; Fig. 3 caption: capped out-of-window segment with sink and
+ * retained KVs.]
+ * m_j = (j >= sink) && (j < n_scored) && (mask ? mask[j] != 0 : r[j] >= tau);
+ * exactly one of r / mask is non-NULL ([B,Hkv,T]).
+ * Outputs (per (b, KV head) unit):
+ *   idx  int32 [B,Hkv,T]: ascending positions j with m_j = 1 (first nret valid),
+ *   nret int32 [B,Hkv]:   number of such positions,
+ *   cnt  int32 [B,Hkv,T]: inclusive prefix count cnt[j] = #{i <= j : m_i}.
+ * Column segment (k_col, v_col both NULL or both set): [B, Hkv, sink + T, D]
+ * contiguous, slot i < sink holds the sink row k[i] (rows i >= T left
+ * unwritten), slot sink + i holds k[idx[i]] for i < nret; likewise for v.
+ * ------------------------------------------------------------------------- */
+lte_status lte_evict_compact(const lte_dims* d, const float* r, const uint8_t* mask,
+                             int32_t n_scored, int32_t* idx, int32_t* nret, int32_t* cnt,
+                             const void* k, const void* v, const lte_strides* kv_strides,
+                             void* k_col, void* v_col, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lte_sparse_attn_prefill -- causal softmax attention of every query over its
+ * per-KV-head attended set.  [LTE paper, Fig. 2 caption (right): per-head
+ * A-plus-column sparsity pattern: sink and window form the "A", retained
+ * tokens the "columns".]
+ * For row t, KV head h, n_t = (t >= w) ? cnt[t - w] : 0:
+ *   S_t = { j < s : j <= t - w }  u  (t - w, t]  u  { idx[i] : max(0, n_t - C) <= i < n_t }
+ *   o[t,q] = sum_{j in S_t} softmax_j(scale * q_t . k_j) v_j,
+ *   lse[q,t] = log sum_{j in S_t} exp(scale * q_t . k_j)   (natural log).
+ * q, o: [B,T,Hq,D]; k, v: [B,T,Hkv,D]; cnt from lte_evict_compact; k_col,
+ * v_col: the column segment written by lte_evict_compact (required).
+ * lse (nullable): fp32 [B,Hq,T].  bf16 inputs: fp32 accumulation, P rounded
+ * to bf16 for the PV product, o rounded to bf16 (round-to-nearest-even).
+ * Workspace: lte_workspace_bytes(d, LTE_WS_PREFILL) bytes (16-byte aligned,
+ * caller-owned; it holds the device error word).
+ * ------------------------------------------------------------------------- */
+lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void* k,
+                                   const void* v, const lte_strides* q_strides,
+                                   const lte_strides* kv_strides, const int32_t* cnt,
+                                   const void* k_col, const void* v_col,
+                                   void* o, const lte_strides* o_strides, float* lse,
+                                   void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Decode cache.  [LTE paper, Fig. 3 caption: circular window segment plus an
+ * out-of-window segment of capped capacity for sink and retained KVs;
+ * "Sparse Linear Attention ...", section "Viewing SWA from the linear-state
+ * perspective": the window as a FIFO of slots.]
+ * All buffers are caller-owned device memory; L = window + sink + cap slots.
+ *   k, v     [B, Hkv, L, D] (dtype): slots [0,w) window ring (token j in slot
+ *            j mod w), [w, w+s) sinks (token j < s in slot w+j once it left
+ *            the window), [w+s, w+s+C) retained ring (the i-th retained token
+ *            of the unit, 0-based, in slot w+s+(i mod C));
+ *   pos      int32 [B, Hkv, L]: token position held by each slot, -1 = empty;
+ *   win_r    fp32  [B, Hkv, w]: score of the token in each window slot;
+ *   ret_total int32 [B, Hkv]: tokens retained so far (the ring's write count);
+ *   meta     int32 [4]: {t = tokens held so far, n_scored = tokens [0,n_scored)
+ *            have a score, internal, internal}. */
+typedef struct {
+  void *k, *v;
+  int32_t* pos;
+  float* win_r;
+  int32_t* ret_total;
+  int32_t* meta;
+} lte_cache;
+
+/* lte_cache_init_from_prefill -- fill an empty cache with the state after a
+ * prompt of T_prompt tokens (T_prompt <= d->T):
+ * window = tokens (T_prompt-1-w, T_prompt-1], sinks that left the window,
+ * retained = idx[max(0,n-C) .. n) with n = cnt[T_prompt-1-w] (0 if negative),
+ * win_r = r of window tokens below n_scored (NaN otherwise),
+ * ret_total = n, meta = {T_prompt, n_scored, 0, 0}.
+ * k, v [B,T,Hkv,D]; r [B,Hkv,T] from lte_score; idx, cnt from
+ * lte_evict_compact run with the same n_scored. */
+lte_status lte_cache_init_from_prefill(const lte_dims* d, const lte_cache* cache,
+                                       const void* k, const void* v,
+                                       const lte_strides* kv_strides, const float* r,
+                                       const int32_t* idx, const int32_t* cnt,
+                                       int32_t T_prompt, int32_t n_scored, void* stream);
+
+/* lte_decode_step -- one generated token for every sequence in the batch.
+ * Reads t = meta[0] on the device (no host synchronisation), then:
+ *  (1) token t-w leaves the window: a sink (t-w < s) moves to its sink slot;
+ *      otherwise it enters the retained ring iff win_r >= tau and C > 0
+ *      (overwriting the oldest when the ring is full), else it is dropped;
+ *  (2) the new token is written to window slot t mod w;
+ *  (3) deferred batched scoring: once score_batch tokens are scorable
+ *      (j + F <= t), the oldest score_batch unscored tokens are scored from
+ *      the window segment (same arithmetic as lte_score);
+ *  (4) attention of q_t over every valid slot (split over the keys, merged
+ *      with log-sum-exp), o_t and lse_t written;  meta[0] = t + 1.
+ * q_t, o_t: [B, Hq, D]; k_t, v_t: [B, Hkv, D]; lse_t (nullable) fp32 [B, Hq].
+ * Requires 1 <= score_batch <= w - P - F (every token is scored before it
+ * leaves the window).  Workspace: lte_workspace_bytes(d, LTE_WS_DECODE).
+ * The same kernels run every step, so a step can be captured in a CUDA graph
+ * and replayed. */
+lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* cache,
+                           const void* q_t, const void* k_t, const void* v_t,
+                           void* o_t, float* lse_t, int32_t score_batch,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1 };
+
+/* Bytes of workspace a call needs (>= 16: the first 16 bytes hold the device
+ * error word).  Returns 0 for invalid dims. */
+size_t lte_workspace_bytes(const lte_dims* d, int32_t which);
+
+/* Zero the error word of a workspace (enqueued on stream). */
+lte_status lte_clear_device_error(void* workspace, void* stream);
+
+/* Synchronise `stream`, then copy the workspace's error word to the host:
+ * *code = 0 if no device-side check failed, else LTE_ERR_TIMEOUT or
+ * LTE_ERR_DEVICE; *where = the id of the wait or check that failed. */
+lte_status lte_read_device_error(const void* workspace, int32_t* code, int32_t* where,
+                                 void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Gated linear attention, the hybrid's companion layer.  ["Sparse Linear
+ * Attention: Viewing SWA from the Perspective of Linear Attention", section
+ * "Background: Linear attention": the state is decayed, the value-key outer
+ * product is written, the query reads; the decay here is diag(a_t).]
+ *   S_t = S_{t-1} diag(a_t) + v_t k_t^T,  o_t = S_t q_t.
+ * q, k: [B,T,H,dk]; v, o: [B,T,H,dv] (dtype); a: fp32 [B,T,H,dk] in (0,1];
+ * state: fp32 [B,H,dv,dk], read as S_0 and overwritten with S_T.
+ * Supported: dk = dv = 128 (bf16) or dk, dv <= 128 (fp32); T % 64 == 0 for
+ * bf16 prefill.  Prefill is chunk-wise (64 tokens); decode is one step.
+ * ------------------------------------------------------------------------- */
+lte_status lte_gla_prefill(int32_t B, int32_t T, int32_t H, int32_t dk, int32_t dv,
+                           int32_t dtype, const void* q, const void* k, const void* v,
+                           const float* a, void* o, float* state, void* stream);
+
+lte_status lte_gla_decode_step(int32_t B, int32_t H, int32_t dk, int32_t dv, int32_t dtype,
+                               const void* q_t, const void* k_t, const void* v_t,
+                               const float* a_t, void* o_t, float* state, void* stream);
+
+/* Library version string (static storage). */
+const char* lte_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LTE_API_H */

@@ -1,0 +1,178 @@
+// Eviction decision, compaction of retained tokens, and decode-cache set-up.
+//
+// "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention
+// and Contextualized Learnable Token Eviction": Fig. 2 caption (r_{j,h}
+// decides whether a KV pair is evicted when it moves out of the sliding
+// window; the attention sink is always kept) and Fig. 3 caption (the
+// out-of-window cache segment has capped capacity and holds the sink and the
+// LTE-retained KVs).
+//
+// compact_kernel: one CTA per (batch, KV head) unit walks the tokens in
+// rounds of one thread per token.  A warp ballot gives each retained token
+// its rank inside the warp, a 32-entry scan over warp totals gives the warp
+// offsets, and a running carry links the rounds.  This yields the ascending
+// retained-position list idx, its length, and the inclusive prefix counts
+// cnt.  The same CTA then copies the sink rows and the retained rows into a
+// contiguous column segment with 16-byte vector loads, so the attention
+// kernels read the "column" keys as dense tiles.
+#include <math.h>
+
+#include "lte_common.cuh"
+#include "lte_internal.h"
+
+namespace lte {
+
+constexpr int kCompactThreads = 1024;
+
+__device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                         int nvec, int lane_in_row) {
+  if (lane_in_row < nvec) dst[lane_in_row] = src[lane_in_row];
+}
+
+__global__ void __launch_bounds__(kCompactThreads)
+compact_kernel(int T, int Hkv, int sink, int n_scored, float tau, const float* __restrict__ r,
+               const uint8_t* __restrict__ mask, int32_t* __restrict__ idx,
+               int32_t* __restrict__ nret, int32_t* __restrict__ cnt, const char* __restrict__ k,
+               const char* __restrict__ v, Strides4 s, int elt, int D, char* __restrict__ k_col,
+               char* __restrict__ v_col) {
+  __shared__ int warp_tot[32];
+  __shared__ int warp_off[32];
+  __shared__ int round_total;
+  const int u = blockIdx.x, b = u / Hkv, h = u % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long row0 = (long long)u * T;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  int carry = 0;
+  for (int base = 0; base < T; base += kCompactThreads) {
+    const int j = base + tid;
+    bool m = false;
+    if (j < T && j >= sink && j < n_scored)
+      m = mask ? (mask[row0 + j] != 0) : (r[row0 + j] >= tau);
+    const unsigned ballot = __ballot_sync(0xffffffffu, m);
+    if (lane == 0) warp_tot[warp] = __popc(ballot);
+    __syncthreads();
+    if (warp == 0) {
+      const int x = warp_tot[lane];
+      int incl = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      warp_off[lane] = incl - x;
+      if (lane == 31) round_total = incl;
+    }
+    __syncthreads();
+    const int pos = carry + warp_off[warp] + __popc(ballot & lt_mask);
+    if (m) idx[row0 + pos] = j;
+    if (j < T) cnt[row0 + j] = pos + (m ? 1 : 0);
+    carry += round_total;
+    __syncthreads();
+  }
+  if (tid == 0) nret[u] = carry;
+  if (k_col == nullptr) return;
+  __syncthreads();   // idx written above is visible to the whole CTA
+
+  // column segment: slot i < sink <- row i; slot sink + i <- row idx[i]
+  const int nvec = D * elt / 16;
+  const int rows_per_pass = kCompactThreads / nvec;
+  const int rr = tid / nvec, lane_in_row = tid % nvec;
+  const int nsink = sink < T ? sink : T;
+  const int total = nsink + carry;
+  const long long col0 = (long long)u * (sink + T);
+  for (int i = rr; i < total; i += rows_per_pass) {
+    const int j = (i < nsink) ? i : idx[row0 + (i - nsink)];
+    const int slot = (i < nsink) ? i : sink + (i - nsink);
+    const long long src = ((long long)b * s.b + (long long)j * s.t + (long long)h * s.h) * elt;
+    const long long dst = (col0 + slot) * D * elt;
+    copy_row(reinterpret_cast<const uint4*>(k + src), reinterpret_cast<uint4*>(k_col + dst), nvec,
+             lane_in_row);
+    copy_row(reinterpret_cast<const uint4*>(v + src), reinterpret_cast<uint4*>(v_col + dst), nvec,
+             lane_in_row);
+  }
+}
+
+cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,
+                          int32_t* idx, int32_t* nret, int32_t* cnt, const void* k,
+                          const void* v, Strides4 s, void* k_col, void* v_col,
+                          cudaStream_t stream) {
+  const int elt = d->dtype == LTE_BF16 ? 2 : 4;
+  compact_kernel<<<d->B * d->Hkv, kCompactThreads, 0, stream>>>(
+      d->T, d->Hkv, d->sink, n_scored, d->tau, r, mask, idx, nret, cnt, (const char*)k,
+      (const char*)v, s, elt, d->D, (char*)k_col, (char*)v_col);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Decode-cache set-up from a prefilled prompt (Fig. 3 layout): window ring,
+// sink slots, retained ring.  One CTA per unit.
+__global__ void __launch_bounds__(256)
+cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap, int T0,
+                  int n_scored, const char* __restrict__ k, const char* __restrict__ v,
+                  Strides4 s, const float* __restrict__ r, const int32_t* __restrict__ idx,
+                  const int32_t* __restrict__ cnt, char* __restrict__ ck, char* __restrict__ cv,
+                  int32_t* __restrict__ pos, float* __restrict__ win_r,
+                  int32_t* __restrict__ ret_total, int32_t* __restrict__ meta) {
+  const int u = blockIdx.x, b = u / Hkv, h = u % Hkv, tid = threadIdx.x;
+  const int L = window + sink + cap;
+  const long long row0 = (long long)u * T;
+  const int last_out = T0 - 1 - window;                 // newest token outside the window
+  const int n = last_out >= 0 ? cnt[row0 + last_out] : 0;
+  const int ret_lo = (n - cap) > 0 ? n - cap : 0;
+
+  // slot -> source token (or -1)
+  for (int slot = tid; slot < L; slot += blockDim.x) {
+    int j = -1;
+    if (slot < window) {
+      // newest token in this window slot, if it is inside (T0-1-w, T0-1]
+      const int jj = T0 - 1 - ((T0 - 1 - slot) % window + window) % window;
+      if (T0 > 0 && jj >= 0 && jj > last_out) j = jj;
+      win_r[(long long)u * window + slot] = (j >= 0 && j < n_scored) ? r[row0 + j] : NAN;
+    } else if (slot < window + sink) {
+      const int jj = slot - window;
+      if (jj <= last_out) j = jj;
+    } else {
+      const int rs = slot - window - sink;
+      // retained ordinal i with i mod C == rs in [ret_lo, n)
+      if (n > 0) {
+        int i = ret_lo + ((rs - ret_lo % cap) % cap + cap) % cap;
+        if (i < n) j = idx[row0 + i];
+      }
+    }
+    pos[(long long)u * L + slot] = j;
+  }
+  __syncthreads();
+  const int nvec = D * elt / 16;
+  for (int i = tid; i < L * nvec; i += blockDim.x) {
+    const int slot = i / nvec, c = i % nvec;
+    const int j = pos[(long long)u * L + slot];
+    if (j < 0) continue;
+    const long long src = ((long long)b * s.b + (long long)j * s.t + (long long)h * s.h) * elt;
+    const long long dst = ((long long)u * L + slot) * D * elt;
+    reinterpret_cast<uint4*>(ck + dst)[c] = reinterpret_cast<const uint4*>(k + src)[c];
+    reinterpret_cast<uint4*>(cv + dst)[c] = reinterpret_cast<const uint4*>(v + src)[c];
+  }
+  if (tid == 0) {
+    ret_total[u] = n;
+    if (u == 0) {
+      meta[0] = T0;
+      meta[1] = n_scored;
+      meta[2] = n_scored;
+      meta[3] = 0;
+    }
+  }
+}
+
+cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, const void* v,
+                       Strides4 s, const float* r, const int32_t* idx, const int32_t* cnt,
+                       int T_prompt, int n_scored, cudaStream_t stream) {
+  const int elt = d->dtype == LTE_BF16 ? 2 : 4;
+  cache_init_kernel<<<d->B * d->Hkv, 256, 0, stream>>>(
+      d->T, d->Hkv, d->D, elt, d->window, d->sink, d->cap, T_prompt, n_scored,
+      (const char*)k, (const char*)v, s, r, idx, cnt, (char*)c->k, (char*)c->v, c->pos,
+      c->win_r, c->ret_total, c->meta);
+  return cudaGetLastError();
+}
+
+}  // namespace lte

@@ -1,0 +1,61 @@
+// Internal host-side launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lte_api.h"
+#include "lte_common.cuh"
+
+namespace lte {
+
+// score_cnn.cu
+bool score_supported(const lte_cnn* cnn);
+cudaError_t score_linear(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
+                         Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
+                         cudaStream_t stream);
+cudaError_t score_ring(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
+                       int score_batch, cudaStream_t stream);
+
+// evict_compact.cu
+cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,
+                          int32_t* idx, int32_t* nret, int32_t* cnt, const void* k,
+                          const void* v, Strides4 s, void* k_col, void* v_col,
+                          cudaStream_t stream);
+cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, const void* v,
+                       Strides4 s, const float* r, const int32_t* idx, const int32_t* cnt,
+                       int T_prompt, int n_scored, cudaStream_t stream);
+
+// attn_prefill_*.cu
+struct PrefillArgs {
+  const lte_dims* d;
+  const void *q, *k, *v;
+  Strides4 qs, kvs, os;
+  const int32_t* cnt;
+  const void *k_col, *v_col;
+  void* o;
+  float* lse;
+  DevError* err;
+  void* scratch;         // workspace after the error word
+  size_t scratch_bytes;
+};
+cudaError_t attn_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t attn_prefill_mma(const PrefillArgs& a, cudaStream_t stream);
+size_t attn_prefill_scratch_bytes(const lte_dims* d);
+
+// decode.cu
+size_t decode_scratch_bytes(const lte_dims* d);
+cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
+                        const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                        float* lse_t, int score_batch, DevError* err, void* scratch,
+                        cudaStream_t stream);
+
+// gla.cu
+cudaError_t gla_prefill(int B, int T, int H, int dk, int dv, int dtype, const void* q,
+                        const void* k, const void* v, const float* a, void* o, float* state,
+                        cudaStream_t stream);
+cudaError_t gla_decode(int B, int H, int dk, int dv, int dtype, const void* q, const void* k,
+                       const void* v, const float* a, void* o, float* state,
+                       cudaStream_t stream);
+
+}  // namespace lte

@@ -1,0 +1,143 @@
+"""Thin host-side helpers over the C ABI: allocate the caller-owned buffers
+(torch device memory) and chain the entry points of one LTE layer.
+
+Nothing here computes: prefill = lte_score (when a CNN is given) ->
+lte_evict_compact -> lte_sparse_attn_prefill; a decode step is one
+lte_decode_step call on a DecodeCache.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import lte as L
+
+
+@dataclass
+class LayerParams:
+    sink: int
+    window: int
+    cap: int
+    tau: float = 0.5
+    scale: float | None = None
+    past1: int = 2
+    past2: int = 1
+
+    def dims(self, B, T, Hq, Hkv, D, dtype) -> L.lte_dims:
+        scale = (1.0 / D ** 0.5) if self.scale is None else self.scale
+        return L.make_dims(B, T, Hq, Hkv, D, self.sink, self.window, self.cap, self.tau, scale, dtype)
+
+
+def cnn_future(w1, w2, past1, past2) -> int:
+    return (w1.shape[3] - 1 - past1) + (w2.shape[2] - 1 - past2)
+
+
+@dataclass
+class PrefillOut:
+    o: torch.Tensor
+    lse: torch.Tensor
+    r: torch.Tensor | None
+    mask: torch.Tensor | None
+    idx: torch.Tensor
+    nret: torch.Tensor
+    cnt: torch.Tensor
+    k_col: torch.Tensor
+    v_col: torch.Tensor
+    n_scored: int
+
+
+class PrefillBuffers:
+    """All buffers one prefill needs, allocated once (reused across calls)."""
+
+    def __init__(self, B, T, Hq, Hkv, D, dtype, sink, dims, device="cuda", want_r=True):
+        dev = torch.device(device)
+        self.dims = dims
+        self.o = torch.empty(B, T, Hq, D, dtype=dtype, device=dev)
+        self.lse = torch.empty(B, Hq, T, dtype=torch.float32, device=dev)
+        self.r = torch.full((B, Hkv, T), float("nan"), dtype=torch.float32, device=dev) if want_r else None
+        self.mask = torch.zeros(B, Hkv, T, dtype=torch.uint8, device=dev) if want_r else None
+        self.idx = torch.empty(B, Hkv, T, dtype=torch.int32, device=dev)
+        self.nret = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(B, Hkv, T, dtype=torch.int32, device=dev)
+        self.k_col = torch.empty(B, Hkv, sink + T, D, dtype=dtype, device=dev)
+        self.v_col = torch.empty(B, Hkv, sink + T, D, dtype=dtype, device=dev)
+        ws = L.lte_workspace_bytes(dims, L.LTE_WS_PREFILL)
+        self.ws = torch.zeros((ws + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+
+
+def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers | None = None,
+            stream=None) -> PrefillOut:
+    """One LTE layer prefill.  Either a fed retention `mask` [B,Hkv,T] (uint8)
+    or `cnn` = (w1, b1, w2, b2) device tensors for live scoring."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
+    if bufs is None:
+        bufs = PrefillBuffers(B, T, Hq, Hkv, D, q.dtype, p.sink, dims, q.device, want_r=cnn is not None)
+    if cnn is not None:
+        w1, b1, w2, b2 = cnn
+        c, _keep = L.make_cnn(w1, b1, w2, b2, p.past1, p.past2)
+        n_scored = max(0, T - cnn_future(w1, w2, p.past1, p.past2))
+        L.lte_score(dims, c, k, v, 0, n_scored, bufs.r, bufs.mask, stream)
+        L.lte_evict_compact(dims, None, bufs.mask, n_scored, bufs.idx, bufs.nret, bufs.cnt, k, v,
+                            bufs.k_col, bufs.v_col, stream)
+    else:
+        n_scored = T
+        L.lte_evict_compact(dims, None, mask, T, bufs.idx, bufs.nret, bufs.cnt, k, v, bufs.k_col,
+                            bufs.v_col, stream)
+    L.lte_sparse_attn_prefill(dims, q, k, v, bufs.cnt, bufs.k_col, bufs.v_col, bufs.o, bufs.lse,
+                              bufs.ws, stream)
+    return PrefillOut(bufs.o, bufs.lse, bufs.r, bufs.mask if cnn is not None else mask, bufs.idx,
+                      bufs.nret, bufs.cnt, bufs.k_col, bufs.v_col, n_scored)
+
+
+class DecodeCache:
+    """Caller-owned decode cache (window ring + sink slots + retained ring)."""
+
+    def __init__(self, B, Hkv, D, dtype, sink, window, cap, device="cuda"):
+        dev = torch.device(device)
+        Ls = window + sink + cap
+        self.k = torch.zeros(B, Hkv, Ls, D, dtype=dtype, device=dev)
+        self.v = torch.zeros(B, Hkv, Ls, D, dtype=dtype, device=dev)
+        self.pos = torch.full((B, Hkv, Ls), -1, dtype=torch.int32, device=dev)
+        self.win_r = torch.full((B, Hkv, window), float("nan"), dtype=torch.float32, device=dev)
+        self.ret_total = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
+        self.meta = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.sink, self.window, self.cap = sink, window, cap
+        self.struct = L.lte_cache(self.k.data_ptr(), self.v.data_ptr(), self.pos.data_ptr(),
+                                  self.win_r.data_ptr(), self.ret_total.data_ptr(),
+                                  self.meta.data_ptr())
+
+    def init_from_prefill(self, dims, k, v, out: PrefillOut, T_prompt, stream=None):
+        L.lte_cache_init_from_prefill(dims, self.struct, k, v, out.r, out.idx, out.cnt, T_prompt,
+                                      out.n_scored, stream)
+
+    def retained_positions(self):
+        """Sorted retained positions per unit (host copy, for checks)."""
+        w, s = self.window, self.sink
+        pos = self.pos[:, :, w + s:].cpu()
+        return [[sorted(int(x) for x in pos[b, h] if x >= 0) for h in range(pos.shape[1])]
+                for b in range(pos.shape[0])]
+
+
+class Decoder:
+    """Runs lte_decode_step with fixed output buffers (graph-capturable)."""
+
+    def __init__(self, dims, cnn, past1, past2, cache: DecodeCache, score_batch, device="cuda"):
+        self.dims = dims
+        w1, b1, w2, b2 = cnn
+        self.cnn, self._keep = L.make_cnn(w1, b1, w2, b2, past1, past2)
+        self.cache = cache
+        self.score_batch = score_batch
+        B, Hq, D = dims.B, dims.Hq, dims.D
+        dt = torch.bfloat16 if dims.dtype == L.LTE_BF16 else torch.float32
+        self.o = torch.empty(B, Hq, D, dtype=dt, device=device)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=device)
+        ws = L.lte_workspace_bytes(dims, L.LTE_WS_DECODE)
+        self.ws = torch.zeros((ws + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+    def step(self, q_t, k_t, v_t, stream=None):
+        L.lte_decode_step(self.dims, self.cnn, self.cache.struct, q_t, k_t, v_t, self.o, self.lse,
+                          self.score_batch, self.ws, stream)
+        return self.o, self.lse

@@ -1,0 +1,80 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/lte_api.h declares; host-side argument validation rejects bad calls
+before any launch (no device needed for those paths)."""
+import ctypes as C
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lte_api.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lte_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sys.path.insert(0, ROOT)
+    from learnable_kv_token_b200 import build
+    path = build.build()
+    return C.CDLL(path), path
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    for n in ("lte_score", "lte_evict_compact", "lte_sparse_attn_prefill", "lte_decode_step",
+              "lte_cache_init_from_prefill", "lte_workspace_bytes", "lte_gla_prefill",
+              "lte_gla_decode_step", "lte_read_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    cdll, path = lib
+    for name in _declared():
+        assert hasattr(cdll, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (lte_\w+)", out))
+    assert set(_declared()) <= exported
+
+
+def test_binding_exposes_same_names(lib):
+    from learnable_kv_token_b200 import lte
+    for name in _declared():
+        if name == "lte_version":
+            continue
+        assert hasattr(lte, name), name
+
+
+def test_host_validation_without_gpu(lib):
+    """Invalid calls return an error status before touching the device."""
+    from learnable_kv_token_b200 import lte as L
+    d = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32)
+    f = L._lib
+    # null pointers -> LTE_ERR_INVALID_ARG
+    assert f.lte_evict_compact(C.byref(d), None, None, 64, None, None, None, None, None, None,
+                               None, None, None) == 1
+    bad = L.make_dims(1, 64, 6, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32)   # Hq % Hkv != 0
+    assert f.lte_workspace_bytes(C.byref(bad), 0) == 0
+    d96 = L.make_dims(1, 64, 4, 4, 96, 4, 16, 8, 0.5, 0.1, L.LTE_F32)     # D not in {64,128}
+    assert f.lte_sparse_attn_prefill(C.byref(d96), None, None, None, None, None, None, None, None,
+                                     None, None, None, None, 0, None) == 2
+    assert f.lte_workspace_bytes(C.byref(d), 0) >= 16
+    assert f.lte_workspace_bytes(C.byref(d), 1) > 16
+    # score: range beyond the receptive field -> invalid
+    cnn = L.lte_cnn(32, 5, 2, 3, 1, 16, 16, 16, 16)
+    assert f.lte_score(C.byref(d), C.byref(cnn), C.c_void_p(16), C.c_void_p(16), None, 0, 63,
+                       C.c_void_p(16), None, None) == 1
+    # decode: score batch larger than the window allows -> invalid
+    dd = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_BF16)
+    cache = L.lte_cache(16, 16, 16, 16, 16, 16)
+    assert f.lte_decode_step(C.byref(dd), C.byref(cnn), C.byref(cache), C.c_void_p(16),
+                             C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), None, 11,
+                             C.c_void_p(16), 1 << 20, None) == 1
+    assert L.version().startswith("lte-b200")
