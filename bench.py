@@ -1,0 +1,453 @@
+"""Benchmark of the LTE sparse-attention hot path on B200.
+
+Default (one GPU): the prefill workload -- B=32, T=4096, 16 query heads over
+4 KV heads, head dim 128, bf16, sink 4, window 512, cap 512, retention mask
+Bernoulli(0.1) fed directly -- one step = lte_evict_compact (compaction and
+column-segment copy) + lte_sparse_attn_prefill.  `value` = B*T tokens per
+second of device time (max over ranks; every rank runs its own batch, so the
+scaling is weak and no collective touches the data path).
+
+Also reported on the same JSON line:
+  roofline     the attention kernel's attended FLOPs / its CUDA-event time
+               against the measured bf16 peak;
+  e2e          the same step from pinned host buffers (H2D of q, k, v, mask
+               and D2H of o inside the timed region);
+  decode       the decode workload (4096-token prompt, B=32, CNN scored live,
+               deferred batch 64): per-layer decode steps rotating over 4
+               layer caches (> L2), captured in a CUDA graph;
+  cpu_baseline the CPU oracle on a bounded sample of the same workload.
+`--impl reference` times the CPU oracle alone (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lte_inputs as LI  # noqa: E402
+
+METRIC = "LTE sparse-attn prefill & decode tokens/s at 1 B200; % tensor/HBM roofline"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def attended_pairs(mask: np.ndarray, sink: int, window: int, cap: int) -> np.ndarray:
+    """|S_t| per (b, h, t) from a fed mask [B,Hkv,T]: window + out-of-window
+    sinks + min(C, retained tokens that left the window).  Work count only."""
+    B, H, T = mask.shape
+    m = mask.astype(np.int64).copy()
+    m[..., :sink] = 0
+    cnt = np.cumsum(m, axis=-1)
+    t = np.arange(T)
+    win = np.minimum(t + 1, window)
+    sinks = np.clip(t - window + 1, 0, sink)
+    n = np.zeros_like(cnt)
+    n[..., window:] = cnt[..., :T - window]
+    return win[None, None] + sinks[None, None] + np.minimum(n, cap)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1])); mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_id(device):
+    """nvidia-smi -i identifier of a torch device (UUID, so that
+    CUDA_VISIBLE_DEVICES remapping does not matter)."""
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return device.index if device.index is not None else 0
+
+
+def source_hash(*files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(kernel_file, launch_units):
+    """DRAM bytes per launch from the committed ncu summary, scaled to this
+    launch by units processed, or None when the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        tr = json.load(f)
+    ent = tr.get(kernel_file)
+    if not ent or ent.get("source_hash") != source_hash(kernel_file):
+        return None
+    return ent["dram_bytes_per_unit"] * launch_units
+
+
+# ------------------------------------------------------------------------- oracle timing
+def oracle_sample(wl, seconds_min, seconds_max, rows_per_unit=None):
+    """Run the CPU oracle on (b, h) units of the workload until seconds_min
+    have elapsed; returns (tokens_equivalent, seconds, description)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import lte_oracle as O
+    g = LI.generator(wl.seed)
+    B = 1
+    q, k, v = LI.qkv(B, wl.T, wl.Hq, wl.Hkv, wl.D, wl.dtype, g)
+    mask = LI.bernoulli_mask(B, wl.Hkv, wl.T, wl.mask_rate, g)
+    G = wl.G
+    rows = list(range(wl.T)) if rows_per_unit is None else \
+        list(range(wl.T - 1, -1, -max(1, wl.T // rows_per_unit)))
+    qn = q.double().numpy(); kn = k.double().numpy(); vn = v.double().numpy()
+    done_rows, t0 = 0, time.perf_counter()
+    units = 0
+    with threadpool_limits(1):
+        for h in range(wl.Hkv):
+            m = O.fed_mask(mask[0, h].numpy(), wl.sink)
+            O.prefill_unit(qn[0, :, h * G:(h + 1) * G], kn[0, :, h], vn[0, :, h], m, wl.sink,
+                           wl.window, wl.cap, wl.scale, rows=rows)
+            done_rows += len(rows)
+            units += 1
+            el = time.perf_counter() - t0
+            if el >= seconds_min or el >= seconds_max:
+                break
+    el = time.perf_counter() - t0
+    desc = f"{units} (batch, KV-head) unit(s) x {len(rows)} rows of the {wl.name} workload"
+    return done_rows / wl.Hkv, el, desc
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = LI.WORKLOADS["prefill"]
+    for _ in range(args.warmup):
+        oracle_sample(wl, 0.0, 1e9, rows_per_unit=128)
+    tok, sec = 0.0, 0.0
+    for _ in range(args.steps):
+        a, b, desc = oracle_sample(wl, 0.0, 1e9, rows_per_unit=128)
+        tok += a; sec += b
+    value = tok / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill B=32 T=4096 Hq=16 Hkv=4 D=128 s=4 w=512 C=512 mask~Bern(0.1)",
+                       "global_batch": wl.B, "seq_len": wl.T, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"per step: {desc} (128 strided rows of KV head 0)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------- GPU arm
+def prefill_bench(args, rank, world, device):
+    from learnable_kv_token_b200 import layer, lte as L
+    wl = LI.WORKLOADS["prefill"]
+    inp = LI.lte_inputs(wl.with_(seed=wl.seed + 1000 * rank), T=wl.T)
+    q, k, v, mask = inp["q"], inp["k"], inp["v"], inp["mask"]
+    B, T, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
+    pairs = attended_pairs(mask.numpy(), wl.sink, wl.window, wl.cap)
+    flops = 4.0 * D * wl.G * float(pairs.sum())         # QK^T + PV per (row, head, key)
+    p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=wl.cap, tau=wl.tau)
+    dims = p.dims(B, T, Hq, Hkv, D, torch.bfloat16)
+    qd, kd, vd, md = (x.to(device) for x in (q, k, v, mask))
+    bufs = layer.PrefillBuffers(B, T, Hq, Hkv, D, torch.bfloat16, wl.sink, dims, device,
+                                want_r=False)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        L.lte_evict_compact(dims, None, md, T, bufs.idx, bufs.nret, bufs.cnt, kd, vd, bufs.k_col,
+                            bufs.v_col, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        L.lte_sparse_attn_prefill(dims, qd, kd, vd, bufs.cnt, bufs.k_col, bufs.v_col, bufs.o,
+                                  bufs.lse, bufs.ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(gpu_id(device)) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = t_start.elapsed_time(t_end)
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms_total = max_over_ranks(ms_total, world, device)
+    attn_ms = max_over_ranks(attn_ms, world, device)
+    ms_step = ms_total / args.steps
+    assert L.lte_read_device_error(bufs.ws) == (0, 0)
+
+    # e2e: pinned host buffers, H2D of the inputs and D2H of o inside the timed region
+    hq, hk, hv, hm = (x.pin_memory() for x in (q, k, v, mask))
+    ho = torch.empty(bufs.o.shape, dtype=bufs.o.dtype).pin_memory()
+    n_e2e = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True); kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True); md.copy_(hm, non_blocking=True)
+        step()
+        ho.copy_(bufs.o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, device)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hm))
+    d2h = ho.numel() * ho.element_size()
+
+    return {
+        "B": B, "T": T, "flops": flops, "pairs": float(pairs.sum()), "ms_step": ms_step,
+        "attn_ms": attn_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+        "launches": 2 * args.steps, "units": B * Hkv * ((T + 16 - 1) // 16),
+        "full_causal_pairs": B * Hkv * T * (T + 1) / 2,
+    }
+
+
+def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
+    from learnable_kv_token_b200 import layer
+    wl = LI.WORKLOADS["decode"]
+    inp = LI.lte_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    q, k, v, cnn = inp["q"], inp["k"], inp["v"], inp["cnn"]
+    B, T0, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
+    p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=wl.cap, tau=wl.tau)
+    qd, kd, vd = (x.to(device) for x in (q, k, v))
+    cd = tuple(x.to(device) for x in cnn)
+    kp, vp, qp = kd[:, :T0].contiguous(), vd[:, :T0].contiguous(), qd[:, :T0].contiguous()
+    dims = p.dims(B, T0, Hq, Hkv, D, torch.bfloat16)
+    torch.cuda.synchronize()
+    tp0 = time.perf_counter()
+    out = layer.prefill(qp, kp, vp, p, cnn=cd)
+    torch.cuda.synchronize()
+    prefill_cnn_ms = 1e3 * (time.perf_counter() - tp0)
+    decs = []
+    for _ in range(n_layers):
+        cache = layer.DecodeCache(B, Hkv, D, torch.bfloat16, wl.sink, wl.window, wl.cap, device)
+        cache.init_from_prefill(dims, kp, vp, out, T0)
+        decs.append(layer.Decoder(dims, cd, p.past1, p.past2, cache, wl.score_batch, device))
+    del out
+    qs = qd[:, T0:].permute(1, 0, 2, 3).contiguous()
+    ks = kd[:, T0:].permute(1, 0, 2, 3).contiguous()
+    vs = vd[:, T0:].permute(1, 0, 2, 3).contiguous()
+    stream = torch.cuda.Stream(device)
+    # warm-up: a few eager steps per layer
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            for d in decs:
+                d.step(qs[i], ks[i], vs[i], stream=stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(steps_per_layer):
+                for d in decs:
+                    t = 3 + i
+                    d.step(qs[t], ks[t], vs[t], stream=stream)
+    graph.replay()                     # warm replay
+    torch.cuda.synchronize()
+    ret = decs[0].cache.ret_total.clone()
+    t_meta = int(decs[0].cache.meta[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    n_steps = steps_per_layer * n_layers
+    ms_step = max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
+    del graph
+    # algorithmic bytes of one layer step (steady state)
+    n_keys = (min(wl.window, t_meta) + wl.sink + torch.clamp(ret, max=wl.cap)).sum().item()
+    units = B * Hkv
+    row = 2 * D * 2                                   # K + V bf16
+    bytes_step = (n_keys * row                        # attended K/V
+                  + 2 * B * Hq * D * 2                # q in, o out
+                  + units * row * 2                   # new token write + leaving-token move
+                  + units * row * (wl.score_batch + 6) / wl.score_batch)   # deferred scoring reads
+    return {"ms_step": ms_step, "bytes": bytes_step, "n_keys": n_keys, "B": B,
+            "prefill_with_cnn_ms": prefill_cnn_ms, "launches": 3 * n_steps}
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lte", choices=["lte", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    from learnable_kv_token_b200 import build as _b  # noqa: F401  (library is prebuilt in-tree)
+
+    pk = peaks()
+    pf = prefill_bench(args, rank, world, device)
+    dec = None if args.no_decode else decode_bench(args, rank, world, device)
+
+    if rank == 0:
+        tokens = pf["B"] * pf["T"] * world
+        value = tokens / (pf["ms_step"] / 1e3)
+        attn_tflops = pf["flops"] / (pf["attn_ms"] / 1e3) / 1e12
+        traffic = traffic_from_profiles("learnable_kv_token_b200/csrc/attn_prefill_mma.cu",
+                                        pf["units"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "prefill B=32 T=4096 Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512 "
+                                   "mask~Bern(0.1) fed; step = evict_compact + sparse_attn_prefill",
+                       "global_batch": pf["B"] * world, "seq_len": pf["T"],
+                       "parallelism": f"dp{world} (independent sequences per GPU)",
+                       "l2": "inputs larger than L2 (q 512 MiB, k/v 128 MiB each)"},
+            "roofline": {"kernel": "attn_prefill_mma_kernel", "bound": "tensor",
+                         "achieved": attn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": attn_tflops / pk["bf16_tflops"],
+                         "frac_of_sustained": attn_tflops / pk["bf16_tflops_sustained"],
+                         "peak_source": pk["source"], "traffic": traffic,
+                         "attended_flops_per_launch": pf["flops"],
+                         "kernel_ms": pf["attn_ms"],
+                         "sparsity_vs_full_causal": pf["pairs"] / pf["full_causal_pairs"]},
+            "clocks": pf["clocks"],
+            "e2e": {"value": pf["B"] * pf["T"] * world / (pf["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": pf["h2d"], "d2h_bytes_per_step": pf["d2h"]},
+            "gpu_launches": pf["launches"] + (dec["launches"] if dec else 0),
+        }
+        if dec is not None:
+            gbs = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
+            line["decode"] = {
+                "workload": "decode B=32, 4096-token prompt, Hq=16 Hkv=4 D=128 bf16 s=4 w=512 "
+                            "C=512, CNN scored live (tau 0.5, deferred batch 64); per-layer steps "
+                            "over 4 layer caches (> L2) in one CUDA graph",
+                "value": dec["B"] * world / (dec["ms_step"] / 1e3), "unit": "tokens/s",
+                "us_per_layer_step": 1e3 * dec["ms_step"],
+                "roofline": {"bound": "hbm", "scope": "whole decode step (3 kernels)",
+                             "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"]},
+                "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
+            }
+        if world == 1:
+            tok, sec, desc = oracle_sample(LI.WORKLOADS["prefill"], args.cpu_seconds,
+                                           2.5 * args.cpu_seconds)
+            line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": 1,
+                                    "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
