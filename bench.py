@@ -327,16 +327,18 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
                 for d in decs:
                     t = 3 + i
                     d.step(qs[t], ks[t], vs[t], stream=stream)
-    graph.replay()                     # warm replay
+    with torch.cuda.stream(stream):    # replay() launches on the current stream
+        graph.replay()                 # warm replay
     torch.cuda.synchronize()
     ret = decs[0].cache.ret_total.clone()
     t_meta = int(decs[0].cache.meta[0])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    e0.record(stream)
-    graph.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     n_steps = steps_per_layer * n_layers
     ms_step = max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
