@@ -205,6 +205,33 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
                            void* o_t, float* lse_t, int32_t score_batch,
                            void* workspace, size_t ws_bytes, void* stream);
 
+/* lte_decode_step_noalloc -- lte_decode_step for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a library
+ * convenience.  Some callers are not allowed to call cudaMalloc: a host
+ * runtime that has reserved the whole device for its own memory pool and
+ * hands a plugin only its input and output buffers, or a latency-critical
+ * loop where the device-wide synchronisation a cudaMalloc can imply is not
+ * acceptable.  This entry point takes the same arguments minus the workspace
+ * and keeps its scratch (error word, split partials, completion counters)
+ * in one file-scope device array of LTE_NOALLOC_SCRATCH_BYTES bytes, which
+ * every GPU that loads the library holds until the process exits.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *  - Limit: returns LTE_ERR_WORKSPACE, launching nothing, when
+ *    lte_workspace_bytes(d, LTE_WS_DECODE) > LTE_NOALLOC_SCRATCH_BYTES
+ *    (4 MiB covers B*Hkv = 128 units x 1028 cache slots x G = 4, D = 128).
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Sharing: all calls on a device share the one array and it keeps the
+ *    last call's contents; every call zeroes the error word and the counters
+ *    it relies on.  Calls that overlap on the GPU (e.g. on two streams at
+ *    once) race on the array: serialise them.
+ *  - Results are the same as lte_decode_step's (same kernels). */
+#define LTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const lte_cache* cache,
+                                   const void* q_t, const void* k_t, const void* v_t,
+                                   void* o_t, float* lse_t, int32_t score_batch, void* stream);
+
 enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1 };
 
 /* Bytes of workspace a call needs (>= 16: the first 16 bytes hold the device

@@ -1,11 +1,19 @@
 """LTE (contextualized Learnable Token Eviction) on B200: a C-ABI CUDA library
 (liblte.so, sm_100a) and its Python binding.
 
-``lte``   - one function per C entry point (argument marshalling only).
+``lte``   - one function per C entry point (argument marshalling only); importing
+            it loads liblte.so and fails if the library is missing.
 ``layer`` - buffer allocation and the call sequence of one layer.
-The binding loads liblte.so on import and fails if it is missing.
+``build`` - compiles liblte.so (importable without the library).
 """
-from .lte import (LteError, lte_cache_init_from_prefill, lte_clear_device_error,  # noqa: F401
-                  lte_decode_step, lte_evict_compact, lte_gla_decode_step, lte_gla_prefill,
-                  lte_read_device_error, lte_score, lte_sparse_attn_prefill, lte_workspace_bytes,
-                  version)
+_LAZY = ("LteError", "lte_cache_init_from_prefill", "lte_clear_device_error", "lte_decode_step",
+         "lte_decode_step_noalloc", "lte_evict_compact", "lte_gla_decode_step", "lte_gla_prefill",
+         "lte_read_device_error", "lte_score", "lte_sparse_attn_prefill", "lte_workspace_bytes",
+         "version")
+
+
+def __getattr__(name):
+    if name in _LAZY:
+        from . import lte
+        return getattr(lte, name)
+    raise AttributeError(name)

@@ -27,6 +27,8 @@
 //     counter) merges them; the last unit advances meta.
 #include <math.h>
 
+#include <mutex>
+
 #include "lte_common.cuh"
 #include "lte_internal.h"
 
@@ -373,6 +375,33 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
   if (d->D == 128)
     return launch_decode_attn<128>(d, c, q_t, o_t, lse_t, part, counters, stream);
   return launch_decode_attn<64>(d, c, q_t, o_t, lse_t, part, counters, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Scratch of lte_decode_step_noalloc, for callers that cannot allocate device
+// memory: one file-scope array per device, zero at module load, held until the
+// process exits.  Host code must not pass the symbol itself to a kernel (on
+// the host it names a stand-in, not device memory): the device address is
+// looked up once per device with that device current, and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LTE_NOALLOC_SCRATCH_BYTES];
+
+cudaError_t noalloc_scratch(void** ptr) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace lte

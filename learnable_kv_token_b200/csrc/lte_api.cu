@@ -197,6 +197,36 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
                                     as_stream(stream)));
 }
 
+lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const lte_cache* cache,
+                                   const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                                   float* lse_t, int32_t score_batch, void* stream) {
+  // Same validation as lte_decode_step, then the static scratch in place of a workspace.
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if ((st = check_cnn(cnn)) != LTE_OK) return st;
+  if (d->dtype != LTE_BF16) return LTE_ERR_UNSUPPORTED;
+  if (cache == nullptr || !cache->k || !cache->v || !cache->pos || !cache->win_r ||
+      !cache->ret_total || !cache->meta)
+    return LTE_ERR_INVALID_ARG;
+  if (!q_t || !k_t || !v_t || !o_t) return LTE_ERR_INVALID_ARG;
+  if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) ||
+      !aligned16(cache->k) || !aligned16(cache->v))
+    return LTE_ERR_INVALID_ARG;
+  if (score_batch < 1 || score_batch > d->window - cnn_past(cnn) - cnn_future(cnn))
+    return LTE_ERR_INVALID_ARG;
+  if (d->Hq / d->Hkv > 16) return LTE_ERR_UNSUPPORTED;
+  if (lte_workspace_bytes(d, LTE_WS_DECODE) > (size_t)LTE_NOALLOC_SCRATCH_BYTES)
+    return LTE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (lte::noalloc_scratch(&scratch) != cudaSuccess) return LTE_ERR_CUDA;
+  // the error word must start at zero for this call (counters are zeroed by the step itself)
+  if (cudaMemsetAsync(scratch, 0, sizeof(lte::DevError), as_stream(stream)) != cudaSuccess)
+    return LTE_ERR_CUDA;
+  return from_cuda(lte::decode_step(d, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch,
+                                    reinterpret_cast<lte::DevError*>(scratch),
+                                    static_cast<char*>(scratch) + kErrBytes, as_stream(stream)));
+}
+
 lte_status lte_clear_device_error(void* workspace, void* stream) {
   if (workspace == nullptr) return LTE_ERR_INVALID_ARG;
   return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(lte::DevError), as_stream(stream)));

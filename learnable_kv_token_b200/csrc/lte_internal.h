@@ -50,6 +50,9 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
                         float* lse_t, int score_batch, DevError* err, void* scratch,
                         cudaStream_t stream);
 
+// decode.cu: the allocation-free variant's scratch (file-scope device array)
+cudaError_t noalloc_scratch(void** ptr);
+
 // gla.cu
 cudaError_t gla_prefill(int B, int T, int H, int dk, int dv, int dtype, const void* q,
                         const void* k, const void* v, const float* a, void* o, float* state,

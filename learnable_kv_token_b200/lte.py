@@ -67,6 +67,8 @@ _SIG = {
                                     C.POINTER(lte_strides), _P, _P, _P, _I, _I, _P],
     "lte_decode_step": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P, _P, _P,
                         _P, _P, _I, _P, C.c_size_t, _P],
+    "lte_decode_step_noalloc": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P,
+                                _P, _P, _P, _P, _I, _P],
     "lte_clear_device_error": [_P, _P],
     "lte_read_device_error": [_P, C.POINTER(C.c_int32), C.POINTER(C.c_int32), _P],
     "lte_gla_prefill": [_I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P],
@@ -167,6 +169,14 @@ def lte_decode_step(dims, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch, wo
     _call("lte_decode_step", C.byref(dims), C.byref(cnn), C.byref(cache), _ptr(q_t), _ptr(k_t),
           _ptr(v_t), _ptr(o_t), _ptr(lse_t), score_batch, _ptr(workspace),
           workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def lte_decode_step_noalloc(dims, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch,
+                            stream=None):
+    """lte_decode_step without a workspace: the library's static device scratch
+    (for callers that cannot allocate device memory; see lte_api.h)."""
+    _call("lte_decode_step_noalloc", C.byref(dims), C.byref(cnn), C.byref(cache), _ptr(q_t),
+          _ptr(k_t), _ptr(v_t), _ptr(o_t), _ptr(lse_t), score_batch, _stream(stream))
 
 
 def lte_clear_device_error(workspace, stream=None):
