@@ -283,7 +283,7 @@ def prefill_bench(args, rank, world, device):
     return {
         "B": B, "T": T, "flops": flops, "pairs": float(pairs.sum()), "ms_step": ms_step,
         "attn_ms": attn_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-        "launches": 2 * args.steps, "units": B * Hkv * ((T + 16 - 1) // 16),
+        "launches": 2 * args.steps, "units": B * Hkv * ((T + 32 - 1) // 32),
         "full_causal_pairs": B * Hkv * T * (T + 1) / 2,
     }
 
@@ -403,7 +403,7 @@ def main():
         tokens = pf["B"] * pf["T"] * world
         value = tokens / (pf["ms_step"] / 1e3)
         attn_tflops = pf["flops"] / (pf["attn_ms"] / 1e3) / 1e12
-        traffic = traffic_from_profiles("learnable_kv_token_b200/csrc/attn_prefill_mma.cu",
+        traffic = traffic_from_profiles("learnable_kv_token_b200/csrc/attn_prefill_tc.cu",
                                         pf["units"])
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -415,7 +415,7 @@ def main():
                        "global_batch": pf["B"] * world, "seq_len": pf["T"],
                        "parallelism": f"dp{world} (independent sequences per GPU)",
                        "l2": "inputs larger than L2 (q 512 MiB, k/v 128 MiB each)"},
-            "roofline": {"kernel": "attn_prefill_mma_kernel", "bound": "tensor",
+            "roofline": {"kernel": "attn_prefill_tc_kernel", "bound": "tensor",
                          "achieved": attn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": attn_tflops / pk["bf16_tflops"],
                          "frac_of_sustained": attn_tflops / pk["bf16_tflops_sustained"],
