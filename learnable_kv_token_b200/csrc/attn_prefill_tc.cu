@@ -7,26 +7,33 @@
 //   S_t = { j < s : j <= t-w } u (t-w, t] u { idx[i] : max(0, n_t-C) <= i < n_t },
 //   n_t = cnt[t-w] (0 for t < w).
 //
-// One CTA computes a 128-row tile: 128/G tokens x the G query heads of one KV
-// head (rows token-major), so each K/V tile it loads serves the whole group.
-// Keys come in tiles of 64 from up to three ranges: the sink slots and the
-// retained slots of the column segment (compacted rows, contiguous) and the
-// window band of the key tensor; each tile is one TMA box per 64-column half.
-// Warp roles (192 threads):
-//   warp 0     TMA producer: Q once, then K and V tiles into a 2-stage ring;
-//   warp 1     TMEM owner and MMA issuer (one thread): S = Q K^T into TMEM,
-//              O += P V with O resident in TMEM for the whole key loop;
-//   warps 2-5  softmax: one thread per row reads its S row from TMEM, applies
-//              the attended-set predicate, keeps the running max and sum,
-//              writes P (bf16) into a 128B-swizzled shared tile for the PV
-//              MMA, and rescales the O row in TMEM only when the running max
-//              grew by more than 2^8 (exact: O and l share the reference max);
-//              then the epilogue reads O, divides by l and stores bf16.
-// The MMA warp issues S_{j+1} before PV_j, so the QK^T of the next tile runs
-// while the softmax of this one is computed.  Every mbarrier wait is bounded
-// (1 s of global time): on expiry the CTA records LTE_ERR_TIMEOUT in the
-// workspace error word, stops issuing work, waits (bounded) for its copies
-// and MMAs in flight, frees its TMEM and exits.
+// Work item: one (batch, KV head) unit and two consecutive 128-row Q tiles
+// (each 128/G tokens x the G query heads of the group, rows token-major).
+// Both Q tiles consume every K/V tile the item loads, so a K/V byte read from
+// L2 serves 256 rows.  Keys come in tiles of 64 from up to three ranges: the
+// sink slots and the retained slots of the column segment (compacted rows,
+// contiguous) and the window band of the key tensor; every tile is one TMA box
+// per 64-column half.  The kernel is persistent (one CTA per SM walks a static
+// heavy-first list of items).  Warp roles (320 threads):
+//   warp 0     TMA producer: Q tiles into a double buffer (the next item's Q
+//              loads while the current item runs), K and V into 3-slot rings (a K slot frees after
+//              its S MMAs, a V slot after its PV MMAs);
+//   warp 1     TMEM owner and MMA issuer (one elected lane): per K/V tile j,
+//              S_A = Q_A K^T, S_B = Q_B K^T, then O_A += P_A V, O_B += P_B V for
+//              tile j-1, so the tensor core computes one Q tile's products while
+//              the other tile's softmax runs; S, O and P of both tiles live in
+//              TMEM (2 x (64 + 128 + 32) of 512 columns);
+//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread per
+//              row reads its S row from TMEM, applies the attended-set
+//              predicate, exp2 via ex2.approx with the scale folded into one
+//              packed FMA, writes P (bf16 pairs) into TMEM, where the PV MMA
+//              reads it as its A operand (only V comes from shared memory),
+//              and rescales its O row in TMEM only when the running max grew by
+//              more than 2^8 (exact: O and l share the reference max); the
+//              epilogue reads O, divides by l and stores bf16 and the lse.
+// Every mbarrier wait is bounded (1 s of global time): on expiry the CTA
+// records LTE_ERR_TIMEOUT in the workspace error word, stops issuing work,
+// waits (bounded) for its copies and MMAs in flight, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -37,31 +44,34 @@
 namespace lte {
 namespace tc {
 
-constexpr int BM = 128;             // rows per CTA (TMEM lanes)
-constexpr int BN = 64;              // keys per tile
+constexpr int BM = 128;             // rows per Q tile (TMEM lanes)
+constexpr int BN = 64;              // keys per K/V tile
 constexpr int HD = 128;             // head dim
-constexpr int kThreads = 192;
-constexpr int kStages = 2;
-constexpr uint32_t kQBytes = BM * HD * 2;      // 32 KiB
-constexpr uint32_t kQHalf = BM * 128;          // one 64-column half of Q: 16 KiB
-constexpr uint32_t kKVBytes = BN * HD * 2;     // 16 KiB (K or V of one tile)
-constexpr uint32_t kKVHalf = BN * 128;         // 8 KiB
-constexpr uint32_t kPBytes = BM * BN * 2;      // 16 KiB
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kQBytes;                              // stage s: K at +s*32K, V at +16K
-constexpr uint32_t kOffP = kOffKV + kStages * 2 * kKVBytes;       // 96 KiB
-constexpr uint32_t kOffBar = kOffP + kPBytes;                     // 112 KiB
+constexpr int kThreads = 320;
+constexpr uint32_t kQTile = BM * HD * 2;          // 32 KiB
+constexpr uint32_t kQHalf = BM * 128;             // 64-column half of a Q tile: 16 KiB
+constexpr uint32_t kQBuf = 2 * kQTile;            // tiles A and B of one item: 64 KiB
+constexpr uint32_t kKV = BN * HD * 2;             // 16 KiB (K or V of one tile)
+constexpr uint32_t kKVHalf = BN * 128;            // 8 KiB
+constexpr int kStages = 3;                        // K/V ring depth
+constexpr uint32_t kOffQ = 0;                     // 2 buffers
+constexpr uint32_t kOffKV = 2 * kQBuf;            // 128 KiB; stage s: K at +s*32K, V at +16K
+constexpr uint32_t kOffBar = kOffKV + kStages * 2 * kKV;   // 224 KiB
 constexpr uint32_t kSmemBytes = kOffBar + 256;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 64;
-constexpr unsigned long long kWaitNs = 1000000000ull;             // bounded waits: 1 s
+constexpr uint32_t kTmemCols = 512;
+__host__ __device__ constexpr uint32_t col_s(int x) { return x == 0 ? 0u : 64u; }     // S of tile x
+__host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256u; }  // O of tile x
+__host__ __device__ constexpr uint32_t col_p(int x) { return x == 0 ? 384u : 416u; }  // P (bf16 pairs)
+constexpr unsigned long long kWaitNs = 1000000000ull;
 
-// barrier slots (8 bytes each) after kOffBar
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KVE = 5, B_SF = 7, B_SFREE = 8, B_PF = 9, B_PVD = 10,
-       B_FIN = 11, kNumBars = 12 };
+enum {
+  B_QF = 0, B_QE = 2, B_KF = 4, B_VF = 7, B_KE = 10, B_VE = 13, B_SF = 16, B_SFREE = 18,
+  B_PF = 20, B_PVD = 22, B_OE = 24, B_FIN = 26, kNumBars = 27
+};
 
 struct Params {
   int T, Hq, Hkv, G, TOK, sink, window, cap;
+  int n_pairs, n_units, n_items;
   float scale_log2;
   const int32_t* cnt;
   __nv_bfloat16* o;
@@ -114,6 +124,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
+// Warp-uniform bounded wait (every lane of the calling warp must call it):
+// the warp proceeds only if every lane saw the phase complete.
+__device__ __forceinline__ bool wwait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      DevError* err, int where) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, err, where);
+  return __all_sync(0xffffffffu, ok);
+}
 // Wait used while shutting down: bounded, ignores the abort flag.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const unsigned long long t0 = gtime();
@@ -137,19 +154,28 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-
+// One lane of a converged warp (elect.sync): the issuing warps run their loops
+// with all 32 lanes, so descriptors and coordinates stay warp-uniform, and
+// only the elected lane issues each TMA copy, MMA or commit.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n .reg .pred P;\n elect.sync _|P, 0xffffffff;\n selp.b32 %0, 1, 0, P;\n}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// 128B-swizzled K-major or MN-major shared-memory matrix descriptor (version 1)
+// 128B-swizzled shared-memory matrix descriptor (version 1)
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// instruction descriptor, kind::f16: bf16 A/B, fp32 D
+// instruction descriptor, kind::f16: bf16 A/B, fp32 D, A K-major
 __host__ __device__ constexpr uint32_t idesc(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -162,6 +188,15 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       "l"(a), "l"(b), "r"(id), "r"(accumulate)
       : "memory");
 }
+// A operand (M x 16, bf16 pairs per 32-bit column, row m in lane m) read from TMEM
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -172,7 +207,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                   "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
 #define LTE_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
                   "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-// 32 consecutive 32-bit TMEM columns of this thread's lane
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -196,18 +230,57 @@ __device__ __forceinline__ void tmem_wait_ld() {
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ float ex2(float x) {   // 2^x, approximate (MUFU)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
-struct Tiles {
-  int start[3], count[3], ntile[3], total;   // 0: sink slots, 1: retained slots, 2: window band
-  __device__ __forceinline__ void at(int it, int& rg, int& key0, int& nk) const {
-    rg = 0;
-    while (rg < 2 && it >= ntile[rg]) { it -= ntile[rg]; ++rg; }
-    key0 = start[rg] + it * BN;
-    nk = min(BN, count[rg] - it * BN);
+// ---------------------------------------------------------------- work items
+struct Item {
+  int b, h, u, t0, t_last;     // tokens [t0, t_last] over both Q tiles
+  // key ranges: 0 sink slots, 1 retained slots (column segment), 2 window band
+  int s0, c0, n0, s1, c1, n1, s2, c2, total;
+  __device__ __forceinline__ void tile(int it, int& rg, int& key0, int& nk) const {
+    int st, cn;
+    if (it < n0) { rg = 0; st = s0; cn = c0; }
+    else if (it < n0 + n1) { rg = 1; it -= n0; st = s1; cn = c1; }
+    else { rg = 2; it -= n0 + n1; st = s2; cn = c2; }
+    key0 = st + it * BN;
+    nk = min(BN, cn - it * BN);
   }
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ Item make_item(const Params& p, int i) {
+  Item m;
+  const int pair = p.n_pairs - 1 - i / p.n_units;   // late (heavy) tokens first
+  m.u = i % p.n_units;
+  m.b = m.u / p.Hkv;
+  m.h = m.u % p.Hkv;
+  m.t0 = pair * 2 * p.TOK;
+  m.t_last = min(m.t0 + 2 * p.TOK - 1, p.T - 1);
+  const long long crow = (long long)m.u * p.T;
+  const int n_first = (m.t0 >= p.window) ? p.cnt[crow + m.t0 - p.window] : 0;
+  const int n_last = (m.t_last >= p.window) ? p.cnt[crow + m.t_last - p.window] : 0;
+  const int lo_min = n_first - p.cap > 0 ? n_first - p.cap : 0;
+  int nsink = m.t_last - p.window + 1;
+  nsink = nsink < 0 ? 0 : (nsink > p.sink ? p.sink : nsink);
+  nsink = nsink > p.T ? p.T : nsink;
+  int r_start = p.sink + lo_min, r_count = (p.cap > 0 && n_last > lo_min) ? n_last - lo_min : 0;
+  if (nsink > 0 && r_count > 0 && r_start - nsink < BN / 2) {   // one slot range [0, end)
+    r_count += r_start;
+    r_start = 0;
+    nsink = 0;
+  }
+  const int w_lo = m.t0 - p.window + 1 > 0 ? m.t0 - p.window + 1 : 0;
+  m.s0 = 0; m.c0 = nsink; m.n0 = (nsink + BN - 1) / BN;
+  m.s1 = r_start; m.c1 = r_count; m.n1 = (r_count + BN - 1) / BN;
+  m.s2 = w_lo; m.c2 = m.t_last - w_lo + 1;
+  m.total = m.n0 + m.n1 + (m.c2 + BN - 1) / BN;
+  return m;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
@@ -225,46 +298,22 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (tid == 0) record_error(p.err, LTE_ERR_DEVICE, 110);
     return;
   }
-  // ---- tile geometry (identical in every thread)
-  const int n_qt = (p.T + p.TOK - 1) / p.TOK;
-  const int t0 = (n_qt - 1 - (int)blockIdx.x) * p.TOK;      // heavy (late) tiles first
-  const int h = blockIdx.y, b = blockIdx.z, u = b * p.Hkv + h;
-  const int t_last = min(t0 + p.TOK - 1, p.T - 1);
-  const long long crow = (long long)u * p.T;
-  Tiles tl;
-  {
-    const int n_first = (t0 >= p.window) ? p.cnt[crow + t0 - p.window] : 0;
-    const int n_last = (t_last >= p.window) ? p.cnt[crow + t_last - p.window] : 0;
-    const int lo_min = n_first - p.cap > 0 ? n_first - p.cap : 0;
-    int nsink = t_last - p.window + 1;
-    nsink = nsink < 0 ? 0 : (nsink > p.sink ? p.sink : nsink);
-    nsink = nsink > p.T ? p.T : nsink;
-    int r_start = p.sink + lo_min, r_count = (p.cap > 0 && n_last > lo_min) ? n_last - lo_min : 0;
-    if (nsink > 0 && r_count > 0 && r_start - nsink < BN / 2) {   // one slot range [0, end)
-      r_count += r_start;
-      r_start = 0;
-      nsink = 0;
-    }
-    const int w_lo = t0 - p.window + 1 > 0 ? t0 - p.window + 1 : 0;
-    tl.start[0] = 0; tl.count[0] = nsink;
-    tl.start[1] = r_start; tl.count[1] = r_count;
-    tl.start[2] = w_lo; tl.count[2] = t_last - w_lo + 1;
-    tl.total = 0;
-    for (int i = 0; i < 3; ++i) { tl.ntile[i] = (tl.count[i] + BN - 1) / BN; tl.total += tl.ntile[i]; }
-  }
-  const int n_tiles = tl.total;
-
   if (tid == 0) {
-    mbar_init(bar(B_Q), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(B_KF + s), 1);
-      mbar_init(bar(B_VF + s), 1);
-      mbar_init(bar(B_KVE + s), 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(bar(B_KF + st), 1);
+      mbar_init(bar(B_VF + st), 1);
+      mbar_init(bar(B_KE + st), 1);
+      mbar_init(bar(B_VE + st), 1);
     }
-    mbar_init(bar(B_SF), 1);
-    mbar_init(bar(B_SFREE), 128);
-    mbar_init(bar(B_PF), 128);
-    mbar_init(bar(B_PVD), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(B_QF + x), 1);
+      mbar_init(bar(B_QE + x), 1);
+      mbar_init(bar(B_SF + x), 1);
+      mbar_init(bar(B_SFREE + x), 128);
+      mbar_init(bar(B_PF + x), 128);
+      mbar_init(bar(B_PVD + x), 1);
+      mbar_init(bar(B_OE + x), 128);
+    }
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -282,211 +331,280 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ======================= TMA producer
-    if (lane == 0) {
-      int issued = 0;
-      mbar_expect_tx(bar(B_Q), kQBytes);
-      tma_load_4d(sbase + kOffQ, &tm_q, bar(B_Q), 0, h * p.G, t0, b);
-      tma_load_4d(sbase + kOffQ + kQHalf, &tm_q, bar(B_Q), 64, h * p.G, t0, b);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j & 1, n = j >> 1;
-        if (j >= kStages && !mbar_wait(bar(B_KVE + s), (n - 1) & 1, abort_flag, p.err, 104)) break;
-        int rg, key0, nk;
-        tl.at(j, rg, key0, nk);
-        const uint32_t kd = sbase + kOffKV + s * 2 * kKVBytes, vd = kd + kKVBytes;
-        mbar_expect_tx(bar(B_KF + s), kKVBytes);
-        if (rg == 2) {
-          tma_load_4d(kd, &tm_k, bar(B_KF + s), 0, h, key0, b);
-          tma_load_4d(kd + kKVHalf, &tm_k, bar(B_KF + s), 64, h, key0, b);
-        } else {
-          tma_load_3d(kd, &tm_kc, bar(B_KF + s), 0, key0, u);
-          tma_load_3d(kd + kKVHalf, &tm_kc, bar(B_KF + s), 64, key0, u);
-        }
-        mbar_expect_tx(bar(B_VF + s), kKVBytes);
-        if (rg == 2) {
-          tma_load_4d(vd, &tm_v, bar(B_VF + s), 0, h, key0, b);
-          tma_load_4d(vd + kKVHalf, &tm_v, bar(B_VF + s), 64, h, key0, b);
-        } else {
-          tma_load_3d(vd, &tm_vc, bar(B_VF + s), 0, key0, u);
-          tma_load_3d(vd + kKVHalf, &tm_vc, bar(B_VF + s), 64, key0, u);
-        }
-        issued = j + 1;
+    // ============================================================ TMA producer
+    // (all 32 lanes run the loop and wait; one elected lane issues)
+    int g = 0, it = 0, issued_k = 0, issued_v = 0, issued_q = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
+      const Item m = make_item(p, i);
+      const int qb = it & 1;
+      if (it >= 2 && !(ok = wwait(bar(B_QE + qb), ((it >> 1) - 1) & 1, abort_flag, p.err, 201)))
+        break;
+      if (elect_one()) {
+        mbar_expect_tx(bar(B_QF + qb), kQBuf);
+        for (int x = 0; x < 2; ++x)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + kOffQ + qb * kQBuf + x * kQTile + hf * kQHalf, &tm_q,
+                        bar(B_QF + qb), hf * 64, m.h * p.G, m.t0 + x * p.TOK, m.b);
       }
-      // drain: every issued copy has landed before the CTA may exit
-      mbar_drain(bar(B_Q), 0);
-      for (int j = issued - kStages > 0 ? issued - kStages : 0; j < issued; ++j) {
-        mbar_drain(bar(B_KF + (j & 1)), (j >> 1) & 1);
-        mbar_drain(bar(B_VF + (j & 1)), (j >> 1) & 1);
+      __syncwarp();
+      issued_q = it + 1;
+      for (int j = 0; j < m.total; ++j, ++g) {
+        const int st = g % kStages, use = g / kStages;
+        int rg, key0, nk;
+        m.tile(j, rg, key0, nk);
+        const uint32_t kd = sbase + kOffKV + st * 2 * kKV, vd = kd + kKV;
+        // K slot frees when both S MMAs of its last tile are done, V slot when both PV are
+        if (use >= 1 && !(ok = wwait(bar(B_KE + st), (use - 1) & 1, abort_flag, p.err, 202)))
+          break;
+        if (elect_one()) {
+          mbar_expect_tx(bar(B_KF + st), kKV);
+          for (int hf = 0; hf < 2; ++hf) {
+            if (rg == 2) tma_load_4d(kd + hf * kKVHalf, &tm_k, bar(B_KF + st), hf * 64, m.h, key0, m.b);
+            else tma_load_3d(kd + hf * kKVHalf, &tm_kc, bar(B_KF + st), hf * 64, key0, m.u);
+          }
+        }
+        __syncwarp();
+        issued_k = g + 1;
+        if (use >= 1 && !(ok = wwait(bar(B_VE + st), (use - 1) & 1, abort_flag, p.err, 203)))
+          break;
+        if (elect_one()) {
+          mbar_expect_tx(bar(B_VF + st), kKV);
+          for (int hf = 0; hf < 2; ++hf) {
+            if (rg == 2) tma_load_4d(vd + hf * kKVHalf, &tm_v, bar(B_VF + st), hf * 64, m.h, key0, m.b);
+            else tma_load_3d(vd + hf * kKVHalf, &tm_vc, bar(B_VF + st), hf * 64, key0, m.u);
+          }
+        }
+        __syncwarp();
+        issued_v = g + 1;
       }
     }
+    // drain: every issued copy has landed before the CTA may exit
+    for (int q = issued_q - 2 > 0 ? issued_q - 2 : 0; q < issued_q; ++q)
+      mbar_drain(bar(B_QF + (q & 1)), (q >> 1) & 1);
+    for (int q = issued_k - kStages > 0 ? issued_k - kStages : 0; q < issued_k; ++q)
+      mbar_drain(bar(B_KF + q % kStages), (q / kStages) & 1);
+    for (int q = issued_v - kStages > 0 ? issued_v - kStages : 0; q < issued_v; ++q)
+      mbar_drain(bar(B_VF + q % kStages), (q / kStages) & 1);
   } else if (warp == 1) {
-    // ======================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc(BM, BN, false);
-      constexpr uint32_t idO = idesc(BM, HD, true);
-      const uint32_t qa = sbase + kOffQ;
-      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, p.err, 101);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j & 1;
-          if (j >= 1 && !(ok = mbar_wait(bar(B_SFREE), (j - 1) & 1, abort_flag, p.err, 102))) break;
-          if (!(ok = mbar_wait(bar(B_KF + s), (j >> 1) & 1, abort_flag, p.err, 101))) break;
-          tc_fence_after();
-          const uint32_t kb = sbase + kOffKV + s * 2 * kKVBytes;
+    // ============================================================ MMA issuer
+    // (all 32 lanes run the loop and wait; one elected lane issues)
+    constexpr uint32_t idS = idesc(BM, BN, false);
+    constexpr uint32_t idO = idesc(BM, HD, true);
+    // descriptors are built once; the start-address field (addr >> 4, low
+    // 14 bits) is then advanced by plain adds (shared addresses < 256 KiB)
+    const uint64_t dq0 = sdesc(sbase + kOffQ, 16, 1024);
+    const uint64_t dk0 = sdesc(sbase + kOffKV, 16, 1024);
+    const uint64_t dv0 = sdesc(sbase + kOffKV + kKV, kKVHalf, 1024);
+    int g0 = 0, it = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
+      const Item m = make_item(p, i);
+      const int qb = it & 1;
+      if (!(ok = wwait(bar(B_QF + qb), (it >> 1) & 1, abort_flag, p.err, 211))) break;
+      const uint64_t dq = dq0 + ((qb * kQBuf) >> 4);
+      for (int j = 0; j <= m.total; ++j) {
+        if (j < m.total) {
+          const int g = g0 + j, st = g % kStages;
+          if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
+          const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
+          for (int x = 0; x < 2; ++x) {
+            if (g >= 1 && !(ok = wwait(bar(B_SFREE + x), (g - 1) & 1, abort_flag, p.err, 213)))
+              break;
+            tc_fence_after();
+            const uint64_t dqx = dq + ((x * kQTile) >> 4);
+            const uint32_t ds = tmem + col_s(x);
+            if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t a = sdesc(qa + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024);
-            const uint64_t bb = sdesc(kb + (kk >> 2) * kKVHalf + (kk & 3) * 32, 16, 1024);
-            mma_f16(tmem + kColS, a, bb, idS, kk > 0);
+              for (int kk = 0; kk < HD / 16; ++kk) {
+                const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
+                const uint32_t offk = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+                mma_f16(ds, dqx + off, dk + offk, idS, kk > 0);
+              }
+              mma_commit(bar(B_SF + x));
+            }
+            __syncwarp();
           }
-          mma_commit(bar(B_SF));
+          if (!ok) break;
+          if (elect_one()) {
+            mma_commit(bar(B_KE + st));
+            if (j == m.total - 1) mma_commit(bar(B_QE + qb));
+          }
+          __syncwarp();
         }
         if (j >= 1) {
-          const int i = j - 1, s = i & 1;
-          if (!(ok = mbar_wait(bar(B_PF), i & 1, abort_flag, p.err, 102))) break;
-          if (!(ok = mbar_wait(bar(B_VF + s), (i >> 1) & 1, abort_flag, p.err, 101))) break;
-          tc_fence_after();
-          const uint32_t vb = sbase + kOffKV + s * 2 * kKVBytes + kKVBytes;
-          const uint32_t pa = sbase + kOffP;
+          const int g = g0 + j - 1, st = g % kStages;
+          if (!(ok = wwait(bar(B_VF + st), (g / kStages) & 1, abort_flag, p.err, 214))) break;
+          const uint64_t dv = dv0 + ((st * 2 * kKV) >> 4);
+          for (int x = 0; x < 2; ++x) {
+            if (!(ok = wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215))) break;
+            if (j == 1 && it >= 1 &&
+                !(ok = wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216)))
+              break;
+            tc_fence_after();
+            const uint32_t tp = tmem + col_p(x);      // P: A operand in TMEM
+            const uint32_t dO = tmem + col_o(x);
+            const uint32_t acc0 = j > 1 ? 1u : 0u;
+            if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t a = sdesc(pa + kk * 32, 16, 1024);
-            const uint64_t bb = sdesc(vb + kk * 2048, kKVHalf, 1024);
-            mma_f16(tmem + kColO, a, bb, idO, (i > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BN / 16; ++kk)
+                mma_f16_ts(dO, tp + 8 * kk, dv + ((kk * 2048) >> 4), idO, kk > 0 ? 1u : acc0);
+              mma_commit(bar(B_PVD + x));
+            }
+            __syncwarp();
           }
-          mma_commit(bar(B_KVE + s));
-          mma_commit(bar(B_PVD));
+          if (!ok) break;
+          if (elect_one()) mma_commit(bar(B_VE + st));
+          __syncwarp();
         }
       }
-      // all MMAs issued by this thread are complete before TMEM is released
-      mma_commit(bar(B_FIN));
-      mbar_drain(bar(B_FIN), 0);
+      g0 += m.total;
     }
+    if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
+    __syncwarp();
+    mbar_drain(bar(B_FIN), 0);
   } else {
-    // ======================= softmax + epilogue (warps 2..5, one row per thread)
+    // ============================================================ softmax + epilogue
+    const int x = (warp - 2) >> 2;                 // Q tile of this warpgroup
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const int g = row % p.G, tt = t0 + row / p.G;
-    const bool row_ok = tt < p.T;
-    int hi_t = 0;
-    if (row_ok && tt >= p.window) hi_t = p.cnt[crow + tt - p.window];
-    const int lo_t = hi_t - p.cap > 0 ? hi_t - p.cap : 0;
-    float m_ref = -INFINITY, l_sum = 0.f;
+    const uint32_t colS = col_s(x), colO = col_o(x), colP = col_p(x);
+    const int g_in_row = row % p.G;
+    int g0 = 0;
     bool ok = true;
-    uint8_t* prow = smem + kOffP + row * 128;
-    for (int j = 0; j < n_tiles; ++j) {
-      ok = mbar_wait(bar(B_SF), j & 1, abort_flag, p.err, 103);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;     // tcgen05.ld is warp-collective
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(lane_addr + kColS, sr[0]);
-      tmem_ld32(lane_addr + kColS + 32, sr[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_SFREE));
-      int rg, key0, nk;
-      tl.at(j, rg, key0, nk);
-      float s[64];
+    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x) {
+      const Item m = make_item(p, i);
+      const int tt = m.t0 + x * p.TOK + row / p.G;
+      const bool row_ok = tt < p.T;
+      int hi_t = 0;
+      if (row_ok && tt >= p.window) hi_t = p.cnt[(long long)m.u * p.T + tt - p.window];
+      const int lo_t = hi_t - p.cap > 0 ? hi_t - p.cap : 0;
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < m.total; ++j) {
+        const int g = g0 + j;
+        ok = mbar_wait(bar(B_SF + x), g & 1, abort_flag, p.err, 221);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;     // tcgen05.ld is warp-collective
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(lane_addr + colS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(lane_addr + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE + x));
+        int rg, key0, nk;
+        m.tile(j, rg, key0, nk);
+        float s[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]) * p.scale_log2;
-      // attended-set predicate (skipped when the whole tile is inside S_t)
-      bool full;
-      if (rg == 2) full = nk == BN && key0 > tt - p.window && key0 + BN - 1 <= tt;
-      else full = nk == BN && key0 >= p.sink && key0 - p.sink >= lo_t && key0 - p.sink + BN <= hi_t;
-      full = full && row_ok;
-      if (!full) {
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
+        // attended-set predicate, skipped when the whole tile is inside S_t
+        bool full;
+        if (rg == 2) full = nk == BN && key0 > tt - p.window && key0 + BN - 1 <= tt;
+        else full = nk == BN && key0 >= p.sink && key0 - p.sink >= lo_t && key0 - p.sink + BN <= hi_t;
+        if (!(full && row_ok)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = key0 + c;
-          bool in;
-          if (rg == 2) in = key <= tt && key > tt - p.window;
-          else if (key < p.sink) in = key <= tt - p.window;
-          else in = key - p.sink >= lo_t && key - p.sink < hi_t;
-          in = in && c < nk && row_ok;
-          if (!in) s[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c) {
+            const int key = key0 + c;
+            bool in;
+            if (rg == 2) in = key <= tt && key > tt - p.window;
+            else if (key < p.sink) in = key <= tt - p.window;
+            else in = key - p.sink >= lo_t && key - p.sink < hi_t;
+            if (!(in && c < nk && row_ok)) s[c] = -INFINITY;
+          }
         }
-      }
-      float mx = -INFINITY;
+        float m8[8];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
-      // lazy rescale: move the reference max only when it grew by > 8 (x256)
-      const bool need = mx > m_ref + 8.f;
-      float corr = 1.f;
-      if (need) {
-        corr = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-        m_ref = mx;
-        l_sum *= corr;
+        for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        mx *= p.scale_log2;                        // scale > 0: max commutes with it
+        const bool need = mx > m_ref + 8.f;        // lazy rescale (x256 headroom)
+        float corr = 1.f;
+        if (need) {
+          corr = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+          m_ref = mx;
+          l_sum *= corr;
+        }
+        const bool any_rescale = __any_sync(0xffffffffu, need && corr != 0.f);
+        if (g >= 1) {      // P buffer free, and O current when this item already ran PV
+          ok = mbar_wait(bar(B_PVD + x), (g - 1) & 1, abort_flag, p.err, 222);
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+        }
+        if (any_rescale) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t orr[32];
+            tmem_ld32(lane_addr + colO + c0, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
+            tmem_st32(lane_addr + colO + c0, orr);
+          }
+          tmem_wait_st();
+        }
+        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(-mu, -mu);
+        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+        uint32_t pk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          float2 z = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), sc2, nm2);
+          z.x = ex2(z.x);
+          z.y = ex2(z.y);
+          acc2[c2 & 3] = __fadd2_rn(acc2[c2 & 3], z);
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(z.x, z.y);
+          pk[c2] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+        tmem_st32(lane_addr + colP, pk);
+        const float2 a01 = __fadd2_rn(acc2[0], acc2[1]), a23 = __fadd2_rn(acc2[2], acc2[3]);
+        const float2 a = __fadd2_rn(a01, a23);
+        l_sum += a.x + a.y;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PF + x));
       }
-      const bool any_rescale = __any_sync(0xffffffffu, need && corr != 0.f);
-      if (j >= 1) {     // PV_{j-1} done: P buffer free, O up to date
-        ok = mbar_wait(bar(B_PVD), (j - 1) & 1, abort_flag, p.err, 103);
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, lse; then hand O back to the MMA warp
+      const int g_last = g0 + m.total - 1;
+      if (m.total > 0) {
+        ok = mbar_wait(bar(B_PVD + x), g_last & 1, abort_flag, p.err, 223);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         tc_fence_after();
-      }
-      if (any_rescale) {
+        const float inv = 1.f / l_sum;
+        __nv_bfloat16* orow = p.o + (long long)m.b * p.os.b + (long long)(row_ok ? tt : 0) * p.os.t +
+                              (long long)(m.h * p.G + g_in_row) * p.os.h;
 #pragma unroll 1
         for (int c0 = 0; c0 < HD; c0 += 32) {
           uint32_t orr[32];
-          tmem_ld32(lane_addr + kColO + c0, orr);
+          tmem_ld32(lane_addr + colO + c0, orr);
           tmem_wait_ld();
+          if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
-          tmem_st32(lane_addr + kColO + c0, orr);
-        }
-        tmem_wait_st();
-      }
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float psum = 0.f;
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2f(s[c8 * 8 + 2 * e] - mu);
-          const float p1 = exp2f(s[c8 * 8 + 2 * e + 1] - mu);
-          psum += p0 + p1;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<uint32_t*>(&v2);
-        }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (row & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      l_sum += psum;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(bar(B_PF));
-    }
-    // ---- epilogue: O / l -> bf16, lse
-    if (ok && n_tiles > 0) ok = mbar_wait(bar(B_PVD), (n_tiles - 1) & 1, abort_flag, p.err, 103);
-    if (__all_sync(0xffffffffu, ok) && n_tiles > 0) {
-      tc_fence_after();
-      const float inv = 1.f / l_sum;
-      __nv_bfloat16* orow = p.o + (long long)b * p.os.b + (long long)(row_ok ? tt : 0) * p.os.t +
-                            (long long)(h * p.G + g) * p.os.h;
-#pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t orr[32];
-        tmem_ld32(lane_addr + kColO + c0, orr);
-        tmem_wait_ld();
-        if (row_ok) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 v;
-            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[e + 2 * f]) * inv,
-                                                        __uint_as_float(orr[e + 2 * f + 1]) * inv);
-              w[f] = *reinterpret_cast<uint32_t*>(&v2);
+              for (int f = 0; f < 4; ++f) {
+                __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[e + 2 * f]) * inv,
+                                                          __uint_as_float(orr[e + 2 * f + 1]) * inv);
+                w[f] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+              *reinterpret_cast<uint4*>(orow + c0 + e) = v;
             }
-            *reinterpret_cast<uint4*>(orow + c0 + e) = v;
           }
         }
+        if (row_ok && p.lse != nullptr)
+          p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
+              (m_ref + log2f(l_sum)) * 0.69314718055994531f;
       }
-      if (row_ok && p.lse != nullptr)
-        p.lse[((long long)b * p.Hq + h * p.G + g) * p.T + tt] =
-            (m_ref + log2f(l_sum)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(bar(B_OE + x));
+      g0 += m.total;
     }
   }
   tc_fence_before();
@@ -529,8 +647,8 @@ static bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t*
 
 bool attn_prefill_tc_supported(const lte_dims* d) {
   const int G = d->Hq / d->Hkv;
-  return d->dtype == LTE_BF16 && d->D == tc::HD && (G == 1 || G == 2 || G == 4 || G == 8 ||
-                                                    G == 16);
+  return d->dtype == LTE_BF16 && d->D == tc::HD &&
+         (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
 cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
@@ -563,13 +681,19 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   Params p{};
   p.T = d->T; p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = G; p.TOK = TOK;
   p.sink = d->sink; p.window = d->window; p.cap = d->cap;
+  p.n_pairs = (d->T + 2 * TOK - 1) / (2 * TOK);
+  p.n_units = d->B * d->Hkv;
+  p.n_items = p.n_pairs * p.n_units;
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.cnt = a.cnt;
   p.o = (__nv_bfloat16*)a.o; p.os = a.os; p.lse = a.lse; p.err = a.err;
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((d->T + TOK - 1) / TOK, d->Hkv, d->B);
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.n_items < n_sm ? p.n_items : n_sm;
   attn_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mkc, mvc, p);
   return cudaGetLastError();
 }
