@@ -255,8 +255,12 @@ lte_status lte_read_device_error(const void* workspace, int32_t* code, int32_t* 
  *   S_t = S_{t-1} diag(a_t) + v_t k_t^T,  o_t = S_t q_t.
  * q, k: [B,T,H,dk]; v, o: [B,T,H,dv] (dtype); a: fp32 [B,T,H,dk] in (0,1];
  * state: fp32 [B,H,dv,dk], read as S_0 and overwritten with S_T.
- * Supported: dk = dv = 128 (bf16) or dk, dv <= 128 (fp32); T % 64 == 0 for
- * bf16 prefill.  Prefill is chunk-wise (64 tokens); decode is one step.
+ * Supported: dk = dv = 128; prefill bf16 with T % 64 == 0 (chunk-wise, 64
+ * tokens per chunk, bf16 operands with fp32 accumulation and an fp32 state);
+ * decode bf16 or fp32 (one step, fp32 arithmetic).  Other shapes return
+ * LTE_ERR_UNSUPPORTED.  The chunk form multiplies q and k by exp(+-sum log a)
+ * over at most 32 tokens, so it needs the product of any 32 consecutive
+ * gates of a channel to stay above ~1e-30 (fp32/bf16 exponent range).
  * ------------------------------------------------------------------------- */
 lte_status lte_gla_prefill(int32_t B, int32_t T, int32_t H, int32_t dk, int32_t dv,
                            int32_t dtype, const void* q, const void* k, const void* v,

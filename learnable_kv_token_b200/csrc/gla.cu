@@ -1,18 +1,365 @@
-// Gated linear attention (the hybrid's companion layer): placeholder until
-// the chunk-wise kernels land; both entry points report "unsupported".
+// Gated linear attention, the linear-attention layer of the laLTE hybrid.
+//
+// "Sparse Linear Attention: Viewing SWA from the Perspective of Linear
+// Attention", section "Background: Linear attention": the state is decayed,
+// the value-key outer product is written, the query reads it:
+//   S_t = S_{t-1} diag(a_t) + v_t k_t^T,   o_t = S_t q_t    (S: d_v x d_k).
+// The hybrid that interleaves this layer with LTE is the one of "Alleviating
+// Forgetfulness of Linear Attention by Hybrid Sparse Attention and
+// Contextualized Learnable Token Eviction" (TL;DR, Abstract).
+//
+// Prefill, chunk-wise (L = 64 tokens).  With b_t = sum_{i<=t} log a_i over
+// the chunk (per key channel) and S_0 the state before the chunk:
+//   o_t  = S_0 (q_t * e^{b_t}) + sum_{s<=t} [(q_t * e^{b_t-b_m}) . (k_s * e^{b_m-b_s})] v_s
+//   S_L  = S_0 diag(e^{b_{L-1}}) + sum_s v_s (k_s * e^{b_{L-1}-b_s})^T
+// (b_m = b at the chunk middle halves the exponent range of the intra-chunk
+// factors).  One CTA per (batch, head) walks the chunks in order; the fp32
+// state stays in MMA accumulator registers for the whole sequence and a bf16
+// copy in shared memory feeds the S_0 q products.  Per chunk: the decay
+// factors (fp32 cumulative log-gates), A = Q~ K~^T masked causal (64x64),
+// O = A V + Qbar S_0^T (64x128), S <- S diag(e^{b_{L-1}}) + V^T Khat (128x128),
+// all on m16n8k16 bf16 MMAs with fp32 accumulation.
+//
+// Decode: one CTA per (batch, head) streams the 128x128 fp32 state once
+// (read, decay, add the outer product, write) with 16-byte accesses and
+// reduces the row-query dot products with warp shuffles.
+#include <math.h>
+
 #include "lte_common.cuh"
 #include "lte_internal.h"
 
 namespace lte {
+namespace gla {
 
-cudaError_t gla_prefill(int, int, int, int, int, int, const void*, const void*, const void*,
-                        const float*, void*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int L = 64, DK = 128, DV = 128;
+constexpr int kThreads = 256;
+
+// shared-memory layout (bytes); [rows][128] bf16 tiles have 256-byte rows with
+// the 16-byte chunks XOR-swizzled by (row mod 8)
+constexpr uint32_t kQbar = 0;                 // q * e^{b_t}          [64][128]
+constexpr uint32_t kQtil = kQbar + 16384;     // q * e^{b_t - b_m}    [64][128]
+constexpr uint32_t kKtil = kQtil + 16384;     // k * e^{b_m - b_s}    [64][128]
+constexpr uint32_t kKhat = kKtil + 16384;     // k * e^{b_last - b_s} [64][128]
+constexpr uint32_t kV = kKhat + 16384;        // v                    [64][128]
+constexpr uint32_t kA = kV + 16384;           // masked A (bf16)      [64][64], 128-byte rows
+constexpr uint32_t kSb = kA + 8192;           // state copy (bf16)    [128][128]
+constexpr uint32_t kLam = kSb + 32768;        // e^{b_last} per key channel (fp32)
+constexpr uint32_t kTot = kLam + 512;         // log-gate totals of each half (2 x 128 fp32)
+constexpr uint32_t kSmem = kTot + 2 * 128 * 4;
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// byte offset of element (r, c) in a swizzled bf16 tile with `rowb`-byte rows
+__device__ __forceinline__ uint32_t sw(int r, int c, int rowb) {
+  return (uint32_t)(r * rowb + ((((c >> 3) ^ (r & 7)) & (rowb / 16 - 1)) << 4) + (c & 7) * 2);
+}
+__device__ __forceinline__ void ldsm4(uint32_t a, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t a, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void mma(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
 }
 
-cudaError_t gla_decode(int, int, int, int, int, const void*, const void*, const void*,
-                       const float*, void*, float*, cudaStream_t) {
-  return cudaErrorNotSupported;
+// A fragment (16 x 16) from a [m][k]-stored tile (row-major A)
+__device__ __forceinline__ void frag_a(uint32_t base, int rowb, int m0, int k0, int lane,
+                                       uint32_t* r) {
+  const int row = m0 + (lane & 7) + ((lane >> 3) & 1) * 8, col = k0 + (lane >> 4) * 8;
+  ldsm4(base + sw(row, col, rowb), r);
+}
+// A fragment (16 x 16) from a [k][m]-stored tile (A^T in memory)
+__device__ __forceinline__ void frag_a_t(uint32_t base, int rowb, int m0, int k0, int lane,
+                                         uint32_t* r) {
+  const int row = k0 + (lane & 7) + (lane >> 4) * 8, col = m0 + ((lane >> 3) & 1) * 8;
+  ldsm4t(base + sw(row, col, rowb), r);
+}
+// B fragments of two n8 tiles (k16 x n16) from a [n][k]-stored tile
+__device__ __forceinline__ void frag_b(uint32_t base, int rowb, int n0, int k0, int lane,
+                                       uint32_t* r) {
+  const int row = n0 + (lane & 7) + (lane >> 4) * 8, col = k0 + ((lane >> 3) & 1) * 8;
+  ldsm4(base + sw(row, col, rowb), r);
+}
+// B fragments of two n8 tiles (k16 x n16) from a [k][n]-stored tile
+__device__ __forceinline__ void frag_b_t(uint32_t base, int rowb, int n0, int k0, int lane,
+                                         uint32_t* r) {
+  const int row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8, col = n0 + (lane >> 4) * 8;
+  ldsm4t(base + sw(row, col, rowb), r);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                   const float* __restrict__ a, __nv_bfloat16* __restrict__ o,
+                   float* __restrict__ state) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int bh = blockIdx.x, b = bh / H, hd = bh % H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, cq = lane & 3;               // accumulator row / column pair
+  const uint32_t s0 = saddr(sm);
+  float* lam = reinterpret_cast<float*>(sm + kLam);
+  float* tot = reinterpret_cast<float*>(sm + kTot);
+  const long long row_stride = (long long)H * DK;        // elements between tokens
+  const long long base_bh = (long long)b * T * row_stride + (long long)hd * DK;
+
+  // ---- state: fp32 master in accumulators (warp: rows 32*(w%4)..+32, cols 64*(w/4)..+64)
+  const int sm0 = (warp & 3) * 32, sn0 = (warp >> 2) * 64;
+  float* st = state + (long long)bh * DV * DK;
+  float sacc[2][8][4];
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 8; ++ni)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = sm0 + mi * 16 + gq + (e >> 1) * 8, j = sn0 + ni * 8 + cq * 2 + (e & 1);
+        sacc[mi][ni][e] = st[i * DK + j];
+      }
+
+  for (int t0 = 0; t0 < T; t0 += L) {
+    // bf16 copy of S_0 for the Qbar S_0^T product
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < 8; ++ni)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int i = sm0 + mi * 16 + gq + hf * 8, j = sn0 + ni * 8 + cq * 2;
+          *reinterpret_cast<uint32_t*>(sm + kSb + sw(i, j, 256)) =
+              pack(sacc[mi][ni][hf * 2], sacc[mi][ni][hf * 2 + 1]);
+        }
+    // raw q -> Qbar slot, k -> Khat slot, v -> V (16-byte async copies)
+    for (int c = tid; c < L * 16; c += kThreads) {
+      const int r = c >> 4, cc = (c & 15) * 8;
+      const long long g = base_bh + (long long)(t0 + r) * row_stride + cc;
+      cp16(s0 + kQbar + sw(r, cc, 256), q + g);
+      cp16(s0 + kKhat + sw(r, cc, 256), k + g);
+      cp16(s0 + kV + sw(r, cc, 256), v + g);
+    }
+    asm volatile("cp.async.commit_group;\n" ::);
+    // cumulative log-gates: thread (j, half) covers 32 tokens of key channel j
+    const int j = tid & 127, half = tid >> 7;
+    float bl[32];
+    {
+      float run = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int t = t0 + half * 32 + i;
+        run += __logf(a[base_bh + (long long)t * row_stride + j]);
+        bl[i] = run;
+      }
+      if (half == 0) tot[j] = run;           // b at the chunk middle (token 31)
+      if (half == 1) tot[128 + j] = run;     // second-half total
+    }
+    asm volatile("cp.async.wait_group 0;\n" ::);
+    __syncthreads();
+    {
+      const float bm = tot[j];
+      const float blast = tot[j] + tot[128 + j];
+      if (half == 0) lam[j] = __expf(blast);
+      const float off = half ? bm : 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = half * 32 + i;
+        const float bt = bl[i] + off;
+        const uint32_t o16 = sw(r, j, 256);
+        __nv_bfloat16* pq = reinterpret_cast<__nv_bfloat16*>(sm + kQbar + o16);
+        __nv_bfloat16* pk = reinterpret_cast<__nv_bfloat16*>(sm + kKhat + o16);
+        const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk);
+        *reinterpret_cast<__nv_bfloat16*>(sm + kQtil + o16) = __float2bfloat16_rn(qv * __expf(bt - bm));
+        *reinterpret_cast<__nv_bfloat16*>(sm + kKtil + o16) = __float2bfloat16_rn(kv * __expf(bm - bt));
+        *pq = __float2bfloat16_rn(qv * __expf(bt));
+        *pk = __float2bfloat16_rn(kv * __expf(blast - bt));
+      }
+    }
+    __syncthreads();
+
+    // ---- A = Q~ K~^T (64 x 64), causal mask s <= t, bf16 -> shared
+    {
+      const int am0 = (warp & 3) * 16, an0 = (warp >> 2) * 32;
+      float acc[4][4] = {};
+#pragma unroll
+      for (int kk = 0; kk < DK; kk += 16) {
+        uint32_t fa[4];
+        frag_a(s0 + kQtil, 256, am0, kk, lane, fa);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          uint32_t fb[4];
+          frag_b(s0 + kKtil, 256, an0 + np * 16, kk, lane, fb);
+          mma(acc[np * 2], fa, fb[0], fb[1]);
+          mma(acc[np * 2 + 1], fa, fb[2], fb[3]);
+        }
+      }
+#pragma unroll
+      for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int t = am0 + gq + hf * 8, s = an0 + ni * 8 + cq * 2;
+          const float x0 = s <= t ? acc[ni][hf * 2] : 0.f;
+          const float x1 = s + 1 <= t ? acc[ni][hf * 2 + 1] : 0.f;
+          *reinterpret_cast<uint32_t*>(sm + kA + sw(t, s, 128)) = pack(x0, x1);
+        }
+    }
+    __syncthreads();
+
+    // ---- O = A V + Qbar S_0^T (64 x 128) -> bf16 output
+    {
+      const int om0 = (warp & 3) * 16, on0 = (warp >> 2) * 64;
+      float acc[8][4] = {};
+#pragma unroll
+      for (int kk = 0; kk < L; kk += 16) {
+        uint32_t fa[4];
+        frag_a(s0 + kA, 128, om0, kk, lane, fa);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t fb[4];
+          frag_b_t(s0 + kV, 256, on0 + np * 16, kk, lane, fb);
+          mma(acc[np * 2], fa, fb[0], fb[1]);
+          mma(acc[np * 2 + 1], fa, fb[2], fb[3]);
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < DK; kk += 16) {
+        uint32_t fa[4];
+        frag_a(s0 + kQbar, 256, om0, kk, lane, fa);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          uint32_t fb[4];
+          frag_b(s0 + kSb, 256, on0 + np * 16, kk, lane, fb);
+          mma(acc[np * 2], fa, fb[0], fb[1]);
+          mma(acc[np * 2 + 1], fa, fb[2], fb[3]);
+        }
+      }
+#pragma unroll
+      for (int ni = 0; ni < 8; ++ni)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int t = om0 + gq + hf * 8, i = on0 + ni * 8 + cq * 2;
+          *reinterpret_cast<uint32_t*>(o + base_bh + (long long)(t0 + t) * row_stride + i) =
+              pack(acc[ni][hf * 2], acc[ni][hf * 2 + 1]);
+        }
+    }
+
+    // ---- S <- S diag(e^{b_last}) + V^T Khat  (128 x 128, K = 64 tokens)
+#pragma unroll
+    for (int ni = 0; ni < 8; ++ni) {
+      const int jj = sn0 + ni * 8 + cq * 2;
+      const float l0 = lam[jj], l1 = lam[jj + 1];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        sacc[mi][ni][0] *= l0; sacc[mi][ni][1] *= l1;
+        sacc[mi][ni][2] *= l0; sacc[mi][ni][3] *= l1;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < L; kk += 16) {
+      uint32_t fa[2][4];
+      frag_a_t(s0 + kV, 256, sm0, kk, lane, fa[0]);
+      frag_a_t(s0 + kV, 256, sm0 + 16, kk, lane, fa[1]);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t fb[4];
+        frag_b_t(s0 + kKhat, 256, sn0 + np * 16, kk, lane, fb);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+          mma(sacc[mi][np * 2], fa[mi], fb[0], fb[1]);
+          mma(sacc[mi][np * 2 + 1], fa[mi], fb[2], fb[3]);
+        }
+      }
+    }
+    __syncthreads();   // every warp is done with this chunk's tiles and S_0 copy
+  }
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 8; ++ni)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = sm0 + mi * 16 + gq + (e >> 1) * 8, jj = sn0 + ni * 8 + cq * 2 + (e & 1);
+        st[i * DK + jj] = sacc[mi][ni][e];
+      }
+}
+
+// ---------------------------------------------------------------- decode
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
+                  const TIn* __restrict__ v, const float* __restrict__ a, TIn* __restrict__ o,
+                  float* __restrict__ state) {
+  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long vb = (long long)bh * DK;
+  float q4[4], k4[4], a4[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    q4[e] = to_f32(q[vb + lane * 4 + e]);
+    k4[e] = to_f32(k[vb + lane * 4 + e]);
+    a4[e] = a[vb + lane * 4 + e];
+  }
+  float* st = state + (long long)bh * DV * DK;
+  constexpr int kRows = DV / 8;                       // rows per warp
+#pragma unroll 4
+  for (int rr = 0; rr < kRows; ++rr) {
+    const int i = warp * kRows + rr;
+    float4* p = reinterpret_cast<float4*>(st + (long long)i * DK) + lane;
+    float4 s4 = *p;
+    const float vi = to_f32(v[(long long)bh * DV + i]);
+    s4.x = fmaf(s4.x, a4[0], vi * k4[0]);
+    s4.y = fmaf(s4.y, a4[1], vi * k4[1]);
+    s4.z = fmaf(s4.z, a4[2], vi * k4[2]);
+    s4.w = fmaf(s4.w, a4[3], vi * k4[3]);
+    *p = s4;
+    float d = s4.x * q4[0] + s4.y * q4[1] + s4.z * q4[2] + s4.w * q4[3];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (lane == 0) o[(long long)bh * DV + i] = from_f32<TIn>(d);
+  }
+}
+
+}  // namespace gla
+
+cudaError_t gla_prefill(int B, int T, int H, int dk, int dv, int dtype, const void* q,
+                        const void* k, const void* v, const float* a, void* o, float* state,
+                        cudaStream_t stream) {
+  if (dtype != LTE_BF16 || dk != gla::DK || dv != gla::DV || T % gla::L != 0)
+    return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(gla::gla_prefill_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, gla::kSmem);
+  if (e != cudaSuccess) return e;
+  gla::gla_prefill_kernel<<<B * H, gla::kThreads, gla::kSmem, stream>>>(
+      T, H, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a,
+      (__nv_bfloat16*)o, state);
+  return cudaGetLastError();
+}
+
+cudaError_t gla_decode(int B, int H, int dk, int dv, int dtype, const void* q, const void* k,
+                       const void* v, const float* a, void* o, float* state,
+                       cudaStream_t stream) {
+  if (dk != gla::DK || dv != gla::DV) return cudaErrorNotSupported;
+  if (dtype == LTE_BF16)
+    gla::gla_decode_kernel<__nv_bfloat16><<<B * H, 256, 0, stream>>>(
+        H, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a,
+        (__nv_bfloat16*)o, state);
+  else
+    gla::gla_decode_kernel<float><<<B * H, 256, 0, stream>>>(
+        H, (const float*)q, (const float*)k, (const float*)v, a, (float*)o, state);
+  return cudaGetLastError();
 }
 
 }  // namespace lte

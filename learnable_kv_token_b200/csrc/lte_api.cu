@@ -258,7 +258,7 @@ lte_status lte_gla_prefill(int32_t B, int32_t T, int32_t H, int32_t dk, int32_t 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned16(o) ||
       !aligned16(state))
     return LTE_ERR_INVALID_ARG;
-  if (dk != 128 || dv != 128) return LTE_ERR_UNSUPPORTED;
+  if (dk != 128 || dv != 128 || dtype != LTE_BF16 || T % 64 != 0) return LTE_ERR_UNSUPPORTED;
   return from_cuda(lte::gla_prefill(B, T, H, dk, dv, dtype, q, k, v, a, o, state,
                                     as_stream(stream)));
 }
