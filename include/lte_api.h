@@ -218,7 +218,8 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
  * no cudaMalloc, cudaFree or other allocating routine.
  *  - Limit: returns LTE_ERR_WORKSPACE, launching nothing, when
  *    lte_workspace_bytes(d, LTE_WS_DECODE) > LTE_NOALLOC_SCRATCH_BYTES
- *    (4 MiB covers B*Hkv = 128 units x 1028 cache slots x G = 4, D = 128).
+ *    (the decode workload -- B*Hkv = 128 units, 1028 cache slots, G = 4,
+ *    D = 128 -- needs about 0.3 MB).
  *  - Set-up: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.

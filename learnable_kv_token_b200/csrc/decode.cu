@@ -1,5 +1,5 @@
-// Decode step of LTE: cache update, deferred batched scoring, split-KV
-// attention with an in-kernel log-sum-exp merge.
+// Decode step of LTE: cache update + deferred batched scoring, then a
+// persistent split-KV attention with an in-kernel log-sum-exp merge.
 //
 // "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention
 // and Contextualized Learnable Token Eviction", Fig. 3 caption: the inference
@@ -11,105 +11,188 @@
 // from the linear-state perspective": each new token overwrites one slot of
 // the window (FIFO).
 //
-// Per step (all kernels read the step index t from meta[0] on the device, so
-// the same launches replay unchanged inside a CUDA graph):
-//  1. decode_update_kernel (one CTA per (batch, KV head) unit): token t-w
-//     leaves its window slot (sink slot, retained ring, or dropped); token t
-//     takes slot t mod w.
-//  2. score_ring (score_cnn.cu): when score_batch tokens are scorable, score
-//     them from the window segment.
-//  3. decode_attn_kernel: the unit's valid slots (window, sinks, retained) are
-//     one logical key list split into chunks of 128 keys, one CTA per chunk;
-//     four warps stream 32 keys each through shared memory with cp.async and
-//     run QK^T and PV on m16n8k16 bf16 MMAs (the G query heads of the group
-//     are rows of the A operand, so each K/V byte is read once per group).
-//     Each CTA writes an (m, l, o) partial; the last CTA of a unit (atomic
-//     counter) merges them; the last unit advances meta.
+// Per step (both kernels read the step index t from meta[0] on the device, so
+// the same two launches replay unchanged inside a CUDA graph):
+//  1. decode_prep_kernel, one CTA per (batch, KV head) unit: token t-w leaves
+//     its window slot (to its sink slot, into the retained ring, or dropped),
+//     token t takes slot t mod w; then, when score_batch tokens are scorable,
+//     the same CTA scores them from the window segment (score_tile, the same
+//     arithmetic as lte_score).
+//  2. decode_attn_kernel, persistent (about one CTA per SM): the valid slots
+//     of all units form one flattened key space that is cut into equal
+//     contiguous ranges, one per CTA.  A CTA streams its range in chunks of
+//     64 keys: TMA copies (128B-swizzled) of the K, V and query rows into a
+//     5-stage ring with bounded mbarrier waits; four warps take 16 keys each and run QK^T and PV on m16n8k16
+//     bf16 MMAs (the G query heads of the group are MMA rows, so each K/V byte
+//     is read once per group) with an online softmax.  At the end of each unit
+//     the CTA writes an (m, l, o) partial; the last CTA of a unit (atomic
+//     counter) merges the partials and writes o_t and lse_t; the last unit
+//     advances meta.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include <mutex>
 
 #include "lte_common.cuh"
 #include "lte_internal.h"
+#include "score_cnn.cuh"
+#include "score_tc.cuh"
 
 namespace lte {
 
-constexpr int kDecKeysPerWarp = 32;
 constexpr int kDecWarps = 4;
-constexpr int kDecKeysPerCta = kDecKeysPerWarp * kDecWarps;
 constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecChunk = 64;            // keys per pipeline stage
+constexpr int kDecStages = 5;
+constexpr int kDecMaxEntries = 256;      // chunk list entries per CTA
+constexpr int kDecMaxParts = 8;          // CTAs sharing one unit
 
-static inline int dec_splits(const lte_dims* d) {
-  const int L = d->window + d->sink + d->cap;
-  return (L + kDecKeysPerCta - 1) / kDecKeysPerCta;
+struct DecGeom {
+  int n_ctas, per_cta, max_parts;
+};
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
 }
 
-// workspace layout after the error word: partials [units][splits][G][D+2] fp32,
+static DecGeom dec_geom(const lte_dims* d) {
+  const long long L = (long long)d->window + d->sink + d->cap;
+  const long long W = (long long)d->B * d->Hkv * L;
+  const long long want = (W + kDecChunk - 1) / kDecChunk;
+  DecGeom g;
+  g.n_ctas = (int)(want < sm_count() ? want : sm_count());
+  if (g.n_ctas < 1) g.n_ctas = 1;
+  g.per_cta = (int)((W + g.n_ctas - 1) / g.n_ctas);
+  g.max_parts = (int)((L + g.per_cta - 1) / g.per_cta) + 1;
+  return g;
+}
+
+// chunk-list bound for one CTA: range chunks + per-unit range splits and flushes
+static bool dec_fits(const lte_dims* d) {
+  const DecGeom g = dec_geom(d);
+  const long long L = (long long)d->window + d->sink + d->cap;
+  const long long units = (g.per_cta + L - 1) / L + 1;
+  const long long rows = (long long)d->B * d->Hkv * L;          // TMA row coordinates are int32
+  return (g.per_cta + kDecChunk - 1) / kDecChunk + 4 * units <= kDecMaxEntries &&
+         g.max_parts <= kDecMaxParts &&
+         rows < (1ll << 31) && (long long)d->B * d->Hq < (1ll << 31);
+}
+
+// workspace after the error word: partials [units][max_parts][G][D+4] fp32,
 // then counters [units + 1] int32.
 size_t decode_scratch_bytes(const lte_dims* d) {
   const size_t units = (size_t)d->B * d->Hkv;
   const size_t G = d->Hq / d->Hkv;
-  return units * dec_splits(d) * G * (d->D + 2) * sizeof(float) + (units + 1) * sizeof(int32_t) +
-         64;
+  return units * dec_geom(d).max_parts * G * (d->D + 4) * sizeof(float) +
+         (units + 1) * sizeof(int32_t) + 64;
+}
+
+bool decode_supported(const lte_dims* d) { return dec_fits(d); }
+
+// Programmatic dependent launch: a kernel may start while its predecessor in
+// the stream finishes; griddepcontrol.wait blocks until the predecessor grid
+// has completed and its memory is visible, launch_dependents lets the next
+// kernel start its own prologue early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128)
-decode_update_kernel(int Hkv, int D, int elt, int window, int sink, int cap, float tau,
-                     const char* __restrict__ k_t, const char* __restrict__ v_t,
-                     char* __restrict__ ck, char* __restrict__ cv, int32_t* __restrict__ pos,
-                     float* __restrict__ win_r, int32_t* __restrict__ ret_total,
-                     const int32_t* __restrict__ meta, int32_t* __restrict__ counters,
-                     int n_units, DevError* err) {
+struct PrepParams {
+  int Hkv, D, elt, window, sink, cap, score_batch, future, n_units;
+  float tau;
+  const char* k_t;
+  const char* v_t;
+  char* ck;
+  char* cv;
+  int32_t* pos;
+  float* win_r;
+  int32_t* ret_total;
+  int32_t* meta;
+  int32_t* counters;
+  DevError* err;
+};
+
+template <typename T, bool kTc>
+__global__ void __launch_bounds__(kTcThreads)
+decode_prep_kernel(PrepParams pp, ScoreParams sp, RingKV<T> kv) {
+  extern __shared__ __align__(128) float smem[];
+  __shared__ int dst_sh;
   const int u = blockIdx.x, tid = threadIdx.x;
-  const int L = window + sink + cap;
-  const int t = meta[0];
-  const int leaving = t - window;
-  const int slot_w = t % window;
+  const int L = pp.window + pp.sink + pp.cap;
+  pdl_wait();              // the previous step's attention has finished with the cache
+  pdl_launch_next();
+  const int t = pp.meta[0];
+  const int n_scored = pp.meta[1];
+  const int leaving = t - pp.window;
+  const int slot_w = t % pp.window;
   const long long urow = (long long)u * L;
-  int dst_slot = -1, rt = 0;
-  bool retained = false;
-  if (leaving >= 0) {
-    if (pos[urow + slot_w] != leaving) {
-      if (tid == 0) record_error(err, LTE_ERR_DEVICE, kWhereDecodeIndex);
-    } else if (leaving < sink) {
-      dst_slot = window + leaving;
-    } else if (cap > 0 && win_r[(long long)u * window + slot_w] >= tau) {
-      rt = ret_total[u];
-      dst_slot = window + sink + rt % cap;
-      retained = true;
-    }
+
+  // ---- (1) cache update; every load is issued before any dependent store
+  const int nvec = pp.D * pp.elt / 16;
+  const long long wsrc = (urow + slot_w) * pp.D * pp.elt;
+  uint4 kw, vw, kn, vn;
+  if (tid < nvec) {
+    kw = reinterpret_cast<const uint4*>(pp.ck + wsrc)[tid];      // leaving token (if any)
+    vw = reinterpret_cast<const uint4*>(pp.cv + wsrc)[tid];
+    kn = reinterpret_cast<const uint4*>(pp.k_t + (long long)u * pp.D * pp.elt)[tid];
+    vn = reinterpret_cast<const uint4*>(pp.v_t + (long long)u * pp.D * pp.elt)[tid];
   }
-  const int nvec = D * elt / 16;
-  const long long wsrc = (urow + slot_w) * D * elt;
-  for (int i = tid; i < nvec; i += blockDim.x) {
-    uint4* kw = reinterpret_cast<uint4*>(ck + wsrc) + i;
-    uint4* vw = reinterpret_cast<uint4*>(cv + wsrc) + i;
-    if (dst_slot >= 0) {
-      const long long dst = (urow + dst_slot) * D * elt;
-      reinterpret_cast<uint4*>(ck + dst)[i] = *kw;
-      reinterpret_cast<uint4*>(cv + dst)[i] = *vw;
+  int rt = 0;
+  if (tid == 0) {
+    int dst = -1;
+    if (leaving >= 0) {
+      const int held = pp.pos[urow + slot_w];
+      const float r = pp.win_r[(long long)u * pp.window + slot_w];
+      rt = pp.ret_total[u];
+      if (held != leaving) record_error(pp.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
+      else if (leaving < pp.sink) dst = pp.window + leaving;
+      else if (pp.cap > 0 && r >= pp.tau) dst = pp.window + pp.sink + rt % pp.cap;
     }
-    *kw = reinterpret_cast<const uint4*>(k_t + (long long)u * D * elt)[i];
-    *vw = reinterpret_cast<const uint4*>(v_t + (long long)u * D * elt)[i];
+    dst_sh = dst;
+  }
+  __syncthreads();
+  const int dst_slot = dst_sh;
+  if (tid < nvec) {
+    if (dst_slot >= 0) {
+      const long long dst = (urow + dst_slot) * pp.D * pp.elt;
+      reinterpret_cast<uint4*>(pp.ck + dst)[tid] = kw;
+      reinterpret_cast<uint4*>(pp.cv + dst)[tid] = vw;
+    }
+    reinterpret_cast<uint4*>(pp.ck + wsrc)[tid] = kn;
+    reinterpret_cast<uint4*>(pp.cv + wsrc)[tid] = vn;
   }
   if (tid == 0) {
-    if (dst_slot >= 0) pos[urow + dst_slot] = leaving;
-    if (retained) ret_total[u] = rt + 1;
-    pos[urow + slot_w] = t;
-    win_r[(long long)u * window + slot_w] = NAN;
-    counters[u] = 0;
-    if (u == 0) counters[n_units] = 0;
+    if (dst_slot >= 0) pp.pos[urow + dst_slot] = leaving;
+    if (dst_slot >= pp.window + pp.sink) pp.ret_total[u] = rt + 1;
+    pp.pos[urow + slot_w] = t;
+    pp.win_r[(long long)u * pp.window + slot_w] = NAN;
+    pp.counters[u] = 0;
+    if (u == 0) pp.counters[pp.n_units] = 0;
+  }
+  __syncthreads();   // the new token is in the window for the scoring below
+
+  // ---- (2) deferred batched scoring of the oldest scorable tokens
+  const bool due = (t - pp.future) - n_scored + 1 >= pp.score_batch;
+  if (u == 0 && tid == 0) pp.meta[2] = due ? n_scored + pp.score_batch : n_scored;
+  if (!due) return;
+  const int b = u / pp.Hkv, h = u % pp.Hkv;
+  const int j_end = n_scored + pp.score_batch;
+  for (int jb = n_scored; jb < j_end; jb += kScoreNT) {
+    if constexpr (kTc)
+      score_tile_tc<RingKV<T>>(sp, kv, b, h, jb, j_end, t + 1, reinterpret_cast<uint8_t*>(smem));
+    else
+      score_tile<T, RingKV<T>>(sp, kv, b, h, jb, j_end, t + 1, smem);
   }
 }
 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32d(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16d(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
 }
 __device__ __forceinline__ void ldsm_x4d(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                          uint32_t& r3, bool trans) {
@@ -133,226 +216,440 @@ __device__ __forceinline__ uint32_t pack_bf16d(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-template <int D>
-__device__ __forceinline__ uint32_t swzd(int r, int c) {
-  return (uint32_t)(r * D * 2 + ((c ^ (r & 7)) << 4));
+struct AttnParams {
+  int Hq, Hkv, G, window, sink, cap, L, n_units, per_cta, max_parts;
+  float scale_log2;
+  const int32_t* ret_total;
+  int32_t* meta;
+  __nv_bfloat16* o_t;
+  float* lse_t;
+  float* part;
+  int32_t* counters;
+  DevError* err;
+};
+
+// 128B-swizzled tile written by TMA: [D/64 column halves][rows][128 bytes];
+// byte offset of 16-byte chunk c of row r
+__device__ __forceinline__ uint32_t sw128(int rows, int r, int c) {
+  return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ unsigned long long gtime_d() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool mbar_try_d(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait (1 s of global time); false when it ran out
+__device__ __forceinline__ bool mbar_wait_d(uint32_t bar, uint32_t parity) {
+  if (mbar_try_d(bar, parity)) return true;
+  const unsigned long long t0 = gtime_d();
+  while (!mbar_try_d(bar, parity))
+    if (gtime_d() - t0 > 1000000000ull) return false;
+  return true;
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                       int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(kDecThreads)
-decode_attn_kernel(int Hq, int Hkv, int window, int sink, int cap, float scale_log2,
-                   const __nv_bfloat16* __restrict__ q_t, const __nv_bfloat16* __restrict__ ck,
-                   const __nv_bfloat16* __restrict__ cv, const int32_t* __restrict__ ret_total,
-                   int32_t* __restrict__ meta, __nv_bfloat16* __restrict__ o_t,
-                   float* __restrict__ lse_t, float* __restrict__ part,
-                   int32_t* __restrict__ counters, int n_units, int n_split) {
-  constexpr int CH = D / 8, KSTEPS = D / 16, DN = D / 8;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* q_sm = smem;                                   // [16][D] bf16
-  uint8_t* kv_sm = smem + 16 * D * 2;                     // per warp: K [32][D], V [32][D]
-  __shared__ float m_sh[kDecWarps][16], l_sh[kDecWarps][16];
-  __shared__ int is_last;
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
+  constexpr int KSTEPS = D / 16, DN = D / 8, HALVES = D / 64;
+  constexpr int kKV = kDecChunk * D * 2;                  // K or V of one stage
+  constexpr int kQ = 16 * D * 2;                          // Q rows of one stage
+  constexpr int kStage = 2 * kKV + kQ;                    // multiple of 1 KiB
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  float* o_sh = reinterpret_cast<float*>(dsm + kDecStages * kStage);    // [warps][16][D]
+  float* m_sh = o_sh + kDecWarps * 16 * D;                               // [warps][16]
+  float* l_sh = m_sh + kDecWarps * 16;                                   // [warps][16]
+  int4* ents = reinterpret_cast<int4*>(l_sh + kDecWarps * 16);           // chunk list
+  uint64_t* full = reinterpret_cast<uint64_t*>(ents + kDecMaxEntries);   // stage barriers
+  int* n_ents = reinterpret_cast<int*>(full + kDecStages);
+  int* is_last = n_ents + 1;
 
-  const int split = blockIdx.x, u = blockIdx.y;
-  const int b = u / Hkv, h = u % Hkv, G = Hq / Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = window + sink + cap;
-  const int t = meta[0];
-  const int nw = min(window, t + 1);
-  int ns = t - window + 1;
-  ns = ns < 0 ? 0 : (ns > sink ? sink : ns);
-  const int rt = ret_total[u];
-  const int nr = min(cap, rt);
-  const int n = nw + ns + nr;
-
-  // Q rows 0..G-1 (rows G..15 zero)
-  for (int i = tid; i < 16 * CH; i += kDecThreads) {
-    const int r = i / CH, c = i % CH;
-    const bool ok = r < G;
-    const __nv_bfloat16* src = q_t + (ok ? ((long long)b * Hq + h * G + r) * D + c * 8 : 0);
-    cp_async16d(smem_u32d(q_sm + swzd<D>(r, c)), src, ok);
+  if ((smem_u32d(dsm) & 1023u) != 0) {          // swizzle atoms need 1 KiB alignment
+    if (tid == 0) record_error(p.err, LTE_ERR_DEVICE, 120);
+    return;
   }
-  // this warp's 32 keys: logical l -> slot
-  const int l0 = split * kDecKeysPerCta + warp * kDecKeysPerWarp;
-  uint8_t* ks = kv_sm + warp * 2 * kDecKeysPerWarp * D * 2;
-  uint8_t* vs = ks + kDecKeysPerWarp * D * 2;
-  const long long ubase = (long long)u * L;
-  for (int i = lane; i < kDecKeysPerWarp * CH; i += 32) {
-    const int r = i / CH, c = i % CH;
-    const int l = l0 + r;
-    const bool ok = l < n;
-    int slot = 0;
-    if (ok) slot = l < nw ? l : (l < nw + ns ? window + (l - nw) : window + sink + (l - nw - ns));
-    const long long a = ok ? (ubase + slot) * D + c * 8 : 0;
-    cp_async16d(smem_u32d(ks + swzd<D>(r, c)), ck + a, ok);
-    cp_async16d(smem_u32d(vs + swzd<D>(r, c)), cv + a, ok);
-  }
-  asm volatile("cp.async.commit_group;\n" ::);
-  asm volatile("cp.async.wait_group 0;\n" ::);
-  __syncthreads();
-
-  uint32_t qf[KSTEPS][4];
-#pragma unroll
-  for (int kst = 0; kst < KSTEPS; ++kst) {
-    const int r = lane & 15, c = kst * 2 + (lane >> 4);
-    ldsm_x4d(smem_u32d(q_sm + swzd<D>(r, c)), qf[kst][0], qf[kst][1], qf[kst][2], qf[kst][3],
-             false);
-  }
-  float s[4][4];
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-#pragma unroll
-  for (int kst = 0; kst < KSTEPS; ++kst) {
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      const int r = np * 16 + ((lane >> 4) << 3) + (lane & 7);
-      const int c = kst * 2 + ((lane >> 3) & 1);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4d(smem_u32d(ks + swzd<D>(r, c)), b0, b1, b2, b3, false);
-      mma_bf16d(s[2 * np], qf[kst], b0, b1);
-      mma_bf16d(s[2 * np + 1], qf[kst], b2, b3);
-    }
-  }
-  // mask keys beyond the list, softmax (exp2 domain)
-  float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int l = l0 + nt * 8 + ((lane & 3) << 1) + (e & 1);
-      s[nt][e] = (l < n) ? s[nt][e] * scale_log2 : -INFINITY;
-      mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
-    }
-  float m_use[2], l_part[2] = {0.f, 0.f};
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
-    mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
-    m_use[hr] = (mx[hr] == -INFINITY) ? 0.f : mx[hr];
-  }
-  uint32_t pf[2][4];
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    float p[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      p[e] = exp2f(s[nt][e] - m_use[e >> 1]);
-      l_part[e >> 1] += p[e];
-    }
-    pf[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16d(p[0], p[1]);
-    pf[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16d(p[2], p[3]);
-  }
-  float o_acc[DN][4];
-#pragma unroll
-  for (int i = 0; i < DN; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o_acc[i][e] = 0.f;
-#pragma unroll
-  for (int kst = 0; kst < 2; ++kst) {
-#pragma unroll
-    for (int dp = 0; dp < DN / 2; ++dp) {
-      const int r = kst * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
-      const int c = dp * 2 + (lane >> 4);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4d(smem_u32d(vs + swzd<D>(r, c)), b0, b1, b2, b3, true);
-      mma_bf16d(o_acc[2 * dp], pf[kst], b0, b1);
-      mma_bf16d(o_acc[2 * dp + 1], pf[kst], b2, b3);
-    }
-  }
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 1);
-    l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 2);
-  }
-  // ---- merge the 4 warps through shared memory (reuses the K/V area)
-  __syncthreads();
-  float* o_sh = reinterpret_cast<float*>(kv_sm);          // [warps][16][D]
-#pragma unroll
-  for (int hr = 0; hr < 2; ++hr) {
-    const int r = (lane >> 2) + hr * 8;
-    if ((lane & 3) == 0) {
-      m_sh[warp][r] = mx[hr];                             // -inf when the warp saw no key
-      l_sh[warp][r] = l_part[hr];
-    }
-#pragma unroll
-    for (int i = 0; i < DN; ++i) {
-      const int dcol = i * 8 + ((lane & 3) << 1);
-      o_sh[(warp * 16 + r) * D + dcol] = o_acc[i][hr * 2];
-      o_sh[(warp * 16 + r) * D + dcol + 1] = o_acc[i][hr * 2 + 1];
-    }
-  }
-  __syncthreads();
-  // CTA partial for rows g < G:  part[u][split][g] = {m, l, o[D]}
-  float* my_part = part + ((long long)u * n_split + split) * G * (D + 2);
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int g = i / D, dd = i % D;
-    float M = -INFINITY;
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, m_sh[w][g]);
-    float acc = 0.f;
-    for (int w = 0; w < kDecWarps; ++w)
-      if (m_sh[w][g] != -INFINITY) acc += o_sh[(w * 16 + g) * D + dd] * exp2f(m_sh[w][g] - M);
-    my_part[g * (D + 2) + 2 + dd] = acc;
-    if (dd == 0) {
-      float l = 0.f;
-      for (int w = 0; w < kDecWarps; ++w)
-        if (m_sh[w][g] != -INFINITY) l += l_sh[w][g] * exp2f(m_sh[w][g] - M);
-      my_part[g * (D + 2)] = M;
-      my_part[g * (D + 2) + 1] = l;
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) is_last = (atomicAdd(&counters[u], 1) == n_split - 1);
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  // ---- last CTA of the unit: merge the splits
-  const float* up = part + (long long)u * n_split * G * (D + 2);
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int g = i / D, dd = i % D;
-    float M = -INFINITY;
-    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, __ldcg(up + (sp * G + g) * (D + 2)));
-    float acc = 0.f, l = 0.f;
-    for (int sp = 0; sp < n_split; ++sp) {
-      const float* pp = up + (sp * G + g) * (D + 2);
-      const float m = __ldcg(pp);
-      if (m == -INFINITY) continue;
-      const float f = exp2f(m - M);
-      l += __ldcg(pp + 1) * f;
-      acc += __ldcg(pp + 2 + dd) * f;
-    }
-    o_t[((long long)b * Hq + h * G + g) * D + dd] = __float2bfloat16_rn(acc / l);
-    if (dd == 0 && lse_t != nullptr)
-      lse_t[(long long)b * Hq + h * G + g] = (M + log2f(l)) * 0.69314718055994531f;
-  }
-  __syncthreads();
+  pdl_launch_next();
   if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(&counters[n_units], 1) == n_units - 1) {
-      meta[0] = t + 1;
-      meta[1] = meta[2];
-    }
+    for (int st = 0; st < kDecStages; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(full + st)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // meta[0] is not written by the preceding update kernel (only by the last
+  // attention CTA of the previous step, which finished before that kernel began)
+  const int t = p.meta[0];
+  pdl_wait();              // the cache update and scoring of this step are visible
+  const int nw = min(p.window, t + 1);
+  int ns = t - p.window + 1;
+  ns = ns < 0 ? 0 : (ns > p.sink ? p.sink : ns);
+  const long long W = (long long)p.n_units * p.L;
+  const long long lo = (long long)blockIdx.x * p.per_cta;
+  const long long hi = lo + p.per_cta < W ? lo + p.per_cta : W;
+
+  // ---- chunk list: (unit, first slot, keys, last-of-unit) over the valid slots of [lo, hi)
+  if (tid == 0) {
+    int n = 0;
+    const int u_lo = (int)(lo / p.L), u_hi = (int)((hi - 1) / p.L);
+    int rt[4];                                   // loads issued together, used below
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rt[k] = (u_lo + k <= u_hi) ? p.ret_total[u_lo + k] : 0;
+    for (int u = u_lo; u <= u_hi; ++u) {
+      const int a = (int)((lo > (long long)u * p.L ? lo : (long long)u * p.L) - (long long)u * p.L);
+      const long long ue = (long long)(u + 1) * p.L;
+      const int bnd = (int)((hi < ue ? hi : ue) - (long long)u * p.L);
+      const int nr = min(p.cap, u - u_lo < 4 ? rt[u - u_lo] : p.ret_total[u]);
+      const int rs[3] = {0, p.window, p.window + p.sink};
+      const int re[3] = {nw, p.window + ns, p.window + p.sink + nr};
+      const int first = n;
+      for (int r = 0; r < 3; ++r) {
+        const int x = max(a, rs[r]), y = min(bnd, re[r]);
+        for (int s = x; s < y && n < kDecMaxEntries; s += kDecChunk)
+          ents[n++] = make_int4(u, s, min(kDecChunk, y - s), 0);
+      }
+      if (n == first && n < kDecMaxEntries) ents[n++] = make_int4(u, 0, 0, 0);   // flush only
+      if (n > 0) ents[n - 1].w = 1;
+    }
+    *n_ents = n;
+  }
+  __syncthreads();
+  const int n_ch = *n_ents;
+
+  // one elected thread issues the TMA copies of chunk i into stage i % kDecStages
+  // (flush-only entries still load rows so that every stage use completes a phase)
+  auto load = [&](int i) {
+    const int4 e = ents[i];
+    const uint32_t st = smem_u32d(dsm + (i % kDecStages) * kStage);
+    const uint32_t bar = smem_u32d(full + i % kDecStages);
+    const int b = e.x / p.Hkv, h = e.x % p.Hkv;
+    const int row = e.x * p.L + e.y;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kStage)
+                 : "memory");
+#pragma unroll
+    for (int hf = 0; hf < HALVES; ++hf) {
+      tma_2d(st + hf * kDecChunk * 128, &tm_k, bar, hf * 64, row);
+      tma_2d(st + kKV + hf * kDecChunk * 128, &tm_v, bar, hf * 64, row);
+      tma_2d(st + 2 * kKV + hf * 16 * 128, &tm_q, bar, hf * 64, b * p.Hq + h * p.G);
+    }
+  };
+
+  float o_acc[DN][4];
+  float m_run[2], l_run[2];
+  auto reset = [&]() {
+#pragma unroll
+    for (int i = 0; i < DN; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o_acc[i][e] = 0.f;
+    m_run[0] = m_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+  };
+  reset();
+
+  int issued = 0;
+  if (tid == 0)
+    for (; issued < kDecStages - 1 && issued < n_ch; ++issued) load(issued);
+  int i = 0;
+#pragma unroll 1
+  for (; i < n_ch; ++i) {
+    if (tid == 0 && i + kDecStages - 1 < n_ch) load(issued++);
+    const bool ok = mbar_wait_d(smem_u32d(full + i % kDecStages), (i / kDecStages) & 1);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) record_error(p.err, LTE_ERR_TIMEOUT, 121);
+      break;
+    }
+    const int4 e = ents[i];
+    const uint8_t* st = dsm + (i % kDecStages) * kStage;
+    const int k0 = warp * 16;                 // this warp's 16 keys of the chunk
+    if (k0 < e.z) {
+      uint32_t qf[KSTEPS][4];
+#pragma unroll
+      for (int kst = 0; kst < KSTEPS; ++kst) {
+        const int r = lane & 15, c = kst * 2 + (lane >> 4);
+        ldsm_x4d(smem_u32d(st + 2 * kKV + sw128(16, r, c)), qf[kst][0], qf[kst][1], qf[kst][2],
+                 qf[kst][3], false);
+      }
+      float s[2][4] = {};
+#pragma unroll
+      for (int kst = 0; kst < KSTEPS; ++kst) {
+        const int r = k0 + ((lane >> 4) << 3) + (lane & 7);
+        const int c = kst * 2 + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4d(smem_u32d(st + sw128(kDecChunk, r, c)), b0, b1, b2, b3, false);
+        mma_bf16d(s[0], qf[kst], b0, b1);
+        mma_bf16d(s[1], qf[kst], b2, b3);
+      }
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int key = k0 + nt * 8 + ((lane & 3) << 1) + (q & 1);
+          s[nt][q] = key < e.z ? s[nt][q] * p.scale_log2 : -INFINITY;
+          mx[q >> 1] = fmaxf(mx[q >> 1], s[nt][q]);
+        }
+      float corr[2], mu[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+        const float m_new = fmaxf(m_run[hr], mx[hr]);
+        mu[hr] = m_new == -INFINITY ? 0.f : m_new;
+        corr[hr] = m_run[hr] == -INFINITY ? 0.f : exp2f(m_run[hr] - mu[hr]);
+        m_run[hr] = m_new;
+        l_run[hr] *= corr[hr];
+      }
+      uint32_t pf[4];
+      {
+        float pv[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            pv[nt][q] = exp2f(s[nt][q] - mu[q >> 1]);
+            l_run[q >> 1] += pv[nt][q];
+          }
+        pf[0] = pack_bf16d(pv[0][0], pv[0][1]);
+        pf[1] = pack_bf16d(pv[0][2], pv[0][3]);
+        pf[2] = pack_bf16d(pv[1][0], pv[1][1]);
+        pf[3] = pack_bf16d(pv[1][2], pv[1][3]);
+      }
+#pragma unroll
+      for (int i2 = 0; i2 < DN; ++i2) {
+        o_acc[i2][0] *= corr[0]; o_acc[i2][1] *= corr[0];
+        o_acc[i2][2] *= corr[1]; o_acc[i2][3] *= corr[1];
+      }
+#pragma unroll
+      for (int dp = 0; dp < DN / 2; ++dp) {
+        const int r = k0 + (((lane >> 3) & 1) << 3) + (lane & 7);
+        const int c = dp * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4d(smem_u32d(st + kKV + sw128(kDecChunk, r, c)), b0, b1, b2, b3, true);
+        mma_bf16d(o_acc[2 * dp], pf, b0, b1);
+        mma_bf16d(o_acc[2 * dp + 1], pf, b2, b3);
+      }
+    }
+    if (e.w) {
+      // ---- end of this CTA's part of unit e.x: merge the warps, publish the partial
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 1);
+        l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 2);
+        const int r = (lane >> 2) + hr * 8;
+        if ((lane & 3) == 0) {
+          m_sh[warp * 16 + r] = m_run[hr];
+          l_sh[warp * 16 + r] = l_run[hr];
+        }
+#pragma unroll
+        for (int i2 = 0; i2 < DN; ++i2) {
+          const int dcol = i2 * 8 + ((lane & 3) << 1);
+          o_sh[(warp * 16 + r) * D + dcol] = o_acc[i2][hr * 2];
+          o_sh[(warp * 16 + r) * D + dcol + 1] = o_acc[i2][hr * 2 + 1];
+        }
+      }
+      __syncthreads();
+      const int u = e.x;
+      const int c_first = (int)(((long long)u * p.L) / p.per_cta);
+      const int c_last = (int)(((long long)u * p.L + p.L - 1) / p.per_cta);
+      const int n_parts = c_last - c_first + 1;
+      // partial layout per (unit, part): [G][D + 4] fp32 = {m, l, pad, pad, o[D]}
+      float* up = p.part + (long long)u * p.max_parts * p.G * (D + 4);
+      float* mine = up + (long long)(blockIdx.x - c_first) * p.G * (D + 4);
+      for (int i2 = tid; i2 < p.G * (D / 4); i2 += kDecThreads) {
+        const int g = i2 / (D / 4), d4 = (i2 % (D / 4)) * 4;
+        float M = -INFINITY;
+        float f[kDecWarps];
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, m_sh[w * 16 + g]);
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+          const float mw = m_sh[w * 16 + g];
+          f[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+          l += l_sh[w * 16 + g] * f[w];
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+          const float4 ow = *reinterpret_cast<const float4*>(o_sh + (w * 16 + g) * D + d4);
+          acc.x += ow.x * f[w]; acc.y += ow.y * f[w]; acc.z += ow.z * f[w]; acc.w += ow.w * f[w];
+        }
+        *reinterpret_cast<float4*>(mine + g * (D + 4) + 4 + d4) = acc;
+        if (d4 == 0) *reinterpret_cast<float4*>(mine + g * (D + 4)) = make_float4(M, l, 0.f, 0.f);
+      }
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) *is_last = atomicAdd(&p.counters[u], 1) == n_parts - 1;
+      __syncthreads();
+      if (*is_last) {
+        __threadfence();
+        const int b = u / p.Hkv, h = u % p.Hkv;
+        for (int i2 = tid; i2 < p.G * (D / 4); i2 += kDecThreads) {
+          const int g = i2 / (D / 4), d4 = (i2 % (D / 4)) * 4;
+          float4 ml[kDecMaxParts], ov[kDecMaxParts];
+#pragma unroll
+          for (int sp = 0; sp < kDecMaxParts; ++sp)       // every load issued before any use
+            if (sp < n_parts) {
+              const float* pp = up + (sp * p.G + g) * (D + 4);
+              ml[sp] = __ldcg(reinterpret_cast<const float4*>(pp));
+              ov[sp] = __ldcg(reinterpret_cast<const float4*>(pp + 4 + d4));
+            }
+          float M = -INFINITY;
+#pragma unroll
+          for (int sp = 0; sp < kDecMaxParts; ++sp) if (sp < n_parts) M = fmaxf(M, ml[sp].x);
+          float l = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int sp = 0; sp < kDecMaxParts; ++sp)
+            if (sp < n_parts && ml[sp].x != -INFINITY) {
+              const float fw = exp2f(ml[sp].x - M);
+              l += ml[sp].y * fw;
+              acc.x += ov[sp].x * fw; acc.y += ov[sp].y * fw;
+              acc.z += ov[sp].z * fw; acc.w += ov[sp].w * fw;
+            }
+          const float inv = 1.f / l;
+          __nv_bfloat16* orow = p.o_t + ((long long)b * p.Hq + h * p.G + g) * D + d4;
+          *reinterpret_cast<uint2*>(orow) =
+              make_uint2(pack_bf16d(acc.x * inv, acc.y * inv), pack_bf16d(acc.z * inv, acc.w * inv));
+          if (d4 == 0 && p.lse_t != nullptr)
+            p.lse_t[(long long)b * p.Hq + h * p.G + g] = (M + log2f(l)) * 0.69314718055994531f;
+        }
+        __syncthreads();
+        if (tid == 0) {
+          __threadfence();
+          if (atomicAdd(&p.counters[p.n_units], 1) == p.n_units - 1) {
+            p.meta[0] = t + 1;
+            p.meta[1] = p.meta[2];
+          }
+        }
+      }
+      reset();
+    }
+    __syncthreads();     // stage i % kDecStages and the merge buffers are free again
+  }
+  // copies issued but not consumed (only after a wait ran out) land before exit
+  if (tid == 0)
+    for (int j = i; j < issued; ++j) mbar_wait_d(smem_u32d(full + j % kDecStages), (j / kDecStages) & 1);
+}
+
+// launch with programmatic stream serialization (see pdl_wait)
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename T>
+static cudaError_t launch_prep(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
+                               const void* k_t, const void* v_t, int score_batch,
+                               int32_t* counters, DevError* err, cudaStream_t stream) {
+  PrepParams pp{};
+  pp.Hkv = d->Hkv; pp.D = d->D; pp.elt = sizeof(T); pp.window = d->window; pp.sink = d->sink;
+  pp.cap = d->cap; pp.score_batch = score_batch;
+  pp.future = (cnn->k1 - 1 - cnn->past1) + (cnn->k2 - 1 - cnn->past2);
+  pp.n_units = d->B * d->Hkv; pp.tau = d->tau;
+  pp.k_t = (const char*)k_t; pp.v_t = (const char*)v_t;
+  pp.ck = (char*)c->k; pp.cv = (char*)c->v; pp.pos = c->pos; pp.win_r = c->win_r;
+  pp.ret_total = c->ret_total; pp.meta = c->meta; pp.counters = counters; pp.err = err;
+  ScoreParams sp = score_params(d, cnn);
+  sp.window = d->window;
+  sp.win_r = c->win_r;
+  const int L = d->window + d->sink + d->cap;
+  RingKV<T> kv{(const T*)c->k, (const T*)c->v, d->Hkv, L, d->window, d->D};
+  // the same scoring tile as lte_score for this shape, so decode scores equal prefill scores
+  if (score_tc_supported(cnn->c_hid, cnn->k1, cnn->k2)) {
+    const size_t smem = score_tc_smem_bytes(d->D, cnn->c_hid, cnn->k2);
+    cudaError_t e = cudaFuncSetAttribute(decode_prep_kernel<T, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_prep_kernel<T, true>, dim3(pp.n_units), dim3(kTcThreads), smem, stream,
+                      pp, sp, kv);
+  }
+  const size_t smem = sizeof(float) * score_smem_floats(d->D, cnn->c_hid, cnn->k1, cnn->k2);
+  cudaError_t e = cudaFuncSetAttribute(decode_prep_kernel<T, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_prep_kernel<T, false>, dim3(pp.n_units), dim3(kScoreThreads), smem,
+                    stream, pp, sp, kv);
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over `rows` rows of D elements, boxes of 64 x box_rows, 128B swizzle
+static bool rows_map(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D>
-static cudaError_t launch_decode_attn(const lte_dims* d, const lte_cache* c, const void* q_t,
-                                      void* o_t, float* lse_t, float* part, int32_t* counters,
-                                      cudaStream_t stream) {
-  const int n_split = dec_splits(d);
-  const int n_units = d->B * d->Hkv;
-  const size_t smem = 16 * D * 2 + (size_t)kDecWarps * 2 * kDecKeysPerWarp * D * 2;
+static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void* q_t, void* o_t,
+                               float* lse_t, float* part, int32_t* counters, DevError* err,
+                               cudaStream_t stream) {
+  const DecGeom g = dec_geom(d);
+  AttnParams p{};
+  p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = d->Hq / d->Hkv; p.window = d->window; p.sink = d->sink;
+  p.cap = d->cap; p.L = d->window + d->sink + d->cap; p.n_units = d->B * d->Hkv;
+  p.per_cta = g.per_cta; p.max_parts = g.max_parts;
+  p.scale_log2 = d->scale * 1.4426950408889634f;
+  p.ret_total = c->ret_total; p.meta = c->meta;
+  p.o_t = (__nv_bfloat16*)o_t; p.lse_t = lse_t; p.part = part; p.counters = counters; p.err = err;
+  CUtensorMap mk, mv, mq;
+  const long long rows = (long long)p.n_units * p.L;
+  if (!rows_map(&mk, c->k, rows, D, kDecChunk) || !rows_map(&mv, c->v, rows, D, kDecChunk) ||
+      !rows_map(&mq, q_t, (long long)d->B * d->Hq, D, 16))
+    return cudaErrorInvalidValue;
+  const size_t stage = 2 * (size_t)kDecChunk * D * 2 + 16 * D * 2;
+  const size_t smem = kDecStages * stage + (size_t)kDecWarps * 16 * D * 4 + 2 * kDecWarps * 16 * 4 +
+                      (size_t)kDecMaxEntries * 16 + kDecStages * 8 + 16;
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(n_split, n_units);
-  decode_attn_kernel<D><<<grid, kDecThreads, smem, stream>>>(
-      d->Hq, d->Hkv, d->window, d->sink, d->cap, d->scale * 1.4426950408889634f,
-      (const __nv_bfloat16*)q_t, (const __nv_bfloat16*)c->k, (const __nv_bfloat16*)c->v,
-      c->ret_total, c->meta, (__nv_bfloat16*)o_t, lse_t, part, counters, n_units, n_split);
-  return cudaGetLastError();
+  return launch_pdl(decode_attn_kernel<D>, dim3(g.n_ctas), dim3(kDecThreads), smem, stream, mk, mv,
+                    mq, p);
 }
 
 cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
@@ -364,17 +661,11 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
   float* part = reinterpret_cast<float*>(scratch);
   int32_t* counters = reinterpret_cast<int32_t*>(
       reinterpret_cast<char*>(scratch) +
-      (size_t)n_units * dec_splits(d) * G * (d->D + 2) * sizeof(float));
-  decode_update_kernel<<<n_units, 128, 0, stream>>>(
-      d->Hkv, d->D, 2, d->window, d->sink, d->cap, d->tau, (const char*)k_t, (const char*)v_t,
-      (char*)c->k, (char*)c->v, c->pos, c->win_r, c->ret_total, c->meta, counters, n_units, err);
-  cudaError_t e = cudaGetLastError();
+      (size_t)n_units * dec_geom(d).max_parts * G * (d->D + 4) * sizeof(float));
+  cudaError_t e = launch_prep<__nv_bfloat16>(d, cnn, c, k_t, v_t, score_batch, counters, err, stream);
   if (e != cudaSuccess) return e;
-  e = score_ring(d, cnn, c, score_batch, stream);
-  if (e != cudaSuccess) return e;
-  if (d->D == 128)
-    return launch_decode_attn<128>(d, c, q_t, o_t, lse_t, part, counters, stream);
-  return launch_decode_attn<64>(d, c, q_t, o_t, lse_t, part, counters, stream);
+  if (d->D == 128) return launch_attn<128>(d, c, q_t, o_t, lse_t, part, counters, err, stream);
+  return launch_attn<64>(d, c, q_t, o_t, lse_t, part, counters, err, stream);
 }
 
 // ---------------------------------------------------------------------------

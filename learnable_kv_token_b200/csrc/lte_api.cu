@@ -192,7 +192,7 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
   if (score_batch < 1 || score_batch > d->window - cnn_past(cnn) - cnn_future(cnn))
     return LTE_ERR_INVALID_ARG;
   const int G = d->Hq / d->Hkv;
-  if (G > 16) return LTE_ERR_UNSUPPORTED;
+  if (G > 16 || !lte::decode_supported(d)) return LTE_ERR_UNSUPPORTED;
   if (workspace == nullptr || !aligned16(workspace)) return LTE_ERR_WORKSPACE;
   if (ws_bytes < lte_workspace_bytes(d, LTE_WS_DECODE)) return LTE_ERR_WORKSPACE;
   return from_cuda(lte::decode_step(d, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch,
@@ -218,7 +218,7 @@ lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const 
     return LTE_ERR_INVALID_ARG;
   if (score_batch < 1 || score_batch > d->window - cnn_past(cnn) - cnn_future(cnn))
     return LTE_ERR_INVALID_ARG;
-  if (d->Hq / d->Hkv > 16) return LTE_ERR_UNSUPPORTED;
+  if (d->Hq / d->Hkv > 16 || !lte::decode_supported(d)) return LTE_ERR_UNSUPPORTED;
   if (lte_workspace_bytes(d, LTE_WS_DECODE) > (size_t)LTE_NOALLOC_SCRATCH_BYTES)
     return LTE_ERR_WORKSPACE;
   void* scratch = nullptr;

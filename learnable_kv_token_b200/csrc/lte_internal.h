@@ -14,8 +14,6 @@ bool score_supported(const lte_cnn* cnn);
 cudaError_t score_linear(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
                          Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
                          cudaStream_t stream);
-cudaError_t score_ring(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
-                       int score_batch, cudaStream_t stream);
 
 // evict_compact.cu
 cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,
@@ -47,6 +45,7 @@ size_t attn_prefill_scratch_bytes(const lte_dims* d);
 
 // decode.cu
 size_t decode_scratch_bytes(const lte_dims* d);
+bool decode_supported(const lte_dims* d);
 cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
                         const void* q_t, const void* k_t, const void* v_t, void* o_t,
                         float* lse_t, int score_batch, DevError* err, void* scratch,

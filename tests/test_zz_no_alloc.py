@@ -52,7 +52,8 @@ def test_noalloc_decode_matches_workspace_variant():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from learnable_kv_token_b200 import lte as L
-    dims = L.make_dims(64, 64, 32, 8, 128, 4, 4096, 8192, 0.5, 0.088, L.LTE_BF16)
+    # 512 units x G = 16 heads x 2 partials per unit x 130 floats ~ 8.5 MB > 4 MiB
+    dims = L.make_dims(64, 64, 128, 8, 128, 4, 512, 512, 0.5, 0.088, L.LTE_BF16)
     assert L.lte_workspace_bytes(dims, L.LTE_WS_DECODE) > 4 << 20
     cnn = L.lte_cnn(32, 5, 2, 3, 1, 16, 16, 16, 16)
     cache = L.lte_cache(16, 16, 16, 16, 16, 16)
