@@ -14,23 +14,29 @@
 // sink slots and the retained slots of the column segment (compacted rows,
 // contiguous) and the window band of the key tensor; every tile is one TMA box
 // per 64-column half.  The kernel is persistent (one CTA per SM walks a static
-// heavy-first list of items).  Warp roles (320 threads):
-//   warp 0     TMA producer: Q tiles into a double buffer (the next item's Q
-//              loads while the current item runs), K and V into 3-slot rings (a K slot frees after
-//              its S MMAs, a V slot after its PV MMAs);
-//   warp 1     TMEM owner and MMA issuer (one elected lane): per K/V tile j,
-//              S_A = Q_A K^T, S_B = Q_B K^T, then O_A += P_A V, O_B += P_B V for
-//              tile j-1, so the tensor core computes one Q tile's products while
-//              the other tile's softmax runs; S, O and P of both tiles live in
-//              TMEM (2 x (64 + 128 + 32) of 512 columns);
-//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one thread per
-//              row reads its S row from TMEM, applies the attended-set
-//              predicate, exp2 via ex2.approx with the scale folded into one
-//              packed FMA, writes P (bf16 pairs) into TMEM, where the PV MMA
-//              reads it as its A operand (only V comes from shared memory),
-//              and rescales its O row in TMEM only when the running max grew by
-//              more than 2^8 (exact: O and l share the reference max); the
-//              epilogue reads O, divides by l and stores bf16 and the lse.
+// heavy-first list of items).
+//
+// TMEM (512 columns): for each Q tile x, S_x (64 fp32 columns; its first 32
+// columns are reused for P_x as bf16 pairs), O_x (128) and Q_x (64, bf16
+// pairs).  Both products read their A operand from TMEM (Q for S = Q K^T, P
+// for O += P V), so shared memory only feeds K and V to the tensor core.
+// Warp roles (320 threads):
+//   warp 0     TMA producer: the item's Q rows into one shared buffer (freed as
+//              soon as both softmax groups copied them into TMEM), K and V
+//              into 4-slot rings (a K slot frees after its S MMAs, a V slot
+//              after its PV MMAs);
+//   warp 1     TMEM owner and MMA issuer (one elected lane), per K/V tile j:
+//              PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  The tensor pipe runs in
+//              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
+//              P_x may then be overwritten and O_x rescaled without a wait;
+//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one thread per row
+//              reads its S row from TMEM, applies the attended-set predicate,
+//              exp2 via ex2.approx with the scale folded into a packed FMA,
+//              writes P into TMEM, and rescales its O row only when the
+//              running max grew by more than 2^8 (exact: O and l share the
+//              reference max).  During an item's last tile it copies the next
+//              item's Q rows into TMEM, so that item's first S overlaps this
+//              item's epilogue (O / l -> bf16, lse).
 // Every mbarrier wait is bounded (1 s of global time): on expiry the CTA
 // records LTE_ERR_TIMEOUT in the workspace error word, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and exits.
@@ -53,20 +59,20 @@ constexpr uint32_t kQHalf = BM * 128;             // 64-column half of a Q tile:
 constexpr uint32_t kQBuf = 2 * kQTile;            // tiles A and B of one item: 64 KiB
 constexpr uint32_t kKV = BN * HD * 2;             // 16 KiB (K or V of one tile)
 constexpr uint32_t kKVHalf = BN * 128;            // 8 KiB
-constexpr int kStages = 3;                        // K/V ring depth
-constexpr uint32_t kOffQ = 0;                     // 2 buffers
-constexpr uint32_t kOffKV = 2 * kQBuf;            // 128 KiB; stage s: K at +s*32K, V at +16K
-constexpr uint32_t kOffBar = kOffKV + kStages * 2 * kKV;   // 224 KiB
+constexpr int kStages = 4;                        // K/V ring depth
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = kQBuf;                // stage s: K at +s*32K, V at +16K
+constexpr uint32_t kOffBar = kOffKV + kStages * 2 * kKV;   // 192 KiB
 constexpr uint32_t kSmemBytes = kOffBar + 256;
 constexpr uint32_t kTmemCols = 512;
-__host__ __device__ constexpr uint32_t col_s(int x) { return x == 0 ? 0u : 64u; }     // S of tile x
-__host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256u; }  // O of tile x
-__host__ __device__ constexpr uint32_t col_p(int x) { return x == 0 ? 384u : 416u; }  // P (bf16 pairs)
+__host__ __device__ constexpr uint32_t col_s(int x) { return x == 0 ? 0u : 64u; }     // S (and P)
+__host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256u; }  // O
+__host__ __device__ constexpr uint32_t col_q(int x) { return x == 0 ? 384u : 448u; }  // Q
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
 enum {
-  B_QF = 0, B_QE = 2, B_KF = 4, B_VF = 7, B_KE = 10, B_VE = 13, B_SF = 16, B_SFREE = 18,
-  B_PF = 20, B_PVD = 22, B_OE = 24, B_FIN = 26, kNumBars = 27
+  B_QF = 0, B_QFREE = 1, B_QC = 2, B_KF = 4, B_VF = 8, B_KE = 12, B_VE = 16, B_SF = 20,
+  B_PF = 22, B_PVD = 24, B_OE = 26, B_FIN = 28, kNumBars = 29
 };
 
 struct Params {
@@ -299,6 +305,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     return;
   }
   if (tid == 0) {
+    mbar_init(bar(B_QF), 1);
+    mbar_init(bar(B_QFREE), 256);
     for (int st = 0; st < kStages; ++st) {
       mbar_init(bar(B_KF + st), 1);
       mbar_init(bar(B_VF + st), 1);
@@ -306,10 +314,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_VE + st), 1);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(bar(B_QF + x), 1);
-      mbar_init(bar(B_QE + x), 1);
+      mbar_init(bar(B_QC + x), 128);
       mbar_init(bar(B_SF + x), 1);
-      mbar_init(bar(B_SFREE + x), 128);
       mbar_init(bar(B_PF + x), 128);
       mbar_init(bar(B_PVD + x), 1);
       mbar_init(bar(B_OE + x), 128);
@@ -337,15 +343,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
       const Item m = make_item(p, i);
-      const int qb = it & 1;
-      if (it >= 2 && !(ok = wwait(bar(B_QE + qb), ((it >> 1) - 1) & 1, abort_flag, p.err, 201)))
-        break;
+      // the shared Q buffer is free once both softmax groups copied the last item's rows
+      if (it >= 1 && !(ok = wwait(bar(B_QFREE), (it - 1) & 1, abort_flag, p.err, 201))) break;
       if (elect_one()) {
-        mbar_expect_tx(bar(B_QF + qb), kQBuf);
+        mbar_expect_tx(bar(B_QF), kQBuf);
         for (int x = 0; x < 2; ++x)
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + kOffQ + qb * kQBuf + x * kQTile + hf * kQHalf, &tm_q,
-                        bar(B_QF + qb), hf * 64, m.h * p.G, m.t0 + x * p.TOK, m.b);
+            tma_load_4d(sbase + kOffQ + x * kQTile + hf * kQHalf, &tm_q, bar(B_QF), hf * 64,
+                        m.h * p.G, m.t0 + x * p.TOK, m.b);
       }
       __syncwarp();
       issued_q = it + 1;
@@ -354,7 +359,6 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         int rg, key0, nk;
         m.tile(j, rg, key0, nk);
         const uint32_t kd = sbase + kOffKV + st * 2 * kKV, vd = kd + kKV;
-        // K slot frees when both S MMAs of its last tile are done, V slot when both PV are
         if (use >= 1 && !(ok = wwait(bar(B_KE + st), (use - 1) & 1, abort_flag, p.err, 202)))
           break;
         if (elect_one()) {
@@ -380,8 +384,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
     }
     // drain: every issued copy has landed before the CTA may exit
-    for (int q = issued_q - 2 > 0 ? issued_q - 2 : 0; q < issued_q; ++q)
-      mbar_drain(bar(B_QF + (q & 1)), (q >> 1) & 1);
+    if (issued_q > 0) mbar_drain(bar(B_QF), (issued_q - 1) & 1);
     for (int q = issued_k - kStages > 0 ? issued_k - kStages : 0; q < issued_k; ++q)
       mbar_drain(bar(B_KF + q % kStages), (q / kStages) & 1);
     for (int q = issued_v - kStages > 0 ? issued_v - kStages : 0; q < issued_v; ++q)
@@ -393,71 +396,69 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     constexpr uint32_t idO = idesc(BM, HD, true);
     // descriptors are built once; the start-address field (addr >> 4, low
     // 14 bits) is then advanced by plain adds (shared addresses < 256 KiB)
-    const uint64_t dq0 = sdesc(sbase + kOffQ, 16, 1024);
     const uint64_t dk0 = sdesc(sbase + kOffKV, 16, 1024);
     const uint64_t dv0 = sdesc(sbase + kOffKV + kKV, kKVHalf, 1024);
     int g0 = 0, it = 0;
     bool ok = true;
+    // PV_x of global tile g (tile j of item it): O_x += P_x V
+    auto issue_pv = [&](int x, int g, int j) -> bool {
+      if (!wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215)) return false;
+      if (j == 0 && it >= 1 && !wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216))
+        return false;                               // the epilogue has read the previous O_x
+      tc_fence_after();
+      const uint64_t dv = dv0 + (((g % kStages) * 2 * kKV) >> 4);
+      const uint32_t tp = tmem + col_s(x), dO = tmem + col_o(x);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_f16_ts(dO, tp + 8 * kk, dv + ((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+      return true;
+    };
     for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
       const Item m = make_item(p, i);
-      const int qb = it & 1;
-      if (!(ok = wwait(bar(B_QF + qb), (it >> 1) & 1, abort_flag, p.err, 211))) break;
-      const uint64_t dq = dq0 + ((qb * kQBuf) >> 4);
-      for (int j = 0; j <= m.total; ++j) {
-        if (j < m.total) {
-          const int g = g0 + j, st = g % kStages;
-          if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
-          const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
-          for (int x = 0; x < 2; ++x) {
-            if (g >= 1 && !(ok = wwait(bar(B_SFREE + x), (g - 1) & 1, abort_flag, p.err, 213)))
-              break;
-            tc_fence_after();
-            const uint64_t dqx = dq + ((x * kQTile) >> 4);
-            const uint32_t ds = tmem + col_s(x);
-            if (elect_one()) {
-#pragma unroll
-              for (int kk = 0; kk < HD / 16; ++kk) {
-                const uint32_t off = ((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4;
-                const uint32_t offk = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-                mma_f16(ds, dqx + off, dk + offk, idS, kk > 0);
-              }
-              mma_commit(bar(B_SF + x));
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
+      for (int j = 0; j < m.total && ok; ++j) {
+        const int g = g0 + j, st = g % kStages;
+        if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
+        if (j >= 1 && !(ok = wwait(bar(B_VF + (g - 1) % kStages), ((g - 1) / kStages) & 1,
+                                   abort_flag, p.err, 214)))
+          break;
+        const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (j >= 1 && !(ok = issue_pv(x, g - 1, j - 1))) break;
+          if (j == 0 && !(ok = wwait(bar(B_QC + x), it & 1, abort_flag, p.err, 213))) break;
+          tc_fence_after();
+          const uint32_t tq = tmem + col_q(x), ds = tmem + col_s(x);
           if (elect_one()) {
-            mma_commit(bar(B_KE + st));
-            if (j == m.total - 1) mma_commit(bar(B_QE + qb));
-          }
-          __syncwarp();
-        }
-        if (j >= 1) {
-          const int g = g0 + j - 1, st = g % kStages;
-          if (!(ok = wwait(bar(B_VF + st), (g / kStages) & 1, abort_flag, p.err, 214))) break;
-          const uint64_t dv = dv0 + ((st * 2 * kKV) >> 4);
-          for (int x = 0; x < 2; ++x) {
-            if (!(ok = wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215))) break;
-            if (j == 1 && it >= 1 &&
-                !(ok = wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216)))
-              break;
-            tc_fence_after();
-            const uint32_t tp = tmem + col_p(x);      // P: A operand in TMEM
-            const uint32_t dO = tmem + col_o(x);
-            const uint32_t acc0 = j > 1 ? 1u : 0u;
-            if (elect_one()) {
 #pragma unroll
-              for (int kk = 0; kk < BN / 16; ++kk)
-                mma_f16_ts(dO, tp + 8 * kk, dv + ((kk * 2048) >> 4), idO, kk > 0 ? 1u : acc0);
-              mma_commit(bar(B_PVD + x));
+            for (int kk = 0; kk < HD / 16; ++kk) {
+              const uint32_t offk = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+              mma_f16_ts(ds, tq + 8 * kk, dk + offk, idS, kk > 0);
             }
-            __syncwarp();
+            mma_commit(bar(B_SF + x));
           }
-          if (!ok) break;
-          if (elect_one()) mma_commit(bar(B_VE + st));
           __syncwarp();
         }
+        if (!ok) break;
+        if (elect_one()) {
+          mma_commit(bar(B_KE + st));
+          if (j >= 1) mma_commit(bar(B_VE + (g - 1) % kStages));
+        }
+        __syncwarp();
       }
+      if (!ok) break;
+      // the item's last tile: PV_A, PV_B, then the epilogue signal
+      const int gl = g0 + m.total - 1;
+      if (!(ok = wwait(bar(B_VF + gl % kStages), (gl / kStages) & 1, abort_flag, p.err, 214))) break;
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (!(ok = issue_pv(x, gl, m.total - 1))) break;
+        if (elect_one()) mma_commit(bar(B_PVD + x));
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (elect_one()) mma_commit(bar(B_VE + gl % kStages));
+      __syncwarp();
       g0 += m.total;
     }
     if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
@@ -469,12 +470,35 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t colS = col_s(x), colO = col_o(x), colP = col_p(x);
+    const uint32_t colS = col_s(x), colO = col_o(x), colQ = col_q(x);
     const int g_in_row = row % p.G;
-    int g0 = 0;
+    // copy this thread's Q row of the shared buffer (128B-swizzled halves) into TMEM
+    auto copy_q = [&](int it) -> bool {
+      bool ok = mbar_wait(bar(B_QF), it & 1, abort_flag, p.err, 224);
+      if (!(ok = __all_sync(0xffffffffu, ok))) return false;
+      const uint8_t* qrow = smem + kOffQ + x * kQTile + row * 128;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + hf * kQHalf + ((c ^ (row & 7)) << 4));
+          r[4 * c] = v4.x; r[4 * c + 1] = v4.y; r[4 * c + 2] = v4.z; r[4 * c + 3] = v4.w;
+        }
+        tmem_st32(lane_addr + colQ + hf * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_QC + x));
+      mbar_arrive(bar(B_QFREE));
+      return true;
+    };
+    int g0 = 0, it = 0;
     bool ok = true;
-    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x) {
+    if (blockIdx.x < p.n_items) ok = copy_q(0);
+    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
       const Item m = make_item(p, i);
+      const bool has_next = i + (int)gridDim.x < p.n_items;
       const int tt = m.t0 + x * p.TOK + row / p.G;
       const bool row_ok = tt < p.T;
       int hi_t = 0;
@@ -490,8 +514,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_ld32(lane_addr + colS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(lane_addr + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_SFREE + x));
+        // S_x of this item's last tile has run, so Q_x is no longer read: load the next item's Q
+        if (j == m.total - 1 && has_next && !(ok = copy_q(it + 1))) break;
         int rg, key0, nk;
         m.tile(j, rg, key0, nk);
         float s[64];
@@ -527,13 +551,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           m_ref = mx;
           l_sum *= corr;
         }
-        const bool any_rescale = __any_sync(0xffffffffu, need && corr != 0.f);
-        if (g >= 1) {      // P buffer free, and O current when this item already ran PV
-          ok = mbar_wait(bar(B_PVD + x), (g - 1) & 1, abort_flag, p.err, 222);
-          if (!(ok = __all_sync(0xffffffffu, ok))) break;
-          tc_fence_after();
-        }
-        if (any_rescale) {
+        // S_x(g) has completed, hence so has PV_x(g-1): O_x is current and P_x is free
+        if (__any_sync(0xffffffffu, need && corr != 0.f)) {
 #pragma unroll 1
           for (int c0 = 0; c0 < HD; c0 += 32) {
             uint32_t orr[32];
@@ -560,7 +579,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           __nv_bfloat162 v2 = __floats2bfloat162_rn(z.x, z.y);
           pk[c2] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        tmem_st32(lane_addr + colP, pk);
+        tmem_st32(lane_addr + colS, pk);           // P_x over the first 32 columns of S_x
         const float2 a01 = __fadd2_rn(acc2[0], acc2[1]), a23 = __fadd2_rn(acc2[2], acc2[3]);
         const float2 a = __fadd2_rn(a01, a23);
         l_sum += a.x + a.y;
@@ -570,38 +589,35 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16, lse; then hand O back to the MMA warp
-      const int g_last = g0 + m.total - 1;
-      if (m.total > 0) {
-        ok = mbar_wait(bar(B_PVD + x), g_last & 1, abort_flag, p.err, 223);
-        if (!(ok = __all_sync(0xffffffffu, ok))) break;
-        tc_fence_after();
-        const float inv = 1.f / l_sum;
-        __nv_bfloat16* orow = p.o + (long long)m.b * p.os.b + (long long)(row_ok ? tt : 0) * p.os.t +
-                              (long long)(m.h * p.G + g_in_row) * p.os.h;
+      ok = mbar_wait(bar(B_PVD + x), it & 1, abort_flag, p.err, 223);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float inv = 1.f / l_sum;
+      __nv_bfloat16* orow = p.o + (long long)m.b * p.os.b + (long long)(row_ok ? tt : 0) * p.os.t +
+                            (long long)(m.h * p.G + g_in_row) * p.os.h;
 #pragma unroll 1
-        for (int c0 = 0; c0 < HD; c0 += 32) {
-          uint32_t orr[32];
-          tmem_ld32(lane_addr + colO + c0, orr);
-          tmem_wait_ld();
-          if (row_ok) {
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t orr[32];
+        tmem_ld32(lane_addr + colO + c0, orr);
+        tmem_wait_ld();
+        if (row_ok) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 v;
-              uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-              for (int f = 0; f < 4; ++f) {
-                __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[e + 2 * f]) * inv,
-                                                          __uint_as_float(orr[e + 2 * f + 1]) * inv);
-                w[f] = *reinterpret_cast<uint32_t*>(&v2);
-              }
-              *reinterpret_cast<uint4*>(orow + c0 + e) = v;
+            for (int f = 0; f < 4; ++f) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[e + 2 * f]) * inv,
+                                                        __uint_as_float(orr[e + 2 * f + 1]) * inv);
+              w[f] = *reinterpret_cast<uint32_t*>(&v2);
             }
+            *reinterpret_cast<uint4*>(orow + c0 + e) = v;
           }
         }
-        if (row_ok && p.lse != nullptr)
-          p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
-              (m_ref + log2f(l_sum)) * 0.69314718055994531f;
       }
+      if (row_ok && p.lse != nullptr)
+        p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
+            (m_ref + log2f(l_sum)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(bar(B_OE + x));
       g0 += m.total;
