@@ -30,13 +30,15 @@
 //              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
 //              P_x may then be overwritten and O_x rescaled without a wait;
 //   warps 2-5  softmax of tile A, warps 6-9 of tile B: one thread per row
-//              reads its S row from TMEM, applies the attended-set predicate,
-//              exp2 via ex2.approx with the scale folded into a packed FMA,
-//              writes P into TMEM, and rescales its O row only when the
-//              running max grew by more than 2^8 (exact: O and l share the
-//              reference max).  During an item's last tile it copies the next
-//              item's Q rows into TMEM, so that item's first S overlaps this
-//              item's epilogue (O / l -> bf16, lse).
+//              reads its S row from TMEM, applies the attended-set predicate
+//              (a 64-bit set of at most two column intervals), exp2 via
+//              ex2.approx with the scale folded into a packed FMA, writes P
+//              into TMEM, and rescales its O row only when the running max
+//              grew by more than 2^8 (exact: O and l share the reference max).
+//              During an item's last tile it copies the next item's Q rows
+//              into TMEM, so that item's first S overlaps this item's
+//              epilogue: O / l -> bf16 rows staged in the (now copied) Q
+//              buffer, written out by TMA stores, and lse.
 // Every mbarrier wait is bounded (1 s of global time): on expiry the CTA
 // records LTE_ERR_TIMEOUT in the workspace error word, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and exits.
@@ -63,7 +65,7 @@ constexpr int kStages = 4;                        // K/V ring depth
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKV = kQBuf;                // stage s: K at +s*32K, V at +16K
 constexpr uint32_t kOffBar = kOffKV + kStages * 2 * kKV;   // 192 KiB
-constexpr uint32_t kSmemBytes = kOffBar + 256;
+constexpr uint32_t kSmemBytes = kOffBar + 512;
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int x) { return x == 0 ? 0u : 64u; }     // S (and P)
 __host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256u; }  // O
@@ -72,16 +74,15 @@ constexpr unsigned long long kWaitNs = 1000000000ull;
 
 enum {
   B_QF = 0, B_QFREE = 1, B_QC = 2, B_KF = 4, B_VF = 8, B_KE = 12, B_VE = 16, B_SF = 20,
-  B_PF = 22, B_PVD = 24, B_OE = 26, B_FIN = 28, kNumBars = 29
+  B_PF = 22, B_PVD = 24, B_OE = 26, B_FIN = 28, B_OST = 29, B_STG = 31, kNumBars = 33
 };
+static_assert(8 * kNumBars + 8 <= 512, "barriers, abort flag and TMEM slot fit the tail");
 
 struct Params {
   int T, Hq, Hkv, G, TOK, sink, window, cap;
   int n_pairs, n_units, n_items;
   float scale_log2;
   const int32_t* cnt;
-  __nv_bfloat16* o;
-  Strides4 os;
   float* lse;
   DevError* err;
 };
@@ -159,6 +160,23 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy shared-memory writes -> visible to the TMA (async proxy)
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // One lane of a converged warp (elect.sync): the issuing warps run their loops
 // with all 32 lanes, so descriptors and coordinates stay warp-uniform, and
@@ -242,6 +260,15 @@ __device__ __forceinline__ float ex2(float x) {   // 2^x, approximate (MUFU)
   return y;
 }
 
+// Columns [a, b) of a 64-key tile as a bit set (empty when b <= a).
+__device__ __forceinline__ uint64_t span_bits(int a, int b) {
+  a = a > 0 ? a : 0;
+  b = b < BN ? b : BN;
+  if (b <= a) return 0ull;
+  const uint64_t ones = (b - a == 64) ? ~0ull : ((1ull << (b - a)) - 1ull);
+  return ones << a;
+}
+
 // ---------------------------------------------------------------- work items
 struct Item {
   int b, h, u, t0, t_last;     // tokens [t0, t_last] over both Q tiles
@@ -291,7 +318,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_kc,
-                       const __grid_constant__ CUtensorMap tm_vc, const Params p) {
+                       const __grid_constant__ CUtensorMap tm_vc,
+                       const __grid_constant__ CUtensorMap tm_o, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = sa(smem);
@@ -321,6 +349,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar(B_OE + x), 128);
     }
     mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(B_OST), 1);
+    mbar_init(bar(B_OST + 1), 1);
+    mbar_init(bar(B_STG), 128);
+    mbar_init(bar(B_STG + 1), 128);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -344,7 +376,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
       const Item m = make_item(p, i);
       // the shared Q buffer is free once both softmax groups copied the last item's rows
+      // out of it and the output store staged in it two items back has been read
       if (it >= 1 && !(ok = wwait(bar(B_QFREE), (it - 1) & 1, abort_flag, p.err, 201))) break;
+      if (it >= 2 && !((ok = wwait(bar(B_OST), (it - 2) & 1, abort_flag, p.err, 204)) &&
+                       (ok = wwait(bar(B_OST + 1), (it - 2) & 1, abort_flag, p.err, 204))))
+        break;
       if (elect_one()) {
         mbar_expect_tx(bar(B_QF), kQBuf);
         for (int x = 0; x < 2; ++x)
@@ -521,19 +557,25 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        // attended-set predicate, skipped when the whole tile is inside S_t
-        bool full;
-        if (rg == 2) full = nk == BN && key0 > tt - p.window && key0 + BN - 1 <= tt;
-        else full = nk == BN && key0 >= p.sink && key0 - p.sink >= lo_t && key0 - p.sink + BN <= hi_t;
-        if (!(full && row_ok)) {
+        // attended-set predicate as a bit set over the tile's columns: the window
+        // band is one interval; a slot tile holds the visible sinks and the
+        // retained slots [lo_t, hi_t), two intervals
+        uint64_t bits = 0ull;
+        if (row_ok) {
+          if (rg == 2) {
+            bits = span_bits(tt - p.window + 1 - key0, min(nk, tt - key0 + 1));
+          } else {
+            const int sink_end = min(p.sink, tt - p.window + 1);
+            bits = span_bits(-key0, min(nk, sink_end - key0)) |
+                   span_bits(p.sink + lo_t - key0, min(nk, p.sink + hi_t - key0));
+          }
+        }
+        if (bits != ~0ull) {
+          const uint32_t b0 = (uint32_t)bits, b1 = (uint32_t)(bits >> 32);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int key = key0 + c;
-            bool in;
-            if (rg == 2) in = key <= tt && key > tt - p.window;
-            else if (key < p.sink) in = key <= tt - p.window;
-            else in = key - p.sink >= lo_t && key - p.sink < hi_t;
-            if (!(in && c < nk && row_ok)) s[c] = -INFINITY;
+          for (int c = 0; c < 32; ++c) {
+            if (!((b0 >> c) & 1u)) s[c] = -INFINITY;
+            if (!((b1 >> c) & 1u)) s[32 + c] = -INFINITY;
           }
         }
         float m8[8];
@@ -588,40 +630,54 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(bar(B_PF + x));
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16, lse; then hand O back to the MMA warp
+      // ---- epilogue: O / l -> bf16 rows staged in this tile's region of the Q
+      // buffer (thread `row` has already copied its row of the next item's Q
+      // out of it), then one TMA store per 64-column half; rows past T are
+      // clipped by the copy
       ok = mbar_wait(bar(B_PVD + x), it & 1, abort_flag, p.err, 223);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const float inv = 1.f / l_sum;
-      __nv_bfloat16* orow = p.o + (long long)m.b * p.os.b + (long long)(row_ok ? tt : 0) * p.os.t +
-                            (long long)(m.h * p.G + g_in_row) * p.os.h;
+      const float inv = __frcp_rn(l_sum);
+      uint8_t* srow = smem + kOffQ + x * kQTile + row * 128;
 #pragma unroll 1
       for (int c0 = 0; c0 < HD; c0 += 32) {
         uint32_t orr[32];
         tmem_ld32(lane_addr + colO + c0, orr);
         tmem_wait_ld();
-        if (row_ok) {
+        uint8_t* half = srow + (c0 >> 6) * kQHalf;
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 v;
-            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+        for (int e = 0; e < 4; ++e) {               // 16-byte chunk (c0 % 64) / 8 + e of the half row
+          uint4 v;
+          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[e + 2 * f]) * inv,
-                                                        __uint_as_float(orr[e + 2 * f + 1]) * inv);
-              w[f] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(orow + c0 + e) = v;
+          for (int f = 0; f < 4; ++f) {
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[8 * e + 2 * f]) * inv,
+                                                      __uint_as_float(orr[8 * e + 2 * f + 1]) * inv);
+            w[f] = *reinterpret_cast<uint32_t*>(&v2);
           }
+          const int chunk = ((c0 & 63) >> 3) + e;
+          *reinterpret_cast<uint4*>(half + ((chunk ^ (row & 7)) << 4)) = v;
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar(B_OE + x));                  // O_x has been read: the next item may overwrite it
       if (row_ok && p.lse != nullptr)
         p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
-            (m_ref + log2f(l_sum)) * 0.69314718055994531f;
-      tc_fence_before();
-      mbar_arrive(bar(B_OE + x));
+            (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+      fence_proxy_async();
+      mbar_arrive(bar(B_STG + x));                  // this row is staged
+      if (row == 0) {
+        if (!mbar_wait(bar(B_STG + x), it & 1, abort_flag, p.err, 225)) break;
+        const uint32_t src = sbase + kOffQ + x * kQTile;
+        tma_store_4d(&tm_o, src, 0, m.h * p.G, m.t0 + x * p.TOK, m.b);
+        tma_store_4d(&tm_o, src + kQHalf, 64, m.h * p.G, m.t0 + x * p.TOK, m.b);
+        bulk_commit();
+        bulk_wait_read();                            // staging rows read: the buffer may be reloaded
+        mbar_arrive(bar(B_OST + x));
+      }
       g0 += m.total;
     }
+    if (row == 0) bulk_wait_all();                 // output stores complete before exit
   }
   tc_fence_before();
   __syncthreads();
@@ -667,16 +723,27 @@ bool attn_prefill_tc_supported(const lte_dims* d) {
          (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
+// Tensor maps need every byte stride a multiple of 16 (pointers are checked at the API).
+bool attn_prefill_tc_layout_ok(const PrefillArgs& a) {
+  const Strides4* ss[3] = {&a.qs, &a.kvs, &a.os};
+  for (const Strides4* s : ss)
+    if ((s->h * 2) % 16 != 0 || (s->t * 2) % 16 != 0 || (s->b * 2) % 16 != 0) return false;
+  return true;
+}
+
 cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   using namespace tc;
   const lte_dims* d = a.d;
   const int G = d->Hq / d->Hkv, TOK = BM / G;
-  CUtensorMap mq, mk, mv, mkc, mvc;
+  CUtensorMap mq, mk, mv, mkc, mvc, mo;
   {
+    // Q rows are loaded and O rows stored in the same box: G heads x TOK tokens
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)d->Hq, (cuuint64_t)d->T, (cuuint64_t)d->B};
     const cuuint64_t st[3] = {(cuuint64_t)a.qs.h * 2, (cuuint64_t)a.qs.t * 2, (cuuint64_t)a.qs.b * 2};
+    const cuuint64_t so[3] = {(cuuint64_t)a.os.h * 2, (cuuint64_t)a.os.t * 2, (cuuint64_t)a.os.b * 2};
     const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)TOK, 1};
     if (!encode(&mq, a.q, 4, dims, st, box)) return cudaErrorInvalidValue;
+    if (!encode(&mo, a.o, 4, dims, so, box)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)d->Hkv, (cuuint64_t)d->T, (cuuint64_t)d->B};
@@ -702,7 +769,7 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   p.n_items = p.n_pairs * p.n_units;
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.cnt = a.cnt;
-  p.o = (__nv_bfloat16*)a.o; p.os = a.os; p.lse = a.lse; p.err = a.err;
+  p.lse = a.lse; p.err = a.err;
   cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -710,7 +777,7 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.n_items < n_sm ? p.n_items : n_sm;
-  attn_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mkc, mvc, p);
+  attn_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mkc, mvc, mo, p);
   return cudaGetLastError();
 }
 

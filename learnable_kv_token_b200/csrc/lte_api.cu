@@ -144,10 +144,12 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
   a.err = reinterpret_cast<lte::DevError*>(workspace);
   a.scratch = static_cast<char*>(workspace) + kErrBytes;
   a.scratch_bytes = ws_bytes - kErrBytes;
-  // bf16, head dim 128: tcgen05/TMEM/TMA kernel; other bf16 shapes: warp-MMA kernel;
-  // fp32: SIMT kernel.  All three are GPU kernels; there is no host path.
+  // bf16, head dim 128, 16-byte strides: tcgen05/TMEM/TMA kernel; other bf16
+  // shapes: warp-MMA kernel; fp32: SIMT kernel.  All three are GPU kernels;
+  // there is no host path.
   cudaError_t e;
-  if (lte::attn_prefill_tc_supported(d)) e = lte::attn_prefill_tc(a, as_stream(stream));
+  if (lte::attn_prefill_tc_supported(d) && lte::attn_prefill_tc_layout_ok(a))
+    e = lte::attn_prefill_tc(a, as_stream(stream));
   else if (d->dtype == LTE_BF16) e = lte::attn_prefill_mma(a, as_stream(stream));
   else e = lte::attn_prefill_simt(a, as_stream(stream));
   return from_cuda(e);

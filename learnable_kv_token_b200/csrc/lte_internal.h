@@ -40,6 +40,7 @@ struct PrefillArgs {
 cudaError_t attn_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t attn_prefill_mma(const PrefillArgs& a, cudaStream_t stream);
 bool attn_prefill_tc_supported(const lte_dims* d);
+bool attn_prefill_tc_layout_ok(const PrefillArgs& a);
 cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
 size_t attn_prefill_scratch_bytes(const lte_dims* d);
 
