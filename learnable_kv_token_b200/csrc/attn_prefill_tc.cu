@@ -20,7 +20,7 @@
 // columns are reused for P_x as bf16 pairs), O_x (128) and Q_x (64, bf16
 // pairs).  Both products read their A operand from TMEM (Q for S = Q K^T, P
 // for O += P V), so shared memory only feeds K and V to the tensor core.
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: the item's Q rows into one shared buffer (freed as
 //              soon as both softmax groups copied them into TMEM), K and V
 //              into 4-slot rings (a K slot frees after its S MMAs, a V slot
@@ -29,7 +29,8 @@
 //              PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  The tensor pipe runs in
 //              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
 //              P_x may then be overwritten and O_x rescaled without a wait;
-//   warps 2-5  softmax of tile A, warps 6-9 of tile B: one thread per row
+//   warps 2-3  idle (they complete warpgroup 0, whose registers go to softmax)
+//   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per row
 //              reads its S row from TMEM, applies the attended-set predicate
 //              (a 64-bit set of at most two column intervals), exp2 via
 //              ex2.approx with the scale folded into a packed FMA, writes P
@@ -55,7 +56,12 @@ namespace tc {
 constexpr int BM = 128;             // rows per Q tile (TMEM lanes)
 constexpr int BN = 64;              // keys per K/V tile
 constexpr int HD = 128;             // head dim
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// register split (setmaxnreg): the launch gives 168 per thread (3 warps per
+// sub-partition); warpgroup 0 (TMA, MMA, two idle warps) drops to 64 and the
+// two softmax warpgroups rise to 216: 4 * 64 + 8 * 216 <= 12 * 168
+constexpr int kRegsLaunch = 168, kRegsIssue = 64, kRegsSoftmax = 216;
+static_assert(4 * kRegsIssue + 8 * kRegsSoftmax <= 12 * kRegsLaunch, "register split fits the launch");
 constexpr uint32_t kQTile = BM * HD * 2;          // 32 KiB
 constexpr uint32_t kQHalf = BM * 128;             // 64-column half of a Q tile: 16 KiB
 constexpr uint32_t kQBuf = 2 * kQTile;            // tiles A and B of one item: 64 KiB
@@ -269,6 +275,32 @@ __device__ __forceinline__ uint64_t span_bits(int a, int b) {
   return ones << a;
 }
 
+// 2^x for a pair of fp32 values on the FMA pipe (the special-function unit
+// evaluates the others).  Range reduction 2^x = 2^n * 2^f with n = round(x),
+// obtained by adding 1.5 * 2^23 (which leaves n in the low mantissa bits),
+// and f = x - n in [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted by least
+// squares on Chebyshev nodes with p(0) = 1 (relative error 1.3e-7, below the
+// bf16 rounding of P by 2^-16; gen_exp2_poly.py prints the fit); 2^n enters
+// as an integer add to the exponent field.  Inputs are clamped to >= -126 so
+// the exponent stays normal: a masked key (x = -inf) gets 2^-126 rather than 0,
+// which no fp32 sum of at least one unit term can register.
+constexpr int kPolyEvery = 0;       // > 0: every kPolyEvery-th pair of S columns takes the polynomial
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(1.340043265e-03f, 1.340043265e-03f), f,
+                        make_float2(9.672171436e-03f, 9.672171436e-03f));
+  q = __ffma2_rn(q, f, make_float2(5.550327152e-02f, 5.550327152e-02f));
+  q = __ffma2_rn(q, f, make_float2(2.402222753e-01f, 2.402222753e-01f));
+  q = __ffma2_rn(q, f, make_float2(6.931471825e-01f, 6.931471825e-01f));
+  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ---------------------------------------------------------------- work items
 struct Item {
   int b, h, u, t0, t_last;     // tokens [t0, t_last] over both Q tiles
@@ -284,17 +316,34 @@ struct Item {
   }
 };
 
-__device__ __forceinline__ Item make_item(const Params& p, int i) {
-  Item m;
+// The retained counts an item's key ranges depend on, loaded one item ahead
+// (each role issues the next item's loads while it works on the current one,
+// so their latency never stalls the pipeline).
+struct ItemCounts {
+  int n_first, n_last;
+};
+__device__ __forceinline__ void item_tokens(const Params& p, int i, int& u, int& t0, int& t_last) {
   const int pair = p.n_pairs - 1 - i / p.n_units;   // late (heavy) tokens first
-  m.u = i % p.n_units;
+  u = i % p.n_units;
+  t0 = pair * 2 * p.TOK;
+  t_last = min(t0 + 2 * p.TOK - 1, p.T - 1);
+}
+__device__ __forceinline__ ItemCounts load_counts(const Params& p, int i) {
+  ItemCounts c{0, 0};
+  if (i >= p.n_items) return c;
+  int u, t0, t_last;
+  item_tokens(p, i, u, t0, t_last);
+  const long long crow = (long long)u * p.T;
+  if (t0 >= p.window) c.n_first = __ldg(p.cnt + crow + t0 - p.window);
+  if (t_last >= p.window) c.n_last = __ldg(p.cnt + crow + t_last - p.window);
+  return c;
+}
+__device__ __forceinline__ Item make_item(const Params& p, int i, const ItemCounts& c) {
+  Item m;
+  item_tokens(p, i, m.u, m.t0, m.t_last);
   m.b = m.u / p.Hkv;
   m.h = m.u % p.Hkv;
-  m.t0 = pair * 2 * p.TOK;
-  m.t_last = min(m.t0 + 2 * p.TOK - 1, p.T - 1);
-  const long long crow = (long long)m.u * p.T;
-  const int n_first = (m.t0 >= p.window) ? p.cnt[crow + m.t0 - p.window] : 0;
-  const int n_last = (m.t_last >= p.window) ? p.cnt[crow + m.t_last - p.window] : 0;
+  const int n_first = c.n_first, n_last = c.n_last;
   const int lo_min = n_first - p.cap > 0 ? n_first - p.cap : 0;
   int nsink = m.t_last - p.window + 1;
   nsink = nsink < 0 ? 0 : (nsink > p.sink ? p.sink : nsink);
@@ -368,141 +417,150 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ============================================================ TMA producer
-    // (all 32 lanes run the loop and wait; one elected lane issues)
-    int g = 0, it = 0, issued_k = 0, issued_v = 0, issued_q = 0;
-    bool ok = true;
-    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
-      const Item m = make_item(p, i);
-      // the shared Q buffer is free once both softmax groups copied the last item's rows
-      // out of it and the output store staged in it two items back has been read
-      if (it >= 1 && !(ok = wwait(bar(B_QFREE), (it - 1) & 1, abort_flag, p.err, 201))) break;
-      if (it >= 2 && !((ok = wwait(bar(B_OST), (it - 2) & 1, abort_flag, p.err, 204)) &&
-                       (ok = wwait(bar(B_OST + 1), (it - 2) & 1, abort_flag, p.err, 204))))
-        break;
-      if (elect_one()) {
-        mbar_expect_tx(bar(B_QF), kQBuf);
-        for (int x = 0; x < 2; ++x)
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + kOffQ + x * kQTile + hf * kQHalf, &tm_q, bar(B_QF), hf * 64,
-                        m.h * p.G, m.t0 + x * p.TOK, m.b);
-      }
-      __syncwarp();
-      issued_q = it + 1;
-      for (int j = 0; j < m.total; ++j, ++g) {
-        const int st = g % kStages, use = g / kStages;
-        int rg, key0, nk;
-        m.tile(j, rg, key0, nk);
-        const uint32_t kd = sbase + kOffKV + st * 2 * kKV, vd = kd + kKV;
-        if (use >= 1 && !(ok = wwait(bar(B_KE + st), (use - 1) & 1, abort_flag, p.err, 202)))
+  if (warp < 4) {
+    // warpgroup 0: its registers go to the softmax warpgroups
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIssue));
+    if (warp == 0) {
+      // ============================================================ TMA producer
+      // (all 32 lanes run the loop and wait; one elected lane issues)
+      int g = 0, it = 0, issued_k = 0, issued_v = 0, issued_q = 0;
+      bool ok = true;
+      ItemCounts cn = load_counts(p, blockIdx.x);
+      for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
+        const Item m = make_item(p, i, cn);
+        cn = load_counts(p, i + gridDim.x);
+        // the shared Q buffer is free once both softmax groups copied the last item's rows
+        // out of it and the output store staged in it two items back has been read
+        if (it >= 1 && !(ok = wwait(bar(B_QFREE), (it - 1) & 1, abort_flag, p.err, 201))) break;
+        if (it >= 2 && !((ok = wwait(bar(B_OST), (it - 2) & 1, abort_flag, p.err, 204)) &&
+                         (ok = wwait(bar(B_OST + 1), (it - 2) & 1, abort_flag, p.err, 204))))
           break;
         if (elect_one()) {
-          mbar_expect_tx(bar(B_KF + st), kKV);
-          for (int hf = 0; hf < 2; ++hf) {
-            if (rg == 2) tma_load_4d(kd + hf * kKVHalf, &tm_k, bar(B_KF + st), hf * 64, m.h, key0, m.b);
-            else tma_load_3d(kd + hf * kKVHalf, &tm_kc, bar(B_KF + st), hf * 64, key0, m.u);
-          }
+          mbar_expect_tx(bar(B_QF), kQBuf);
+          for (int x = 0; x < 2; ++x)
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + kOffQ + x * kQTile + hf * kQHalf, &tm_q, bar(B_QF), hf * 64,
+                          m.h * p.G, m.t0 + x * p.TOK, m.b);
         }
         __syncwarp();
-        issued_k = g + 1;
-        if (use >= 1 && !(ok = wwait(bar(B_VE + st), (use - 1) & 1, abort_flag, p.err, 203)))
-          break;
-        if (elect_one()) {
-          mbar_expect_tx(bar(B_VF + st), kKV);
-          for (int hf = 0; hf < 2; ++hf) {
-            if (rg == 2) tma_load_4d(vd + hf * kKVHalf, &tm_v, bar(B_VF + st), hf * 64, m.h, key0, m.b);
-            else tma_load_3d(vd + hf * kKVHalf, &tm_vc, bar(B_VF + st), hf * 64, key0, m.u);
-          }
-        }
-        __syncwarp();
-        issued_v = g + 1;
-      }
-    }
-    // drain: every issued copy has landed before the CTA may exit
-    if (issued_q > 0) mbar_drain(bar(B_QF), (issued_q - 1) & 1);
-    for (int q = issued_k - kStages > 0 ? issued_k - kStages : 0; q < issued_k; ++q)
-      mbar_drain(bar(B_KF + q % kStages), (q / kStages) & 1);
-    for (int q = issued_v - kStages > 0 ? issued_v - kStages : 0; q < issued_v; ++q)
-      mbar_drain(bar(B_VF + q % kStages), (q / kStages) & 1);
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
-    // (all 32 lanes run the loop and wait; one elected lane issues)
-    constexpr uint32_t idS = idesc(BM, BN, false);
-    constexpr uint32_t idO = idesc(BM, HD, true);
-    // descriptors are built once; the start-address field (addr >> 4, low
-    // 14 bits) is then advanced by plain adds (shared addresses < 256 KiB)
-    const uint64_t dk0 = sdesc(sbase + kOffKV, 16, 1024);
-    const uint64_t dv0 = sdesc(sbase + kOffKV + kKV, kKVHalf, 1024);
-    int g0 = 0, it = 0;
-    bool ok = true;
-    // PV_x of global tile g (tile j of item it): O_x += P_x V
-    auto issue_pv = [&](int x, int g, int j) -> bool {
-      if (!wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215)) return false;
-      if (j == 0 && it >= 1 && !wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216))
-        return false;                               // the epilogue has read the previous O_x
-      tc_fence_after();
-      const uint64_t dv = dv0 + (((g % kStages) * 2 * kKV) >> 4);
-      const uint32_t tp = tmem + col_s(x), dO = tmem + col_o(x);
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_f16_ts(dO, tp + 8 * kk, dv + ((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
-      const Item m = make_item(p, i);
-      for (int j = 0; j < m.total && ok; ++j) {
-        const int g = g0 + j, st = g % kStages;
-        if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
-        if (j >= 1 && !(ok = wwait(bar(B_VF + (g - 1) % kStages), ((g - 1) / kStages) & 1,
-                                   abort_flag, p.err, 214)))
-          break;
-        const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (j >= 1 && !(ok = issue_pv(x, g - 1, j - 1))) break;
-          if (j == 0 && !(ok = wwait(bar(B_QC + x), it & 1, abort_flag, p.err, 213))) break;
-          tc_fence_after();
-          const uint32_t tq = tmem + col_q(x), ds = tmem + col_s(x);
+        issued_q = it + 1;
+        for (int j = 0; j < m.total; ++j, ++g) {
+          const int st = g % kStages, use = g / kStages;
+          int rg, key0, nk;
+          m.tile(j, rg, key0, nk);
+          const uint32_t kd = sbase + kOffKV + st * 2 * kKV, vd = kd + kKV;
+          if (use >= 1 && !(ok = wwait(bar(B_KE + st), (use - 1) & 1, abort_flag, p.err, 202)))
+            break;
           if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
-              const uint32_t offk = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
-              mma_f16_ts(ds, tq + 8 * kk, dk + offk, idS, kk > 0);
+            mbar_expect_tx(bar(B_KF + st), kKV);
+            for (int hf = 0; hf < 2; ++hf) {
+              if (rg == 2) tma_load_4d(kd + hf * kKVHalf, &tm_k, bar(B_KF + st), hf * 64, m.h, key0, m.b);
+              else tma_load_3d(kd + hf * kKVHalf, &tm_kc, bar(B_KF + st), hf * 64, key0, m.u);
             }
-            mma_commit(bar(B_SF + x));
+          }
+          __syncwarp();
+          issued_k = g + 1;
+          if (use >= 1 && !(ok = wwait(bar(B_VE + st), (use - 1) & 1, abort_flag, p.err, 203)))
+            break;
+          if (elect_one()) {
+            mbar_expect_tx(bar(B_VF + st), kKV);
+            for (int hf = 0; hf < 2; ++hf) {
+              if (rg == 2) tma_load_4d(vd + hf * kKVHalf, &tm_v, bar(B_VF + st), hf * 64, m.h, key0, m.b);
+              else tma_load_3d(vd + hf * kKVHalf, &tm_vc, bar(B_VF + st), hf * 64, key0, m.u);
+            }
+          }
+          __syncwarp();
+          issued_v = g + 1;
+        }
+      }
+      // drain: every issued copy has landed before the CTA may exit
+      if (issued_q > 0) mbar_drain(bar(B_QF), (issued_q - 1) & 1);
+      for (int q = issued_k - kStages > 0 ? issued_k - kStages : 0; q < issued_k; ++q)
+        mbar_drain(bar(B_KF + q % kStages), (q / kStages) & 1);
+      for (int q = issued_v - kStages > 0 ? issued_v - kStages : 0; q < issued_v; ++q)
+        mbar_drain(bar(B_VF + q % kStages), (q / kStages) & 1);
+    } else if (warp == 1) {
+      // ============================================================ MMA issuer
+      // (all 32 lanes run the loop and wait; one elected lane issues)
+      constexpr uint32_t idS = idesc(BM, BN, false);
+      constexpr uint32_t idO = idesc(BM, HD, true);
+      // descriptors are built once; the start-address field (addr >> 4, low
+      // 14 bits) is then advanced by plain adds (shared addresses < 256 KiB)
+      const uint64_t dk0 = sdesc(sbase + kOffKV, 16, 1024);
+      const uint64_t dv0 = sdesc(sbase + kOffKV + kKV, kKVHalf, 1024);
+      int g0 = 0, it = 0;
+      bool ok = true;
+      // PV_x of global tile g (tile j of item it): O_x += P_x V
+      auto issue_pv = [&](int x, int g, int j) -> bool {
+        if (!wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215)) return false;
+        if (j == 0 && it >= 1 && !wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216))
+          return false;                               // the epilogue has read the previous O_x
+        tc_fence_after();
+        const uint64_t dv = dv0 + (((g % kStages) * 2 * kKV) >> 4);
+        const uint32_t tp = tmem + col_s(x), dO = tmem + col_o(x);
+        if (elect_one()) {
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_f16_ts(dO, tp + 8 * kk, dv + ((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        return true;
+      };
+      ItemCounts cn = load_counts(p, blockIdx.x);
+      for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
+        const Item m = make_item(p, i, cn);
+        cn = load_counts(p, i + gridDim.x);
+        for (int j = 0; j < m.total && ok; ++j) {
+          const int g = g0 + j, st = g % kStages;
+          if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
+          if (j >= 1 && !(ok = wwait(bar(B_VF + (g - 1) % kStages), ((g - 1) / kStages) & 1,
+                                     abort_flag, p.err, 214)))
+            break;
+          const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j >= 1 && !(ok = issue_pv(x, g - 1, j - 1))) break;
+            if (j == 0 && !(ok = wwait(bar(B_QC + x), it & 1, abort_flag, p.err, 213))) break;
+            tc_fence_after();
+            const uint32_t tq = tmem + col_q(x), ds = tmem + col_s(x);
+            if (elect_one()) {
+  #pragma unroll
+              for (int kk = 0; kk < HD / 16; ++kk) {
+                const uint32_t offk = ((kk >> 2) * kKVHalf + (kk & 3) * 32) >> 4;
+                mma_f16_ts(ds, tq + 8 * kk, dk + offk, idS, kk > 0);
+              }
+              mma_commit(bar(B_SF + x));
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (elect_one()) {
+            mma_commit(bar(B_KE + st));
+            if (j >= 1) mma_commit(bar(B_VE + (g - 1) % kStages));
           }
           __syncwarp();
         }
         if (!ok) break;
-        if (elect_one()) {
-          mma_commit(bar(B_KE + st));
-          if (j >= 1) mma_commit(bar(B_VE + (g - 1) % kStages));
+        // the item's last tile: PV_A, PV_B, then the epilogue signal
+        const int gl = g0 + m.total - 1;
+        if (!(ok = wwait(bar(B_VF + gl % kStages), (gl / kStages) & 1, abort_flag, p.err, 214))) break;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (!(ok = issue_pv(x, gl, m.total - 1))) break;
+          if (elect_one()) mma_commit(bar(B_PVD + x));
+          __syncwarp();
         }
+        if (!ok) break;
+        if (elect_one()) mma_commit(bar(B_VE + gl % kStages));
         __syncwarp();
+        g0 += m.total;
       }
-      if (!ok) break;
-      // the item's last tile: PV_A, PV_B, then the epilogue signal
-      const int gl = g0 + m.total - 1;
-      if (!(ok = wwait(bar(B_VF + gl % kStages), (gl / kStages) & 1, abort_flag, p.err, 214))) break;
-      for (int x = 0; x < 2 && ok; ++x) {
-        if (!(ok = issue_pv(x, gl, m.total - 1))) break;
-        if (elect_one()) mma_commit(bar(B_PVD + x));
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (elect_one()) mma_commit(bar(B_VE + gl % kStages));
+      if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
       __syncwarp();
-      g0 += m.total;
+      mbar_drain(bar(B_FIN), 0);
     }
-    if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
-    __syncwarp();
-    mbar_drain(bar(B_FIN), 0);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ============================================================ softmax + epilogue
-    const int x = (warp - 2) >> 2;                 // Q tile of this warpgroup
+    const int x = (warp - 4) >> 2;                 // Q tile of this warpgroup
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
@@ -532,17 +590,48 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     int g0 = 0, it = 0;
     bool ok = true;
     if (blockIdx.x < p.n_items) ok = copy_q(0);
+    // this row's retained count n_t = cnt[t - w] of item i (0 if none), loaded one item ahead
+    auto row_count = [&](int i) -> int {
+      if (i >= p.n_items) return 0;
+      int u, t0, t_last;
+      item_tokens(p, i, u, t0, t_last);
+      const int t = t0 + x * p.TOK + row / p.G;
+      return (t < p.T && t >= p.window) ? __ldg(p.cnt + (long long)u * p.T + t - p.window) : 0;
+    };
+    ItemCounts cn = load_counts(p, blockIdx.x);
+    int hi_next = row_count(blockIdx.x);
     for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
-      const Item m = make_item(p, i);
+      const Item m = make_item(p, i, cn);
+      const int hi_t = hi_next;
+      cn = load_counts(p, i + gridDim.x);
+      hi_next = row_count(i + gridDim.x);
       const bool has_next = i + (int)gridDim.x < p.n_items;
       const int tt = m.t0 + x * p.TOK + row / p.G;
       const bool row_ok = tt < p.T;
-      int hi_t = 0;
-      if (row_ok && tt >= p.window) hi_t = p.cnt[(long long)m.u * p.T + tt - p.window];
       const int lo_t = hi_t - p.cap > 0 ? hi_t - p.cap : 0;
+      // attended-set predicate of tile j as a bit set over its columns: the
+      // window band is one interval; a slot tile holds the visible sinks and
+      // the retained slots [lo_t, hi_t), two intervals.  It does not depend on
+      // S, so each tile's set is built while the warp waits for that S.
+      auto tile_bits = [&](int j) -> uint64_t {
+        int rg, key0, nk;
+        m.tile(j, rg, key0, nk);
+        if (!row_ok) return 0ull;
+        if (rg == 2) return span_bits(tt - p.window + 1 - key0, min(nk, tt - key0 + 1));
+        const int sink_end = min(p.sink, tt - p.window + 1);
+        return span_bits(-key0, min(nk, sink_end - key0)) |
+               span_bits(p.sink + lo_t - key0, min(nk, p.sink + hi_t - key0));
+      };
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = 0; j < m.total; ++j) {
         const int g = g0 + j;
+        uint32_t b0, b1;
+        {
+          const uint64_t bits = tile_bits(j);
+          b0 = (uint32_t)bits;
+          b1 = (uint32_t)(bits >> 32);
+        }
+        asm volatile("" : "+r"(b0), "+r"(b1));     // computed before the wait below
         ok = mbar_wait(bar(B_SF + x), g & 1, abort_flag, p.err, 221);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;     // tcgen05.ld is warp-collective
         tc_fence_after();
@@ -550,28 +639,10 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_ld32(lane_addr + colS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(lane_addr + colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        // S_x of this item's last tile has run, so Q_x is no longer read: load the next item's Q
-        if (j == m.total - 1 && has_next && !(ok = copy_q(it + 1))) break;
-        int rg, key0, nk;
-        m.tile(j, rg, key0, nk);
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        // attended-set predicate as a bit set over the tile's columns: the window
-        // band is one interval; a slot tile holds the visible sinks and the
-        // retained slots [lo_t, hi_t), two intervals
-        uint64_t bits = 0ull;
-        if (row_ok) {
-          if (rg == 2) {
-            bits = span_bits(tt - p.window + 1 - key0, min(nk, tt - key0 + 1));
-          } else {
-            const int sink_end = min(p.sink, tt - p.window + 1);
-            bits = span_bits(-key0, min(nk, sink_end - key0)) |
-                   span_bits(p.sink + lo_t - key0, min(nk, p.sink + hi_t - key0));
-          }
-        }
-        if (bits != ~0ull) {
-          const uint32_t b0 = (uint32_t)bits, b1 = (uint32_t)(bits >> 32);
+        if ((b0 & b1) != ~0u) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             if (!((b0 >> c) & 1u)) s[c] = -INFINITY;
@@ -615,8 +686,12 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
           float2 z = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), sc2, nm2);
-          z.x = ex2(z.x);
-          z.y = ex2(z.y);
+          if (kPolyEvery > 0 && c2 % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+            z = exp2_poly2(z);
+          } else {
+            z.x = ex2(z.x);
+            z.y = ex2(z.y);
+          }
           acc2[c2 & 3] = __fadd2_rn(acc2[c2 & 3], z);
           __nv_bfloat162 v2 = __floats2bfloat162_rn(z.x, z.y);
           pk[c2] = *reinterpret_cast<uint32_t*>(&v2);
@@ -628,6 +703,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PF + x));
+        // S_x of this item's last tile has run, so Q_x is no longer read: load the
+        // next item's Q (overlapping this tile's PV, which reads only P and V)
+        if (j == m.total - 1 && has_next && !(ok = copy_q(it + 1))) break;
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 rows staged in this tile's region of the Q
