@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import lte_inputs as LI  # noqa: E402
+from learnable_kv_token_b200 import dist as DI  # noqa: E402
 
 METRIC = "LTE sparse-attn prefill & decode tokens/s at 1 B200; % tensor/HBM roofline"
 
@@ -212,7 +213,7 @@ def run_reference(args, rank, world):
 def prefill_bench(args, rank, world, device):
     from learnable_kv_token_b200 import layer, lte as L
     wl = LI.WORKLOADS["prefill"]
-    inp = LI.lte_inputs(wl.with_(seed=wl.seed + 1000 * rank), T=wl.T)
+    inp = LI.lte_inputs(wl.with_(seed=DI.shard_seed(wl.seed, rank)), T=wl.T)
     q, k, v, mask = inp["q"], inp["k"], inp["v"], inp["mask"]
     B, T, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
     pairs = attended_pairs(mask.numpy(), wl.sink, wl.window, wl.cap)
@@ -240,7 +241,7 @@ def prefill_bench(args, rank, world, device):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
+    DI.barrier(world)
     torch.cuda.synchronize()
     with Clocks(gpu_id(device)) as clk:
         t_start.record(stream)
@@ -248,11 +249,11 @@ def prefill_bench(args, rank, world, device):
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize()
-    barrier(world)
+    DI.barrier(world)
     ms_total = t_start.elapsed_time(t_end)
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    ms_total = max_over_ranks(ms_total, world, device)
-    attn_ms = max_over_ranks(attn_ms, world, device)
+    ms_total = DI.max_over_ranks(ms_total, world, device)
+    attn_ms = DI.max_over_ranks(attn_ms, world, device)
     ms_step = ms_total / args.steps
     assert L.lte_read_device_error(bufs.ws) == (0, 0)
 
@@ -269,14 +270,14 @@ def prefill_bench(args, rank, world, device):
 
     e2e_step()
     torch.cuda.synchronize()
-    barrier(world)
+    DI.barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(n_e2e):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, device)
+    e2e_ms = DI.max_over_ranks(e0.elapsed_time(e1) / n_e2e, world, device)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hm))
     d2h = ho.numel() * ho.element_size()
 
@@ -291,7 +292,7 @@ def prefill_bench(args, rank, world, device):
 def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
     from learnable_kv_token_b200 import layer
     wl = LI.WORKLOADS["decode"]
-    inp = LI.lte_inputs(wl.with_(seed=wl.seed + 1000 * rank))
+    inp = LI.lte_inputs(wl.with_(seed=DI.shard_seed(wl.seed, rank)))
     q, k, v, cnn = inp["q"], inp["k"], inp["v"], inp["cnn"]
     B, T0, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
     p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=wl.cap, tau=wl.tau)
@@ -333,7 +334,7 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
     ret = decs[0].cache.ret_total.clone()
     t_meta = int(decs[0].cache.meta[0])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
+    DI.barrier(world)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -341,7 +342,7 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
         e1.record(stream)
     torch.cuda.synchronize()
     n_steps = steps_per_layer * n_layers
-    ms_step = max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
+    ms_step = DI.max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
     del graph
     # algorithmic bytes of one layer step (steady state)
     n_keys = (min(wl.window, t_meta) + wl.sink + torch.clamp(ret, max=wl.cap)).sum().item()
@@ -352,20 +353,7 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
                   + units * row * 2                   # new token write + leaving-token move
                   + units * row * (wl.score_batch + 6) / wl.score_batch)   # deferred scoring reads
     return {"ms_step": ms_step, "bytes": bytes_step, "n_keys": n_keys, "B": B,
-            "prefill_with_cnn_ms": prefill_cnn_ms, "launches": 3 * n_steps}
-
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-
-
-def max_over_ranks(x, world, device):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+            "prefill_with_cnn_ms": prefill_cnn_ms, "launches": 2 * n_steps}
 
 
 def main():
@@ -379,9 +367,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = DI.env_ranks()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -389,10 +375,7 @@ def main():
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+    DI.init(world, "nccl", device, timeout_s=120)
     from learnable_kv_token_b200 import build as _b  # noqa: F401  (library is prebuilt in-tree)
 
     pk = peaks()
@@ -400,8 +383,7 @@ def main():
     dec = None if args.no_decode else decode_bench(args, rank, world, device)
 
     if rank == 0:
-        tokens = pf["B"] * pf["T"] * world
-        value = tokens / (pf["ms_step"] / 1e3)
+        value = DI.job_throughput(pf["B"] * pf["T"], world, pf["ms_step"] / 1e3)
         attn_tflops = pf["flops"] / (pf["attn_ms"] / 1e3) / 1e12
         traffic = traffic_from_profiles("learnable_kv_token_b200/csrc/attn_prefill_tc.cu",
                                         pf["units"])
@@ -424,7 +406,8 @@ def main():
                          "kernel_ms": pf["attn_ms"],
                          "sparsity_vs_full_causal": pf["pairs"] / pf["full_causal_pairs"]},
             "clocks": pf["clocks"],
-            "e2e": {"value": pf["B"] * pf["T"] * world / (pf["e2e_ms"] / 1e3), "unit": "tokens/s",
+            "e2e": {"value": DI.job_throughput(pf["B"] * pf["T"], world, pf["e2e_ms"] / 1e3),
+                    "unit": "tokens/s",
                     "h2d_bytes_per_step": pf["h2d"], "d2h_bytes_per_step": pf["d2h"]},
             "gpu_launches": pf["launches"] + (dec["launches"] if dec else 0),
         }
@@ -434,9 +417,9 @@ def main():
                 "workload": "decode B=32, 4096-token prompt, Hq=16 Hkv=4 D=128 bf16 s=4 w=512 "
                             "C=512, CNN scored live (tau 0.5, deferred batch 64); per-layer steps "
                             "over 4 layer caches (> L2) in one CUDA graph",
-                "value": dec["B"] * world / (dec["ms_step"] / 1e3), "unit": "tokens/s",
+                "value": DI.job_throughput(dec["B"], world, dec["ms_step"] / 1e3), "unit": "tokens/s",
                 "us_per_layer_step": 1e3 * dec["ms_step"],
-                "roofline": {"bound": "hbm", "scope": "whole decode step (3 kernels)",
+                "roofline": {"bound": "hbm", "scope": "whole decode step (2 kernels)",
                              "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"]},
                 "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
@@ -447,8 +430,7 @@ def main():
             line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": 1,
                                     "kind": "oracle", "sample": desc}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    DI.shutdown(world)
 
 
 if __name__ == "__main__":

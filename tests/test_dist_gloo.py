@@ -1,0 +1,116 @@
+"""Multi-rank host path of the data-parallel bench, as world-size-2 gloo ranks
+on the CPU (spawned processes, rendezvous on 127.0.0.1).
+
+Checked: the job time is the max over ranks and the job throughput the
+weak-scaling aggregate; every rank draws its own reproducible sequences; a
+rank that dies before the barrier makes the survivor fail within the
+process-group timeout instead of waiting for ever."""
+import hashlib
+import multiprocessing as mp
+import os
+import socket
+
+import pytest
+
+WORLD = 2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _env(rank, port):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(WORLD), LOCAL_RANK=str(rank))
+
+
+def _digest(t):
+    return hashlib.sha256(t.contiguous().view(-1).view(dtype=__import__("torch").uint8)
+                          .numpy().tobytes()).hexdigest()[:16]
+
+
+def _tiny_inputs(rank):
+    import lte_inputs as LI
+    from learnable_kv_token_b200 import dist as DI
+    wl = LI.WORKLOADS["tiny"]
+    inp = LI.lte_inputs(wl.with_(seed=DI.shard_seed(wl.seed, rank)), T=wl.T)
+    extra = inp["mask"] if "mask" in inp else inp["cnn"][0]
+    return _digest(inp["q"]) + _digest(inp["k"]) + _digest(extra)
+
+
+def _rank_main(rank, port, q):
+    try:
+        _env(rank, port)
+        import torch.distributed as tdist
+        from learnable_kv_token_b200 import dist as DI
+        r, w, _ = DI.env_ranks()
+        DI.init(w, "gloo", timeout_s=30)
+        t_ms = 10.0 + 5.0 * r                      # the slower rank defines the job time
+        job_ms = DI.max_over_ranks(t_ms, w)
+        DI.barrier(w)
+        thr = DI.job_throughput(1000.0, w, job_ms / 1e3)
+        digests = [None] * w
+        tdist.all_gather_object(digests, _tiny_inputs(r))
+        DI.shutdown(w)
+        q.put((rank, "ok", job_ms, thr, digests))
+    except Exception as e:  # reported to the parent
+        q.put((rank, "error", repr(e), None, None))
+
+
+def _dying_rank_main(rank, port, q):
+    try:
+        _env(rank, port)
+        from learnable_kv_token_b200 import dist as DI
+        DI.init(WORLD, "gloo", timeout_s=5)
+        if rank == 1:
+            q.put((rank, "exited", None))
+            q.close()
+            q.join_thread()                        # the message is out before the hard exit
+            os._exit(0)                            # leaves without joining the barrier
+        try:
+            DI.barrier(WORLD)
+            q.put((rank, "no-error", None))
+        except Exception as e:
+            q.put((rank, "error", type(e).__name__))
+    except Exception as e:
+        q.put((rank, "setup-error", repr(e)))
+
+
+def _run(target, timeout):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=target, args=(r, port, q)) for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    out = []
+    try:
+        for _ in range(WORLD):
+            out.append(q.get(timeout=timeout))
+    finally:
+        for p in procs:
+            p.join(timeout=10)
+            if p.is_alive():
+                p.kill()                           # our own child, by its handle
+                p.join()
+    return sorted(out, key=lambda t: t[0])
+
+
+def test_job_time_throughput_and_shards():
+    res = _run(_rank_main, timeout=120)
+    for rank, status, *rest in res:
+        assert status == "ok", (rank, rest)
+    (_, _, job0, thr0, dig0), (_, _, job1, thr1, dig1) = res
+    assert job0 == job1 == 15.0                    # max over ranks, seen alike by both
+    assert thr0 == thr1 == pytest.approx(1000.0 * WORLD / 0.015)
+    assert dig0 == dig1 and dig0[0] != dig0[1]     # each rank its own sequences
+    assert dig0 == [_tiny_inputs(0), _tiny_inputs(1)]   # reproducible from the rank alone
+
+
+def test_dead_rank_fails_the_barrier_instead_of_hanging():
+    res = _run(_dying_rank_main, timeout=90)
+    status = {r: s for r, s, _ in res}
+    assert status[1] == "exited"
+    assert status[0] == "error", res
