@@ -213,6 +213,8 @@ def run_reference(args, rank, world):
 def prefill_bench(args, rank, world, device):
     from learnable_kv_token_b200 import layer, lte as L
     wl = LI.WORKLOADS["prefill"]
+    if args.batch:                                  # smaller case for profiler captures
+        wl = wl.with_(B=args.batch)
     inp = LI.lte_inputs(wl.with_(seed=DI.shard_seed(wl.seed, rank)), T=wl.T)
     q, k, v, mask = inp["q"], inp["k"], inp["v"], inp["mask"]
     B, T, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
@@ -363,7 +365,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="lte", choices=["lte", "reference"])
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle CPU sample length (0 skips the cpu_baseline leg)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="prefill batch override for profiler captures (default: the workload's)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -392,11 +397,12 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pf["ms_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "prefill B=32 T=4096 Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512 "
+            "config": {"workload": f"prefill B={pf['B']} T=4096 Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512 "
                                    "mask~Bern(0.1) fed; step = evict_compact + sparse_attn_prefill",
                        "global_batch": pf["B"] * world, "seq_len": pf["T"],
                        "parallelism": f"dp{world} (independent sequences per GPU)",
-                       "l2": "inputs larger than L2 (q 512 MiB, k/v 128 MiB each)"},
+                       "l2": f"inputs larger than L2 (q {pf['B'] * pf['T'] * 16 * 128 * 2 >> 20} MiB, "
+                             f"k/v {pf['B'] * pf['T'] * 4 * 128 * 2 >> 20} MiB each)"},
             "roofline": {"kernel": "attn_prefill_tc_kernel", "bound": "tensor",
                          "achieved": attn_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": attn_tflops / pk["bf16_tflops"],
@@ -424,7 +430,7 @@ def main():
                              "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"]},
                 "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
             }
-        if world == 1:
+        if world == 1 and args.cpu_seconds > 0:
             tok, sec, desc = oracle_sample(LI.WORKLOADS["prefill"], args.cpu_seconds,
                                            2.5 * args.cpu_seconds)
             line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": 1,
