@@ -50,6 +50,7 @@ constexpr int kDecMaxParts = 8;          // CTAs sharing one unit
 
 struct DecGeom {
   int n_ctas, per_cta, max_parts;
+  bool single;             // one whole unit per CTA: no partials, no merge
 };
 
 static int sm_count() {
@@ -63,10 +64,21 @@ static DecGeom dec_geom(const lte_dims* d) {
   const long long W = (long long)d->B * d->Hkv * L;
   const long long want = (W + kDecChunk - 1) / kDecChunk;
   DecGeom g;
+  const long long units = (long long)d->B * d->Hkv;
+  if (units <= sm_count()) {
+    // the units fit one wave: a CTA streams one whole unit and writes its
+    // output itself (no split of a unit, hence no partials to merge)
+    g.n_ctas = (int)units;
+    g.per_cta = (int)L;
+    g.max_parts = 1;
+    g.single = true;
+    return g;
+  }
   g.n_ctas = (int)(want < sm_count() ? want : sm_count());
   if (g.n_ctas < 1) g.n_ctas = 1;
   g.per_cta = (int)((W + g.n_ctas - 1) / g.n_ctas);
   g.max_parts = (int)((L + g.per_cta - 1) / g.per_cta) + 1;
+  g.single = false;
   return g;
 }
 
@@ -217,7 +229,7 @@ __device__ __forceinline__ uint32_t pack_bf16d(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 struct AttnParams {
-  int Hq, Hkv, G, window, sink, cap, L, n_units, per_cta, max_parts;
+  int Hq, Hkv, G, window, sink, cap, L, n_units, per_cta, max_parts, single;
   float scale_log2;
   const int32_t* ret_total;
   int32_t* meta;
@@ -281,6 +293,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   uint64_t* full = reinterpret_cast<uint64_t*>(ents + kDecMaxEntries);   // stage barriers
   int* n_ents = reinterpret_cast<int*>(full + kDecStages);
   int* is_last = n_ents + 1;
+  int* t_sh = n_ents + 2;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((smem_u32d(dsm) & 1023u) != 0) {          // swizzle atoms need 1 KiB alignment
@@ -293,44 +306,28 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(full + st)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // meta[0] is not written by the preceding update kernel (only by the last
-  // attention CTA of the previous step, which finished before that kernel began)
-  const int t = p.meta[0];
+  // meta[0] is not written by the preceding update kernel (only by the
+  // attention grid of the previous step, which finished before that kernel
+  // began).  Thread 0 reads it once for the CTA, then takes a ticket: the
+  // CTA holding the last ticket advances meta at its end, when every CTA has
+  // read the step index.
+  int t = 0, ticket = 0;
+  if (tid == 0) t = p.meta[0];
   pdl_wait();              // the cache update and scoring of this step are visible
+  if (tid == 0)
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(ticket)
+                 : "l"(p.counters + p.n_units)
+                 : "memory");
+  if (tid == 0) *t_sh = t;
+  __syncthreads();
+  t = *t_sh;
   const int nw = min(p.window, t + 1);
   int ns = t - p.window + 1;
   ns = ns < 0 ? 0 : (ns > p.sink ? p.sink : ns);
   const long long W = (long long)p.n_units * p.L;
   const long long lo = (long long)blockIdx.x * p.per_cta;
   const long long hi = lo + p.per_cta < W ? lo + p.per_cta : W;
-
-  // ---- chunk list: (unit, first slot, keys, last-of-unit) over the valid slots of [lo, hi)
-  if (tid == 0) {
-    int n = 0;
-    const int u_lo = (int)(lo / p.L), u_hi = (int)((hi - 1) / p.L);
-    int rt[4];                                   // loads issued together, used below
-#pragma unroll
-    for (int k = 0; k < 4; ++k) rt[k] = (u_lo + k <= u_hi) ? p.ret_total[u_lo + k] : 0;
-    for (int u = u_lo; u <= u_hi; ++u) {
-      const int a = (int)((lo > (long long)u * p.L ? lo : (long long)u * p.L) - (long long)u * p.L);
-      const long long ue = (long long)(u + 1) * p.L;
-      const int bnd = (int)((hi < ue ? hi : ue) - (long long)u * p.L);
-      const int nr = min(p.cap, u - u_lo < 4 ? rt[u - u_lo] : p.ret_total[u]);
-      const int rs[3] = {0, p.window, p.window + p.sink};
-      const int re[3] = {nw, p.window + ns, p.window + p.sink + nr};
-      const int first = n;
-      for (int r = 0; r < 3; ++r) {
-        const int x = max(a, rs[r]), y = min(bnd, re[r]);
-        for (int s = x; s < y && n < kDecMaxEntries; s += kDecChunk)
-          ents[n++] = make_int4(u, s, min(kDecChunk, y - s), 0);
-      }
-      if (n == first && n < kDecMaxEntries) ents[n++] = make_int4(u, 0, 0, 0);   // flush only
-      if (n > 0) ents[n - 1].w = 1;
-    }
-    *n_ents = n;
-  }
-  __syncthreads();
-  const int n_ch = *n_ents;
 
   // one elected thread issues the TMA copies of chunk i into stage i % kDecStages
   // (flush-only entries still load rows so that every stage use completes a phase)
@@ -350,6 +347,41 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
   };
 
+  // ---- chunk list: (unit, first slot, keys, last-of-unit) over the valid slots of [lo, hi).
+  // The window chunks of the first unit need no retained count: their copies
+  // start while the count loads.
+  int issued = 0;
+  if (tid == 0) {
+    int n = 0;
+    const int u_lo = (int)(lo / p.L), u_hi = (int)((hi - 1) / p.L);
+    int rt[4];                                   // loads issued together, used below
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rt[k] = (u_lo + k <= u_hi) ? p.ret_total[u_lo + k] : 0;
+    for (int u = u_lo; u <= u_hi; ++u) {
+      const int a = (int)((lo > (long long)u * p.L ? lo : (long long)u * p.L) - (long long)u * p.L);
+      const long long ue = (long long)(u + 1) * p.L;
+      const int bnd = (int)((hi < ue ? hi : ue) - (long long)u * p.L);
+      const int rs[3] = {0, p.window, p.window + p.sink};
+      const int first = n;
+      for (int r = 0; r < 3; ++r) {
+        const int re = r == 0 ? nw
+                     : r == 1 ? p.window + ns
+                              : p.window + p.sink +
+                                    min(p.cap, u - u_lo < 4 ? rt[u - u_lo] : p.ret_total[u]);
+        const int x = max(a, rs[r]), y = min(bnd, re);
+        for (int s = x; s < y && n < kDecMaxEntries; s += kDecChunk)
+          ents[n++] = make_int4(u, s, min(kDecChunk, y - s), 0);
+        if (u == u_lo && r == 0)
+          for (; issued < kDecStages - 1 && issued < n; ++issued) load(issued);
+      }
+      if (n == first && n < kDecMaxEntries) ents[n++] = make_int4(u, 0, 0, 0);   // flush only
+      if (n > 0) ents[n - 1].w = 1;
+    }
+    *n_ents = n;
+  }
+  __syncthreads();
+  const int n_ch = *n_ents;
+
   float o_acc[DN][4];
   float m_run[2], l_run[2];
   auto reset = [&]() {
@@ -362,7 +394,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   };
   reset();
 
-  int issued = 0;
   if (tid == 0)
     for (; issued < kDecStages - 1 && issued < n_ch; ++issued) load(issued);
   int i = 0;
@@ -465,6 +496,35 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       }
       __syncthreads();
       const int u = e.x;
+      if (p.single) {
+        // the CTA holds the whole unit: combine its warps and write o_t, lse_t
+        const int b = u / p.Hkv, h = u % p.Hkv;
+        for (int i2 = tid; i2 < p.G * (D / 4); i2 += kDecThreads) {
+          const int g = i2 / (D / 4), d4 = (i2 % (D / 4)) * 4;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, m_sh[w * 16 + g]);
+          float l = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < kDecWarps; ++w) {
+            const float mw = m_sh[w * 16 + g];
+            const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            l += l_sh[w * 16 + g] * f;
+            const float4 ow = *reinterpret_cast<const float4*>(o_sh + (w * 16 + g) * D + d4);
+            acc.x += ow.x * f; acc.y += ow.y * f; acc.z += ow.z * f; acc.w += ow.w * f;
+          }
+          const float inv = 1.f / l;
+          __nv_bfloat16* orow = p.o_t + ((long long)b * p.Hq + h * p.G + g) * D + d4;
+          *reinterpret_cast<uint2*>(orow) =
+              make_uint2(pack_bf16d(acc.x * inv, acc.y * inv), pack_bf16d(acc.z * inv, acc.w * inv));
+          if (d4 == 0 && p.lse_t != nullptr)
+            p.lse_t[(long long)b * p.Hq + h * p.G + g] = (M + log2f(l)) * 0.69314718055994531f;
+        }
+        reset();
+        __syncthreads();   // stage i % kDecStages and the merge buffers are free again
+        continue;
+      }
       const int c_first = (int)(((long long)u * p.L) / p.per_cta);
       const int c_last = (int)(((long long)u * p.L + p.L - 1) / p.per_cta);
       const int n_parts = c_last - c_first + 1;
@@ -530,14 +590,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           if (d4 == 0 && p.lse_t != nullptr)
             p.lse_t[(long long)b * p.Hq + h * p.G + g] = (M + log2f(l)) * 0.69314718055994531f;
         }
-        __syncthreads();
-        if (tid == 0) {
-          __threadfence();
-          if (atomicAdd(&p.counters[p.n_units], 1) == p.n_units - 1) {
-            p.meta[0] = t + 1;
-            p.meta[1] = p.meta[2];
-          }
-        }
       }
       reset();
     }
@@ -546,6 +598,11 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   // copies issued but not consumed (only after a wait ran out) land before exit
   if (tid == 0)
     for (int j = i; j < issued; ++j) mbar_wait_d(smem_u32d(full + j % kDecStages), (j / kDecStages) & 1);
+  // every CTA has read the step index before taking its ticket: the last one advances it
+  if (tid == 0 && ticket == (int)gridDim.x - 1) {
+    p.meta[0] = t + 1;
+    p.meta[1] = p.meta[2];
+  }
 }
 
 // launch with programmatic stream serialization (see pdl_wait)
@@ -633,7 +690,7 @@ static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void
   AttnParams p{};
   p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = d->Hq / d->Hkv; p.window = d->window; p.sink = d->sink;
   p.cap = d->cap; p.L = d->window + d->sink + d->cap; p.n_units = d->B * d->Hkv;
-  p.per_cta = g.per_cta; p.max_parts = g.max_parts;
+  p.per_cta = g.per_cta; p.max_parts = g.max_parts; p.single = g.single ? 1 : 0;
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.ret_total = c->ret_total; p.meta = c->meta;
   p.o_t = (__nv_bfloat16*)o_t; p.lse_t = lse_t; p.part = part; p.counters = counters; p.err = err;

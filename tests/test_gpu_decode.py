@@ -87,6 +87,31 @@ def test_decode_vs_oracle_simulation(layer, cfg):
                 assert rs[b][h] == ret_ref[t - T0], (b, h, t)
 
 
+def test_decode_split_kv_path(layer):
+    """More (batch, KV head) units than SMs: units are split across CTAs and
+    the last CTA of each unit merges the partials.  Sampled units vs the oracle."""
+    B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = 40, 8, 4, 64, 2, 32, 16, 60, 30, 8
+    assert B * Hkv > torch.cuda.get_device_properties(0).multi_processor_count
+    T = T0 + steps
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 91, w_std=0.1)
+    G = Hq // Hkv
+    units = [(0, 0), (7, 3), (19, 1), (26, 2), (39, 3)]
+    r_or = {(b, h): O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h))
+            for b in range(B) for h in range(Hkv)}
+    tau, margin = clean_tau(np.stack(list(r_or.values())))
+    assert margin > 1e-5
+    o_g, lse_g, rets, _, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, Ds,
+                                         check_every=11)
+    for b, h in units:
+        o_ref, lse_ref, sets, ret_ref, _ = O.decode_unit(
+            f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]), f64(v[b, :, h]), T0, sink,
+            window, cap, tau, oracle_cnn(cnn, h), Ds, scale_of(D))
+        assert_attention_close(f64(o_g[:, b, h * G:(h + 1) * G]), f64(lse_g[:, b, h * G:(h + 1) * G]),
+                               o_ref, lse_ref, torch.bfloat16, f"unit {b},{h}")
+        for t, rs in rets.items():
+            assert rs[b][h] == ret_ref[t - T0], (b, h, t)
+
+
 def test_decode_score_batch_invariance(layer):
     """Deferred-scoring batch sizes give bit-identical outputs and caches."""
     B, Hq, Hkv, D, sink, window, cap, T0, steps = 1, 8, 2, 128, 4, 80, 24, 150, 100
