@@ -29,7 +29,7 @@
 //              PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  The tensor pipe runs in
 //              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
 //              P_x may then be overwritten and O_x rescaled without a wait;
-//   warps 2-3  idle (they complete warpgroup 0, whose registers go to softmax)
+//   warps 2-3  output stores of tiles A and B (TMA stores of the staged rows)
 //   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per row
 //              reads its S row from TMEM, applies the attended-set predicate
 //              (a 64-bit set of at most two column intervals), exp2 via
@@ -58,7 +58,7 @@ constexpr int BN = 64;              // keys per K/V tile
 constexpr int HD = 128;             // head dim
 constexpr int kThreads = 384;
 // register split (setmaxnreg): the launch gives 168 per thread (3 warps per
-// sub-partition); warpgroup 0 (TMA, MMA, two idle warps) drops to 64 and the
+// sub-partition); warpgroup 0 (TMA, MMA, two store warps) drops to 64 and the
 // two softmax warpgroups rise to 216: 4 * 64 + 8 * 216 <= 12 * 168
 constexpr int kRegsLaunch = 168, kRegsIssue = 64, kRegsSoftmax = 216;
 static_assert(4 * kRegsIssue + 8 * kRegsSoftmax <= 12 * kRegsLaunch, "register split fits the launch");
@@ -556,6 +556,32 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
       __syncwarp();
       mbar_drain(bar(B_FIN), 0);
+    } else {
+      // ============================================================ output stores
+      // warp 2 stores tile A, warp 3 tile B: once all 128 rows of the tile are
+      // staged in its region of the Q buffer, one TMA store per 64-column half
+      // (rows past T are clipped by the copy); the region is released for the
+      // next Q load when the store has read it.  Keeping this wait off the
+      // softmax warps keeps their next tile on time.
+      const int x = warp - 2;
+      int it = 0;
+      for (int i = blockIdx.x; i < p.n_items; i += gridDim.x, ++it) {
+        int u, t0, t_last;
+        item_tokens(p, i, u, t0, t_last);
+        if (!wwait(bar(B_STG + x), it & 1, abort_flag, p.err, 225)) break;
+        if (elect_one()) {
+          const uint32_t src = sbase + kOffQ + x * kQTile;
+          const int b = u / p.Hkv, h = u % p.Hkv;
+          tma_store_4d(&tm_o, src, 0, h * p.G, t0 + x * p.TOK, b);
+          tma_store_4d(&tm_o, src + kQHalf, 64, h * p.G, t0 + x * p.TOK, b);
+          bulk_commit();
+          bulk_wait_read();                          // staging rows read: the buffer may be reloaded
+          mbar_arrive(bar(B_OST + x));
+        }
+        __syncwarp();
+      }
+      if (elect_one()) bulk_wait_all();            // output stores complete before exit
+      __syncwarp();
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
@@ -718,13 +744,14 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const float inv = __frcp_rn(l_sum);
       uint8_t* srow = smem + kOffQ + x * kQTile + row * 128;
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t orr[32];
-        tmem_ld32(lane_addr + colO + c0, orr);
+      for (int c0 = 0; c0 < HD; c0 += 64) {        // one 64-column half per wait
+        uint32_t orr[64];
+        tmem_ld32(lane_addr + colO + c0, *reinterpret_cast<uint32_t(*)[32]>(&orr[0]));
+        tmem_ld32(lane_addr + colO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&orr[32]));
         tmem_wait_ld();
         uint8_t* half = srow + (c0 >> 6) * kQHalf;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {               // 16-byte chunk (c0 % 64) / 8 + e of the half row
+        for (int e = 0; e < 8; ++e) {               // 16-byte chunk e of the half row
           uint4 v;
           uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
@@ -733,8 +760,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                       __uint_as_float(orr[8 * e + 2 * f + 1]) * inv);
             w[f] = *reinterpret_cast<uint32_t*>(&v2);
           }
-          const int chunk = ((c0 & 63) >> 3) + e;
-          *reinterpret_cast<uint4*>(half + ((chunk ^ (row & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(half + ((e ^ (row & 7)) << 4)) = v;
         }
       }
       tc_fence_before();
@@ -743,19 +769,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
             (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       fence_proxy_async();
-      mbar_arrive(bar(B_STG + x));                  // this row is staged
-      if (row == 0) {
-        if (!mbar_wait(bar(B_STG + x), it & 1, abort_flag, p.err, 225)) break;
-        const uint32_t src = sbase + kOffQ + x * kQTile;
-        tma_store_4d(&tm_o, src, 0, m.h * p.G, m.t0 + x * p.TOK, m.b);
-        tma_store_4d(&tm_o, src + kQHalf, 64, m.h * p.G, m.t0 + x * p.TOK, m.b);
-        bulk_commit();
-        bulk_wait_read();                            // staging rows read: the buffer may be reloaded
-        mbar_arrive(bar(B_OST + x));
-      }
+      mbar_arrive(bar(B_STG + x));                  // this row is staged (warp 2 + x stores it)
       g0 += m.total;
     }
-    if (row == 0) bulk_wait_all();                 // output stores complete before exit
   }
   tc_fence_before();
   __syncthreads();
