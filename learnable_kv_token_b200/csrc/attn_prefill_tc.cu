@@ -278,27 +278,36 @@ __device__ __forceinline__ uint64_t span_bits(int a, int b) {
 // 2^x for a pair of fp32 values on the FMA pipe (the special-function unit
 // evaluates the others).  Range reduction 2^x = 2^n * 2^f with n = round(x),
 // obtained by adding 1.5 * 2^23 (which leaves n in the low mantissa bits),
-// and f = x - n in [-1/2, 1/2]; 2^f by a degree-5 polynomial fitted by least
-// squares on Chebyshev nodes with p(0) = 1 (relative error 1.3e-7, below the
-// bf16 rounding of P by 2^-16; gen_exp2_poly.py prints the fit); 2^n enters
-// as an integer add to the exponent field.  Inputs are clamped to >= -126 so
-// the exponent stays normal: a masked key (x = -inf) gets 2^-126 rather than 0,
-// which no fp32 sum of at least one unit term can register.
+// and f = x - n in [-1/2, 1/2]; 2^f by a degree-3 polynomial, a weighted
+// least-squares fit of the relative error on Chebyshev nodes with p(0) = 1
+// (relative error <= 1.2e-4, mean 4e-5: below the bf16 rounding of P, 2^-9,
+// and, on the fraction of terms it serves, far below the lse tolerance;
+// gen_exp2_poly.py prints the fit); 2^n enters as an integer add to the
+// exponent field.  Inputs are clamped to >= -127: a masked key (x = -inf)
+// then has n = -127, f = 0, p(0) = 1 and an exponent field of 0, so its P is
+// exactly +0 as from the special-function unit (the key rows of a ragged tile
+// past the valid ones may hold any finite value, and 0 * V must stay 0);
+// x in (-127, -126.5) gives a denormal below 2^-126 instead of 2^x.
 constexpr int kPolyEvery = 0;       // > 0: every kPolyEvery-th pair of S columns takes the polynomial
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
   const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
   const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
   const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(make_float2(1.340043265e-03f, 1.340043265e-03f), f,
-                        make_float2(9.672171436e-03f, 9.672171436e-03f));
-  q = __ffma2_rn(q, f, make_float2(5.550327152e-02f, 5.550327152e-02f));
-  q = __ffma2_rn(q, f, make_float2(2.402222753e-01f, 2.402222753e-01f));
-  q = __ffma2_rn(q, f, make_float2(6.931471825e-01f, 6.931471825e-01f));
+  float2 q = __ffma2_rn(make_float2(5.459282547e-02f, 5.459282547e-02f), f,
+                        make_float2(2.422178388e-01f, 2.422178388e-01f));
+  q = __ffma2_rn(q, f, make_float2(6.933686137e-01f, 6.933686137e-01f));
   q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// max of three fp32 values in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // ---------------------------------------------------------------- work items
@@ -677,11 +686,13 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         float m8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int e = 0; e < 8; ++e) {              // columns e, e + 8, ..., e + 56
+          m8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+          m8[e] = fmax3(m8[e], s[24 + e], s[32 + e]);
+          m8[e] = fmax3(m8[e], s[40 + e], s[48 + e]);
+          m8[e] = fmaxf(m8[e], s[56 + e]);
+        }
+        float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         mx *= p.scale_log2;                        // scale > 0: max commutes with it
         const bool need = mx > m_ref + 8.f;        // lazy rescale (x256 headroom)
         float corr = 1.f;
