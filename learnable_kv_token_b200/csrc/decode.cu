@@ -709,6 +709,457 @@ static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void
                     mq, p);
 }
 
+// ---------------------------------------------------------------------------
+// Fused decode step, used when every (batch, KV head) unit gets a CTA of its
+// own (units <= SMs) and the CNN fits the tensor-core scoring tile: one
+// launch per step.  320 threads (the scoring tile's size), per unit:
+//   warp 8     cache update: token t-w leaves slot t mod w (to its sink slot,
+//              into the retained ring, or dropped), token t takes the slot;
+//              the rows are written to global memory, fenced for the async
+//              proxy, and the new retained count is published through an
+//              mbarrier;
+//   warp 9     TMA producer: 64-slot chunks of K and V into a ring of
+//              192 KiB.  The window chunks the update cannot touch go first
+//              (their copies overlap the update); the chunk holding slot
+//              t mod w, the sinks and the retained ring follow once the
+//              update has landed;
+//   warps 0..NS-1  one per ring stage (NS = 6 at D = 128, 8 at D = 64):
+//              chunk c goes to stage and warp c mod NS, so a warp only ever
+//              waits for the next phase of its own stage (a phase parity
+//              cannot alias).  QK^T and PV on m16n8k16 bf16 MMAs with the G
+//              query heads as MMA rows (the query rows are staged once in
+//              shared memory), online softmax per chunk, the stage released
+//              through an mbarrier -- the warps never wait for one another;
+// then the NS (m, l, o) partials are merged in shared memory and o_t,
+// lse_t written; when the deferred batch is due the same CTA scores it
+// (score_tile_tc, the arithmetic of lte_score).  The step counter lives in
+// the cache: every CTA reads meta[0..1], then takes a ticket on meta[3]; the
+// last ticket advances t (and n_scored) and resets the ticket.
+constexpr int kFuUpdWarp = 8, kFuProdWarp = 9;
+constexpr int kFuRingBytes = 192 * 1024;
+// ring stages (= attention warps) for head dim D: at most 192 KiB and 8 warps
+__host__ __device__ constexpr int fu_stages(int D) {
+  return kFuRingBytes / (4 * kDecChunk * D) < 8 ? kFuRingBytes / (4 * kDecChunk * D) : 8;
+}
+
+struct FusedParams {
+  int Hq, Hkv, G, window, sink, cap, L, score_batch, future;
+  float tau, scale_log2;
+  const __nv_bfloat16* q_t;
+  const __nv_bfloat16* k_t;
+  const __nv_bfloat16* v_t;
+  __nv_bfloat16* ck;
+  __nv_bfloat16* cv;
+  int32_t* pos;
+  float* win_r;
+  int32_t* ret_total;
+  int32_t* meta;
+  __nv_bfloat16* o_t;
+  float* lse_t;
+  DevError* err;
+};
+
+// The chunks of one step, in issue order: the window chunks except the one
+// holding slot t mod w (index kw), then chunk kw, then the sink slots, then
+// the retained slots.  nw valid window slots, ns sinks, nr retained (nr is
+// known once the update has run).
+struct FuChunks {
+  int nw, kw, ns, nr, window, sink;
+  __device__ __forceinline__ int nwc() const { return (nw + kDecChunk - 1) / kDecChunk; }
+  __device__ __forceinline__ int early() const { return nwc() - 1; }
+  __device__ __forceinline__ int count() const {
+    return nwc() + (ns + kDecChunk - 1) / kDecChunk + (nr + kDecChunk - 1) / kDecChunk;
+  }
+  __device__ __forceinline__ void get(int c, int& slot0, int& nk) const {
+    const int a = nwc();
+    if (c < a) {
+      const int k = c < a - 1 ? (c < kw ? c : c + 1) : kw;
+      slot0 = k * kDecChunk;
+      nk = min(kDecChunk, nw - slot0);
+      return;
+    }
+    c -= a;
+    const int bs = (ns + kDecChunk - 1) / kDecChunk;
+    if (c < bs) {
+      slot0 = window + c * kDecChunk;
+      nk = min(kDecChunk, ns - c * kDecChunk);
+      return;
+    }
+    c -= bs;
+    slot0 = window + sink + c * kDecChunk;
+    nk = min(kDecChunk, nr - c * kDecChunk);
+  }
+};
+
+// bounded wait that also gives up when the CTA is aborting
+__device__ __forceinline__ bool fu_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                        DevError* err, int where) {
+  if (mbar_try_d(bar, parity)) return true;
+  const unsigned long long t0 = gtime_d();
+  while (true) {
+    if (mbar_try_d(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (gtime_d() - t0 > 1000000000ull) {
+      record_error(err, LTE_ERR_TIMEOUT, where);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const FusedParams p, const ScoreParams sp, const RingKV<__nv_bfloat16> kv) {
+  constexpr int KSTEPS = D / 16, DN = D / 8, HALVES = D / 64;
+  constexpr int kKV = kDecChunk * D * 2;                  // K or V of one chunk
+  constexpr int kStage = 2 * kKV;
+  constexpr int NS = fu_stages(D);                        // stages = attention warps
+  constexpr int kQBytes = 16 * D * 2;                     // the group's query rows (16, zero padded)
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  uint8_t* sq = dsm + kFuRingBytes;                       // 128B-swizzled like the K tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kFuRingBytes + kQBytes);
+  uint64_t* empty = full + NS;
+  uint64_t* upd = empty + NS;
+  int* sh = reinterpret_cast<int*>(upd + 1);   // t, n_scored, retained count, abort, ticket
+  volatile int* abort_flag = sh + 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.x, b = u / p.Hkv, h = u % p.Hkv;
+  if ((smem_u32d(dsm) & 1023u) != 0) {          // swizzle atoms need 1 KiB alignment
+    if (tid == 0) record_error(p.err, LTE_ERR_DEVICE, 130);
+    return;
+  }
+  pdl_launch_next();
+  if (tid == 0) {
+    for (int st = 0; st < NS; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(full + st)));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(empty + st)));
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(upd)));
+    sh[3] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  pdl_wait();              // the previous step has completed: cache and meta are current
+  if (tid == 0) {
+    sh[0] = p.meta[0];
+    sh[1] = p.meta[1];
+    int ticket;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(ticket)
+                 : "l"(p.meta + 3)
+                 : "memory");
+    sh[4] = ticket;
+  }
+  __syncthreads();
+  const int t = sh[0], n_scored = sh[1];
+  const int slot_w = t % p.window, leaving = t - p.window;
+  const long long urow = (long long)u * p.L;
+  FuChunks ch;
+  ch.window = p.window;
+  ch.sink = p.sink;
+  ch.nw = min(p.window, t + 1);
+  ch.kw = slot_w / kDecChunk;
+  {
+    const int ns = t - p.window + 1;
+    ch.ns = ns < 0 ? 0 : (ns > p.sink ? p.sink : ns);
+  }
+  ch.nr = 0;
+  constexpr int kUnknown = 1 << 30;
+  // the attention warps' running (m, l, o) over their chunks
+  float o_acc[DN][4];
+#pragma unroll
+  for (int i = 0; i < DN; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o_acc[i][e] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+  if (warp == kFuUpdWarp) {
+    // ---------------------------------------------------------------- cache update
+    constexpr int NV = D * 2 / 16;               // 16-byte vectors per row
+    const int e = lane & 15;
+    const bool is_v = lane >= 16;
+    const long long wrow = (urow + slot_w) * D;
+    uint4 new4 = make_uint4(0, 0, 0, 0), old4 = make_uint4(0, 0, 0, 0);
+    if (e < NV) {                                // every load before any dependent store
+      new4 = reinterpret_cast<const uint4*>((is_v ? p.v_t : p.k_t) + (long long)u * D)[e];
+      old4 = reinterpret_cast<const uint4*>((is_v ? p.cv : p.ck) + wrow)[e];
+    }
+    int dst = -1, rt = 0;
+    if (lane == 0) {
+      rt = p.ret_total[u];
+      if (leaving >= 0) {
+        const int held = p.pos[urow + slot_w];
+        const float r = p.win_r[(long long)u * p.window + slot_w];
+        if (held != leaving) record_error(p.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
+        else if (leaving < p.sink) dst = p.window + leaving;
+        else if (p.cap > 0 && r >= p.tau) dst = p.window + p.sink + rt % p.cap;
+      }
+    }
+    dst = __shfl_sync(0xffffffffu, dst, 0);
+    if (e < NV) {
+      __nv_bfloat16* base = is_v ? p.cv : p.ck;
+      if (dst >= 0) reinterpret_cast<uint4*>(base + (urow + dst) * D)[e] = old4;
+      reinterpret_cast<uint4*>(base + wrow)[e] = new4;
+    }
+    if (lane == 0) {
+      if (dst >= 0) p.pos[urow + dst] = leaving;
+      const int rt_new = rt + (dst >= p.window + p.sink ? 1 : 0);
+      if (rt_new != rt) p.ret_total[u] = rt_new;
+      p.pos[urow + slot_w] = t;
+      p.win_r[(long long)u * p.window + slot_w] = NAN;
+      sh[2] = rt_new;
+    }
+    fence_proxy_async_global();                  // the rows are read next by TMA copies
+    __syncwarp();
+    if (lane == 0)
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32d(upd)) : "memory");
+  } else if (warp == kFuProdWarp) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int n_ch = kUnknown, c = 0;
+      const int E = ch.early();
+      for (;; ++c) {
+        if (c >= E && n_ch == kUnknown) {
+          if (!fu_wait(smem_u32d(upd), 0, abort_flag, p.err, 133)) break;
+          fence_proxy_async_global();
+          ch.nr = min(p.cap, sh[2]);
+          n_ch = ch.count();
+        }
+        if (c >= n_ch) break;
+        const int st = c % NS;
+        if (c >= NS && !fu_wait(smem_u32d(empty + st), ((c / NS) - 1) & 1, abort_flag, p.err, 134))
+          break;
+        int slot0, nk;
+        ch.get(c, slot0, nk);
+        const uint32_t dst = smem_u32d(dsm + st * kStage), bar = smem_u32d(full + st);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kStage)
+                     : "memory");
+        const int row = (int)(urow + slot0);
+#pragma unroll
+        for (int hf = 0; hf < HALVES; ++hf) {
+          tma_2d(dst + hf * kDecChunk * 128, &tm_k, bar, hf * 64, row);
+          tma_2d(dst + kKV + hf * kDecChunk * 128, &tm_v, bar, hf * 64, row);
+        }
+      }
+      // the copies issued last have landed before shared memory is reused
+      for (int j = c - NS > 0 ? c - NS : 0; j < c; ++j)
+        mbar_wait_d(smem_u32d(full + j % NS), (j / NS) & 1);
+    }
+  } else if (warp < NS) {
+    // ---------------------------------------------------------------- attention
+    {
+      // the group's query rows (the MMA A operand; rows >= G are zero), staged once
+      const __nv_bfloat16* q0 = p.q_t + ((long long)b * p.Hq + h * p.G) * D;
+      for (int i = tid; i < 16 * (D / 8); i += 32 * NS) {
+        const int r = i / (D / 8), cc = i % (D / 8);
+        const uint4 v = r < p.G ? *reinterpret_cast<const uint4*>(q0 + (long long)r * D + cc * 8)
+                                : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sq + sw128(16, r, cc)) = v;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NS) : "memory");   // attention warps only
+    }
+    int n_ch = kUnknown;
+    const int E = ch.early();
+#pragma unroll 1
+    for (int c = warp;; c += NS) {
+      if (c >= E && n_ch == kUnknown) {
+        if (!__all_sync(0xffffffffu, fu_wait(smem_u32d(upd), 0, abort_flag, p.err, 132))) break;
+        ch.nr = min(p.cap, sh[2]);
+        n_ch = ch.count();
+      }
+      if (c >= n_ch) break;
+      const int st = c % NS;
+      if (!__all_sync(0xffffffffu,
+                      fu_wait(smem_u32d(full + st), (c / NS) & 1, abort_flag, p.err, 131)))
+        break;
+      int slot0, nk;
+      ch.get(c, slot0, nk);
+      const uint8_t* sk = dsm + st * kStage;
+      float s[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[i][e] = 0.f;
+#pragma unroll
+      for (int kst = 0; kst < KSTEPS; ++kst) {
+        uint32_t qf[4];
+        ldsm_x4d(smem_u32d(sq + sw128(16, lane & 15, kst * 2 + (lane >> 4))), qf[0], qf[1], qf[2],
+                 qf[3], false);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {         // 16 keys per pair of n8 tiles
+          const int r = np * 16 + ((lane >> 4) << 3) + (lane & 7);
+          const int cc = kst * 2 + ((lane >> 3) & 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4d(smem_u32d(sk + sw128(kDecChunk, r, cc)), b0, b1, b2, b3, false);
+          mma_bf16d(s[2 * np], qf, b0, b1);
+          mma_bf16d(s[2 * np + 1], qf, b2, b3);
+        }
+      }
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int key = nt * 8 + ((lane & 3) << 1) + (q & 1);
+          s[nt][q] = key < nk ? s[nt][q] * p.scale_log2 : -INFINITY;
+          mx[q >> 1] = fmaxf(mx[q >> 1], s[nt][q]);
+        }
+      float corr[2], mu[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+        const float m_new = fmaxf(m_run[hr], mx[hr]);
+        mu[hr] = m_new == -INFINITY ? 0.f : m_new;
+        corr[hr] = m_run[hr] == -INFINITY ? 0.f : exp2f(m_run[hr] - mu[hr]);
+        m_run[hr] = m_new;
+        l_run[hr] *= corr[hr];
+      }
+#pragma unroll
+      for (int i = 0; i < DN; ++i) {
+        o_acc[i][0] *= corr[0]; o_acc[i][1] *= corr[0];
+        o_acc[i][2] *= corr[1]; o_acc[i][3] *= corr[1];
+      }
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t pf[4];
+        {
+          float pv[2][4];
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              pv[x][q] = exp2f(s[2 * np + x][q] - mu[q >> 1]);
+              l_run[q >> 1] += pv[x][q];
+            }
+          pf[0] = pack_bf16d(pv[0][0], pv[0][1]);
+          pf[1] = pack_bf16d(pv[0][2], pv[0][3]);
+          pf[2] = pack_bf16d(pv[1][0], pv[1][1]);
+          pf[3] = pack_bf16d(pv[1][2], pv[1][3]);
+        }
+#pragma unroll
+        for (int dp = 0; dp < DN / 2; ++dp) {
+          const int r = np * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
+          const int cc = dp * 2 + (lane >> 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4d(smem_u32d(sk + kKV + sw128(kDecChunk, r, cc)), b0, b1, b2, b3, true);
+          mma_bf16d(o_acc[2 * dp], pf, b0, b1);
+          mma_bf16d(o_acc[2 * dp + 1], pf, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32d(empty + st))
+                     : "memory");
+    }
+    // finish this warp's row sums (the quad of lanes shares a row)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 1);
+      l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 2);
+    }
+  }
+  __syncthreads();         // every chunk is consumed and every copy has landed
+  if (warp < NS) {
+    float* o_sh = reinterpret_cast<float*>(dsm);                 // [warps][16][D]
+    float* m_sh = o_sh + NS * 16 * D;                  // [warps][16]
+    float* l_sh = m_sh + NS * 16;                      // [warps][16]
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = (lane >> 2) + hr * 8;
+      if ((lane & 3) == 0) {
+        m_sh[warp * 16 + r] = m_run[hr];
+        l_sh[warp * 16 + r] = l_run[hr];
+      }
+#pragma unroll
+      for (int i = 0; i < DN; ++i) {
+        const int dcol = i * 8 + ((lane & 3) << 1);
+        *reinterpret_cast<float2*>(o_sh + (warp * 16 + r) * D + dcol) =
+            make_float2(o_acc[i][hr * 2], o_acc[i][hr * 2 + 1]);
+      }
+    }
+  }
+  __syncthreads();         // the partials are in shared memory
+  const bool aborted = *abort_flag != 0;
+  if (!aborted) {
+    const float* o_sh = reinterpret_cast<const float*>(dsm);
+    const float* m_sh = o_sh + NS * 16 * D;
+    const float* l_sh = m_sh + NS * 16;
+    for (int i2 = tid; i2 < p.G * (D / 4); i2 += kTcThreads) {
+      const int g = i2 / (D / 4), d4 = (i2 % (D / 4)) * 4;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NS; ++w) M = fmaxf(M, m_sh[w * 16 + g]);
+      float l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < NS; ++w) {
+        const float mw = m_sh[w * 16 + g];
+        const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        l += l_sh[w * 16 + g] * f;
+        const float4 ow = *reinterpret_cast<const float4*>(o_sh + (w * 16 + g) * D + d4);
+        acc.x += ow.x * f; acc.y += ow.y * f; acc.z += ow.z * f; acc.w += ow.w * f;
+      }
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.o_t + ((long long)b * p.Hq + h * p.G + g) * D + d4;
+      *reinterpret_cast<uint2*>(orow) =
+          make_uint2(pack_bf16d(acc.x * inv, acc.y * inv), pack_bf16d(acc.z * inv, acc.w * inv));
+      if (d4 == 0 && p.lse_t != nullptr)
+        p.lse_t[(long long)b * p.Hq + h * p.G + g] = (M + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+  // ---- deferred batched scoring of the oldest scorable tokens of this unit
+  const bool due = (t - p.future) - n_scored + 1 >= p.score_batch;
+  if (due && !aborted) {
+    __syncthreads();       // the partials have been read: shared memory is free
+    const int j_end = n_scored + p.score_batch;
+    for (int jb = n_scored; jb < j_end; jb += kScoreNT)
+      score_tile_tc<RingKV<__nv_bfloat16>>(sp, kv, b, h, jb, j_end, t + 1, dsm);
+  }
+  // every CTA read meta before taking its ticket: the last one advances the step
+  if (tid == 0 && sh[4] == (int)gridDim.x - 1) {
+    p.meta[0] = t + 1;
+    p.meta[1] = due ? n_scored + p.score_batch : n_scored;
+    p.meta[3] = 0;
+  }
+}
+
+template <int D>
+static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
+                                const void* q_t, const void* k_t, const void* v_t, void* o_t,
+                                float* lse_t, int score_batch, DevError* err, cudaStream_t stream) {
+  FusedParams p{};
+  p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = d->Hq / d->Hkv; p.window = d->window; p.sink = d->sink;
+  p.cap = d->cap; p.L = d->window + d->sink + d->cap; p.score_batch = score_batch;
+  p.future = (cnn->k1 - 1 - cnn->past1) + (cnn->k2 - 1 - cnn->past2);
+  p.tau = d->tau; p.scale_log2 = d->scale * 1.4426950408889634f;
+  p.q_t = (const __nv_bfloat16*)q_t; p.k_t = (const __nv_bfloat16*)k_t;
+  p.v_t = (const __nv_bfloat16*)v_t;
+  p.ck = (__nv_bfloat16*)c->k; p.cv = (__nv_bfloat16*)c->v; p.pos = c->pos; p.win_r = c->win_r;
+  p.ret_total = c->ret_total; p.meta = c->meta;
+  p.o_t = (__nv_bfloat16*)o_t; p.lse_t = lse_t; p.err = err;
+  ScoreParams sp = score_params(d, cnn);
+  sp.window = d->window;
+  sp.win_r = c->win_r;
+  const RingKV<__nv_bfloat16> kv{(const __nv_bfloat16*)c->k, (const __nv_bfloat16*)c->v, d->Hkv,
+                                 p.L, d->window, d->D};
+  CUtensorMap mk, mv;
+  const long long rows = (long long)d->B * d->Hkv * p.L;
+  if (!rows_map(&mk, c->k, rows, D, kDecChunk) || !rows_map(&mv, c->v, rows, D, kDecChunk))
+    return cudaErrorInvalidValue;
+  constexpr int NS = fu_stages(D);
+  const size_t smem = kFuRingBytes + 16 * D * 2 + (2 * NS + 1) * 8 + 8 * sizeof(int);
+  // the merge buffers (8 x 16 x D + 256 floats) and the scoring tile reuse the ring
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_fused_kernel<D>, dim3(d->B * d->Hkv), dim3(kTcThreads), smem, stream, mk,
+                    mv, p, sp, kv);
+}
+
 cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
                         const void* q_t, const void* k_t, const void* v_t, void* o_t,
                         float* lse_t, int score_batch, DevError* err, void* scratch,
@@ -719,6 +1170,12 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
   int32_t* counters = reinterpret_cast<int32_t*>(
       reinterpret_cast<char*>(scratch) +
       (size_t)n_units * dec_geom(d).max_parts * G * (d->D + 4) * sizeof(float));
+  // one fused launch when every unit has a CTA of its own and the scorer is the tensor-core tile
+  if (dec_geom(d).single && score_tc_supported(cnn->c_hid, cnn->k1, cnn->k2) &&
+      score_tc_smem_bytes(d->D, cnn->c_hid, cnn->k2) <= (size_t)kFuRingBytes) {
+    if (d->D == 128) return launch_fused<128>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
+    return launch_fused<64>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
+  }
   cudaError_t e = launch_prep<__nv_bfloat16>(d, cnn, c, k_t, v_t, score_batch, counters, err, stream);
   if (e != cudaSuccess) return e;
   if (d->D == 128) return launch_attn<128>(d, c, q_t, o_t, lse_t, part, counters, err, stream);
