@@ -354,8 +354,14 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
                   + 2 * B * Hq * D * 2                # q in, o out
                   + units * row * 2                   # new token write + leaving-token move
                   + units * row * (wl.score_batch + 6) / wl.score_batch)   # deferred scoring reads
+    # the library fuses the whole step into one kernel when every (batch, KV head)
+    # unit gets its own CTA (units <= SMs) and the CNN fits its tensor-core scoring
+    # tile (c_hid * k1 <= 160); otherwise a step is an update kernel + an attention kernel
+    n_sm = torch.cuda.get_device_properties(device).multi_processor_count
+    fused = units <= n_sm and wl.c_hid * wl.k1 <= 160
     return {"ms_step": ms_step, "bytes": bytes_step, "n_keys": n_keys, "B": B,
-            "prefill_with_cnn_ms": prefill_cnn_ms, "launches": 2 * n_steps}
+            "prefill_with_cnn_ms": prefill_cnn_ms, "fused": fused,
+            "launches": (1 if fused else 2) * n_steps}
 
 
 def main():
@@ -425,7 +431,9 @@ def main():
                             "over 4 layer caches (> L2) in one CUDA graph",
                 "value": DI.job_throughput(dec["B"], world, dec["ms_step"] / 1e3), "unit": "tokens/s",
                 "us_per_layer_step": 1e3 * dec["ms_step"],
-                "roofline": {"bound": "hbm", "scope": "whole decode step (2 kernels)",
+                "roofline": {"bound": "hbm",
+                             "scope": "whole decode step (" + ("one fused kernel" if dec["fused"]
+                                                               else "2 kernels") + ")",
                              "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"]},
                 "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
