@@ -726,10 +726,11 @@ static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void
 //   warps 0..NS-1  one per ring stage (NS = 6 at D = 128, 8 at D = 64):
 //              chunk c goes to stage and warp c mod NS, so a warp only ever
 //              waits for the next phase of its own stage (a phase parity
-//              cannot alias).  QK^T and PV on m16n8k16 bf16 MMAs with the G
-//              query heads as MMA rows (the query rows are staged once in
-//              shared memory), online softmax per chunk, the stage released
-//              through an mbarrier -- the warps never wait for one another;
+//              cannot alias).  K Q^T and V^T P^T on m16n8k16 bf16 MMAs with
+//              the keys (resp. head dims) as MMA rows and the G query heads as
+//              the 8 (or 16) columns, online softmax per chunk, the stage
+//              released through an mbarrier -- the warps never wait for one
+//              another;
 // then the NS (m, l, o) partials are merged in shared memory and o_t,
 // lse_t written; when the deferred batch is due the same CTA scores it
 // (score_tile_tc, the arithmetic of lte_score).  The step counter lives in
@@ -810,18 +811,25 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-template <int D>
+// 8x8 bf16 matrix held one row pair per lane (row lane/4, columns 2(lane%4), +1),
+// transposed in registers
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// NT: tiles of 8 query heads per KV head (1 for G <= 8, 2 for G <= 16)
+template <int D, int NT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const FusedParams p, const ScoreParams sp, const RingKV<__nv_bfloat16> kv) {
-  constexpr int KSTEPS = D / 16, DN = D / 8, HALVES = D / 64;
+  constexpr int KSTEPS = D / 16, DM = D / 16, HALVES = D / 64;
   constexpr int kKV = kDecChunk * D * 2;                  // K or V of one chunk
   constexpr int kStage = 2 * kKV;
   constexpr int NS = fu_stages(D);                        // stages = attention warps
-  constexpr int kQBytes = 16 * D * 2;                     // the group's query rows (16, zero padded)
   extern __shared__ __align__(1024) uint8_t dsm[];
-  uint8_t* sq = dsm + kFuRingBytes;                       // 128B-swizzled like the K tiles
-  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kFuRingBytes + kQBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kFuRingBytes);
   uint64_t* empty = full + NS;
   uint64_t* upd = empty + NS;
   int* sh = reinterpret_cast<int*>(upd + 1);   // t, n_scored, retained count, abort, ticket
@@ -833,6 +841,10 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     return;
   }
   pdl_launch_next();
+  if (warp == kFuProdWarp && lane == 0) {         // the descriptors do not depend on the previous step
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_v)) : "memory");
+  }
   if (tid == 0) {
     for (int st = 0; st < NS; ++st) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32d(full + st)));
@@ -868,13 +880,17 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
   ch.nr = 0;
   constexpr int kUnknown = 1 << 30;
-  // the attention warps' running (m, l, o) over their chunks
-  float o_acc[DN][4];
+  // the attention warps' running (m, l, O^T) per head over their chunks
+  float o[DM][NT][4];
 #pragma unroll
-  for (int i = 0; i < DN; ++i)
+  for (int i = 0; i < DM; ++i)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o_acc[i][e] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[i][n][e] = 0.f;
+  float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) m_run[n][0] = m_run[n][1] = -INFINITY, l_run[n][0] = l_run[n][1] = 0.f;
 
   if (warp == kFuUpdWarp) {
     // ---------------------------------------------------------------- cache update
@@ -950,16 +966,25 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
   } else if (warp < NS) {
     // ---------------------------------------------------------------- attention
+    // Transposed products, keys as the MMA M dimension and the group's query
+    // heads as N (NT tiles of 8): S^T = K Q^T (A = K rows by ldmatrix, B = Q^T
+    // held in registers) and O^T += V^T P^T (A = V^T by ldmatrix.trans, B =
+    // P^T: the S^T accumulator fragment of 16 keys x 8 heads is rounded to
+    // bf16 and transposed in registers with movmatrix).
+    uint32_t qb[NT][KSTEPS][2];                  // B fragments of Q^T (heads >= G are 0)
     {
-      // the group's query rows (the MMA A operand; rows >= G are zero), staged once
       const __nv_bfloat16* q0 = p.q_t + ((long long)b * p.Hq + h * p.G) * D;
-      for (int i = tid; i < 16 * (D / 8); i += 32 * NS) {
-        const int r = i / (D / 8), cc = i % (D / 8);
-        const uint4 v = r < p.G ? *reinterpret_cast<const uint4*>(q0 + (long long)r * D + cc * 8)
-                                : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sq + sw128(16, r, cc)) = v;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int head = n * 8 + (lane >> 2);
+#pragma unroll
+        for (int kst = 0; kst < KSTEPS; ++kst)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            qb[n][kst][e] = head < p.G ? *reinterpret_cast<const uint32_t*>(
+                                             q0 + (long long)head * D + kst * 16 + e * 8 + ((lane & 3) << 1))
+                                       : 0u;
       }
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * NS) : "memory");   // attention warps only
     }
     int n_ch = kUnknown;
     const int E = ch.early();
@@ -978,109 +1003,124 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       int slot0, nk;
       ch.get(c, slot0, nk);
       const uint8_t* sk = dsm + st * kStage;
-      float s[8][4];
+      // S^T for the chunk's 64 keys: 4 tiles of 16 keys
+      float s[4][NT][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[i][e] = 0.f;
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int kst = 0; kst < KSTEPS; ++kst) {
-        uint32_t qf[4];
-        ldsm_x4d(smem_u32d(sq + sw128(16, lane & 15, kst * 2 + (lane >> 4))), qf[0], qf[1], qf[2],
-                 qf[3], false);
+          for (int e = 0; e < 4; ++e) s[mt][n][e] = 0.f;
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {         // 16 keys per pair of n8 tiles
-          const int r = np * 16 + ((lane >> 4) << 3) + (lane & 7);
-          const int cc = kst * 2 + ((lane >> 3) & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4d(smem_u32d(sk + sw128(kDecChunk, r, cc)), b0, b1, b2, b3, false);
-          mma_bf16d(s[2 * np], qf, b0, b1);
-          mma_bf16d(s[2 * np + 1], qf, b2, b3);
+      for (int kst = 0; kst < KSTEPS; ++kst)
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int r = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+          uint32_t a[4];
+          ldsm_x4d(smem_u32d(sk + sw128(kDecChunk, r, kst * 2 + (lane >> 4))), a[0], a[1], a[2],
+                   a[3], false);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16d(s[mt][n], a, qb[n][kst][0], qb[n][kst][1]);
         }
-      }
-      float mx[2] = {-INFINITY, -INFINITY};
+      // per head (columns 2(lane%4), +1 of each n tile): mask, scale, max over the keys
+      float mx[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+      for (int n = 0; n < NT; ++n) mx[n][0] = mx[n][1] = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int key = nt * 8 + ((lane & 3) << 1) + (q & 1);
-          s[nt][q] = key < nk ? s[nt][q] * p.scale_log2 : -INFINITY;
-          mx[q >> 1] = fmaxf(mx[q >> 1], s[nt][q]);
-        }
-      float corr[2], mu[2];
+      for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
-        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
-        const float m_new = fmaxf(m_run[hr], mx[hr]);
-        mu[hr] = m_new == -INFINITY ? 0.f : m_new;
-        corr[hr] = m_run[hr] == -INFINITY ? 0.f : exp2f(m_run[hr] - mu[hr]);
-        m_run[hr] = m_new;
-        l_run[hr] *= corr[hr];
-      }
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int i = 0; i < DN; ++i) {
-        o_acc[i][0] *= corr[0]; o_acc[i][1] *= corr[0];
-        o_acc[i][2] *= corr[1]; o_acc[i][3] *= corr[1];
-      }
+          for (int e = 0; e < 4; ++e) {
+            const int key = mt * 16 + (lane >> 2) + ((e >> 1) << 3);
+            s[mt][n][e] = key < nk ? s[mt][n][e] * p.scale_log2 : -INFINITY;
+            mx[n][e & 1] = fmaxf(mx[n][e & 1], s[mt][n][e]);
+          }
+      float corr[NT][2], mu[NT][2];
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t pf[4];
-        {
-          float pv[2][4];
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-          for (int x = 0; x < 2; ++x)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              pv[x][q] = exp2f(s[2 * np + x][q] - mu[q >> 1]);
-              l_run[q >> 1] += pv[x][q];
-            }
-          pf[0] = pack_bf16d(pv[0][0], pv[0][1]);
-          pf[1] = pack_bf16d(pv[0][2], pv[0][3]);
-          pf[2] = pack_bf16d(pv[1][0], pv[1][1]);
-          pf[3] = pack_bf16d(pv[1][2], pv[1][3]);
+        for (int j = 0; j < 2; ++j) {
+          float v = mx[n][j];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          const float m_new = fmaxf(m_run[n][j], v);
+          mu[n][j] = m_new == -INFINITY ? 0.f : m_new;
+          corr[n][j] = m_run[n][j] == -INFINITY ? 0.f : exp2f(m_run[n][j] - mu[n][j]);
+          m_run[n][j] = m_new;
+          l_run[n][j] *= corr[n][j];
         }
 #pragma unroll
-        for (int dp = 0; dp < DN / 2; ++dp) {
-          const int r = np * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
-          const int cc = dp * 2 + (lane >> 4);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4d(smem_u32d(sk + kKV + sw128(kDecChunk, r, cc)), b0, b1, b2, b3, true);
-          mma_bf16d(o_acc[2 * dp], pf, b0, b1);
-          mma_bf16d(o_acc[2 * dp + 1], pf, b2, b3);
+      for (int i = 0; i < DM; ++i)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          o[i][n][0] *= corr[n][0]; o[i][n][1] *= corr[n][1];
+          o[i][n][2] *= corr[n][0]; o[i][n][3] *= corr[n][1];
         }
-      }
+      // P^T as B fragments: for key tile mt, {keys 0-7, keys 8-15} x 8 heads
+      uint32_t pb[4][NT][2];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float pv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pv[e] = exp2f(s[mt][n][e] - mu[n][e & 1]);
+            l_run[n][e & 1] += pv[e];
+          }
+          pb[mt][n][0] = movmatrix_t(pack_bf16d(pv[0], pv[1]));
+          pb[mt][n][1] = movmatrix_t(pack_bf16d(pv[2], pv[3]));
+        }
+      // O^T += V^T P^T: d tiles of 16 x key steps of 16
+#pragma unroll
+      for (int i = 0; i < DM; ++i)
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int r = mt * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int cc = i * 2 + ((lane >> 3) & 1);
+          uint32_t a[4];
+          ldsm_x4d(smem_u32d(sk + kKV + sw128(kDecChunk, r, cc)), a[0], a[1], a[2], a[3], true);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16d(o[i][n], a, pb[mt][n][0], pb[mt][n][1]);
+        }
       __syncwarp();
       if (lane == 0)
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32d(empty + st))
                      : "memory");
     }
-    // finish this warp's row sums (the quad of lanes shares a row)
+    // finish this warp's per-head sums (lanes with equal lane % 4 share heads)
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 1);
-      l_run[hr] += __shfl_xor_sync(0xffffffffu, l_run[hr], 2);
-    }
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        l_run[n][j] += __shfl_xor_sync(0xffffffffu, l_run[n][j], 4);
+        l_run[n][j] += __shfl_xor_sync(0xffffffffu, l_run[n][j], 8);
+        l_run[n][j] += __shfl_xor_sync(0xffffffffu, l_run[n][j], 16);
+      }
   }
   __syncthreads();         // every chunk is consumed and every copy has landed
   if (warp < NS) {
-    float* o_sh = reinterpret_cast<float*>(dsm);                 // [warps][16][D]
-    float* m_sh = o_sh + NS * 16 * D;                  // [warps][16]
-    float* l_sh = m_sh + NS * 16;                      // [warps][16]
+    float* o_sh = reinterpret_cast<float*>(dsm);                 // [warps][16 heads][D]
+    float* m_sh = o_sh + NS * 16 * D;                            // [warps][16]
+    float* l_sh = m_sh + NS * 16;                                // [warps][16]
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int r = (lane >> 2) + hr * 8;
-      if ((lane & 3) == 0) {
-        m_sh[warp * 16 + r] = m_run[hr];
-        l_sh[warp * 16 + r] = l_run[hr];
-      }
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int i = 0; i < DN; ++i) {
-        const int dcol = i * 8 + ((lane & 3) << 1);
-        *reinterpret_cast<float2*>(o_sh + (warp * 16 + r) * D + dcol) =
-            make_float2(o_acc[i][hr * 2], o_acc[i][hr * 2 + 1]);
+      for (int j = 0; j < 2; ++j) {
+        const int head = n * 8 + ((lane & 3) << 1) + j;
+        if (lane < 4) {
+          m_sh[warp * 16 + head] = m_run[n][j];
+          l_sh[warp * 16 + head] = l_run[n][j];
+        }
+#pragma unroll
+        for (int i = 0; i < DM; ++i) {
+          float* row = o_sh + (warp * 16 + head) * D + i * 16 + (lane >> 2);
+          row[0] = o[i][n][j];
+          row[8] = o[i][n][2 + j];
+        }
       }
-    }
   }
   __syncthreads();         // the partials are in shared memory
   const bool aborted = *abort_flag != 0;
@@ -1127,7 +1167,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 }
 
-template <int D>
+template <int D, int NT>
 static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte_cache* c,
                                 const void* q_t, const void* k_t, const void* v_t, void* o_t,
                                 float* lse_t, int score_batch, DevError* err, cudaStream_t stream) {
@@ -1151,12 +1191,12 @@ static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte
   if (!rows_map(&mk, c->k, rows, D, kDecChunk) || !rows_map(&mv, c->v, rows, D, kDecChunk))
     return cudaErrorInvalidValue;
   constexpr int NS = fu_stages(D);
-  const size_t smem = kFuRingBytes + 16 * D * 2 + (2 * NS + 1) * 8 + 8 * sizeof(int);
+  const size_t smem = kFuRingBytes + (2 * NS + 1) * 8 + 8 * sizeof(int);
   // the merge buffers (8 x 16 x D + 256 floats) and the scoring tile reuse the ring
-  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<D, NT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_fused_kernel<D>, dim3(d->B * d->Hkv), dim3(kTcThreads), smem, stream, mk,
+  return launch_pdl(decode_fused_kernel<D, NT>, dim3(d->B * d->Hkv), dim3(kTcThreads), smem, stream, mk,
                     mv, p, sp, kv);
 }
 
@@ -1173,8 +1213,12 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
   // one fused launch when every unit has a CTA of its own and the scorer is the tensor-core tile
   if (dec_geom(d).single && score_tc_supported(cnn->c_hid, cnn->k1, cnn->k2) &&
       score_tc_smem_bytes(d->D, cnn->c_hid, cnn->k2) <= (size_t)kFuRingBytes) {
-    if (d->D == 128) return launch_fused<128>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
-    return launch_fused<64>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
+    const bool g8 = G <= 8;
+    if (d->D == 128)
+      return g8 ? launch_fused<128, 1>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream)
+                : launch_fused<128, 2>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
+    return g8 ? launch_fused<64, 1>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream)
+              : launch_fused<64, 2>(d, cnn, c, q_t, k_t, v_t, o_t, lse_t, score_batch, err, stream);
   }
   cudaError_t e = launch_prep<__nv_bfloat16>(d, cnn, c, k_t, v_t, score_batch, counters, err, stream);
   if (e != cudaSuccess) return e;

@@ -64,6 +64,8 @@ def _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, score_batch, ch
     (1, 4, 1, 64, 2, 40, 5, 50, 90, 1),
     (2, 16, 4, 128, 4, 128, 300, 20, 200, 64),      # prompt shorter than the window
     (1, 4, 2, 128, 3, 32, 0, 100, 60, 8),           # cap 0: sink + window only
+    (1, 16, 1, 128, 4, 64, 40, 130, 70, 16),        # G = 16: two tiles of 8 query heads
+    (2, 16, 2, 64, 2, 48, 20, 90, 60, 4),           # G = 8, head dim 64
 ])
 def test_decode_vs_oracle_simulation(layer, cfg):
     B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = cfg
