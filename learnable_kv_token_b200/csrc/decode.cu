@@ -277,6 +277,15 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, uin
       : "memory");
 }
 
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                       int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -682,6 +691,21 @@ static bool rows_map(CUtensorMap* m, const void* base, long long rows, int D, in
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over `rows` rows of D elements seen as (64 columns, row,
+// D/64 column halves): one box of 64 x box_rows x D/64 lands as [half][row][128 B],
+// 128B-swizzled -- the layout of D/64 separate 2-D boxes, in one copy.
+static bool rows_map_halves(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(D / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(D / 64)};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void* q_t, void* o_t,
                                float* lse_t, float* part, int32_t* counters, DevError* err,
@@ -718,12 +742,12 @@ static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void
 //              the rows are written to global memory, fenced for the async
 //              proxy, and the new retained count is published through an
 //              mbarrier;
-//   warp 9     TMA producer: 64-slot chunks of K and V into a ring of
-//              192 KiB.  The window chunks the update cannot touch go first
+//   warp 9     TMA producer: 64-slot chunks of K and V (one 3-D box each)
+//              into a ring of up to 192 KiB.  The window chunks the update cannot touch go first
 //              (their copies overlap the update); the chunk holding slot
 //              t mod w, the sinks and the retained ring follow once the
 //              update has landed;
-//   warps 0..NS-1  one per ring stage (NS = 6 at D = 128, 8 at D = 64):
+//   warps 0..NS-1  one per ring stage (NS = 6 at D = 128, 7 at D = 64):
 //              chunk c goes to stage and warp c mod NS, so a warp only ever
 //              waits for the next phase of its own stage (a phase parity
 //              cannot alias).  K Q^T and V^T P^T on m16n8k16 bf16 MMAs with
@@ -731,16 +755,21 @@ static cudaError_t launch_attn(const lte_dims* d, const lte_cache* c, const void
 //              the 8 (or 16) columns, online softmax per chunk, the stage
 //              released through an mbarrier -- the warps never wait for one
 //              another;
+//   warp NS    takes the step ticket (below) once the step index is known,
+//              off the path of the copies;
 // then the NS (m, l, o) partials are merged in shared memory and o_t,
 // lse_t written; when the deferred batch is due the same CTA scores it
 // (score_tile_tc, the arithmetic of lte_score).  The step counter lives in
 // the cache: every CTA reads meta[0..1], then takes a ticket on meta[3]; the
-// last ticket advances t (and n_scored) and resets the ticket.
+// last ticket advances t (and n_scored) and resets the ticket.  The partials
+// are stored in rows padded to D + 4 floats, so that the lanes of a warp write
+// distinct banks.
 constexpr int kFuUpdWarp = 8, kFuProdWarp = 9;
 constexpr int kFuRingBytes = 192 * 1024;
-// ring stages (= attention warps) for head dim D: at most 192 KiB and 8 warps
+// ring stages (= attention warps) for head dim D: at most 192 KiB and 7 warps
+// (warp NS takes the step ticket)
 __host__ __device__ constexpr int fu_stages(int D) {
-  return kFuRingBytes / (4 * kDecChunk * D) < 8 ? kFuRingBytes / (4 * kDecChunk * D) : 8;
+  return kFuRingBytes / (4 * kDecChunk * D) < 7 ? kFuRingBytes / (4 * kDecChunk * D) : 7;
 }
 
 struct FusedParams {
@@ -824,10 +853,11 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const FusedParams p, const ScoreParams sp, const RingKV<__nv_bfloat16> kv) {
-  constexpr int KSTEPS = D / 16, DM = D / 16, HALVES = D / 64;
+  constexpr int KSTEPS = D / 16, DM = D / 16;
   constexpr int kKV = kDecChunk * D * 2;                  // K or V of one chunk
   constexpr int kStage = 2 * kKV;
   constexpr int NS = fu_stages(D);                        // stages = attention warps
+  constexpr int kRowF = D + 4;     // partial rows padded: the per-lane stores hit distinct banks
   extern __shared__ __align__(1024) uint8_t dsm[];
   uint64_t* full = reinterpret_cast<uint64_t*>(dsm + kFuRingBytes);
   uint64_t* empty = full + NS;
@@ -858,6 +888,11 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   if (tid == 0) {
     sh[0] = p.meta[0];
     sh[1] = p.meta[1];
+  }
+  __syncthreads();
+  if (warp == NS && lane == 0) {
+    // the step ticket, taken after the step index was read and used only at the
+    // end, so that this round trip is off the path of the copies and the update
     int ticket;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                  : "=r"(ticket)
@@ -865,7 +900,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                  : "memory");
     sh[4] = ticket;
   }
-  __syncthreads();
   const int t = sh[0], n_scored = sh[1];
   const int slot_w = t % p.window, leaving = t - p.window;
   const long long urow = (long long)u * p.L;
@@ -954,11 +988,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kStage)
                      : "memory");
         const int row = (int)(urow + slot0);
-#pragma unroll
-        for (int hf = 0; hf < HALVES; ++hf) {
-          tma_2d(dst + hf * kDecChunk * 128, &tm_k, bar, hf * 64, row);
-          tma_2d(dst + kKV + hf * kDecChunk * 128, &tm_v, bar, hf * 64, row);
-        }
+        tma_3d(dst, &tm_k, bar, 0, row, 0);          // all D/64 column halves in one box
+        tma_3d(dst + kKV, &tm_v, bar, 0, row, 0);
       }
       // the copies issued last have landed before shared memory is reused
       for (int j = c - NS > 0 ? c - NS : 0; j < c; ++j)
@@ -1102,8 +1133,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
   __syncthreads();         // every chunk is consumed and every copy has landed
   if (warp < NS) {
-    float* o_sh = reinterpret_cast<float*>(dsm);                 // [warps][16 heads][D]
-    float* m_sh = o_sh + NS * 16 * D;                            // [warps][16]
+    float* o_sh = reinterpret_cast<float*>(dsm);                 // [warps][16 heads][D + 4]
+    float* m_sh = o_sh + NS * 16 * kRowF;                        // [warps][16]
     float* l_sh = m_sh + NS * 16;                                // [warps][16]
 #pragma unroll
     for (int n = 0; n < NT; ++n)
@@ -1116,7 +1147,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
 #pragma unroll
         for (int i = 0; i < DM; ++i) {
-          float* row = o_sh + (warp * 16 + head) * D + i * 16 + (lane >> 2);
+          float* row = o_sh + (warp * 16 + head) * kRowF + i * 16 + (lane >> 2);
           row[0] = o[i][n][j];
           row[8] = o[i][n][2 + j];
         }
@@ -1126,7 +1157,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const bool aborted = *abort_flag != 0;
   if (!aborted) {
     const float* o_sh = reinterpret_cast<const float*>(dsm);
-    const float* m_sh = o_sh + NS * 16 * D;
+    const float* m_sh = o_sh + NS * 16 * kRowF;
     const float* l_sh = m_sh + NS * 16;
     for (int i2 = tid; i2 < p.G * (D / 4); i2 += kTcThreads) {
       const int g = i2 / (D / 4), d4 = (i2 % (D / 4)) * 4;
@@ -1140,7 +1171,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const float mw = m_sh[w * 16 + g];
         const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
         l += l_sh[w * 16 + g] * f;
-        const float4 ow = *reinterpret_cast<const float4*>(o_sh + (w * 16 + g) * D + d4);
+        const float4 ow = *reinterpret_cast<const float4*>(o_sh + (w * 16 + g) * kRowF + d4);
         acc.x += ow.x * f; acc.y += ow.y * f; acc.z += ow.z * f; acc.w += ow.w * f;
       }
       const float inv = 1.f / l;
@@ -1188,7 +1219,8 @@ static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte
                                  p.L, d->window, d->D};
   CUtensorMap mk, mv;
   const long long rows = (long long)d->B * d->Hkv * p.L;
-  if (!rows_map(&mk, c->k, rows, D, kDecChunk) || !rows_map(&mv, c->v, rows, D, kDecChunk))
+  if (!rows_map_halves(&mk, c->k, rows, D, kDecChunk) ||
+      !rows_map_halves(&mv, c->v, rows, D, kDecChunk))
     return cudaErrorInvalidValue;
   constexpr int NS = fu_stages(D);
   const size_t smem = kFuRingBytes + (2 * NS + 1) * 8 + 8 * sizeof(int);
