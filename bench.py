@@ -359,7 +359,7 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
     # tile (c_hid * k1 <= 160); otherwise a step is an update kernel + an attention kernel
     n_sm = torch.cuda.get_device_properties(device).multi_processor_count
     fused = units <= n_sm and wl.c_hid * wl.k1 <= 160
-    return {"ms_step": ms_step, "bytes": bytes_step, "n_keys": n_keys, "B": B,
+    return {"ms_step": ms_step, "bytes": bytes_step, "n_keys": n_keys, "B": B, "units": units,
             "prefill_with_cnn_ms": prefill_cnn_ms, "fused": fused,
             "launches": (1 if fused else 2) * n_steps}
 
@@ -435,7 +435,10 @@ def main():
                              "scope": "whole decode step (" + ("one fused kernel" if dec["fused"]
                                                                else "2 kernels") + ")",
                              "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                             "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"]},
+                             "frac": gbs / pk["hbm_gbs"], "bytes_per_step": dec["bytes"],
+                             "traffic": (traffic_from_profiles("learnable_kv_token_b200/csrc/decode.cu",
+                                                               dec["units"])
+                                         if dec["fused"] else None)},
                 "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
             }
         if world == 1 and args.cpu_seconds > 0:
