@@ -248,6 +248,21 @@ lte_status lte_clear_device_error(void* workspace, void* stream);
 lte_status lte_read_device_error(const void* workspace, int32_t* code, int32_t* where,
                                  void* stream);
 
+/* lte_wait_probe -- diagnostic: shows on the live device that a bounded wait
+ * ends in an error status instead of a hang.  The pages have no counterpart;
+ * it exercises the failure path of the library's device waits (the bounded
+ * mbarrier wait of the fused decode step).  One small kernel: a thread
+ * arrives on an mbarrier once the device word *flag equals `expect`, another
+ * waits for that barrier for at most limit_ns.  If the flag never holds
+ * `expect`, the wait runs out after ~limit_ns, LTE_ERR_TIMEOUT is recorded in
+ * the workspace's error word (read it with lte_read_device_error) and the
+ * kernel returns; otherwise the error word is left as it was.
+ * flag: device int32, 4-byte aligned, read only.  limit_ns in [1e3, 1e10].
+ * workspace: any workspace of >= 16 bytes (only its error word is used).
+ * Errors: LTE_ERR_INVALID_ARG (flag, limit), LTE_ERR_WORKSPACE, LTE_ERR_CUDA. */
+lte_status lte_wait_probe(const int32_t* flag, int32_t expect, int64_t limit_ns, void* workspace,
+                          void* stream);
+
 /* ---------------------------------------------------------------------------
  * Gated linear attention, the hybrid's companion layer.  ["Sparse Linear
  * Attention: Viewing SWA from the Perspective of Linear Attention", section

@@ -821,20 +821,10 @@ struct FuChunks {
   }
 };
 
-// bounded wait that also gives up when the CTA is aborting
+// bounded wait (1 s) that also gives up when the CTA is aborting
 __device__ __forceinline__ bool fu_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                         DevError* err, int where) {
-  if (mbar_try_d(bar, parity)) return true;
-  const unsigned long long t0 = gtime_d();
-  while (true) {
-    if (mbar_try_d(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (gtime_d() - t0 > 1000000000ull) {
-      record_error(err, LTE_ERR_TIMEOUT, where);
-      *abort_flag = 1;
-      return false;
-    }
-  }
+  return mbar_wait_bounded(bar, parity, 1000000000ull, abort_flag, err, where);
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");

@@ -251,6 +251,15 @@ lte_status lte_read_device_error(const void* workspace, int32_t* code, int32_t* 
   return LTE_OK;
 }
 
+lte_status lte_wait_probe(const int32_t* flag, int32_t expect, int64_t limit_ns, void* workspace,
+                          void* stream) {
+  if (flag == nullptr || reinterpret_cast<uintptr_t>(flag) % 4 != 0) return LTE_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return LTE_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace)) return LTE_ERR_WORKSPACE;
+  return from_cuda(lte::wait_probe(flag, expect, (unsigned long long)limit_ns,
+                                   reinterpret_cast<lte::DevError*>(workspace), as_stream(stream)));
+}
+
 lte_status lte_gla_prefill(int32_t B, int32_t T, int32_t H, int32_t dk, int32_t dv,
                            int32_t dtype, const void* q, const void* k, const void* v,
                            const float* a, void* o, float* state, void* stream) {

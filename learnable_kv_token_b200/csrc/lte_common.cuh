@@ -23,6 +23,7 @@ enum : int32_t {
   kWhereAttnTmemWait = 103,
   kWhereDecodeIndex = 201,
   kWhereDecodeMeta = 202,
+  kWhereWaitProbe = 301,
 };
 
 // Bounded spin: iterations after which a device wait gives up.
@@ -31,6 +32,47 @@ constexpr long long kSpinLimit = 1ll << 26;
 __device__ __forceinline__ void record_error(DevError* e, int32_t code, int32_t where) {
   if (e == nullptr) return;
   if (atomicCAS(&e->code, 0, code) == 0) atomicExch(&e->where, where);
+}
+
+// Global time in nanoseconds.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// True once phase `parity` of the shared-memory mbarrier at `bar` has completed.
+__device__ __forceinline__ bool mbar_try_wait_parity(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of an mbarrier: true once the phase has
+// completed; false when the CTA is aborting (*abort_flag set by another wait)
+// or when limit_ns of global time have passed, in which case it records
+// LTE_ERR_TIMEOUT (site `where`) in the error word and sets *abort_flag so that
+// the CTA's other waits give up as well.  No wait of the library spins for ever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns,
+                                                  volatile int* abort_flag, DevError* err,
+                                                  int32_t where) {
+  if (mbar_try_wait_parity(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait_parity(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > limit_ns) {
+      record_error(err, LTE_ERR_TIMEOUT, where);
+      *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

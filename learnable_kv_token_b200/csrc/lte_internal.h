@@ -55,6 +55,10 @@ cudaError_t decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* 
 // decode.cu: the allocation-free variant's scratch (file-scope device array)
 cudaError_t noalloc_scratch(void** ptr);
 
+// diag.cu
+cudaError_t wait_probe(const int32_t* flag, int32_t expect, unsigned long long limit_ns,
+                       DevError* err, cudaStream_t stream);
+
 // gla.cu
 cudaError_t gla_prefill(int B, int T, int H, int dk, int dv, int dtype, const void* q,
                         const void* k, const void* v, const float* a, void* o, float* state,

@@ -71,6 +71,7 @@ _SIG = {
                                 _P, _P, _P, _P, _I, _P],
     "lte_clear_device_error": [_P, _P],
     "lte_read_device_error": [_P, C.POINTER(C.c_int32), C.POINTER(C.c_int32), _P],
+    "lte_wait_probe": [_P, _I, C.c_int64, _P, _P],
     "lte_gla_prefill": [_I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P],
     "lte_gla_decode_step": [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P],
 }
@@ -187,6 +188,14 @@ def lte_read_device_error(workspace, stream=None):
     code, where = C.c_int32(0), C.c_int32(0)
     _call("lte_read_device_error", _ptr(workspace), C.byref(code), C.byref(where), _stream(stream))
     return code.value, where.value
+
+
+def lte_wait_probe(flag, expect, limit_ns, workspace, stream=None):
+    """Diagnostic: a bounded device wait on an mbarrier that arrives only once
+    the device int32 `flag` equals `expect`; if it never does, the wait runs
+    out after limit_ns and LTE_ERR_TIMEOUT lands in the workspace error word."""
+    _call("lte_wait_probe", _ptr(flag), int(expect), int(limit_ns), _ptr(workspace),
+          _stream(stream))
 
 
 def lte_gla_prefill(q, k, v, a, o, state, stream=None):

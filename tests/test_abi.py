@@ -77,4 +77,9 @@ def test_host_validation_without_gpu(lib):
     assert f.lte_decode_step(C.byref(dd), C.byref(cnn), C.byref(cache), C.c_void_p(16),
                              C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), None, 11,
                              C.c_void_p(16), 1 << 20, None) == 1
+    # wait probe: null or misaligned flag, limit out of range, missing workspace
+    assert f.lte_wait_probe(None, 1, 1000000, C.c_void_p(16), None) == 1
+    assert f.lte_wait_probe(C.c_void_p(18), 1, 1000000, C.c_void_p(16), None) == 1
+    assert f.lte_wait_probe(C.c_void_p(16), 1, 10, C.c_void_p(16), None) == 1
+    assert f.lte_wait_probe(C.c_void_p(16), 1, 1000000, None, None) == 5
     assert L.version().startswith("lte-b200")
