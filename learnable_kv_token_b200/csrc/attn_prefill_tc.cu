@@ -122,20 +122,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the CTA is aborting or the wait ran out (then aborts).
+// Bounded wait (the library's mbar_wait_bounded): false if the CTA is aborting
+// or the wait ran out (then aborts).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           DevError* err, int where) {
-  if (mbar_try(bar, parity)) return true;
-  const unsigned long long t0 = gtime();
-  while (true) {
-    if (mbar_try(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (gtime() - t0 > kWaitNs) {
-      record_error(err, LTE_ERR_TIMEOUT, where);
-      *abort_flag = 1;
-      return false;
-    }
-  }
+  return mbar_wait_bounded(bar, parity, kWaitNs, abort_flag, err, where);
 }
 // Warp-uniform bounded wait (every lane of the calling warp must call it):
 // the warp proceeds only if every lane saw the phase complete.
