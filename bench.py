@@ -364,6 +364,103 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
             "launches": (1 if fused else 2) * n_steps}
 
 
+def rows_bench(args, rank, world, device, lte_decode_ms):
+    """The hot-path rows outside the two headline steps, each launch timed alone
+    with CUDA events after warm-up, on the hybrid workload (B=32, 4096-token
+    prompts, Hq=16 / Hkv=4, D=128, the CNN scored live, tau 0.5): retention
+    scoring (a1), compaction with the column copy (a2), sparse-attention prefill
+    over the scored mask (a3 at the scored retention rate), gated linear
+    attention prefill and decode step (a7); and the laLTE pair -- one gated
+    linear-attention layer followed by one LTE layer -- as tokens/s."""
+    from learnable_kv_token_b200 import layer
+    from learnable_kv_token_b200 import lte as L
+    wl = LI.WORKLOADS["hybrid"]
+    B, T, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
+    seed = DI.shard_seed(wl.seed, rank)
+    inp = LI.lte_inputs(wl.with_(seed=seed), T=T)
+    q, k, v = (inp[x].to(device) for x in ("q", "k", "v"))
+    cnn = tuple(x.to(device) for x in inp["cnn"])
+    p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=wl.cap, tau=wl.tau)
+    dims = p.dims(B, T, Hq, Hkv, D, torch.bfloat16)
+    bufs = layer.PrefillBuffers(B, T, Hq, Hkv, D, torch.bfloat16, wl.sink, dims, device, want_r=True)
+    c, _keep = L.make_cnn(*cnn, p.past1, p.past2)
+    n_scored = T - layer.cnn_future(cnn[0], cnn[2], p.past1, p.past2)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return DI.max_over_ranks(e0.elapsed_time(e1) / reps, world, device)
+
+    t_score = timed(lambda: L.lte_score(dims, c, k, v, 0, n_scored, bufs.r, bufs.mask, stream))
+    t_compact = timed(lambda: L.lte_evict_compact(dims, None, bufs.mask, n_scored, bufs.idx,
+                                                  bufs.nret, bufs.cnt, k, v, bufs.k_col,
+                                                  bufs.v_col, stream))
+    t_attn = timed(lambda: L.lte_sparse_attn_prefill(dims, q, k, v, bufs.cnt, bufs.k_col,
+                                                     bufs.v_col, bufs.o, bufs.lse, bufs.ws, stream))
+    assert L.lte_read_device_error(bufs.ws) == (0, 0)
+    mask = bufs.mask.cpu().numpy()
+    nret = int(bufs.nret.sum())
+    pairs = attended_pairs(mask, wl.sink, wl.window, wl.cap).sum()
+    attn_flops = 4.0 * D * wl.G * float(pairs)
+    score_flops = 2.0 * B * Hkv * n_scored * (wl.c_hid * 2 * D * wl.k1 + wl.c_hid * wl.k2)
+    score_bytes = B * T * Hkv * D * 2 * 2 + B * Hkv * n_scored * 5
+    compact_bytes = (B * Hkv * T * (1 + 8) + B * Hkv * 4
+                     + 2 * (wl.sink * B * Hkv + nret) * 2 * D * 2)
+    del bufs, q, k, v
+
+    H, dk = 16, 128
+    gq, gk, gv, ga = (x.to(device) for x in LI.gla_inputs(B, T, H, dk, dk, LI.generator(seed + 1000)))
+    go = torch.empty_like(gv)
+    state = torch.zeros(B, H, dk, dk, dtype=torch.float32, device=device)
+    t_gla = timed(lambda: L.lte_gla_prefill(gq, gk, gv, ga, go, state, stream))
+    q1, k1_, v1, a1, o1 = (x[:, 0].contiguous() for x in (gq, gk, gv, ga, go))
+    # decode steps rotate over 6 layer states (6 x 32 MiB > L2), as a layer stack would
+    states = [state.clone() for _ in range(6)]
+    it_st = iter(range(1 << 30))
+    t_gla_dec = timed(lambda: L.lte_gla_decode_step(q1, k1_, v1, a1, o1, states[next(it_st) % 6],
+                                                    stream), reps=60)
+    gla_bytes = B * T * H * dk * (4 * 2 + 4) + B * H * dk * dk * 4
+    gla_dec_bytes = 2 * B * H * dk * dk * 4 + B * H * dk * (4 * 2 + 4)
+    pk = peaks()
+
+    def hbm(nbytes, ms):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / pk["hbm_gbs"], "bytes": nbytes}
+
+    def tensor(flops, ms):
+        tf = flops / (ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tf / pk["bf16_tflops"], "flops": flops}
+
+    lte_prefill_ms = t_score + t_compact + t_attn
+    return {
+        "workload": "hybrid B=32 T=4096 (prompt) Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512, CNN "
+                    "32ch k5/k3 scored live, tau 0.5; GLA 16 heads dk=dv=128, chunk 64",
+        "a1_score_ms": t_score, "a1_roofline": tensor(score_flops, t_score),
+        "a1_bytes_rate": hbm(score_bytes, t_score),
+        "a2_compact_ms": t_compact, "a2_roofline": hbm(compact_bytes, t_compact),
+        "a3_attn_ms": t_attn, "a3_roofline": tensor(attn_flops, t_attn),
+        "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
+        "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),
+        "a7_gla_decode_us": 1e3 * t_gla_dec, "a7_decode_roofline": hbm(gla_dec_bytes, t_gla_dec),
+        "pair_prefill": {"value": DI.job_throughput(B * T, world, (t_gla + lte_prefill_ms) / 1e3),
+                         "unit": "tokens/s", "ms": t_gla + lte_prefill_ms},
+        "pair_decode": (None if lte_decode_ms is None else
+                        {"value": DI.job_throughput(B, world, (t_gla_dec + lte_decode_ms) / 1e3),
+                         "unit": "tokens/s", "us": 1e3 * (t_gla_dec + lte_decode_ms)}),
+        "launches": 2 + 5 * 3 + 5 + 50,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -371,6 +468,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="lte", choices=["lte", "reference"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the per-row measurements (scoring, compaction, GLA, hybrid pair)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle CPU sample length (0 skips the cpu_baseline leg)")
     ap.add_argument("--batch", type=int, default=0,
@@ -392,6 +491,8 @@ def main():
     pk = peaks()
     pf = prefill_bench(args, rank, world, device)
     dec = None if args.no_decode else decode_bench(args, rank, world, device)
+    rows = None if args.no_rows else rows_bench(args, rank, world, device,
+                                                dec["ms_step"] if dec else None)
 
     if rank == 0:
         value = DI.job_throughput(pf["B"] * pf["T"], world, pf["ms_step"] / 1e3)
@@ -441,6 +542,8 @@ def main():
                                          if dec["fused"] else None)},
                 "prompt_prefill_with_cnn_ms": dec["prefill_with_cnn_ms"],
             }
+        if rows is not None:
+            line["rows"] = {k: v for k, v in rows.items() if k != "launches"}
         if world == 1 and args.cpu_seconds > 0:
             tok, sec, desc = oracle_sample(LI.WORKLOADS["prefill"], args.cpu_seconds,
                                            2.5 * args.cpu_seconds)
