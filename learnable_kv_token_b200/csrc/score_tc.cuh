@@ -32,12 +32,13 @@ __host__ __device__ inline bool score_tc_supported(int c_hid, int k1, int k2) {
   return c_hid * k1 <= kTcN && kScoreNT + k1 + k2 - 2 <= kTcRows;
 }
 
-// shared memory (bytes): x [80][2D] bf16 | W hi, lo [160][64] bf16 | u [c_hid][NU] fp32;
-// Z [80][160] fp32 reuses the x and W region after the GEMM.
+// shared memory (bytes): x [80][2D] bf16 | W hi, lo [160][64] bf16 | u [c_hid][NU] fp32 |
+// layer-2 weights and layer-1 biases [c_hid * (k2 + 1)] fp32; Z [160][80] fp32 reuses the x
+// and W region after the GEMM.
 __host__ __device__ inline size_t score_tc_smem_bytes(int D, int c_hid, int k2) {
   const size_t xw = (size_t)kTcRows * 2 * D * 2 + 2 * (size_t)kTcN * kTcKC * 2;
   const size_t z = (size_t)kTcRows * kTcN * 4;
-  return (xw > z ? xw : z) + (size_t)c_hid * (kScoreNT + k2 - 1) * 4;
+  return (xw > z ? xw : z) + (size_t)c_hid * (kScoreNT + k2 - 1) * 4 + (size_t)c_hid * (k2 + 1) * 4;
 }
 
 namespace stc {
@@ -62,6 +63,55 @@ __device__ __forceinline__ void mma(float* c, const uint32_t* a, uint32_t b0, ui
 }
 }  // namespace stc
 
+// Layers 1 (tap sum, bias, SiLU) and 2 (+ sigmoid, threshold) of a tile, after
+// the GEMM, shared by every tensor-core scoring kernel so that a token's score
+// is the same instruction sequence wherever it is computed.  zs holds Z
+// transposed, [160 columns][R rows] (the tap sum then reads consecutive rows:
+// conflict-free); u gets [c_hid][NU], NU = NT + k2 - 1; wsm c_hid * (k2 + 1)
+// floats for w2 and b1 of head h.  Row r of Z is x position jb - past2 - past1 + r.
+// Writes the scores of tokens [jb, min(jb + NT, j_end)).  All threads call it.
+__device__ __forceinline__ void score_tail(const ScoreParams& p, const float* zs, int R, float* us,
+                                           float* wsm, int NT, int b, int h, int jb, int j_end,
+                                           int T_avail) {
+  const int tid = threadIdx.x, nthreads = blockDim.x;
+  const int NU = NT + p.k2 - 1, nw2 = p.c_hid * p.k2;
+  float* w2s = wsm;
+  float* b1s = wsm + nw2;
+  for (int i = tid; i < nw2; i += nthreads) w2s[i] = p.w2[(long long)h * nw2 + i];
+  for (int i = tid; i < p.c_hid; i += nthreads) b1s[i] = p.b1[h * p.c_hid + i];
+  __syncthreads();
+  // ---- u[c][q] = SiLU(b1[c] + sum_kk Z[q + kk][c*k1 + kk]); 0 outside the tokens
+  const int u0 = jb - p.past2;
+  for (int i = tid; i < p.c_hid * NU; i += nthreads) {
+    const int c = i / NU, q = i % NU;
+    const int ug = u0 + q;
+    float z = 0.f;
+    for (int kk = 0; kk < p.k1; ++kk) z += zs[(c * p.k1 + kk) * R + q + kk];
+    us[c * NU + q] = (ug >= 0 && ug < T_avail) ? siluf_(b1s[c] + z) : 0.f;
+  }
+  __syncthreads();
+  // ---- layer 2 + sigmoid + threshold (fp32), one thread per token
+  if (tid < NT) {
+    const int j = jb + tid;
+    if (j < j_end) {
+      float z = p.b2[h];
+      for (int c = 0; c < p.c_hid; ++c) {
+#pragma unroll 3
+        for (int kk = 0; kk < p.k2; ++kk) z = fmaf(w2s[c * p.k2 + kk], us[c * NU + tid + kk], z);
+      }
+      const float r = sigmoidf_(z);
+      if (p.win_r != nullptr) {
+        p.win_r[(long long)(b * p.Hkv + h) * p.window + (j % p.window)] = r;
+      } else {
+        const long long o = (long long)(b * p.Hkv + h) * p.T + j;
+        p.r[o] = r;
+        if (p.mask) p.mask[o] = (j >= p.sink && r >= p.tau) ? 1 : 0;
+      }
+    }
+  }
+  __syncthreads();   // shared memory is reused next
+}
+
 // Scores of tokens [jb, min(jb + 64, j_end)) of unit (b, h); tokens [0, T_avail)
 // exist.  Called by all kTcThreads threads (it synchronises the CTA).
 template <typename KV>
@@ -76,10 +126,11 @@ __device__ __forceinline__ void score_tile_tc(const ScoreParams& p, const KV& kv
   uint8_t* xs = smem;                                          // [80][2D] bf16
   uint8_t* whi = smem + kTcRows * xrow_b;                      // [160][64] bf16
   uint8_t* wlo = whi + kTcN * kTcKC * 2;
-  float* zs = reinterpret_cast<float*>(smem);                  // [80][160] fp32 (after GEMM)
+  float* zs = reinterpret_cast<float*>(smem);                  // [160][80] fp32 (after GEMM)
   const size_t xw = (size_t)kTcRows * xrow_b + 2 * (size_t)kTcN * kTcKC * 2;
   const size_t zb = (size_t)kTcRows * kTcN * 4;
   float* us = reinterpret_cast<float*>(smem + (xw > zb ? xw : zb));   // [c_hid][NU]
+  float* wsm = us + p.c_hid * NU;                              // w2, b1 of head h
 
   // ---- x rows [x0, x0 + 80): [k; v] of existing tokens, zero elsewhere
   const int cpr = xrow_b / 16;                                 // 16-byte chunks per row
@@ -152,40 +203,9 @@ __device__ __forceinline__ void score_tile_tc(const ScoreParams& p, const KV& kv
     for (int e = 0; e < 4; ++e) {
       const int row = mt * 16 + (lane >> 2) + (e >> 1) * 8;
       const int col = nh * 80 + nt * 8 + (lane & 3) * 2 + (e & 1);
-      zs[row * kTcN + col] = acc[nt][e];
+      zs[col * kTcRows + row] = acc[nt][e];
     }
-  __syncthreads();
-
-  // ---- u[c][q] = SiLU(b1[c] + sum_kk Z[q + kk][c*k1 + kk]); 0 outside the tokens
-  const int u0 = jb - p.past2;
-  for (int i = tid; i < p.c_hid * NU; i += kTcThreads) {
-    const int c = i / NU, q = i % NU;
-    const int ug = u0 + q;
-    float z = 0.f;
-    for (int kk = 0; kk < p.k1; ++kk) z += zs[(q + kk) * kTcN + c * p.k1 + kk];
-    us[c * NU + q] = (ug >= 0 && ug < T_avail) ? siluf_(p.b1[h * p.c_hid + c] + z) : 0.f;
-  }
-  __syncthreads();
-
-  // ---- layer 2 + sigmoid + threshold (fp32)
-  if (tid < kScoreNT) {
-    const int j = jb + tid;
-    if (j < j_end) {
-      float z = p.b2[h];
-      const float* w2h = p.w2 + (long long)h * p.c_hid * p.k2;
-      for (int c = 0; c < p.c_hid; ++c)
-        for (int kk = 0; kk < p.k2; ++kk) z = fmaf(w2h[c * p.k2 + kk], us[c * NU + tid + kk], z);
-      const float r = sigmoidf_(z);
-      if (p.win_r != nullptr) {
-        p.win_r[(long long)(b * p.Hkv + h) * p.window + (j % p.window)] = r;
-      } else {
-        const long long o = (long long)(b * p.Hkv + h) * p.T + j;
-        p.r[o] = r;
-        if (p.mask) p.mask[o] = (j >= p.sink && r >= p.tau) ? 1 : 0;
-      }
-    }
-  }
-  __syncthreads();   // shared memory is reused by the next tile
+  score_tail(p, zs, kTcRows, us, wsm, kScoreNT, b, h, jb, j_end, T_avail);
 }
 
 }  // namespace lte

@@ -204,3 +204,29 @@ def test_decode_full_size_sampled(layer):
                                        torch.bfloat16, f"unit {b},{h} step {t}")
                 compared += 1
     assert compared >= len(rets)
+
+
+def test_decode_scores_equal_lte_score_bitwise(layer):
+    """The decode step's deferred scores (the tensor-core tile inside the step)
+    equal lte_score's (the persistent kernel) bit for bit, token by token."""
+    B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = 2, 8, 2, 128, 4, 96, 20, 150, 120, 16
+    T = T0 + steps
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 17, w_std=0.1)
+    _, _, _, cache, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, 0.5, T0, Ds)
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=0.5)
+    full = layer.prefill(q.cuda(), k.cuda(), v.cuda(), p, cnn=tuple(x.cuda() for x in cnn))
+    torch.cuda.synchronize()
+    pos = cache.pos[:, :, :window].cpu()
+    wr = cache.win_r.cpu().view(torch.int32)
+    r = full.r.cpu().view(torch.int32)
+    n_scored = int(cache.meta[1])
+    F = 3                                   # future reach of the 5- and 3-tap layers
+    checked = 0
+    for b in range(B):
+        for h in range(Hkv):
+            for sl in range(window):
+                j = int(pos[b, h, sl])
+                if T0 - F <= j < n_scored:  # scored by the decode step, not by the prompt's prefill
+                    assert int(wr[b, h, sl]) == int(r[b, h, j]), (b, h, j)
+                    checked += 1
+    assert checked >= B * Hkv * 32
