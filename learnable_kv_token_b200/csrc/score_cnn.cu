@@ -122,7 +122,10 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
     *reinterpret_cast<__nv_bfloat16*>(wlo + off) = lo;
   }
 
-  // x rows of tile `t` into registers: row r holds [k; v] of token x0 + r, 0 outside
+  score_stage_w2(p, h, wsm);                                   // once; visible after the first barrier
+
+  // x rows of tile `t` into registers: row r holds [k; v] of token x0 + r, 0 outside.
+  // The loads are volatile asm, so they are issued here, ahead of the MMAs they overlap.
   uint4 xr[kPXVec];
   auto load_x = [&](int t) {
     const int b = t / tiles_per_unit, jb = p.j_begin + (t % tiles_per_unit) * NT;
@@ -136,7 +139,9 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
         if (xg >= 0 && xg < p.T_avail) {
           const int e = c * 8;
           const __nv_bfloat16* src = e < p.D ? kv.krow(b, h, xg) + e : kv.vrow(b, h, xg) + (e - p.D);
-          val = *reinterpret_cast<const uint4*>(src);
+          asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                       : "l"(src));
         }
       }
       xr[v] = val;
@@ -208,7 +213,7 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
         const int col = nq * 40 + nt * 8 + (lane & 3) * 2 + (e & 1);
         zs[col * kPRows + row] = acc[nt][e];
       }
-    score_tail(p, zs, kPRows, us, wsm, NT, b, h, jb, j_last, p.T_avail);   // ends with a barrier
+    score_tail(p, zs, kPRows, us, wsm, NT, b, h, jb, j_last, p.T_avail);   // barriers at both ends
   }
 }
 

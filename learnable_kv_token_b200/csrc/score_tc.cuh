@@ -63,23 +63,35 @@ __device__ __forceinline__ void mma(float* c, const uint32_t* a, uint32_t b0, ui
 }
 }  // namespace stc
 
+// Layer-2 weights and layer-1 biases of head h into shared memory (wsm:
+// c_hid * (k2 + 1) floats).  Visible to the CTA after its next barrier.
+__device__ __forceinline__ void score_stage_w2(const ScoreParams& p, int h, float* wsm) {
+  const int nw2 = p.c_hid * p.k2;
+  for (int i = threadIdx.x; i < nw2; i += blockDim.x) wsm[i] = p.w2[(long long)h * nw2 + i];
+  for (int i = threadIdx.x; i < p.c_hid; i += blockDim.x) wsm[nw2 + i] = p.b1[h * p.c_hid + i];
+}
+
+constexpr int kL2Groups = 4;       // layer 2: threads per token, one channel group each
+
 // Layers 1 (tap sum, bias, SiLU) and 2 (+ sigmoid, threshold) of a tile, after
 // the GEMM, shared by every tensor-core scoring kernel so that a token's score
 // is the same instruction sequence wherever it is computed.  zs holds Z
 // transposed, [160 columns][R rows] (the tap sum then reads consecutive rows:
-// conflict-free); u gets [c_hid][NU], NU = NT + k2 - 1; wsm c_hid * (k2 + 1)
-// floats for w2 and b1 of head h.  Row r of Z is x position jb - past2 - past1 + r.
-// Writes the scores of tokens [jb, min(jb + NT, j_end)).  All threads call it.
+// conflict-free); u gets [c_hid][NU], NU = NT + k2 - 1; wsm holds w2 and b1 of
+// head h (score_stage_w2, staged before the caller's last barrier).  Row r of Z
+// is x position jb - past2 - past1 + r.  Layer 2 runs kL2Groups threads per
+// token, each summing a contiguous group of hidden channels in order; the
+// partial sums are added in a fixed tree order.  Writes the scores of tokens
+// [jb, min(jb + NT, j_end)).  All threads call it; it begins and ends with a
+// barrier.
 __device__ __forceinline__ void score_tail(const ScoreParams& p, const float* zs, int R, float* us,
-                                           float* wsm, int NT, int b, int h, int jb, int j_end,
-                                           int T_avail) {
+                                           const float* wsm, int NT, int b, int h, int jb,
+                                           int j_end, int T_avail) {
   const int tid = threadIdx.x, nthreads = blockDim.x;
   const int NU = NT + p.k2 - 1, nw2 = p.c_hid * p.k2;
-  float* w2s = wsm;
-  float* b1s = wsm + nw2;
-  for (int i = tid; i < nw2; i += nthreads) w2s[i] = p.w2[(long long)h * nw2 + i];
-  for (int i = tid; i < p.c_hid; i += nthreads) b1s[i] = p.b1[h * p.c_hid + i];
-  __syncthreads();
+  const float* w2s = wsm;
+  const float* b1s = wsm + nw2;
+  __syncthreads();                                           // Z (and wsm) are in shared memory
   // ---- u[c][q] = SiLU(b1[c] + sum_kk Z[q + kk][c*k1 + kk]); 0 outside the tokens
   const int u0 = jb - p.past2;
   for (int i = tid; i < p.c_hid * NU; i += nthreads) {
@@ -90,16 +102,24 @@ __device__ __forceinline__ void score_tail(const ScoreParams& p, const float* zs
     us[c * NU + q] = (ug >= 0 && ug < T_avail) ? siluf_(b1s[c] + z) : 0.f;
   }
   __syncthreads();
-  // ---- layer 2 + sigmoid + threshold (fp32), one thread per token
-  if (tid < NT) {
-    const int j = jb + tid;
-    if (j < j_end) {
-      float z = p.b2[h];
-      for (int c = 0; c < p.c_hid; ++c) {
-#pragma unroll 3
-        for (int kk = 0; kk < p.k2; ++kk) z = fmaf(w2s[c * p.k2 + kk], us[c * NU + tid + kk], z);
-      }
-      const float r = sigmoidf_(z);
+  // ---- layer 2 + sigmoid + threshold (fp32)
+  const int per_g = (p.c_hid + kL2Groups - 1) / kL2Groups;
+  for (int i0 = 0; i0 < NT * kL2Groups; i0 += nthreads) {    // uniform trip count (shuffles)
+    const int i = i0 + tid;
+    const int tok = i / kL2Groups, grp = i % kL2Groups;
+    const bool live = i < NT * kL2Groups;
+    float part = 0.f;
+    if (live) {
+      const int c_end = min(p.c_hid, (grp + 1) * per_g);
+      for (int c = grp * per_g; c < c_end; ++c)
+        for (int kk = 0; kk < p.k2; ++kk) part = fmaf(w2s[c * p.k2 + kk], us[c * NU + tok + kk], part);
+    }
+    // groups are lanes 4k..4k+3 of a warp: ((g0 + g1) + (g2 + g3)), the same on every lane
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    const int j = jb + tok;
+    if (live && grp == 0 && j < j_end) {
+      const float r = sigmoidf_(p.b2[h] + part);
       if (p.win_r != nullptr) {
         p.win_r[(long long)(b * p.Hkv + h) * p.window + (j % p.window)] = r;
       } else {
@@ -131,6 +151,7 @@ __device__ __forceinline__ void score_tile_tc(const ScoreParams& p, const KV& kv
   const size_t zb = (size_t)kTcRows * kTcN * 4;
   float* us = reinterpret_cast<float*>(smem + (xw > zb ? xw : zb));   // [c_hid][NU]
   float* wsm = us + p.c_hid * NU;                              // w2, b1 of head h
+  score_stage_w2(p, h, wsm);                                   // visible after the next barrier
 
   // ---- x rows [x0, x0 + 80): [k; v] of existing tokens, zero elsewhere
   const int cpr = xrow_b / 16;                                 // 16-byte chunks per row
@@ -205,7 +226,7 @@ __device__ __forceinline__ void score_tile_tc(const ScoreParams& p, const KV& kv
       const int col = nh * 80 + nt * 8 + (lane & 3) * 2 + (e & 1);
       zs[col * kTcRows + row] = acc[nt][e];
     }
-  score_tail(p, zs, kTcRows, us, wsm, kScoreNT, b, h, jb, j_end, T_avail);
+  score_tail(p, zs, kTcRows, us, wsm, kScoreNT, b, h, jb, j_end, T_avail);   // barrier first
 }
 
 }  // namespace lte
