@@ -15,7 +15,9 @@
 // (b_m = b at the chunk middle halves the exponent range of the intra-chunk
 // factors).  One CTA per (batch, head) walks the chunks in order; the fp32
 // state stays in MMA accumulator registers for the whole sequence and a bf16
-// copy in shared memory feeds the S_0 q products.  Per chunk: the decay
+// copy in shared memory feeds the S_0 q products.  The next chunk's q, k, v
+// (cp.async into the other of two shared input sets) and decay gates (into
+// registers) load while the current chunk computes.  Per chunk: the decay
 // factors (fp32 cumulative log-gates), A = Q~ K~^T masked causal (64x64),
 // O = A V + Qbar S_0^T (64x128), S <- S diag(e^{b_{L-1}}) + V^T Khat (128x128),
 // all on m16n8k16 bf16 MMAs with fp32 accumulation.
@@ -35,13 +37,14 @@ constexpr int L = 64, DK = 128, DV = 128;
 constexpr int kThreads = 256;
 
 // shared-memory layout (bytes); [rows][128] bf16 tiles have 256-byte rows with
-// the 16-byte chunks XOR-swizzled by (row mod 8)
-constexpr uint32_t kQbar = 0;                 // q * e^{b_t}          [64][128]
-constexpr uint32_t kQtil = kQbar + 16384;     // q * e^{b_t - b_m}    [64][128]
-constexpr uint32_t kKtil = kQtil + 16384;     // k * e^{b_m - b_s}    [64][128]
-constexpr uint32_t kKhat = kKtil + 16384;     // k * e^{b_last - b_s} [64][128]
-constexpr uint32_t kV = kKhat + 16384;        // v                    [64][128]
-constexpr uint32_t kA = kV + 16384;           // masked A (bf16)      [64][64], 128-byte rows
+// the 16-byte chunks XOR-swizzled by (row mod 8).  Two input sets alternate
+// between chunks: while chunk c computes from set c mod 2, the copies of chunk
+// c+1 land in the other set.  In a set, q becomes Q~ and k becomes K~ in place.
+constexpr uint32_t kSet = 3 * 16384;          // one input set: q, k, v [64][128] bf16
+constexpr uint32_t kSetQ = 0, kSetK = 16384, kSetV = 32768;
+constexpr uint32_t kQbar = 2 * kSet;          // q * e^{b_t}          [64][128]
+constexpr uint32_t kKhat = kQbar + 16384;     // k * e^{b_last - b_s} [64][128]
+constexpr uint32_t kA = kKhat + 16384;        // masked A (bf16)      [64][64], 128-byte rows
 constexpr uint32_t kSb = kA + 8192;           // state copy (bf16)    [128][128]
 constexpr uint32_t kLam = kSb + 32768;        // e^{b_last} per key channel (fp32)
 constexpr uint32_t kTot = kLam + 512;         // log-gate totals of each half (2 x 128 fp32)
@@ -133,7 +136,31 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
         sacc[mi][ni][e] = st[i * DK + j];
       }
 
-  for (int t0 = 0; t0 < T; t0 += L) {
+  // inputs of chunk t0 -> input set `set` (async copies, one commit group)
+  auto load_qkv = [&](int t0, int set) {
+    const uint32_t sb = s0 + set * kSet;
+    for (int c = tid; c < L * 16; c += kThreads) {
+      const int r = c >> 4, cc = (c & 15) * 8;
+      const long long g = base_bh + (long long)(t0 + r) * row_stride + cc;
+      cp16(sb + kSetQ + sw(r, cc, 256), q + g);
+      cp16(sb + kSetK + sw(r, cc, 256), k + g);
+      cp16(sb + kSetV + sw(r, cc, 256), v + g);
+    }
+  };
+  // decay gates of chunk t0: thread (j, half) holds 32 tokens of key channel j
+  const int j = tid & 127, half = tid >> 7;
+  float a_cur[32], a_nxt[32];
+  auto load_a = [&](int t0, float (&dst)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      dst[i] = __ldg(a + base_bh + (long long)(t0 + half * 32 + i) * row_stride + j);
+  };
+  load_qkv(0, 0);
+  asm volatile("cp.async.commit_group;\n" ::);
+  load_a(0, a_cur);
+
+  for (int t0 = 0, set = 0; t0 < T; t0 += L, set ^= 1) {
+    const uint32_t sq = kSetQ + set * kSet, sk = kSetK + set * kSet, sv = kSetV + set * kSet;
     // bf16 copy of S_0 for the Qbar S_0^T product
 #pragma unroll
     for (int mi = 0; mi < 2; ++mi)
@@ -141,34 +168,29 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
       for (int ni = 0; ni < 8; ++ni)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          const int i = sm0 + mi * 16 + gq + hf * 8, j = sn0 + ni * 8 + cq * 2;
-          *reinterpret_cast<uint32_t*>(sm + kSb + sw(i, j, 256)) =
+          const int i = sm0 + mi * 16 + gq + hf * 8, jj = sn0 + ni * 8 + cq * 2;
+          *reinterpret_cast<uint32_t*>(sm + kSb + sw(i, jj, 256)) =
               pack(sacc[mi][ni][hf * 2], sacc[mi][ni][hf * 2 + 1]);
         }
-    // raw q -> Qbar slot, k -> Khat slot, v -> V (16-byte async copies)
-    for (int c = tid; c < L * 16; c += kThreads) {
-      const int r = c >> 4, cc = (c & 15) * 8;
-      const long long g = base_bh + (long long)(t0 + r) * row_stride + cc;
-      cp16(s0 + kQbar + sw(r, cc, 256), q + g);
-      cp16(s0 + kKhat + sw(r, cc, 256), k + g);
-      cp16(s0 + kV + sw(r, cc, 256), v + g);
-    }
+    // the next chunk's inputs start loading (the other set is free: the
+    // previous chunk ended with a barrier)
+    const bool more = t0 + L < T;
+    if (more) load_qkv(t0 + L, set ^ 1);
     asm volatile("cp.async.commit_group;\n" ::);
-    // cumulative log-gates: thread (j, half) covers 32 tokens of key channel j
-    const int j = tid & 127, half = tid >> 7;
+    if (more) load_a(t0 + L, a_nxt);
+    // cumulative log-gates
     float bl[32];
     {
       float run = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int t = t0 + half * 32 + i;
-        run += __logf(a[base_bh + (long long)t * row_stride + j]);
+        run += __logf(a_cur[i]);
         bl[i] = run;
       }
       if (half == 0) tot[j] = run;           // b at the chunk middle (token 31)
       if (half == 1) tot[128 + j] = run;     // second-half total
     }
-    asm volatile("cp.async.wait_group 0;\n" ::);
+    asm volatile("cp.async.wait_group 1;\n" ::);   // this chunk's set has landed
     __syncthreads();
     {
       const float bm = tot[j];
@@ -180,15 +202,17 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
         const int r = half * 32 + i;
         const float bt = bl[i] + off;
         const uint32_t o16 = sw(r, j, 256);
-        __nv_bfloat16* pq = reinterpret_cast<__nv_bfloat16*>(sm + kQbar + o16);
-        __nv_bfloat16* pk = reinterpret_cast<__nv_bfloat16*>(sm + kKhat + o16);
+        __nv_bfloat16* pq = reinterpret_cast<__nv_bfloat16*>(sm + sq + o16);
+        __nv_bfloat16* pk = reinterpret_cast<__nv_bfloat16*>(sm + sk + o16);
         const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk);
-        *reinterpret_cast<__nv_bfloat16*>(sm + kQtil + o16) = __float2bfloat16_rn(qv * __expf(bt - bm));
-        *reinterpret_cast<__nv_bfloat16*>(sm + kKtil + o16) = __float2bfloat16_rn(kv * __expf(bm - bt));
-        *pq = __float2bfloat16_rn(qv * __expf(bt));
-        *pk = __float2bfloat16_rn(kv * __expf(blast - bt));
+        *reinterpret_cast<__nv_bfloat16*>(sm + kQbar + o16) = __float2bfloat16_rn(qv * __expf(bt));
+        *reinterpret_cast<__nv_bfloat16*>(sm + kKhat + o16) = __float2bfloat16_rn(kv * __expf(blast - bt));
+        *pq = __float2bfloat16_rn(qv * __expf(bt - bm));       // Q~ in place
+        *pk = __float2bfloat16_rn(kv * __expf(bm - bt));       // K~ in place
       }
     }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a_cur[i] = a_nxt[i];
     __syncthreads();
 
     // ---- A = Q~ K~^T (64 x 64), causal mask s <= t, bf16 -> shared
@@ -198,11 +222,11 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
 #pragma unroll
       for (int kk = 0; kk < DK; kk += 16) {
         uint32_t fa[4];
-        frag_a(s0 + kQtil, 256, am0, kk, lane, fa);
+        frag_a(s0 + sq, 256, am0, kk, lane, fa);
 #pragma unroll
         for (int np = 0; np < 2; ++np) {
           uint32_t fb[4];
-          frag_b(s0 + kKtil, 256, an0 + np * 16, kk, lane, fb);
+          frag_b(s0 + sk, 256, an0 + np * 16, kk, lane, fb);
           mma(acc[np * 2], fa, fb[0], fb[1]);
           mma(acc[np * 2 + 1], fa, fb[2], fb[3]);
         }
@@ -230,7 +254,7 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
 #pragma unroll
         for (int np = 0; np < 4; ++np) {
           uint32_t fb[4];
-          frag_b_t(s0 + kV, 256, on0 + np * 16, kk, lane, fb);
+          frag_b_t(s0 + sv, 256, on0 + np * 16, kk, lane, fb);
           mma(acc[np * 2], fa, fb[0], fb[1]);
           mma(acc[np * 2 + 1], fa, fb[2], fb[3]);
         }
@@ -271,8 +295,8 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
 #pragma unroll
     for (int kk = 0; kk < L; kk += 16) {
       uint32_t fa[2][4];
-      frag_a_t(s0 + kV, 256, sm0, kk, lane, fa[0]);
-      frag_a_t(s0 + kV, 256, sm0 + 16, kk, lane, fa[1]);
+      frag_a_t(s0 + sv, 256, sm0, kk, lane, fa[0]);
+      frag_a_t(s0 + sv, 256, sm0 + 16, kk, lane, fa[1]);
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t fb[4];
