@@ -52,8 +52,9 @@ score_cnn_tc_kernel(ScoreParams p, KV kv) {
 // bf16 hi + lo (all 2D input channels, 160 KiB at D = 128), converted once,
 // and walks that head's token tiles of all sequences: 48 x rows per tile
 // (42 scored tokens with a 5- and a 3-tap layer), 12 warps = 3 row tiles x 4
-// column quarters of 40.  A tile's x rows are loaded into registers while the
-// previous tile's MMAs run.  Every accumulator receives exactly the MMA
+// column quarters of 40.  Two buffers alternate: one holds a tile's x rows,
+// then (once the GEMM has read them) its Z; the next tile's x rows are copied
+// into the other buffer (cp.async) while this tile's MMAs run.  Every accumulator receives exactly the MMA
 // sequence of score_tile_tc (input-channel chunks of 64, steps of 16, hi then
 // lo), and the tap sum, SiLU and layer 2 are the same code path, so each score
 // is bit-identical to the decode step's.
@@ -62,13 +63,24 @@ constexpr int kPWarps = 12;
 constexpr int kPThreads = 32 * kPWarps;
 constexpr int kPXVec = 4;          // x-row 16-byte vectors per thread and tile at D <= 128
 
+// one x/Z buffer: x [48][2D] bf16, later Z [160][48] fp32
+__host__ __device__ inline size_t score_persist_buf_bytes(int D) {
+  const size_t x = (size_t)kPRows * 2 * D * 2, z = (size_t)kPRows * kTcN * 4;
+  return x > z ? x : z;
+}
 __host__ __device__ inline size_t score_persist_smem_bytes(int D, int c_hid, int k1, int k2) {
   const int NT = kPRows - (k1 + k2 - 2);
   return 2 * (size_t)kTcN * 2 * D * 2                 // W hi, lo: [2D/64 chunks][160][64] bf16
-         + (size_t)kPRows * 2 * D * 2                 // x: [48][2D] bf16
-         + (size_t)kPRows * kTcN * 4                  // Z: [160][48] fp32
+         + 2 * score_persist_buf_bytes(D)             // two x / Z buffers
          + (size_t)c_hid * (NT + k2 - 1) * 4          // u: [c_hid][NU] fp32
          + (size_t)c_hid * (k2 + 1) * 4;              // w2, b1 of the head
+}
+
+// 16-byte async copy global -> shared; src_bytes = 0 writes zeros
+__device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void ldsm2_p(uint32_t a, uint32_t& r0, uint32_t& r1) {
@@ -89,9 +101,9 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
   const size_t wchunk = (size_t)kTcN * kTcKC * 2;              // bytes of one [160][64] chunk
   uint8_t* whi = smem_p;
   uint8_t* wlo = whi + n_chunks * wchunk;
-  uint8_t* xs = wlo + n_chunks * wchunk;                       // [48][2D] bf16
-  float* zs = reinterpret_cast<float*>(xs + (size_t)kPRows * xrow_b);   // [160][48]
-  float* us = zs + kPRows * kTcN;                              // [c_hid][NU]
+  const size_t bufb = score_persist_buf_bytes(p.D);
+  uint8_t* buf0 = wlo + n_chunks * wchunk;                     // x of even tiles, then their Z
+  float* us = reinterpret_cast<float*>(buf0 + 2 * bufb);       // [c_hid][NU]
   float* wsm = us + p.c_hid * NU;                              // w2, b1 of head h
 
   const int h = blockIdx.x % p.Hkv;
@@ -124,46 +136,40 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
 
   score_stage_w2(p, h, wsm);                                   // once; visible after the first barrier
 
-  // x rows of tile `t` into registers: row r holds [k; v] of token x0 + r, 0 outside.
-  // The loads are volatile asm, so they are issued here, ahead of the MMAs they overlap.
-  uint4 xr[kPXVec];
-  auto load_x = [&](int t) {
+  // x rows of tile `t` into buffer `xs` (async): row r holds [k; v] of token
+  // x0 + r, zeros outside the tokens; one commit group per tile
+  auto load_x = [&](int t, uint8_t* xs) {
     const int b = t / tiles_per_unit, jb = p.j_begin + (t % tiles_per_unit) * NT;
     const int x0 = jb - p.past2 - p.past1;
+    const uint32_t xa = stc::sa(xs);
 #pragma unroll
     for (int v = 0; v < kPXVec; ++v) {
       const int i = tid + v * kPThreads;
-      uint4 val = make_uint4(0, 0, 0, 0);
       if (i < kPRows * cpr) {
         const int r = i / cpr, c = i % cpr, xg = x0 + r;
-        if (xg >= 0 && xg < p.T_avail) {
-          const int e = c * 8;
-          const __nv_bfloat16* src = e < p.D ? kv.krow(b, h, xg) + e : kv.vrow(b, h, xg) + (e - p.D);
-          asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                       : "l"(src));
-        }
+        const bool ok = xg >= 0 && xg < p.T_avail;
+        const int xc = ok ? xg : 0, e = c * 8;
+        const __nv_bfloat16* src = e < p.D ? kv.krow(b, h, xc) + e : kv.vrow(b, h, xc) + (e - p.D);
+        cp16_zfill(xa + sw(r, c, xrow_b), src, ok ? 16 : 0);
       }
-      xr[v] = val;
     }
-  };
-  auto store_x = [&]() {
-#pragma unroll
-    for (int v = 0; v < kPXVec; ++v) {
-      const int i = tid + v * kPThreads;
-      if (i < kPRows * cpr) *reinterpret_cast<uint4*>(xs + sw(i / cpr, i % cpr, xrow_b)) = xr[v];
-    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
   };
 
   const int mt = warp % 3, nq = warp / 3;                      // rows 16*mt, columns 40*nq
-  load_x(slot);
+  load_x(slot, buf0);
+  int par = 0;
 #pragma unroll 1
-  for (int t = slot; t < n_tiles; t += n_slots) {
+  for (int t = slot; t < n_tiles; t += n_slots, par ^= 1) {
     const int b = t / tiles_per_unit, jb = p.j_begin + (t % tiles_per_unit) * NT;
     const int j_last = min(jb + NT, p.j_end);
-    store_x();
+    uint8_t* xs = buf0 + par * bufb;                           // this tile's x, then its Z
+    float* zs = reinterpret_cast<float*>(xs);                  // [160][48]
+    // the other buffer held the previous tile's Z, which its tail has finished reading
+    if (t + n_slots < n_tiles) load_x(t + n_slots, buf0 + (par ^ 1) * bufb);
+    else asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");   // this tile's x has landed
     __syncthreads();                                           // x (and, first time, W) ready
-    if (t + n_slots < n_tiles) load_x(t + n_slots);            // lands during the MMAs below
 
     // ---- Z = X (48 x 2D) . W (2D x 160), weights split hi/lo
     float acc[5][4];
@@ -205,6 +211,7 @@ score_persist_tc_kernel(ScoreParams p, LinearKV<__nv_bfloat16> kv, int B) {
         }
       }
     }
+    __syncthreads();                                           // every warp has read x: Z replaces it
 #pragma unroll
     for (int nt = 0; nt < 5; ++nt)
 #pragma unroll
