@@ -22,9 +22,11 @@
 // for O += P V), so shared memory only feeds K and V to the tensor core.
 // Warp roles (384 threads, three warpgroups):
 //   warp 0     TMA producer: the item's Q rows into one shared buffer (freed as
-//              soon as both softmax groups copied them into TMEM), K and V
-//              into 4-slot rings (a K slot frees after its S MMAs, a V slot
-//              after its PV MMAs);
+//              soon as both softmax groups copied them into TMEM), the K and V
+//              tiles of a key tile into one stage of a 4-stage ring (one
+//              barrier per stage for both; a stage frees once the tile's PV
+//              MMAs have run -- each MMA-warp wait is costly, so the issuer
+//              waits once per key tile);
 //   warp 1     TMEM owner and MMA issuer (one elected lane), per K/V tile j:
 //              PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  The tensor pipe runs in
 //              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
@@ -78,9 +80,11 @@ __host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256
 __host__ __device__ constexpr uint32_t col_q(int x) { return x == 0 ? 384u : 448u; }  // Q
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
+// mbarriers: KF / KE = a K/V ring stage is full / free again (one per stage)
 enum {
-  B_QF = 0, B_QFREE = 1, B_QC = 2, B_KF = 4, B_VF = 8, B_KE = 12, B_VE = 16, B_SF = 20,
-  B_PF = 22, B_PVD = 24, B_OE = 26, B_FIN = 28, B_OST = 29, B_STG = 31, kNumBars = 33
+  B_QF = 0, B_QFREE = 1, B_QC = 2, B_KF = 4, B_KE = B_KF + kStages, B_SF = B_KE + kStages,
+  B_PF = B_SF + 2, B_PVD = B_PF + 2, B_OE = B_PVD + 2, B_FIN = B_OE + 2, B_OST = B_FIN + 1,
+  B_STG = B_OST + 2, kNumBars = B_STG + 2
 };
 static_assert(8 * kNumBars + 8 <= 512, "barriers, abort flag and TMEM slot fit the tail");
 
@@ -386,9 +390,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(B_QFREE), 256);
     for (int st = 0; st < kStages; ++st) {
       mbar_init(bar(B_KF + st), 1);
-      mbar_init(bar(B_VF + st), 1);
       mbar_init(bar(B_KE + st), 1);
-      mbar_init(bar(B_VE + st), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(B_QC + x), 128);
@@ -423,7 +425,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     if (warp == 0) {
       // ============================================================ TMA producer
       // (all 32 lanes run the loop and wait; one elected lane issues)
-      int g = 0, it = 0, issued_k = 0, issued_v = 0, issued_q = 0;
+      int g = 0, it = 0, issued_k = 0, issued_q = 0;
       bool ok = true;
       ItemCounts cn = load_counts(p, blockIdx.x);
       for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
@@ -452,33 +454,26 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (use >= 1 && !(ok = wwait(bar(B_KE + st), (use - 1) & 1, abort_flag, p.err, 202)))
             break;
           if (elect_one()) {
-            mbar_expect_tx(bar(B_KF + st), kKV);
+            mbar_expect_tx(bar(B_KF + st), 2 * kKV);
             for (int hf = 0; hf < 2; ++hf) {
-              if (rg == 2) tma_load_4d(kd + hf * kKVHalf, &tm_k, bar(B_KF + st), hf * 64, m.h, key0, m.b);
-              else tma_load_3d(kd + hf * kKVHalf, &tm_kc, bar(B_KF + st), hf * 64, key0, m.u);
+              if (rg == 2) {
+                tma_load_4d(kd + hf * kKVHalf, &tm_k, bar(B_KF + st), hf * 64, m.h, key0, m.b);
+                tma_load_4d(vd + hf * kKVHalf, &tm_v, bar(B_KF + st), hf * 64, m.h, key0, m.b);
+              } else {
+                tma_load_3d(kd + hf * kKVHalf, &tm_kc, bar(B_KF + st), hf * 64, key0, m.u);
+                tma_load_3d(vd + hf * kKVHalf, &tm_vc, bar(B_KF + st), hf * 64, key0, m.u);
+              }
             }
           }
           __syncwarp();
           issued_k = g + 1;
-          if (use >= 1 && !(ok = wwait(bar(B_VE + st), (use - 1) & 1, abort_flag, p.err, 203)))
-            break;
-          if (elect_one()) {
-            mbar_expect_tx(bar(B_VF + st), kKV);
-            for (int hf = 0; hf < 2; ++hf) {
-              if (rg == 2) tma_load_4d(vd + hf * kKVHalf, &tm_v, bar(B_VF + st), hf * 64, m.h, key0, m.b);
-              else tma_load_3d(vd + hf * kKVHalf, &tm_vc, bar(B_VF + st), hf * 64, key0, m.u);
-            }
-          }
-          __syncwarp();
-          issued_v = g + 1;
         }
       }
       // drain: every issued copy has landed before the CTA may exit
       if (issued_q > 0) mbar_drain(bar(B_QF), (issued_q - 1) & 1);
       for (int q = issued_k - kStages > 0 ? issued_k - kStages : 0; q < issued_k; ++q)
         mbar_drain(bar(B_KF + q % kStages), (q / kStages) & 1);
-      for (int q = issued_v - kStages > 0 ? issued_v - kStages : 0; q < issued_v; ++q)
-        mbar_drain(bar(B_VF + q % kStages), (q / kStages) & 1);
+
     } else if (warp == 1) {
       // ============================================================ MMA issuer
       // (all 32 lanes run the loop and wait; one elected lane issues)
@@ -513,9 +508,6 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int j = 0; j < m.total && ok; ++j) {
           const int g = g0 + j, st = g % kStages;
           if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
-          if (j >= 1 && !(ok = wwait(bar(B_VF + (g - 1) % kStages), ((g - 1) / kStages) & 1,
-                                     abort_flag, p.err, 214)))
-            break;
           const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
           for (int x = 0; x < 2 && ok; ++x) {
             if (j >= 1 && !(ok = issue_pv(x, g - 1, j - 1))) break;
@@ -533,23 +525,19 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             __syncwarp();
           }
           if (!ok) break;
-          if (elect_one()) {
-            mma_commit(bar(B_KE + st));
-            if (j >= 1) mma_commit(bar(B_VE + (g - 1) % kStages));
-          }
+          if (j >= 1 && elect_one()) mma_commit(bar(B_KE + (g - 1) % kStages));   // tile g-1 done
           __syncwarp();
         }
         if (!ok) break;
         // the item's last tile: PV_A, PV_B, then the epilogue signal
         const int gl = g0 + m.total - 1;
-        if (!(ok = wwait(bar(B_VF + gl % kStages), (gl / kStages) & 1, abort_flag, p.err, 214))) break;
         for (int x = 0; x < 2 && ok; ++x) {
           if (!(ok = issue_pv(x, gl, m.total - 1))) break;
           if (elect_one()) mma_commit(bar(B_PVD + x));
           __syncwarp();
         }
         if (!ok) break;
-        if (elect_one()) mma_commit(bar(B_VE + gl % kStages));
+        if (elect_one()) mma_commit(bar(B_KE + gl % kStages));
         __syncwarp();
         g0 += m.total;
       }
