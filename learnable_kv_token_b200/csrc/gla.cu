@@ -338,21 +338,46 @@ gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
   }
   float* st = state + (long long)bh * DV * DK;
   constexpr int kRows = DV / 8;                       // rows per warp
-#pragma unroll 4
+  // every row's loads first (16 x 512 B in flight per warp), then update and store
+  float4 s4[kRows];
+  float vi[kRows];
+#pragma unroll
   for (int rr = 0; rr < kRows; ++rr) {
     const int i = warp * kRows + rr;
-    float4* p = reinterpret_cast<float4*>(st + (long long)i * DK) + lane;
-    float4 s4 = *p;
-    const float vi = to_f32(v[(long long)bh * DV + i]);
-    s4.x = fmaf(s4.x, a4[0], vi * k4[0]);
-    s4.y = fmaf(s4.y, a4[1], vi * k4[1]);
-    s4.z = fmaf(s4.z, a4[2], vi * k4[2]);
-    s4.w = fmaf(s4.w, a4[3], vi * k4[3]);
-    *p = s4;
-    float d = s4.x * q4[0] + s4.y * q4[1] + s4.z * q4[2] + s4.w * q4[3];
+    s4[rr] = reinterpret_cast<const float4*>(st + (long long)i * DK)[lane];
+    vi[rr] = to_f32(v[(long long)bh * DV + i]);
+  }
+  float d[kRows];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-    if (lane == 0) o[(long long)bh * DV + i] = from_f32<TIn>(d);
+  for (int rr = 0; rr < kRows; ++rr) {
+    const int i = warp * kRows + rr;
+    float4 x = s4[rr];
+    x.x = fmaf(x.x, a4[0], vi[rr] * k4[0]);
+    x.y = fmaf(x.y, a4[1], vi[rr] * k4[1]);
+    x.z = fmaf(x.z, a4[2], vi[rr] * k4[2]);
+    x.w = fmaf(x.w, a4[3], vi[rr] * k4[3]);
+    reinterpret_cast<float4*>(st + (long long)i * DK)[lane] = x;
+    d[rr] = x.x * q4[0] + x.y * q4[1] + x.z * q4[2] + x.w * q4[3];
+  }
+  // the 16 row sums across the 32 lanes: at each step a lane keeps half of its
+  // values and adds its partner's copy of them (lanes paired over bit 4, 3, 2,
+  // 1, then 0 -- the same pairing tree as a plain butterfly per row)
+#pragma unroll
+  for (int half = kRows / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int jj = 0; jj < half; ++jj) {
+      const float send = upper ? d[jj] : d[jj + half];
+      const float keep = upper ? d[jj + half] : d[jj];
+      d[jj] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+    }
+  }
+  d[0] += __shfl_xor_sync(0xffffffffu, d[0], 1);
+  // lane -> row: bits 4, 3, 2, 1 of the lane select the row's bits 3, 2, 1, 0
+  if ((lane & 1) == 0) {
+    const int row = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                    ((lane >> 1) & 1);
+    o[(long long)bh * DV + warp * kRows + row] = from_f32<TIn>(d[0]);
   }
 }
 
