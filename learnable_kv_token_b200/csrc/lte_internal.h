@@ -15,6 +15,12 @@ cudaError_t score_linear(const lte_dims* d, const lte_cnn* cnn, const void* k, c
                          Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
                          cudaStream_t stream);
 
+// score_tcgen05.cu
+bool score_tcgen05_supported(const lte_dims* d, const lte_cnn* cnn, Strides4 s);
+cudaError_t score_tcgen05(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
+                          Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
+                          cudaStream_t stream);
+
 // evict_compact.cu
 cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,
                           int32_t* idx, int32_t* nret, int32_t* cnt, const void* k,

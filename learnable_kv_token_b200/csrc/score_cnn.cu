@@ -292,6 +292,8 @@ cudaError_t score_linear(const lte_dims* d, const lte_cnn* cnn, const void* k, c
   const int tiles = (j_end - j_begin + kScoreNT - 1) / kScoreNT;
   if (tiles == 0) return cudaSuccess;
   if (d->dtype == LTE_BF16) {
+    if (score_tcgen05_supported(d, cnn, s))
+      return score_tcgen05(d, cnn, k, v, s, j_begin, j_end, r, mask, stream);
     const LinearKV<__nv_bfloat16> kv{(const __nv_bfloat16*)k, (const __nv_bfloat16*)v, s};
     if (persist_supported(d, cnn)) return launch_persist(p, kv, d->B, stream);
     if (score_tc_supported(cnn->c_hid, cnn->k1, cnn->k2)) return launch_tc(p, kv, d->B, tiles, stream);

@@ -8,8 +8,8 @@ import torch
 
 import lte_inputs as LI
 from oracle import lte_oracle as O
-from tests.gpu_util import (MASK_BAND, assert_attention_close, clean_tau, f64, oracle_cnn,
-                            scale_of)
+from tests.gpu_util import (MASK_BAND, R_TOL, assert_attention_close, clean_tau, f64,
+                            oracle_cnn, scale_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -206,9 +206,10 @@ def test_decode_full_size_sampled(layer):
     assert compared >= len(rets)
 
 
-def test_decode_scores_equal_lte_score_bitwise(layer):
-    """The decode step's deferred scores (the tensor-core tile inside the step)
-    equal lte_score's (the persistent kernel) bit for bit, token by token."""
+def test_decode_scores_match_lte_score(layer):
+    """The decode step's deferred scores (the warp-MMA tile inside the step)
+    and lte_score's (the tcgen05 kernel) are the same function of the same
+    tokens: each within R_TOL of the oracle's score, token by token."""
     B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = 2, 8, 2, 128, 4, 96, 20, 150, 120, 16
     T = T0 + steps
     q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 17, w_std=0.1)
@@ -217,16 +218,18 @@ def test_decode_scores_equal_lte_score_bitwise(layer):
     full = layer.prefill(q.cuda(), k.cuda(), v.cuda(), p, cnn=tuple(x.cuda() for x in cnn))
     torch.cuda.synchronize()
     pos = cache.pos[:, :, :window].cpu()
-    wr = cache.win_r.cpu().view(torch.int32)
-    r = full.r.cpu().view(torch.int32)
+    wr = f64(cache.win_r)
+    r = f64(full.r)
     n_scored = int(cache.meta[1])
     F = 3                                   # future reach of the 5- and 3-tap layers
     checked = 0
     for b in range(B):
         for h in range(Hkv):
+            ro = O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h))
             for sl in range(window):
                 j = int(pos[b, h, sl])
                 if T0 - F <= j < n_scored:  # scored by the decode step, not by the prompt's prefill
-                    assert int(wr[b, h, sl]) == int(r[b, h, j]), (b, h, j)
+                    assert abs(wr[b, h, sl] - ro[j]) <= R_TOL, (b, h, j)
+                    assert abs(r[b, h, j] - ro[j]) <= R_TOL, (b, h, j)
                     checked += 1
     assert checked >= B * Hkv * 32

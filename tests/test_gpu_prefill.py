@@ -86,6 +86,46 @@ def test_score_causal_variant(L):
             np.testing.assert_allclose(f64(r[b, h]), ro, atol=R_TOL, rtol=0)
 
 
+@pytest.mark.parametrize("B,T,Hkv,D,c_hid,past1,past2", [
+    (3, 1500, 2, 64, 32, 2, 1),       # head dim 64, several sequences and heads
+    (2, 1000, 4, 128, 20, 4, 2),      # fewer hidden channels than columns per tap; causal taps
+    (1, 40, 1, 128, 32, 2, 1),        # a sequence shorter than one tile
+])
+def test_score_tensor_core_shapes(L, B, T, Hkv, D, c_hid, past1, past2):
+    """bf16 scores from the tcgen05 scorer, with k and v strided views into one
+    packed [B, T, Hkv, 2, D] tensor, against the oracle; a split launch gives
+    the same values bit for bit."""
+    g = LI.generator(23)
+    kv = (torch.randn(B, T, Hkv, 2, D, generator=g) / math.sqrt(D)).to(torch.bfloat16)
+    k, v = kv[:, :, :, 0], kv[:, :, :, 1]
+    w1, _, w2, _ = LI.cnn_weights(Hkv, D, c_hid, 5, 3, g, 0.05)
+    cnn = (w1, 0.1 * torch.randn(Hkv, c_hid, generator=g), w2, 0.1 * torch.randn(Hkv, generator=g))
+    kvd = kv.cuda()
+    kd, vd = kvd[:, :, :, 0], kvd[:, :, :, 1]
+    cd = _dev(*cnn)
+    dims = L.make_dims(B, T, Hkv, Hkv, D, 4, 64, 32, 0.5, 1.0 / math.sqrt(D), torch.bfloat16)
+    c, _keep = L.make_cnn(*cd, past1, past2)
+    F = (5 - 1 - past1) + (3 - 1 - past2)
+    n = T - F
+    r = torch.full((B, Hkv, T), float("nan"), device="cuda")
+    m = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+    L.lte_score(dims, c, kd, vd, 0, n, r, m)
+    cut = min(n, 233)
+    r2 = torch.full_like(r, float("nan"))
+    L.lte_score(dims, c, kd, vd, 0, cut, r2)
+    L.lte_score(dims, c, kd, vd, cut, n, r2)
+    torch.cuda.synchronize()
+    assert torch.equal(r[..., :n], r2[..., :n])
+    assert torch.isnan(r[..., n:]).all()
+    for b in range(B):
+        for h in range(Hkv):
+            ro = O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h, past1, past2))
+            np.testing.assert_allclose(f64(r[b, h])[:n], ro[:n], atol=R_TOL, rtol=0)
+            clear = np.abs(ro[:n] - 0.5) > MASK_BAND
+            mo = O.retention_mask(ro, 4, 0.5)
+            np.testing.assert_array_equal(m[b, h].cpu().numpy()[:n][clear], mo[:n][clear])
+
+
 # --------------------------------------------------------------------------- compaction
 @pytest.mark.parametrize("T,sink,p,n_scored", [(1000, 4, 0.1, 1000), (3001, 0, 0.5, 2990),
                                                (77, 4, 1.0, 77), (64, 2, 0.0, 64), (3, 4, 1.0, 3),
