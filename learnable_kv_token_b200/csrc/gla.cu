@@ -9,18 +9,23 @@
 // Contextualized Learnable Token Eviction" (TL;DR, Abstract).
 //
 // Prefill, chunk-wise (L = 64 tokens).  With b_t = sum_{i<=t} log a_i over
-// the chunk (per key channel) and S_0 the state before the chunk:
-//   o_t  = S_0 (q_t * e^{b_t}) + sum_{s<=t} [(q_t * e^{b_t-b_m}) . (k_s * e^{b_m-b_s})] v_s
-//   S_L  = S_0 diag(e^{b_{L-1}}) + sum_s v_s (k_s * e^{b_{L-1}-b_s})^T
-// (b_m = b at the chunk middle halves the exponent range of the intra-chunk
-// factors).  One CTA per (batch, head) walks the chunks in order; the fp32
-// state stays in MMA accumulator registers for the whole sequence and a bf16
-// copy in shared memory feeds the S_0 q products.  The next chunk's q, k, v
-// (cp.async into the other of two shared input sets) and decay gates (into
-// registers) load while the current chunk computes.  Per chunk: the decay
-// factors (fp32 cumulative log-gates), A = Q~ K~^T masked causal (64x64),
-// O = A V + Qbar S_0^T (64x128), S <- S diag(e^{b_{L-1}}) + V^T Khat (128x128),
-// all on m16n8k16 bf16 MMAs with fp32 accumulation.
+// the chunk (per key channel), m = 31 the chunk middle, S_0 the state before
+// the chunk, Q~_t = q_t * e^{b_t-b_m} and K~_s = k_s * e^{b_m-b_s}:
+//   o_t  = (S_0 diag(e^{b_m})) Q~_t + sum_{s<=t} (Q~_t . K~_s) v_s
+//   S_L  = (S_0 diag(e^{b_m}) + sum_s v_s K~_s^T) diag(e^{b_{L-1}-b_m})
+// (expanding the products gives the recurrence's S_0 diag(e^{b_{L-1}}) +
+// sum_s v_s (k_s * e^{b_{L-1}-b_s})^T and S_0 (q_t * e^{b_t}); the middle
+// reference halves the range of the intra-chunk factors).  The factors are
+// running products of the gates (of a within the second half, of 1/a
+// backwards through the first), so no logarithm or exponential is evaluated.
+// One CTA per (batch, head) walks the chunks in order; the fp32 state stays
+// in MMA accumulator registers for the whole sequence and a bf16 copy of
+// S_0 diag(e^{b_m}) in shared memory feeds the Q~ products.  The next chunk's
+// q, k, v (cp.async into the other of two shared input sets) and gates (into
+// registers) load while the current chunk computes.  Per chunk: Q~ and K~
+// (in place), A = Q~ K~^T masked causal (64x64), O = A V + Q~ (S_0
+// diag(e^{b_m}))^T (64x128), the state update (128x128), all on m16n8k16
+// bf16 MMAs with fp32 accumulation.
 //
 // Decode: one CTA per (batch, head) streams the 128x128 fp32 state once
 // (read, decay, add the outer product, write) with 16-byte accesses and
@@ -39,16 +44,15 @@ constexpr int kThreads = 256;
 // shared-memory layout (bytes); [rows][128] bf16 tiles have 256-byte rows with
 // the 16-byte chunks XOR-swizzled by (row mod 8).  Two input sets alternate
 // between chunks: while chunk c computes from set c mod 2, the copies of chunk
-// c+1 land in the other set.  In a set, q becomes Q~ and k becomes K~ in place.
-constexpr uint32_t kSet = 3 * 16384;          // one input set: q, k, v [64][128] bf16
-constexpr uint32_t kSetQ = 0, kSetK = 16384, kSetV = 32768;
-constexpr uint32_t kQbar = 2 * kSet;          // q * e^{b_t}          [64][128]
-constexpr uint32_t kKhat = kQbar + 16384;     // k * e^{b_last - b_s} [64][128]
-constexpr uint32_t kA = kKhat + 16384;        // masked A (bf16)      [64][64], 128-byte rows
-constexpr uint32_t kSb = kA + 8192;           // state copy (bf16)    [128][128]
-constexpr uint32_t kLam = kSb + 32768;        // e^{b_last} per key channel (fp32)
-constexpr uint32_t kTot = kLam + 512;         // log-gate totals of each half (2 x 128 fp32)
-constexpr uint32_t kSmem = kTot + 2 * 128 * 4;
+// c+1 land in the other set.  In a set, q becomes Q~, k becomes K~ and the
+// gates a become the decay factors x_t, all in place.
+constexpr uint32_t kSet = 3 * 16384 + L * DK * 4;   // one input set: q, k, v [64][128] bf16, a [64][128] fp32
+constexpr uint32_t kSetQ = 0, kSetK = 16384, kSetV = 32768, kSetA = 49152;
+constexpr uint32_t kA = 2 * kSet;             // masked A (bf16)      [64][64], 128-byte rows
+constexpr uint32_t kSb = kA + 8192;           // S_0 diag(e^{b_m}) (bf16) [128][128]
+constexpr uint32_t kLamM = kSb + 32768;       // e^{b_m} per key channel (fp32)
+constexpr uint32_t kLamR = kLamM + 512;       // e^{b_last - b_m} per key channel (fp32)
+constexpr uint32_t kSmem = kLamR + 512;
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -77,6 +81,13 @@ __device__ __forceinline__ void mma(float* c, const uint32_t* a, uint32_t b0, ui
 __device__ __forceinline__ uint32_t pack(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// 1/x by the special-function unit (rcp.approx: within 1 ulp, far below the
+// bf16 rounding the decay factors feed into)
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
@@ -117,8 +128,8 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = lane & 3;               // accumulator row / column pair
   const uint32_t s0 = saddr(sm);
-  float* lam = reinterpret_cast<float*>(sm + kLam);
-  float* tot = reinterpret_cast<float*>(sm + kTot);
+  float* lam_m = reinterpret_cast<float*>(sm + kLamM);
+  float* lam_r = reinterpret_cast<float*>(sm + kLamR);
   const long long row_stride = (long long)H * DK;        // elements between tokens
   const long long base_bh = (long long)b * T * row_stride + (long long)hd * DK;
 
@@ -146,74 +157,107 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
       cp16(sb + kSetK + sw(r, cc, 256), k + g);
       cp16(sb + kSetV + sw(r, cc, 256), v + g);
     }
+    for (int c = tid; c < L * 32; c += kThreads) {       // gates: plain [64][128] fp32 rows
+      const int r = c >> 5, cc = (c & 31) * 4;
+      cp16(sb + kSetA + (r * DK + cc) * 4, a + base_bh + (long long)(t0 + r) * row_stride + cc);
+    }
   };
-  // decay gates of chunk t0: thread (j, half) holds 32 tokens of key channel j
+  // gate math: thread (j, half) walks 32 tokens of key channel j
   const int j = tid & 127, half = tid >> 7;
-  float a_cur[32], a_nxt[32];
-  auto load_a = [&](int t0, float (&dst)[32]) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      dst[i] = __ldg(a + base_bh + (long long)(t0 + half * 32 + i) * row_stride + j);
-  };
   load_qkv(0, 0);
   asm volatile("cp.async.commit_group;\n" ::);
-  load_a(0, a_cur);
 
   for (int t0 = 0, set = 0; t0 < T; t0 += L, set ^= 1) {
     const uint32_t sq = kSetQ + set * kSet, sk = kSetK + set * kSet, sv = kSetV + set * kSet;
-    // bf16 copy of S_0 for the Qbar S_0^T product
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-      for (int ni = 0; ni < 8; ++ni)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int i = sm0 + mi * 16 + gq + hf * 8, jj = sn0 + ni * 8 + cq * 2;
-          *reinterpret_cast<uint32_t*>(sm + kSb + sw(i, jj, 256)) =
-              pack(sacc[mi][ni][hf * 2], sacc[mi][ni][hf * 2 + 1]);
-        }
     // the next chunk's inputs start loading (the other set is free: the
     // previous chunk ended with a barrier)
-    const bool more = t0 + L < T;
-    if (more) load_qkv(t0 + L, set ^ 1);
+    if (t0 + L < T) load_qkv(t0 + L, set ^ 1);
     asm volatile("cp.async.commit_group;\n" ::);
-    if (more) load_a(t0 + L, a_nxt);
-    // cumulative log-gates
-    float bl[32];
-    {
-      float run = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        run += __logf(a_cur[i]);
-        bl[i] = run;
-      }
-      if (half == 0) tot[j] = run;           // b at the chunk middle (token 31)
-      if (half == 1) tot[128 + j] = run;     // second-half total
-    }
     asm volatile("cp.async.wait_group 1;\n" ::);   // this chunk's set has landed
     __syncthreads();
+    // ---- decay factors x_t = e^{b_t - b_m}, written over the gates (the
+    // thread reads a_i before it writes x_i).  First half (warps 0-3): the
+    // product of 1/a_i over t < i <= m, built backwards from the middle;
+    // second half (warps 4-7): the product of a_i over m < i <= t.
+    float* X = reinterpret_cast<float*>(sm + kSetA + set * kSet);   // [64][128]
     {
-      const float bm = tot[j];
-      const float blast = tot[j] + tot[128 + j];
-      if (half == 0) lam[j] = __expf(blast);
-      const float off = half ? bm : 0.f;
+      float* Xj = X + half * 32 * DK + j;        // column j of this thread's 32 rows
+      float g[32];                               // this thread's 32 gates, then factors
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = half * 32 + i;
-        const float bt = bl[i] + off;
-        const uint32_t o16 = sw(r, j, 256);
-        __nv_bfloat16* pq = reinterpret_cast<__nv_bfloat16*>(sm + sq + o16);
-        __nv_bfloat16* pk = reinterpret_cast<__nv_bfloat16*>(sm + sk + o16);
-        const float qv = __bfloat162float(*pq), kv = __bfloat162float(*pk);
-        *reinterpret_cast<__nv_bfloat16*>(sm + kQbar + o16) = __float2bfloat16_rn(qv * __expf(bt));
-        *reinterpret_cast<__nv_bfloat16*>(sm + kKhat + o16) = __float2bfloat16_rn(kv * __expf(blast - bt));
-        *pq = __float2bfloat16_rn(qv * __expf(bt - bm));       // Q~ in place
-        *pk = __float2bfloat16_rn(kv * __expf(bm - bt));       // K~ in place
+      for (int i = 0; i < 32; ++i) g[i] = Xj[i * DK];
+      float pa = 1.f;                            // running product of a
+      if (half == 0) {
+        float pr = 1.f;                          // running product of 1/a
+#pragma unroll
+        for (int i = 31; i >= 0; --i) {
+          const float ai = g[i];
+          g[i] = pr;
+          pr *= rcp_approx(ai);
+          pa *= ai;
+        }
+        lam_m[j] = pa;                           // e^{b_m}: product of a over the first half
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          pa *= g[i];
+          g[i] = pa;
+        }
+        lam_r[j] = pa;                           // e^{b_last - b_m}
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Xj[i * DK] = g[i];
+    }
+    __syncthreads();
+    // ---- Q~ = q x_t and K~ = k / x_t in place, 8 channels (16 bytes) per access
+    {
+      constexpr int kItems = L * 16 / kThreads;  // (row, 16-byte group) pairs per thread
+      uint4 qv[kItems], kv[kItems];
+      float4 x0[kItems], x1[kItems];
+#pragma unroll
+      for (int it = 0; it < kItems; ++it) {
+        const int c = tid + it * kThreads, r = c >> 4, g = (c & 15) * 8;
+        const uint32_t o16 = sw(r, g, 256);
+        qv[it] = *reinterpret_cast<const uint4*>(sm + sq + o16);
+        kv[it] = *reinterpret_cast<const uint4*>(sm + sk + o16);
+        x0[it] = *reinterpret_cast<const float4*>(X + r * DK + g);
+        x1[it] = *reinterpret_cast<const float4*>(X + r * DK + g + 4);
+      }
+#pragma unroll
+      for (int it = 0; it < kItems; ++it) {
+        const int c = tid + it * kThreads, r = c >> 4, g = (c & 15) * 8;
+        const uint32_t o16 = sw(r, g, 256);
+        const float xs[8] = {x0[it].x, x0[it].y, x0[it].z, x0[it].w,
+                             x1[it].x, x1[it].y, x1[it].z, x1[it].w};
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv[it]);
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv[it]);
+        uint32_t qo[4], ko[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(&qw[e]);
+          const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(&kw[e]);
+          const float xa = xs[2 * e], xb = xs[2 * e + 1];
+          qo[e] = pack(__low2float(q2) * xa, __high2float(q2) * xb);
+          ko[e] = pack(__low2float(k2) * rcp_approx(xa), __high2float(k2) * rcp_approx(xb));
+        }
+        *reinterpret_cast<uint4*>(sm + sq + o16) = make_uint4(qo[0], qo[1], qo[2], qo[3]);
+        *reinterpret_cast<uint4*>(sm + sk + o16) = make_uint4(ko[0], ko[1], ko[2], ko[3]);
       }
     }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) a_cur[i] = a_nxt[i];
     __syncthreads();
+    // bf16 copy of S_0 diag(e^{b_m}) for the O product
+#pragma unroll
+    for (int ni = 0; ni < 8; ++ni) {
+      const int jj = sn0 + ni * 8 + cq * 2;
+      const float m0 = lam_m[jj], m1 = lam_m[jj + 1];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int i = sm0 + mi * 16 + gq + hf * 8;
+          *reinterpret_cast<uint32_t*>(sm + kSb + sw(i, jj, 256)) =
+              pack(sacc[mi][ni][hf * 2] * m0, sacc[mi][ni][hf * 2 + 1] * m1);
+        }
+    }
 
     // ---- A = Q~ K~^T (64 x 64), causal mask s <= t, bf16 -> shared
     {
@@ -243,7 +287,7 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
     }
     __syncthreads();
 
-    // ---- O = A V + Qbar S_0^T (64 x 128) -> bf16 output
+    // ---- O = A V + Q~ (S_0 diag(e^{b_m}))^T (64 x 128) -> bf16 output
     {
       const int om0 = (warp & 3) * 16, on0 = (warp >> 2) * 64;
       float acc[8][4] = {};
@@ -262,7 +306,7 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
 #pragma unroll
       for (int kk = 0; kk < DK; kk += 16) {
         uint32_t fa[4];
-        frag_a(s0 + kQbar, 256, om0, kk, lane, fa);
+        frag_a(s0 + sq, 256, om0, kk, lane, fa);
 #pragma unroll
         for (int np = 0; np < 4; ++np) {
           uint32_t fb[4];
@@ -281,17 +325,20 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
         }
     }
 
-    // ---- S <- S diag(e^{b_last}) + V^T Khat  (128 x 128, K = 64 tokens)
+    // ---- S <- (S diag(e^{b_m}) + V^T K~) diag(e^{b_last - b_m})  (128 x 128, K = 64 tokens)
+    auto scale_cols = [&](const float* f) {
 #pragma unroll
-    for (int ni = 0; ni < 8; ++ni) {
-      const int jj = sn0 + ni * 8 + cq * 2;
-      const float l0 = lam[jj], l1 = lam[jj + 1];
+      for (int ni = 0; ni < 8; ++ni) {
+        const int jj = sn0 + ni * 8 + cq * 2;
+        const float l0 = f[jj], l1 = f[jj + 1];
 #pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        sacc[mi][ni][0] *= l0; sacc[mi][ni][1] *= l1;
-        sacc[mi][ni][2] *= l0; sacc[mi][ni][3] *= l1;
+        for (int mi = 0; mi < 2; ++mi) {
+          sacc[mi][ni][0] *= l0; sacc[mi][ni][1] *= l1;
+          sacc[mi][ni][2] *= l0; sacc[mi][ni][3] *= l1;
+        }
       }
-    }
+    };
+    scale_cols(lam_m);
 #pragma unroll
     for (int kk = 0; kk < L; kk += 16) {
       uint32_t fa[2][4];
@@ -300,7 +347,7 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t fb[4];
-        frag_b_t(s0 + kKhat, 256, sn0 + np * 16, kk, lane, fb);
+        frag_b_t(s0 + sk, 256, sn0 + np * 16, kk, lane, fb);
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
           mma(sacc[mi][np * 2], fa[mi], fb[0], fb[1]);
@@ -308,6 +355,7 @@ gla_prefill_kernel(int T, int H, const __nv_bfloat16* __restrict__ q,
         }
       }
     }
+    scale_cols(lam_r);
     __syncthreads();   // every warp is done with this chunk's tiles and S_0 copy
   }
 #pragma unroll
