@@ -141,3 +141,73 @@ class Decoder:
         L.lte_decode_step(self.dims, self.cnn, self.cache.struct, q_t, k_t, v_t, self.o, self.lse,
                           self.score_batch, self.ws, stream)
         return self.o, self.lse
+
+
+class HostPrefill:
+    """Prefill of a batch that lives in pinned host memory, streamed through
+    the device in sub-batches of `chunk` sequences.
+
+    Two device slots alternate.  Sub-batch c is copied in on one stream, computed
+    (lte_evict_compact with a fed mask, then lte_sparse_attn_prefill) on a
+    second and copied out on a third, so the input copy of c + 1 and the output
+    copy of c - 1 overlap the compute of c, and the two copy directions overlap
+    each other.  The copies are the only work outside the library's kernels."""
+
+    def __init__(self, B, T, Hq, Hkv, D, dtype, p: LayerParams, chunk, device="cuda"):
+        if B % chunk:
+            raise ValueError("the batch must be a multiple of the sub-batch")
+        dev = torch.device(device)
+        self.B, self.T, self.chunk, self.p = B, T, chunk, p
+        self.dims = p.dims(chunk, T, Hq, Hkv, D, dtype)
+        self.slots = []
+        for _ in range(2):
+            self.slots.append(dict(
+                q=torch.empty(chunk, T, Hq, D, dtype=dtype, device=dev),
+                k=torch.empty(chunk, T, Hkv, D, dtype=dtype, device=dev),
+                v=torch.empty(chunk, T, Hkv, D, dtype=dtype, device=dev),
+                mask=torch.empty(chunk, Hkv, T, dtype=torch.uint8, device=dev),
+                bufs=PrefillBuffers(chunk, T, Hq, Hkv, D, dtype, p.sink, self.dims, dev, want_r=False)))
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.in_done, self.comp_done, self.out_done = ev(), ev(), ev()
+
+    def run(self, hq, hk, hv, hmask, ho, stream=None):
+        """hq, hk, hv [B,T,H,D], hmask [B,Hkv,T] uint8 and ho [B,T,Hq,D]: pinned host
+        tensors.  Work is ordered after `stream` (default: the current stream),
+        which in turn waits for the last output copy."""
+        stream = torch.cuda.current_stream() if stream is None else stream
+        start = torch.cuda.Event()
+        start.record(stream)
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.wait_event(start)
+        n = self.B // self.chunk
+        for c in range(n):
+            s, sl = c % 2, self.slots[c % 2]
+            b0, b1 = c * self.chunk, (c + 1) * self.chunk
+            if c >= 2:
+                self.s_in.wait_event(self.comp_done[s])       # the slot's inputs have been read
+            with torch.cuda.stream(self.s_in):
+                sl["q"].copy_(hq[b0:b1], non_blocking=True)
+                sl["k"].copy_(hk[b0:b1], non_blocking=True)
+                sl["v"].copy_(hv[b0:b1], non_blocking=True)
+                sl["mask"].copy_(hmask[b0:b1], non_blocking=True)
+            self.in_done[s].record(self.s_in)
+            self.s_comp.wait_event(self.in_done[s])
+            if c >= 2:
+                self.s_comp.wait_event(self.out_done[s])      # the slot's o has been copied out
+            bufs = sl["bufs"]
+            L.lte_evict_compact(self.dims, None, sl["mask"], self.T, bufs.idx, bufs.nret, bufs.cnt,
+                                sl["k"], sl["v"], bufs.k_col, bufs.v_col, self.s_comp)
+            L.lte_sparse_attn_prefill(self.dims, sl["q"], sl["k"], sl["v"], bufs.cnt, bufs.k_col,
+                                      bufs.v_col, bufs.o, bufs.lse, bufs.ws, self.s_comp)
+            self.comp_done[s].record(self.s_comp)
+            self.s_out.wait_event(self.comp_done[s])
+            with torch.cuda.stream(self.s_out):
+                ho[b0:b1].copy_(bufs.o, non_blocking=True)
+            self.out_done[s].record(self.s_out)
+        stream.wait_stream(self.s_out)
+        stream.wait_stream(self.s_comp)
+        stream.wait_stream(self.s_in)
+
+    def device_errors(self):
+        return [L.lte_read_device_error(sl["bufs"].ws) for sl in self.slots]
