@@ -148,7 +148,7 @@ def traffic_from_profiles(kernel_file, launch_units):
     with open(path) as f:
         tr = json.load(f)
     ent = tr.get(kernel_file)
-    if not ent or ent.get("source_hash") != source_hash(kernel_file):
+    if not ent or ent.get("source_hash") != source_hash(*ent.get("sources", [kernel_file])):
         return None
     return ent["dram_bytes_per_unit"] * launch_units
 
@@ -374,6 +374,8 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
     from learnable_kv_token_b200 import layer
     from learnable_kv_token_b200 import lte as L
     wl = LI.WORKLOADS["hybrid"]
+    if args.batch:                                  # smaller case for profiler captures
+        wl = wl.with_(B=args.batch)
     B, T, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
     seed = DI.shard_seed(wl.seed, rank)
     inp = LI.lte_inputs(wl.with_(seed=seed), T=T)
@@ -442,7 +444,7 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
 
     lte_prefill_ms = t_score + t_compact + t_attn
     return {
-        "workload": "hybrid B=32 T=4096 (prompt) Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512, CNN "
+        "workload": f"hybrid B={B} T=4096 (prompt) Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512, CNN "
                     "32ch k5/k3 scored live, tau 0.5; GLA 16 heads dk=dv=128, chunk 64",
         "a1_score_ms": t_score, "a1_roofline": tensor(score_flops, t_score),
         "a1_bytes_rate": hbm(score_bytes, t_score),
@@ -472,7 +474,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle CPU sample length (0 skips the cpu_baseline leg)")
     ap.add_argument("--batch", type=int, default=0,
-                    help="prefill batch override for profiler captures (default: the workload's)")
+                    help="batch override of the prefill and per-row workloads, for profiler "
+                         "captures (default: the workloads')")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
