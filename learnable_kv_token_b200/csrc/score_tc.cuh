@@ -12,7 +12,8 @@
 // (relative weight error ~2^-17).  Layer 2 (c_hid -> 1, k2 taps) and the
 // sigmoid run in fp32.  Every value is produced by a fixed sequence of
 // instructions independent of where its token falls in the tile, so a
-// token's score is bit-identical in lte_score and in the decode step.
+// token's score does not depend on the tile or the addressing mode (the
+// decode step's ring or a [B,T,H,D] tensor).
 //
 // CTA: 320 threads (10 warps = 5 row tiles of 16 x 2 column halves of 80);
 // a tile covers kScoreNT = 64 output tokens (NX = 64 + k1 + k2 - 2 <= 80 rows
