@@ -6,7 +6,11 @@ by one.
   retention mask Bernoulli(0.1) fed;
 * long-context sweep: B=4, T=16384, w=1024, C in {0, 1024, 4096, 16384} x
   per-head retention rates ~ U[0, 2*rate] clipped, rate in {0, 5, 25, 100} %
-  (rate 100 % with C = 16384 is full causal attention).
+  (rate 100 % with C = 16384 is full causal attention);
+* laLTE hybrid pair: B=32 x 4096-token prompts, the CNN scored live (sampled
+  units against the oracle's scores), and the gated linear-attention layer
+  (16 heads, dk = dv = 128) through prefill and 256 decode steps (sampled
+  heads against the oracle's recurrence).
 Rows are sampled at the window / sink / cap boundaries, the ragged end, and
 uniformly in between."""
 import numpy as np
@@ -73,3 +77,64 @@ def test_sweep_sampled(layer, sweep_inputs, cap, rate):
     torch.cuda.synchronize()
     rng = np.random.default_rng(cap + int(rate * 1000))
     _check(q, k, v, mask, out, [(0, 0), (3, 3)], wl.sink, wl.window, cap, rng)
+
+
+# --------------------------------------------------------------------------- laLTE hybrid pair
+def test_hybrid_scores_sampled():
+    """lte_score at the hybrid workload's size (B=32, 4096-token prompts, Hkv=4,
+    D=128, the CNN live): sampled units against the oracle's scores, masks exact
+    off the band around tau."""
+    from learnable_kv_token_b200 import lte as L
+    from oracle import lte_oracle as O
+    from tests.gpu_util import MASK_BAND, R_TOL, oracle_cnn
+    wl = LI.WORKLOADS["hybrid"]
+    inp = LI.lte_inputs(wl, T=wl.T)
+    k, v, cnn = inp["k"], inp["v"], inp["cnn"]
+    B, T, Hkv = wl.B, wl.T, wl.Hkv
+    dims = L.make_dims(B, T, wl.Hq, Hkv, wl.D, wl.sink, wl.window, wl.cap, wl.tau, scale_of(wl.D),
+                       wl.dtype)
+    c, _keep = L.make_cnn(*(x.cuda() for x in cnn), wl.past1, wl.past2)
+    n = T - 3
+    r = torch.full((B, Hkv, T), float("nan"), device="cuda")
+    m = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
+    L.lte_score(dims, c, k.cuda(), v.cuda(), 0, n, r, m)
+    torch.cuda.synchronize()
+    assert torch.isfinite(r[..., :n]).all()
+    for b, h in [(0, 0), (7, 2), (19, 1), (31, 3)]:
+        ro = O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h, wl.past1, wl.past2))
+        np.testing.assert_allclose(f64(r[b, h])[:n], ro[:n], atol=R_TOL, rtol=0)
+        clear = np.abs(ro[:n] - wl.tau) > MASK_BAND
+        np.testing.assert_array_equal(m[b, h].cpu().numpy()[:n][clear],
+                                      O.retention_mask(ro, wl.sink, wl.tau)[:n][clear])
+
+
+def test_hybrid_gla_sampled():
+    """The gated linear-attention layer of the pair at full size: prefill of
+    B=32 x 4096 tokens x 16 heads (dk = dv = 128), then 256 decode steps; sampled
+    heads against the oracle's token-by-token recurrence (outputs of every token
+    and the final state, max-abs error relative to max |reference| <= 1e-2)."""
+    from learnable_kv_token_b200 import lte as L
+    from oracle import gla_oracle as GO
+    wl = LI.WORKLOADS["hybrid"]
+    B, T, H, dk, steps = wl.B, wl.T, 16, 128, wl.decode_steps
+    q, k, v, a = LI.gla_inputs(B, T + steps, H, dk, dk, LI.generator(wl.seed + 1000))
+    qd, kd, vd, ad = (x.cuda() for x in (q, k, v, a))
+    o = torch.empty(B, T, H, dk, dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(B, H, dk, dk, dtype=torch.float32, device="cuda")
+    L.lte_gla_prefill(qd[:, :T].contiguous(), kd[:, :T].contiguous(), vd[:, :T].contiguous(),
+                      ad[:, :T].contiguous(), o, st)
+    od = torch.empty(steps, B, H, dk, dtype=torch.bfloat16, device="cuda")
+    for t in range(steps):
+        L.lte_gla_decode_step(qd[:, T + t].contiguous(), kd[:, T + t].contiguous(),
+                              vd[:, T + t].contiguous(), ad[:, T + t].contiguous(), od[t], st)
+    torch.cuda.synchronize()
+
+    def rel(got, ref):
+        return float(np.abs(got - ref).max() / np.abs(ref).max())
+
+    for b, h in [(0, 0), (17, 9), (31, 15)]:
+        o_ref, S_ref = GO.gla_recurrent(f64(q[b, :, h]), f64(k[b, :, h]), f64(v[b, :, h]),
+                                        f64(a[b, :, h]))
+        assert rel(f64(o[b, :, h]), o_ref[:T]) <= 1e-2, (b, h)
+        assert rel(f64(od[:, b, h]), o_ref[T:]) <= 1e-2, (b, h)
+        assert rel(f64(st[b, h]), S_ref) <= 1e-2, (b, h)
