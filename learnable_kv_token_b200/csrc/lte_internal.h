@@ -69,6 +69,8 @@ cudaError_t wait_probe(const int32_t* flag, int32_t expect, unsigned long long l
 cudaError_t gla_prefill(int B, int T, int H, int dk, int dv, int dtype, const void* q,
                         const void* k, const void* v, const float* a, void* o, float* state,
                         cudaStream_t stream);
+cudaError_t gla_prefill_tc(int B, int T, int H, const void* q, const void* k, const void* v,
+                           const float* a, void* o, float* state, cudaStream_t stream);
 cudaError_t gla_decode(int B, int H, int dk, int dv, int dtype, const void* q, const void* k,
                        const void* v, const float* a, void* o, float* state,
                        cudaStream_t stream);
