@@ -28,8 +28,9 @@
 //     S_0 diag(e^{b_m}) (the B operand of O) and into S_0 diag(e^{b_last});
 //     the masked A goes to shared memory as bf16 (over the set's consumed gate
 //     table), then O = A V + Q~ S_0'^T (M = 64, K = 64 + 128) and
-//     S += V^T Khat (M = 128, K = 64) run; one thread then requests chunk
-//     c + 2's inputs into the freed set, and O is stored as bf16.
+//     S += V^T Khat (M = 128, K = 64) run; O is staged as bf16 behind the
+//     masked A and written by TMA stores, after which one thread requests
+//     chunk c + 2's inputs into the freed set.
 // TMEM holds the fp32 state S (columns 0-127, lane = value channel) for the
 // whole sequence and one 64-row accumulator (columns 128-255: A of a chunk,
 // then its O; a 64-row accumulator keeps row r in lane 32 (r / 16) + r % 16).
@@ -106,7 +107,8 @@ constexpr int kBarGate = 1, kBarTmem = 2;                // named barriers of th
 __global__ void __launch_bounds__(kThreads, 1)
 gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                      int T, int H, __nv_bfloat16* __restrict__ o, float* __restrict__ state) {
+                      const __grid_constant__ CUtensorMap tm_o, int T, int H,
+                      float* __restrict__ state) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const int bh = blockIdx.x, b = bh / H, hd = bh % H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -116,8 +118,6 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   const uint32_t bar_g = s0 + kBar + 24;                 // gate work of set s done: + 8 s
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kBar + 40);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kBar + 44);
-  const long long row_stride = (long long)H * DK;        // elements between tokens
-  const long long base_bh = (long long)b * T * row_stride + (long long)hd * DK;
   float* st = state + (long long)bh * DV * DK;
   const int n_chunks = T / L;
 
@@ -208,18 +208,19 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // ---- Q~ = q x and K~ = k / x in place, Khat = K~ e^{b_last - b_m} in its buffer
       {
         const float* X = reinterpret_cast<const float*>(sset + kSetA);
-#pragma unroll 2
+        const int c16 = gt & 15, col = c16 * 8;            // the same 8 channels in every item
+        const float4 l0 = *reinterpret_cast<const float4*>(lam_r + col);
+        const float4 l1 = *reinterpret_cast<const float4*>(lam_r + col + 4);
+        const float ls[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
         for (int it = 0; it < L * 16 / kGroup; ++it) {
-          const int ci = gt + it * kGroup, r = ci >> 4, c16 = ci & 15, col = c16 * 8;
+          const int r = (gt + it * kGroup) >> 4;
           const uint32_t off = swz(L, r, c16);
           const uint4 qv = *reinterpret_cast<const uint4*>(sset + kSetQ + off);
           const uint4 kv = *reinterpret_cast<const uint4*>(sset + kSetK + off);
           const float4 x0 = *reinterpret_cast<const float4*>(X + r * DK + col);
           const float4 x1 = *reinterpret_cast<const float4*>(X + r * DK + col + 4);
-          const float4 l0 = *reinterpret_cast<const float4*>(lam_r + col);
-          const float4 l1 = *reinterpret_cast<const float4*>(lam_r + col + 4);
           const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-          const float ls[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
           const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv);
           const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv);
           uint32_t qo[4], ko[4], ho[4];
@@ -294,12 +295,17 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int j = c0 + e;
-          const float x0 = __uint_as_float(r[e]) * lam_m[j], x1 = __uint_as_float(r[e + 1]) * lam_m[j + 1];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(lam_m + c0 + e);
+          const float4 r4 = *reinterpret_cast<const float4*>(lam_r + c0 + e);
+          const float x0 = __uint_as_float(r[e]) * m4.x, x1 = __uint_as_float(r[e + 1]) * m4.y;
+          const float x2 = __uint_as_float(r[e + 2]) * m4.z, x3 = __uint_as_float(r[e + 3]) * m4.w;
           pk[e / 2] = pack2(x0, x1);
-          r[e] = __float_as_uint(x0 * lam_r[j]);
-          r[e + 1] = __float_as_uint(x1 * lam_r[j + 1]);
+          pk[e / 2 + 1] = pack2(x2, x3);
+          r[e] = __float_as_uint(x0 * r4.x);
+          r[e + 1] = __float_as_uint(x1 * r4.y);
+          r[e + 2] = __float_as_uint(x2 * r4.z);
+          r[e + 3] = __float_as_uint(x3 * r4.w);
         }
         tmem_st32(lane_addr + kColS + c0, r);
 #pragma unroll
@@ -363,13 +369,10 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       ok = mbar_wait_bounded(bar_mma, phase & 1, kWait, abort_flag, nullptr, 0);
       ++phase;
       tc_fence_after();
-      // the set is free: chunk c + 2's inputs start loading into it
-      if (tid == 0 && ok && c + 2 < n_chunks) {
-        load_chunk(c + 2);
-        ++n_issued;
-      }
-      // ---- O -> bf16 rows of the output (row t = 16 quad + lane on lanes 0-15;
-      // columns 64 hc .. + 63)
+      // ---- O -> bf16 rows (row t = 16 quad + lane on lanes 0-15; columns
+      // 64 hc .. + 63), staged as a [64][128] 128B-swizzled tile behind the
+      // masked A in the set's consumed gate table, then one TMA store per half
+      const uint32_t stage = kSetA + kHalf;
 #pragma unroll 1
       for (int c0 = hc * 64; c0 < hc * 64 + 64; c0 += 32) {
         uint32_t r[32];
@@ -377,17 +380,29 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tmem_wait_ld();
         if (lane < 16) {
           const int t = quad * 16 + lane;
-          uint4* dst = reinterpret_cast<uint4*>(o + base_bh + (long long)(c * L + t) * row_stride + c0);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pack2(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
-                                pack2(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
-                                pack2(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
-                                pack2(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7])));
+            *reinterpret_cast<uint4*>(sm + set * kSet + stage + swz(L, t, c0 / 8 + e)) =
+                make_uint4(pack2(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
+                           pack2(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
+                           pack2(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
+                           pack2(__uint_as_float(r[8 * e + 6]), __uint_as_float(r[8 * e + 7])));
         }
       }
+      fence_proxy_async();                                 // staged rows -> the TMA store
       tc_fence_before();
       if (!(ok = group_and(kBarTmem, kGroup, ok))) break;  // the accumulator is reused next
+      if (tid == 0) {
+        tma_store_4d(&tm_o, sb + stage, 0, hd, c * L, b);
+        tma_store_4d(&tm_o, sb + stage + kHalf, 64, hd, c * L, b);
+        bulk_commit();
+        bulk_wait_read();                                  // the staging has been read
+        // the set is free: chunk c + 2's inputs start loading into it
+        if (c + 2 < n_chunks) {
+          load_chunk(c + 2);
+          ++n_issued;
+        }
+      }
     }
     if (!ok && tid == 0) {                                 // MMAs in flight end before exit
       mma_commit(bar_mma);
@@ -419,6 +434,7 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       }
     }
   }
+  if (tid == 0) bulk_wait_all();                         // output stores complete before exit
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -433,21 +449,20 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 cudaError_t gla_prefill_tc(int B, int T, int H, const void* q, const void* k, const void* v,
                            const float* a, void* o, float* state, cudaStream_t stream) {
   using namespace glatc;
-  CUtensorMap mq, mk, mv, ma;
+  CUtensorMap mq, mk, mv, ma, mo;
   const cuuint64_t dims[4] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t sb[3] = {(cuuint64_t)DK * 2, (cuuint64_t)H * DK * 2, (cuuint64_t)T * H * DK * 2};
   const cuuint64_t sf[3] = {(cuuint64_t)DK * 4, (cuuint64_t)H * DK * 4, (cuuint64_t)T * H * DK * 4};
   const cuuint32_t box_b[4] = {64, 1, (cuuint32_t)L, 1}, box_f[4] = {(cuuint32_t)DK, 1, (cuuint32_t)L, 1};
   if (!tc::encode(&mq, q, 4, dims, sb, box_b) || !tc::encode(&mk, k, 4, dims, sb, box_b) ||
-      !tc::encode(&mv, v, 4, dims, sb, box_b) ||
+      !tc::encode(&mv, v, 4, dims, sb, box_b) || !tc::encode(&mo, o, 4, dims, sb, box_b) ||
       !tc::encode_ex(&ma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_NONE, a, 4, dims,
                      sf, box_f))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(gla_prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  gla_prefill_tc_kernel<<<B * H, kThreads, kSmem, stream>>>(mq, mk, mv, ma, T, H,
-                                                            (__nv_bfloat16*)o, state);
+  gla_prefill_tc_kernel<<<B * H, kThreads, kSmem, stream>>>(mq, mk, mv, ma, mo, T, H, state);
   return cudaGetLastError();
 }
 
