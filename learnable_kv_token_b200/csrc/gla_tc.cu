@@ -28,9 +28,9 @@
 //     S_0 diag(e^{b_m}) (the B operand of O) and into S_0 diag(e^{b_last});
 //     the masked A goes to shared memory as bf16 (over the set's consumed gate
 //     table), then O = A V + Q~ S_0'^T (M = 64, K = 64 + 128) and
-//     S += V^T Khat (M = 128, K = 64) run; O is staged as bf16 behind the
-//     masked A and written by TMA stores, after which one thread requests
-//     chunk c + 2's inputs into the freed set.
+//     S += V^T Khat (M = 128, K = 64) run; one thread requests chunk c + 2's
+//     inputs into the freed set, and O is staged as bf16 in the S_0' buffer
+//     and written by TMA stores.
 // TMEM holds the fp32 state S (columns 0-127, lane = value channel) for the
 // whole sequence and one 64-row accumulator (columns 128-255: A of a chunk,
 // then its O; a 64-row accumulator keeps row r in lane 32 (r / 16) + r % 16).
@@ -273,6 +273,7 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const float* lam_m = reinterpret_cast<const float*>(sm + kLam + set * 2 * DK * 4);
       const float* lam_r = lam_m + DK;
       ok = mbar_wait_bounded(bar_g + 8 * set, (c >> 1) & 1, kWait, abort_flag, nullptr, 0);
+      if (tid == 0) bulk_wait_read();                      // the previous output tile has left S_0'
       if (!(ok = group_and(kBarTmem, kGroup, ok))) break;
 
       // ---- A = Q~ K~^T (64 x 64, K = 128) into the 64-row accumulator
@@ -369,10 +370,15 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       ok = mbar_wait_bounded(bar_mma, phase & 1, kWait, abort_flag, nullptr, 0);
       ++phase;
       tc_fence_after();
+      // the set is free: chunk c + 2's inputs start loading into it
+      if (tid == 0 && ok && c + 2 < n_chunks) {
+        load_chunk(c + 2);
+        ++n_issued;
+      }
       // ---- O -> bf16 rows (row t = 16 quad + lane on lanes 0-15; columns
-      // 64 hc .. + 63), staged as a [64][128] 128B-swizzled tile behind the
-      // masked A in the set's consumed gate table, then one TMA store per half
-      const uint32_t stage = kSetA + kHalf;
+      // 64 hc .. + 63), staged as a [64][128] 128B-swizzled tile in the S_0'
+      // buffer (free until the next state pass), then one TMA store per half;
+      // thread 0 waits for the store to have read it before that pass
 #pragma unroll 1
       for (int c0 = hc * 64; c0 < hc * 64 + 64; c0 += 32) {
         uint32_t r[32];
@@ -382,7 +388,7 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           const int t = quad * 16 + lane;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            *reinterpret_cast<uint4*>(sm + set * kSet + stage + swz(L, t, c0 / 8 + e)) =
+            *reinterpret_cast<uint4*>(sm + kSb + swz(L, t, c0 / 8 + e)) =
                 make_uint4(pack2(__uint_as_float(r[8 * e]), __uint_as_float(r[8 * e + 1])),
                            pack2(__uint_as_float(r[8 * e + 2]), __uint_as_float(r[8 * e + 3])),
                            pack2(__uint_as_float(r[8 * e + 4]), __uint_as_float(r[8 * e + 5])),
@@ -393,15 +399,9 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       tc_fence_before();
       if (!(ok = group_and(kBarTmem, kGroup, ok))) break;  // the accumulator is reused next
       if (tid == 0) {
-        tma_store_4d(&tm_o, sb + stage, 0, hd, c * L, b);
-        tma_store_4d(&tm_o, sb + stage + kHalf, 64, hd, c * L, b);
+        tma_store_4d(&tm_o, s0 + kSb, 0, hd, c * L, b);
+        tma_store_4d(&tm_o, s0 + kSb + kHalf, 64, hd, c * L, b);
         bulk_commit();
-        bulk_wait_read();                                  // the staging has been read
-        // the set is free: chunk c + 2's inputs start loading into it
-        if (c + 2 < n_chunks) {
-          load_chunk(c + 2);
-          ++n_issued;
-        }
       }
     }
     if (!ok && tid == 0) {                                 // MMAs in flight end before exit
