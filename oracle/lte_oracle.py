@@ -25,7 +25,10 @@ Readings taken where the pages are silent (each is restated where used):
 
 * window (t-w, t] holds w keys including the current token;
 * the cap C counts retained tokens only (sinks are extra); when more than C
-  tokens qualify, the C most recent are kept (FIFO ring);
+  tokens qualify, the C most recent are kept (FIFO ring) -- policy "recent".
+  The pages leave the capped segment's policy open; policy "first" keeps the
+  first C retained tokens instead (later ones are dropped once the segment is
+  full);
 * retain iff r >= tau; the first s tokens are sinks and are never "retained";
 * CNN: conv1d over the channel concatenation [k; v] (k first), PyTorch
   cross-correlation convention, per-layer zero padding outside [0, n), a
@@ -178,18 +181,24 @@ def compact(m) -> tuple[np.ndarray, int, np.ndarray]:
 # (3) attended set and attention  [LTE, Fig. 2 right: A-plus-column pattern]
 # ---------------------------------------------------------------------------
 
-def attended_set(t: int, m, sink: int, window: int, cap: int) -> list[int]:
+CAP_RECENT, CAP_FIRST = "recent", "first"     # policies of the capped segment
+
+
+def attended_set(t: int, m, sink: int, window: int, cap: int,
+                 policy: str = CAP_RECENT) -> list[int]:
     """Key positions query t attends to, for one KV head.
 
-    S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t,
-    Ret_t = the `cap` largest j in [s, t-w] with m_j = 1 (the C most recent
-    tokens that were kept when they left the window).
+    S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t, with Ret_t drawn from the
+    tokens j in [s, t-w] with m_j = 1 (kept when they left the window):
+    policy "recent": the `cap` largest such j (the C most recent);
+    policy "first":  the `cap` smallest such j (the segment fills, then later
+    retained tokens are dropped).
     """
     keys = set(range(0, min(sink, t + 1)))
     keys |= set(range(max(0, t - window + 1), t + 1))
     candidates = [j for j in range(sink, t - window + 1) if m[j]]
     if cap > 0:
-        keys |= set(candidates[-cap:])
+        keys |= set(candidates[-cap:] if policy == CAP_RECENT else candidates[:cap])
     return sorted(keys)
 
 
@@ -210,7 +219,7 @@ def attend(q_rows, K, V, scale: float):
 
 
 def prefill_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
-                 rows=None):
+                 rows=None, policy: str = CAP_RECENT):
     """Prefill of one (batch element, KV head) unit.
 
     q [T, G, D] (the G query heads that share this KV head), k, v [T, D],
@@ -224,13 +233,14 @@ def prefill_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
     k = _f64(k)
     v = _f64(v)
     for t in (range(T) if rows is None else rows):
-        S = attended_set(t, m, sink, window, cap)
+        S = attended_set(t, m, sink, window, cap, policy)
         o[t], lse[t] = attend(q[t], k[S], v[S], scale)
         count[t] = len(S)
     return o, lse, count
 
 
-def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | None = None):
+def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | None = None,
+            policy: str = CAP_RECENT):
     """Prefill over a batch: q [B,T,Hq,D], k, v [B,T,Hkv,D], masks [B,Hkv,T].
 
     GQA: query head qh uses KV head qh // (Hq // Hkv).  Returns o [B,T,Hq,D],
@@ -247,7 +257,7 @@ def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | Non
     for b in range(B):
         for h in range(Hkv):
             ou, lu, cu = prefill_unit(q[b, :, h * G:(h + 1) * G], k[b, :, h], v[b, :, h],
-                                      masks[b, h], sink, window, cap, scale)
+                                      masks[b, h], sink, window, cap, scale, policy=policy)
             o[b, :, h * G:(h + 1) * G] = ou
             lse[b, h * G:(h + 1) * G] = lu.T
             count[b, h] = cu
@@ -266,8 +276,11 @@ class DecodeCache:
 
     * window ring: w slots, token j lives in slot j mod w while in (t-w, t];
     * sink slots: s slots, token j < s moves to slot j when it leaves the window;
-    * retained ring: C slots, the i-th retained token (0-based) goes to slot
-      i mod C, overwriting the oldest one (the cap keeps the C most recent);
+    * retained ring: C slots.  Policy "recent": the i-th retained token
+      (0-based) goes to slot i mod C, overwriting the oldest one (the cap
+      keeps the C most recent).  Policy "first": the i-th retained token goes
+      to slot i while i < C and is dropped afterwards (ret_total then counts
+      the stored tokens);
     * r of window tokens, filled by deferred batched scoring.
     """
     D: int
@@ -291,6 +304,7 @@ class DecodeCache:
     t: int = 0              # tokens received so far
     n_scored: int = 0       # tokens [0, n_scored) have a score
     fed: np.ndarray | None = None   # optional fed mask instead of the CNN
+    policy: str = CAP_RECENT
 
     def __post_init__(self):
         w, s, C, D = self.window, self.sink, self.cap, self.D
@@ -344,7 +358,10 @@ class DecodeCache:
             else:
                 assert leaving < self.n_scored, "token left the window unscored"
                 r = self.win_r[slot]
-                if r >= self.tau and self.cap > 0:
+                keep = r >= self.tau and self.cap > 0
+                if keep and self.policy == CAP_FIRST and self.ret_total >= self.cap:
+                    keep = False                     # the segment is full: dropped
+                if keep:
                     rs = self.ret_total % self.cap
                     self.ret_k[rs] = self.win_k[slot]
                     self.ret_v[rs] = self.win_v[slot]
@@ -384,7 +401,8 @@ class DecodeCache:
 
 
 def decode_unit(q, k, v, T0: int, sink: int, window: int, cap: int, tau: float,
-                cnn: CNN | None, score_batch: int, scale: float, fed=None):
+                cnn: CNN | None, score_batch: int, scale: float, fed=None,
+                policy: str = CAP_RECENT):
     """Feed tokens 0..T-1 of one unit through the cache; for every token
     t >= T0 return its attention output, lse and attended positions.
 
@@ -392,7 +410,7 @@ def decode_unit(q, k, v, T0: int, sink: int, window: int, cap: int, tau: float,
     cache updates as decoding (no attention output is kept for it).
     """
     cache = DecodeCache(D=k.shape[1], sink=sink, window=window, cap=cap, tau=tau,
-                        cnn=cnn, score_batch=score_batch)
+                        cnn=cnn, score_batch=score_batch, policy=policy)
     cache.fed = None if fed is None else np.asarray(fed)
     outs, lses, sets, rets = [], [], [], []
     for t in range(k.shape[0]):
@@ -404,11 +422,14 @@ def decode_unit(q, k, v, T0: int, sink: int, window: int, cap: int, tau: float,
     return np.array(outs), np.array(lses), sets, rets, cache
 
 
-def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int):
+def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int,
+                       policy: str = CAP_RECENT):
     """The cache contents after a prompt of T0 tokens, read off the prefill
     mask: window = positions (T0-1-w, T0-1], sinks = j < s with j <= T0-1-w,
     retained = the C most recent j in [s, T0-1-w] with m_j = 1, with the
-    i-th retained token (0-based over all retained) in ring slot i mod C.
+    i-th retained token (0-based over all retained) in ring slot i mod C
+    (policy "first": the C earliest such j, the i-th in slot i, and ret_total
+    counts the stored ones).
 
     Returns dict of position arrays (-1 = empty) and ret_total.
     """
@@ -420,6 +441,8 @@ def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int):
     for j in range(min(sink, last_out + 1)):
         sink_pos[j] = j
     ret = [j for j in range(sink, last_out + 1) if m[j]]
+    if policy == CAP_FIRST:
+        ret = ret[:cap]
     ret_pos = np.full(cap, -1, dtype=np.int64)
     for i, j in enumerate(ret):
         if cap > 0:

@@ -28,6 +28,19 @@ def brute_member(j, t, m, s, w, C):
     return newer < C
 
 
+def brute_member_first(j, t, m, s, w, C):
+    """Policy "first": a retained token that left the window survives iff
+    fewer than C retained tokens left the window before it."""
+    if j > t or j < 0:
+        return False
+    if j < s or j > t - w:
+        return True
+    if not m[j]:
+        return False
+    older = sum(1 for i in range(s, j) if m[i])
+    return older < C
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_attended_set_vs_bruteforce(seed):
     rng = np.random.default_rng(seed)
@@ -42,6 +55,38 @@ def test_attended_set_vs_bruteforce(seed):
             S = O.attended_set(t, m, s, w, C)
             ref = [j for j in range(T) if brute_member(j, t, m, s, w, C)]
             assert S == ref, (T, s, w, C, t)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_attended_set_first_policy_vs_bruteforce(seed):
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(25):
+        T = int(rng.integers(1, 48))
+        s = int(rng.integers(0, 5))
+        w = int(rng.integers(1, 14))
+        C = int(rng.choice([0, 1, 2, 3, 8, 100]))
+        p = float(rng.choice([0.0, 0.3, 0.7, 1.0]))
+        m = O.fed_mask((rng.random(T) < p).astype(np.uint8), s)
+        for t in range(T):
+            S = O.attended_set(t, m, s, w, C, O.CAP_FIRST)
+            ref = [j for j in range(T) if brute_member_first(j, t, m, s, w, C)]
+            assert S == ref, (T, s, w, C, t)
+            if C >= T:                       # the cap never binds: both policies agree
+                assert S == O.attended_set(t, m, s, w, C, O.CAP_RECENT)
+
+
+def test_first_policy_closed_forms():
+    """r == 1: the first C tokens past the sink stay for good; the count
+    formula min(C, cnt[t-w]) is the same as for the most recent C."""
+    T, s, w, C = 120, 3, 10, 7
+    ones = O.fed_mask(np.ones(T, np.uint8), s)
+    _, _, cnt = O.compact(ones)
+    for t in range(T):
+        S = O.attended_set(t, ones, s, w, C, O.CAP_FIRST)
+        n = cnt[t - w] if t - w >= 0 else 0
+        ret = [j for j in S if s <= j <= t - w]
+        assert ret == list(range(s, s + min(C, n)))
+        assert len(S) == min(t + 1, w) + len([j for j in range(s) if j <= t - w]) + min(C, n)
 
 
 def test_closed_forms():
