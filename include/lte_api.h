@@ -60,15 +60,25 @@ typedef enum {
 
 typedef enum { LTE_F32 = 0, LTE_BF16 = 1 } lte_dtype;
 
+/* Which retained tokens the capped out-of-window segment keeps once more
+ * than C qualify.  [LTE paper, Fig. 3 caption: the segment has capped
+ * capacity; the pages leave the policy open.]
+ *   LTE_CAP_RECENT: the C most recent (a ring; the oldest is overwritten);
+ *   LTE_CAP_FIRST:  the first C (later retained tokens are dropped once the
+ *                   segment is full). */
+typedef enum { LTE_CAP_RECENT = 0, LTE_CAP_FIRST = 1 } lte_cap_policy;
+
 /* Shapes and method parameters of one LTE layer.
  * sink = s >= 0, window = w >= 1, cap = C >= 0 (retained tokens only; sinks
  * are extra), tau = retention threshold (retain iff r >= tau), scale =
- * softmax scale (1/sqrt(D) in the usual setting), dtype of q/k/v/o/caches. */
+ * softmax scale (1/sqrt(D) in the usual setting), dtype of q/k/v/o/caches,
+ * cap_policy = lte_cap_policy (0, the C most recent, when zero-initialised). */
 typedef struct {
   int32_t B, T, Hq, Hkv, D;
   int32_t sink, window, cap;
   float tau, scale;
   int32_t dtype;
+  int32_t cap_policy;
 } lte_dims;
 
 /* Element strides of a [B, T, H, D] tensor (D stride is 1). */

@@ -80,7 +80,8 @@ struct KeyRanges {
 
 template <int D>
 __global__ void __launch_bounds__(kMmaThreads, 2)
-attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, float scale_log2,
+attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, int cap_policy,
+                        float scale_log2,
                         const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                         const __nv_bfloat16* __restrict__ v, Strides4 qs, Strides4 kvs,
                         const int32_t* __restrict__ cnt, const __nv_bfloat16* __restrict__ k_col,
@@ -118,8 +119,8 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, f
   // ---- key ranges of the tile
   KeyRanges kr;
   {
-    const int n_first = (t0 >= window) ? cnt[crow + t0 - window] : 0;
-    const int n_last = (t_last >= window) ? cnt[crow + t_last - window] : 0;
+    const int n_first = (t0 >= window) ? held_retained(cnt[crow + t0 - window], cap, cap_policy) : 0;
+    const int n_last = (t_last >= window) ? held_retained(cnt[crow + t_last - window], cap, cap_policy) : 0;
     const int lo_min = n_first - cap > 0 ? n_first - cap : 0;
     int nsink = t_last - window + 1;
     nsink = nsink < 0 ? 0 : (nsink > sink ? sink : nsink);
@@ -181,7 +182,7 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, f
     const int tt = t0 + rho % TOK;
     t_row[hr] = tt;
     int hi = 0;
-    if (tt < T && tt >= window) hi = cnt[crow + tt - window];
+    if (tt < T && tt >= window) hi = held_retained(cnt[crow + tt - window], cap, cap_policy);
     hi_row[hr] = hi;
     lo_row[hr] = hi - cap > 0 ? hi - cap : 0;
   }
@@ -360,7 +361,7 @@ static cudaError_t launch_mma(const PrefillArgs& a, cudaStream_t stream) {
   dim3 grid((d->T + TOK - 1) / TOK, d->Hkv, d->B);
   const float scale_log2 = d->scale * 1.4426950408889634f;
   attn_prefill_mma_kernel<D><<<grid, kMmaThreads, smem, stream>>>(
-      d->T, d->Hq, d->Hkv, d->sink, d->window, d->cap, scale_log2,
+      d->T, d->Hq, d->Hkv, d->sink, d->window, d->cap, d->cap_policy, scale_log2,
       (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v, a.qs,
       a.kvs, a.cnt, (const __nv_bfloat16*)a.k_col, (const __nv_bfloat16*)a.v_col,
       (__nv_bfloat16*)a.o, a.os, a.lse);

@@ -25,7 +25,7 @@ constexpr int kSimtMaxD = 128;
 
 __global__ void __launch_bounds__(kSimtThreads)
 attn_prefill_simt_kernel(int T, int Hq, int Hkv, int D, int sink, int window, int cap,
-                         float scale, const float* __restrict__ q, const float* __restrict__ k,
+                         int cap_policy, float scale, const float* __restrict__ q, const float* __restrict__ k,
                          const float* __restrict__ v, Strides4 qs, Strides4 kvs,
                          const int32_t* __restrict__ cnt, const float* __restrict__ k_col,
                          const float* __restrict__ v_col, float* __restrict__ o, Strides4 os,
@@ -52,12 +52,12 @@ attn_prefill_simt_kernel(int T, int Hq, int Hkv, int D, int sink, int window, in
   // per-row retained range [lo_t, hi_t) of the compacted list
   int hi_t = 0, lo_t = 0;
   if (t < T && t >= window) {
-    hi_t = cnt[crow + t - window];
+    hi_t = held_retained(cnt[crow + t - window], cap, cap_policy);
     lo_t = hi_t - cap > 0 ? hi_t - cap : 0;
   }
   // tile-wide ranges
-  const int n_first = (t0 >= window) ? cnt[crow + t0 - window] : 0;
-  const int n_last = (t_last >= window) ? cnt[crow + t_last - window] : 0;
+  const int n_first = (t0 >= window) ? held_retained(cnt[crow + t0 - window], cap, cap_policy) : 0;
+  const int n_last = (t_last >= window) ? held_retained(cnt[crow + t_last - window], cap, cap_policy) : 0;
   const int lo_min = n_first - cap > 0 ? n_first - cap : 0;
   int nsink = t_last - window + 1;
   nsink = nsink < 0 ? 0 : (nsink > sink ? sink : nsink);
@@ -159,7 +159,7 @@ cudaError_t attn_prefill_simt(const PrefillArgs& a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   attn_prefill_simt_kernel<<<grid, kSimtThreads, smem, stream>>>(
-      d->T, d->Hq, d->Hkv, d->D, d->sink, d->window, d->cap, d->scale, (const float*)a.q,
+      d->T, d->Hq, d->Hkv, d->D, d->sink, d->window, d->cap, d->cap_policy, d->scale, (const float*)a.q,
       (const float*)a.k, (const float*)a.v, a.qs, a.kvs, a.cnt, (const float*)a.k_col,
       (const float*)a.v_col, (float*)a.o, a.os, a.lse);
   return cudaGetLastError();

@@ -89,7 +89,7 @@ enum {
 static_assert(8 * kNumBars + 8 <= 512, "barriers, abort flag and TMEM slot fit the tail");
 
 struct Params {
-  int T, Hq, Hkv, G, TOK, sink, window, cap;
+  int T, Hq, Hkv, G, TOK, sink, window, cap, cap_policy;
   int n_pairs, n_units, n_items;
   float scale_log2;
   const int32_t* cnt;
@@ -174,8 +174,8 @@ __device__ __forceinline__ ItemCounts load_counts(const Params& p, int i) {
   int u, t0, t_last;
   item_tokens(p, i, u, t0, t_last);
   const long long crow = (long long)u * p.T;
-  if (t0 >= p.window) c.n_first = __ldg(p.cnt + crow + t0 - p.window);
-  if (t_last >= p.window) c.n_last = __ldg(p.cnt + crow + t_last - p.window);
+  if (t0 >= p.window) c.n_first = held_retained(__ldg(p.cnt + crow + t0 - p.window), p.cap, p.cap_policy);
+  if (t_last >= p.window) c.n_last = held_retained(__ldg(p.cnt + crow + t_last - p.window), p.cap, p.cap_policy);
   return c;
 }
 __device__ __forceinline__ Item make_item(const Params& p, int i, const ItemCounts& c) {
@@ -446,7 +446,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       int u, t0, t_last;
       item_tokens(p, i, u, t0, t_last);
       const int t = t0 + x * p.TOK + row / p.G;
-      return (t < p.T && t >= p.window) ? __ldg(p.cnt + (long long)u * p.T + t - p.window) : 0;
+      return (t < p.T && t >= p.window)
+                 ? held_retained(__ldg(p.cnt + (long long)u * p.T + t - p.window), p.cap, p.cap_policy)
+                 : 0;
     };
     ItemCounts cn = load_counts(p, blockIdx.x);
     int hi_next = row_count(blockIdx.x);
@@ -657,7 +659,7 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   }
   Params p{};
   p.T = d->T; p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = G; p.TOK = TOK;
-  p.sink = d->sink; p.window = d->window; p.cap = d->cap;
+  p.sink = d->sink; p.window = d->window; p.cap = d->cap; p.cap_policy = d->cap_policy;
   p.n_pairs = (d->T + 2 * TOK - 1) / (2 * TOK);
   p.n_units = d->B * d->Hkv;
   p.n_items = p.n_pairs * p.n_units;

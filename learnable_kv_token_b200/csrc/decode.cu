@@ -115,7 +115,7 @@ __device__ __forceinline__ void pdl_launch_next() {
 
 // ---------------------------------------------------------------------------
 struct PrepParams {
-  int Hkv, D, elt, window, sink, cap, score_batch, future, n_units;
+  int Hkv, D, elt, window, sink, cap, cap_policy, score_batch, future, n_units;
   float tau;
   const char* k_t;
   const char* v_t;
@@ -163,7 +163,8 @@ decode_prep_kernel(PrepParams pp, ScoreParams sp, RingKV<T> kv) {
       rt = pp.ret_total[u];
       if (held != leaving) record_error(pp.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
       else if (leaving < pp.sink) dst = pp.window + leaving;
-      else if (pp.cap > 0 && r >= pp.tau) dst = pp.window + pp.sink + rt % pp.cap;
+      else if (pp.cap > 0 && r >= pp.tau && (pp.cap_policy == LTE_CAP_RECENT || rt < pp.cap))
+        dst = pp.window + pp.sink + rt % pp.cap;       // under LTE_CAP_FIRST a full segment drops it
     }
     dst_sh = dst;
   }
@@ -637,7 +638,7 @@ static cudaError_t launch_prep(const lte_dims* d, const lte_cnn* cnn, const lte_
                                int32_t* counters, DevError* err, cudaStream_t stream) {
   PrepParams pp{};
   pp.Hkv = d->Hkv; pp.D = d->D; pp.elt = sizeof(T); pp.window = d->window; pp.sink = d->sink;
-  pp.cap = d->cap; pp.score_batch = score_batch;
+  pp.cap = d->cap; pp.cap_policy = d->cap_policy; pp.score_batch = score_batch;
   pp.future = (cnn->k1 - 1 - cnn->past1) + (cnn->k2 - 1 - cnn->past2);
   pp.n_units = d->B * d->Hkv; pp.tau = d->tau;
   pp.k_t = (const char*)k_t; pp.v_t = (const char*)v_t;
@@ -773,7 +774,7 @@ __host__ __device__ constexpr int fu_stages(int D) {
 }
 
 struct FusedParams {
-  int Hq, Hkv, G, window, sink, cap, L, score_batch, future;
+  int Hq, Hkv, G, window, sink, cap, cap_policy, L, score_batch, future;
   float tau, scale_log2;
   const __nv_bfloat16* q_t;
   const __nv_bfloat16* k_t;
@@ -935,7 +936,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const float r = p.win_r[(long long)u * p.window + slot_w];
         if (held != leaving) record_error(p.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
         else if (leaving < p.sink) dst = p.window + leaving;
-        else if (p.cap > 0 && r >= p.tau) dst = p.window + p.sink + rt % p.cap;
+        else if (p.cap > 0 && r >= p.tau && (p.cap_policy == LTE_CAP_RECENT || rt < p.cap))
+          dst = p.window + p.sink + rt % p.cap;         // under LTE_CAP_FIRST a full segment drops it
       }
     }
     dst = __shfl_sync(0xffffffffu, dst, 0);
@@ -1194,7 +1196,8 @@ static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte
                                 float* lse_t, int score_batch, DevError* err, cudaStream_t stream) {
   FusedParams p{};
   p.Hq = d->Hq; p.Hkv = d->Hkv; p.G = d->Hq / d->Hkv; p.window = d->window; p.sink = d->sink;
-  p.cap = d->cap; p.L = d->window + d->sink + d->cap; p.score_batch = score_batch;
+  p.cap = d->cap; p.cap_policy = d->cap_policy; p.L = d->window + d->sink + d->cap;
+  p.score_batch = score_batch;
   p.future = (cnn->k1 - 1 - cnn->past1) + (cnn->k2 - 1 - cnn->past2);
   p.tau = d->tau; p.scale_log2 = d->scale * 1.4426950408889634f;
   p.q_t = (const __nv_bfloat16*)q_t; p.k_t = (const __nv_bfloat16*)k_t;

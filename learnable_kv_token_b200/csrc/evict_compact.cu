@@ -108,8 +108,8 @@ cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask
 // Decode-cache set-up from a prefilled prompt (Fig. 3 layout): window ring,
 // sink slots, retained ring.  One CTA per unit.
 __global__ void __launch_bounds__(256)
-cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap, int T0,
-                  int n_scored, const char* __restrict__ k, const char* __restrict__ v,
+cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap, int cap_policy,
+                  int T0, int n_scored, const char* __restrict__ k, const char* __restrict__ v,
                   Strides4 s, const float* __restrict__ r, const int32_t* __restrict__ idx,
                   const int32_t* __restrict__ cnt, char* __restrict__ ck, char* __restrict__ cv,
                   int32_t* __restrict__ pos, float* __restrict__ win_r,
@@ -118,7 +118,9 @@ cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap,
   const int L = window + sink + cap;
   const long long row0 = (long long)u * T;
   const int last_out = T0 - 1 - window;                 // newest token outside the window
-  const int n = last_out >= 0 ? cnt[row0 + last_out] : 0;
+  // retained tokens the segment holds (all that left with a keep decision, or
+  // under LTE_CAP_FIRST at most the first C), the i-th in ring slot i mod C
+  const int n = last_out >= 0 ? held_retained(cnt[row0 + last_out], cap, cap_policy) : 0;
   const int ret_lo = (n - cap) > 0 ? n - cap : 0;
 
   // slot -> source token (or -1)
@@ -169,7 +171,7 @@ cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, con
                        int T_prompt, int n_scored, cudaStream_t stream) {
   const int elt = d->dtype == LTE_BF16 ? 2 : 4;
   cache_init_kernel<<<d->B * d->Hkv, 256, 0, stream>>>(
-      d->T, d->Hkv, d->D, elt, d->window, d->sink, d->cap, T_prompt, n_scored,
+      d->T, d->Hkv, d->D, elt, d->window, d->sink, d->cap, d->cap_policy, T_prompt, n_scored,
       (const char*)k, (const char*)v, s, r, idx, cnt, (char*)c->k, (char*)c->v, c->pos,
       c->win_r, c->ret_total, c->meta);
   return cudaGetLastError();

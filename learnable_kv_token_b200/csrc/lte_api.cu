@@ -24,6 +24,7 @@ lte_status check_dims(const lte_dims* d) {
   if (d->Hq % d->Hkv != 0) return LTE_ERR_INVALID_ARG;
   if (d->sink < 0 || d->window < 1 || d->cap < 0) return LTE_ERR_INVALID_ARG;
   if (d->dtype != LTE_F32 && d->dtype != LTE_BF16) return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy != LTE_CAP_RECENT && d->cap_policy != LTE_CAP_FIRST) return LTE_ERR_INVALID_ARG;
   if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return LTE_ERR_INVALID_ARG;
   if (std::isnan(d->tau)) return LTE_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LTE_ERR_UNSUPPORTED;

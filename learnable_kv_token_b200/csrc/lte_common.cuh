@@ -75,6 +75,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Retained tokens a row (or the cache) holds when n have left the window with
+// a keep decision: under LTE_CAP_FIRST only the first C are stored, so the
+// slot range [max(0, n' - C), n') of the compacted list, n' = this value,
+// covers both policies.
+__host__ __device__ __forceinline__ int held_retained(int n, int cap, int policy) {
+  return (policy == LTE_CAP_FIRST && n > cap) ? cap : n;
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

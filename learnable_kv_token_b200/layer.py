@@ -23,10 +23,12 @@ class LayerParams:
     scale: float | None = None
     past1: int = 2
     past2: int = 1
+    cap_policy: int = L.LTE_CAP_RECENT      # or L.LTE_CAP_FIRST
 
     def dims(self, B, T, Hq, Hkv, D, dtype) -> L.lte_dims:
         scale = (1.0 / D ** 0.5) if self.scale is None else self.scale
-        return L.make_dims(B, T, Hq, Hkv, D, self.sink, self.window, self.cap, self.tau, scale, dtype)
+        return L.make_dims(B, T, Hq, Hkv, D, self.sink, self.window, self.cap, self.tau, scale, dtype,
+                           self.cap_policy)
 
 
 def cnn_future(w1, w2, past1, past2) -> int:

@@ -21,6 +21,7 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 LTE_F32, LTE_BF16 = 0, 1
+LTE_CAP_RECENT, LTE_CAP_FIRST = 0, 1
 LTE_WS_PREFILL, LTE_WS_DECODE = 0, 1
 STATUS = {0: "LTE_OK", 1: "LTE_ERR_INVALID_ARG", 2: "LTE_ERR_UNSUPPORTED", 3: "LTE_ERR_CUDA",
           4: "LTE_ERR_TIMEOUT", 5: "LTE_ERR_WORKSPACE", 6: "LTE_ERR_DEVICE"}
@@ -35,7 +36,8 @@ class LteError(RuntimeError):
 class lte_dims(C.Structure):
     _fields_ = [("B", C.c_int32), ("T", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32),
                 ("D", C.c_int32), ("sink", C.c_int32), ("window", C.c_int32), ("cap", C.c_int32),
-                ("tau", C.c_float), ("scale", C.c_float), ("dtype", C.c_int32)]
+                ("tau", C.c_float), ("scale", C.c_float), ("dtype", C.c_int32),
+                ("cap_policy", C.c_int32)]
 
 
 class lte_strides(C.Structure):
@@ -118,9 +120,11 @@ def dtype_code(dt: torch.dtype) -> int:
     raise ValueError(f"unsupported dtype {dt}")
 
 
-def make_dims(B, T, Hq, Hkv, D, sink, window, cap, tau, scale, dtype) -> lte_dims:
+def make_dims(B, T, Hq, Hkv, D, sink, window, cap, tau, scale, dtype,
+              cap_policy=LTE_CAP_RECENT) -> lte_dims:
     return lte_dims(B, T, Hq, Hkv, D, sink, window, cap, float(tau), float(scale),
-                    dtype_code(dtype) if isinstance(dtype, torch.dtype) else int(dtype))
+                    dtype_code(dtype) if isinstance(dtype, torch.dtype) else int(dtype),
+                    int(cap_policy))
 
 
 def make_cnn(w1, b1, w2, b2, past1, past2) -> tuple[lte_cnn, tuple]:

@@ -62,6 +62,10 @@ def test_host_validation_without_gpu(lib):
                                None, None, None) == 1
     bad = L.make_dims(1, 64, 6, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32)   # Hq % Hkv != 0
     assert f.lte_workspace_bytes(C.byref(bad), 0) == 0
+    pol = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, cap_policy=2)  # no such policy
+    assert f.lte_workspace_bytes(C.byref(pol), 0) == 0
+    first = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, L.LTE_CAP_FIRST)
+    assert f.lte_workspace_bytes(C.byref(first), 0) >= 16
     d96 = L.make_dims(1, 64, 4, 4, 96, 4, 16, 8, 0.5, 0.1, L.LTE_F32)     # D not in {64,128}
     assert f.lte_sparse_attn_prefill(C.byref(d96), None, None, None, None, None, None, None, None,
                                      None, None, None, None, 0, None) == 2

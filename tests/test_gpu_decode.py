@@ -27,12 +27,13 @@ def _inputs(B, Hq, Hkv, D, T_total, seed, w_std):
     return q, k, v, cnn
 
 
-def _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, score_batch, check_every=0):
+def _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, score_batch, check_every=0,
+                cap_policy=0):
     """Prefill the prompt on the GPU, set up the cache, decode the rest.
     Returns o [steps,B,Hq,D], lse [steps,B,Hq], retained sets at checkpoints."""
     B, T_total, Hq, D = q.shape
     Hkv = k.shape[2]
-    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=tau)
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=tau, cap_policy=cap_policy)
     qd, kd, vd = (x.cuda() for x in (q, k, v))
     cd = tuple(x.cuda() for x in cnn)
     kp, vp = kd[:, :T0].contiguous(), vd[:, :T0].contiguous()
@@ -87,6 +88,38 @@ def test_decode_vs_oracle_simulation(layer, cfg):
                                    o_ref, lse_ref, torch.bfloat16, f"unit {b},{h}")
             for t, rs in rets.items():
                 assert rs[b][h] == ret_ref[t - T0], (b, h, t)
+
+
+@pytest.mark.parametrize("cfg", [
+    # B, Hq, Hkv, D, sink, window, cap, T0, steps, score_batch
+    (2, 8, 2, 128, 4, 64, 6, 300, 120, 16),         # one fused launch per step
+    (40, 8, 4, 64, 2, 32, 5, 60, 40, 8),            # more units than SMs: two launches per step
+])
+def test_decode_cap_first_policy(layer, cfg):
+    """LTE_CAP_FIRST through cache set-up and decode: the segment keeps the
+    first C retained tokens and drops later ones; outputs and retained sets
+    against the oracle's simulation with policy "first" (sampled units)."""
+    from learnable_kv_token_b200 import lte as L
+    B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = cfg
+    T = T0 + steps
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 60 + B, w_std=0.1)
+    G = Hq // Hkv
+    units = [(b, h) for b in range(B) for h in range(Hkv)][:: max(1, (B * Hkv) // 6)]
+    r_or = {(b, h): O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h))
+            for b in range(B) for h in range(Hkv)}
+    tau, margin = clean_tau(np.stack(list(r_or.values())))
+    assert margin > 1e-5
+    o_g, lse_g, rets, _, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, Ds,
+                                         check_every=13, cap_policy=L.LTE_CAP_FIRST)
+    for b, h in units:
+        o_ref, lse_ref, sets, ret_ref, _ = O.decode_unit(
+            f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]), f64(v[b, :, h]), T0, sink,
+            window, cap, tau, oracle_cnn(cnn, h), Ds, scale_of(D), policy=O.CAP_FIRST)
+        assert_attention_close(f64(o_g[:, b, h * G:(h + 1) * G]), f64(lse_g[:, b, h * G:(h + 1) * G]),
+                               o_ref, lse_ref, torch.bfloat16, f"unit {b},{h}")
+        for t, rs in rets.items():
+            assert rs[b][h] == ret_ref[t - T0], (b, h, t)
+        assert len(ret_ref[-1]) <= cap
 
 
 def test_decode_split_kv_path(layer):

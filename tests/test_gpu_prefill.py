@@ -177,8 +177,8 @@ def test_compact_from_scores(L):
 
 
 # --------------------------------------------------------------------------- attention
-def _run_prefill(layer, q, k, v, mask, sink, window, cap, scale=None):
-    p = layer.LayerParams(sink=sink, window=window, cap=cap, scale=scale)
+def _run_prefill(layer, q, k, v, mask, sink, window, cap, scale=None, cap_policy=0):
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, scale=scale, cap_policy=cap_policy)
     qd, kd, vd, md = _dev(q, k, v, mask)
     out = layer.prefill(qd, kd, vd, p, mask=md)
     torch.cuda.synchronize()
@@ -210,6 +210,37 @@ def test_prefill_fed_mask_parity(layer, case):
     for b in range(B):
         for h in range(Hkv):
             o_ref, lse_ref, _ = oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap, scale_of(D))
+            o_g = f64(out.o[b, :, h * G:(h + 1) * G])
+            lse_g = f64(out.lse[b, h * G:(h + 1) * G]).T
+            assert_attention_close(o_g, lse_g, o_ref, lse_ref, dtype, f"unit {b},{h}")
+
+
+FIRST_CASES = [
+    # B, T, Hq, Hkv, D, dtype, sink, window, cap, rate: the cap binds early
+    (2, 1100, 8, 2, 128, torch.bfloat16, 4, 128, 24, 0.3),     # tcgen05 kernel
+    (2, 333, 4, 1, 64, torch.bfloat16, 2, 37, 5, 0.5),         # warp-MMA kernel (head dim 64)
+    (1, 400, 2, 2, 128, torch.float32, 3, 20, 7, 0.5),         # fp32 kernel
+    (1, 700, 16, 4, 128, torch.bfloat16, 4, 64, 300, 0.2),     # the cap never binds
+]
+
+
+@pytest.mark.parametrize("case", FIRST_CASES)
+def test_prefill_cap_first_policy(layer, case):
+    """LTE_CAP_FIRST: rows attend to the first C retained tokens instead of the
+    C most recent, in every prefill kernel, against the oracle's policy "first"."""
+    from learnable_kv_token_b200 import lte as L
+    B, T, Hq, Hkv, D, dtype, sink, window, cap, rate = case
+    g = LI.generator(300 + T)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, dtype, g)
+    mask = LI.bernoulli_mask(B, Hkv, T, rate, g)
+    out = _run_prefill(layer, q, k, v, mask, sink, window, cap, cap_policy=L.LTE_CAP_FIRST)
+    masks = fed_masks(mask, sink)
+    G = Hq // Hkv
+    rows = list(range(T))
+    for b in range(B):
+        for h in range(Hkv):
+            o_ref, lse_ref, _ = oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap,
+                                            scale_of(D), policy=O.CAP_FIRST)
             o_g = f64(out.o[b, :, h * G:(h + 1) * G])
             lse_g = f64(out.lse[b, h * G:(h + 1) * G]).T
             assert_attention_close(o_g, lse_g, o_ref, lse_ref, dtype, f"unit {b},{h}")
