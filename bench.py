@@ -319,12 +319,12 @@ def prefill_bench(args, rank, world, device):
     assert L.lte_read_device_error(bufs.ws) == (0, 0)
 
     # e2e: pinned host buffers, H2D of the inputs and D2H of o inside the timed
-    # region, through layer.HostPrefill (sub-batches of 8 sequences: the copies
+    # region, through layer.HostPrefill (sub-batches of 4 sequences: the copies
     # in and out overlap each other and the compute)
     hq, hk, hv, hm = (x.pin_memory() for x in (q, k, v, mask))
     ho = torch.empty(bufs.o.shape, dtype=bufs.o.dtype).pin_memory()
     n_e2e = max(3, min(args.steps, 10))
-    hp = layer.HostPrefill(B, T, Hq, Hkv, D, torch.bfloat16, p, chunk=8 if B % 8 == 0 else B,
+    hp = layer.HostPrefill(B, T, Hq, Hkv, D, torch.bfloat16, p, chunk=4 if B % 4 == 0 else B,
                            device=device)
     hp.run(hq, hk, hv, hm, ho, stream)
     torch.cuda.synchronize()
@@ -586,7 +586,7 @@ def main():
             "e2e": {"value": DI.job_throughput(pf["B"] * pf["T"], world, pf["e2e_ms"] / 1e3),
                     "unit": "tokens/s",
                     "h2d_bytes_per_step": pf["h2d"], "d2h_bytes_per_step": pf["d2h"],
-                    "path": "layer.HostPrefill: sub-batches of 8 sequences, copies in/out "
+                    "path": "layer.HostPrefill: sub-batches of 4 sequences, copies in/out "
                             "overlapping the compute", "o_equals_device_step": pf["e2e_ok"]},
             "gpu_launches": pf["launches"] + (dec["launches"] if dec else 0),
         }
