@@ -12,9 +12,11 @@
 // the state in TMEM.  This file holds the recurrent decode step and the
 // dispatch.
 //
-// Decode: one CTA per (batch, head) streams the 128x128 fp32 state once
-// (read, decay, add the outer product, write) with 16-byte accesses and
-// reduces the row-query dot products with warp shuffles.
+// Decode: two CTAs of four warps per (batch, head), one per half of the value
+// rows, stream the 128x128 fp32 state once (read, decay, add the outer
+// product, write) with 16-byte accesses and reduce the row-query dot products
+// with warp shuffles.  (Twice as many, smaller CTAs spread the states evenly
+// over the SMs: with one CTA per state, 3 or 4 states land on each SM.)
 #include <math.h>
 
 #include "lte_common.cuh"
@@ -27,11 +29,12 @@ constexpr int DK = 128, DV = 128;
 
 // ---------------------------------------------------------------- decode
 template <typename TIn>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
                   const TIn* __restrict__ v, const float* __restrict__ a, TIn* __restrict__ o,
                   float* __restrict__ state) {
-  const int bh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x >> 1, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row0 = (blockIdx.x & 1) * (DV / 2);       // this CTA's half of the value rows
   const long long vb = (long long)bh * DK;
   float q4[4], k4[4], a4[4];
 #pragma unroll
@@ -41,20 +44,20 @@ gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
     a4[e] = a[vb + lane * 4 + e];
   }
   float* st = state + (long long)bh * DV * DK;
-  constexpr int kRows = DV / 8;                       // rows per warp
+  constexpr int kRows = 16;                           // rows per warp (4 warps per half)
   // every row's loads first (16 x 512 B in flight per warp), then update and store
   float4 s4[kRows];
   float vi[kRows];
 #pragma unroll
   for (int rr = 0; rr < kRows; ++rr) {
-    const int i = warp * kRows + rr;
+    const int i = row0 + warp * kRows + rr;
     s4[rr] = reinterpret_cast<const float4*>(st + (long long)i * DK)[lane];
     vi[rr] = to_f32(v[(long long)bh * DV + i]);
   }
   float d[kRows];
 #pragma unroll
   for (int rr = 0; rr < kRows; ++rr) {
-    const int i = warp * kRows + rr;
+    const int i = row0 + warp * kRows + rr;
     float4 x = s4[rr];
     x.x = fmaf(x.x, a4[0], vi[rr] * k4[0]);
     x.y = fmaf(x.y, a4[1], vi[rr] * k4[1]);
@@ -81,7 +84,7 @@ gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
   if ((lane & 1) == 0) {
     const int row = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
                     ((lane >> 1) & 1);
-    o[(long long)bh * DV + warp * kRows + row] = from_f32<TIn>(d[0]);
+    o[(long long)bh * DV + row0 + warp * kRows + row] = from_f32<TIn>(d[0]);
   }
 }
 
@@ -100,11 +103,11 @@ cudaError_t gla_decode(int B, int H, int dk, int dv, int dtype, const void* q, c
                        cudaStream_t stream) {
   if (dk != gla::DK || dv != gla::DV) return cudaErrorNotSupported;
   if (dtype == LTE_BF16)
-    gla::gla_decode_kernel<__nv_bfloat16><<<B * H, 256, 0, stream>>>(
+    gla::gla_decode_kernel<__nv_bfloat16><<<B * H * 2, 128, 0, stream>>>(
         H, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a,
         (__nv_bfloat16*)o, state);
   else
-    gla::gla_decode_kernel<float><<<B * H, 256, 0, stream>>>(
+    gla::gla_decode_kernel<float><<<B * H * 2, 128, 0, stream>>>(
         H, (const float*)q, (const float*)k, (const float*)v, a, (float*)o, state);
   return cudaGetLastError();
 }
