@@ -7,14 +7,17 @@
 // out-of-window cache segment has capped capacity and holds the sink and the
 // LTE-retained KVs).
 //
-// compact_kernel: one CTA per (batch, KV head) unit walks the tokens in
-// rounds of one thread per token.  A warp ballot gives each retained token
-// its rank inside the warp, a 32-entry scan over warp totals gives the warp
-// offsets, and a running carry links the rounds.  This yields the ascending
-// retained-position list idx, its length, and the inclusive prefix counts
-// cnt.  The same CTA then copies the sink rows and the retained rows into a
-// contiguous column segment with 16-byte vector loads, so the attention
-// kernels read the "column" keys as dense tiles.
+// compact_kernel: kCompactSplit CTAs per (batch, KV head) unit.  Each walks
+// all of the unit's tokens in rounds of one thread per token (the mask is a
+// few KiB): a warp ballot gives each retained token its rank inside the warp,
+// a 32-entry scan over warp totals gives the warp offsets, and a running carry
+// links the rounds.  This yields the ascending retained-position list idx, its
+// length, and the inclusive prefix counts cnt; CTA part p writes the entries
+// of its p-th share of the rounds.  Each CTA then copies the retained rows of
+// those rounds (whose idx entries it wrote itself), and part 0 the sink rows,
+// into a contiguous column segment with 16-byte vector loads, so the
+// attention kernels read the "column" keys as dense tiles.  (Splitting a unit
+// over several CTAs spreads the copy over more SMs than there are units.)
 #include <math.h>
 
 #include "lte_common.cuh"
@@ -23,6 +26,7 @@
 namespace lte {
 
 constexpr int kCompactThreads = 1024;
+constexpr int kCompactSplit = 4;   // CTAs per unit
 
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                          int nvec, int lane_in_row) {
@@ -38,17 +42,35 @@ compact_kernel(int T, int Hkv, int sink, int n_scored, float tau, const float* _
   __shared__ int warp_tot[32];
   __shared__ int warp_off[32];
   __shared__ int round_total;
-  const int u = blockIdx.x, b = u / Hkv, h = u % Hkv;
+  const int u = blockIdx.x / kCompactSplit, part = blockIdx.x % kCompactSplit;
+  const int b = u / Hkv, h = u % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_rounds = (T + kCompactThreads - 1) / kCompactThreads;
+  const int r_lo = (int)((long long)n_rounds * part / kCompactSplit);
+  const int r_hi = (int)((long long)n_rounds * (part + 1) / kCompactSplit);
   const long long row0 = (long long)u * T;
   const unsigned lt_mask = (1u << lane) - 1u;
 
-  int carry = 0;
-  for (int base = 0; base < T; base += kCompactThreads) {
+  int carry = 0, own_lo = 0, own_hi = 0;                 // retained ordinals of this CTA's rounds
+  constexpr int kAhead = 8;                              // rounds whose decisions load together
+  bool mk[kAhead];
+  for (int base = 0, rnd = 0; base < T; base += kCompactThreads, ++rnd) {
+    if (rnd % kAhead == 0) {                             // this thread's next kAhead decisions
+#pragma unroll
+      for (int a = 0; a < kAhead; ++a) {
+        const int jj = base + a * kCompactThreads + tid;
+        mk[a] = false;
+        if (jj < T && jj >= sink && jj < n_scored)
+          mk[a] = mask ? (mask[row0 + jj] != 0) : (r[row0 + jj] >= tau);
+      }
+    }
+    const bool mine = rnd >= r_lo && rnd < r_hi;          // rounds whose entries this CTA writes
+    if (rnd == r_lo) own_lo = carry;
     const int j = base + tid;
     bool m = false;
-    if (j < T && j >= sink && j < n_scored)
-      m = mask ? (mask[row0 + j] != 0) : (r[row0 + j] >= tau);
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a)
+      if (a == rnd % kAhead) m = mk[a];
     const unsigned ballot = __ballot_sync(0xffffffffu, m);
     if (lane == 0) warp_tot[warp] = __popc(ballot);
     __syncthreads();
@@ -65,25 +87,29 @@ compact_kernel(int T, int Hkv, int sink, int n_scored, float tau, const float* _
     }
     __syncthreads();
     const int pos = carry + warp_off[warp] + __popc(ballot & lt_mask);
-    if (m) idx[row0 + pos] = j;
-    if (j < T) cnt[row0 + j] = pos + (m ? 1 : 0);
+    if (mine && m) idx[row0 + pos] = j;
+    if (mine && j < T) cnt[row0 + j] = pos + (m ? 1 : 0);
     carry += round_total;
+    if (rnd == r_hi - 1) own_hi = carry;
     __syncthreads();
   }
-  if (tid == 0) nret[u] = carry;
+  if (r_lo >= r_hi) own_lo = own_hi = carry;
+  if (tid == 0 && part == 0) nret[u] = carry;
   if (k_col == nullptr) return;
-  __syncthreads();   // idx written above is visible to the whole CTA
+  __syncthreads();   // this CTA's idx entries are visible to all of its threads
 
   // column segment: slot i < sink <- row i; slot sink + i <- row idx[i]
   const int nvec = D * elt / 16;
   const int rows_per_pass = kCompactThreads / nvec;
   const int rr = tid / nvec, lane_in_row = tid % nvec;
-  const int nsink = sink < T ? sink : T;
-  const int total = nsink + carry;
+  const int nsink = (part == 0) ? (sink < T ? sink : T) : 0;
+  const int total = nsink + (own_hi - own_lo);
   const long long col0 = (long long)u * (sink + T);
+  // rows: the sinks (part 0), then retained ordinals [own_lo, own_hi)
   for (int i = rr; i < total; i += rows_per_pass) {
-    const int j = (i < nsink) ? i : idx[row0 + (i - nsink)];
-    const int slot = (i < nsink) ? i : sink + (i - nsink);
+    const int o = own_lo + (i - nsink);
+    const int j = (i < nsink) ? i : idx[row0 + o];
+    const int slot = (i < nsink) ? i : sink + o;
     const long long src = ((long long)b * s.b + (long long)j * s.t + (long long)h * s.h) * elt;
     const long long dst = (col0 + slot) * D * elt;
     copy_row(reinterpret_cast<const uint4*>(k + src), reinterpret_cast<uint4*>(k_col + dst), nvec,
@@ -98,7 +124,7 @@ cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask
                           const void* v, Strides4 s, void* k_col, void* v_col,
                           cudaStream_t stream) {
   const int elt = d->dtype == LTE_BF16 ? 2 : 4;
-  compact_kernel<<<d->B * d->Hkv, kCompactThreads, 0, stream>>>(
+  compact_kernel<<<d->B * d->Hkv * kCompactSplit, kCompactThreads, 0, stream>>>(
       d->T, d->Hkv, d->sink, n_scored, d->tau, r, mask, idx, nret, cnt, (const char*)k,
       (const char*)v, s, elt, d->D, (char*)k_col, (char*)v_col);
   return cudaGetLastError();
