@@ -28,7 +28,9 @@ Readings taken where the pages are silent (each is restated where used):
   tokens qualify, the C most recent are kept (FIFO ring) -- policy "recent".
   The pages leave the capped segment's policy open; policy "first" keeps the
   first C retained tokens instead (later ones are dropped once the segment is
-  full);
+  full); policy "lowest" drops, when a retained token arrives at a full
+  segment, the one with the lowest retention score among the C held and the
+  newcomer (equal scores: the older token goes);
 * retain iff r >= tau; the first s tokens are sinks and are never "retained";
 * CNN: conv1d over the channel concatenation [k; v] (k first), PyTorch
   cross-correlation convention, per-layer zero padding outside [0, n), a
@@ -181,24 +183,45 @@ def compact(m) -> tuple[np.ndarray, int, np.ndarray]:
 # (3) attended set and attention  [LTE, Fig. 2 right: A-plus-column pattern]
 # ---------------------------------------------------------------------------
 
-CAP_RECENT, CAP_FIRST = "recent", "first"     # policies of the capped segment
+CAP_RECENT, CAP_FIRST, CAP_LOWEST = "recent", "first", "lowest"   # capped-segment policies
+
+
+def top_by_score(candidates, r, cap: int) -> list[int]:
+    """The `cap` candidates j with the largest (r_j, j), i.e. the highest
+    retention scores, the later token first among equal scores.
+
+    This is what policy "lowest" holds after the candidates have arrived one by
+    one (in position order) at a segment of capacity C that, when full, drops
+    the lowest-scoring of its C tokens and the newcomer: a token is dropped
+    exactly when C others that beat it have arrived, so the survivors are the
+    C best of all arrivals.  ``test_oracle_sets`` checks this against the
+    arrival-by-arrival simulation."""
+    ranked = sorted(candidates, key=lambda j: (float(r[j]), j), reverse=True)
+    return ranked[:cap]
 
 
 def attended_set(t: int, m, sink: int, window: int, cap: int,
-                 policy: str = CAP_RECENT) -> list[int]:
+                 policy: str = CAP_RECENT, r=None) -> list[int]:
     """Key positions query t attends to, for one KV head.
 
     S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t, with Ret_t drawn from the
     tokens j in [s, t-w] with m_j = 1 (kept when they left the window):
     policy "recent": the `cap` largest such j (the C most recent);
     policy "first":  the `cap` smallest such j (the segment fills, then later
-    retained tokens are dropped).
+    retained tokens are dropped);
+    policy "lowest": the `cap` such j with the highest scores r_j (the
+    lowest-scoring token is dropped when the segment overflows; `r` required).
     """
     keys = set(range(0, min(sink, t + 1)))
     keys |= set(range(max(0, t - window + 1), t + 1))
     candidates = [j for j in range(sink, t - window + 1) if m[j]]
     if cap > 0:
-        keys |= set(candidates[-cap:] if policy == CAP_RECENT else candidates[:cap])
+        if policy == CAP_RECENT:
+            keys |= set(candidates[-cap:])
+        elif policy == CAP_FIRST:
+            keys |= set(candidates[:cap])
+        else:
+            keys |= set(top_by_score(candidates, r, cap))
     return sorted(keys)
 
 
@@ -219,12 +242,13 @@ def attend(q_rows, K, V, scale: float):
 
 
 def prefill_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
-                 rows=None, policy: str = CAP_RECENT):
+                 rows=None, policy: str = CAP_RECENT, r=None):
     """Prefill of one (batch element, KV head) unit.
 
     q [T, G, D] (the G query heads that share this KV head), k, v [T, D],
-    m [T] retention mask.  Returns o [T, G, D], lse [T, G] and the attended
-    count per row (rows not in `rows` are left as NaN / -1).
+    m [T] retention mask, r [T] retention scores (policy "lowest" only).
+    Returns o [T, G, D], lse [T, G] and the attended count per row (rows not
+    in `rows` are left as NaN / -1).
     """
     T, G, D = q.shape
     o = np.full((T, G, v.shape[1]), np.nan)
@@ -233,15 +257,16 @@ def prefill_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
     k = _f64(k)
     v = _f64(v)
     for t in (range(T) if rows is None else rows):
-        S = attended_set(t, m, sink, window, cap, policy)
+        S = attended_set(t, m, sink, window, cap, policy, r)
         o[t], lse[t] = attend(q[t], k[S], v[S], scale)
         count[t] = len(S)
     return o, lse, count
 
 
 def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | None = None,
-            policy: str = CAP_RECENT):
-    """Prefill over a batch: q [B,T,Hq,D], k, v [B,T,Hkv,D], masks [B,Hkv,T].
+            policy: str = CAP_RECENT, r=None):
+    """Prefill over a batch: q [B,T,Hq,D], k, v [B,T,Hkv,D], masks [B,Hkv,T]
+    (and scores r [B,Hkv,T] under policy "lowest").
 
     GQA: query head qh uses KV head qh // (Hq // Hkv).  Returns o [B,T,Hq,D],
     lse [B,Hq,T], count [B,Hkv,T].
@@ -257,7 +282,8 @@ def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | Non
     for b in range(B):
         for h in range(Hkv):
             ou, lu, cu = prefill_unit(q[b, :, h * G:(h + 1) * G], k[b, :, h], v[b, :, h],
-                                      masks[b, h], sink, window, cap, scale, policy=policy)
+                                      masks[b, h], sink, window, cap, scale, policy=policy,
+                                      r=None if r is None else r[b, h])
             o[b, :, h * G:(h + 1) * G] = ou
             lse[b, h * G:(h + 1) * G] = lu.T
             count[b, h] = cu
@@ -280,7 +306,10 @@ class DecodeCache:
       (0-based) goes to slot i mod C, overwriting the oldest one (the cap
       keeps the C most recent).  Policy "first": the i-th retained token goes
       to slot i while i < C and is dropped afterwards (ret_total then counts
-      the stored tokens);
+      the stored tokens).  Policy "lowest": the i-th retained token goes to
+      slot i while i < C; afterwards it replaces the held token with the
+      lowest (score, position) unless its own score is lower (ret_total counts
+      the stored tokens; ret_r holds their scores);
     * r of window tokens, filled by deferred batched scoring.
     """
     D: int
@@ -300,6 +329,7 @@ class DecodeCache:
     ret_k: np.ndarray = field(init=False)
     ret_v: np.ndarray = field(init=False)
     ret_pos: np.ndarray = field(init=False)
+    ret_r: np.ndarray = field(init=False)     # score of each retained slot's token
     ret_total: int = 0
     t: int = 0              # tokens received so far
     n_scored: int = 0       # tokens [0, n_scored) have a score
@@ -314,6 +344,7 @@ class DecodeCache:
         self.sink_pos = np.full(s, -1, dtype=np.int64)
         self.ret_k = np.zeros((C, D)); self.ret_v = np.zeros((C, D))
         self.ret_pos = np.full(C, -1, dtype=np.int64)
+        self.ret_r = np.full(C, np.nan)
 
     # -- deferred scoring ---------------------------------------------------
     def _score_from_window(self, j: int) -> float:
@@ -359,14 +390,23 @@ class DecodeCache:
                 assert leaving < self.n_scored, "token left the window unscored"
                 r = self.win_r[slot]
                 keep = r >= self.tau and self.cap > 0
-                if keep and self.policy == CAP_FIRST and self.ret_total >= self.cap:
+                rs = self.ret_total % self.cap if self.cap > 0 else 0
+                full = self.ret_total >= self.cap
+                if keep and self.policy == CAP_FIRST and full:
                     keep = False                     # the segment is full: dropped
+                if keep and self.policy == CAP_LOWEST and full:
+                    # drop the lowest (score, position) of the held tokens and the
+                    # newcomer; the newcomer is the latest, so it stays iff its
+                    # score is not below the lowest held score
+                    rs = min(range(self.cap), key=lambda i: (self.ret_r[i], self.ret_pos[i]))
+                    keep = r >= self.ret_r[rs]
                 if keep:
-                    rs = self.ret_total % self.cap
                     self.ret_k[rs] = self.win_k[slot]
                     self.ret_v[rs] = self.win_v[slot]
                     self.ret_pos[rs] = leaving
-                    self.ret_total += 1
+                    self.ret_r[rs] = r
+                    if not (self.policy == CAP_LOWEST and full):
+                        self.ret_total += 1
         slot = t % w
         self.win_k[slot] = _f64(k_t); self.win_v[slot] = _f64(v_t)
         self.win_pos[slot] = t; self.win_r[slot] = np.nan
@@ -423,13 +463,14 @@ def decode_unit(q, k, v, T0: int, sink: int, window: int, cap: int, tau: float,
 
 
 def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int,
-                       policy: str = CAP_RECENT):
+                       policy: str = CAP_RECENT, r=None):
     """The cache contents after a prompt of T0 tokens, read off the prefill
     mask: window = positions (T0-1-w, T0-1], sinks = j < s with j <= T0-1-w,
     retained = the C most recent j in [s, T0-1-w] with m_j = 1, with the
     i-th retained token (0-based over all retained) in ring slot i mod C
     (policy "first": the C earliest such j, the i-th in slot i, and ret_total
-    counts the stored ones).
+    counts the stored ones; policy "lowest": the C such j with the highest
+    scores, in position order in slots 0, 1, ..., ret_total = their number).
 
     Returns dict of position arrays (-1 = empty) and ret_total.
     """
@@ -443,6 +484,8 @@ def cache_after_prompt(k, v, m, T0: int, sink: int, window: int, cap: int,
     ret = [j for j in range(sink, last_out + 1) if m[j]]
     if policy == CAP_FIRST:
         ret = ret[:cap]
+    elif policy == CAP_LOWEST:
+        ret = sorted(top_by_score(ret, r, cap))
     ret_pos = np.full(cap, -1, dtype=np.int64)
     for i, j in enumerate(ret):
         if cap > 0:

@@ -28,12 +28,13 @@ def _inputs(B, Hq, Hkv, D, T_total, seed, w_std):
 
 
 def _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, score_batch, check_every=0,
-                cap_policy=0):
+                cap_policy=0, past1=2, past2=1):
     """Prefill the prompt on the GPU, set up the cache, decode the rest.
     Returns o [steps,B,Hq,D], lse [steps,B,Hq], retained sets at checkpoints."""
     B, T_total, Hq, D = q.shape
     Hkv = k.shape[2]
-    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=tau, cap_policy=cap_policy)
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=tau, cap_policy=cap_policy,
+                          past1=past1, past2=past2)
     qd, kd, vd = (x.cuda() for x in (q, k, v))
     cd = tuple(x.cuda() for x in cnn)
     kp, vp = kd[:, :T0].contiguous(), vd[:, :T0].contiguous()
@@ -120,6 +121,32 @@ def test_decode_cap_first_policy(layer, cfg):
         for t, rs in rets.items():
             assert rs[b][h] == ret_ref[t - T0], (b, h, t)
         assert len(ret_ref[-1]) <= cap
+
+
+@pytest.mark.parametrize("score_batch", [1, 8])
+def test_decode_causal_cnn(layer, score_batch):
+    """A CNN that reads the past only (past1 = k1 - 1, past2 = k2 - 1): every
+    token is scored as it arrives, with no deferral; outputs and retained sets
+    against the oracle's simulation with the same taps."""
+    B, Hq, Hkv, D, sink, window, cap, T0, steps = 2, 8, 2, 128, 4, 48, 12, 150, 90
+    T = T0 + steps
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 77, w_std=0.1)
+    G = Hq // Hkv
+    r_or = {(b, h): O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h, 4, 2))
+            for b in range(B) for h in range(Hkv)}
+    tau, margin = clean_tau(np.stack(list(r_or.values())))
+    assert margin > 1e-5
+    o_g, lse_g, rets, _, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0,
+                                         score_batch, check_every=11, past1=4, past2=2)
+    for b in range(B):
+        for h in range(Hkv):
+            o_ref, lse_ref, sets, ret_ref, _ = O.decode_unit(
+                f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]), f64(v[b, :, h]), T0, sink,
+                window, cap, tau, oracle_cnn(cnn, h, 4, 2), score_batch, scale_of(D))
+            assert_attention_close(f64(o_g[:, b, h * G:(h + 1) * G]), f64(lse_g[:, b, h * G:(h + 1) * G]),
+                                   o_ref, lse_ref, torch.bfloat16, f"unit {b},{h}")
+            for t, rs in rets.items():
+                assert rs[b][h] == ret_ref[t - T0], (b, h, t)
 
 
 def test_decode_split_kv_path(layer):

@@ -1,7 +1,7 @@
 """Pins for the oracle's decode cache simulation (no GPU).
 
 The simulation holds the inference cache slot by slot (window ring, sink
-slots, retained ring under either cap policy, scores computed from the
+slots, retained ring under each cap policy, scores computed from the
 window in deferred batches).  It is an independent formulation of the prefill set formula, so
 the two are checked against each other: every decode output equals the
 prefill row of the concatenated sequence, for several scoring batch sizes.
@@ -28,7 +28,7 @@ def _setup(seed, T=90, D=6, G=2, C1=4):
                                           (2, 0, 9, 5, 30), (3, 3, 10, 0, 15),
                                           (4, 2, 7, 100, 1)])
 @pytest.mark.parametrize("score_batch", [1, 3])
-@pytest.mark.parametrize("policy", [O.CAP_RECENT, O.CAP_FIRST])
+@pytest.mark.parametrize("policy", [O.CAP_RECENT, O.CAP_FIRST, O.CAP_LOWEST])
 def test_decode_equals_prefill(seed, s, w, C, T0, score_batch, policy):
     q, k, v, cnn = _setup(seed)
     T = k.shape[0]
@@ -40,12 +40,12 @@ def test_decode_equals_prefill(seed, s, w, C, T0, score_batch, policy):
                                               policy=policy)
     r = O.cnn_scores(k, v, cnn)
     m = O.retention_mask(r, s, tau)
-    o_p, lse_p, _ = O.prefill_unit(q, k, v, m, s, w, C, scale, policy=policy)
+    o_p, lse_p, _ = O.prefill_unit(q, k, v, m, s, w, C, scale, policy=policy, r=r)
     for i, t in enumerate(range(T0, T)):
-        assert sets[i] == O.attended_set(t, m, s, w, C, policy), t
+        assert sets[i] == O.attended_set(t, m, s, w, C, policy, r), t
         np.testing.assert_allclose(o_d[i], o_p[t], atol=1e-12, rtol=0)
         np.testing.assert_allclose(lse_d[i], lse_p[t], atol=1e-12, rtol=0)
-        ret = [j for j in O.attended_set(t, m, s, w, C, policy) if s <= j <= t - w]
+        ret = [j for j in O.attended_set(t, m, s, w, C, policy, r) if s <= j <= t - w]
         assert rets[i] == ret
 
 
@@ -61,7 +61,7 @@ def test_scoring_batch_invariance():
         assert sets == outs[0][1] and rets == outs[0][2]
 
 
-@pytest.mark.parametrize("policy", [O.CAP_RECENT, O.CAP_FIRST])
+@pytest.mark.parametrize("policy", [O.CAP_RECENT, O.CAP_FIRST, O.CAP_LOWEST])
 def test_cache_after_prompt_matches_simulation(policy):
     q, k, v, cnn = _setup(5, T=70)
     s, w, C, tau = 3, 11, 4, 0.5
@@ -70,10 +70,13 @@ def test_cache_after_prompt_matches_simulation(policy):
     for T0 in (1, 5, 11, 12, 20, 47, 70):
         *_, cache = O.decode_unit(q[:T0], k[:T0], v[:T0], T0, s, w, C, tau, cnn, 1, 0.3,
                                   policy=policy)
-        st = O.cache_after_prompt(k, v, m, T0, s, w, C, policy)
+        st = O.cache_after_prompt(k, v, m, T0, s, w, C, policy, r)
         np.testing.assert_array_equal(st["win_pos"], cache.win_pos)
         np.testing.assert_array_equal(st["sink_pos"], cache.sink_pos)
-        np.testing.assert_array_equal(st["ret_pos"], cache.ret_pos)
+        if policy == O.CAP_LOWEST:      # replacements land in the dropped token's slot
+            assert sorted(st["ret_pos"]) == sorted(cache.ret_pos)
+        else:
+            np.testing.assert_array_equal(st["ret_pos"], cache.ret_pos)
         assert st["ret_total"] == cache.ret_total
 
 

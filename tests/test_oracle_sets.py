@@ -41,6 +41,33 @@ def brute_member_first(j, t, m, s, w, C):
     return older < C
 
 
+def brute_member_lowest(j, t, m, r, s, w, C):
+    """Policy "lowest": a retained token that left the window survives iff
+    fewer than C of the retained tokens that left the window by row t beat
+    it (a higher score, or an equal score and a later position)."""
+    if j > t or j < 0:
+        return False
+    if j < s or j > t - w:
+        return True
+    if not m[j]:
+        return False
+    better = sum(1 for i in range(s, t - w + 1)
+                 if m[i] and i != j and (r[i] > r[j] or (r[i] == r[j] and i > j)))
+    return better < C
+
+
+def arrivals_lowest(order, r, C):
+    """The segment after the tokens of `order` arrive one at a time: each is
+    appended and, past C entries, the entry with the lowest (score, position)
+    is removed (which may be the newcomer)."""
+    held = []
+    for j in order:
+        held.append(j)
+        if len(held) > C:
+            held.remove(min(held, key=lambda i: (r[i], i)))
+    return sorted(held)
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_attended_set_vs_bruteforce(seed):
     rng = np.random.default_rng(seed)
@@ -87,6 +114,59 @@ def test_first_policy_closed_forms():
         ret = [j for j in S if s <= j <= t - w]
         assert ret == list(range(s, s + min(C, n)))
         assert len(S) == min(t + 1, w) + len([j for j in range(s) if j <= t - w]) + min(C, n)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_attended_set_lowest_policy_vs_bruteforce(seed):
+    """Scores drawn from a few levels, so that equal scores occur often."""
+    rng = np.random.default_rng(200 + seed)
+    for _ in range(25):
+        T = int(rng.integers(1, 48))
+        s = int(rng.integers(0, 5))
+        w = int(rng.integers(1, 14))
+        C = int(rng.choice([0, 1, 2, 3, 8, 100]))
+        r = rng.integers(0, 5, T) / 4.0
+        m = O.retention_mask(r, s, float(rng.choice([0.0, 0.25, 0.5])))
+        for t in range(T):
+            S = O.attended_set(t, m, s, w, C, O.CAP_LOWEST, r)
+            ref = [j for j in range(T) if brute_member_lowest(j, t, m, r, s, w, C)]
+            assert S == ref, (T, s, w, C, t)
+            if C >= T:                       # the cap never binds: all policies agree
+                assert S == O.attended_set(t, m, s, w, C, O.CAP_RECENT)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_lowest_top_scores_equal_arrivals(seed):
+    """The closed form (the C best of all arrivals) equals the segment built
+    arrival by arrival with a drop of the lowest (score, position)."""
+    rng = np.random.default_rng(300 + seed)
+    for _ in range(40):
+        n = int(rng.integers(0, 60))
+        C = int(rng.integers(1, 12))
+        r = rng.integers(0, int(rng.choice([3, 50])), n) / 7.0
+        order = list(range(n))
+        for k in range(n + 1):
+            assert sorted(O.top_by_score(order[:k], r, C)) == arrivals_lowest(order[:k], r, C)
+
+
+def test_lowest_policy_closed_forms():
+    """Scores rising with position: the lowest is always the oldest, so the
+    segment is the C most recent (policy "recent"); falling scores: the
+    newcomer is always the lowest, so the first C stay (policy "first")."""
+    T, s, w, C = 110, 3, 9, 6
+    ones = O.fed_mask(np.ones(T, np.uint8), s)
+    up = np.linspace(0.1, 0.9, T)
+    down = up[::-1].copy()
+    for t in range(T):
+        assert (O.attended_set(t, ones, s, w, C, O.CAP_LOWEST, up) ==
+                O.attended_set(t, ones, s, w, C, O.CAP_RECENT))
+        assert (O.attended_set(t, ones, s, w, C, O.CAP_LOWEST, down) ==
+                O.attended_set(t, ones, s, w, C, O.CAP_FIRST))
+    # equal scores everywhere: ties go against the older token, as in "recent"
+    flat = np.full(T, 0.5)
+    for t in range(T):
+        assert (O.attended_set(t, ones, s, w, C, O.CAP_LOWEST, flat) ==
+                O.attended_set(t, ones, s, w, C, O.CAP_RECENT))
 
 
 def test_closed_forms():
