@@ -65,8 +65,15 @@ typedef enum { LTE_F32 = 0, LTE_BF16 = 1 } lte_dtype;
  * capacity; the pages leave the policy open.]
  *   LTE_CAP_RECENT: the C most recent (a ring; the oldest is overwritten);
  *   LTE_CAP_FIRST:  the first C (later retained tokens are dropped once the
- *                   segment is full). */
-typedef enum { LTE_CAP_RECENT = 0, LTE_CAP_FIRST = 1 } lte_cap_policy;
+ *                   segment is full);
+ *   LTE_CAP_LOWEST: when a retained token arrives at a full segment, the
+ *                   token with the lowest (score r, position) among the C
+ *                   held and the newcomer is dropped -- equal scores drop the
+ *                   older token.  The segment then holds the C retained
+ *                   tokens with the highest (r, position) so far.  Needs the
+ *                   scores: prefill takes lifetimes from
+ *                   lte_retained_lifetimes, the decode cache its ret_r. */
+typedef enum { LTE_CAP_RECENT = 0, LTE_CAP_FIRST = 1, LTE_CAP_LOWEST = 2 } lte_cap_policy;
 
 /* Shapes and method parameters of one LTE layer.
  * sink = s >= 0, window = w >= 1, cap = C >= 0 (retained tokens only; sinks
@@ -135,16 +142,40 @@ lte_status lte_evict_compact(const lte_dims* d, const float* r, const uint8_t* m
                              void* k_col, void* v_col, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * lte_retained_lifetimes -- for LTE_CAP_LOWEST, the retained counts during
+ * which each retained token is held.  [LTE paper, Fig. 3 caption: capped
+ * out-of-window segment; the drop-the-lowest-score reading of the cap.]
+ * Token i of the compacted list (0-based, position idx[i], score
+ * r[idx[i]]) is beaten by token i' != i when r[idx[i']] > r[idx[i]], or the
+ * scores are equal and i' > i.  Then, per (b, KV head) unit:
+ *   death[i] = the smallest n > i such that at least C of the tokens
+ *              0 .. n-1 beat token i, or T + 1 if there is none;
+ * the segment holds token i exactly while the retained count n satisfies
+ * i < n < death[i].  r: fp32 [B,Hkv,T] (the scores behind the mask);
+ * idx, nret from lte_evict_compact; death: int32 [B,Hkv,T], entries
+ * i >= nret left unwritten.  Requires d->cap_policy == LTE_CAP_LOWEST.
+ * Work: O(nret^2) comparisons per unit, none when nret <= C.
+ * ------------------------------------------------------------------------- */
+lte_status lte_retained_lifetimes(const lte_dims* d, const float* r, const int32_t* idx,
+                                  const int32_t* nret, int32_t* death, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lte_sparse_attn_prefill -- causal softmax attention of every query over its
  * per-KV-head attended set.  [LTE paper, Fig. 2 caption (right): per-head
  * A-plus-column sparsity pattern: sink and window form the "A", retained
  * tokens the "columns".]
  * For row t, KV head h, n_t = (t >= w) ? cnt[t - w] : 0:
- *   S_t = { j < s : j <= t - w }  u  (t - w, t]  u  { idx[i] : max(0, n_t - C) <= i < n_t }
+ *   S_t = { j < s : j <= t - w }  u  (t - w, t]  u  { idx[i] : i in R_t }, where
+ *   R_t = [max(0, n_t - C), n_t)               under LTE_CAP_RECENT,
+ *         [0, min(n_t, C))                     under LTE_CAP_FIRST,
+ *         { i < n_t : death[i] > n_t }         under LTE_CAP_LOWEST;
  *   o[t,q] = sum_{j in S_t} softmax_j(scale * q_t . k_j) v_j,
  *   lse[q,t] = log sum_{j in S_t} exp(scale * q_t . k_j)   (natural log).
  * q, o: [B,T,Hq,D]; k, v: [B,T,Hkv,D]; cnt from lte_evict_compact; k_col,
- * v_col: the column segment written by lte_evict_compact (required).
+ * v_col: the column segment written by lte_evict_compact (required); death:
+ * from lte_retained_lifetimes, required under LTE_CAP_LOWEST, else ignored.
+ * Under LTE_CAP_LOWEST every row scans retained slots [0, n_t), so its cost
+ * grows with n_t rather than with C once the cap binds.
  * lse (nullable): fp32 [B,Hq,T].  bf16 inputs: fp32 accumulation, P rounded
  * to bf16 for the PV product, o rounded to bf16 (round-to-nearest-even).
  * Workspace: lte_workspace_bytes(d, LTE_WS_PREFILL) bytes (16-byte aligned,
@@ -153,7 +184,7 @@ lte_status lte_evict_compact(const lte_dims* d, const float* r, const uint8_t* m
 lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void* k,
                                    const void* v, const lte_strides* q_strides,
                                    const lte_strides* kv_strides, const int32_t* cnt,
-                                   const void* k_col, const void* v_col,
+                                   const int32_t* death, const void* k_col, const void* v_col,
                                    void* o, const lte_strides* o_strides, float* lse,
                                    void* workspace, size_t ws_bytes, void* stream);
 
@@ -166,39 +197,57 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
  *   k, v     [B, Hkv, L, D] (dtype): slots [0,w) window ring (token j in slot
  *            j mod w), [w, w+s) sinks (token j < s in slot w+j once it left
  *            the window), [w+s, w+s+C) retained ring (the i-th retained token
- *            of the unit, 0-based, in slot w+s+(i mod C));
+ *            of the unit, 0-based, in slot w+s+(i mod C); under
+ *            LTE_CAP_FIRST and LTE_CAP_LOWEST slots fill in order and never
+ *            wrap, and under LTE_CAP_LOWEST a newcomer takes the slot of the
+ *            token it displaces);
  *   pos      int32 [B, Hkv, L]: token position held by each slot, -1 = empty;
  *   win_r    fp32  [B, Hkv, w]: score of the token in each window slot;
- *   ret_total int32 [B, Hkv]: tokens retained so far (the ring's write count);
+ *   ret_total int32 [B, Hkv]: tokens retained so far (the ring's write count;
+ *            the number held, at most C, under LTE_CAP_FIRST / LOWEST);
  *   meta     int32 [4]: {t = tokens held so far, n_scored = tokens [0,n_scored)
- *            have a score, internal, internal}. */
+ *            have a score, internal, internal};
+ *   ret_r    fp32  [B, Hkv, C]: score of the token in each retained slot
+ *            (required under LTE_CAP_LOWEST, else may be NULL). */
 typedef struct {
   void *k, *v;
   int32_t* pos;
   float* win_r;
   int32_t* ret_total;
   int32_t* meta;
+  float* ret_r;
 } lte_cache;
 
 /* lte_cache_init_from_prefill -- fill an empty cache with the state after a
  * prompt of T_prompt tokens (T_prompt <= d->T):
  * window = tokens (T_prompt-1-w, T_prompt-1], sinks that left the window,
- * retained = idx[max(0,n-C) .. n) with n = cnt[T_prompt-1-w] (0 if negative),
+ * with n = cnt[T_prompt-1-w] (0 if negative) the retained tokens are
+ *   LTE_CAP_RECENT: idx[max(0,n-C) .. n), the i-th in ring slot i mod C,
+ *                   ret_total = n;
+ *   LTE_CAP_FIRST:  idx[0 .. min(n,C)), in slots 0, 1, ..., ret_total = min(n,C);
+ *   LTE_CAP_LOWEST: idx[i] for i < n with death[i] > n, in that order in
+ *                   slots 0, 1, ..., with ret_r = their scores and
+ *                   ret_total = their number;
  * win_r = r of window tokens below n_scored (NaN otherwise),
- * ret_total = n, meta = {T_prompt, n_scored, 0, 0}.
+ * meta = {T_prompt, n_scored, 0, 0}.
  * k, v [B,T,Hkv,D]; r [B,Hkv,T] from lte_score; idx, cnt from
- * lte_evict_compact run with the same n_scored. */
+ * lte_evict_compact run with the same n_scored; death (LTE_CAP_LOWEST only,
+ * else ignored) from lte_retained_lifetimes. */
 lte_status lte_cache_init_from_prefill(const lte_dims* d, const lte_cache* cache,
                                        const void* k, const void* v,
                                        const lte_strides* kv_strides, const float* r,
                                        const int32_t* idx, const int32_t* cnt,
+                                       const int32_t* death,
                                        int32_t T_prompt, int32_t n_scored, void* stream);
 
 /* lte_decode_step -- one generated token for every sequence in the batch.
  * Reads t = meta[0] on the device (no host synchronisation), then:
  *  (1) token t-w leaves the window: a sink (t-w < s) moves to its sink slot;
- *      otherwise it enters the retained ring iff win_r >= tau and C > 0
- *      (overwriting the oldest when the ring is full), else it is dropped;
+ *      otherwise it enters the retained segment iff win_r >= tau and C > 0,
+ *      else it is dropped.  When the segment is full, LTE_CAP_RECENT
+ *      overwrites the oldest, LTE_CAP_FIRST drops the newcomer, and
+ *      LTE_CAP_LOWEST replaces the held token with the lowest (ret_r, pos)
+ *      if win_r is not below that score (else drops the newcomer);
  *  (2) the new token is written to window slot t mod w;
  *  (3) deferred batched scoring: once score_batch tokens are scorable
  *      (j + F <= t), the oldest score_batch unscored tokens are scored from

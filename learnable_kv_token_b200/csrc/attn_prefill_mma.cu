@@ -3,7 +3,9 @@
 // "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention
 // and Contextualized Learnable Token Eviction", Fig. 2 caption (right):
 // per-head A-plus-column sparsity; row t of KV head h attends to
-//   S_t = { j < s : j <= t-w } u (t-w, t] u { idx[i] : max(0, n_t-C) <= i < n_t }.
+//   S_t = { j < s : j <= t-w } u (t-w, t] u { idx[i] : max(0, n_t-C) <= i < n_t }
+// (first-C cap: i in [0, min(n_t, C)); drop-the-lowest-score cap: i < n_t with
+// death[i] > n_t, the lifetimes from lte_retained_lifetimes).
 //
 // Design.  A CTA owns 64 query rows that share one KV head: 64/G tokens x
 // the G query heads of the group, so every K/V tile it loads serves all G
@@ -84,7 +86,8 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
                         float scale_log2,
                         const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                         const __nv_bfloat16* __restrict__ v, Strides4 qs, Strides4 kvs,
-                        const int32_t* __restrict__ cnt, const __nv_bfloat16* __restrict__ k_col,
+                        const int32_t* __restrict__ cnt, const int32_t* __restrict__ death,
+                        const __nv_bfloat16* __restrict__ k_col,
                         const __nv_bfloat16* __restrict__ v_col, __nv_bfloat16* __restrict__ o,
                         Strides4 os, float* __restrict__ lse) {
   constexpr int CH = D / 8;            // 16-byte chunks per row
@@ -103,6 +106,7 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
   const int t_last = min(t0 + TOK - 1, T - 1);
   const long long crow = (long long)u * T;
   const long long col_base = (long long)u * (sink + T);
+  const bool lowest = death != nullptr;      // held set filtered by lifetime, scanned from 0
 
   // ---- Q tile: row rho = g*TOK + i  <-  q[b, t0+i, h*G+g, :]
   for (int i = tid; i < kMmaRows * CH; i += kMmaThreads) {
@@ -121,7 +125,7 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
   {
     const int n_first = (t0 >= window) ? held_retained(cnt[crow + t0 - window], cap, cap_policy) : 0;
     const int n_last = (t_last >= window) ? held_retained(cnt[crow + t_last - window], cap, cap_policy) : 0;
-    const int lo_min = n_first - cap > 0 ? n_first - cap : 0;
+    const int lo_min = n_first - cap > 0 && !lowest ? n_first - cap : 0;
     int nsink = t_last - window + 1;
     nsink = nsink < 0 ? 0 : (nsink > sink ? sink : nsink);
     nsink = nsink > T ? T : nsink;
@@ -184,7 +188,7 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
     int hi = 0;
     if (tt < T && tt >= window) hi = held_retained(cnt[crow + tt - window], cap, cap_policy);
     hi_row[hr] = hi;
-    lo_row[hr] = hi - cap > 0 ? hi - cap : 0;
+    lo_row[hr] = hi - cap > 0 && !lowest ? hi - cap : 0;
   }
   // tile-wide bounds for the "every row sees every key" fast path
   const int lo_all = max(lo_row[0], lo_row[1]);
@@ -248,7 +252,7 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
       full = (nk == kMmaKeys) && key0 > max(t_row[0], t_row[1]) - window &&
              key0 + kMmaKeys - 1 <= min(t_row[0], t_row[1]);
     } else {
-      full = (nk == kMmaKeys) && key0 >= sink && (key0 - sink) >= lo_all &&
+      full = !lowest && (nk == kMmaKeys) && key0 >= sink && (key0 - sink) >= lo_all &&
              (key0 - sink + kMmaKeys) <= hi_all;
     }
     full = __all_sync(0xffffffffu, full);
@@ -265,7 +269,8 @@ attn_prefill_mma_kernel(int T, int Hq, int Hkv, int sink, int window, int cap, i
           if (ok) {
             if (rg == 2) ok = key <= tt && key > tt - window;
             else if (key < sink) ok = key <= tt - window;
-            else ok = (key - sink) >= lo_row[hr] && (key - sink) < hi_row[hr];
+            else ok = (key - sink) >= lo_row[hr] && (key - sink) < hi_row[hr] &&
+                      (!lowest || __ldg(death + crow + key - sink) > hi_row[hr]);
           }
           if (!ok) s[nt][e] = -INFINITY;
         }
@@ -363,7 +368,7 @@ static cudaError_t launch_mma(const PrefillArgs& a, cudaStream_t stream) {
   attn_prefill_mma_kernel<D><<<grid, kMmaThreads, smem, stream>>>(
       d->T, d->Hq, d->Hkv, d->sink, d->window, d->cap, d->cap_policy, scale_log2,
       (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v, a.qs,
-      a.kvs, a.cnt, (const __nv_bfloat16*)a.k_col, (const __nv_bfloat16*)a.v_col,
+      a.kvs, a.cnt, a.death, (const __nv_bfloat16*)a.k_col, (const __nv_bfloat16*)a.v_col,
       (__nv_bfloat16*)a.o, a.os, a.lse);
   return cudaGetLastError();
 }

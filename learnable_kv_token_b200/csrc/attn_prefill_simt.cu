@@ -5,7 +5,9 @@
 // query attends, per KV head, to the attention sink, the sliding window and
 // the LTE-retained tokens (the "A-plus-column" pattern).  For row t:
 //   S_t = { j < s : j <= t-w } u (t-w, t] u { idx[i] : max(0, n_t-C) <= i < n_t },
-//   n_t = cnt[t-w] (0 for t < w).
+//   n_t = cnt[t-w] (0 for t < w); under the first-C cap the range is
+//   [0, min(n_t, C)), under the drop-the-lowest-score cap { i < n_t :
+//   death[i] > n_t } (death from lte_retained_lifetimes).
 //
 // One CTA handles 32 rows of one query head.  Keys stream in chunks of 32
 // from three ranges (sink slots and retained slots of the column segment,
@@ -27,7 +29,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 attn_prefill_simt_kernel(int T, int Hq, int Hkv, int D, int sink, int window, int cap,
                          int cap_policy, float scale, const float* __restrict__ q, const float* __restrict__ k,
                          const float* __restrict__ v, Strides4 qs, Strides4 kvs,
-                         const int32_t* __restrict__ cnt, const float* __restrict__ k_col,
+                         const int32_t* __restrict__ cnt, const int32_t* __restrict__ death,
+                         const float* __restrict__ k_col,
                          const float* __restrict__ v_col, float* __restrict__ o, Strides4 os,
                          float* __restrict__ lse) {
   extern __shared__ float sm[];
@@ -50,15 +53,16 @@ attn_prefill_simt_kernel(int T, int Hq, int Hkv, int D, int sink, int window, in
                          : 0.f;
   }
   // per-row retained range [lo_t, hi_t) of the compacted list
+  const bool lowest = death != nullptr;      // held set filtered by lifetime, scanned from 0
   int hi_t = 0, lo_t = 0;
   if (t < T && t >= window) {
     hi_t = held_retained(cnt[crow + t - window], cap, cap_policy);
-    lo_t = hi_t - cap > 0 ? hi_t - cap : 0;
+    lo_t = hi_t - cap > 0 && !lowest ? hi_t - cap : 0;
   }
   // tile-wide ranges
   const int n_first = (t0 >= window) ? held_retained(cnt[crow + t0 - window], cap, cap_policy) : 0;
   const int n_last = (t_last >= window) ? held_retained(cnt[crow + t_last - window], cap, cap_policy) : 0;
-  const int lo_min = n_first - cap > 0 ? n_first - cap : 0;
+  const int lo_min = n_first - cap > 0 && !lowest ? n_first - cap : 0;
   int nsink = t_last - window + 1;
   nsink = nsink < 0 ? 0 : (nsink > sink ? sink : nsink);
   nsink = nsink > T ? T : nsink;
@@ -105,7 +109,8 @@ attn_prefill_simt_kernel(int T, int Hq, int Hkv, int D, int sink, int window, in
         if (ok) {
           if (rg == 2) ok = key <= t && key > t - window;
           else if (key < sink) ok = key <= t - window;
-          else ok = (key - sink) >= lo_t && (key - sink) < hi_t;
+          else ok = (key - sink) >= lo_t && (key - sink) < hi_t &&
+                    (!lowest || death[crow + key - sink] > hi_t);
         }
         float s = -INFINITY;
         if (ok) {
@@ -160,7 +165,7 @@ cudaError_t attn_prefill_simt(const PrefillArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   attn_prefill_simt_kernel<<<grid, kSimtThreads, smem, stream>>>(
       d->T, d->Hq, d->Hkv, d->D, d->sink, d->window, d->cap, d->cap_policy, d->scale, (const float*)a.q,
-      (const float*)a.k, (const float*)a.v, a.qs, a.kvs, a.cnt, (const float*)a.k_col,
+      (const float*)a.k, (const float*)a.v, a.qs, a.kvs, a.cnt, a.death, (const float*)a.k_col,
       (const float*)a.v_col, (float*)a.o, a.os, a.lse);
   return cudaGetLastError();
 }

@@ -5,7 +5,11 @@
 // and Contextualized Learnable Token Eviction", Fig. 2 caption (right): the
 // per-head A-plus-column pattern.  Row t of KV head h attends to
 //   S_t = { j < s : j <= t-w } u (t-w, t] u { idx[i] : max(0, n_t-C) <= i < n_t },
-//   n_t = cnt[t-w] (0 for t < w).
+//   n_t = cnt[t-w] (0 for t < w).  Under the first-C cap the retained range is
+//   [0, min(n_t, C)); under the drop-the-lowest-score cap it is { i < n_t :
+//   death[i] > n_t } (lifetimes from lte_retained_lifetimes): the kernel
+//   instance for that policy scans retained slots from 0 and ANDs a lifetime
+//   bit set into each retained tile's predicate.
 //
 // Work item: one (batch, KV head) unit and two consecutive 128-row Q tiles
 // (each 128/G tokens x the G query heads of the group, rows token-major).
@@ -93,6 +97,7 @@ struct Params {
   int n_pairs, n_units, n_items;
   float scale_log2;
   const int32_t* cnt;
+  const int32_t* death;   // lifetimes of retained slots (drop-the-lowest-score cap), else NULL
   float* lse;
   DevError* err;
 };
@@ -184,7 +189,7 @@ __device__ __forceinline__ Item make_item(const Params& p, int i, const ItemCoun
   m.b = m.u / p.Hkv;
   m.h = m.u % p.Hkv;
   const int n_first = c.n_first, n_last = c.n_last;
-  const int lo_min = n_first - p.cap > 0 ? n_first - p.cap : 0;
+  const int lo_min = n_first - p.cap > 0 && p.death == nullptr ? n_first - p.cap : 0;
   int nsink = m.t_last - p.window + 1;
   nsink = nsink < 0 ? 0 : (nsink > p.sink ? p.sink : nsink);
   nsink = nsink > p.T ? p.T : nsink;
@@ -202,6 +207,18 @@ __device__ __forceinline__ Item make_item(const Params& p, int i, const ItemCoun
   return m;
 }
 
+// Retained slots i = i0 + c (c < 64) held at count n: 0 <= i < n and death[i] > n.
+__device__ __forceinline__ uint64_t alive_bits(const int32_t* __restrict__ death_u, int i0, int n) {
+  uint64_t bits = 0ull;
+#pragma unroll 8
+  for (int c = 0; c < BN; ++c) {
+    const int i = i0 + c;
+    if (i >= 0 && i < n && __ldg(death_u + i) > n) bits |= 1ull << c;
+  }
+  return bits;
+}
+
+template <bool kLowest>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -460,7 +477,7 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const bool has_next = i + (int)gridDim.x < p.n_items;
       const int tt = m.t0 + x * p.TOK + row / p.G;
       const bool row_ok = tt < p.T;
-      const int lo_t = hi_t - p.cap > 0 ? hi_t - p.cap : 0;
+      const int lo_t = hi_t - p.cap > 0 && !kLowest ? hi_t - p.cap : 0;
       // attended-set predicate of tile j as a bit set over its columns: the
       // window band is one interval; a slot tile holds the visible sinks and
       // the retained slots [lo_t, hi_t), two intervals.  It does not depend on
@@ -471,8 +488,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (!row_ok) return 0ull;
         if (rg == 2) return span_bits(tt - p.window + 1 - key0, min(nk, tt - key0 + 1));
         const int sink_end = min(p.sink, tt - p.window + 1);
-        return span_bits(-key0, min(nk, sink_end - key0)) |
-               span_bits(p.sink + lo_t - key0, min(nk, p.sink + hi_t - key0));
+        uint64_t ret = span_bits(p.sink + lo_t - key0, min(nk, p.sink + hi_t - key0));
+        if constexpr (kLowest) {
+          if (ret != 0ull) ret &= alive_bits(p.death + (long long)m.u * p.T, key0 - p.sink, hi_t);
+        }
+        return span_bits(-key0, min(nk, sink_end - key0)) | ret;
       };
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = 0; j < m.total; ++j) {
@@ -665,15 +685,17 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   p.n_items = p.n_pairs * p.n_units;
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.cnt = a.cnt;
+  p.death = a.death;
   p.lse = a.lse; p.err = a.err;
-  cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kernel = a.death != nullptr ? attn_prefill_tc_kernel<true> : attn_prefill_tc_kernel<false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, n_sm = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const int grid = p.n_items < n_sm ? p.n_items : n_sm;
-  attn_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mkc, mvc, mo, p);
+  kernel<<<grid, kThreads, kSmemBytes, stream>>>(mq, mk, mv, mkc, mvc, mo, p);
   return cudaGetLastError();
 }
 

@@ -113,6 +113,69 @@ __device__ __forceinline__ void pdl_launch_next() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The retained slot holding the lowest (score, position), over slots [0, cap)
+// of one unit: each lane scans every 32nd slot, then a shuffle tree.  Called by
+// a whole warp; every lane returns the same slot and score.
+__device__ __forceinline__ int lowest_slot(const float* __restrict__ ret_r,
+                                           const int32_t* __restrict__ ret_pos, int cap,
+                                           float& r_min) {
+  const int lane = threadIdx.x & 31;
+  float br = INFINITY;
+  int bp = 0x7fffffff, bs = -1;
+  for (int i = lane; i < cap; i += 32) {
+    const float x = ret_r[i];
+    const int p = ret_pos[i];
+    if (x < br || (x == br && p < bp)) br = x, bp = p, bs = i;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const float xr = __shfl_xor_sync(0xffffffffu, br, o);
+    const int xp = __shfl_xor_sync(0xffffffffu, bp, o);
+    const int xs = __shfl_xor_sync(0xffffffffu, bs, o);
+    if (xr < br || (xr == br && xp < bp)) br = xr, bp = xp, bs = xs;
+  }
+  r_min = br;
+  return bs;
+}
+
+// Where token `leaving` goes when it leaves the window (-1: dropped), and the
+// retained count afterwards.  Called by a whole warp (LTE_CAP_LOWEST looks for
+// the lowest held score when the segment is full); `held`/`r`/`rt` are read by
+// every lane.  Under LTE_CAP_LOWEST the newcomer's score is written to its slot.
+__device__ __forceinline__ int leaving_dst(int leaving, int held, float r, int rt, int window,
+                                           int sink, int cap, int cap_policy, float tau,
+                                           const int32_t* __restrict__ urow_pos,
+                                           float* __restrict__ u_ret_r, DevError* err,
+                                           int& rt_new) {
+  const int lane = threadIdx.x & 31;
+  rt_new = rt;
+  if (leaving < 0) return -1;
+  if (held != leaving) {
+    if (lane == 0) record_error(err, LTE_ERR_DEVICE, kWhereDecodeIndex);
+    return -1;
+  }
+  if (leaving < sink) return window + leaving;
+  if (cap == 0 || !(r >= tau)) return -1;
+  if (cap_policy == LTE_CAP_RECENT) {
+    rt_new = rt + 1;
+    return window + sink + rt % cap;
+  }
+  if (rt < cap) {                                 // FIRST and LOWEST fill slots in order
+    rt_new = rt + 1;
+    if (cap_policy == LTE_CAP_LOWEST && lane == 0) u_ret_r[rt] = r;
+    return window + sink + rt;
+  }
+  if (cap_policy == LTE_CAP_FIRST) return -1;    // a full segment drops the newcomer
+  float r_min;
+  const int m = lowest_slot(u_ret_r, urow_pos + window + sink, cap, r_min);
+  // the newcomer is the latest token, so it beats the lowest held one iff its
+  // score is not below it
+  if (m < 0 || r < r_min) return -1;
+  __syncwarp();                                   // every lane has read the old score
+  if (lane == 0) u_ret_r[m] = r;
+  return window + sink + m;
+}
+
 // ---------------------------------------------------------------------------
 struct PrepParams {
   int Hkv, D, elt, window, sink, cap, cap_policy, score_batch, future, n_units;
@@ -127,6 +190,7 @@ struct PrepParams {
   int32_t* meta;
   int32_t* counters;
   DevError* err;
+  float* ret_r;
 };
 
 template <typename T, bool kTc>
@@ -154,19 +218,17 @@ decode_prep_kernel(PrepParams pp, ScoreParams sp, RingKV<T> kv) {
     kn = reinterpret_cast<const uint4*>(pp.k_t + (long long)u * pp.D * pp.elt)[tid];
     vn = reinterpret_cast<const uint4*>(pp.v_t + (long long)u * pp.D * pp.elt)[tid];
   }
-  int rt = 0;
-  if (tid == 0) {
-    int dst = -1;
+  if (tid < 32) {
+    int rt_new = 0, dst = -1;
     if (leaving >= 0) {
       const int held = pp.pos[urow + slot_w];
       const float r = pp.win_r[(long long)u * pp.window + slot_w];
-      rt = pp.ret_total[u];
-      if (held != leaving) record_error(pp.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
-      else if (leaving < pp.sink) dst = pp.window + leaving;
-      else if (pp.cap > 0 && r >= pp.tau && (pp.cap_policy == LTE_CAP_RECENT || rt < pp.cap))
-        dst = pp.window + pp.sink + rt % pp.cap;       // under LTE_CAP_FIRST a full segment drops it
+      const int rt = pp.ret_total[u];
+      dst = leaving_dst(leaving, held, r, rt, pp.window, pp.sink, pp.cap, pp.cap_policy, pp.tau,
+                        pp.pos + urow, pp.ret_r + (long long)u * pp.cap, pp.err, rt_new);
+      if (tid == 0 && rt_new != rt) pp.ret_total[u] = rt_new;
     }
-    dst_sh = dst;
+    if (tid == 0) dst_sh = dst;
   }
   __syncthreads();
   const int dst_slot = dst_sh;
@@ -181,7 +243,6 @@ decode_prep_kernel(PrepParams pp, ScoreParams sp, RingKV<T> kv) {
   }
   if (tid == 0) {
     if (dst_slot >= 0) pp.pos[urow + dst_slot] = leaving;
-    if (dst_slot >= pp.window + pp.sink) pp.ret_total[u] = rt + 1;
     pp.pos[urow + slot_w] = t;
     pp.win_r[(long long)u * pp.window + slot_w] = NAN;
     pp.counters[u] = 0;
@@ -644,6 +705,7 @@ static cudaError_t launch_prep(const lte_dims* d, const lte_cnn* cnn, const lte_
   pp.k_t = (const char*)k_t; pp.v_t = (const char*)v_t;
   pp.ck = (char*)c->k; pp.cv = (char*)c->v; pp.pos = c->pos; pp.win_r = c->win_r;
   pp.ret_total = c->ret_total; pp.meta = c->meta; pp.counters = counters; pp.err = err;
+  pp.ret_r = c->ret_r;
   ScoreParams sp = score_params(d, cnn);
   sp.window = d->window;
   sp.win_r = c->win_r;
@@ -788,6 +850,7 @@ struct FusedParams {
   __nv_bfloat16* o_t;
   float* lse_t;
   DevError* err;
+  float* ret_r;
 };
 
 // The chunks of one step, in issue order: the window chunks except the one
@@ -928,19 +991,15 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       new4 = reinterpret_cast<const uint4*>((is_v ? p.v_t : p.k_t) + (long long)u * D)[e];
       old4 = reinterpret_cast<const uint4*>((is_v ? p.cv : p.ck) + wrow)[e];
     }
-    int dst = -1, rt = 0;
-    if (lane == 0) {
-      rt = p.ret_total[u];
-      if (leaving >= 0) {
-        const int held = p.pos[urow + slot_w];
-        const float r = p.win_r[(long long)u * p.window + slot_w];
-        if (held != leaving) record_error(p.err, LTE_ERR_DEVICE, kWhereDecodeIndex);
-        else if (leaving < p.sink) dst = p.window + leaving;
-        else if (p.cap > 0 && r >= p.tau && (p.cap_policy == LTE_CAP_RECENT || rt < p.cap))
-          dst = p.window + p.sink + rt % p.cap;         // under LTE_CAP_FIRST a full segment drops it
-      }
+    const int rt = p.ret_total[u];
+    int dst = -1, rt_new = rt;
+    if (leaving >= 0) {
+      const int held = p.pos[urow + slot_w];
+      const float r = p.win_r[(long long)u * p.window + slot_w];
+      dst = leaving_dst(leaving, held, r, rt, p.window, p.sink, p.cap, p.cap_policy, p.tau,
+                        p.pos + urow, p.ret_r + (long long)u * p.cap, p.err, rt_new);
     }
-    dst = __shfl_sync(0xffffffffu, dst, 0);
+    __syncwarp();                                // every lane has read the slots' positions
     if (e < NV) {
       __nv_bfloat16* base = is_v ? p.cv : p.ck;
       if (dst >= 0) reinterpret_cast<uint4*>(base + (urow + dst) * D)[e] = old4;
@@ -948,7 +1007,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     if (lane == 0) {
       if (dst >= 0) p.pos[urow + dst] = leaving;
-      const int rt_new = rt + (dst >= p.window + p.sink ? 1 : 0);
       if (rt_new != rt) p.ret_total[u] = rt_new;
       p.pos[urow + slot_w] = t;
       p.win_r[(long long)u * p.window + slot_w] = NAN;
@@ -1203,7 +1261,7 @@ static cudaError_t launch_fused(const lte_dims* d, const lte_cnn* cnn, const lte
   p.q_t = (const __nv_bfloat16*)q_t; p.k_t = (const __nv_bfloat16*)k_t;
   p.v_t = (const __nv_bfloat16*)v_t;
   p.ck = (__nv_bfloat16*)c->k; p.cv = (__nv_bfloat16*)c->v; p.pos = c->pos; p.win_r = c->win_r;
-  p.ret_total = c->ret_total; p.meta = c->meta;
+  p.ret_total = c->ret_total; p.meta = c->meta; p.ret_r = c->ret_r;
   p.o_t = (__nv_bfloat16*)o_t; p.lse_t = lse_t; p.err = err;
   ScoreParams sp = score_params(d, cnn);
   sp.window = d->window;

@@ -131,16 +131,84 @@ cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask
 }
 
 // ---------------------------------------------------------------------------
+// Lifetimes of retained tokens under the drop-the-lowest-score cap
+// (LTE_CAP_LOWEST).  The segment after n arrivals holds the C best of them by
+// (score, ordinal): a token is dropped -- possibly on arrival -- exactly when
+// the C-th token that beats it has arrived.  So death[i] = max(i, j*) + 1,
+// j* the ordinal at which the count of tokens beating i reaches C, scanning
+// ordinals in order (T + 1 if it never does).
+// One thread per ordinal, kLifeThreads ordinals per CTA; the unit's compacted
+// scores pass through shared memory in tiles, read by every thread of the CTA
+// at the same address (broadcast).  A CTA stops once all its threads have
+// found their j*.
+constexpr int kLifeThreads = 256;
+constexpr int kLifeTile = 2048;
+
+__global__ void __launch_bounds__(kLifeThreads)
+lifetimes_kernel(int T, int cap, const float* __restrict__ r, const int32_t* __restrict__ idx,
+                 const int32_t* __restrict__ nret, int32_t* __restrict__ death) {
+  __shared__ float rc[kLifeTile];
+  const int chunks = (T + kLifeThreads - 1) / kLifeThreads;
+  const int u = blockIdx.x / chunks, tid = threadIdx.x;
+  const long long row0 = (long long)u * T;
+  const int n = nret[u];
+  const int i0 = (blockIdx.x % chunks) * kLifeThreads;
+  if (i0 >= n) return;
+  const int i = i0 + tid;
+  const bool valid = i < n;
+  if (cap == 0 || n <= cap) {
+    // C = 0: zero beaters suffice, every token is dropped on arrival (i + 1);
+    // n <= C: at most n - 1 < C others, nobody is ever dropped
+    if (valid) death[row0 + i] = cap == 0 ? i + 1 : T + 1;
+    return;
+  }
+  const float ri = valid ? r[row0 + idx[row0 + i]] : 0.f;
+  int beaten = 0, dies = T + 1;
+  bool found = !valid;
+  for (int j0 = 0; j0 < n; j0 += kLifeTile) {
+    const int nj = min(kLifeTile, n - j0);
+    __syncthreads();                                 // the previous tile has been read
+    for (int jj = tid; jj < nj; jj += kLifeThreads) rc[jj] = r[row0 + idx[row0 + j0 + jj]];
+    __syncthreads();
+    if (!found) {
+      for (int jj = 0; jj < nj; ++jj) {
+        const int j = j0 + jj;
+        const float x = rc[jj];
+        beaten += (x > ri || (x == ri && j > i)) ? 1 : 0;   // j == i never counts
+        if (beaten == cap) {
+          dies = max(i, j) + 1;
+          found = true;
+          break;
+        }
+      }
+    }
+    if (__syncthreads_and(found)) break;
+  }
+  if (valid) death[row0 + i] = dies;
+}
+
+cudaError_t retained_lifetimes(const lte_dims* d, const float* r, const int32_t* idx,
+                               const int32_t* nret, int32_t* death, cudaStream_t stream) {
+  const long long ctas = (long long)((d->T + kLifeThreads - 1) / kLifeThreads) * d->B * d->Hkv;
+  if (ctas > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  lifetimes_kernel<<<(unsigned)ctas, kLifeThreads, 0, stream>>>(d->T, d->cap, r, idx, nret, death);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Decode-cache set-up from a prefilled prompt (Fig. 3 layout): window ring,
 // sink slots, retained ring.  One CTA per unit.
 __global__ void __launch_bounds__(256)
 cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap, int cap_policy,
                   int T0, int n_scored, const char* __restrict__ k, const char* __restrict__ v,
                   Strides4 s, const float* __restrict__ r, const int32_t* __restrict__ idx,
-                  const int32_t* __restrict__ cnt, char* __restrict__ ck, char* __restrict__ cv,
-                  int32_t* __restrict__ pos, float* __restrict__ win_r,
-                  int32_t* __restrict__ ret_total, int32_t* __restrict__ meta) {
+                  const int32_t* __restrict__ cnt, const int32_t* __restrict__ death,
+                  char* __restrict__ ck, char* __restrict__ cv, int32_t* __restrict__ pos,
+                  float* __restrict__ win_r, int32_t* __restrict__ ret_total,
+                  int32_t* __restrict__ meta, float* __restrict__ ret_r) {
+  __shared__ int warp_tot[8];
   const int u = blockIdx.x, b = u / Hkv, h = u % Hkv, tid = threadIdx.x;
+  const bool lowest = cap_policy == LTE_CAP_LOWEST;
   const int L = window + sink + cap;
   const long long row0 = (long long)u * T;
   const int last_out = T0 - 1 - window;                 // newest token outside the window
@@ -162,13 +230,44 @@ cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap,
       if (jj <= last_out) j = jj;
     } else {
       const int rs = slot - window - sink;
-      // retained ordinal i with i mod C == rs in [ret_lo, n)
-      if (n > 0) {
+      // retained ordinal i with i mod C == rs in [ret_lo, n) (LTE_CAP_LOWEST: below)
+      if (n > 0 && !lowest) {
         int i = ret_lo + ((rs - ret_lo % cap) % cap + cap) % cap;
         if (i < n) j = idx[row0 + i];
       }
     }
     pos[(long long)u * L + slot] = j;
+  }
+  int held = n;
+  if (lowest) {
+    // the tokens held at count n, i < n with death[i] > n, in ordinal order in
+    // slots 0, 1, ...: a ballot rank per warp plus the warp offsets, per round
+    // of 256 ordinals
+    const int lane = tid & 31, warp = tid >> 5;
+    int carry = 0;
+    for (int base = 0; base < n; base += 256) {
+      const int i = base + tid;
+      const bool keep = i < n && death[row0 + i] > n;
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      __syncthreads();                                // the previous round's totals are read
+      if (lane == 0) warp_tot[warp] = __popc(bal);
+      __syncthreads();
+      int off = carry, tot = 0;
+      for (int w = 0; w < 8; ++w) {
+        if (w < warp) off += warp_tot[w];
+        tot += warp_tot[w];
+      }
+      const int slot = off + __popc(bal & ((1u << lane) - 1u));
+      if (keep && slot < cap) {
+        const int j = idx[row0 + i];
+        pos[(long long)u * L + window + sink + slot] = j;
+        ret_r[(long long)u * cap + slot] = r[row0 + j];
+      }
+      carry += tot;
+    }
+    held = carry < cap ? carry : cap;
+    for (int slot = held + tid; slot < cap; slot += blockDim.x)
+      ret_r[(long long)u * cap + slot] = NAN;
   }
   __syncthreads();
   const int nvec = D * elt / 16;
@@ -182,7 +281,7 @@ cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap,
     reinterpret_cast<uint4*>(cv + dst)[c] = reinterpret_cast<const uint4*>(v + src)[c];
   }
   if (tid == 0) {
-    ret_total[u] = n;
+    ret_total[u] = held;
     if (u == 0) {
       meta[0] = T0;
       meta[1] = n_scored;
@@ -194,12 +293,12 @@ cache_init_kernel(int T, int Hkv, int D, int elt, int window, int sink, int cap,
 
 cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, const void* v,
                        Strides4 s, const float* r, const int32_t* idx, const int32_t* cnt,
-                       int T_prompt, int n_scored, cudaStream_t stream) {
+                       const int32_t* death, int T_prompt, int n_scored, cudaStream_t stream) {
   const int elt = d->dtype == LTE_BF16 ? 2 : 4;
   cache_init_kernel<<<d->B * d->Hkv, 256, 0, stream>>>(
       d->T, d->Hkv, d->D, elt, d->window, d->sink, d->cap, d->cap_policy, T_prompt, n_scored,
-      (const char*)k, (const char*)v, s, r, idx, cnt, (char*)c->k, (char*)c->v, c->pos,
-      c->win_r, c->ret_total, c->meta);
+      (const char*)k, (const char*)v, s, r, idx, cnt, death, (char*)c->k, (char*)c->v, c->pos,
+      c->win_r, c->ret_total, c->meta, c->ret_r);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,9 @@ lte_status check_dims(const lte_dims* d) {
   if (d->Hq % d->Hkv != 0) return LTE_ERR_INVALID_ARG;
   if (d->sink < 0 || d->window < 1 || d->cap < 0) return LTE_ERR_INVALID_ARG;
   if (d->dtype != LTE_F32 && d->dtype != LTE_BF16) return LTE_ERR_INVALID_ARG;
-  if (d->cap_policy != LTE_CAP_RECENT && d->cap_policy != LTE_CAP_FIRST) return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy != LTE_CAP_RECENT && d->cap_policy != LTE_CAP_FIRST &&
+      d->cap_policy != LTE_CAP_LOWEST)
+    return LTE_ERR_INVALID_ARG;
   if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return LTE_ERR_INVALID_ARG;
   if (std::isnan(d->tau)) return LTE_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LTE_ERR_UNSUPPORTED;
@@ -112,6 +114,15 @@ lte_status lte_evict_compact(const lte_dims* d, const float* r, const uint8_t* m
                                       v_col, as_stream(stream)));
 }
 
+lte_status lte_retained_lifetimes(const lte_dims* d, const float* r, const int32_t* idx,
+                                  const int32_t* nret, int32_t* death, void* stream) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (d->cap_policy != LTE_CAP_LOWEST) return LTE_ERR_INVALID_ARG;
+  if (!r || !idx || !nret || !death) return LTE_ERR_INVALID_ARG;
+  return from_cuda(lte::retained_lifetimes(d, r, idx, nret, death, as_stream(stream)));
+}
+
 size_t lte_workspace_bytes(const lte_dims* d, int32_t which) {
   if (check_dims(d) != LTE_OK) return 0;
   if (which == LTE_WS_PREFILL) return kErrBytes + lte::attn_prefill_scratch_bytes(d);
@@ -122,12 +133,13 @@ size_t lte_workspace_bytes(const lte_dims* d, int32_t which) {
 lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void* k,
                                    const void* v, const lte_strides* q_strides,
                                    const lte_strides* kv_strides, const int32_t* cnt,
-                                   const void* k_col, const void* v_col, void* o,
-                                   const lte_strides* o_strides, float* lse, void* workspace,
-                                   size_t ws_bytes, void* stream) {
+                                   const int32_t* death, const void* k_col, const void* v_col,
+                                   void* o, const lte_strides* o_strides, float* lse,
+                                   void* workspace, size_t ws_bytes, void* stream) {
   lte_status st = check_dims(d);
   if (st != LTE_OK) return st;
   if (!q || !k || !v || !cnt || !k_col || !v_col || !o) return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy == LTE_CAP_LOWEST && death == nullptr) return LTE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_col) || !aligned16(v_col) ||
       !aligned16(o))
     return LTE_ERR_INVALID_ARG;
@@ -142,6 +154,7 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
   if ((st = get_strides(d, kv_strides, d->Hkv, &a.kvs)) != LTE_OK) return st;
   if ((st = get_strides(d, o_strides, d->Hq, &a.os)) != LTE_OK) return st;
   a.cnt = cnt; a.k_col = k_col; a.v_col = v_col; a.o = o; a.lse = lse;
+  a.death = d->cap_policy == LTE_CAP_LOWEST ? death : nullptr;
   a.err = reinterpret_cast<lte::DevError*>(workspace);
   a.scratch = static_cast<char*>(workspace) + kErrBytes;
   a.scratch_bytes = ws_bytes - kErrBytes;
@@ -159,7 +172,8 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
 lte_status lte_cache_init_from_prefill(const lte_dims* d, const lte_cache* cache, const void* k,
                                        const void* v, const lte_strides* kv_strides,
                                        const float* r, const int32_t* idx, const int32_t* cnt,
-                                       int32_t T_prompt, int32_t n_scored, void* stream) {
+                                       const int32_t* death, int32_t T_prompt, int32_t n_scored,
+                                       void* stream) {
   lte_status st = check_dims(d);
   if (st != LTE_OK) return st;
   if (cache == nullptr || !cache->k || !cache->v || !cache->pos || !cache->win_r ||
@@ -171,10 +185,13 @@ lte_status lte_cache_init_from_prefill(const lte_dims* d, const lte_cache* cache
   if (T_prompt > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return LTE_ERR_INVALID_ARG;
   if (T_prompt > d->window && (!idx || !cnt)) return LTE_ERR_INVALID_ARG;
   if (n_scored > 0 && r == nullptr) return LTE_ERR_INVALID_ARG;
+  const bool lowest = d->cap_policy == LTE_CAP_LOWEST;
+  if (lowest && (cache->ret_r == nullptr || (T_prompt > d->window && (!death || !r))))
+    return LTE_ERR_INVALID_ARG;
   Strides4 s;
   if ((st = get_strides(d, kv_strides, d->Hkv, &s)) != LTE_OK) return st;
-  return from_cuda(lte::cache_init(d, cache, k, v, s, r, idx, cnt, T_prompt, n_scored,
-                                   as_stream(stream)));
+  return from_cuda(lte::cache_init(d, cache, k, v, s, r, idx, cnt, lowest ? death : nullptr,
+                                   T_prompt, n_scored, as_stream(stream)));
 }
 
 lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cache* cache,
@@ -188,6 +205,7 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
   if (cache == nullptr || !cache->k || !cache->v || !cache->pos || !cache->win_r ||
       !cache->ret_total || !cache->meta)
     return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy == LTE_CAP_LOWEST && cache->ret_r == nullptr) return LTE_ERR_INVALID_ARG;
   if (!q_t || !k_t || !v_t || !o_t) return LTE_ERR_INVALID_ARG;
   if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) ||
       !aligned16(cache->k) || !aligned16(cache->v))
@@ -215,6 +233,7 @@ lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const 
   if (cache == nullptr || !cache->k || !cache->v || !cache->pos || !cache->win_r ||
       !cache->ret_total || !cache->meta)
     return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy == LTE_CAP_LOWEST && cache->ret_r == nullptr) return LTE_ERR_INVALID_ARG;
   if (!q_t || !k_t || !v_t || !o_t) return LTE_ERR_INVALID_ARG;
   if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(o_t) ||
       !aligned16(cache->k) || !aligned16(cache->v))

@@ -26,9 +26,11 @@ cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask
                           int32_t* idx, int32_t* nret, int32_t* cnt, const void* k,
                           const void* v, Strides4 s, void* k_col, void* v_col,
                           cudaStream_t stream);
+cudaError_t retained_lifetimes(const lte_dims* d, const float* r, const int32_t* idx,
+                               const int32_t* nret, int32_t* death, cudaStream_t stream);
 cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, const void* v,
                        Strides4 s, const float* r, const int32_t* idx, const int32_t* cnt,
-                       int T_prompt, int n_scored, cudaStream_t stream);
+                       const int32_t* death, int T_prompt, int n_scored, cudaStream_t stream);
 
 // attn_prefill_*.cu
 struct PrefillArgs {
@@ -36,6 +38,7 @@ struct PrefillArgs {
   const void *q, *k, *v;
   Strides4 qs, kvs, os;
   const int32_t* cnt;
+  const int32_t* death;  // retained lifetimes (LTE_CAP_LOWEST), else NULL
   const void *k_col, *v_col;
   void* o;
   float* lse;

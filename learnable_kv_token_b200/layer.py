@@ -47,6 +47,7 @@ class PrefillOut:
     k_col: torch.Tensor
     v_col: torch.Tensor
     n_scored: int
+    death: torch.Tensor | None = None      # retained lifetimes (LTE_CAP_LOWEST)
 
 
 class PrefillBuffers:
@@ -64,19 +65,27 @@ class PrefillBuffers:
         self.cnt = torch.empty(B, Hkv, T, dtype=torch.int32, device=dev)
         self.k_col = torch.empty(B, Hkv, sink + T, D, dtype=dtype, device=dev)
         self.v_col = torch.empty(B, Hkv, sink + T, D, dtype=dtype, device=dev)
+        self.death = (torch.empty(B, Hkv, T, dtype=torch.int32, device=dev)
+                      if dims.cap_policy == L.LTE_CAP_LOWEST else None)
         ws = L.lte_workspace_bytes(dims, L.LTE_WS_PREFILL)
         self.ws = torch.zeros((ws + 15) // 16 * 16, dtype=torch.uint8, device=dev)
 
 
 def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers | None = None,
-            stream=None) -> PrefillOut:
-    """One LTE layer prefill.  Either a fed retention `mask` [B,Hkv,T] (uint8)
-    or `cnn` = (w1, b1, w2, b2) device tensors for live scoring."""
+            stream=None, scores=None) -> PrefillOut:
+    """One LTE layer prefill.  Either a fed retention `mask` [B,Hkv,T] (uint8),
+    fed `scores` [B,Hkv,T] (fp32, retained iff >= tau), or `cnn` = (w1, b1,
+    w2, b2) device tensors for live scoring.  LTE_CAP_LOWEST needs scores
+    (fed or live): they rank the retained tokens."""
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
+    lowest = p.cap_policy == L.LTE_CAP_LOWEST
+    if lowest and cnn is None and scores is None:
+        raise ValueError("LTE_CAP_LOWEST ranks retained tokens by score: pass cnn or scores")
     if bufs is None:
         bufs = PrefillBuffers(B, T, Hq, Hkv, D, q.dtype, p.sink, dims, q.device, want_r=cnn is not None)
+    r = scores
     if cnn is not None:
         w1, b1, w2, b2 = cnn
         c, _keep = L.make_cnn(w1, b1, w2, b2, p.past1, p.past2)
@@ -84,14 +93,22 @@ def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers |
         L.lte_score(dims, c, k, v, 0, n_scored, bufs.r, bufs.mask, stream)
         L.lte_evict_compact(dims, None, bufs.mask, n_scored, bufs.idx, bufs.nret, bufs.cnt, k, v,
                             bufs.k_col, bufs.v_col, stream)
+        r = bufs.r
+    elif scores is not None:
+        n_scored = T
+        L.lte_evict_compact(dims, scores, None, T, bufs.idx, bufs.nret, bufs.cnt, k, v, bufs.k_col,
+                            bufs.v_col, stream)
     else:
         n_scored = T
         L.lte_evict_compact(dims, None, mask, T, bufs.idx, bufs.nret, bufs.cnt, k, v, bufs.k_col,
                             bufs.v_col, stream)
+    if lowest:
+        L.lte_retained_lifetimes(dims, r, bufs.idx, bufs.nret, bufs.death, stream)
     L.lte_sparse_attn_prefill(dims, q, k, v, bufs.cnt, bufs.k_col, bufs.v_col, bufs.o, bufs.lse,
-                              bufs.ws, stream)
-    return PrefillOut(bufs.o, bufs.lse, bufs.r, bufs.mask if cnn is not None else mask, bufs.idx,
-                      bufs.nret, bufs.cnt, bufs.k_col, bufs.v_col, n_scored)
+                              bufs.ws, stream, death=bufs.death if lowest else None)
+    return PrefillOut(bufs.o, bufs.lse, r, bufs.mask if cnn is not None else mask, bufs.idx,
+                      bufs.nret, bufs.cnt, bufs.k_col, bufs.v_col, n_scored,
+                      bufs.death if lowest else None)
 
 
 class DecodeCache:
@@ -106,14 +123,16 @@ class DecodeCache:
         self.win_r = torch.full((B, Hkv, window), float("nan"), dtype=torch.float32, device=dev)
         self.ret_total = torch.zeros(B, Hkv, dtype=torch.int32, device=dev)
         self.meta = torch.zeros(4, dtype=torch.int32, device=dev)
+        # scores of the retained slots' tokens (read under LTE_CAP_LOWEST only)
+        self.ret_r = torch.full((B, Hkv, max(cap, 1)), float("nan"), dtype=torch.float32, device=dev)
         self.sink, self.window, self.cap = sink, window, cap
         self.struct = L.lte_cache(self.k.data_ptr(), self.v.data_ptr(), self.pos.data_ptr(),
                                   self.win_r.data_ptr(), self.ret_total.data_ptr(),
-                                  self.meta.data_ptr())
+                                  self.meta.data_ptr(), self.ret_r.data_ptr())
 
     def init_from_prefill(self, dims, k, v, out: PrefillOut, T_prompt, stream=None):
         L.lte_cache_init_from_prefill(dims, self.struct, k, v, out.r, out.idx, out.cnt, T_prompt,
-                                      out.n_scored, stream)
+                                      out.n_scored, stream, death=out.death)
 
     def retained_positions(self):
         """Sorted retained positions per unit (host copy, for checks)."""
@@ -158,6 +177,8 @@ class HostPrefill:
     def __init__(self, B, T, Hq, Hkv, D, dtype, p: LayerParams, chunk, device="cuda"):
         if B % chunk:
             raise ValueError("the batch must be a multiple of the sub-batch")
+        if p.cap_policy == L.LTE_CAP_LOWEST:
+            raise ValueError("a fed mask carries no scores to rank retained tokens by")
         dev = torch.device(device)
         self.B, self.T, self.chunk, self.p = B, T, chunk, p
         self.dims = p.dims(chunk, T, Hq, Hkv, D, dtype)

@@ -21,7 +21,7 @@ if not os.path.exists(LIB_PATH):
 _lib = C.CDLL(LIB_PATH)
 
 LTE_F32, LTE_BF16 = 0, 1
-LTE_CAP_RECENT, LTE_CAP_FIRST = 0, 1
+LTE_CAP_RECENT, LTE_CAP_FIRST, LTE_CAP_LOWEST = 0, 1, 2
 LTE_WS_PREFILL, LTE_WS_DECODE = 0, 1
 STATUS = {0: "LTE_OK", 1: "LTE_ERR_INVALID_ARG", 2: "LTE_ERR_UNSUPPORTED", 3: "LTE_ERR_CUDA",
           4: "LTE_ERR_TIMEOUT", 5: "LTE_ERR_WORKSPACE", 6: "LTE_ERR_DEVICE"}
@@ -52,7 +52,7 @@ class lte_cnn(C.Structure):
 
 class lte_cache(C.Structure):
     _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("pos", C.c_void_p), ("win_r", C.c_void_p),
-                ("ret_total", C.c_void_p), ("meta", C.c_void_p)]
+                ("ret_total", C.c_void_p), ("meta", C.c_void_p), ("ret_r", C.c_void_p)]
 
 
 _P = C.c_void_p
@@ -62,11 +62,12 @@ _SIG = {
                   _P, _P, _P],
     "lte_evict_compact": [C.POINTER(lte_dims), _P, _P, _I, _P, _P, _P, _P, _P,
                           C.POINTER(lte_strides), _P, _P, _P],
+    "lte_retained_lifetimes": [C.POINTER(lte_dims), _P, _P, _P, _P, _P],
     "lte_sparse_attn_prefill": [C.POINTER(lte_dims), _P, _P, _P, C.POINTER(lte_strides),
-                                C.POINTER(lte_strides), _P, _P, _P, _P, C.POINTER(lte_strides),
-                                _P, _P, C.c_size_t, _P],
+                                C.POINTER(lte_strides), _P, _P, _P, _P, _P,
+                                C.POINTER(lte_strides), _P, _P, C.c_size_t, _P],
     "lte_cache_init_from_prefill": [C.POINTER(lte_dims), C.POINTER(lte_cache), _P, _P,
-                                    C.POINTER(lte_strides), _P, _P, _P, _I, _I, _P],
+                                    C.POINTER(lte_strides), _P, _P, _P, _P, _I, _I, _P],
     "lte_decode_step": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P, _P, _P,
                         _P, _P, _I, _P, C.c_size_t, _P],
     "lte_decode_step_noalloc": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P,
@@ -157,16 +158,24 @@ def lte_evict_compact(dims, r, mask, n_scored, idx, nret, cnt, k=None, v=None, k
           _ptr(cnt), _ptr(k), _ptr(v), st, _ptr(k_col), _ptr(v_col), _stream(stream))
 
 
-def lte_sparse_attn_prefill(dims, q, k, v, cnt, k_col, v_col, o, lse, workspace, stream=None):
-    _call("lte_sparse_attn_prefill", C.byref(dims), _ptr(q), _ptr(k), _ptr(v),
-          C.byref(_strides(q)), C.byref(_strides(k)), _ptr(cnt), _ptr(k_col), _ptr(v_col), _ptr(o),
-          C.byref(_strides(o)), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+def lte_retained_lifetimes(dims, r, idx, nret, death, stream=None):
+    _call("lte_retained_lifetimes", C.byref(dims), _ptr(r), _ptr(idx), _ptr(nret), _ptr(death),
           _stream(stream))
 
 
-def lte_cache_init_from_prefill(dims, cache, k, v, r, idx, cnt, T_prompt, n_scored, stream=None):
+def lte_sparse_attn_prefill(dims, q, k, v, cnt, k_col, v_col, o, lse, workspace, stream=None,
+                            death=None):
+    _call("lte_sparse_attn_prefill", C.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+          C.byref(_strides(q)), C.byref(_strides(k)), _ptr(cnt), _ptr(death), _ptr(k_col),
+          _ptr(v_col), _ptr(o), C.byref(_strides(o)), _ptr(lse), _ptr(workspace),
+          workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def lte_cache_init_from_prefill(dims, cache, k, v, r, idx, cnt, T_prompt, n_scored, stream=None,
+                                death=None):
     _call("lte_cache_init_from_prefill", C.byref(dims), C.byref(cache), _ptr(k), _ptr(v),
-          C.byref(_strides(k)), _ptr(r), _ptr(idx), _ptr(cnt), T_prompt, n_scored, _stream(stream))
+          C.byref(_strides(k)), _ptr(r), _ptr(idx), _ptr(cnt), _ptr(death), T_prompt, n_scored,
+          _stream(stream))
 
 
 def lte_decode_step(dims, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch, workspace,

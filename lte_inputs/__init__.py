@@ -121,6 +121,14 @@ def bernoulli_mask(B, Hkv, T, p, g) -> torch.Tensor:
     return (u < p).to(torch.uint8)
 
 
+def grid_scores(B, Hkv, T, levels, g) -> torch.Tensor:
+    """fp32 [B,Hkv,T] scores drawn uniformly from {0, 1/levels, ..., (levels-1)/levels}:
+    exact in fp32 (levels a power of two), with equal scores frequent when
+    levels is small."""
+    x = torch.randint(0, levels, (B, Hkv, T), generator=g, dtype=torch.int64)
+    return x.to(torch.float32) / levels
+
+
 def rate_mask(B, Hkv, T, rate, g) -> torch.Tensor:
     """Per-KV-head rates ~ U[0, 2*rate] clipped to [0,1], then Bernoulli per
     token; rate >= 1 gives every token."""

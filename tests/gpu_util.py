@@ -62,14 +62,16 @@ def fed_masks(mask: torch.Tensor, sink: int) -> np.ndarray:
     return m
 
 
-def oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap, scale, policy=O.CAP_RECENT):
-    """Oracle o [len(rows), G, D], lse [len(rows), G] for one unit."""
+def oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap, scale, policy=O.CAP_RECENT,
+                r=None):
+    """Oracle o [len(rows), G, D], lse [len(rows), G] for one unit (r [B,Hkv,T]:
+    the scores, for policy "lowest")."""
     Hq, Hkv = q.shape[2], k.shape[2]
     G = Hq // Hkv
     qn = f64(q[b, :, h * G:(h + 1) * G])
     kn, vn = f64(k[b, :, h]), f64(v[b, :, h])
     o, lse, cnt = O.prefill_unit(qn, kn, vn, masks[b, h], sink, window, cap, scale, rows=rows,
-                                 policy=policy)
+                                 policy=policy, r=None if r is None else f64(r[b, h]))
     return o[rows], lse[rows], cnt[rows]
 
 

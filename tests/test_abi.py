@@ -31,7 +31,7 @@ def test_header_declares_expected_entry_points():
     names = _declared()
     for n in ("lte_score", "lte_evict_compact", "lte_sparse_attn_prefill", "lte_decode_step",
               "lte_cache_init_from_prefill", "lte_workspace_bytes", "lte_gla_prefill",
-              "lte_gla_decode_step", "lte_read_device_error"):
+              "lte_gla_decode_step", "lte_read_device_error", "lte_retained_lifetimes"):
         assert n in names
 
 
@@ -62,13 +62,22 @@ def test_host_validation_without_gpu(lib):
                                None, None, None) == 1
     bad = L.make_dims(1, 64, 6, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32)   # Hq % Hkv != 0
     assert f.lte_workspace_bytes(C.byref(bad), 0) == 0
-    pol = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, cap_policy=2)  # no such policy
+    pol = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, cap_policy=3)  # no such policy
     assert f.lte_workspace_bytes(C.byref(pol), 0) == 0
     first = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, L.LTE_CAP_FIRST)
     assert f.lte_workspace_bytes(C.byref(first), 0) >= 16
     d96 = L.make_dims(1, 64, 4, 4, 96, 4, 16, 8, 0.5, 0.1, L.LTE_F32)     # D not in {64,128}
     assert f.lte_sparse_attn_prefill(C.byref(d96), None, None, None, None, None, None, None, None,
-                                     None, None, None, None, 0, None) == 2
+                                     None, None, None, None, None, 0, None) == 2
+    # LTE_CAP_LOWEST: lifetimes need that policy and all pointers; the attention
+    # needs the lifetimes
+    low = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_F32, L.LTE_CAP_LOWEST)
+    p16 = C.c_void_p(16)
+    assert f.lte_workspace_bytes(C.byref(low), 0) >= 16
+    assert f.lte_retained_lifetimes(C.byref(d), p16, p16, p16, p16, None) == 1
+    assert f.lte_retained_lifetimes(C.byref(low), p16, p16, None, p16, None) == 1
+    assert f.lte_sparse_attn_prefill(C.byref(low), p16, p16, p16, None, None, p16, None, p16, p16,
+                                     p16, None, None, p16, 1 << 20, None) == 1
     assert f.lte_workspace_bytes(C.byref(d), 0) >= 16
     assert f.lte_workspace_bytes(C.byref(d), 1) > 16
     # score: range beyond the receptive field -> invalid
@@ -80,6 +89,11 @@ def test_host_validation_without_gpu(lib):
     cache = L.lte_cache(16, 16, 16, 16, 16, 16)
     assert f.lte_decode_step(C.byref(dd), C.byref(cnn), C.byref(cache), C.c_void_p(16),
                              C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), None, 11,
+                             C.c_void_p(16), 1 << 20, None) == 1
+    # decode under LTE_CAP_LOWEST without the retained slots' scores -> invalid
+    dl = L.make_dims(1, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_BF16, L.LTE_CAP_LOWEST)
+    assert f.lte_decode_step(C.byref(dl), C.byref(cnn), C.byref(cache), C.c_void_p(16),
+                             C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), None, 4,
                              C.c_void_p(16), 1 << 20, None) == 1
     # wait probe: null or misaligned flag, limit out of range, missing workspace
     assert f.lte_wait_probe(None, 1, 1000000, C.c_void_p(16), None) == 1

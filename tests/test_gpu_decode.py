@@ -123,6 +123,45 @@ def test_decode_cap_first_policy(layer, cfg):
         assert len(ret_ref[-1]) <= cap
 
 
+@pytest.mark.parametrize("cfg", [
+    # B, Hq, Hkv, D, sink, window, cap, T0, steps, score_batch
+    (2, 8, 2, 128, 2, 32, 6, 100, 100, 8),          # one fused launch per step
+    (2, 8, 2, 128, 2, 32, 6, 40, 160, 4),           # the segment fills during decode
+])
+def test_decode_cap_lowest_policy(layer, cfg):
+    """LTE_CAP_LOWEST through lifetimes, cache set-up and decode: a retained
+    token arriving at a full segment replaces the lowest-scoring held one (or
+    is dropped); outputs and retained sets against the oracle's simulation.
+    The seed is one where no two retained candidates' scores are within
+    2e-5 of each other (20x the fp32 score tolerance), so the ranking is the
+    same in fp32 and float64; the test asserts that gap."""
+    from learnable_kv_token_b200 import lte as L
+    B, Hq, Hkv, D, sink, window, cap, T0, steps, Ds = cfg
+    T = T0 + steps
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T, 531, w_std=0.5)
+    G = Hq // Hkv
+    r_or = {(b, h): O.cnn_scores(f64(k[b, :, h]), f64(v[b, :, h]), oracle_cnn(cnn, h))
+            for b in range(B) for h in range(Hkv)}
+    tau, margin = clean_tau(np.stack(list(r_or.values())), 0.55, 0.85)
+    assert margin > 1e-5
+    for x in r_or.values():
+        kept = np.sort(x[np.isfinite(x) & (x >= tau)])
+        assert np.diff(kept).min() > 20 * R_TOL
+    o_g, lse_g, rets, cache, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, tau, T0, Ds,
+                                             check_every=7, cap_policy=L.LTE_CAP_LOWEST)
+    ret_total = cache.ret_total.cpu()
+    for b in range(B):
+        for h in range(Hkv):
+            o_ref, lse_ref, sets, ret_ref, c_ref = O.decode_unit(
+                f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]), f64(v[b, :, h]), T0, sink,
+                window, cap, tau, oracle_cnn(cnn, h), Ds, scale_of(D), policy=O.CAP_LOWEST)
+            assert_attention_close(f64(o_g[:, b, h * G:(h + 1) * G]), f64(lse_g[:, b, h * G:(h + 1) * G]),
+                                   o_ref, lse_ref, torch.bfloat16, f"unit {b},{h}")
+            for t, rs in rets.items():
+                assert rs[b][h] == ret_ref[t - T0], (b, h, t)
+            assert int(ret_total[b, h]) == c_ref.ret_total <= cap
+
+
 @pytest.mark.parametrize("score_batch", [1, 8])
 def test_decode_causal_cnn(layer, score_batch):
     """A CNN that reads the past only (past1 = k1 - 1, past2 = k2 - 1): every

@@ -246,6 +246,76 @@ def test_prefill_cap_first_policy(layer, case):
             assert_attention_close(o_g, lse_g, o_ref, lse_ref, dtype, f"unit {b},{h}")
 
 
+LOWEST_CASES = [
+    # B, T, Hq, Hkv, D, dtype, sink, window, cap, score levels (few levels: many equal scores)
+    (2, 1100, 8, 2, 128, torch.bfloat16, 4, 128, 24, 1024),   # tcgen05 kernel
+    (1, 900, 16, 4, 128, torch.bfloat16, 4, 64, 40, 8),       # tcgen05 kernel, G = 4, ties
+    (2, 333, 4, 1, 64, torch.bfloat16, 2, 37, 5, 16),         # warp-MMA kernel (head dim 64)
+    (1, 400, 2, 2, 128, torch.float32, 3, 20, 7, 256),        # fp32 kernel
+    (1, 700, 16, 4, 128, torch.bfloat16, 4, 64, 300, 64),     # the cap binds late
+    (1, 300, 8, 2, 128, torch.bfloat16, 2, 30, 0, 64),        # cap 0
+]
+
+
+def _run_prefill_scores(layer, q, k, v, r, sink, window, cap, cap_policy):
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=0.5, cap_policy=cap_policy)
+    qd, kd, vd, rd = _dev(q, k, v, r)
+    out = layer.prefill(qd, kd, vd, p, scores=rd)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("case", LOWEST_CASES)
+def test_prefill_cap_lowest_policy(layer, case):
+    """LTE_CAP_LOWEST: each row attends to the C retained tokens with the
+    highest (score, position) among those that left the window, in every
+    prefill kernel, against the oracle's policy "lowest".  The scores are fed
+    (exact in fp32, so both sides rank the same values)."""
+    from learnable_kv_token_b200 import lte as L
+    B, T, Hq, Hkv, D, dtype, sink, window, cap, levels = case
+    g = LI.generator(400 + T)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, dtype, g)
+    r = LI.grid_scores(B, Hkv, T, levels, g)
+    out = _run_prefill_scores(layer, q, k, v, r, sink, window, cap, L.LTE_CAP_LOWEST)
+    masks = np.stack([[O.retention_mask(f64(r[b, h]), sink, 0.5) for h in range(Hkv)]
+                      for b in range(B)])
+    G = Hq // Hkv
+    rows = list(range(T))
+    for b in range(B):
+        for h in range(Hkv):
+            o_ref, lse_ref, _ = oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap,
+                                            scale_of(D), policy=O.CAP_LOWEST, r=r)
+            o_g = f64(out.o[b, :, h * G:(h + 1) * G])
+            lse_g = f64(out.lse[b, h * G:(h + 1) * G]).T
+            assert_attention_close(o_g, lse_g, o_ref, lse_ref, dtype, f"unit {b},{h}")
+
+
+@pytest.mark.parametrize("levels,cap", [(8, 6), (1024, 6), (4, 1), (64, 0), (64, 500)])
+def test_retained_lifetimes_vs_oracle(layer, levels, cap):
+    """lte_retained_lifetimes, exactly: for every retained count n, the ordinals
+    i < n with death[i] > n are the oracle's C best of the first n retained
+    tokens (and the compacted list equals the oracle's)."""
+    from learnable_kv_token_b200 import lte as L
+    B, T, Hq, Hkv, D, sink, window = 2, 700, 4, 2, 64, 3, 16
+    g = LI.generator(500 + levels + cap)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, torch.bfloat16, g)
+    r = LI.grid_scores(B, Hkv, T, levels, g)
+    out = _run_prefill_scores(layer, q, k, v, r, sink, window, cap, L.LTE_CAP_LOWEST)
+    idx, nret, death = out.idx.cpu().numpy(), out.nret.cpu().numpy(), out.death.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv):
+            rr = f64(r[b, h])
+            cand, n_all, _ = O.compact(O.retention_mask(rr, sink, 0.5))
+            assert int(nret[b, h]) == n_all
+            np.testing.assert_array_equal(idx[b, h, :n_all], cand)
+            d = death[b, h, :n_all]
+            assert (d > np.arange(n_all)).all() and (d <= T + 1).all()
+            for n in range(n_all + 1):
+                held = [i for i in range(n) if d[i] > n]
+                best = set(O.top_by_score(list(cand[:n]), rr, cap))
+                assert held == [i for i in range(n) if cand[i] in best], (b, h, n)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("special", ["window_covers_all", "retain_none", "retain_all", "cap_zero"])
 def test_prefill_special_cases(layer, dtype, special):
