@@ -291,6 +291,68 @@ def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | Non
 
 
 # ---------------------------------------------------------------------------
+# (3b) backward of the prefill attention for fixed attended sets
+#      [LTE, Abstract: the model is trained end to end; the pages give no rule
+#      for differentiating the eviction decisions, so the sets S_t are held
+#      fixed and only the softmax attention over them is differentiated]
+# ---------------------------------------------------------------------------
+
+def prefill_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float, do,
+                          policy: str = CAP_RECENT, r=None):
+    """Gradients of L = sum_t <do_t, o_t> for one (batch element, KV head)
+    unit, o_t the prefill output over the fixed attended set S_t.
+
+    q, do [T, G, D]; k, v [T, D].  Row by row, with P the softmax weights of
+    row t over S_t and o_t = P V_S:
+      dP = do_t V_S^T,  D_t = <do_t, o_t> per head,  dS = P * (dP - D_t),
+      dq_t = scale dS K_S,  dk_S += scale dS^T q_t,  dv_S += P^T do_t.
+    A position attended both from the window and, later, from the retained
+    segment receives both contributions in the same dk / dv row.
+    Returns dq [T, G, D], dk [T, D], dv [T, D] (float64)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    T, G, D = q.shape
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for t in range(T):
+        S = attended_set(t, m, sink, window, cap, policy, r)
+        Ks, Vs = k[S], v[S]
+        logits = scale * (q[t] @ Ks.T)                        # [G, n]
+        P = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        o = P @ Vs
+        dP = do[t] @ Vs.T
+        Dt = (do[t] * o).sum(axis=1, keepdims=True)
+        dS = P * (dP - Dt)
+        dq[t] = scale * (dS @ Ks)
+        dk[S] += scale * (dS.T @ q[t])
+        dv[S] += P.T @ do[t]
+    return dq, dk, dv
+
+
+def prefill_backward(q, k, v, masks, sink: int, window: int, cap: int, do,
+                     scale: float | None = None, policy: str = CAP_RECENT, r=None):
+    """prefill_backward_unit over a batch: q, do [B,T,Hq,D], k, v [B,T,Hkv,D],
+    masks (and r) [B,Hkv,T].  GQA as in ``prefill``: dk, dv of KV head h sum
+    the contributions of its G query heads.  Returns dq, dk, dv (float64)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hkv):
+            gq, gk, gv = prefill_backward_unit(
+                q[b, :, h * G:(h + 1) * G], k[b, :, h], v[b, :, h], masks[b, h], sink, window,
+                cap, scale, do[b, :, h * G:(h + 1) * G], policy, None if r is None else r[b, h])
+            dq[b, :, h * G:(h + 1) * G] = gq
+            dk[b, :, h] = gk
+            dv[b, :, h] = gv
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
 # (4) decode: the inference cache simulated slot by slot  [LTE, Fig. 3]
 #     window as a FIFO of w slots  [SWA-LA, "Viewing SWA from the
 #     linear-state perspective": one slot overwritten per token]
