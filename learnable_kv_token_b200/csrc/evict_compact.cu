@@ -27,6 +27,7 @@ namespace lte {
 
 constexpr int kCompactThreads = 1024;
 constexpr int kCompactSplit = 4;   // CTAs per unit
+constexpr int kCompactPad = 64;    // zeroed slots after the retained rows (one key tile)
 
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                          int nvec, int lane_in_row) {
@@ -116,6 +117,25 @@ compact_kernel(int T, int Hkv, int sink, int n_scored, float tau, const float* _
              lane_in_row);
     copy_row(reinterpret_cast<const uint4*>(v + src), reinterpret_cast<uint4*>(v_col + dst), nvec,
              lane_in_row);
+  }
+  // zero rows (part 3): the sink slots a short sequence leaves empty, [T, sink),
+  // and the kCompactPad slots after the last retained row.  A 64-row tile the
+  // attention kernels load from the segment then holds zeros, never stale
+  // memory, past its valid rows: a masked key has P = 0, and 0 times a stale
+  // NaN or Inf would still poison the output.
+  if (part == kCompactSplit - 1) {
+    const int z0 = sink + carry, z1 = min(sink + T, sink + carry + kCompactPad);
+    const int e0 = T < sink ? T : sink, n_e = sink - e0;     // empty sink slots
+    const int nz = n_e + (z1 > z0 ? z1 - z0 : 0);
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    for (int i = rr; i < nz; i += rows_per_pass) {
+      const int slot = i < n_e ? e0 + i : z0 + (i - n_e);
+      const long long dst = (col0 + slot) * D * elt;
+      if (lane_in_row < nvec) {
+        reinterpret_cast<uint4*>(k_col + dst)[lane_in_row] = zero;
+        reinterpret_cast<uint4*>(v_col + dst)[lane_in_row] = zero;
+      }
+    }
   }
 }
 

@@ -246,6 +246,41 @@ def test_prefill_cap_first_policy(layer, case):
             assert_attention_close(o_g, lse_g, o_ref, lse_ref, dtype, f"unit {b},{h}")
 
 
+@pytest.mark.parametrize("case", [
+    # B, T, Hq, Hkv, D, dtype, sink, window, cap, rate
+    (1, 300, 8, 2, 128, torch.bfloat16, 0, 16, 3, 0.7),      # tcgen05 kernel, no sink
+    (1, 300, 8, 8, 128, torch.bfloat16, 0, 16, 3, 0.7),      # tcgen05 kernel, G = 1
+    (1, 20, 4, 1, 128, torch.bfloat16, 40, 8, 4, 0.5),       # more sink slots than tokens
+    (1, 333, 4, 1, 64, torch.bfloat16, 2, 37, 5, 0.5),       # warp-MMA kernel
+])
+def test_prefill_stale_column_segment(layer, case):
+    """The column segment's buffers start as NaN (stale memory): compaction
+    writes the rows past the retained ones that a 64-row tile can reach, so the
+    output is still finite and equal to the oracle's."""
+    B, T, Hq, Hkv, D, dtype, sink, window, cap, rate = case
+    g = LI.generator(600 + T)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, dtype, g)
+    mask = LI.bernoulli_mask(B, Hkv, T, rate, g)
+    p = layer.LayerParams(sink=sink, window=window, cap=cap)
+    qd, kd, vd, md = _dev(q, k, v, mask)
+    dims = p.dims(B, T, Hq, Hkv, D, dtype)
+    bufs = layer.PrefillBuffers(B, T, Hq, Hkv, D, dtype, sink, dims, "cuda", want_r=False)
+    bufs.k_col.fill_(float("nan"))
+    bufs.v_col.fill_(float("nan"))
+    out = layer.prefill(qd, kd, vd, p, mask=md, bufs=bufs)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out.o.float()).all()) and bool(torch.isfinite(out.lse).all())
+    masks = fed_masks(mask, sink)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hkv):
+            o_ref, lse_ref, _ = oracle_rows(q, k, v, masks, b, h, list(range(T)), sink, window, cap,
+                                            scale_of(D))
+            assert_attention_close(f64(out.o[b, :, h * G:(h + 1) * G]),
+                                   f64(out.lse[b, h * G:(h + 1) * G]).T, o_ref, lse_ref, dtype,
+                                   f"unit {b},{h}")
+
+
 LOWEST_CASES = [
     # B, T, Hq, Hkv, D, dtype, sink, window, cap, score levels (few levels: many equal scores)
     (2, 1100, 8, 2, 128, torch.bfloat16, 4, 128, 24, 1024),   # tcgen05 kernel
