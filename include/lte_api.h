@@ -133,8 +133,11 @@ lte_status lte_score(const lte_dims* d, const lte_cnn* cnn,
  *   nret int32 [B,Hkv]:   number of such positions,
  *   cnt  int32 [B,Hkv,T]: inclusive prefix count cnt[j] = #{i <= j : m_i}.
  * Column segment (k_col, v_col both NULL or both set): [B, Hkv, sink + T, D]
- * contiguous, slot i < sink holds the sink row k[i] (rows i >= T left
- * unwritten), slot sink + i holds k[idx[i]] for i < nret; likewise for v.
+ * contiguous, slot i < sink holds the sink row k[i] (zeros for i >= T),
+ * slot sink + i holds k[idx[i]] for i < nret, and the next 64 slots (those
+ * within the segment) are zeros, so that every 64-row tile the attention
+ * kernels read holds finite values; likewise for v.  Later slots are left
+ * unwritten.
  * ------------------------------------------------------------------------- */
 lte_status lte_evict_compact(const lte_dims* d, const float* r, const uint8_t* mask,
                              int32_t n_scored, int32_t* idx, int32_t* nret, int32_t* cnt,
@@ -187,6 +190,36 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
                                    const int32_t* death, const void* k_col, const void* v_col,
                                    void* o, const lte_strides* o_strides, float* lse,
                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * lte_sparse_attn_backward -- gradients of the prefill sparse attention with
+ * the attended sets held fixed.  [LTE paper, Abstract: the hybrids are
+ * trained end to end; the pages give no gradient for the eviction decisions,
+ * so S_t (as in lte_sparse_attn_prefill) is fixed and only the softmax
+ * attention over it is differentiated.]  With P the softmax weights of row t
+ * (recomputed from lse), o the forward output and dO its incoming gradient:
+ *   D_t = <dO_t, o_t>,  dS = P * (dO V^T - D_t),
+ *   dq = scale dS K,  dk = scale dS^T Q,  dv = P^T dO,
+ * summed, for dk and dv, over the G query heads of a KV head and over every
+ * way a position is attended (window band, sink slot, retained slot).
+ * q, o, dO: [B,T,Hq,D] bf16 contiguous; k, v: [B,T,Hkv,D] bf16 contiguous;
+ * cnt, idx, nret, k_col, v_col: from lte_evict_compact (the column segment
+ * is required); death: from lte_retained_lifetimes, required under
+ * LTE_CAP_LOWEST, else ignored; o and lse (natural log, [B,Hq,T]): from
+ * lte_sparse_attn_prefill on the same inputs.
+ * Outputs (overwritten): dq fp32 [B,T,Hq,D], dk, dv fp32 [B,T,Hkv,D].
+ * Arithmetic: fp32 accumulation; P and dS rounded to bf16 for the products;
+ * dk and dv of retained and sink positions add fp32 partial sums with
+ * atomics, so their last bits may vary between runs.
+ * bf16 only, G = Hq/Hkv dividing 64 (else LTE_ERR_UNSUPPORTED).
+ * Workspace: lte_workspace_bytes(d, LTE_WS_BACKWARD) (error word + D_t).
+ * ------------------------------------------------------------------------- */
+lte_status lte_sparse_attn_backward(const lte_dims* d, const void* q, const void* k, const void* v,
+                                    const int32_t* cnt, const int32_t* death, const int32_t* idx,
+                                    const int32_t* nret, const void* k_col, const void* v_col,
+                                    const void* o, const float* lse, const void* dO, float* dq,
+                                    float* dk, float* dv, void* workspace, size_t ws_bytes,
+                                    void* stream);
 
 /* ---------------------------------------------------------------------------
  * Decode cache.  [LTE paper, Fig. 3 caption: circular window segment plus an
@@ -292,7 +325,7 @@ lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const 
                                    const void* q_t, const void* k_t, const void* v_t,
                                    void* o_t, float* lse_t, int32_t score_batch, void* stream);
 
-enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1 };
+enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1, LTE_WS_BACKWARD = 2 };
 
 /* Bytes of workspace a call needs (>= 16: the first 16 bytes hold the device
  * error word).  Returns 0 for invalid dims. */

@@ -127,7 +127,38 @@ size_t lte_workspace_bytes(const lte_dims* d, int32_t which) {
   if (check_dims(d) != LTE_OK) return 0;
   if (which == LTE_WS_PREFILL) return kErrBytes + lte::attn_prefill_scratch_bytes(d);
   if (which == LTE_WS_DECODE) return kErrBytes + lte::decode_scratch_bytes(d);
+  if (which == LTE_WS_BACKWARD) return kErrBytes + lte::attn_backward_scratch_bytes(d);
   return 0;
+}
+
+lte_status lte_sparse_attn_backward(const lte_dims* d, const void* q, const void* k, const void* v,
+                                    const int32_t* cnt, const int32_t* death, const int32_t* idx,
+                                    const int32_t* nret, const void* k_col, const void* v_col,
+                                    const void* o, const float* lse, const void* dO, float* dq,
+                                    float* dk, float* dv, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (!q || !k || !v || !cnt || !idx || !nret || !k_col || !v_col || !o || !lse || !dO || !dq ||
+      !dk || !dv)
+    return LTE_ERR_INVALID_ARG;
+  if (d->cap_policy == LTE_CAP_LOWEST && death == nullptr) return LTE_ERR_INVALID_ARG;
+  const void* vec[] = {q, k, v, k_col, v_col, o, dO, dq, dk, dv};
+  for (const void* p : vec)
+    if (!aligned16(p)) return LTE_ERR_INVALID_ARG;
+  if (d->dtype != LTE_BF16) return LTE_ERR_UNSUPPORTED;
+  const int G = d->Hq / d->Hkv;
+  if (64 % G != 0 || G > 16) return LTE_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned16(workspace)) return LTE_ERR_WORKSPACE;
+  if (ws_bytes < lte_workspace_bytes(d, LTE_WS_BACKWARD)) return LTE_ERR_WORKSPACE;
+  lte::BackwardArgs a{};
+  a.d = d;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO;
+  a.cnt = cnt; a.death = d->cap_policy == LTE_CAP_LOWEST ? death : nullptr; a.idx = idx;
+  a.nret = nret; a.k_col = k_col; a.v_col = v_col; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.scratch = static_cast<char*>(workspace) + kErrBytes;
+  return from_cuda(lte::attn_backward(a, as_stream(stream)));
 }
 
 lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void* k,

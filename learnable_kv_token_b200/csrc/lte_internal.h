@@ -53,6 +53,19 @@ bool attn_prefill_tc_layout_ok(const PrefillArgs& a);
 cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
 size_t attn_prefill_scratch_bytes(const lte_dims* d);
 
+// attn_backward_mma.cu
+struct BackwardArgs {
+  const lte_dims* d;
+  const void *q, *k, *v, *o, *dO;   // contiguous [B,T,H,D] bf16
+  const int32_t *cnt, *death, *idx, *nret;
+  const void *k_col, *v_col;
+  const float* lse;
+  float *dq, *dk, *dv;
+  void* scratch;                    // workspace after the error word
+};
+size_t attn_backward_scratch_bytes(const lte_dims* d);
+cudaError_t attn_backward(const BackwardArgs& a, cudaStream_t stream);
+
 // decode.cu
 size_t decode_scratch_bytes(const lte_dims* d);
 bool decode_supported(const lte_dims* d);

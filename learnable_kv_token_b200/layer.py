@@ -111,6 +111,24 @@ def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers |
                       bufs.death if lowest else None)
 
 
+def backward(q, k, v, out: PrefillOut, do, p: LayerParams, stream=None):
+    """Gradients (fp32) of the prefill attention for the attended sets that
+    `out` (from prefill on the same q, k, v) used, given dO = do.
+    Returns dq [B,T,Hq,D], dk, dv [B,T,Hkv,D]."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
+    dev = q.device
+    dq = torch.empty(B, T, Hq, D, dtype=torch.float32, device=dev)
+    dk = torch.empty(B, T, Hkv, D, dtype=torch.float32, device=dev)
+    dv = torch.empty(B, T, Hkv, D, dtype=torch.float32, device=dev)
+    ws_bytes = L.lte_workspace_bytes(dims, L.LTE_WS_BACKWARD)
+    ws = torch.zeros((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    L.lte_sparse_attn_backward(dims, q, k, v, out.cnt, out.death, out.idx, out.nret, out.k_col,
+                               out.v_col, out.o, out.lse, do, dq, dk, dv, ws, stream)
+    return dq, dk, dv
+
+
 class DecodeCache:
     """Caller-owned decode cache (window ring + sink slots + retained ring)."""
 

@@ -22,7 +22,7 @@ _lib = C.CDLL(LIB_PATH)
 
 LTE_F32, LTE_BF16 = 0, 1
 LTE_CAP_RECENT, LTE_CAP_FIRST, LTE_CAP_LOWEST = 0, 1, 2
-LTE_WS_PREFILL, LTE_WS_DECODE = 0, 1
+LTE_WS_PREFILL, LTE_WS_DECODE, LTE_WS_BACKWARD = 0, 1, 2
 STATUS = {0: "LTE_OK", 1: "LTE_ERR_INVALID_ARG", 2: "LTE_ERR_UNSUPPORTED", 3: "LTE_ERR_CUDA",
           4: "LTE_ERR_TIMEOUT", 5: "LTE_ERR_WORKSPACE", 6: "LTE_ERR_DEVICE"}
 
@@ -66,6 +66,7 @@ _SIG = {
     "lte_sparse_attn_prefill": [C.POINTER(lte_dims), _P, _P, _P, C.POINTER(lte_strides),
                                 C.POINTER(lte_strides), _P, _P, _P, _P, _P,
                                 C.POINTER(lte_strides), _P, _P, C.c_size_t, _P],
+    "lte_sparse_attn_backward": [C.POINTER(lte_dims)] + [_P] * 16 + [C.c_size_t, _P],
     "lte_cache_init_from_prefill": [C.POINTER(lte_dims), C.POINTER(lte_cache), _P, _P,
                                     C.POINTER(lte_strides), _P, _P, _P, _P, _I, _I, _P],
     "lte_decode_step": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P, _P, _P,
@@ -168,6 +169,14 @@ def lte_sparse_attn_prefill(dims, q, k, v, cnt, k_col, v_col, o, lse, workspace,
     _call("lte_sparse_attn_prefill", C.byref(dims), _ptr(q), _ptr(k), _ptr(v),
           C.byref(_strides(q)), C.byref(_strides(k)), _ptr(cnt), _ptr(death), _ptr(k_col),
           _ptr(v_col), _ptr(o), C.byref(_strides(o)), _ptr(lse), _ptr(workspace),
+          workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def lte_sparse_attn_backward(dims, q, k, v, cnt, death, idx, nret, k_col, v_col, o, lse, do, dq,
+                             dk, dv, workspace, stream=None):
+    _call("lte_sparse_attn_backward", C.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(cnt),
+          _ptr(death), _ptr(idx), _ptr(nret), _ptr(k_col), _ptr(v_col), _ptr(o), _ptr(lse), _ptr(do),
+          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
           workspace.numel() * workspace.element_size(), _stream(stream))
 
 
