@@ -466,10 +466,23 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
     t_attn = timed(lambda: L.lte_sparse_attn_prefill(dims, q, k, v, bufs.cnt, bufs.k_col,
                                                      bufs.v_col, bufs.o, bufs.lse, bufs.ws, stream))
     assert L.lte_read_device_error(bufs.ws) == (0, 0)
+    # backward of the attention (fixed attended sets); dO = q stands in for the
+    # incoming gradient (any [B,T,Hq,D] tensor: the work does not depend on it)
+    dq = torch.empty(B, T, Hq, D, dtype=torch.float32, device=device)
+    dk = torch.empty(B, T, Hkv, D, dtype=torch.float32, device=device)
+    dv = torch.empty_like(dk)
+    ws_b = torch.zeros(L.lte_workspace_bytes(dims, L.LTE_WS_BACKWARD) + 16, dtype=torch.uint8,
+                       device=device)
+    t_bwd = timed(lambda: L.lte_sparse_attn_backward(dims, q, k, v, bufs.cnt, None, bufs.idx,
+                                                     bufs.nret, bufs.k_col, bufs.v_col, bufs.o,
+                                                     bufs.lse, q, dq, dk, dv, ws_b, stream))
+    assert L.lte_read_device_error(ws_b) == (0, 0)
+    del dq, dk, dv, ws_b
     mask = bufs.mask.cpu().numpy()
     nret = int(bufs.nret.sum())
     pairs = attended_pairs(mask, wl.sink, wl.window, wl.cap).sum()
     attn_flops = 4.0 * D * wl.G * float(pairs)
+    bwd_flops = 2.5 * attn_flops           # S, dP, dQ, dK, dV over the attended pairs
     score_flops = 2.0 * B * Hkv * n_scored * (wl.c_hid * 2 * D * wl.k1 + wl.c_hid * wl.k2)
     score_bytes = B * T * Hkv * D * 2 * 2 + B * Hkv * n_scored * 5
     compact_bytes = (B * Hkv * T * (1 + 8) + B * Hkv * 4
@@ -510,6 +523,9 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
         "a2_compact_ms": t_compact, "a2_roofline": hbm(compact_bytes, t_compact),
         "a3_attn_ms": t_attn, "a3_roofline": tensor(attn_flops, t_attn),
         "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
+        "a3b_backward_ms": t_bwd, "a3b_roofline": tensor(bwd_flops, t_bwd),
+        "a3b_note": "lte_sparse_attn_backward (delta, dQ, dK/dV window, dK/dV column: 4 "
+                    "launches, mma.sync) on the same scored mask; FLOPs = 2.5 x the forward's",
         "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),
         "a7_gla_decode_us": 1e3 * t_gla_dec, "a7_decode_roofline": hbm(gla_dec_bytes, t_gla_dec),
         "pair_prefill": {"value": DI.job_throughput(B * T, world, (t_gla + lte_prefill_ms) / 1e3),
@@ -517,7 +533,7 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
         "pair_decode": (None if lte_decode_ms is None else
                         {"value": DI.job_throughput(B, world, (t_gla_dec + lte_decode_ms) / 1e3),
                          "unit": "tokens/s", "us": 1e3 * (t_gla_dec + lte_decode_ms)}),
-        "launches": 2 + 5 * 3 + 5 + 50,
+        "launches": 2 + 5 * 3 + 5 + 50 + 4 * 7,
     }
 
 
