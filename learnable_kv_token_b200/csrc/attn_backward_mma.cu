@@ -36,6 +36,7 @@
 #include "lte_common.cuh"
 #include "lte_internal.h"
 #include "mma_sync.cuh"
+#include "attn_backward.cuh"
 
 namespace lte {
 namespace bwd {
@@ -44,23 +45,6 @@ constexpr int kRows = 64;      // query rows per tile (tokens x heads)
 constexpr int kKeys = 64;      // keys per tile
 constexpr int kThreads = 128;  // four warps, 16 rows (dQ) or 16 keys (dK, dV) each
 constexpr int kSplitRows = 32; // row tiles per CTA of the column pass
-
-struct Args {
-  int T, Hq, Hkv, G, TOK, sink, window, cap, cap_policy;
-  float scale, scale_log2;
-  const __nv_bfloat16 *q, *k, *v, *o, *dO, *k_col, *v_col;
-  const int32_t *cnt, *death, *idx, *nret;
-  const float* lse;       // natural log, [B, Hq, T]
-  float* delta;           // [B, Hq, T]
-  float *dq, *dk, *dv;    // fp32, [B,T,Hq,D] and [B,T,Hkv,D]
-};
-
-// retained count a row sees and the start of its retained range
-__device__ __forceinline__ void row_range(const Args& a, long long crow, int t, int& lo, int& hi) {
-  hi = 0;
-  if (t < a.T && t >= a.window) hi = held_retained(__ldg(a.cnt + crow + t - a.window), a.cap, a.cap_policy);
-  lo = (a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
-}
 
 // ---------------------------------------------------------------- D_t
 template <int D>
@@ -595,19 +579,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const Args a, int
 }
 
 template <int D>
-cudaError_t launch(const Args& a, int B, cudaStream_t stream) {
+cudaError_t launch(const Args& a, int B, bool dq_tc, DevError* err, cudaStream_t stream) {
   const long long rows = (long long)B * a.T * a.Hq;
   bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(rows, a.o, a.dO, a.T, a.Hq,
                                                                        a.delta);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem_dq = 2 * (size_t)kRows * D * 2 + 2 * 2 * (size_t)kKeys * D * 2;
-  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem_dq);
-  if (e != cudaSuccess) return e;
-  const int n_tiles = (a.T + a.TOK - 1) / a.TOK;
-  bwd_dq_kernel<D><<<dim3(n_tiles, a.Hkv, B), kThreads, smem_dq, stream>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (dq_tc) {
+    if ((e = attn_backward_dq_tc(a, B, err, stream)) != cudaSuccess) return e;
+  } else {
+    const size_t smem_dq = 2 * (size_t)kRows * D * 2 + 2 * 2 * (size_t)kKeys * D * 2;
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_dq);
+    if (e != cudaSuccess) return e;
+    const int n_tiles = (a.T + a.TOK - 1) / a.TOK;
+    bwd_dq_kernel<D><<<dim3(n_tiles, a.Hkv, B), kThreads, smem_dq, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const size_t smem_kv = 2 * (size_t)kKeys * D * 2 + 2 * 2 * (size_t)kRows * D * 2 +
                          2 * 2 * kRows * sizeof(float) + 2 * 3 * kRows * sizeof(int);
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -646,8 +634,10 @@ cudaError_t attn_backward(const BackwardArgs& g, cudaStream_t stream) {
   a.cnt = g.cnt; a.death = g.death; a.idx = g.idx; a.nret = g.nret; a.lse = g.lse;
   a.delta = reinterpret_cast<float*>(g.scratch);
   a.dq = g.dq; a.dk = g.dk; a.dv = g.dv;
-  if (d->D == 128) return bwd::launch<128>(a, d->B, stream);
-  return bwd::launch<64>(a, d->B, stream);
+  // dQ on tcgen05 where it applies (head dim 128), else on the warp-MMA kernel
+  const bool dq_tc = attn_backward_dq_tc_supported(d);
+  if (d->D == 128) return bwd::launch<128>(a, d->B, dq_tc, g.err, stream);
+  return bwd::launch<64>(a, d->B, dq_tc, g.err, stream);
 }
 
 }  // namespace lte

@@ -1,0 +1,303 @@
+// dQ of the prefill sparse attention's backward on 5th-generation tensor
+// cores (tcgen05 + TMEM), head dim 128, bf16 operands, fp32 accumulation.
+//
+// "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention
+// and Contextualized Learnable Token Eviction", Abstract (trained end to end)
+// and Fig. 2 caption (right): the attended sets S_t, held fixed.  Per query
+// row, with P recomputed from the forward's lse and D_t = <dO_t, o_t>:
+//   dS = P * (dO V^T - D_t),   dQ = scale dS K.
+//
+// One CTA of 128 threads per 128 query rows (128/G tokens x the G heads of a
+// KV head, token-major), one row per thread; two CTAs share an SM (112 KiB of
+// shared memory and 256 TMEM columns each).  Q and dO stay in shared memory;
+// per 64-key tile of the forward's key ranges (sink slots and retained slots
+// of the column segment, window band of k):
+//   1. K and V of the tile arrive by cp.async (zero-filled past the tile's
+//      valid rows) in the 128-byte-swizzled K-major layout;
+//   2. one thread issues S = Q K^T and dP = dO V^T (M128 N64 K128, both
+//      operands in shared memory) into TMEM and commits;
+//   3. each thread reads its row of S and dP, forms P (masked keys 0) and
+//      dS = P (dP - D_t), and writes dS as bf16 into shared memory (the A
+//      operand of the next product);
+//   4. one thread issues dQ += dS K (M128 N128 K64; K as an N-contiguous B
+//      operand) into the TMEM accumulator and commits; the tile's buffers are
+//      reused once that product has completed.
+// Every wait is bounded; on expiry the CTA records LTE_ERR_TIMEOUT, drains
+// what it issued, frees its TMEM and leaves.
+#include <math.h>
+
+#include "attn_backward.cuh"
+#include "lte_common.cuh"
+#include "lte_internal.h"
+#include "tc_ptx.cuh"
+
+namespace lte {
+namespace bwdtc {
+
+using namespace tc;
+
+constexpr int HD = 128;
+constexpr int kRowsTc = 128;                    // query rows per CTA
+constexpr int kKeysTc = 64;                     // keys per tile
+constexpr int kThreadsTc = 128;
+constexpr uint32_t kQ = 0;                      // [128][128] bf16: two 64-column halves of 16 KiB
+constexpr uint32_t kDO = 32768;                 // same for dO
+constexpr uint32_t kK = 65536;                  // [64][128]: two halves of 8 KiB
+constexpr uint32_t kV = 81920;
+constexpr uint32_t kDS = 98304;                 // [128][64] bf16 (one half)
+constexpr uint32_t kBar = 114688;               // bar_s, bar_q, abort flag, TMEM slot
+constexpr int kSmemBytes = kBar + 64;
+constexpr int kTmemCols = 256;                  // S 0..63, dP 64..127, dQ 128..255
+constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128;
+
+// byte offset of 16-byte chunk c16 (0..15) of row r in a K-major [rows][128]
+// bf16 tile stored as two 64-column halves, 128-byte swizzle
+__device__ __forceinline__ uint32_t sw(int rows, int r, int c16) {
+  return (uint32_t)((c16 >> 3) * rows * 128 + r * 128 + ((((c16 & 7) ^ (r & 7))) << 4));
+}
+__device__ __forceinline__ void cpa16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+__device__ __forceinline__ void cpa_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
+__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Args a, DevError* err) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sb = sa(sm);
+  if ((sb & 1023u) != 0) {                      // swizzle atoms need 1 KiB alignment
+    if (threadIdx.x == 0) record_error(err, LTE_ERR_DEVICE, 403);
+    return;
+  }
+  const uint32_t bar_s = sb + kBar, bar_q = sb + kBar + 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kBar + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kBar + 20);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int G = a.G, TOK = kRowsTc / G;
+  const int n_tiles = (a.T + TOK - 1) / TOK;
+  const int t0 = (n_tiles - 1 - (int)blockIdx.x) * TOK;          // late (heavy) tiles first
+  const int h = blockIdx.y, b = blockIdx.z, u = b * a.Hkv + h;
+  const int t_last = min(t0 + TOK - 1, a.T - 1);
+  const long long crow = (long long)u * a.T;
+  const long long col_base = (long long)u * (a.sink + a.T);
+  const bool lowest = a.death != nullptr;
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_q, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     sa(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // Q and dO rows (row rho = token * G + head; rows past T zero)
+  for (int i = tid; i < kRowsTc * 16; i += kThreadsTc) {
+    const int r = i >> 4, c = i & 15;
+    const int tt = t0 + r / G, g = r % G;
+    const bool ok = tt < a.T;
+    const long long off = ok ? (((long long)b * a.T + tt) * a.Hq + h * G + g) * HD + c * 8 : 0;
+    cpa16(sb + kQ + sw(kRowsTc, r, c), a.q + off, ok);
+    cpa16(sb + kDO + sw(kRowsTc, r, c), a.dO + off, ok);
+  }
+  cpa_commit();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+
+  // this thread's row
+  const int tt = t0 + tid / G, gq = tid % G;
+  int lo_r, hi_r;
+  bwd::row_range(a, crow, tt, lo_r, hi_r);
+  if (lowest) lo_r = 0;
+  float lse2 = 0.f, dl = 0.f;
+  if (tt < a.T) {
+    const long long li = ((long long)b * a.Hq + h * G + gq) * a.T + tt;
+    lse2 = a.lse[li] * 1.4426950408889634f;
+    dl = a.delta[li];
+  }
+
+  // key ranges of the tile: 0 sink slots, 1 retained slots, 2 window band
+  int start[3], count[3];
+  {
+    int lo_f, n_first, lo_l, n_last;
+    bwd::row_range(a, crow, t0, lo_f, n_first);
+    bwd::row_range(a, crow, t_last, lo_l, n_last);
+    const int lo_min = lowest ? 0 : lo_f;
+    int nsink = t_last - a.window + 1;
+    nsink = nsink < 0 ? 0 : (nsink > a.sink ? a.sink : nsink);
+    nsink = nsink > a.T ? a.T : nsink;
+    const int w_lo = t0 - a.window + 1 > 0 ? t0 - a.window + 1 : 0;
+    start[0] = 0; count[0] = nsink;
+    start[1] = a.sink + lo_min; count[1] = (a.cap > 0 && n_last > lo_min) ? n_last - lo_min : 0;
+    start[2] = w_lo; count[2] = t_last - w_lo + 1;
+  }
+  const int n0 = (count[0] + kKeysTc - 1) / kKeysTc, n1 = (count[1] + kKeysTc - 1) / kKeysTc;
+  const int total = n0 + n1 + (count[2] + kKeysTc - 1) / kKeysTc;
+
+  const uint32_t id_s = idesc(kRowsTc, kKeysTc, false);     // S, dP: K-major A and B
+  const uint32_t id_q = idesc(kRowsTc, HD, true);           // dQ: K as an N-contiguous B
+  bool ok = true;
+  int issued_q = 0;                                         // dQ products committed
+  for (int j = 0; j < total && ok; ++j) {
+    int rg, it = j;
+    if (it < n0) rg = 0;
+    else if (it < n0 + n1) { rg = 1; it -= n0; }
+    else { rg = 2; it -= n0 + n1; }
+    const int key0 = start[rg] + it * kKeysTc;
+    const int nk = min(kKeysTc, count[rg] - it * kKeysTc);
+    // 1. K, V of the tile (the previous tile's products have completed)
+    for (int i = tid; i < kKeysTc * 16; i += kThreadsTc) {
+      const int r = i >> 4, c = i & 15;
+      const bool v_ok = r < nk;
+      long long e = 0;
+      if (v_ok) {
+        const int key = key0 + r;
+        e = rg == 2 ? (((long long)b * a.T + key) * a.Hkv + h) * HD + c * 8
+                    : (col_base + key) * HD + c * 8;
+      }
+      const __nv_bfloat16* kb = rg == 2 ? a.k : a.k_col;
+      const __nv_bfloat16* vb = rg == 2 ? a.v : a.v_col;
+      cpa16(sb + kK + sw(kKeysTc, r, c), kb + e, v_ok);
+      cpa16(sb + kV + sw(kKeysTc, r, c), vb + e, v_ok);
+    }
+    cpa_commit();
+    cpa_wait_all();
+    fence_proxy_async();                                     // generic writes -> tensor core
+    __syncthreads();
+    // 2. S = Q K^T, dP = dO V^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dq_ = sdesc(sb + kQ, 16, 1024), ddo = sdesc(sb + kDO, 16, 1024);
+      const uint64_t dk = sdesc(sb + kK, 16, 1024), dv = sdesc(sb + kV, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t oa = ((ks >> 2) * (kRowsTc * 128) + (ks & 3) * 32) >> 4;
+        const uint32_t ob = ((ks >> 2) * (kKeysTc * 128) + (ks & 3) * 32) >> 4;
+        mma_f16(tmem + kColS, dq_ + oa, dk + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16(tmem + kColDP, ddo + oa, dv + ob, id_s, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_s);
+    }
+    ok = mbar_wait(bar_s, j & 1, abort_flag, err, 401);
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc_fence_after();
+    // 3. P and dS of this row
+    {
+      uint32_t rs[32], rp[32];
+      uint32_t pkd[32];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        tmem_ld32(lane_addr + kColS + half * 32, rs);
+        tmem_ld32(lane_addr + kColDP + half * 32, rp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float ds2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kk = half * 32 + c + e, key = key0 + kk;
+            bool m = kk < nk && tt < a.T;
+            if (m) {
+              if (rg == 2) m = key <= tt && key > tt - a.window;
+              else if (key < a.sink) m = key <= tt - a.window;
+              else
+                m = (key - a.sink) >= lo_r && (key - a.sink) < hi_r &&
+                    (!lowest || __ldg(a.death + crow + key - a.sink) > hi_r);
+            }
+            const float p = m ? exp2f(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -lse2)) : 0.f;
+            ds2[e] = p * (__uint_as_float(rp[c + e]) - dl);
+          }
+          pkd[half * 16 + (c >> 1)] = pk2(ds2[0], ds2[1]);
+        }
+      }
+      // the dS row (64 keys = 128 bytes) into the swizzled K-major A operand
+      uint8_t* row = sm + kDS + tid * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(row + ((c ^ (tid & 7)) << 4)) =
+            make_uint4(pkd[4 * c], pkd[4 * c + 1], pkd[4 * c + 2], pkd[4 * c + 3]);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    // 4. dQ += dS K
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dds = sdesc(sb + kDS, 16, 1024);
+      const uint64_t dkb = sdesc(sb + kK, kKeysTc * 128, 1024);   // K: N-contiguous, halves 8 KiB apart
+#pragma unroll
+      for (int ks = 0; ks < kKeysTc / 16; ++ks)
+        mma_f16(tmem + kColDQ, dds + ((ks * 32) >> 4), dkb + ((ks * 2048) >> 4), id_q,
+                (j > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(bar_q);
+    }
+    ++issued_q;
+    ok = mbar_wait(bar_q, j & 1, abort_flag, err, 402);
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc_fence_after();
+  }
+  if (ok) {
+    // dQ row: scale, fp32 out (every lane loads: tcgen05.ld is warp-collective)
+    float* out = a.dq + (((long long)b * a.T + min(tt, a.T - 1)) * a.Hq + h * G + gq) * HD;
+#pragma unroll 1
+    for (int c0 = 0; c0 < HD; c0 += 32) {
+      uint32_t r[32];
+      if (total > 0) {
+        tmem_ld32(lane_addr + kColDQ + c0, r);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0u;
+      }
+      if (tt < a.T) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(out + c0 + e) =
+              make_float4(__uint_as_float(r[e]) * a.scale, __uint_as_float(r[e + 1]) * a.scale,
+                          __uint_as_float(r[e + 2]) * a.scale, __uint_as_float(r[e + 3]) * a.scale);
+      }
+    }
+  } else if (tid == 0) {
+    // drain the products this CTA issued before its TMEM is freed
+    mbar_drain(bar_s, 0);
+    mbar_drain(bar_s, 1);
+    if (issued_q > 0) mbar_drain(bar_q, (issued_q - 1) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+}
+
+}  // namespace bwdtc
+
+bool attn_backward_dq_tc_supported(const lte_dims* d) {
+  const int G = d->Hq / d->Hkv;
+  return d->D == bwdtc::HD && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
+}
+
+cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
+  using namespace bwdtc;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int TOK = kRowsTc / a.G;
+  const int n_tiles = (a.T + TOK - 1) / TOK;
+  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsTc, kSmemBytes, stream>>>(a, err);
+  return cudaGetLastError();
+}
+
+}  // namespace lte

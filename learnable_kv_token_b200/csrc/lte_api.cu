@@ -157,6 +157,7 @@ lte_status lte_sparse_attn_backward(const lte_dims* d, const void* q, const void
   a.cnt = cnt; a.death = d->cap_policy == LTE_CAP_LOWEST ? death : nullptr; a.idx = idx;
   a.nret = nret; a.k_col = k_col; a.v_col = v_col; a.lse = lse;
   a.dq = dq; a.dk = dk; a.dv = dv;
+  a.err = reinterpret_cast<lte::DevError*>(workspace);
   a.scratch = static_cast<char*>(workspace) + kErrBytes;
   return from_cuda(lte::attn_backward(a, as_stream(stream)));
 }

@@ -111,10 +111,11 @@ def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers |
                       bufs.death if lowest else None)
 
 
-def backward(q, k, v, out: PrefillOut, do, p: LayerParams, stream=None):
+def backward(q, k, v, out: PrefillOut, do, p: LayerParams, stream=None, check_errors=False):
     """Gradients (fp32) of the prefill attention for the attended sets that
     `out` (from prefill on the same q, k, v) used, given dO = do.
-    Returns dq [B,T,Hq,D], dk, dv [B,T,Hkv,D]."""
+    Returns dq [B,T,Hq,D], dk, dv [B,T,Hkv,D].  check_errors: synchronise and
+    raise if a device-side check or wait failed."""
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
     dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
@@ -126,6 +127,10 @@ def backward(q, k, v, out: PrefillOut, do, p: LayerParams, stream=None):
     ws = torch.zeros((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
     L.lte_sparse_attn_backward(dims, q, k, v, out.cnt, out.death, out.idx, out.nret, out.k_col,
                                out.v_col, out.o, out.lse, do, dq, dk, dv, ws, stream)
+    if check_errors:
+        code, where = L.lte_read_device_error(ws, stream)
+        if code != 0:
+            raise L.LteError(f"lte_sparse_attn_backward (device check {where})", code)
     return dq, dk, dv
 
 

@@ -69,7 +69,7 @@ def test_backward_vs_oracle(layer, case):
         mask = LI.bernoulli_mask(B, Hkv, T, src, g)
         out = layer.prefill(qd, kd, vd, p, mask=mask.cuda())
         masks, r64 = fed_masks(mask, sink), None
-    dq, dk, dv = layer.backward(qd, kd, vd, out, dod, p)
+    dq, dk, dv = layer.backward(qd, kd, vd, out, dod, p, check_errors=True)
     torch.cuda.synchronize()
     rq, rk, rv = O.prefill_backward(f64(q), f64(k), f64(v), masks, sink, window, cap, f64(do),
                                     scale_of(D), opol, r64)
@@ -90,7 +90,7 @@ def test_backward_gradient_check_direction(layer):
     p = layer.LayerParams(sink=sink, window=window, cap=cap)
     qd, kd, vd, dod, md = (x.cuda() for x in (q, k, v, do, mask))
     out = layer.prefill(qd, kd, vd, p, mask=md)
-    dq, _, _ = layer.backward(qd, kd, vd, out, dod, p)
+    dq, _, _ = layer.backward(qd, kd, vd, out, dod, p, check_errors=True)
     # the oracle's forward in float64 along q + eps * e, e a random direction
     e = LI.normal((B, T, Hq, D), 1.0, torch.float32, g)
     masks = fed_masks(mask, sink)
