@@ -525,7 +525,7 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
         "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
         "a3b_backward_ms": t_bwd, "a3b_roofline": tensor(bwd_flops, t_bwd),
         "a3b_note": "lte_sparse_attn_backward (delta, dQ, dK/dV window, dK/dV column: 4 "
-                    "launches, mma.sync) on the same scored mask; FLOPs = 2.5 x the forward's",
+                    "launches, tcgen05) on the same scored mask; FLOPs = 2.5 x the forward's",
         "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),
         "a7_gla_decode_us": 1e3 * t_gla_dec, "a7_decode_roofline": hbm(gla_dec_bytes, t_gla_dec),
         "pair_prefill": {"value": DI.job_throughput(B * T, world, (t_gla + lte_prefill_ms) / 1e3),

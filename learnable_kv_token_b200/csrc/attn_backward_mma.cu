@@ -596,6 +596,7 @@ cudaError_t launch(const Args& a, int B, bool dq_tc, DevError* err, cudaStream_t
     bwd_dq_kernel<D><<<dim3(n_tiles, a.Hkv, B), kThreads, smem_dq, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (dq_tc) return attn_backward_dkdv_tc(a, B, err, stream);   // dK, dV on tcgen05 as well
   const size_t smem_kv = 2 * (size_t)kKeys * D * 2 + 2 * 2 * (size_t)kRows * D * 2 +
                          2 * 2 * kRows * sizeof(float) + 2 * 3 * kRows * sizeof(int);
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -634,7 +635,7 @@ cudaError_t attn_backward(const BackwardArgs& g, cudaStream_t stream) {
   a.cnt = g.cnt; a.death = g.death; a.idx = g.idx; a.nret = g.nret; a.lse = g.lse;
   a.delta = reinterpret_cast<float*>(g.scratch);
   a.dq = g.dq; a.dk = g.dk; a.dv = g.dv;
-  // dQ on tcgen05 where it applies (head dim 128), else on the warp-MMA kernel
+  // tcgen05 kernels where they apply (head dim 128), else the warp-MMA kernels
   const bool dq_tc = attn_backward_dq_tc_supported(d);
   if (d->D == 128) return bwd::launch<128>(a, d->B, dq_tc, g.err, stream);
   return bwd::launch<64>(a, d->B, dq_tc, g.err, stream);

@@ -282,11 +282,368 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
                  : "memory");
 }
 
+// ---------------------------------------------------------------- dK, dV
+// One CTA of 256 threads per 128-key tile (keys of k for the window part,
+// kColumn = false; slots of the column segment, kColumn = true, for this
+// CTA's share of the attending rows).  Keys are the MMA rows: per 64-row
+// tile of attending query rows,
+//   S^T = K Q^T, dP^T = V dO^T            (M128 N64 K128, SS)
+//   P^T, dS^T = P^T (dP^T - D)             (thread pair per key row, 32 columns each)
+//   dV += P^T dO, dK += dS^T Q             (M128 N128 K64; dO, Q as N-contiguous B)
+// with Q and dO of the next row tile loading (cp.async, double-buffered)
+// while the current one is processed.  TMEM: S^T 0..63, dP^T 64..127,
+// dV 128..255, dK 256..383.
+constexpr int kKeysKV = 128;
+constexpr int kRowsKV = 64;
+constexpr int kThreadsKV = 256;
+constexpr int kSplitRowsKV = 32;                  // row tiles per CTA of the column pass
+constexpr uint32_t kvK = 0;                       // [128][128]: halves of 16 KiB
+constexpr uint32_t kvV = 32768;
+constexpr uint32_t kvQD = 65536;                  // [2 stages][Q, dO][64][128]: halves of 8 KiB
+constexpr uint32_t kvStage = 32768;               // one stage: Q then dO (16 KiB each)
+constexpr uint32_t kvPT = 131072;                 // P^T  [128][64] (one half)
+constexpr uint32_t kvDST = 147456;                // dS^T [128][64]
+constexpr uint32_t kvMeta = 163840;               // [2 stages][64] x {lse2, D, t, lo, hi}
+constexpr uint32_t kvBar = kvMeta + 2 * 5 * kRowsKV * 4;   // bar_s, bar_kv, abort, TMEM slot, range
+constexpr int kvSmemBytes = kvBar + 64;
+constexpr int kvTmemCols = 512;
+constexpr uint32_t kvColS = 0, kvColDP = 64, kvColDV = 128, kvColDK = 256;
+
+template <bool kColumn>
+__global__ void __launch_bounds__(kThreadsKV, 1)
+bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const uint32_t sb = sa(sm);
+  if ((sb & 1023u) != 0) {
+    if (threadIdx.x == 0) record_error(err, LTE_ERR_DEVICE, 413);
+    return;
+  }
+  const uint32_t bar_s = sb + kvBar, bar_kv = sb + kvBar + 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kvBar + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kvBar + 20);
+  int* range_sh = reinterpret_cast<int*>(sm + kvBar + 24);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int G = a.G, TOK = kRowsKV / G;
+  const int h = blockIdx.y, b = blockIdx.z, u = b * a.Hkv + h;
+  const long long crow = (long long)u * a.T;
+  const long long col_base = (long long)u * (a.sink + a.T);
+  const bool lowest = a.death != nullptr;
+  const int tile = kColumn ? (int)blockIdx.x / n_split : (int)blockIdx.x;
+  const int split = kColumn ? (int)blockIdx.x % n_split : 0;
+  const int k0 = tile * kKeysKV;
+  const int nk = kColumn ? min(kKeysKV, a.sink + __ldg(a.nret + u) - k0) : min(kKeysKV, a.T - k0);
+  if (nk <= 0) return;
+
+  // token range of the attending rows (as in the warp-MMA kernel)
+  if (tid == 0) {
+    int lo_t, hi_t;
+    if constexpr (!kColumn) {
+      lo_t = k0;
+      hi_t = min(a.T - 1, k0 + nk - 1 + a.window - 1);
+    } else {
+      lo_t = a.T;
+      hi_t = -1;
+      const int s_end = min(min(a.sink, k0 + nk), a.T);
+      if (k0 < s_end) {
+        lo_t = k0 + a.window;
+        hi_t = a.T - 1;
+      }
+      const int i0 = max(k0, a.sink) - a.sink, i1 = k0 + nk - a.sink;
+      if (i1 > i0 && a.cap > 0 && (a.cap_policy != LTE_CAP_FIRST || i0 < a.cap)) {
+        int l = a.window, r = a.T;
+        while (l < r) {
+          const int m = (l + r) >> 1;
+          if (__ldg(a.cnt + crow + m - a.window) > i0) r = m; else l = m + 1;
+        }
+        if (l < a.T) {
+          long long bound;
+          if (a.cap_policy == LTE_CAP_RECENT) bound = (long long)i1 + a.cap;
+          else if (a.cap_policy == LTE_CAP_FIRST) bound = 1ll << 40;
+          else {
+            int md = 0;
+            for (int i = i0; i < i1; ++i) md = max(md, __ldg(a.death + crow + i));
+            bound = md;
+          }
+          int l2 = l, r2 = a.T;
+          while (l2 < r2) {
+            const int m = (l2 + r2) >> 1;
+            if ((long long)__ldg(a.cnt + crow + m - a.window) >= bound) r2 = m; else l2 = m + 1;
+          }
+          if (l2 > l) {
+            lo_t = min(lo_t, l);
+            hi_t = max(hi_t, l2 - 1);
+          }
+        }
+      }
+    }
+    int rt0 = lo_t / TOK, rt1 = hi_t / TOK;
+    if (lo_t > hi_t) rt0 = 1, rt1 = 0;
+    if constexpr (kColumn) {
+      if (rt0 <= rt1) {
+        const int first = rt0 + split * kSplitRowsKV;
+        rt1 = min(rt1, first + kSplitRowsKV - 1);
+        rt0 = first;
+      }
+    }
+    range_sh[0] = rt0;
+    range_sh[1] = rt1;
+  }
+  __syncthreads();
+  const int rt0 = range_sh[0], n_rt = range_sh[1] - range_sh[0] + 1;
+  if (n_rt <= 0) return;                               // nothing attends (uniform)
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_kv, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     sa(tmem_slot)),
+                 "r"(kvTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // K, V of the tile (resident; rows past nk zero)
+  for (int i = tid; i < kKeysKV * 16; i += kThreadsKV) {
+    const int r = i >> 4, c = i & 15;
+    const bool ok = r < nk;
+    long long e = 0;
+    if (ok) {
+      if constexpr (kColumn) e = (col_base + k0 + r) * HD + c * 8;
+      else e = (((long long)b * a.T + k0 + r) * a.Hkv + h) * HD + c * 8;
+    }
+    cpa16(sb + kvK + sw(kKeysKV, r, c), (kColumn ? a.k_col : a.k) + e, ok);
+    cpa16(sb + kvV + sw(kKeysKV, r, c), (kColumn ? a.v_col : a.v) + e, ok);
+  }
+  // Q, dO and the row data of row tile `it` into stage it & 1
+  auto load_rows = [&](int it) {
+    const int st = it & 1, t0 = (rt0 + it) * TOK;
+    const uint32_t qs = sb + kvQD + st * kvStage;
+    for (int i = tid; i < kRowsKV * 16; i += kThreadsKV) {
+      const int r = i >> 4, c = i & 15;
+      const int tt = t0 + r / G, g = r % G;
+      const bool ok = tt < a.T;
+      const long long off = ok ? (((long long)b * a.T + tt) * a.Hq + h * G + g) * HD + c * 8 : 0;
+      cpa16(qs + sw(kRowsKV, r, c), a.q + off, ok);
+      cpa16(qs + 16384 + sw(kRowsKV, r, c), a.dO + off, ok);
+    }
+    if (tid < kRowsKV) {
+      const int r = tid, tt = t0 + r / G, g = r % G;
+      float* mf = reinterpret_cast<float*>(sm + kvMeta) + st * 5 * kRowsKV;
+      int* mi = reinterpret_cast<int*>(mf);
+      float l2 = 0.f, dd = 0.f;
+      if (tt < a.T) {
+        const long long li = ((long long)b * a.Hq + h * G + g) * a.T + tt;
+        l2 = a.lse[li] * 1.4426950408889634f;
+        dd = a.delta[li];
+      }
+      int lo, hi;
+      bwd::row_range(a, crow, tt, lo, hi);
+      if (lowest) lo = 0;
+      mf[r] = l2;
+      mf[kRowsKV + r] = dd;
+      mi[2 * kRowsKV + r] = tt;
+      mi[3 * kRowsKV + r] = lo;
+      mi[4 * kRowsKV + r] = hi;
+    }
+  };
+  load_rows(0);
+  cpa_commit();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int key_row = tid & 127, half = tid >> 7;       // this thread: key row, column half
+  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  // this key's identity for the masks
+  const int kpos = k0 + key_row;                         // position (window) or slot (column)
+  int kdeath = 0;
+  if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
+
+  const uint32_t id_s = idesc(kKeysKV, kRowsKV, false);
+  const uint32_t id_o = idesc(kKeysKV, HD, true);
+  bool ok = true;
+  int kv_issued = 0;
+  for (int it = 0; it < n_rt && ok; ++it) {
+    const int st = it & 1;
+    const uint32_t qs = sb + kvQD + st * kvStage, ds_ = qs + 16384;
+    // this stage's rows have landed
+    cpa_wait_all();
+    fence_proxy_async();
+    __syncthreads();
+    // S^T = K Q^T, dP^T = V dO^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dk = sdesc(sb + kvK, 16, 1024), dv = sdesc(sb + kvV, 16, 1024);
+      const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(ds_, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
+        const uint32_t ob = ((ks >> 2) * (kRowsKV * 128) + (ks & 3) * 32) >> 4;
+        mma_f16(tmem + kvColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16(tmem + kvColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_s);
+    }
+    // the previous tile's dV, dK products are done: its stage and P^T / dS^T are free
+    if (it > 0) {
+      ok = mbar_wait(bar_kv, (it - 1) & 1, abort_flag, err, 411);
+      if (!__syncthreads_and(ok)) { ok = false; break; }
+    }
+    if (it + 1 < n_rt) load_rows(it + 1);
+    cpa_commit();
+    ok = mbar_wait(bar_s, it & 1, abort_flag, err, 412);
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc_fence_after();
+    // P^T and dS^T: 32 row-columns of this key row
+    {
+      uint32_t rs[32], rp[32];
+      tmem_ld32(lane_addr + kvColS + half * 32, rs);
+      tmem_ld32(lane_addr + kvColDP + half * 32, rp);
+      tmem_wait_ld();
+      const float* mf = reinterpret_cast<const float*>(sm + kvMeta) + st * 5 * kRowsKV;
+      const int* mi = reinterpret_cast<const int*>(mf);
+      uint32_t pp[16], pd[16];
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float p2[2], d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int rho = half * 32 + c + e;
+          const int tt = mi[2 * kRowsKV + rho];
+          bool m = key_row < nk && tt < a.T;
+          if (m) {
+            if constexpr (!kColumn) {
+              m = kpos <= tt && kpos > tt - a.window;
+            } else if (kpos < a.sink) {
+              m = kpos <= tt - a.window;
+            } else {
+              const int i = kpos - a.sink, hi = mi[4 * kRowsKV + rho];
+              m = i >= mi[3 * kRowsKV + rho] && i < hi && (!lowest || kdeath > hi);
+            }
+          }
+          const float p = m ? exp2f(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -mf[rho])) : 0.f;
+          p2[e] = p;
+          d2[e] = p * (__uint_as_float(rp[c + e]) - mf[kRowsKV + rho]);
+        }
+        pp[c >> 1] = pk2(p2[0], p2[1]);
+        pd[c >> 1] = pk2(d2[0], d2[1]);
+      }
+      // chunks 4 half .. 4 half + 3 of the key row (swizzled K-major, one half)
+      uint8_t* prow = sm + kvPT + key_row * 128;
+      uint8_t* drow = sm + kvDST + key_row * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int ch = half * 4 + c;
+        const uint32_t o = (uint32_t)((ch ^ (key_row & 7)) << 4);
+        *reinterpret_cast<uint4*>(prow + o) = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+        *reinterpret_cast<uint4*>(drow + o) = make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    // dV += P^T dO, dK += dS^T Q
+    if (tid == 0) {
+      tc_fence_after();
+      const uint64_t dpt = sdesc(sb + kvPT, 16, 1024), ddst = sdesc(sb + kvDST, 16, 1024);
+      const uint64_t dob = sdesc(ds_, kRowsKV * 128, 1024), qb = sdesc(qs, kRowsKV * 128, 1024);
+#pragma unroll
+      for (int ks = 0; ks < kRowsKV / 16; ++ks) {
+        const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
+        mma_f16(tmem + kvColDV, dpt + ((ks * 32) >> 4), dob + ((ks * 2048) >> 4), id_o, acc);
+        mma_f16(tmem + kvColDK, ddst + ((ks * 32) >> 4), qb + ((ks * 2048) >> 4), id_o, acc);
+      }
+      mma_commit(bar_kv);
+    }
+    ++kv_issued;
+  }
+  if (ok && kv_issued > 0) {
+    ok = mbar_wait(bar_kv, (kv_issued - 1) & 1, abort_flag, err, 414);
+    ok = __syncthreads_and(ok);
+  }
+  cpa_wait_all();
+  if (ok) {
+    tc_fence_after();
+    // this thread: key row, dims [64 half, 64 half + 64) of dK and dV
+    int pos = kpos;
+    bool store = key_row < nk;
+    if constexpr (kColumn) {
+      if (store) {
+        pos = kpos < a.sink ? kpos : __ldg(a.idx + crow + kpos - a.sink);
+        store = pos < a.T;
+      }
+    }
+    const long long rowoff = (((long long)b * a.T + (store ? pos : 0)) * a.Hkv + h) * HD;
+#pragma unroll 1
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+      uint32_t rk[32], rv[32];
+      tmem_ld32(lane_addr + kvColDK + c0, rk);
+      tmem_ld32(lane_addr + kvColDV + c0, rv);
+      tmem_wait_ld();
+      if (store) {
+        float* dkr = a.dk + rowoff + c0;
+        float* dvr = a.dv + rowoff + c0;
+        if constexpr (kColumn) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            atomicAdd(dkr + e, __uint_as_float(rk[e]) * a.scale);
+            atomicAdd(dvr + e, __uint_as_float(rv[e]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            *reinterpret_cast<float4*>(dkr + e) =
+                make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
+                            __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale);
+            *reinterpret_cast<float4*>(dvr + e) =
+                make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
+                            __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3]));
+          }
+        }
+      }
+    }
+  } else if (tid == 0) {
+    mbar_drain(bar_s, 0);
+    mbar_drain(bar_s, 1);
+    if (kv_issued > 0) mbar_drain(bar_kv, (kv_issued - 1) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kvTmemCols)
+                 : "memory");
+}
+
 }  // namespace bwdtc
 
 bool attn_backward_dq_tc_supported(const lte_dims* d) {
   const int G = d->Hq / d->Hkv;
   return d->D == bwdtc::HD && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
+}
+
+cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
+  using namespace bwdtc;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kvSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kvSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int n_ktiles = (a.T + kKeysKV - 1) / kKeysKV;
+  bwd_dkdv_tc_kernel<false><<<dim3(n_ktiles, a.Hkv, B), kThreadsKV, kvSmemBytes, stream>>>(a, 1, err);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int TOK = kRowsKV / a.G;
+  const int n_ctiles = (a.sink + a.T + kKeysKV - 1) / kKeysKV;
+  const int n_split = ((a.T + TOK - 1) / TOK + kSplitRowsKV - 1) / kSplitRowsKV;
+  const long long gx = (long long)n_ctiles * n_split;
+  if (gx > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  bwd_dkdv_tc_kernel<true><<<dim3((unsigned)gx, a.Hkv, B), kThreadsKV, kvSmemBytes, stream>>>(
+      a, n_split, err);
+  return cudaGetLastError();
 }
 
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {

@@ -70,6 +70,7 @@ namespace bwd { struct Args; }
 // attn_backward_tc.cu: dQ on tcgen05 (head dim 128, G in {1, 2, 4, 8, 16})
 bool attn_backward_dq_tc_supported(const lte_dims* d);
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream);
+cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream);
 
 // decode.cu
 size_t decode_scratch_bytes(const lte_dims* d);
