@@ -61,6 +61,23 @@ __device__ __forceinline__ void cpa16(uint32_t dst, const void* src, bool valid)
 }
 __device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 __device__ __forceinline__ void cpa_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
+// bits [a, b) of a 64-bit set (empty when b <= a), clipped to [0, 64)
+__device__ __forceinline__ uint64_t span64(int a, int b) {
+  a = a > 0 ? a : 0;
+  b = b < 64 ? b : 64;
+  if (b <= a) return 0ull;
+  const uint64_t ones = (b - a == 64) ? ~0ull : ((1ull << (b - a)) - 1ull);
+  return ones << a;
+}
+// first index i in [0, n) with v[i] > x for a nondecreasing v (n if none)
+__device__ __forceinline__ int first_above(const int* v, int n, int x) {
+  int l = 0, r = n;
+  while (l < r) {
+    const int m = (l + r) >> 1;
+    if (v[m] > x) r = m; else l = m + 1;
+  }
+  return l;
+}
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -147,16 +164,21 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
 
   const uint32_t id_s = idesc(kRowsTc, kKeysTc, false);     // S, dP: K-major A and B
   const uint32_t id_q = idesc(kRowsTc, HD, true);           // dQ: K as an N-contiguous B
-  bool ok = true;
-  int issued_q = 0;                                         // dQ products committed
-  for (int j = 0; j < total && ok; ++j) {
-    int rg, it = j;
+  // tile j: range, first key, valid keys
+  auto tile_of = [&](int j, int& rg, int& key0, int& nk) {
+    int it = j;
     if (it < n0) rg = 0;
     else if (it < n0 + n1) { rg = 1; it -= n0; }
     else { rg = 2; it -= n0 + n1; }
-    const int key0 = start[rg] + it * kKeysTc;
-    const int nk = min(kKeysTc, count[rg] - it * kKeysTc);
-    // 1. K, V of the tile (the previous tile's products have completed)
+    key0 = start[rg] + it * kKeysTc;
+    nk = min(kKeysTc, count[rg] - it * kKeysTc);
+  };
+  // K (which = 0) or V (which = 1) rows of tile j into their buffer, zero past nk
+  auto load_kv = [&](int j, int which) {
+    int rg, key0, nk;
+    tile_of(j, rg, key0, nk);
+    const __nv_bfloat16* base = which == 0 ? (rg == 2 ? a.k : a.k_col) : (rg == 2 ? a.v : a.v_col);
+    const uint32_t dst = sb + (which == 0 ? kK : kV);
     for (int i = tid; i < kKeysTc * 16; i += kThreadsTc) {
       const int r = i >> 4, c = i & 15;
       const bool v_ok = r < nk;
@@ -166,12 +188,21 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
         e = rg == 2 ? (((long long)b * a.T + key) * a.Hkv + h) * HD + c * 8
                     : (col_base + key) * HD + c * 8;
       }
-      const __nv_bfloat16* kb = rg == 2 ? a.k : a.k_col;
-      const __nv_bfloat16* vb = rg == 2 ? a.v : a.v_col;
-      cpa16(sb + kK + sw(kKeysTc, r, c), kb + e, v_ok);
-      cpa16(sb + kV + sw(kKeysTc, r, c), vb + e, v_ok);
+      cpa16(dst + sw(kKeysTc, r, c), base + e, v_ok);
     }
-    cpa_commit();
+  };
+  bool ok = true;
+  int issued_q = 0;                                         // dQ products committed
+  if (total > 0) {
+    load_kv(0, 0);
+    load_kv(0, 1);
+  }
+  cpa_commit();
+  for (int j = 0; j < total && ok; ++j) {
+    int rg, key0, nk;
+    tile_of(j, rg, key0, nk);
+    // 1. K and V of tile j have landed (V was fetched while tile j - 1 was
+    //    being processed, K once tile j - 1's dQ product had completed)
     cpa_wait_all();
     fence_proxy_async();                                     // generic writes -> tensor core
     __syncthreads();
@@ -192,7 +223,26 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
     ok = mbar_wait(bar_s, j & 1, abort_flag, err, 401);
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc_fence_after();
-    // 3. P and dS of this row
+    if (j + 1 < total) load_kv(j + 1, 1);                  // V is free once dP is done
+    cpa_commit();
+    // 3. P and dS of this row.  The row's keys in the tile form at most two
+    //    intervals (sink slots, retained slots [lo, hi)) or one (window band)
+    uint64_t bits = 0ull;
+    if (tt < a.T) {
+      if (rg == 2) {
+        bits = span64(tt - a.window + 1 - key0, min(nk, tt - key0 + 1));
+      } else {
+        const int sink_end = min(a.sink, tt - a.window + 1);
+        uint64_t ret = span64(a.sink + lo_r - key0, min(nk, a.sink + hi_r - key0));
+        if (lowest && ret != 0ull) {                   // lifetimes: held at count hi_r
+#pragma unroll 4
+          for (int kk = 0; kk < kKeysTc; ++kk)
+            if (((ret >> kk) & 1ull) && __ldg(a.death + crow + key0 + kk - a.sink) <= hi_r)
+              ret &= ~(1ull << kk);
+        }
+        bits = span64(-key0, min(nk, sink_end - key0)) | ret;
+      }
+    }
     {
       uint32_t rs[32], rp[32];
       uint32_t pkd[32];
@@ -201,21 +251,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
         tmem_ld32(lane_addr + kColS + half * 32, rs);
         tmem_ld32(lane_addr + kColDP + half * 32, rp);
         tmem_wait_ld();
+        const uint32_t hb = (uint32_t)(bits >> (half * 32));
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float ds2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int kk = half * 32 + c + e, key = key0 + kk;
-            bool m = kk < nk && tt < a.T;
-            if (m) {
-              if (rg == 2) m = key <= tt && key > tt - a.window;
-              else if (key < a.sink) m = key <= tt - a.window;
-              else
-                m = (key - a.sink) >= lo_r && (key - a.sink) < hi_r &&
-                    (!lowest || __ldg(a.death + crow + key - a.sink) > hi_r);
-            }
-            const float p = m ? exp2f(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -lse2)) : 0.f;
+            const float p = ((hb >> (c + e)) & 1u)
+                                ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -lse2))
+                                : 0.f;
             ds2[e] = p * (__uint_as_float(rp[c + e]) - dl);
           }
           pkd[half * 16 + (c >> 1)] = pk2(ds2[0], ds2[1]);
@@ -246,7 +290,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
     ok = mbar_wait(bar_q, j & 1, abort_flag, err, 402);
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc_fence_after();
+    if (j + 1 < total) load_kv(j + 1, 0);                  // K is free once dQ is done
+    cpa_commit();
   }
+  cpa_wait_all();
   if (ok) {
     // dQ row: scale, fp32 out (every lane loads: tcgen05.ld is warp-collective)
     float* out = a.dq + (((long long)b * a.T + min(tt, a.T - 1)) * a.Hq + h * G + gq) * HD;
@@ -505,6 +552,30 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
       tmem_wait_ld();
       const float* mf = reinterpret_cast<const float*>(sm + kvMeta) + st * 5 * kRowsKV;
       const int* mi = reinterpret_cast<const int*>(mf);
+      // the rows of this tile that attend to this key: one interval of the
+      // (token-major) rows; tokens past T never attend
+      const int t0r = (rt0 + it) * TOK;
+      const int r_end = min(kRowsKV, (a.T - t0r) * G);
+      int r_a = 0, r_b = 0;
+      if (key_row < nk) {
+        if constexpr (!kColumn) {
+          r_a = (kpos - t0r) * G;                          // tokens [kpos, kpos + w)
+          r_b = (kpos + a.window - t0r) * G;
+        } else if (kpos < a.sink) {
+          r_a = (kpos + a.window - t0r) * G;               // tokens >= kpos + w
+          r_b = kRowsKV;
+        } else {
+          // lo(t) <= i < hi(t) (and, lowest, hi(t) < death): hi and lo grow with
+          // t over the rows of tokens below T (the searches stop there)
+          const int i = kpos - a.sink, n = max(r_end, 0);
+          r_a = first_above(mi + 4 * kRowsKV, n, i);               // hi > i
+          r_b = first_above(mi + 3 * kRowsKV, n, i);               // lo > i
+          if (lowest) r_b = min(r_b, first_above(mi + 4 * kRowsKV, n, kdeath - 1));
+        }
+        r_a = max(r_a, 0);
+        r_b = min(r_b, r_end);
+      }
+      const uint32_t hb = (uint32_t)(span64(r_a, r_b) >> (half * 32));
       uint32_t pp[16], pd[16];
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
@@ -512,19 +583,9 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int rho = half * 32 + c + e;
-          const int tt = mi[2 * kRowsKV + rho];
-          bool m = key_row < nk && tt < a.T;
-          if (m) {
-            if constexpr (!kColumn) {
-              m = kpos <= tt && kpos > tt - a.window;
-            } else if (kpos < a.sink) {
-              m = kpos <= tt - a.window;
-            } else {
-              const int i = kpos - a.sink, hi = mi[4 * kRowsKV + rho];
-              m = i >= mi[3 * kRowsKV + rho] && i < hi && (!lowest || kdeath > hi);
-            }
-          }
-          const float p = m ? exp2f(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -mf[rho])) : 0.f;
+          const float p = ((hb >> (c + e)) & 1u)
+                              ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -mf[rho]))
+                              : 0.f;
           p2[e] = p;
           d2[e] = p * (__uint_as_float(rp[c + e]) - mf[kRowsKV + rho]);
         }
@@ -587,10 +648,15 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         float* dkr = a.dk + rowoff + c0;
         float* dvr = a.dv + rowoff + c0;
         if constexpr (kColumn) {
+          // 16-byte vector atomics (rows are 512-byte aligned, c0 + e a multiple of 4)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            atomicAdd(dkr + e, __uint_as_float(rk[e]) * a.scale);
-            atomicAdd(dvr + e, __uint_as_float(rv[e]));
+          for (int e = 0; e < 32; e += 4) {
+            atomicAdd(reinterpret_cast<float4*>(dkr + e),
+                      make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
+                                  __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale));
+            atomicAdd(reinterpret_cast<float4*>(dvr + e),
+                      make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
+                                  __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3])));
           }
         } else {
 #pragma unroll
