@@ -334,12 +334,13 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
 // kColumn = false; slots of the column segment, kColumn = true, for this
 // CTA's share of the attending rows).  Keys are the MMA rows: per 64-row
 // tile of attending query rows,
-//   S^T = K Q^T, dP^T = V dO^T            (M128 N64 K128, SS)
+//   S^T = K Q^T, dP^T = V dO^T            (M128 N64 K128)
 //   P^T, dS^T = P^T (dP^T - D)             (thread pair per key row, 32 columns each)
 //   dV += P^T dO, dK += dS^T Q             (M128 N128 K64; dO, Q as N-contiguous B)
 // with Q and dO of the next row tile loading (cp.async, double-buffered)
-// while the current one is processed.  TMEM: S^T 0..63, dP^T 64..127,
-// dV 128..255, dK 256..383.
+// while the current one is processed.  K and V are copied into TMEM once, and
+// P^T, dS^T are written over S^T, dP^T, so that every product reads its A
+// operand from TMEM.
 constexpr int kKeysKV = 128;
 constexpr int kRowsKV = 64;
 constexpr int kThreadsKV = 256;
@@ -348,13 +349,23 @@ constexpr uint32_t kvK = 0;                       // [128][128]: halves of 16 Ki
 constexpr uint32_t kvV = 32768;
 constexpr uint32_t kvQD = 65536;                  // [2 stages][Q, dO][64][128]: halves of 8 KiB
 constexpr uint32_t kvStage = 32768;               // one stage: Q then dO (16 KiB each)
-constexpr uint32_t kvPT = 131072;                 // P^T  [128][64] (one half)
-constexpr uint32_t kvDST = 147456;                // dS^T [128][64]
-constexpr uint32_t kvMeta = 163840;               // [2 stages][64] x {lse2, D, t, lo, hi}
+constexpr uint32_t kvMeta = 131072;               // [2 stages][64] x {lse2, D, t, lo, hi}
 constexpr uint32_t kvBar = kvMeta + 2 * 5 * kRowsKV * 4;   // bar_s, bar_kv, abort, TMEM slot, range
 constexpr int kvSmemBytes = kvBar + 64;
 constexpr int kvTmemCols = 512;
-constexpr uint32_t kvColS = 0, kvColDP = 64, kvColDV = 128, kvColDK = 256;
+// S^T 0..63 (P^T over its first 32 as bf16 pairs), dP^T 64..127 (dS^T over its
+// first 32), dV 128..255, dK 256..383, K 384..447 and V 448..511 (bf16 pairs)
+constexpr uint32_t kvColS = 0, kvColDP = 64, kvColDV = 128, kvColDK = 256, kvColK = 384,
+                   kvColV = 448;
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 
 template <bool kColumn>
 __global__ void __launch_bounds__(kThreadsKV, 1)
@@ -464,8 +475,13 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     cpa16(sb + kvK + sw(kKeysKV, r, c), (kColumn ? a.k_col : a.k) + e, ok);
     cpa16(sb + kvV + sw(kKeysKV, r, c), (kColumn ? a.v_col : a.v) + e, ok);
   }
-  // Q, dO and the row data of row tile `it` into stage it & 1
-  auto load_rows = [&](int it) {
+  // Q, dO of row tile `it` into stage it & 1 (cp.async), and its row data:
+  // issue_rows starts the loads of lse, D and the retained count into
+  // registers (threads < 64, one row each); put_rows, called after other
+  // work, stores them, so that their latency is off the critical path
+  float m_l2 = 0.f, m_dd = 0.f;
+  int m_cnt = 0;
+  auto issue_rows = [&](int it) {
     const int st = it & 1, t0 = (rt0 + it) * TOK;
     const uint32_t qs = sb + kvQD + st * kvStage;
     for (int i = tid; i < kRowsKV * 16; i += kThreadsKV) {
@@ -478,25 +494,31 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     }
     if (tid < kRowsKV) {
       const int r = tid, tt = t0 + r / G, g = r % G;
-      float* mf = reinterpret_cast<float*>(sm + kvMeta) + st * 5 * kRowsKV;
-      int* mi = reinterpret_cast<int*>(mf);
-      float l2 = 0.f, dd = 0.f;
+      m_l2 = 0.f; m_dd = 0.f; m_cnt = 0;
       if (tt < a.T) {
         const long long li = ((long long)b * a.Hq + h * G + g) * a.T + tt;
-        l2 = a.lse[li] * 1.4426950408889634f;
-        dd = a.delta[li];
+        m_l2 = __ldg(a.lse + li);
+        m_dd = __ldg(a.delta + li);
+        if (tt >= a.window) m_cnt = __ldg(a.cnt + crow + tt - a.window);
       }
-      int lo, hi;
-      bwd::row_range(a, crow, tt, lo, hi);
-      if (lowest) lo = 0;
-      mf[r] = l2;
-      mf[kRowsKV + r] = dd;
+    }
+  };
+  auto put_rows = [&](int it) {
+    if (tid < kRowsKV) {
+      const int st = it & 1, r = tid, tt = (rt0 + it) * TOK + r / G;
+      float* mf = reinterpret_cast<float*>(sm + kvMeta) + st * 5 * kRowsKV;
+      int* mi = reinterpret_cast<int*>(mf);
+      const int hi = (tt < a.T && tt >= a.window) ? held_retained(m_cnt, a.cap, a.cap_policy) : 0;
+      const int lo = (!lowest && a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
+      mf[r] = m_l2 * 1.4426950408889634f;
+      mf[kRowsKV + r] = m_dd;
       mi[2 * kRowsKV + r] = tt;
       mi[3 * kRowsKV + r] = lo;
       mi[4 * kRowsKV + r] = hi;
     }
   };
-  load_rows(0);
+  issue_rows(0);
+  put_rows(0);
   cpa_commit();
   tc_fence_before();
   __syncthreads();
@@ -509,6 +531,25 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   int kdeath = 0;
   if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
 
+  // K and V rows into TMEM (A operands of S^T and dP^T): this thread's half of
+  // its key row, 64 dims = 32 columns of bf16 pairs
+  cpa_wait_all();
+  __syncthreads();
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const uint8_t* src = sm + (which == 0 ? kvK : kvV) + half * kKeysKV * 128 + key_row * 128;
+    uint32_t r[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v4 = *reinterpret_cast<const uint4*>(src + ((c ^ (key_row & 7)) << 4));
+      r[4 * c] = v4.x; r[4 * c + 1] = v4.y; r[4 * c + 2] = v4.z; r[4 * c + 3] = v4.w;
+    }
+    tmem_st32(lane_addr + (which == 0 ? kvColK : kvColV) + half * 32, r);
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+
   const uint32_t id_s = idesc(kKeysKV, kRowsKV, false);
   const uint32_t id_o = idesc(kKeysKV, HD, true);
   bool ok = true;
@@ -520,26 +561,26 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     cpa_wait_all();
     fence_proxy_async();
     __syncthreads();
-    // S^T = K Q^T, dP^T = V dO^T
+    // S^T = K Q^T, dP^T = V dO^T (K, V from TMEM).  They overwrite P^T, dS^T of
+    // the previous tile, whose products were issued earlier: the tensor pipe
+    // runs them in issue order
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t dk = sdesc(sb + kvK, 16, 1024), dv = sdesc(sb + kvV, 16, 1024);
       const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(ds_, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < HD / 16; ++ks) {
-        const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
         const uint32_t ob = ((ks >> 2) * (kRowsKV * 128) + (ks & 3) * 32) >> 4;
-        mma_f16(tmem + kvColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
-        mma_f16(tmem + kvColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16_ts(tmem + kvColS, tmem + kvColK + 8 * ks, dq + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16_ts(tmem + kvColDP, tmem + kvColV + 8 * ks, ddo + ob, id_s, ks > 0 ? 1u : 0u);
       }
       mma_commit(bar_s);
     }
-    // the previous tile's dV, dK products are done: its stage and P^T / dS^T are free
+    // the previous tile's dV, dK products are done: its Q / dO stage is free
     if (it > 0) {
       ok = mbar_wait(bar_kv, (it - 1) & 1, abort_flag, err, 411);
       if (!__syncthreads_and(ok)) { ok = false; break; }
     }
-    if (it + 1 < n_rt) load_rows(it + 1);
+    if (it + 1 < n_rt) issue_rows(it + 1);
     cpa_commit();
     ok = mbar_wait(bar_s, it & 1, abort_flag, err, 412);
     if (!__syncthreads_and(ok)) { ok = false; break; }
@@ -592,30 +633,27 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         pp[c >> 1] = pk2(p2[0], p2[1]);
         pd[c >> 1] = pk2(d2[0], d2[1]);
       }
-      // chunks 4 half .. 4 half + 3 of the key row (swizzled K-major, one half)
-      uint8_t* prow = sm + kvPT + key_row * 128;
-      uint8_t* drow = sm + kvDST + key_row * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int ch = half * 4 + c;
-        const uint32_t o = (uint32_t)((ch ^ (key_row & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + o) = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
-        *reinterpret_cast<uint4*>(drow + o) = make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
-      }
+      // P^T, dS^T over the first 32 columns of S^T, dP^T (16 per half), once
+      // both threads of the key row have read their columns
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      tmem_st16(lane_addr + kvColS + half * 16, pp);
+      tmem_st16(lane_addr + kvColDP + half * 16, pd);
+      tmem_wait_st();
     }
-    fence_proxy_async();
+    if (it + 1 < n_rt) put_rows(it + 1);               // the next stage's row data
     tc_fence_before();
     __syncthreads();
-    // dV += P^T dO, dK += dS^T Q
+    // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM)
     if (tid == 0) {
       tc_fence_after();
-      const uint64_t dpt = sdesc(sb + kvPT, 16, 1024), ddst = sdesc(sb + kvDST, 16, 1024);
       const uint64_t dob = sdesc(ds_, kRowsKV * 128, 1024), qb = sdesc(qs, kRowsKV * 128, 1024);
 #pragma unroll
       for (int ks = 0; ks < kRowsKV / 16; ++ks) {
         const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
-        mma_f16(tmem + kvColDV, dpt + ((ks * 32) >> 4), dob + ((ks * 2048) >> 4), id_o, acc);
-        mma_f16(tmem + kvColDK, ddst + ((ks * 32) >> 4), qb + ((ks * 2048) >> 4), id_o, acc);
+        mma_f16_ts(tmem + kvColDV, tmem + kvColS + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
+        mma_f16_ts(tmem + kvColDK, tmem + kvColDP + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
       }
       mma_commit(bar_kv);
     }
