@@ -31,7 +31,8 @@ def test_header_declares_expected_entry_points():
     names = _declared()
     for n in ("lte_score", "lte_evict_compact", "lte_sparse_attn_prefill", "lte_decode_step",
               "lte_cache_init_from_prefill", "lte_workspace_bytes", "lte_gla_prefill",
-              "lte_gla_decode_step", "lte_read_device_error", "lte_retained_lifetimes"):
+              "lte_gla_decode_step", "lte_read_device_error", "lte_retained_lifetimes",
+              "lte_sparse_attn_backward"):
         assert n in names
 
 
@@ -95,6 +96,20 @@ def test_host_validation_without_gpu(lib):
     assert f.lte_decode_step(C.byref(dl), C.byref(cnn), C.byref(cache), C.c_void_p(16),
                              C.c_void_p(16), C.c_void_p(16), C.c_void_p(16), None, 4,
                              C.c_void_p(16), 1 << 20, None) == 1
+    # backward: null pointers, fp32 (unsupported), lowest-score policy without
+    # lifetimes, workspace too small
+    bb = L.make_dims(1, 64, 4, 4, 128, 4, 16, 8, 0.5, 0.125, L.LTE_BF16)
+    p = [C.c_void_p(16)] * 16                                 # 15 tensors and the workspace
+    ws_need = f.lte_workspace_bytes(C.byref(bb), L.LTE_WS_BACKWARD)
+    assert ws_need >= 16 + 4 * 64 * 4
+    assert f.lte_sparse_attn_backward(C.byref(bb), *([None] * 16), 0, None) == 1
+    assert f.lte_sparse_attn_backward(C.byref(bb), *p, ws_need - 16, None) == 5
+    bf = L.make_dims(1, 64, 4, 4, 128, 4, 16, 8, 0.5, 0.125, L.LTE_F32)
+    assert f.lte_sparse_attn_backward(C.byref(bf), *p, 1 << 20, None) == 2
+    bl = L.make_dims(1, 64, 4, 4, 128, 4, 16, 8, 0.5, 0.125, L.LTE_BF16, L.LTE_CAP_LOWEST)
+    pl = list(p)
+    pl[4] = None                                              # death
+    assert f.lte_sparse_attn_backward(C.byref(bl), *pl, 1 << 20, None) == 1
     # wait probe: null or misaligned flag, limit out of range, missing workspace
     assert f.lte_wait_probe(None, 1, 1000000, C.c_void_p(16), None) == 1
     assert f.lte_wait_probe(C.c_void_p(18), 1, 1000000, C.c_void_p(16), None) == 1
