@@ -139,6 +139,56 @@ def cnn_scores(k, v, cnn: CNN, n_avail: int | None = None) -> np.ndarray:
     return r
 
 
+def cnn_backward(k, v, cnn: CNN, dr, n_scored: int):
+    """Gradients of L = sum_{j < n_scored} dr[j] r[j] through the scoring CNN
+    of one (batch element, KV head) unit, r as in ``cnn_scores`` with
+    n_avail = n (the whole sequence).  [LTE, Abstract: trained end to end;
+    the pages fix no dL/dr, so dr is an input.]
+
+    Chain rule through the two layers, written out:
+      dz2[j] = dr[j] r[j] (1 - r[j])                     (j < n_scored, else 0)
+      du[c, i]  = sum_kk w2[c, kk] dz2[i - kk + past2]   (u read at j + kk - past2)
+      dz1[c, i] = du[c, i] SiLU'(z1[c, i]),  SiLU'(z) = s(z) (1 + z (1 - s(z)))
+      dx[ch, m] = sum_{c, kk} w1[c, ch, kk] dz1[c, m - kk + past1]
+      dw1[c, ch, kk] = sum_i dz1[c, i] x[ch, i + kk - past1],  db1 = sum_i dz1
+      dw2[c, kk] = sum_j dz2[j] u[c, j + kk - past2],       db2 = sum_j dz2
+    with every shifted read 0 outside [0, n), as in the forward.
+    Returns dk, dv [n, D], dw1 [C1, 2D, K1], db1 [C1], dw2 [C1, K2], db2."""
+    k, v = _f64(k), _f64(v)
+    n, D = k.shape
+    x = np.concatenate([k, v], axis=1).T                      # [2D, n]
+    w1, w2 = _f64(cnn.w1), _f64(cnn.w2)
+    c1, _, k1 = w1.shape
+    k2 = w2.shape[1]
+    z1 = np.zeros((c1, n))
+    for kk in range(k1):
+        z1 += w1[:, :, kk] @ _shifted(x, kk - cnn.past1)
+    z1 += _f64(cnn.b1)[:, None]
+    u = silu(z1)
+    z2 = np.full(n, float(cnn.b2))
+    for kk in range(k2):
+        z2 += w2[:, kk] @ _shifted(u, kk - cnn.past2)
+    r = sigmoid(z2)
+    g = np.zeros(n)
+    g[:n_scored] = _f64(dr)[:n_scored]
+    dz2 = g * r * (1.0 - r)
+    du = np.zeros((c1, n))
+    dw2 = np.zeros((c1, k2))
+    for kk in range(k2):
+        us = _shifted(u, kk - cnn.past2)                      # us[:, j] = u[:, j + kk - past2]
+        dw2[:, kk] = us @ dz2
+        du += w2[:, kk][:, None] * _shifted(dz2[None, :], -(kk - cnn.past2))
+    sg = sigmoid(z1)
+    dz1 = du * sg * (1.0 + z1 * (1.0 - sg))
+    dx = np.zeros_like(x)
+    dw1 = np.zeros_like(w1)
+    for kk in range(k1):
+        xs = _shifted(x, kk - cnn.past1)
+        dw1[:, :, kk] = dz1 @ xs.T
+        dx += w1[:, :, kk].T @ _shifted(dz1, -(kk - cnn.past1))
+    return (dx[:D].T.copy(), dx[D:].T.copy(), dw1, dz1.sum(axis=1), dw2, float(dz2.sum()))
+
+
 # ---------------------------------------------------------------------------
 # (2) eviction decision and compaction  [LTE, Fig. 2 and Fig. 3]
 # ---------------------------------------------------------------------------
