@@ -422,6 +422,11 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
             "launches": (1 if fused else 2) * n_steps}
 
 
+# fp32 FMA throughput of one B200 from its unit counts and clock (no measured
+# fp32 peak is recorded): 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def rows_bench(args, rank, world, device, lte_decode_ms):
     """The hot-path rows outside the two headline steps, each launch timed alone
     with CUDA events after warm-up, on the hybrid workload (B=32, 4096-token
@@ -477,12 +482,24 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
                                                      bufs.nret, bufs.k_col, bufs.v_col, bufs.o,
                                                      bufs.lse, q, dq, dk, dv, ws_b, stream))
     assert L.lte_read_device_error(ws_b) == (0, 0)
-    del dq, dk, dv, ws_b
+    # backward through the scoring CNN (dL/dr = the scores themselves stand in
+    # for an incoming gradient: the work does not depend on its values)
+    dw1 = torch.empty_like(cnn[0]); db1 = torch.empty_like(cnn[1])
+    dw2 = torch.empty_like(cnn[2]); db2 = torch.empty_like(cnn[3])
+    ws_s = torch.zeros(L.lte_score_backward_workspace_bytes(dims, c) + 16, dtype=torch.uint8,
+                       device=device)
+    t_sbwd = timed(lambda: L.lte_score_backward(dims, c, k, v, n_scored, bufs.r, dk, dv, dw1, db1,
+                                                dw2, db2, ws_s, stream))
+    assert L.lte_read_device_error(ws_s) == (0, 0)
+    del dq, dk, dv, ws_b, ws_s, dw1, db1, dw2, db2
     mask = bufs.mask.cpu().numpy()
     nret = int(bufs.nret.sum())
     pairs = attended_pairs(mask, wl.sink, wl.window, wl.cap).sum()
     attn_flops = 4.0 * D * wl.G * float(pairs)
     bwd_flops = 2.5 * attn_flops           # S, dP, dQ, dK, dV over the attended pairs
+    # CNN backward: layer 1 recomputed, dx and dw1 (each 2 c_hid 2D k1 flops per
+    # position), layer 2 terms (small)
+    sbwd_flops = 3.0 * 2 * B * Hkv * T * wl.c_hid * 2 * D * wl.k1
     score_flops = 2.0 * B * Hkv * n_scored * (wl.c_hid * 2 * D * wl.k1 + wl.c_hid * wl.k2)
     score_bytes = B * T * Hkv * D * 2 * 2 + B * Hkv * n_scored * 5
     compact_bytes = (B * Hkv * T * (1 + 8) + B * Hkv * 4
@@ -524,6 +541,13 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
         "a3_attn_ms": t_attn, "a3_roofline": tensor(attn_flops, t_attn),
         "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
         "a3b_backward_ms": t_bwd, "a3b_roofline": tensor(bwd_flops, t_bwd),
+        "a1b_score_backward_ms": t_sbwd,
+        "a1b_roofline": {"bound": "alu", "achieved": sbwd_flops / (t_sbwd / 1e3) / 1e12,
+                         "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
+                         "frac": sbwd_flops / (t_sbwd / 1e3) / 1e12 / FP32_FMA_TFLOPS,
+                         "flops": sbwd_flops,
+                         "note": "lte_score_backward, fp32 SIMT; peak = 148 SMs x 128 fp32 lanes "
+                                 "x 2 flops x 1.965 GHz"},
         "a3b_note": "lte_sparse_attn_backward (delta, dQ, dK/dV window, dK/dV column: 4 "
                     "launches, tcgen05) on the same scored mask; FLOPs = 2.5 x the forward's",
         "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),
@@ -533,7 +557,7 @@ def rows_bench(args, rank, world, device, lte_decode_ms):
         "pair_decode": (None if lte_decode_ms is None else
                         {"value": DI.job_throughput(B, world, (t_gla_dec + lte_decode_ms) / 1e3),
                          "unit": "tokens/s", "us": 1e3 * (t_gla_dec + lte_decode_ms)}),
-        "launches": 2 + 5 * 3 + 5 + 50 + 4 * 7,
+        "launches": 2 + 5 * 3 + 5 + 50 + 4 * 7 + 4 * 7,
     }
 
 

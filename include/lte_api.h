@@ -122,6 +122,28 @@ lte_status lte_score(const lte_dims* d, const lte_cnn* cnn,
                      float* r, uint8_t* mask, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * lte_score_backward -- gradients through the scoring CNN, given dL/dr.
+ * [LTE paper, Abstract: trained end to end; Fig. 2 caption: the CNN.  The
+ * pages give no rule for dL/dr (the eviction decision is discrete), so it is
+ * an input.]  With r computed as in lte_score over the whole sequence (each
+ * layer's input 0 outside [0, T)) and L = sum_{j < n_scored} dr[j] r[j]:
+ *   dk, dv (fp32 [B,T,Hkv,D], contiguous): dL/dk, dL/dv ADDED to their
+ *          contents (so the attention backward's gradients can be summed in);
+ *   dw1 [Hkv,c_hid,2D,k1], db1 [Hkv,c_hid], dw2 [Hkv,c_hid,k2], db2 [Hkv]
+ *          (fp32): dL/dweights summed over the batch, OVERWRITTEN.
+ * k, v as in lte_score (kv_strides may be NULL); dr: fp32 [B,Hkv,T], entries
+ * j >= n_scored ignored; 0 <= n_scored <= T - F.  fp32 SIMT arithmetic; the
+ * weight gradients add fp32 partial sums with atomics (last bits may vary).
+ * Workspace: lte_score_backward_workspace_bytes(d, cnn) bytes (error word and
+ * 2 x B x Hkv x c_hid x T floats).
+ * ------------------------------------------------------------------------- */
+size_t lte_score_backward_workspace_bytes(const lte_dims* d, const lte_cnn* cnn);
+lte_status lte_score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
+                              const lte_strides* kv_strides, int32_t n_scored, const float* dr,
+                              float* dk, float* dv, float* dw1, float* db1, float* dw2, float* db2,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * lte_evict_compact -- eviction decision and compaction of retained tokens.
  * [LTE paper, Fig. 2 caption: a KV pair is kept or evicted when it moves out
  * of the window; Fig. 3 caption: capped out-of-window segment with sink and

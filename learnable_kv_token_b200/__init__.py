@@ -8,7 +8,8 @@
 """
 _LAZY = ("LteError", "lte_cache_init_from_prefill", "lte_clear_device_error", "lte_decode_step",
          "lte_decode_step_noalloc", "lte_evict_compact", "lte_gla_decode_step", "lte_gla_prefill",
-         "lte_read_device_error", "lte_retained_lifetimes", "lte_score", "lte_sparse_attn_backward",
+         "lte_read_device_error", "lte_retained_lifetimes", "lte_score", "lte_score_backward",
+         "lte_score_backward_workspace_bytes", "lte_sparse_attn_backward",
          "lte_sparse_attn_prefill", "lte_workspace_bytes",
          "version")
 

@@ -131,6 +131,29 @@ size_t lte_workspace_bytes(const lte_dims* d, int32_t which) {
   return 0;
 }
 
+size_t lte_score_backward_workspace_bytes(const lte_dims* d, const lte_cnn* cnn) {
+  if (check_dims(d) != LTE_OK || check_cnn(cnn) != LTE_OK) return 0;
+  return kErrBytes + lte::score_backward_scratch_bytes(d, cnn);
+}
+
+lte_status lte_score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
+                              const lte_strides* kv_strides, int32_t n_scored, const float* dr,
+                              float* dk, float* dv, float* dw1, float* db1, float* dw2, float* db2,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if ((st = check_cnn(cnn)) != LTE_OK) return st;
+  if (!k || !v || !dr || !dk || !dv || !dw1 || !db1 || !dw2 || !db2) return LTE_ERR_INVALID_ARG;
+  if (n_scored < 0 || n_scored > d->T - cnn_future(cnn)) return LTE_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace)) return LTE_ERR_WORKSPACE;
+  if (ws_bytes < lte_score_backward_workspace_bytes(d, cnn)) return LTE_ERR_WORKSPACE;
+  Strides4 s;
+  if ((st = get_strides(d, kv_strides, d->Hkv, &s)) != LTE_OK) return st;
+  return from_cuda(lte::score_backward(d, cnn, k, v, s, n_scored, dr, dk, dv, dw1, db1, dw2, db2,
+                                       static_cast<char*>(workspace) + kErrBytes,
+                                       as_stream(stream)));
+}
+
 lte_status lte_sparse_attn_backward(const lte_dims* d, const void* q, const void* k, const void* v,
                                     const int32_t* cnt, const int32_t* death, const int32_t* idx,
                                     const int32_t* nret, const void* k_col, const void* v_col,

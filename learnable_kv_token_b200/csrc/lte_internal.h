@@ -21,6 +21,13 @@ cudaError_t score_tcgen05(const lte_dims* d, const lte_cnn* cnn, const void* k, 
                           Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
                           cudaStream_t stream);
 
+// score_backward.cu
+size_t score_backward_scratch_bytes(const lte_dims* d, const lte_cnn* cnn);
+cudaError_t score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
+                           Strides4 s, int n_scored, const float* dr, float* dk, float* dv,
+                           float* dw1, float* db1, float* dw2, float* db2, void* scratch,
+                           cudaStream_t stream);
+
 // evict_compact.cu
 cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,
                           int32_t* idx, int32_t* nret, int32_t* cnt, const void* k,

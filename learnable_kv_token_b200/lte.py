@@ -67,6 +67,8 @@ _SIG = {
                                 C.POINTER(lte_strides), _P, _P, _P, _P, _P,
                                 C.POINTER(lte_strides), _P, _P, C.c_size_t, _P],
     "lte_sparse_attn_backward": [C.POINTER(lte_dims)] + [_P] * 16 + [C.c_size_t, _P],
+    "lte_score_backward": [C.POINTER(lte_dims), C.POINTER(lte_cnn), _P, _P, C.POINTER(lte_strides),
+                           _I] + [_P] * 8 + [C.c_size_t, _P],
     "lte_cache_init_from_prefill": [C.POINTER(lte_dims), C.POINTER(lte_cache), _P, _P,
                                     C.POINTER(lte_strides), _P, _P, _P, _P, _I, _I, _P],
     "lte_decode_step": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P, _P, _P,
@@ -85,10 +87,12 @@ for _name, _args in _SIG.items():
     _f.restype = C.c_int
 _lib.lte_workspace_bytes.argtypes = [C.POINTER(lte_dims), _I]
 _lib.lte_workspace_bytes.restype = C.c_size_t
+_lib.lte_score_backward_workspace_bytes.argtypes = [C.POINTER(lte_dims), C.POINTER(lte_cnn)]
+_lib.lte_score_backward_workspace_bytes.restype = C.c_size_t
 _lib.lte_version.argtypes = []
 _lib.lte_version.restype = C.c_char_p
 
-EXPORTED = tuple(_SIG) + ("lte_workspace_bytes", "lte_version")
+EXPORTED = tuple(_SIG) + ("lte_workspace_bytes", "lte_score_backward_workspace_bytes", "lte_version")
 
 
 def _call(name, *args):
@@ -170,6 +174,17 @@ def lte_sparse_attn_prefill(dims, q, k, v, cnt, k_col, v_col, o, lse, workspace,
           C.byref(_strides(q)), C.byref(_strides(k)), _ptr(cnt), _ptr(death), _ptr(k_col),
           _ptr(v_col), _ptr(o), C.byref(_strides(o)), _ptr(lse), _ptr(workspace),
           workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def lte_score_backward_workspace_bytes(dims, cnn) -> int:
+    return int(_lib.lte_score_backward_workspace_bytes(C.byref(dims), C.byref(cnn)))
+
+
+def lte_score_backward(dims, cnn, k, v, n_scored, dr, dk, dv, dw1, db1, dw2, db2, workspace,
+                       stream=None):
+    _call("lte_score_backward", C.byref(dims), C.byref(cnn), _ptr(k), _ptr(v), C.byref(_strides(k)),
+          n_scored, _ptr(dr), _ptr(dk), _ptr(dv), _ptr(dw1), _ptr(db1), _ptr(dw2), _ptr(db2),
+          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
 
 
 def lte_sparse_attn_backward(dims, q, k, v, cnt, death, idx, nret, k_col, v_col, o, lse, do, dq,
