@@ -84,16 +84,23 @@ __global__ void __launch_bounds__(kThreads) cnnb_z1_kernel(const Args a) {
       ws[t] = a.w1[(((long long)h * C + c) * 2 * a.D + ch0 + r / K1) * K1 + r % K1];
     }
     __syncthreads();
+    for (int ch = 0; ch < kChanChunk; ++ch) {
+      // the 8 + k1 - 1 inputs this thread's 8 positions read, once per channel
+      float xr[8 + kMaxK - 1];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int c = c0 + q * 32;
-      if (c >= C) continue;
-      for (int ch = 0; ch < kChanChunk; ++ch)
-        for (int kk = 0; kk < K1; ++kk) {
+      for (int t = 0; t < 8 + kMaxK - 1; ++t) xr[t] = t < 8 + K1 - 1 ? xs[ch][i0 + t] : 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int c = c0 + q * 32;
+        if (c >= C) continue;
+#pragma unroll
+        for (int kk = 0; kk < kMaxK; ++kk) {
+          if (kk >= K1) break;
           const float w = ws[(c * kChanChunk + ch) * K1 + kk];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(w, xs[ch][i0 + e + kk], acc[q][e]);
+          for (int e = 0; e < 8; ++e) acc[q][e] = fmaf(w, xr[e + kk], acc[q][e]);
         }
+      }
     }
   }
 #pragma unroll
@@ -194,13 +201,19 @@ __global__ void __launch_bounds__(kThreads) cnnb_dx_kernel(const Args a) {
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    for (int c = 0; c < C; ++c)
-      for (int kk = 0; kk < K1; ++kk) {
-        const float w = ws[(c * kChanChunk + chl) * K1 + kk];
-        // dz1 at m - kk + past1, m = p0 + i0 + e  ->  index i0 + e - kk + P1 + F1
+    for (int c = 0; c < C; ++c) {
+      // dz1 at m - kk + past1, m = p0 + i0 + e  ->  index i0 + e + (k1 - 1 - kk)
+      float zr[8 + kMaxK - 1];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, dzs[c][i0 + e - kk + P1 + F1], acc[e]);
+      for (int t = 0; t < 8 + kMaxK - 1; ++t) zr[t] = t < 8 + K1 - 1 ? dzs[c][i0 + t] : 0.f;
+#pragma unroll
+      for (int rk = 0; rk < kMaxK; ++rk) {             // rk = k1 - 1 - kk
+        if (rk >= K1) break;
+        const float w = ws[(c * kChanChunk + chl) * K1 + (K1 - 1 - rk)];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, zr[e + rk], acc[e]);
       }
+    }
     const int ch = ch0 + chl;
     const bool is_v = ch >= a.D;
     float* dst = is_v ? a.dv : a.dk;
