@@ -12,7 +12,8 @@
 //   D_t = <dO_t, o_t>,  dP = dO V^T,  dS = P * (dP - D_t),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO.
 //
-// Kernels, in stream order:
+// Kernels, in stream order (head dim 128 runs the tcgen05 dQ and dK/dV kernels
+// of attn_backward_tc.cu in place of the two warp-MMA ones):
 //   bwd_delta_kernel   D_t per (row, query head) from dO and o;
 //   bwd_dq_kernel      one CTA per 64 query rows (64/G tokens x the G heads of
 //                      a KV head), the forward's key ranges (sink slots and
