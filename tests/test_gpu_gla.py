@@ -2,7 +2,7 @@
 recurrent decode step) against the oracle's float64 token-by-token
 recurrence, on identical seeded inputs.
 
-Tolerance: bf16 operands with fp32 accumulation, judged as max-abs error
+Tolerance: bf16 operands with fp32 accumulation, measured as max-abs error
 relative to max |reference| (<= 1e-2 for bf16, <= 1e-5 for the fp32 decode
 arithmetic), on both the outputs and the final state."""
 import numpy as np
