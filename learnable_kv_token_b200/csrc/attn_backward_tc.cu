@@ -332,40 +332,31 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
 // ---------------------------------------------------------------- dK, dV
 // One CTA of 256 threads per 128-key tile (keys of k for the window part,
 // kColumn = false; slots of the column segment, kColumn = true, for this
-// CTA's share of the attending rows).  Keys are the MMA rows: per 64-row
+// CTA's share of the attending rows).  Keys are the MMA rows: per 128-row
 // tile of attending query rows,
-//   S^T = K Q^T, dP^T = V dO^T            (M128 N64 K128)
-//   P^T, dS^T = P^T (dP^T - D)             (thread pair per key row, 32 columns each)
-//   dV += P^T dO, dK += dS^T Q             (M128 N128 K64; dO, Q as N-contiguous B)
+//   S^T = K Q^T, dP^T = V dO^T            (M128 N128 K128)
+//   P^T, dS^T = P^T (dP^T - D)             (thread pair per key row, 64 rows each)
+//   dV += P^T dO, dK += dS^T Q             (M128 N128 K128; dO, Q as N-contiguous B)
 // with Q and dO of the next row tile loading (cp.async, double-buffered)
-// while the current one is processed.  K and V are copied into TMEM once, and
-// P^T, dS^T are written over S^T, dP^T, so that every product reads its A
-// operand from TMEM.
+// while the current one is processed.  P^T and dS^T are written over S^T and
+// dP^T in TMEM and read from there as A operands; the four accumulators fill
+// the 512 TMEM columns.
 constexpr int kKeysKV = 128;
-constexpr int kRowsKV = 64;
+constexpr int kRowsKV = 128;
 constexpr int kThreadsKV = 256;
-constexpr int kSplitRowsKV = 32;                  // row tiles per CTA of the column pass
+constexpr int kSplitRowsKV = 16;                  // row tiles per CTA of the column pass
 constexpr uint32_t kvK = 0;                       // [128][128]: halves of 16 KiB
 constexpr uint32_t kvV = 32768;
-constexpr uint32_t kvQD = 65536;                  // [2 stages][Q, dO][64][128]: halves of 8 KiB
-constexpr uint32_t kvStage = 32768;               // one stage: Q then dO (16 KiB each)
-constexpr uint32_t kvMeta = 131072;               // [2 stages][64] x {lse2, D, t, lo, hi}
+constexpr uint32_t kvQD = 65536;                  // [2 stages][Q, dO][128][128]: halves of 16 KiB
+constexpr uint32_t kvQBytes = kRowsKV * 128 * 2;  // one Q (or dO) tile
+constexpr uint32_t kvStage = 2 * kvQBytes;        // one stage: Q then dO
+constexpr uint32_t kvMeta = kvQD + 2 * kvStage;   // [2 stages][128] x {lse2, D, t, lo, hi}
 constexpr uint32_t kvBar = kvMeta + 2 * 5 * kRowsKV * 4;   // bar_s, bar_kv, abort, TMEM slot, range
 constexpr int kvSmemBytes = kvBar + 64;
 constexpr int kvTmemCols = 512;
-// S^T 0..63 (P^T over its first 32 as bf16 pairs), dP^T 64..127 (dS^T over its
-// first 32), dV 128..255, dK 256..383, K 384..447 and V 448..511 (bf16 pairs)
-constexpr uint32_t kvColS = 0, kvColDP = 64, kvColDV = 128, kvColDK = 256, kvColK = 384,
-                   kvColV = 448;
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
+// S^T 0..127 (P^T over its first 64 as bf16 pairs), dP^T 128..255 (dS^T over its
+// first 64), dV 256..383, dK 384..511
+constexpr uint32_t kvColS = 0, kvColDP = 128, kvColDV = 256, kvColDK = 384;
 
 template <bool kColumn>
 __global__ void __launch_bounds__(kThreadsKV, 1)
@@ -490,7 +481,7 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
       const bool ok = tt < a.T;
       const long long off = ok ? (((long long)b * a.T + tt) * a.Hq + h * G + g) * HD + c * 8 : 0;
       cpa16(qs + sw(kRowsKV, r, c), a.q + off, ok);
-      cpa16(qs + 16384 + sw(kRowsKV, r, c), a.dO + off, ok);
+      cpa16(qs + kvQBytes + sw(kRowsKV, r, c), a.dO + off, ok);
     }
     if (tid < kRowsKV) {
       const int r = tid, tt = t0 + r / G, g = r % G;
@@ -531,23 +522,7 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   int kdeath = 0;
   if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
 
-  // K and V rows into TMEM (A operands of S^T and dP^T): this thread's half of
-  // its key row, 64 dims = 32 columns of bf16 pairs
   cpa_wait_all();
-  __syncthreads();
-#pragma unroll
-  for (int which = 0; which < 2; ++which) {
-    const uint8_t* src = sm + (which == 0 ? kvK : kvV) + half * kKeysKV * 128 + key_row * 128;
-    uint32_t r[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 v4 = *reinterpret_cast<const uint4*>(src + ((c ^ (key_row & 7)) << 4));
-      r[4 * c] = v4.x; r[4 * c + 1] = v4.y; r[4 * c + 2] = v4.z; r[4 * c + 3] = v4.w;
-    }
-    tmem_st32(lane_addr + (which == 0 ? kvColK : kvColV) + half * 32, r);
-  }
-  tmem_wait_st();
-  tc_fence_before();
   __syncthreads();
 
   const uint32_t id_s = idesc(kKeysKV, kRowsKV, false);
@@ -556,7 +531,7 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   int kv_issued = 0;
   for (int it = 0; it < n_rt && ok; ++it) {
     const int st = it & 1;
-    const uint32_t qs = sb + kvQD + st * kvStage, ds_ = qs + 16384;
+    const uint32_t qs = sb + kvQD + st * kvStage, ds_ = qs + kvQBytes;
     // this stage's rows have landed
     cpa_wait_all();
     fence_proxy_async();
@@ -566,12 +541,14 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     // runs them in issue order
     if (tid == 0) {
       tc_fence_after();
+      const uint64_t dk = sdesc(sb + kvK, 16, 1024), dv = sdesc(sb + kvV, 16, 1024);
       const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(ds_, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < HD / 16; ++ks) {
+        const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
         const uint32_t ob = ((ks >> 2) * (kRowsKV * 128) + (ks & 3) * 32) >> 4;
-        mma_f16_ts(tmem + kvColS, tmem + kvColK + 8 * ks, dq + ob, id_s, ks > 0 ? 1u : 0u);
-        mma_f16_ts(tmem + kvColDP, tmem + kvColV + 8 * ks, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16(tmem + kvColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
+        mma_f16(tmem + kvColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
       }
       mma_commit(bar_s);
     }
@@ -587,9 +564,11 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     tc_fence_after();
     // P^T and dS^T: 32 row-columns of this key row
     {
-      uint32_t rs[32], rp[32];
-      tmem_ld32(lane_addr + kvColS + half * 32, rs);
-      tmem_ld32(lane_addr + kvColDP + half * 32, rp);
+      uint32_t rs[64], rp[64];
+      tmem_ld32(lane_addr + kvColS + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
+      tmem_ld32(lane_addr + kvColS + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
+      tmem_ld32(lane_addr + kvColDP + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&rp[0]));
+      tmem_ld32(lane_addr + kvColDP + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rp[32]));
       tmem_wait_ld();
       const float* mf = reinterpret_cast<const float*>(sm + kvMeta) + st * 5 * kRowsKV;
       const int* mi = reinterpret_cast<const int*>(mf);
@@ -616,15 +595,15 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         r_a = max(r_a, 0);
         r_b = min(r_b, r_end);
       }
-      const uint32_t hb = (uint32_t)(span64(r_a, r_b) >> (half * 32));
-      uint32_t pp[16], pd[16];
+      const uint64_t hb = span64(r_a - half * 64, r_b - half * 64);   // this thread's 64 rows
+      uint32_t pp[32], pd[32];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
+      for (int c = 0; c < 64; c += 2) {
         float p2[2], d2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int rho = half * 32 + c + e;
-          const float p = ((hb >> (c + e)) & 1u)
+          const int rho = half * 64 + c + e;
+          const float p = ((hb >> (c + e)) & 1ull)
                               ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -mf[rho]))
                               : 0.f;
           p2[e] = p;
@@ -633,13 +612,13 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         pp[c >> 1] = pk2(p2[0], p2[1]);
         pd[c >> 1] = pk2(d2[0], d2[1]);
       }
-      // P^T, dS^T over the first 32 columns of S^T, dP^T (16 per half), once
+      // P^T, dS^T over the first 64 columns of S^T, dP^T (32 per half), once
       // both threads of the key row have read their columns
       tc_fence_before();
       __syncthreads();
       tc_fence_after();
-      tmem_st16(lane_addr + kvColS + half * 16, pp);
-      tmem_st16(lane_addr + kvColDP + half * 16, pd);
+      tmem_st32(lane_addr + kvColS + half * 32, pp);
+      tmem_st32(lane_addr + kvColDP + half * 32, pd);
       tmem_wait_st();
     }
     if (it + 1 < n_rt) put_rows(it + 1);               // the next stage's row data
