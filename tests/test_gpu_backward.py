@@ -46,6 +46,9 @@ CASES = [
     (1, 300, 8, 8, 128, 0, 16, 3, "recent", 0.7),       # G = 1, no sink
     (1, 260, 16, 1, 64, 5, 50, 0, "recent", 0.6),       # G = 16, cap 0
     (1, 200, 4, 2, 128, 3, 400, 10, "recent", 0.5),     # window longer than the sequence
+    (1, 300, 16, 1, 128, 4, 48, 12, "recent", 0.5),     # G = 16 on the tcgen05 kernels
+    (1, 260, 16, 2, 128, 2, 40, 9, "first", 0.4),       # G = 8
+    (2, 190, 4, 2, 128, 1, 30, 6, "lowest", 16),        # G = 2, lowest-score policy
 ]
 POLICY = {"recent": (0, O.CAP_RECENT), "first": (1, O.CAP_FIRST), "lowest": (2, O.CAP_LOWEST)}
 
