@@ -36,7 +36,10 @@ Readings taken where the pages are silent (each is restated where used):
   cross-correlation convention, per-layer zero padding outside [0, n), a
   token is scorable only once its whole receptive field exists;
 * softmax scale is a parameter (1/sqrt(D) by default); KV head of query head
-  q is q // (Hq / Hkv).
+  q is q // (Hq / Hkv);
+* backward: the pages say the model is trained end to end but give no
+  gradient for the keep/evict decision, so the attention backward holds the
+  attended sets fixed, and the CNN backward takes dL/dr as an input.
 
 Parity pins: every function here is checked in ``tests/test_oracle_*.py``
 against something other than itself (library routines on special cases,
