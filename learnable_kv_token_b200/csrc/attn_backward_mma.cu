@@ -305,47 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const Args a, int
   // token range of the rows that attend to the tile's keys
   if (tid == 0) {
     int lo_t, hi_t;
-    if constexpr (!kColumn) {
-      lo_t = k0;
-      hi_t = min(a.T - 1, k0 + nk - 1 + a.window - 1);
-    } else {
-      lo_t = a.T;
-      hi_t = -1;
-      const int s_end = min(min(a.sink, k0 + nk), a.T);
-      if (k0 < s_end) {                                   // sink slots: rows t >= j + w
-        lo_t = k0 + a.window;
-        hi_t = a.T - 1;
-      }
-      const int i0 = max(k0, a.sink) - a.sink, i1 = k0 + nk - a.sink;
-      if (i1 > i0 && a.cap > 0 && (a.cap_policy != LTE_CAP_FIRST || i0 < a.cap)) {
-        // first row with cnt[t - w] > i0 (cnt is nondecreasing in t)
-        int l = a.window, r = a.T;
-        while (l < r) {
-          const int m = (l + r) >> 1;
-          if (__ldg(a.cnt + crow + m - a.window) > i0) r = m; else l = m + 1;
-        }
-        if (l < a.T) {
-          // last row whose retained count can still hold one of the slots
-          long long bound;                                // rows need cnt[t - w] < bound
-          if (a.cap_policy == LTE_CAP_RECENT) bound = (long long)i1 + a.cap;
-          else if (a.cap_policy == LTE_CAP_FIRST) bound = 1ll << 40;
-          else {
-            int md = 0;
-            for (int i = i0; i < i1; ++i) md = max(md, __ldg(a.death + crow + i));
-            bound = md;
-          }
-          int l2 = l, r2 = a.T;                           // first row with cnt >= bound
-          while (l2 < r2) {
-            const int m = (l2 + r2) >> 1;
-            if ((long long)__ldg(a.cnt + crow + m - a.window) >= bound) r2 = m; else l2 = m + 1;
-          }
-          if (l2 > l) {
-            lo_t = min(lo_t, l);
-            hi_t = max(hi_t, l2 - 1);
-          }
-        }
-      }
-    }
+    attending_tokens(a, crow, kColumn, k0, nk, lo_t, hi_t);
     range_sh[0] = lo_t;
     range_sh[1] = hi_t;
   }

@@ -383,48 +383,10 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   const int nk = kColumn ? min(kKeysKV, a.sink + __ldg(a.nret + u) - k0) : min(kKeysKV, a.T - k0);
   if (nk <= 0) return;
 
-  // token range of the attending rows (as in the warp-MMA kernel)
+  // token range of the attending rows
   if (tid == 0) {
     int lo_t, hi_t;
-    if constexpr (!kColumn) {
-      lo_t = k0;
-      hi_t = min(a.T - 1, k0 + nk - 1 + a.window - 1);
-    } else {
-      lo_t = a.T;
-      hi_t = -1;
-      const int s_end = min(min(a.sink, k0 + nk), a.T);
-      if (k0 < s_end) {
-        lo_t = k0 + a.window;
-        hi_t = a.T - 1;
-      }
-      const int i0 = max(k0, a.sink) - a.sink, i1 = k0 + nk - a.sink;
-      if (i1 > i0 && a.cap > 0 && (a.cap_policy != LTE_CAP_FIRST || i0 < a.cap)) {
-        int l = a.window, r = a.T;
-        while (l < r) {
-          const int m = (l + r) >> 1;
-          if (__ldg(a.cnt + crow + m - a.window) > i0) r = m; else l = m + 1;
-        }
-        if (l < a.T) {
-          long long bound;
-          if (a.cap_policy == LTE_CAP_RECENT) bound = (long long)i1 + a.cap;
-          else if (a.cap_policy == LTE_CAP_FIRST) bound = 1ll << 40;
-          else {
-            int md = 0;
-            for (int i = i0; i < i1; ++i) md = max(md, __ldg(a.death + crow + i));
-            bound = md;
-          }
-          int l2 = l, r2 = a.T;
-          while (l2 < r2) {
-            const int m = (l2 + r2) >> 1;
-            if ((long long)__ldg(a.cnt + crow + m - a.window) >= bound) r2 = m; else l2 = m + 1;
-          }
-          if (l2 > l) {
-            lo_t = min(lo_t, l);
-            hi_t = max(hi_t, l2 - 1);
-          }
-        }
-      }
-    }
+    bwd::attending_tokens(a, crow, kColumn, k0, nk, lo_t, hi_t);
     int rt0 = lo_t / TOK, rt1 = hi_t / TOK;
     if (lo_t > hi_t) rt0 = 1, rt1 = 0;
     if constexpr (kColumn) {
