@@ -1,12 +1,15 @@
 """Data-parallel plumbing of the LTE hot path.
 
 "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention and
-Contextualized Learnable Token Eviction", Sec. 3 (method): LTE scores, evicts
-and attends per (sequence, KV head); sequences never exchange data.  Data
-parallelism therefore shards whole sequences over ranks (one process per GPU)
-and the data path has no collective: the host needs only a barrier around the
-timed region and a max over ranks of each device-timed interval, which is how
-the job's time is defined (the slowest rank finishes the job).
+Contextualized Learnable Token Eviction", Fig. 2 and Fig. 3 captions: LTE
+scores, evicts and attends per (sequence, KV head); sequences never exchange
+data.  Data parallelism therefore shards whole sequences over ranks (one
+process per GPU) and the forward data path has no collective: the host needs
+only a barrier around the timed region and a max over ranks of each
+device-timed interval, which is how the job's time is defined (the slowest
+rank finishes the job).  Training adds one exchange: the gradients of the
+scoring CNN's weights, shared by all sequences, are summed over ranks
+(all_reduce_sum_).
 """
 from __future__ import annotations
 
@@ -65,3 +68,19 @@ def job_throughput(units_per_rank: float, world: int, seconds: float) -> float:
     """Whole-job throughput under weak scaling: every rank processes
     `units_per_rank` and the job takes the slowest rank's `seconds`."""
     return units_per_rank * world / seconds
+
+
+def all_reduce_sum_(tensors, world: int) -> None:
+    """Sum each tensor over all ranks, in place.  Used for the scoring CNN's
+    weight gradients, which lte_score_backward sums over a rank's own sequences
+    only.  The tensors (one dtype and device) are coalesced into one buffer,
+    so the exchange is a single all-reduce (NCCL on GPUs, gloo on the CPU)."""
+    if world <= 1 or not tensors:
+        return
+    flat = torch.cat([t.reshape(-1) for t in tensors])
+    tdist.all_reduce(flat, op=tdist.ReduceOp.SUM)
+    off = 0
+    for t in tensors:
+        n = t.numel()
+        t.copy_(flat[off:off + n].view_as(t))
+        off += n

@@ -59,6 +59,41 @@ def _rank_main(rank, port, q):
         q.put((rank, "error", repr(e), None, None))
 
 
+def _cnn_grads(rank):
+    """The oracle's CNN weight gradients of rank `rank`'s shard (two sequences,
+    one KV head, small sizes), as float64 tensors."""
+    import numpy as np
+    import torch
+    from learnable_kv_token_b200 import dist as DI
+    from oracle import lte_oracle as O
+    rng = np.random.default_rng(DI.shard_seed(5, rank))
+    n, D, c1 = 24, 3, 4
+    # the same weights on every rank (a shared model), each rank its own sequences
+    w = O.CNN(np.random.default_rng(5).standard_normal((c1, 2 * D, 5)) * 0.5,
+              np.zeros(c1), np.random.default_rng(6).standard_normal((c1, 3)) * 0.5, 0.1, 2, 1)
+    acc = None
+    for _ in range(2):
+        k, v, dr = rng.standard_normal((n, D)), rng.standard_normal((n, D)), rng.standard_normal(n)
+        _, _, dw1, db1, dw2, db2 = O.cnn_backward(k, v, w, dr, n - w.future)
+        g = [dw1, db1, dw2, np.array([db2])]
+        acc = g if acc is None else [a + b for a, b in zip(acc, g)]
+    return [torch.tensor(x) for x in acc]
+
+
+def _grad_rank_main(rank, port, q):
+    try:
+        _env(rank, port)
+        from learnable_kv_token_b200 import dist as DI
+        r, w, _ = DI.env_ranks()
+        DI.init(w, "gloo", timeout_s=30)
+        grads = _cnn_grads(r)
+        DI.all_reduce_sum_(grads, w)
+        DI.shutdown(w)
+        q.put((rank, "ok", [g.numpy() for g in grads]))
+    except Exception as e:  # reported to the parent
+        q.put((rank, "error", repr(e)))
+
+
 def _dying_rank_main(rank, port, q):
     try:
         _env(rank, port)
@@ -114,3 +149,17 @@ def test_dead_rank_fails_the_barrier_instead_of_hanging():
     status = {r: s for r, s, _ in res}
     assert status[1] == "exited"
     assert status[0] == "error", res
+
+
+def test_cnn_weight_gradients_sum_over_ranks():
+    """Data-parallel training: the CNN weight gradients each rank computes on
+    its own sequences are summed over ranks by one coalesced all-reduce; every
+    rank ends with the sum of both shards' gradients."""
+    import numpy as np
+    res = _run(_grad_rank_main, timeout=120)
+    for rank, status, payload in res:
+        assert status == "ok", (rank, payload)
+    want = [a.numpy() + b.numpy() for a, b in zip(_cnn_grads(0), _cnn_grads(1))]
+    for _, _, got in res:
+        for g, w_ in zip(got, want):
+            np.testing.assert_allclose(g, w_, rtol=0, atol=1e-12)
