@@ -32,7 +32,7 @@ def test_header_declares_expected_entry_points():
     for n in ("lte_score", "lte_evict_compact", "lte_sparse_attn_prefill", "lte_decode_step",
               "lte_cache_init_from_prefill", "lte_workspace_bytes", "lte_gla_prefill",
               "lte_gla_decode_step", "lte_read_device_error", "lte_retained_lifetimes",
-              "lte_sparse_attn_backward"):
+              "lte_sparse_attn_backward", "lte_score_backward"):
         assert n in names
 
 
@@ -110,6 +110,18 @@ def test_host_validation_without_gpu(lib):
     pl = list(p)
     pl[4] = None                                              # death
     assert f.lte_sparse_attn_backward(C.byref(bl), *pl, 1 << 20, None) == 1
+    # CNN backward: null pointers, n_scored past the receptive field, short workspace
+    cb = L.make_dims(2, 64, 4, 4, 64, 4, 16, 8, 0.5, 0.125, L.LTE_BF16)
+    cnn5 = L.lte_cnn(32, 5, 2, 3, 1, 16, 16, 16, 16)
+    need = f.lte_score_backward_workspace_bytes(C.byref(cb), C.byref(cnn5))
+    assert need >= 16 + 2 * 2 * 4 * 32 * 64 * 4
+    q16 = [C.c_void_p(16)] * 8                                # dr, dk, dv, dw1, db1, dw2, db2, ws
+    assert f.lte_score_backward(C.byref(cb), C.byref(cnn5), p16, p16, None, 61,
+                                *([None] * 8), need, None) == 1
+    assert f.lte_score_backward(C.byref(cb), C.byref(cnn5), p16, p16, None, 62, *q16, need,
+                                None) == 1                     # T - F = 61
+    assert f.lte_score_backward(C.byref(cb), C.byref(cnn5), p16, p16, None, 61, *q16, need - 16,
+                                None) == 5
     # wait probe: null or misaligned flag, limit out of range, missing workspace
     assert f.lte_wait_probe(None, 1, 1000000, C.c_void_p(16), None) == 1
     assert f.lte_wait_probe(C.c_void_p(18), 1, 1000000, C.c_void_p(16), None) == 1
