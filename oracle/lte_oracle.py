@@ -253,28 +253,34 @@ def top_by_score(candidates, r, cap: int) -> list[int]:
     return ranked[:cap]
 
 
-def attended_set(t: int, m, sink: int, window: int, cap: int,
+def retained_set(t: int, m, sink: int, window: int, cap: int,
                  policy: str = CAP_RECENT, r=None) -> list[int]:
-    """Key positions query t attends to, for one KV head.
-
-    S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t, with Ret_t drawn from the
-    tokens j in [s, t-w] with m_j = 1 (kept when they left the window):
+    """Ret_t: the retained tokens query t attends to, drawn from the tokens j
+    in [s, t-w] with m_j = 1 (kept when they left the window):
     policy "recent": the `cap` largest such j (the C most recent);
     policy "first":  the `cap` smallest such j (the segment fills, then later
     retained tokens are dropped);
     policy "lowest": the `cap` such j with the highest scores r_j (the
     lowest-scoring token is dropped when the segment overflows; `r` required).
+    Every member lies outside the window and the sink."""
+    candidates = [j for j in range(sink, t - window + 1) if m[j]]
+    if cap <= 0:
+        return []
+    if policy == CAP_RECENT:
+        return candidates[-cap:]
+    if policy == CAP_FIRST:
+        return candidates[:cap]
+    return sorted(top_by_score(candidates, r, cap))
+
+
+def attended_set(t: int, m, sink: int, window: int, cap: int,
+                 policy: str = CAP_RECENT, r=None) -> list[int]:
+    """Key positions query t attends to, for one KV head:
+    S_t = ([0, s) n [0, t])  u  (t-w, t]  u  Ret_t  (Ret_t: ``retained_set``).
     """
     keys = set(range(0, min(sink, t + 1)))
     keys |= set(range(max(0, t - window + 1), t + 1))
-    candidates = [j for j in range(sink, t - window + 1) if m[j]]
-    if cap > 0:
-        if policy == CAP_RECENT:
-            keys |= set(candidates[-cap:])
-        elif policy == CAP_FIRST:
-            keys |= set(candidates[:cap])
-        else:
-            keys |= set(top_by_score(candidates, r, cap))
+    keys |= set(retained_set(t, m, sink, window, cap, policy, r))
     return sorted(keys)
 
 
@@ -351,7 +357,7 @@ def prefill(q, k, v, masks, sink: int, window: int, cap: int, scale: float | Non
 # ---------------------------------------------------------------------------
 
 def prefill_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float, do,
-                          policy: str = CAP_RECENT, r=None):
+                          policy: str = CAP_RECENT, r=None, o_out=None):
     """Gradients of L = sum_t <do_t, o_t> for one (batch element, KV head)
     unit, o_t the prefill output over the fixed attended set S_t.
 
@@ -361,6 +367,9 @@ def prefill_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: f
       dq_t = scale dS K_S,  dk_S += scale dS^T q_t,  dv_S += P^T do_t.
     A position attended both from the window and, later, from the retained
     segment receives both contributions in the same dk / dv row.
+    o_out [T, G, D] (optional): the forward output as stored (e.g. rounded to
+    bf16), used for D_t in place of the exact o -- the usual contract of an
+    attention backward that is handed the forward's output; None = exact.
     Returns dq [T, G, D], dk [T, D], dv [T, D] (float64)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     T, G, D = q.shape
@@ -373,7 +382,7 @@ def prefill_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: f
         logits = scale * (q[t] @ Ks.T)                        # [G, n]
         P = np.exp(logits - logits.max(axis=1, keepdims=True))
         P /= P.sum(axis=1, keepdims=True)
-        o = P @ Vs
+        o = P @ Vs if o_out is None else _f64(o_out[t])
         dP = do[t] @ Vs.T
         Dt = (do[t] * o).sum(axis=1, keepdims=True)
         dS = P * (dP - Dt)
@@ -384,10 +393,11 @@ def prefill_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: f
 
 
 def prefill_backward(q, k, v, masks, sink: int, window: int, cap: int, do,
-                     scale: float | None = None, policy: str = CAP_RECENT, r=None):
+                     scale: float | None = None, policy: str = CAP_RECENT, r=None, o_out=None):
     """prefill_backward_unit over a batch: q, do [B,T,Hq,D], k, v [B,T,Hkv,D],
-    masks (and r) [B,Hkv,T].  GQA as in ``prefill``: dk, dv of KV head h sum
-    the contributions of its G query heads.  Returns dq, dk, dv (float64)."""
+    masks (and r) [B,Hkv,T], o_out [B,T,Hq,D] (optional, the stored forward
+    output for D_t).  GQA as in ``prefill``: dk, dv of KV head h sum the
+    contributions of its G query heads.  Returns dq, dk, dv (float64)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, T, Hq, D = q.shape
     Hkv = k.shape[2]
@@ -398,11 +408,89 @@ def prefill_backward(q, k, v, masks, sink: int, window: int, cap: int, do,
         for h in range(Hkv):
             gq, gk, gv = prefill_backward_unit(
                 q[b, :, h * G:(h + 1) * G], k[b, :, h], v[b, :, h], masks[b, h], sink, window,
-                cap, scale, do[b, :, h * G:(h + 1) * G], policy, None if r is None else r[b, h])
+                cap, scale, do[b, :, h * G:(h + 1) * G], policy, None if r is None else r[b, h],
+                None if o_out is None else o_out[b, :, h * G:(h + 1) * G])
             dq[b, :, h * G:(h + 1) * G] = gq
             dk[b, :, h] = gk
             dv[b, :, h] = gv
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# (3c) relaxed retention for training  [LTE, Abstract: the CNN and the model
+#      are trained end to end; Fig. 2 caption: r_{j,h} decides whether a KV
+#      pair is kept.  The pages give no rule for how the loss reaches r, so this
+#      reading is taken: the attended sets stay the hard ones (r >= tau, the
+#      cap policy), and every retained-segment key j of row t (j in Ret_t)
+#      enters the softmax with weight r_j, i.e. its logit gains log r_j.
+#      Window and sink keys are unweighted.  r then receives
+#        dL/dr_j = sum over rows t with j in Ret_t, heads g, of dS_{t,g,j} / r_j,
+#      dS the gradient at the logits.  With r = 1 everything reduces to the
+#      hard attention above.]
+# ---------------------------------------------------------------------------
+
+def _relaxed_row(t, q_t, k, v, m, sink, window, cap, scale, r, policy, r_rank):
+    """Logits and the pieces of row t under relaxed retention: keys S (list),
+    the bias vector (log r_j on Ret_t, else 0), logits [G, |S|]."""
+    S = attended_set(t, m, sink, window, cap, policy, r_rank)
+    ret = set(retained_set(t, m, sink, window, cap, policy, r_rank))
+    bias = np.array([math.log(r[j]) if j in ret else 0.0 for j in S])
+    logits = scale * (q_t @ k[S].T) + bias[None, :]
+    return S, ret, logits
+
+
+def prefill_relaxed_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float, r,
+                         rows=None, policy: str = CAP_RECENT):
+    """Relaxed-retention prefill of one (batch element, KV head) unit: as
+    ``prefill_unit``, with the logit of every key j in Ret_t raised by
+    log r_j (r [T] > 0 on retained tokens: the retention scores; they also
+    rank the tokens under policy "lowest").  Returns o [T, G, D], lse [T, G]."""
+    q, k, v, r = _f64(q), _f64(k), _f64(v), _f64(r)
+    T, G, D = q.shape
+    o = np.full((T, G, v.shape[1]), np.nan)
+    lse = np.full((T, G), np.nan)
+    for t in (range(T) if rows is None else rows):
+        S, _, logits = _relaxed_row(t, q[t], k, v, m, sink, window, cap, scale, r, policy, r)
+        mx = logits.max(axis=1, keepdims=True)
+        p = np.exp(logits - mx)
+        l = p.sum(axis=1, keepdims=True)
+        o[t] = (p @ v[S]) / l
+        lse[t] = (mx + np.log(l))[:, 0]
+    return o, lse
+
+
+def prefill_relaxed_backward_unit(q, k, v, m, sink: int, window: int, cap: int, scale: float,
+                                  do, r, policy: str = CAP_RECENT, o_out=None):
+    """Gradients of L = sum_t <do_t, o_t> under relaxed retention, for one unit.
+
+    Row by row, with P the softmax weights over S_t (logits with the log r
+    bias) and o_t = P V_S:  dP = do_t V_S^T,  D_t = <do_t, o_t>,
+    dS = P * (dP - D_t),  dq_t = scale dS K_S,  dk_S += scale dS^T q_t,
+    dv_S += P^T do_t,  and for j in Ret_t:  dr_j += sum_g dS[g, j] / r_j.
+    o_out: as in ``prefill_backward_unit`` (the stored output for D_t).
+    Returns dq [T, G, D], dk [T, D], dv [T, D], dr [T] (float64)."""
+    q, k, v, do, r = _f64(q), _f64(k), _f64(v), _f64(do), _f64(r)
+    T, G, D = q.shape
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dr = np.zeros(T)
+    for t in range(T):
+        S, ret, logits = _relaxed_row(t, q[t], k, v, m, sink, window, cap, scale, r, policy, r)
+        P = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        Vs, Ks = v[S], k[S]
+        o = P @ Vs if o_out is None else _f64(o_out[t])
+        dP = do[t] @ Vs.T
+        Dt = (do[t] * o).sum(axis=1, keepdims=True)
+        dS = P * (dP - Dt)
+        dq[t] = scale * (dS @ Ks)
+        dk[S] += scale * (dS.T @ q[t])
+        dv[S] += P.T @ do[t]
+        for c, j in enumerate(S):
+            if j in ret:
+                dr[j] += dS[:, c].sum() / r[j]
+    return dq, dk, dv, dr
 
 
 # ---------------------------------------------------------------------------

@@ -119,3 +119,34 @@ def test_batched_backward_splits_heads():
             np.testing.assert_array_equal(dq[b, :, 2 * h:2 * h + 2], gq)
             np.testing.assert_array_equal(dk[b, :, h], gk)
             np.testing.assert_array_equal(dv[b, :, h], gv)
+
+
+def test_stored_output_for_delta_vs_autograd():
+    """With o_out (the forward output as stored, here rounded to bf16) the
+    backward uses D_t = <do_t, o_out_t>.  That is the exact gradient of
+    L + sum_t c_t lse_t with the constants c_t = <do_t, o_t - o_out_t> (the
+    lse term adds c_t P to the logits' gradient): checked with torch autograd
+    for dq, dk and dv, and o_out = o reproduces the plain backward."""
+    T, G, D, s, w, C = 48, 2, 8, 2, 7, 5
+    q, k, v, do, r, m = _case(21, T, G, D, s, w, C, 0.5)
+    scale = 0.45
+    o, _, _ = O.prefill_unit(q, k, v, m, s, w, C, scale)
+    o_st = torch.tensor(o).to(torch.bfloat16).double().numpy()
+    dq, dk, dv = O.prefill_backward_unit(q, k, v, m, s, w, C, scale, do, o_out=o_st)
+    member = np.zeros((T, T), dtype=bool)
+    for t in range(T):
+        member[t, O.attended_set(t, m, s, w, C)] = True
+    c = torch.tensor((do * (o - o_st)).sum(-1))                  # [T, G], constants
+    qt, kt, vt = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    logits = (scale * torch.einsum("tgd,jd->tgj", qt, kt)).masked_fill(
+        ~torch.tensor(member)[:, None, :], float("-inf"))
+    ot = torch.einsum("tgj,jd->tgd", torch.softmax(logits, dim=-1), vt)
+    loss = (ot * torch.tensor(do)).sum() + (c * torch.logsumexp(logits, dim=-1)).sum()
+    loss.backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-11, rtol=0)
+    assert np.abs(dq - O.prefill_backward_unit(q, k, v, m, s, w, C, scale, do)[0]).max() > 0
+    same = O.prefill_backward_unit(q, k, v, m, s, w, C, scale, do, o_out=o)
+    for a, b in zip(same, O.prefill_backward_unit(q, k, v, m, s, w, C, scale, do)):
+        np.testing.assert_allclose(a, b, atol=1e-13, rtol=0)
