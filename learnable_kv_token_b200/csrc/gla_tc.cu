@@ -34,6 +34,15 @@
 // TMEM holds the fp32 state S (columns 0-127, lane = value channel) for the
 // whole sequence and one 64-row accumulator (columns 128-255: A of a chunk,
 // then its O; a 64-row accumulator keeps row r in lane 32 (r / 16) + r % 16).
+// Range.  The factors x_t and 1/x_t are products of up to 32 gates (or their
+// reciprocals), so the chunk form needs them inside the fp32/bf16 exponent
+// range.  The gate group checks every chunk: when some key channel's product
+// of 32 gates falls below 2^-100 (a gate near 0 -- or exactly 0 -- within a
+// chunk), that chunk instead runs the recurrence itself, token by token, in
+// fp32 on the state held in registers (the TMEM group: thread (row, half)
+// updates S[row, 64 half .. + 63] and the halves' partial o_t[row] are added
+// through shared memory).  So every gate in [0, 1] gives the recurrence's
+// result; only the speed of such chunks differs.
 // Every mbarrier wait is bounded; a CTA that gives up writes NaN into its
 // final state, so the failure is visible to the caller.
 #include <math.h>
@@ -118,6 +127,7 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   const uint32_t bar_g = s0 + kBar + 24;                 // gate work of set s done: + 8 s
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kBar + 40);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kBar + 44);
+  volatile int* exact = reinterpret_cast<volatile int*>(sm + kBar + 48);   // per set: 1 = recurrence
   float* st = state + (long long)bh * DV * DK;
   const int n_chunks = T / L;
 
@@ -176,6 +186,11 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // ---- decay factors x_t over the gates (in place): thread (j, half) walks
       // key channel j backwards through the first half (product of 1/a over
       // t < i <= m) or forwards through the second (product of a over m < i <= t)
+      // The chunk form is used only when, in every channel, the product of each
+      // half's 32 gates is >= 2^-100 (then every factor and its reciprocal stays
+      // within 2^+-100); otherwise the table keeps the raw gates for the
+      // recurrence (`exact`).  NaN or zero gates fail the test too.
+      bool in_range;
       {
         const int j = gt & (DK - 1), half = gt >> 7;
         float* Xj = reinterpret_cast<float*>(sset + kSetA) + half * 32 * DK + j;
@@ -192,6 +207,7 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             pr *= rcp_approx(ai);
             pa *= ai;
           }
+          in_range = pa >= 0x1p-100f && pr <= 0x1p100f;
           lam_m[j] = pa;                                   // e^{b_m}
         } else {
 #pragma unroll
@@ -199,11 +215,23 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             pa *= g[i];
             g[i] = pa;
           }
+          in_range = pa >= 0x1p-100f;
           lam_r[j] = pa;                                   // e^{b_last - b_m}
         }
+        in_range = group_and(kBarGate, kGroup, in_range);
+        if (in_range) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) Xj[i * DK] = g[i];
+          for (int i = 0; i < 32; ++i) Xj[i * DK] = g[i];
+        }
       }
+      if (!in_range) {                                     // chunk c runs the recurrence
+        if (gt == 0) {
+          exact[set] = 1;
+          mbar_arrive(bar_g + 8 * set);
+        }
+        continue;
+      }
+      if (gt == 0) exact[set] = 0;
       group_sync(kBarGate, kGroup);
       // ---- Q~ = q x and K~ = k / x in place, Khat = K~ e^{b_last - b_m} in its buffer
       {
@@ -275,6 +303,81 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       ok = mbar_wait_bounded(bar_g + 8 * set, (c >> 1) & 1, kWait, abort_flag, nullptr, 0);
       if (tid == 0) bulk_wait_read();                      // the previous output tile has left S_0'
       if (!(ok = group_and(kBarTmem, kGroup, ok))) break;
+
+      if (exact[set]) {
+        // ---- the recurrence, token by token, on raw q, k, v and gates: this
+        // thread holds S[row, 64 hc .. + 63] in registers; the half hc = 1 hands
+        // its part of o_t[row] to hc = 0 through the set's (unused) Khat buffer,
+        // which writes o_t as bf16 into the staging tile
+        const uint8_t* sset = sm + set * kSet;
+        float* xbuf = reinterpret_cast<float*>(sm + set * kSet + kSetKhat);   // [2][128]
+        float S[64];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + kColS + hc * 64 + 32 * h2, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) S[32 * h2 + e] = __uint_as_float(r[e]);
+        }
+#pragma unroll 1
+        for (int t = 0; t < L; ++t) {
+          const float* at = reinterpret_cast<const float*>(sset + kSetA) + t * DK + hc * 64;
+          const uint32_t vo = swz(L, t, row >> 3) + (row & 7) * 2;
+          const float vt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sset + kSetV + vo));
+          float o = 0.f;
+#pragma unroll
+          for (int e8 = 0; e8 < 8; ++e8) {                 // 16-byte chunk hc * 8 + e8 of row t
+            const uint32_t off = swz(L, t, hc * 8 + e8);
+            const uint4 kv = *reinterpret_cast<const uint4*>(sset + kSetK + off);
+            const uint4 qv = *reinterpret_cast<const uint4*>(sset + kSetQ + off);
+            const float4 a0 = *reinterpret_cast<const float4*>(at + 8 * e8);
+            const float4 a1 = *reinterpret_cast<const float4*>(at + 8 * e8 + 4);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv);
+            const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162*>(&kw[e]);
+              const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162*>(&qw[e]);
+              float& s0v = S[8 * e8 + 2 * e];
+              float& s1v = S[8 * e8 + 2 * e + 1];
+              s0v = fmaf(s0v, av[2 * e], vt * __low2float(k2));
+              s1v = fmaf(s1v, av[2 * e + 1], vt * __high2float(k2));
+              o = fmaf(s0v, __low2float(q2), o);
+              o = fmaf(s1v, __high2float(q2), o);
+            }
+          }
+          if (hc == 1) xbuf[(t & 1) * DV + row] = o;
+          group_sync(kBarTmem, kGroup);
+          if (hc == 0) {
+            o += xbuf[(t & 1) * DV + row];
+            *reinterpret_cast<__nv_bfloat16*>(sm + kSb + vo) = __float2bfloat16_rn(o);
+          }
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t r[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(S[32 * h2 + e]);
+          tmem_st32(lane_addr + kColS + hc * 64 + 32 * h2, r);
+        }
+        tmem_wait_st();
+        fence_proxy_async();                               // staged rows -> the TMA store
+        tc_fence_before();
+        if (!(ok = group_and(kBarTmem, kGroup, ok))) break;   // the set has been read
+        if (tid == 0) {
+          tc_fence_after();
+          if (c + 2 < n_chunks) {
+            load_chunk(c + 2);
+            ++n_issued;
+          }
+          tma_store_4d(&tm_o, s0 + kSb, 0, hd, c * L, b);
+          tma_store_4d(&tm_o, s0 + kSb + kHalf, 64, hd, c * L, b);
+          bulk_commit();
+        }
+        continue;
+      }
 
       // ---- A = Q~ K~^T (64 x 64, K = 128) into the 64-row accumulator
       if (tid == 0) {

@@ -48,6 +48,36 @@ def test_gla_prefill_vs_recurrence(L, B, T, H, gates, init):
     assert rel_err(f64(st), S_ref) <= 1e-2
 
 
+@pytest.mark.parametrize("kind", ["all-0.05", "sparse-zeros", "alternating"])
+def test_gla_prefill_any_gate(L, kind):
+    """Gates far below the chunk form's range: a = 0.05 everywhere (the product
+    of 32 gates is 2e-42), and typical gates with a = 0 or 1e-3 at a few
+    (token, channel) entries, and chunks that alternate between the two.  The
+    chunks whose gates leave the range run the recurrence token by token; the
+    result still matches the float64 recurrence at relative 1e-2, and the
+    final state too (the state then flows into the next chunk of either kind)."""
+    B, T, H = 2, 320, 2
+    g = LI.generator(4000 + len(kind))
+    q, k, v, a = LI.gla_inputs(B, T, H, 128, 128, g)
+    if kind == "all-0.05":
+        a = torch.full_like(a, 0.05)
+    elif kind == "sparse-zeros":
+        pick = torch.rand(a.shape, generator=g) < 2e-3
+        a = torch.where(pick, torch.where(torch.rand(a.shape, generator=g) < 0.5, 0.0, 1e-3), a)
+    else:                             # chunks 1, 3 of each sequence at 0.05, the others typical
+        for c in (1, 3):
+            a[:, 64 * c:64 * (c + 1)] = 0.05
+    S0 = torch.randn(B, H, 128, 128, generator=g) * 0.05
+    o = torch.empty_like(q, device="cuda")
+    st = S0.clone().cuda()
+    L.lte_gla_prefill(q.cuda(), k.cuda(), v.cuda(), a.cuda(), o, st)
+    torch.cuda.synchronize()
+    o_ref, S_ref = GO.gla(f64(q), f64(k), f64(v), f64(a), S0=f64(S0))
+    assert np.isfinite(f64(o)).all() and np.isfinite(f64(st)).all()
+    assert rel_err(f64(o), o_ref) <= 1e-2
+    assert rel_err(f64(st), S_ref) <= 1e-2
+
+
 @pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, 1e-2), (torch.float32, 1e-5)])
 def test_gla_decode_continues_recurrence(L, dtype, tol):
     B, T0, steps, H = 2, 128, 12, 2
