@@ -422,6 +422,86 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
             "launches": (1 if fused else 2) * n_steps}
 
 
+def sweep_bench(args, rank, world, device, only=None, reps=5):
+    """The long-context sparsity sweep: B=4, T=16384, Hq=16 / Hkv=4, D=128, bf16,
+    s=4, w=1024, C in {0, 1024, 4096, 16384} x retention rate in {0, 5, 25,
+    100} %, per-KV-head rates ~ U[0, 2 rate] clipped (rate 100 % retains every
+    token, so C = 16384 is full causal attention).  Per point: compaction once,
+    then `reps` attention launches timed with CUDA events after 2 warm-ups;
+    the attended FLOPs are counted exactly from the drawn mask.  Inputs are
+    larger than L2 (q 256 MiB).  `only` = (cap, rate) restricts it to one point
+    (profiler captures)."""
+    from learnable_kv_token_b200 import layer, lte as L
+    wl = LI.WORKLOADS["sweep"]
+    B = args.batch or wl.B
+    T, Hq, Hkv, D = wl.T, wl.Hq, wl.Hkv, wl.D
+    seed = DI.shard_seed(wl.seed, rank)
+    g = LI.generator(seed)
+    q, k, v = (x.to(device) for x in LI.qkv(B, T, Hq, Hkv, D, wl.dtype, g))
+    stream = torch.cuda.current_stream(device)
+    pk = peaks()
+    points = []
+    bufs = None
+    for cap in LI.SWEEP_CAPS:
+        for rate in LI.SWEEP_RATES:
+            if only is not None and (cap, rate) != only:
+                continue
+            mask = LI.rate_mask(B, Hkv, T, rate, LI.generator(seed + 1000 + cap + int(rate * 100)))
+            pairs = attended_pairs(mask.numpy(), wl.sink, wl.window, cap)
+            flops = 4.0 * D * wl.G * float(pairs.sum())
+            p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=cap, tau=wl.tau)
+            dims = p.dims(B, T, Hq, Hkv, D, torch.bfloat16)
+            if bufs is None:
+                bufs = layer.PrefillBuffers(B, T, Hq, Hkv, D, torch.bfloat16, wl.sink, dims, device,
+                                            want_r=False)
+            md = mask.to(device)
+
+            def compact():
+                L.lte_evict_compact(dims, None, md, T, bufs.idx, bufs.nret, bufs.cnt, k, v,
+                                    bufs.k_col, bufs.v_col, stream)
+
+            def attn():
+                L.lte_sparse_attn_prefill(dims, q, k, v, bufs.cnt, bufs.k_col, bufs.v_col, bufs.o,
+                                          bufs.lse, bufs.ws, stream)
+
+            def timed(fn, n):
+                for _ in range(2):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(n):
+                    fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                return DI.max_over_ranks(e0.elapsed_time(e1) / n, world, device)
+
+            t_c = timed(compact, 3)
+            compact()
+            t_a = timed(attn, reps)
+            assert L.lte_read_device_error(bufs.ws) == (0, 0)
+            tf = flops / (t_a / 1e3) / 1e12
+            rates = mask[..., wl.sink:].float().mean(dim=-1)
+            points.append({
+                "cap": cap, "rate": rate, "attended_flops": flops,
+                "frac_of_full_causal": float(pairs.sum()) / (B * Hkv * T * (T + 1) / 2),
+                "head_rate_min": float(rates.min()), "head_rate_max": float(rates.max()),
+                "attn_ms": t_a, "compact_ms": t_c,
+                "tokens_per_s": DI.job_throughput(B * T, world, (t_a + t_c) / 1e3),
+                "achieved_tflops": tf, "frac": tf / pk["bf16_tflops"],
+                "frac_of_sustained": tf / pk["bf16_tflops_sustained"]})
+            del md
+    del q, k, v, bufs
+    worst = min(points, key=lambda x: x["frac"]) if points else None
+    return {"workload": f"sweep B={B} T={T} Hq=16 Hkv=4 D=128 bf16 s=4 w=1024, C x per-head "
+                        "rate ~ U[0, 2 rate] clipped; step = evict_compact + sparse_attn_prefill; "
+                        "inputs larger than L2",
+            "peak": pk["bf16_tflops"], "peak_source": pk["source"], "points": points,
+            "worst": None if worst is None else {"cap": worst["cap"], "rate": worst["rate"],
+                                                 "frac": worst["frac"]},
+            "launches": len(points) * (5 + reps + 2 + 1)}
+
+
 # fp32 FMA throughput of one B200 from its unit counts and clock (no measured
 # fp32 peak is recorded): 148 SMs x 128 lanes x 2 flops x 1.965 GHz
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -572,6 +652,10 @@ def main():
                     help="skip the per-row measurements (scoring, compaction, GLA, hybrid pair)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="oracle CPU sample length (0 skips the cpu_baseline leg)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the long-context sparsity sweep (16 points)")
+    ap.add_argument("--sweep-only", default=None, metavar="CAP,RATE",
+                    help="run only this sweep point (e.g. 16384,0.05), for profiler captures")
     ap.add_argument("--batch", type=int, default=0,
                     help="batch override of the prefill and per-row workloads, for profiler "
                          "captures (default: the workloads')")
@@ -593,10 +677,18 @@ def main():
     from learnable_kv_token_b200 import build as _b  # noqa: F401  (library is prebuilt in-tree)
 
     pk = peaks()
+    if args.sweep_only:
+        c_, r_ = args.sweep_only.split(",")
+        sw = sweep_bench(args, rank, world, device, only=(int(c_), float(r_)))
+        if rank == 0:
+            print(json.dumps({"sweep": sw}), flush=True)
+        DI.shutdown(world)
+        return
     pf = prefill_bench(args, rank, world, device)
     dec = None if args.no_decode else decode_bench(args, rank, world, device)
     rows = None if args.no_rows else rows_bench(args, rank, world, device,
                                                 dec["ms_step"] if dec else None)
+    sweep = None if args.no_sweep else sweep_bench(args, rank, world, device)
 
     if rank == 0:
         value = DI.job_throughput(pf["B"] * pf["T"], world, pf["ms_step"] / 1e3)
@@ -650,6 +742,9 @@ def main():
             }
         if rows is not None:
             line["rows"] = {k: v for k, v in rows.items() if k != "launches"}
+        if sweep is not None:
+            line.setdefault("rows", {})["sweep"] = {k: v for k, v in sweep.items()
+                                                    if k != "launches"}
         if world == 1 and args.cpu_seconds > 0:
             tok, sec, desc = oracle_sample(LI.WORKLOADS["prefill"], args.cpu_seconds / 2,
                                            1.25 * args.cpu_seconds)

@@ -213,6 +213,25 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
                                    void* o, const lte_strides* o_strides, float* lse,
                                    void* workspace, size_t ws_bytes, void* stream);
 
+/* Which kernel family a call runs.  Every family is GPU code and gives the
+ * same results within the stated tolerances; they differ in speed. */
+typedef enum {
+  LTE_KERNEL_TCGEN05 = 1,   /* 5th-generation tensor cores (tcgen05, TMEM, TMA) */
+  LTE_KERNEL_MMA_SYNC = 2,  /* warp-level mma.sync tensor-core kernels (slower) */
+  LTE_KERNEL_SIMT = 3       /* fp32 CUDA-core kernels (fp32 inputs) */
+} lte_kernel_kind;
+
+/* lte_sparse_attn_prefill_kernel -- the kernel family lte_sparse_attn_prefill
+ * would run for these dims and strides (same meaning as in that call; NULL =
+ * contiguous), written to *kind.  The tcgen05 kernel serves bf16 with head
+ * dim 128, G in {1,2,4,8,16} and byte strides that are multiples of 16; other
+ * bf16 shapes run the mma.sync kernel, fp32 runs the SIMT kernel.  Host only:
+ * launches nothing.  Errors: LTE_ERR_INVALID_ARG / LTE_ERR_UNSUPPORTED as the
+ * call itself would return for these dims and strides. */
+lte_status lte_sparse_attn_prefill_kernel(const lte_dims* d, const lte_strides* q_strides,
+                                          const lte_strides* kv_strides,
+                                          const lte_strides* o_strides, int32_t* kind);
+
 /* ---------------------------------------------------------------------------
  * lte_sparse_attn_backward -- gradients of the prefill sparse attention with
  * the attended sets held fixed.  [LTE paper, Abstract: the hybrids are
@@ -242,6 +261,56 @@ lte_status lte_sparse_attn_backward(const lte_dims* d, const void* q, const void
                                     const void* o, const float* lse, const void* dO, float* dq,
                                     float* dk, float* dv, void* workspace, size_t ws_bytes,
                                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Relaxed retention for training.  [LTE paper, Abstract: the model, CNN
+ * included, is trained end to end; Fig. 2 caption: the score r_{j,h} decides
+ * whether a KV pair is kept.  The pages give no rule for how the loss reaches
+ * r; the reading taken here:]  the attended sets stay the hard ones (as in
+ * lte_sparse_attn_prefill: r >= tau, the cap policy), and every key j that
+ * row t attends through the retained segment (j in R_t's positions) enters
+ * the softmax with weight r_j -- its logit gains log r_j.  Sink and window
+ * keys are unweighted.  With r = 1 the calls equal the hard ones.
+ *
+ * lte_sparse_attn_prefill_relaxed -- o and lse as lte_sparse_attn_prefill
+ * with those weights:
+ *   o[t,q] = sum_{j in S_t} w_j exp(scale q_t.k_j) v_j / sum_{j in S_t} w_j exp(scale q_t.k_j),
+ *   lse[q,t] = log sum_{j in S_t} w_j exp(scale q_t.k_j),  w_j = r_j on retained
+ *   keys, 1 otherwise.
+ * lte_sparse_attn_backward_relaxed -- dq, dk, dv as lte_sparse_attn_backward
+ * for that forward, and
+ *   dr[j] = sum over rows t (and their G query heads) attending j through
+ *           the retained segment of dS_{t,j} / r_j   (dS: dL/dlogit),
+ *   dr: fp32 [B,Hkv,T], OVERWRITTEN (0 where no row attends j that way) --
+ *   the dL/dr that lte_score_backward takes.
+ * Arguments as in lte_sparse_attn_prefill / lte_sparse_attn_backward with
+ * contiguous [B,T,H,D] layouts, plus r: fp32 [B,Hkv,T] > 0 on retained tokens
+ * (clamped below at 1e-30; the scores behind the mask, e.g. from lte_score)
+ * and idx, nret from lte_evict_compact.  Supported: bf16, head dim 128,
+ * G in {1,2,4,8,16} (tcgen05 kernels), else LTE_ERR_UNSUPPORTED.
+ * Workspace: lte_workspace_bytes(d, LTE_WS_RELAXED) (error word, per-slot log
+ * weights, D_t); the calls share nothing through it.  dk, dv of retained and
+ * sink positions and dr add fp32 partial sums with atomics.
+ * ------------------------------------------------------------------------- */
+lte_status lte_sparse_attn_prefill_relaxed(const lte_dims* d, const void* q, const void* k,
+                                           const void* v, const int32_t* cnt, const int32_t* death,
+                                           const int32_t* idx, const int32_t* nret,
+                                           const void* k_col, const void* v_col, const float* r,
+                                           void* o, float* lse, void* workspace, size_t ws_bytes,
+                                           void* stream);
+lte_status lte_sparse_attn_backward_relaxed(const lte_dims* d, const void* q, const void* k,
+                                            const void* v, const int32_t* cnt,
+                                            const int32_t* death, const int32_t* idx,
+                                            const int32_t* nret, const void* k_col,
+                                            const void* v_col, const float* r, const void* o,
+                                            const float* lse, const void* dO, float* dq,
+                                            float* dk, float* dv, float* dr, void* workspace,
+                                            size_t ws_bytes, void* stream);
+
+/* lte_sparse_attn_backward_kernel -- the kernel family lte_sparse_attn_backward
+ * would run for these dims (*kind): LTE_KERNEL_TCGEN05 for head dim 128,
+ * LTE_KERNEL_MMA_SYNC for head dim 64.  Host only.  Errors as the call's. */
+lte_status lte_sparse_attn_backward_kernel(const lte_dims* d, int32_t* kind);
 
 /* ---------------------------------------------------------------------------
  * Decode cache.  [LTE paper, Fig. 3 caption: circular window segment plus an
@@ -341,13 +410,27 @@ lte_status lte_decode_step(const lte_dims* d, const lte_cnn* cnn, const lte_cach
  *    last call's contents; every call zeroes the error word and the counters
  *    it relies on.  Calls that overlap on the GPU (e.g. on two streams at
  *    once) race on the array: serialise them.
+ *  - Device errors: the error word lives in the array too; every call
+ *    clears it first, and lte_noalloc_read_device_error reads it.  Check it
+ *    after a call (before the next one clears it) as you would check a
+ *    workspace with lte_read_device_error.
+ *  - The cached address belongs to the device's primary context.  After
+ *    cudaDeviceReset (or anything else that destroys that context) the entry
+ *    point must not be called again in this process.
  *  - Results are the same as lte_decode_step's (same kernels). */
 #define LTE_NOALLOC_SCRATCH_BYTES (4u << 20)
 lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const lte_cache* cache,
                                    const void* q_t, const void* k_t, const void* v_t,
                                    void* o_t, float* lse_t, int32_t score_batch, void* stream);
 
-enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1, LTE_WS_BACKWARD = 2 };
+/* lte_noalloc_read_device_error -- the device error word of the last
+ * lte_decode_step_noalloc call on the current device: synchronises `stream`,
+ * then *code = 0 or LTE_ERR_TIMEOUT / LTE_ERR_DEVICE and *where = the id of
+ * the wait or check that failed (where may be NULL).  Allocates nothing.
+ * Errors: LTE_ERR_INVALID_ARG (code NULL), LTE_ERR_CUDA. */
+lte_status lte_noalloc_read_device_error(int32_t* code, int32_t* where, void* stream);
+
+enum { LTE_WS_PREFILL = 0, LTE_WS_DECODE = 1, LTE_WS_BACKWARD = 2, LTE_WS_RELAXED = 3 };
 
 /* Bytes of workspace a call needs (>= 16: the first 16 bytes hold the device
  * error word).  Returns 0 for invalid dims. */
@@ -383,14 +466,16 @@ lte_status lte_wait_probe(const int32_t* flag, int32_t expect, int64_t limit_ns,
  * "Background: Linear attention": the state is decayed, the value-key outer
  * product is written, the query reads; the decay here is diag(a_t).]
  *   S_t = S_{t-1} diag(a_t) + v_t k_t^T,  o_t = S_t q_t.
- * q, k: [B,T,H,dk]; v, o: [B,T,H,dv] (dtype); a: fp32 [B,T,H,dk] in (0,1];
+ * q, k: [B,T,H,dk]; v, o: [B,T,H,dv] (dtype); a: fp32 [B,T,H,dk] in [0,1];
  * state: fp32 [B,H,dv,dk], read as S_0 and overwritten with S_T.
  * Supported: dk = dv = 128; prefill bf16 with T % 64 == 0 (chunk-wise, 64
  * tokens per chunk, bf16 operands with fp32 accumulation and an fp32 state);
  * decode bf16 or fp32 (one step, fp32 arithmetic).  Other shapes return
- * LTE_ERR_UNSUPPORTED.  The chunk form multiplies q and k by exp(+-sum log a)
- * over at most 32 tokens, so it needs the product of any 32 consecutive
- * gates of a channel to stay above ~1e-30 (fp32/bf16 exponent range).
+ * LTE_ERR_UNSUPPORTED.  Any gate in [0, 1] is accepted.  The chunk form
+ * multiplies q and k by products of up to 32 gates (or their reciprocals);
+ * a chunk in which some channel's product of 32 gates falls below 2^-100 runs
+ * the recurrence token by token instead (fp32 state, same result within the
+ * stated tolerance, slower for that chunk).
  * ------------------------------------------------------------------------- */
 lte_status lte_gla_prefill(int32_t B, int32_t T, int32_t H, int32_t dk, int32_t dv,
                            int32_t dtype, const void* q, const void* k, const void* v,

@@ -18,6 +18,11 @@ struct Args {
   const float* lse;       // natural log, [B, Hq, T]
   float* delta;           // [B, Hq, T]
   float *dq, *dk, *dv;    // fp32, [B,T,Hq,D] and [B,T,Hkv,D]
+  // relaxed retention (NULL otherwise): logit offset per column-segment slot
+  // ([B*Hkv][sink + T] + 64 padding, log r_j / scale on retained slots, 0 on
+  // sinks) and dL/dr ([B,Hkv,T], accumulated with atomics onto zeros)
+  const float* bias;
+  float* dr;
 };
 
 // retained count a row sees and the start of its retained range

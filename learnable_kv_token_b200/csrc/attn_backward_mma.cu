@@ -596,8 +596,14 @@ cudaError_t attn_backward(const BackwardArgs& g, cudaStream_t stream) {
   a.cnt = g.cnt; a.death = g.death; a.idx = g.idx; a.nret = g.nret; a.lse = g.lse;
   a.delta = reinterpret_cast<float*>(g.scratch);
   a.dq = g.dq; a.dk = g.dk; a.dv = g.dv;
+  a.bias = g.bias; a.dr = g.dr;
   // tcgen05 kernels where they apply (head dim 128), else the warp-MMA kernels
   const bool dq_tc = attn_backward_dq_tc_supported(d);
+  if ((g.bias != nullptr || g.dr != nullptr) && !dq_tc) return cudaErrorNotSupported;
+  if (g.dr != nullptr) {
+    const cudaError_t e = cudaMemsetAsync(g.dr, 0, (size_t)d->B * d->Hkv * d->T * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
   if (d->D == 128) return bwd::launch<128>(a, d->B, dq_tc, g.err, stream);
   return bwd::launch<64>(a, d->B, dq_tc, g.err, stream);
 }

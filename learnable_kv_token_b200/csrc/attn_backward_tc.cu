@@ -243,6 +243,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
         bits = span64(-key0, min(nk, sink_end - key0)) | ret;
       }
     }
+    // relaxed retention: the column slots' logit offsets (0 on sinks)
+    const float* brow = (a.bias != nullptr && rg != 2) ? a.bias + col_base + key0 : nullptr;
     {
       uint32_t rs[32], rp[32];
       uint32_t pkd[32];
@@ -252,6 +254,12 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
         tmem_ld32(lane_addr + kColDP + half * 32, rp);
         tmem_wait_ld();
         const uint32_t hb = (uint32_t)(bits >> (half * 32));
+        if (brow != nullptr) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if ((hb >> c) & 1u)
+              rs[c] = __float_as_uint(__uint_as_float(rs[c]) + __ldg(brow + half * 32 + c));
+        }
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float ds2[2];
@@ -483,6 +491,10 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   const int kpos = k0 + key_row;                         // position (window) or slot (column)
   int kdeath = 0;
   if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
+  // relaxed retention: log2 of this slot's weight r (0 for sinks and window keys),
+  // and the partial sum of dS over the rows this thread sees, for dL/dr
+  float bk2 = 0.f, dr_acc = 0.f;
+  if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
 
   cpa_wait_all();
   __syncthreads();
@@ -566,10 +578,11 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         for (int e = 0; e < 2; ++e) {
           const int rho = half * 64 + c + e;
           const float p = ((hb >> (c + e)) & 1ull)
-                              ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -mf[rho]))
+                              ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, bk2 - mf[rho]))
                               : 0.f;
           p2[e] = p;
           d2[e] = p * (__uint_as_float(rp[c + e]) - mf[kRowsKV + rho]);
+          if constexpr (kColumn) dr_acc += d2[e];
         }
         pp[c >> 1] = pk2(p2[0], p2[1]);
         pd[c >> 1] = pk2(d2[0], d2[1]);
@@ -615,6 +628,10 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
         pos = kpos < a.sink ? kpos : __ldg(a.idx + crow + kpos - a.sink);
         store = pos < a.T;
       }
+    }
+    // dL/dr of a retained slot: sum of dS over its rows, over r (both halves add)
+    if constexpr (kColumn) {
+      if (store && a.dr != nullptr && kpos >= a.sink) atomicAdd(a.dr + crow + pos, dr_acc * ex2(-bk2));
     }
     const long long rowoff = (((long long)b * a.T + (store ? pos : 0)) * a.Hkv + h) * HD;
 #pragma unroll 1

@@ -24,28 +24,34 @@
 // columns are reused for P_x as bf16 pairs), O_x (128) and Q_x (64, bf16
 // pairs).  Both products read their A operand from TMEM (Q for S = Q K^T, P
 // for O += P V), so shared memory only feeds K and V to the tensor core.
-// Warp roles (384 threads, three warpgroups):
+// Warp roles (512 threads, four warpgroups):
 //   warp 0     TMA producer: the item's Q rows into one shared buffer (freed as
-//              soon as both softmax groups copied them into TMEM), the K and V
-//              tiles of a key tile into one stage of a 4-stage ring (one
-//              barrier per stage for both; a stage frees once the tile's PV
-//              MMAs have run -- each MMA-warp wait is costly, so the issuer
-//              waits once per key tile);
-//   warp 1     TMEM owner and MMA issuer (one elected lane), per K/V tile j:
-//              PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  The tensor pipe runs in
-//              issue order, so when S_x(j) has completed, PV_x(j-1) has too:
-//              P_x may then be overwritten and O_x rescaled without a wait;
-//   warps 2-3  output stores of tiles A and B (TMA stores of the staged rows)
+//              soon as they are copied into TMEM), the K and V tiles of a key
+//              tile into one stage of a 4-stage ring (one barrier per stage for
+//              both; a stage frees once the tile's PV MMAs have run -- each
+//              MMA-warp wait is costly, so the issuer waits once per key tile);
+//   warp 1     TMEM owner and MMA issuer (one elected lane).  It walks one
+//              stream of key tiles across items, per tile g: PV_A(g-1), S_A(g),
+//              PV_B(g-1), S_B(g), also across an item boundary, so the next
+//              item's first products follow the last ones without a gap.  The
+//              tensor pipe runs in issue order, so when S_x(g) has completed,
+//              PV_x(g-1) has too: P_x may then be overwritten and O_x rescaled
+//              without a wait;
+//   warps 2-3  output stores of tiles A and B (TMA stores of the staged rows);
 //   warps 4-7  softmax of tile A, warps 8-11 of tile B: one thread per row
 //              reads its S row from TMEM, applies the attended-set predicate
 //              (a 64-bit set of at most two column intervals), exp2 via
 //              ex2.approx with the scale folded into a packed FMA, writes P
 //              into TMEM, and rescales its O row only when the running max
 //              grew by more than 2^8 (exact: O and l share the reference max).
-//              During an item's last tile it copies the next item's Q rows
-//              into TMEM, so that item's first S overlaps this item's
-//              epilogue: O / l -> bf16 rows staged in the (now copied) Q
-//              buffer, written out by TMA stores, and lse.
+//              At an item's end it hands l and the max to the epilogue through
+//              shared memory and goes straight on to the next item;
+//   warps 12-15 item boundaries, off the softmax path: once S_x of an item's
+//              last tile has run, copy the next item's Q rows of tile x from
+//              the shared buffer into TMEM; once PV_x of the last tile has run,
+//              O / l -> bf16 rows staged in the (now copied) Q buffer for the
+//              store warps, and lse.  The next item's first PV_x waits only for
+//              O_x to have been read.
 // Every mbarrier wait is bounded (1 s of global time): on expiry the CTA
 // records LTE_ERR_TIMEOUT in the workspace error word, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and exits.
@@ -63,12 +69,14 @@ namespace tc {
 constexpr int BM = 128;             // rows per Q tile (TMEM lanes)
 constexpr int BN = 64;              // keys per K/V tile
 constexpr int HD = 128;             // head dim
-constexpr int kThreads = 384;
-// register split (setmaxnreg): the launch gives 168 per thread (3 warps per
-// sub-partition); warpgroup 0 (TMA, MMA, two store warps) drops to 64 and the
-// two softmax warpgroups rise to 216: 4 * 64 + 8 * 216 <= 12 * 168
-constexpr int kRegsLaunch = 168, kRegsIssue = 64, kRegsSoftmax = 216;
-static_assert(4 * kRegsIssue + 8 * kRegsSoftmax <= 12 * kRegsLaunch, "register split fits the launch");
+constexpr int kThreads = 512;
+// register split (setmaxnreg): the launch gives 128 per thread (4 warps per
+// sub-partition); warpgroup 0 (TMA, MMA, two store warps) drops to 72, the
+// epilogue warpgroup to 88, and the two softmax warpgroups rise to 176:
+// 4 * 72 + 4 * 88 + 8 * 176 <= 16 * 128
+constexpr int kRegsLaunch = 128, kRegsIssue = 72, kRegsEpi = 88, kRegsSoftmax = 176;
+static_assert(4 * kRegsIssue + 4 * kRegsEpi + 8 * kRegsSoftmax <= 16 * kRegsLaunch,
+              "register split fits the launch");
 constexpr uint32_t kQTile = BM * HD * 2;          // 32 KiB
 constexpr uint32_t kQHalf = BM * 128;             // 64-column half of a Q tile: 16 KiB
 constexpr uint32_t kQBuf = 2 * kQTile;            // tiles A and B of one item: 64 KiB
@@ -78,18 +86,25 @@ constexpr int kStages = 4;                        // K/V ring depth
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKV = kQBuf;                // stage s: K at +s*32K, V at +16K
 constexpr uint32_t kOffBar = kOffKV + kStages * 2 * kKV;   // 192 KiB
-constexpr uint32_t kSmemBytes = kOffBar + 512;
+constexpr uint32_t kOffLM = kOffBar + 512;        // l and max per row: [item parity][tile][row][2]
+constexpr uint32_t kSmemBytes = kOffLM + 2 * 2 * 128 * 8;
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int x) { return x == 0 ? 0u : 64u; }     // S (and P)
 __host__ __device__ constexpr uint32_t col_o(int x) { return x == 0 ? 128u : 256u; }  // O
 __host__ __device__ constexpr uint32_t col_q(int x) { return x == 0 ? 384u : 448u; }  // Q
 
-// mbarriers: KF / KE = a K/V ring stage is full / free again (one per stage)
+// mbarriers: KF / KE = a K/V ring stage is full / free again (one per stage);
+// LM = a tile's l and max are in shared memory (one per tile and item parity,
+// so that a one-tile item cannot complete a phase before the last one was seen)
 enum {
   B_QF = 0, B_QFREE = 1, B_QC = 2, B_KF = 4, B_KE = B_KF + kStages, B_SF = B_KE + kStages,
   B_PF = B_SF + 2, B_PVD = B_PF + 2, B_OE = B_PVD + 2, B_FIN = B_OE + 2, B_OST = B_FIN + 1,
-  B_STG = B_OST + 2, kNumBars = B_STG + 2
+  B_STG = B_OST + 2, B_LM = B_STG + 2, B_SL = B_LM + 4, kNumBars = B_SL + 2
 };
+// SL_x: S_x of an item's last tile has completed (one phase per item).  The
+// epilogue warpgroup waits on it before it overwrites Q_x; it cannot wait on
+// SF_x for that tile, since it may arrive more than one phase early, where a
+// parity wait would pass on an older phase.
 static_assert(8 * kNumBars + 8 <= 512, "barriers, abort flag and TMEM slot fit the tail");
 
 struct Params {
@@ -98,6 +113,8 @@ struct Params {
   float scale_log2;
   const int32_t* cnt;
   const int32_t* death;   // lifetimes of retained slots (drop-the-lowest-score cap), else NULL
+  const float* bias;      // relaxed retention: logit offset per column-segment slot, else NULL
+  int col_stride;         // slots per unit of the column segment (sink + T)
   float* lse;
   DevError* err;
 };
@@ -109,34 +126,6 @@ __device__ __forceinline__ uint64_t span_bits(int a, int b) {
   if (b <= a) return 0ull;
   const uint64_t ones = (b - a == 64) ? ~0ull : ((1ull << (b - a)) - 1ull);
   return ones << a;
-}
-
-// 2^x for a pair of fp32 values on the FMA pipe (the special-function unit
-// evaluates the others).  Range reduction 2^x = 2^n * 2^f with n = round(x),
-// obtained by adding 1.5 * 2^23 (which leaves n in the low mantissa bits),
-// and f = x - n in [-1/2, 1/2]; 2^f by a degree-3 polynomial, a weighted
-// least-squares fit of the relative error on Chebyshev nodes with p(0) = 1
-// (relative error <= 1.2e-4, mean 4e-5: below the bf16 rounding of P, 2^-9,
-// and, on the fraction of terms it serves, far below the lse tolerance;
-// gen_exp2_poly.py prints the fit); 2^n enters as an integer add to the
-// exponent field.  Inputs are clamped to >= -127: a masked key (x = -inf)
-// then has n = -127, f = 0, p(0) = 1 and an exponent field of 0, so its P is
-// exactly +0 as from the special-function unit (the key rows of a ragged tile
-// past the valid ones may hold any finite value, and 0 * V must stay 0);
-// x in (-127, -126.5) gives a denormal below 2^-126 instead of 2^x.
-constexpr int kPolyEvery = 0;       // > 0: every kPolyEvery-th pair of S columns takes the polynomial
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -127.f);
-  x.y = fmaxf(x.y, -127.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 q = __ffma2_rn(make_float2(5.459282547e-02f, 5.459282547e-02f), f,
-                        make_float2(2.422178388e-01f, 2.422178388e-01f));
-  q = __ffma2_rn(q, f, make_float2(6.933686137e-01f, 6.933686137e-01f));
-  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // max of three fp32 values in one instruction
@@ -218,7 +207,10 @@ __device__ __forceinline__ uint64_t alive_bits(const int32_t* __restrict__ death
   return bits;
 }
 
-template <bool kLowest>
+// kRelax: relaxed retention for training -- every retained-segment key's
+// logit gains log r (p.bias, in units of the raw score q.k), so its softmax
+// weight is scaled by r; window and sink keys are unchanged.
+template <bool kLowest, bool kRelax>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -257,6 +249,9 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mbar_init(bar(B_OST + 1), 1);
     mbar_init(bar(B_STG), 128);
     mbar_init(bar(B_STG + 1), 128);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(B_LM + i), 128);
+    mbar_init(bar(B_SL), 1);
+    mbar_init(bar(B_SL + 1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -336,12 +331,11 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       // 14 bits) is then advanced by plain adds (shared addresses < 256 KiB)
       const uint64_t dk0 = sdesc(sbase + kOffKV, 16, 1024);
       const uint64_t dv0 = sdesc(sbase + kOffKV + kKV, kKVHalf, 1024);
-      int g0 = 0, it = 0;
       bool ok = true;
-      // PV_x of global tile g (tile j of item it): O_x += P_x V
-      auto issue_pv = [&](int x, int g, int j) -> bool {
+      // PV_x of global tile g (tile j of item `item`): O_x += P_x V
+      auto issue_pv = [&](int x, int g, int j, int item) -> bool {
         if (!wwait(bar(B_PF + x), g & 1, abort_flag, p.err, 215)) return false;
-        if (j == 0 && it >= 1 && !wwait(bar(B_OE + x), (it - 1) & 1, abort_flag, p.err, 216))
+        if (j == 0 && item >= 1 && !wwait(bar(B_OE + x), (item - 1) & 1, abort_flag, p.err, 216))
           return false;                               // the epilogue has read the previous O_x
         tc_fence_after();
         const uint64_t dv = dv0 + (((g % kStages) * 2 * kKV) >> 4);
@@ -354,16 +348,23 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         __syncwarp();
         return true;
       };
+      // key tile g is tile j of item `it`; tile g - 1 is tile jp of item itp
+      int g = 0, it = 0, prev_total = 0;
       ItemCounts cn = load_counts(p, blockIdx.x);
       for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
         const Item m = make_item(p, i, cn);
         cn = load_counts(p, i + gridDim.x);
-        for (int j = 0; j < m.total && ok; ++j) {
-          const int g = g0 + j, st = g % kStages;
+        for (int j = 0; j < m.total && ok; ++j, ++g) {
+          const int st = g % kStages;
           if (!(ok = wwait(bar(B_KF + st), (g / kStages) & 1, abort_flag, p.err, 212))) break;
           const uint64_t dk = dk0 + ((st * 2 * kKV) >> 4);
+          const int jp = j >= 1 ? j - 1 : prev_total - 1, itp = j >= 1 ? it : it - 1;
           for (int x = 0; x < 2 && ok; ++x) {
-            if (j >= 1 && !(ok = issue_pv(x, g - 1, j - 1))) break;
+            if (g >= 1) {
+              if (!(ok = issue_pv(x, g - 1, jp, itp))) break;
+              if (j == 0 && elect_one()) mma_commit(bar(B_PVD + x));   // item itp's O_x is final
+              __syncwarp();
+            }
             if (j == 0 && !(ok = wwait(bar(B_QC + x), it & 1, abort_flag, p.err, 213))) break;
             tc_fence_after();
             const uint32_t tq = tmem + col_q(x), ds = tmem + col_s(x);
@@ -374,25 +375,25 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mma_f16_ts(ds, tq + 8 * kk, dk + offk, idS, kk > 0);
               }
               mma_commit(bar(B_SF + x));
+              if (j == m.total - 1) mma_commit(bar(B_SL + x));   // Q_x of this item is done with
             }
             __syncwarp();
           }
           if (!ok) break;
-          if (j >= 1 && elect_one()) mma_commit(bar(B_KE + (g - 1) % kStages));   // tile g-1 done
+          if (g >= 1 && elect_one()) mma_commit(bar(B_KE + (g - 1) % kStages));   // tile g-1 done
           __syncwarp();
         }
-        if (!ok) break;
-        // the item's last tile: PV_A, PV_B, then the epilogue signal
-        const int gl = g0 + m.total - 1;
+        prev_total = m.total;
+      }
+      // the last tile: PV_A, PV_B, then the epilogue signals
+      if (ok && g >= 1) {
         for (int x = 0; x < 2 && ok; ++x) {
-          if (!(ok = issue_pv(x, gl, m.total - 1))) break;
+          if (!(ok = issue_pv(x, g - 1, prev_total - 1, it - 1))) break;
           if (elect_one()) mma_commit(bar(B_PVD + x));
           __syncwarp();
         }
-        if (!ok) break;
-        if (elect_one()) mma_commit(bar(B_KE + gl % kStages));
+        if (ok && elect_one()) mma_commit(bar(B_KE + (g - 1) % kStages));
         __syncwarp();
-        g0 += m.total;
       }
       if (elect_one()) mma_commit(bar(B_FIN));       // all MMAs of this warp are complete
       __syncwarp();
@@ -424,39 +425,17 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (elect_one()) bulk_wait_all();            // output stores complete before exit
       __syncwarp();
     }
-  } else {
+  } else if (warp < 12) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    // ============================================================ softmax + epilogue
+    // ============================================================ softmax
     const int x = (warp - 4) >> 2;                 // Q tile of this warpgroup
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t colS = col_s(x), colO = col_o(x), colQ = col_q(x);
-    const int g_in_row = row % p.G;
-    // copy this thread's Q row of the shared buffer (128B-swizzled halves) into TMEM
-    auto copy_q = [&](int it) -> bool {
-      bool ok = mbar_wait(bar(B_QF), it & 1, abort_flag, p.err, 224);
-      if (!(ok = __all_sync(0xffffffffu, ok))) return false;
-      const uint8_t* qrow = smem + kOffQ + x * kQTile + row * 128;
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + hf * kQHalf + ((c ^ (row & 7)) << 4));
-          r[4 * c] = v4.x; r[4 * c + 1] = v4.y; r[4 * c + 2] = v4.z; r[4 * c + 3] = v4.w;
-        }
-        tmem_st32(lane_addr + colQ + hf * 32, r);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_QC + x));
-      mbar_arrive(bar(B_QFREE));
-      return true;
-    };
+    const uint32_t colS = col_s(x), colO = col_o(x);
+    float2* lm = reinterpret_cast<float2*>(smem + kOffLM) + x * 128 + row;   // + 256 * parity
     int g0 = 0, it = 0;
     bool ok = true;
-    if (blockIdx.x < p.n_items) ok = copy_q(0);
     // this row's retained count n_t = cnt[t - w] of item i (0 if none), loaded one item ahead
     auto row_count = [&](int i) -> int {
       if (i >= p.n_items) return 0;
@@ -474,7 +453,6 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int hi_t = hi_next;
       cn = load_counts(p, i + gridDim.x);
       hi_next = row_count(i + gridDim.x);
-      const bool has_next = i + (int)gridDim.x < p.n_items;
       const int tt = m.t0 + x * p.TOK + row / p.G;
       const bool row_ok = tt < p.T;
       const int lo_t = hi_t - p.cap > 0 && !kLowest ? hi_t - p.cap : 0;
@@ -514,6 +492,15 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
+        if constexpr (kRelax) {
+          int rg, key0, nk;
+          m.tile(j, rg, key0, nk);
+          if (rg != 2) {                           // column-segment slots: + log r (0 on sinks)
+            const float* brow = p.bias + (long long)m.u * p.col_stride + key0;   // padded by 64
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] += __ldg(brow + c);
+          }
+        }
         if ((b0 & b1) != ~0u) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -560,12 +547,8 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
           float2 z = __ffma2_rn(make_float2(s[2 * c2], s[2 * c2 + 1]), sc2, nm2);
-          if (kPolyEvery > 0 && c2 % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-            z = exp2_poly2(z);
-          } else {
-            z.x = ex2(z.x);
-            z.y = ex2(z.y);
-          }
+          z.x = ex2(z.x);
+          z.y = ex2(z.y);
           acc2[c2 & 3] = __fadd2_rn(acc2[c2 & 3], z);
           __nv_bfloat162 v2 = __floats2bfloat162_rn(z.x, z.y);
           pk[c2] = *reinterpret_cast<uint32_t*>(&v2);
@@ -577,48 +560,107 @@ attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PF + x));
-        // S_x of this item's last tile has run, so Q_x is no longer read: load the
-        // next item's Q (overlapping this tile's PV, which reads only P and V)
-        if (j == m.total - 1 && has_next && !(ok = copy_q(it + 1))) break;
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16 rows staged in this tile's region of the Q
-      // buffer (thread `row` has already copied its row of the next item's Q
-      // out of it), then one TMA store per 64-column half; rows past T are
-      // clipped by the copy
-      ok = mbar_wait(bar(B_PVD + x), it & 1, abort_flag, p.err, 223);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      tc_fence_after();
-      const float inv = __frcp_rn(l_sum);
-      uint8_t* srow = smem + kOffQ + x * kQTile + row * 128;
-#pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 64) {        // one 64-column half per wait
-        uint32_t orr[64];
-        tmem_ld32(lane_addr + colO + c0, *reinterpret_cast<uint32_t(*)[32]>(&orr[0]));
-        tmem_ld32(lane_addr + colO + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&orr[32]));
-        tmem_wait_ld();
-        uint8_t* half = srow + (c0 >> 6) * kQHalf;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {               // 16-byte chunk e of the half row
-          uint4 v;
-          uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-          for (int f = 0; f < 4; ++f) {
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[8 * e + 2 * f]) * inv,
-                                                      __uint_as_float(orr[8 * e + 2 * f + 1]) * inv);
-            w[f] = *reinterpret_cast<uint32_t*>(&v2);
-          }
-          *reinterpret_cast<uint4*>(half + ((e ^ (row & 7)) << 4)) = v;
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(B_OE + x));                  // O_x has been read: the next item may overwrite it
-      if (row_ok && p.lse != nullptr)
-        p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
-            (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
-      fence_proxy_async();
-      mbar_arrive(bar(B_STG + x));                  // this row is staged (warp 2 + x stores it)
+      // the item's l and max for the epilogue warpgroup (slot and barrier of this item's parity)
+      lm[256 * (it & 1)] = make_float2(l_sum, m_ref);
+      mbar_arrive(bar(B_LM + 2 * x + (it & 1)));
       g0 += m.total;
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    // ============================================================ item boundaries
+    const int quad = warp & 3;                     // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int g_in_row = row % p.G;
+    const float2* lm = reinterpret_cast<const float2*>(smem + kOffLM) + row;
+    // copy this thread's row of Q tile x from the shared buffer (128B-swizzled
+    // halves) into TMEM; the caller has seen the buffer's Q copy land
+    auto copy_q = [&](int x) {
+      const uint8_t* qrow = smem + kOffQ + x * kQTile + row * 128;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(qrow + hf * kQHalf + ((c ^ (row & 7)) << 4));
+          r[4 * c] = v4.x; r[4 * c + 1] = v4.y; r[4 * c + 2] = v4.z; r[4 * c + 3] = v4.w;
+        }
+        tmem_st32(lane_addr + col_q(x) + hf * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_QC + x));
+      mbar_arrive(bar(B_QFREE));
+    };
+    int it = 0;
+    bool ok = true;
+    if (blockIdx.x < p.n_items) {
+      ok = wwait(bar(B_QF), 0, abort_flag, p.err, 224);
+      if (ok) {
+        copy_q(0);
+        copy_q(1);
+      }
+    }
+    ItemCounts cn = load_counts(p, blockIdx.x);
+    for (int i = blockIdx.x; ok && i < p.n_items; i += gridDim.x, ++it) {
+      const Item m = make_item(p, i, cn);
+      cn = load_counts(p, i + gridDim.x);
+      // the next item's Q: tile x's rows go into TMEM once S_x of this item's last
+      // tile has run (Q_x is no longer read), overlapping that tile's softmax
+      if (i + (int)gridDim.x < p.n_items) {
+        if (!(ok = wwait(bar(B_QF), (it + 1) & 1, abort_flag, p.err, 224))) break;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (!(ok = wwait(bar(B_SL + x), it & 1, abort_flag, p.err, 226))) break;
+          tc_fence_after();
+          copy_q(x);
+        }
+        if (!ok) break;
+      }
+      // ---- epilogue: O / l -> bf16 rows staged in tile x's region of the Q
+      // buffer (the next item's rows have been copied out of it, and the store
+      // of the previous item has read it), then warp 2 + x stores them; rows
+      // past T are clipped by the copy
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (!(ok = wwait(bar(B_LM + 2 * x + (it & 1)), (it >> 1) & 1, abort_flag, p.err, 227)))
+          break;
+        if (!(ok = wwait(bar(B_PVD + x), it & 1, abort_flag, p.err, 223))) break;
+        if (it >= 1 && !(ok = wwait(bar(B_OST + x), (it - 1) & 1, abort_flag, p.err, 228))) break;
+        tc_fence_after();
+        const float2 lmv = lm[256 * (it & 1) + 128 * x];
+        const float l_sum = lmv.x, m_ref = lmv.y;
+        const float inv = __frcp_rn(l_sum);
+        uint8_t* srow = smem + kOffQ + x * kQTile + row * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < HD; c0 += 32) {      // 32 columns per wait
+          uint32_t orr[32];
+          tmem_ld32(lane_addr + col_o(x) + c0, orr);
+          tmem_wait_ld();
+          uint8_t* half = srow + (c0 >> 6) * kQHalf;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {             // 16-byte chunk (c0 % 64) / 8 + e of the half row
+            uint4 v;
+            uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[8 * e + 2 * f]) * inv,
+                                                        __uint_as_float(orr[8 * e + 2 * f + 1]) * inv);
+              w[f] = *reinterpret_cast<uint32_t*>(&v2);
+            }
+            const int chunk = ((c0 & 63) >> 3) + e;
+            *reinterpret_cast<uint4*>(half + ((chunk ^ (row & 7)) << 4)) = v;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_OE + x));                // O_x has been read: the next item may overwrite it
+        const int tt = m.t0 + x * p.TOK + row / p.G;
+        if (tt < p.T && p.lse != nullptr)
+          p.lse[((long long)m.b * p.Hq + m.h * p.G + g_in_row) * p.T + tt] =
+              (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
+        fence_proxy_async();
+        mbar_arrive(bar(B_STG + x));                // this row is staged (warp 2 + x stores it)
+      }
     }
   }
   tc_fence_before();
@@ -686,8 +728,14 @@ cudaError_t attn_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   p.scale_log2 = d->scale * 1.4426950408889634f;
   p.cnt = a.cnt;
   p.death = a.death;
+  p.bias = a.bias;
+  p.col_stride = d->sink + d->T;
   p.lse = a.lse; p.err = a.err;
-  auto kernel = a.death != nullptr ? attn_prefill_tc_kernel<true> : attn_prefill_tc_kernel<false>;
+  auto kernel = a.death != nullptr
+                    ? (a.bias != nullptr ? attn_prefill_tc_kernel<true, true>
+                                         : attn_prefill_tc_kernel<true, false>)
+                    : (a.bias != nullptr ? attn_prefill_tc_kernel<false, true>
+                                         : attn_prefill_tc_kernel<false, false>);
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;

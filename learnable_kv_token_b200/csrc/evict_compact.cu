@@ -216,6 +216,46 @@ cudaError_t retained_lifetimes(const lte_dims* d, const float* r, const int32_t*
 }
 
 // ---------------------------------------------------------------------------
+// Relaxed retention (training): the logit offset of every column-segment slot,
+// log r / scale for the retained token in the slot (so that adding it to the
+// raw score q.k multiplies the key's softmax weight by r), 0 for the sink
+// slots, the empty slots and 64 padding floats at the end (the attention
+// kernels read a whole 64-slot tile of offsets).  r is clamped below at 1e-30.
+__global__ void __launch_bounds__(256)
+slot_bias_kernel(long long n_slots, int T, int sink, float inv_scale, const float* __restrict__ r,
+                 const int32_t* __restrict__ idx, const int32_t* __restrict__ nret,
+                 float* __restrict__ bias) {
+  const long long stride = (long long)sink + T;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_slots + 64;
+       e += (long long)gridDim.x * blockDim.x) {
+    float b = 0.f;
+    if (e < n_slots) {
+      const long long u = e / stride;
+      const int i = (int)(e - u * stride) - sink;
+      if (i >= 0 && i < __ldg(nret + u)) {
+        const int j = __ldg(idx + u * T + i);
+        b = logf(fmaxf(__ldg(r + u * T + j), 1e-30f)) * inv_scale;
+      }
+    }
+    bias[e] = b;
+  }
+}
+
+size_t slot_bias_floats(const lte_dims* d) {
+  return (size_t)d->B * d->Hkv * ((size_t)d->sink + d->T) + 64;
+}
+
+cudaError_t slot_bias(const lte_dims* d, const float* r, const int32_t* idx, const int32_t* nret,
+                      float* bias, cudaStream_t stream) {
+  const long long n_slots = (long long)d->B * d->Hkv * ((long long)d->sink + d->T);
+  long long blocks = (n_slots + 64 + 255) / 256;
+  blocks = blocks > 148 * 16 ? 148 * 16 : blocks;
+  slot_bias_kernel<<<(unsigned)blocks, 256, 0, stream>>>(n_slots, d->T, d->sink, 1.0f / d->scale, r,
+                                                         idx, nret, bias);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Decode-cache set-up from a prefilled prompt (Fig. 3 layout): window ring,
 // sink slots, retained ring.  One CTA per unit.
 __global__ void __launch_bounds__(256)

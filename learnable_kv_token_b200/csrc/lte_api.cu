@@ -123,11 +123,18 @@ lte_status lte_retained_lifetimes(const lte_dims* d, const float* r, const int32
   return from_cuda(lte::retained_lifetimes(d, r, idx, nret, death, as_stream(stream)));
 }
 
+// relaxed-retention workspace: error word, the slot offsets, then (backward) D_t
+inline size_t relaxed_bias_bytes(const lte_dims* d) {
+  return (lte::slot_bias_floats(d) * sizeof(float) + 255) & ~(size_t)255;
+}
+
 size_t lte_workspace_bytes(const lte_dims* d, int32_t which) {
   if (check_dims(d) != LTE_OK) return 0;
   if (which == LTE_WS_PREFILL) return kErrBytes + lte::attn_prefill_scratch_bytes(d);
   if (which == LTE_WS_DECODE) return kErrBytes + lte::decode_scratch_bytes(d);
   if (which == LTE_WS_BACKWARD) return kErrBytes + lte::attn_backward_scratch_bytes(d);
+  if (which == LTE_WS_RELAXED)
+    return kErrBytes + relaxed_bias_bytes(d) + lte::attn_backward_scratch_bytes(d);
   return 0;
 }
 
@@ -224,6 +231,118 @@ lte_status lte_sparse_attn_prefill(const lte_dims* d, const void* q, const void*
   return from_cuda(e);
 }
 
+// Shared checks of the relaxed-retention calls (contiguous bf16, head dim 128,
+// the tcgen05 kernels' group sizes).
+static lte_status check_relaxed(const lte_dims* d, const int32_t* death, const void* workspace,
+                                size_t ws_bytes) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (d->cap_policy == LTE_CAP_LOWEST && death == nullptr) return LTE_ERR_INVALID_ARG;
+  if (d->dtype != LTE_BF16 || !lte::attn_prefill_tc_supported(d) ||
+      !lte::attn_backward_dq_tc_supported(d))
+    return LTE_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned16(workspace)) return LTE_ERR_WORKSPACE;
+  if (ws_bytes < lte_workspace_bytes(d, LTE_WS_RELAXED)) return LTE_ERR_WORKSPACE;
+  return LTE_OK;
+}
+
+lte_status lte_sparse_attn_prefill_relaxed(const lte_dims* d, const void* q, const void* k,
+                                           const void* v, const int32_t* cnt, const int32_t* death,
+                                           const int32_t* idx, const int32_t* nret,
+                                           const void* k_col, const void* v_col, const float* r,
+                                           void* o, float* lse, void* workspace, size_t ws_bytes,
+                                           void* stream) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (!q || !k || !v || !cnt || !idx || !nret || !k_col || !v_col || !r || !o)
+    return LTE_ERR_INVALID_ARG;
+  const void* vec[] = {q, k, v, k_col, v_col, o};
+  for (const void* p : vec)
+    if (!aligned16(p)) return LTE_ERR_INVALID_ARG;
+  if ((st = check_relaxed(d, death, workspace, ws_bytes)) != LTE_OK) return st;
+  float* bias = reinterpret_cast<float*>(static_cast<char*>(workspace) + kErrBytes);
+  cudaError_t e = lte::slot_bias(d, r, idx, nret, bias, as_stream(stream));
+  if (e != cudaSuccess) return LTE_ERR_CUDA;
+  lte::PrefillArgs a{};
+  a.d = d;
+  a.q = q; a.k = k; a.v = v;
+  get_strides(d, nullptr, d->Hq, &a.qs);
+  get_strides(d, nullptr, d->Hkv, &a.kvs);
+  get_strides(d, nullptr, d->Hq, &a.os);
+  a.cnt = cnt; a.k_col = k_col; a.v_col = v_col; a.o = o; a.lse = lse;
+  a.death = d->cap_policy == LTE_CAP_LOWEST ? death : nullptr;
+  a.err = reinterpret_cast<lte::DevError*>(workspace);
+  a.scratch = nullptr;
+  a.scratch_bytes = 0;
+  a.bias = bias;
+  return from_cuda(lte::attn_prefill_tc(a, as_stream(stream)));
+}
+
+lte_status lte_sparse_attn_backward_relaxed(const lte_dims* d, const void* q, const void* k,
+                                            const void* v, const int32_t* cnt,
+                                            const int32_t* death, const int32_t* idx,
+                                            const int32_t* nret, const void* k_col,
+                                            const void* v_col, const float* r, const void* o,
+                                            const float* lse, const void* dO, float* dq,
+                                            float* dk, float* dv, float* dr, void* workspace,
+                                            size_t ws_bytes, void* stream) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (!q || !k || !v || !cnt || !idx || !nret || !k_col || !v_col || !r || !o || !lse || !dO ||
+      !dq || !dk || !dv || !dr)
+    return LTE_ERR_INVALID_ARG;
+  const void* vec[] = {q, k, v, k_col, v_col, o, dO, dq, dk, dv};
+  for (const void* p : vec)
+    if (!aligned16(p)) return LTE_ERR_INVALID_ARG;
+  if ((st = check_relaxed(d, death, workspace, ws_bytes)) != LTE_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  float* bias = reinterpret_cast<float*>(ws + kErrBytes);
+  cudaError_t e = lte::slot_bias(d, r, idx, nret, bias, as_stream(stream));
+  if (e != cudaSuccess) return LTE_ERR_CUDA;
+  lte::BackwardArgs a{};
+  a.d = d;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO;
+  a.cnt = cnt; a.death = d->cap_policy == LTE_CAP_LOWEST ? death : nullptr; a.idx = idx;
+  a.nret = nret; a.k_col = k_col; a.v_col = v_col; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.err = reinterpret_cast<lte::DevError*>(workspace);
+  a.scratch = ws + kErrBytes + relaxed_bias_bytes(d);
+  a.bias = bias;
+  a.dr = dr;
+  return from_cuda(lte::attn_backward(a, as_stream(stream)));
+}
+
+lte_status lte_sparse_attn_prefill_kernel(const lte_dims* d, const lte_strides* q_strides,
+                                          const lte_strides* kv_strides,
+                                          const lte_strides* o_strides, int32_t* kind) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (kind == nullptr) return LTE_ERR_INVALID_ARG;
+  const int G = d->Hq / d->Hkv;
+  if (d->dtype == LTE_BF16 && (64 % G != 0 || G > 16)) return LTE_ERR_UNSUPPORTED;
+  lte::PrefillArgs a{};
+  a.d = d;
+  if ((st = get_strides(d, q_strides, d->Hq, &a.qs)) != LTE_OK) return st;
+  if ((st = get_strides(d, kv_strides, d->Hkv, &a.kvs)) != LTE_OK) return st;
+  if ((st = get_strides(d, o_strides, d->Hq, &a.os)) != LTE_OK) return st;
+  if (lte::attn_prefill_tc_supported(d) && lte::attn_prefill_tc_layout_ok(a))
+    *kind = LTE_KERNEL_TCGEN05;
+  else
+    *kind = d->dtype == LTE_BF16 ? LTE_KERNEL_MMA_SYNC : LTE_KERNEL_SIMT;
+  return LTE_OK;
+}
+
+lte_status lte_sparse_attn_backward_kernel(const lte_dims* d, int32_t* kind) {
+  lte_status st = check_dims(d);
+  if (st != LTE_OK) return st;
+  if (kind == nullptr) return LTE_ERR_INVALID_ARG;
+  if (d->dtype != LTE_BF16) return LTE_ERR_UNSUPPORTED;
+  const int G = d->Hq / d->Hkv;
+  if (64 % G != 0 || G > 16) return LTE_ERR_UNSUPPORTED;
+  *kind = lte::attn_backward_dq_tc_supported(d) ? LTE_KERNEL_TCGEN05 : LTE_KERNEL_MMA_SYNC;
+  return LTE_OK;
+}
+
 lte_status lte_cache_init_from_prefill(const lte_dims* d, const lte_cache* cache, const void* k,
                                        const void* v, const lte_strides* kv_strides,
                                        const float* r, const int32_t* idx, const int32_t* cnt,
@@ -306,6 +425,13 @@ lte_status lte_decode_step_noalloc(const lte_dims* d, const lte_cnn* cnn, const 
   return from_cuda(lte::decode_step(d, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_batch,
                                     reinterpret_cast<lte::DevError*>(scratch),
                                     static_cast<char*>(scratch) + kErrBytes, as_stream(stream)));
+}
+
+lte_status lte_noalloc_read_device_error(int32_t* code, int32_t* where, void* stream) {
+  if (code == nullptr) return LTE_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (lte::noalloc_scratch(&scratch) != cudaSuccess) return LTE_ERR_CUDA;
+  return lte_read_device_error(scratch, code, where, stream);
 }
 
 lte_status lte_clear_device_error(void* workspace, void* stream) {

@@ -35,6 +35,12 @@ cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask
                           cudaStream_t stream);
 cudaError_t retained_lifetimes(const lte_dims* d, const float* r, const int32_t* idx,
                                const int32_t* nret, int32_t* death, cudaStream_t stream);
+// relaxed retention: bias[u][slot] = log(r[u][idx[u][slot - s]]) / scale on the
+// retained slots of the column segment, 0 elsewhere (slots [0, s + T) plus 64
+// zero floats of padding at the end)
+size_t slot_bias_floats(const lte_dims* d);
+cudaError_t slot_bias(const lte_dims* d, const float* r, const int32_t* idx, const int32_t* nret,
+                      float* bias, cudaStream_t stream);
 cudaError_t cache_init(const lte_dims* d, const lte_cache* c, const void* k, const void* v,
                        Strides4 s, const float* r, const int32_t* idx, const int32_t* cnt,
                        const int32_t* death, int T_prompt, int n_scored, cudaStream_t stream);
@@ -52,6 +58,7 @@ struct PrefillArgs {
   DevError* err;
   void* scratch;         // workspace after the error word
   size_t scratch_bytes;
+  const float* bias;     // relaxed retention: logit offset per column-segment slot, else NULL
 };
 cudaError_t attn_prefill_simt(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t attn_prefill_mma(const PrefillArgs& a, cudaStream_t stream);
@@ -70,6 +77,8 @@ struct BackwardArgs {
   float *dq, *dk, *dv;
   DevError* err;                    // the workspace's error word
   void* scratch;                    // workspace after the error word
+  const float* bias;                // relaxed retention: slot logit offsets, else NULL
+  float* dr;                        // relaxed retention: dL/dr [B,Hkv,T], else NULL
 };
 size_t attn_backward_scratch_bytes(const lte_dims* d);
 cudaError_t attn_backward(const BackwardArgs& a, cudaStream_t stream);

@@ -111,6 +111,50 @@ def prefill(q, k, v, p: LayerParams, mask=None, cnn=None, bufs: PrefillBuffers |
                       bufs.death if lowest else None)
 
 
+def prefill_relaxed(q, k, v, out: PrefillOut, r, p: LayerParams, stream=None):
+    """Training-time forward with relaxed retention over the attended sets of
+    `out` (from prefill on the same q, k, v): every retained-segment key j
+    enters the softmax with weight r[j] (r [B,Hkv,T] fp32, the scores behind
+    the retention mask).  Returns (o, lse, workspace); pass the workspace on
+    to backward_relaxed."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, T, dtype=torch.float32, device=q.device)
+    ws_bytes = L.lte_workspace_bytes(dims, L.LTE_WS_RELAXED)
+    ws = torch.zeros((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=q.device)
+    L.lte_sparse_attn_prefill_relaxed(dims, q, k, v, out.cnt, out.death, out.idx, out.nret,
+                                      out.k_col, out.v_col, r, o, lse, ws, stream)
+    return o, lse, ws
+
+
+def backward_relaxed(q, k, v, out: PrefillOut, r, o, lse, do, p: LayerParams, ws=None,
+                     stream=None, check_errors=False):
+    """Gradients of the relaxed-retention forward (o, lse from
+    prefill_relaxed): dq [B,T,Hq,D], dk, dv [B,T,Hkv,D] and dr [B,Hkv,T]
+    (fp32), dr being the dL/dr that lte_score_backward takes."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    dims = p.dims(B, T, Hq, Hkv, D, q.dtype)
+    dev = q.device
+    dq = torch.empty(B, T, Hq, D, dtype=torch.float32, device=dev)
+    dk = torch.empty(B, T, Hkv, D, dtype=torch.float32, device=dev)
+    dv = torch.empty(B, T, Hkv, D, dtype=torch.float32, device=dev)
+    dr = torch.empty(B, Hkv, T, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws_bytes = L.lte_workspace_bytes(dims, L.LTE_WS_RELAXED)
+        ws = torch.zeros((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    L.lte_sparse_attn_backward_relaxed(dims, q, k, v, out.cnt, out.death, out.idx, out.nret,
+                                       out.k_col, out.v_col, r, o, lse, do, dq, dk, dv, dr, ws,
+                                       stream)
+    if check_errors:
+        code, where = L.lte_read_device_error(ws, stream)
+        if code != 0:
+            raise L.LteError(f"lte_sparse_attn_backward_relaxed (device check {where})", code)
+    return dq, dk, dv, dr
+
+
 def backward(q, k, v, out: PrefillOut, do, p: LayerParams, stream=None, check_errors=False):
     """Gradients (fp32) of the prefill attention for the attended sets that
     `out` (from prefill on the same q, k, v) used, given dO = do.
@@ -185,6 +229,10 @@ class Decoder:
         L.lte_decode_step(self.dims, self.cnn, self.cache.struct, q_t, k_t, v_t, self.o, self.lse,
                           self.score_batch, self.ws, stream)
         return self.o, self.lse
+
+    def device_error(self, stream=None):
+        """(code, where) of this decoder's workspace error word (synchronises)."""
+        return L.lte_read_device_error(self.ws, stream)
 
 
 class HostPrefill:

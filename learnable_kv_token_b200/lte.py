@@ -22,7 +22,8 @@ _lib = C.CDLL(LIB_PATH)
 
 LTE_F32, LTE_BF16 = 0, 1
 LTE_CAP_RECENT, LTE_CAP_FIRST, LTE_CAP_LOWEST = 0, 1, 2
-LTE_WS_PREFILL, LTE_WS_DECODE, LTE_WS_BACKWARD = 0, 1, 2
+LTE_WS_PREFILL, LTE_WS_DECODE, LTE_WS_BACKWARD, LTE_WS_RELAXED = 0, 1, 2, 3
+LTE_KERNEL_TCGEN05, LTE_KERNEL_MMA_SYNC, LTE_KERNEL_SIMT = 1, 2, 3
 STATUS = {0: "LTE_OK", 1: "LTE_ERR_INVALID_ARG", 2: "LTE_ERR_UNSUPPORTED", 3: "LTE_ERR_CUDA",
           4: "LTE_ERR_TIMEOUT", 5: "LTE_ERR_WORKSPACE", 6: "LTE_ERR_DEVICE"}
 
@@ -67,6 +68,8 @@ _SIG = {
                                 C.POINTER(lte_strides), _P, _P, _P, _P, _P,
                                 C.POINTER(lte_strides), _P, _P, C.c_size_t, _P],
     "lte_sparse_attn_backward": [C.POINTER(lte_dims)] + [_P] * 16 + [C.c_size_t, _P],
+    "lte_sparse_attn_prefill_relaxed": [C.POINTER(lte_dims)] + [_P] * 13 + [C.c_size_t, _P],
+    "lte_sparse_attn_backward_relaxed": [C.POINTER(lte_dims)] + [_P] * 18 + [C.c_size_t, _P],
     "lte_score_backward": [C.POINTER(lte_dims), C.POINTER(lte_cnn), _P, _P, C.POINTER(lte_strides),
                            _I] + [_P] * 8 + [C.c_size_t, _P],
     "lte_cache_init_from_prefill": [C.POINTER(lte_dims), C.POINTER(lte_cache), _P, _P,
@@ -75,6 +78,11 @@ _SIG = {
                         _P, _P, _I, _P, C.c_size_t, _P],
     "lte_decode_step_noalloc": [C.POINTER(lte_dims), C.POINTER(lte_cnn), C.POINTER(lte_cache), _P,
                                 _P, _P, _P, _P, _I, _P],
+    "lte_noalloc_read_device_error": [C.POINTER(C.c_int32), C.POINTER(C.c_int32), _P],
+    "lte_sparse_attn_prefill_kernel": [C.POINTER(lte_dims), C.POINTER(lte_strides),
+                                       C.POINTER(lte_strides), C.POINTER(lte_strides),
+                                       C.POINTER(C.c_int32)],
+    "lte_sparse_attn_backward_kernel": [C.POINTER(lte_dims), C.POINTER(C.c_int32)],
     "lte_clear_device_error": [_P, _P],
     "lte_read_device_error": [_P, C.POINTER(C.c_int32), C.POINTER(C.c_int32), _P],
     "lte_wait_probe": [_P, _I, C.c_int64, _P, _P],
@@ -195,6 +203,21 @@ def lte_sparse_attn_backward(dims, q, k, v, cnt, death, idx, nret, k_col, v_col,
           workspace.numel() * workspace.element_size(), _stream(stream))
 
 
+def lte_sparse_attn_prefill_relaxed(dims, q, k, v, cnt, death, idx, nret, k_col, v_col, r, o, lse,
+                                    workspace, stream=None):
+    _call("lte_sparse_attn_prefill_relaxed", C.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(cnt),
+          _ptr(death), _ptr(idx), _ptr(nret), _ptr(k_col), _ptr(v_col), _ptr(r), _ptr(o), _ptr(lse),
+          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+
+
+def lte_sparse_attn_backward_relaxed(dims, q, k, v, cnt, death, idx, nret, k_col, v_col, r, o, lse,
+                                     do, dq, dk, dv, dr, workspace, stream=None):
+    _call("lte_sparse_attn_backward_relaxed", C.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(cnt),
+          _ptr(death), _ptr(idx), _ptr(nret), _ptr(k_col), _ptr(v_col), _ptr(r), _ptr(o), _ptr(lse),
+          _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dr), _ptr(workspace),
+          workspace.numel() * workspace.element_size(), _stream(stream))
+
+
 def lte_cache_init_from_prefill(dims, cache, k, v, r, idx, cnt, T_prompt, n_scored, stream=None,
                                 death=None):
     _call("lte_cache_init_from_prefill", C.byref(dims), C.byref(cache), _ptr(k), _ptr(v),
@@ -215,6 +238,31 @@ def lte_decode_step_noalloc(dims, cnn, cache, q_t, k_t, v_t, o_t, lse_t, score_b
     (for callers that cannot allocate device memory; see lte_api.h)."""
     _call("lte_decode_step_noalloc", C.byref(dims), C.byref(cnn), C.byref(cache), _ptr(q_t),
           _ptr(k_t), _ptr(v_t), _ptr(o_t), _ptr(lse_t), score_batch, _stream(stream))
+
+
+def lte_noalloc_read_device_error(stream=None):
+    """(code, where) of the error word in lte_decode_step_noalloc's static
+    scratch (the last call on the current device); synchronises the stream."""
+    code, where = C.c_int32(0), C.c_int32(0)
+    _call("lte_noalloc_read_device_error", C.byref(code), C.byref(where), _stream(stream))
+    return code.value, where.value
+
+
+def lte_sparse_attn_prefill_kernel(dims, q_strides=None, kv_strides=None, o_strides=None):
+    """Kernel family (LTE_KERNEL_*) lte_sparse_attn_prefill runs for these dims
+    and lte_strides (None = contiguous).  Host only."""
+    kind = C.c_int32(0)
+    ref = (lambda s: None if s is None else C.byref(s))
+    _call("lte_sparse_attn_prefill_kernel", C.byref(dims), ref(q_strides), ref(kv_strides),
+          ref(o_strides), C.byref(kind))
+    return kind.value
+
+
+def lte_sparse_attn_backward_kernel(dims):
+    """Kernel family (LTE_KERNEL_*) lte_sparse_attn_backward runs for these dims."""
+    kind = C.c_int32(0)
+    _call("lte_sparse_attn_backward_kernel", C.byref(dims), C.byref(kind))
+    return kind.value
 
 
 def lte_clear_device_error(workspace, stream=None):

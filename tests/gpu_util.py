@@ -24,6 +24,12 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").double().numpy()
 
 
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """float64 values rounded to bf16 (round to nearest even) and widened back:
+    the storage format of a bf16 output."""
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+
+
 def oracle_cnn(cnn, h: int, past1=2, past2=1) -> O.CNN:
     w1, b1, w2, b2 = (f64(x) for x in cnn)
     return O.CNN(w1[h], b1[h], w2[h], float(b2[h]), past1, past2)
@@ -77,3 +83,49 @@ def oracle_rows(q, k, v, masks, b, h, rows, sink, window, cap, scale, policy=O.C
 
 def scale_of(D):
     return 1.0 / math.sqrt(D)
+
+
+# Gradients of the attention (bf16 products, fp32 accumulation): every element
+# of a row (one position of dk / dv, one (position, head) of dq) within
+# GRAD_ROW of that row's largest reference entry, plus GRAD_ABS.  P and dS are
+# rounded to bf16 (2^-9 relative) before the products that use them, so a
+# gradient sum carries about 2^-8 relative error per term, well inside 2e-2;
+# a missing or doubled contribution to one row (a slot attended from many
+# rows) moves that row by far more.
+GRAD_ROW = 2e-2
+GRAD_ABS = 1e-6
+
+
+def assert_grad_close(g, ref, what="", extra=None):
+    """Element-wise gate of a gradient tensor [..., D] against the oracle's:
+    |g - ref| <= GRAD_ROW * max_row |ref| + GRAD_ABS (+ extra, an allowance
+    per element derived from the arithmetic, see dq_delta_allowance) at every
+    element.  Returns the largest error relative to its row's scale."""
+    g, ref = np.asarray(g, np.float64), np.asarray(ref, np.float64)
+    row = np.abs(ref).max(axis=-1, keepdims=True)
+    err = np.abs(g - ref)
+    bound = GRAD_ROW * row + GRAD_ABS
+    if extra is not None:
+        bound = bound + np.asarray(extra, np.float64)
+    bound = np.broadcast_to(bound, err.shape)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(int(np.argmax(err - bound)), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} element(s) outside the row bound; worst at "
+                             f"{i}: |err| {err[i]:.3g} > {bound[i]:.3g} (row max {row[i[:-1] + (0,)]:.3g}; row {i[:-1]})")
+    return float((err / np.maximum(row, 1e-30)).max())
+
+
+# The backward takes D_t = <dO_t, o_t> from the forward's stored output o.
+# That o differs from the exact one by at most 2^-8 |o| per element (P and
+# the output rounded to bf16), so D_t is off by up to 2^-8 sum_d |dO_td o_td|,
+# which moves dq_t by scale * dD_t * (P K)_t (dS = P (dP - D_t)).  On rows
+# with many keys this is far below the row gate; on rows with two or three
+# keys, where dq is a near-cancelling sum, it is not.
+def dq_delta_allowance(do, o, pk, scale):
+    """Per-element allowance for dq [..., D]: do, o the incoming gradient and
+    the oracle's output, pk the oracle's attention-weighted keys sum_j P_j k_j
+    (all [..., D])."""
+    do, o, pk = (np.asarray(x, np.float64) for x in (do, o, pk))
+    dD = 2.0 ** -8 * np.abs(do * o).sum(axis=-1, keepdims=True)
+    return scale * dD * np.abs(pk)

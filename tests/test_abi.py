@@ -128,3 +128,34 @@ def test_host_validation_without_gpu(lib):
     assert f.lte_wait_probe(C.c_void_p(16), 1, 10, C.c_void_p(16), None) == 1
     assert f.lte_wait_probe(C.c_void_p(16), 1, 1000000, None, None) == 5
     assert L.version().startswith("lte-b200")
+
+
+def test_kernel_choice_is_reported(lib):
+    """lte_sparse_attn_prefill_kernel / lte_sparse_attn_backward_kernel say
+    which kernel family the call runs, so a caller can see when a shape or a
+    stride leaves the tcgen05 kernels (host only, no GPU needed)."""
+    from learnable_kv_token_b200 import lte as L
+    mk = lambda D, dt, Hq=16, Hkv=4: L.make_dims(2, 256, Hq, Hkv, D, 4, 64, 32, 0.5, 0.1, dt)
+    assert L.lte_sparse_attn_prefill_kernel(mk(128, L.LTE_BF16)) == L.LTE_KERNEL_TCGEN05
+    assert L.lte_sparse_attn_prefill_kernel(mk(64, L.LTE_BF16)) == L.LTE_KERNEL_MMA_SYNC
+    assert L.lte_sparse_attn_prefill_kernel(mk(128, L.LTE_F32)) == L.LTE_KERNEL_SIMT
+    # q rows spaced by 1032 elements (2064 bytes, a multiple of 16) stay on tcgen05;
+    # an element stride of 8 per row but 8 + 4 per head is rejected as unaligned
+    ok = L.lte_strides(256 * 16 * 1032, 16 * 1032, 1032)
+    assert L.lte_sparse_attn_prefill_kernel(mk(128, L.LTE_BF16), ok, None, None) == \
+        L.LTE_KERNEL_TCGEN05
+    with pytest.raises(L.LteError) as ei:
+        L.lte_sparse_attn_prefill_kernel(mk(128, L.LTE_BF16), L.lte_strides(8, 8, 12), None, None)
+    assert ei.value.status == 1
+    with pytest.raises(L.LteError) as ei:                    # G = 32 is not supported in bf16
+        L.lte_sparse_attn_prefill_kernel(mk(128, L.LTE_BF16, Hq=32, Hkv=1))
+    assert ei.value.status == 2
+    assert L.lte_sparse_attn_backward_kernel(mk(128, L.LTE_BF16)) == L.LTE_KERNEL_TCGEN05
+    assert L.lte_sparse_attn_backward_kernel(mk(64, L.LTE_BF16)) == L.LTE_KERNEL_MMA_SYNC
+    with pytest.raises(L.LteError) as ei:
+        L.lte_sparse_attn_backward_kernel(mk(128, L.LTE_F32))
+    assert ei.value.status == 2
+    f = L._lib
+    assert f.lte_noalloc_read_device_error(None, None, None) == 1
+    assert f.lte_sparse_attn_prefill_kernel(C.byref(mk(128, L.LTE_BF16)), None, None, None,
+                                            None) == 1

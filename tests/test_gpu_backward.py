@@ -5,23 +5,28 @@ policies, GQA group sizes 1 to 16 and head dims 64 and 128.
 
 Tolerance.  The oracle works in float64 on the same bf16 inputs.  The kernels
 round P and dS to bf16 (relative 2^-9 each) before the products that use
-them and take D_t = <dO_t, o_t> from the bf16 output o, so every term of a
-gradient sum carries a relative error of about 2^-8.  Summed over hundreds of
-terms with mixed signs this gives a relative Frobenius error of a few 1e-3;
-the bound is 1e-2 per tensor, and 5e-2 of the tensor's largest entry for any
-single element."""
+them, so every term of a gradient sum carries a relative error of about
+2^-8.  D_t = <dO_t, o_t> is taken, as the call's contract states, from the
+forward output as stored (bf16); the oracle is given its own o rounded to
+bf16 for D_t, and dq gets an allowance for the forward output's own error
+in D_t (tests/gpu_util.dq_delta_allowance: it matters only on rows with few
+keys, where dq is a near-cancelling sum).  Every element must lie
+within 2e-2 of its row's largest reference entry (a row: one position of dk
+or dv, one (position, head) of dq), so a missing or doubled contribution to
+any one position fails; the relative Frobenius error of each tensor must also
+stay below 1e-2."""
 import numpy as np
 import pytest
 import torch
 
 import lte_inputs as LI
 from oracle import lte_oracle as O
-from tests.gpu_util import f64, fed_masks, scale_of
+from tests.gpu_util import (assert_grad_close, bf16_round, dq_delta_allowance, f64, fed_masks,
+                            scale_of)
 
 pytestmark = pytest.mark.gpu
 
 REL_FRO = 1e-2
-REL_MAX = 5e-2
 
 
 @pytest.fixture(scope="module")
@@ -30,11 +35,11 @@ def layer():
     return layer
 
 
-def _close(g, ref, what):
+def _close(g, ref, what, extra=None):
     g, ref = np.asarray(g, np.float64), np.asarray(ref, np.float64)
     fro = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
-    mx = np.abs(g - ref).max() / max(np.abs(ref).max(), 1e-30)
-    assert fro <= REL_FRO and mx <= REL_MAX, f"{what}: relative Frobenius {fro:.2e}, max {mx:.2e}"
+    assert fro <= REL_FRO, f"{what}: relative Frobenius {fro:.2e}"
+    mx = assert_grad_close(g, ref, what, extra)
     return fro, mx
 
 
@@ -74,11 +79,15 @@ def test_backward_vs_oracle(layer, case):
         masks, r64 = fed_masks(mask, sink), None
     dq, dk, dv = layer.backward(qd, kd, vd, out, dod, p, check_errors=True)
     torch.cuda.synchronize()
+    # D_t comes from the forward's stored output: the oracle's o rounded to bf16
+    o_ref, _, _ = O.prefill(f64(q), f64(k), f64(v), masks, sink, window, cap, scale_of(D), opol, r64)
+    pk, _, _ = O.prefill(f64(q), f64(k), f64(k), masks, sink, window, cap, scale_of(D), opol, r64)
     rq, rk, rv = O.prefill_backward(f64(q), f64(k), f64(v), masks, sink, window, cap, f64(do),
-                                    scale_of(D), opol, r64)
+                                    scale_of(D), opol, r64, o_out=bf16_round(o_ref))
+    extra = {"dq": dq_delta_allowance(f64(do), o_ref, pk, scale_of(D)), "dk": None, "dv": None}
     for name, a, b in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
-        fro, mx = _close(f64(a), b, f"{name} {case}")
-        print(f"{name}: relative Frobenius {fro:.2e}, max {mx:.2e}")
+        fro, mx = _close(f64(a), b, f"{name} {case}", extra[name])
+        print(f"{name}: relative Frobenius {fro:.2e}, worst element / row max {mx:.2e}")
 
 
 def test_backward_gradient_check_direction(layer):

@@ -138,3 +138,41 @@ def test_hybrid_gla_sampled():
         assert rel(f64(o[b, :, h]), o_ref[:T]) <= 1e-2, (b, h)
         assert rel(f64(od[:, b, h]), o_ref[T:]) <= 1e-2, (b, h)
         assert rel(f64(st[b, h]), S_ref) <= 1e-2, (b, h)
+
+
+# --------------------------------------------------------------------------- attention backward
+def test_backward_bench_shape_sampled(layer):
+    """lte_sparse_attn_backward at the bench's shape -- B=32, T=4096, Hq=16 /
+    Hkv=4, D=128, s=4, w=512, C=512, a fed Bernoulli(0.5) retention mask, so the
+    cap binds from t ~ 1500 on and a retained slot is attended from ~1000 rows
+    (the column pass's multi-CTA atomics at full depth) -- against the oracle's
+    prefill_backward_unit for two whole units: every element of dq, dk and dv
+    within 2e-2 of its row's largest reference entry (D_t from the oracle's own
+    o rounded to bf16, the forward's stored output)."""
+    from oracle import lte_oracle as O
+    from tests.gpu_util import assert_grad_close, bf16_round, dq_delta_allowance
+    B, T, Hq, Hkv, D, sink, window, cap = 32, 4096, 16, 4, 128, 4, 512, 512
+    G = Hq // Hkv
+    g = LI.generator(4242)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, torch.bfloat16, g)
+    do = LI.normal((B, T, Hq, D), 1.0, torch.bfloat16, g)
+    mask = LI.bernoulli_mask(B, Hkv, T, 0.5, g)
+    p = layer.LayerParams(sink=sink, window=window, cap=cap)
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    out = layer.prefill(qd, kd, vd, p, mask=mask.cuda())
+    dq, dk, dv = layer.backward(qd, kd, vd, out, dod, p, check_errors=True)
+    torch.cuda.synchronize()
+    masks = fed_masks(mask, sink)
+    for b, h in [(0, 0), (31, 3)]:
+        o_ref, _, _ = O.prefill_unit(f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]),
+                                     f64(v[b, :, h]), masks[b, h], sink, window, cap, scale_of(D))
+        rq, rk, rv = O.prefill_backward_unit(f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]),
+                                             f64(v[b, :, h]), masks[b, h], sink, window, cap,
+                                             scale_of(D), f64(do[b, :, h * G:(h + 1) * G]),
+                                             o_out=bf16_round(o_ref))
+        pk, _, _ = O.prefill_unit(f64(q[b, :, h * G:(h + 1) * G]), f64(k[b, :, h]),
+                                  f64(k[b, :, h]), masks[b, h], sink, window, cap, scale_of(D))
+        assert_grad_close(f64(dq[b, :, h * G:(h + 1) * G]), rq, f"dq unit {b},{h}",
+                          dq_delta_allowance(f64(do[b, :, h * G:(h + 1) * G]), o_ref, pk, scale_of(D)))
+        assert_grad_close(f64(dk[b, :, h]), rk, f"dk unit {b},{h}")
+        assert_grad_close(f64(dv[b, :, h]), rv, f"dv unit {b},{h}")

@@ -463,3 +463,34 @@ def test_device_error_word_clean(L, layer):
     layer.prefill(qd, kd, vd, p, mask=md, bufs=bufs)
     assert L.lte_read_device_error(bufs.ws) == (0, 0)
     del out_bufs
+
+
+def test_prefill_repeatable_long_items(layer):
+    """The tcgen05 prefill kernel gives bit-identical o and lse on repeated
+    launches over items with many key tiles (w = 1024, 16 retained-segment
+    tiles): the roles that hand work on at item boundaries (next Q rows into
+    TMEM, l and the max to the epilogue) wait on one phase per item, so a
+    role that runs ahead cannot pass on an older phase.  A race there shows
+    as launch-to-launch differences; the first launch is also checked
+    against the oracle on sampled rows."""
+    B, T, Hq, Hkv, D, s, w, C = 4, 4096, 16, 4, 128, 4, 1024, 1024
+    g = LI.generator(77)
+    q, k, v = LI.qkv(B, T, Hq, Hkv, D, torch.bfloat16, g)
+    mask = LI.bernoulli_mask(B, Hkv, T, 0.4, g)
+    p = layer.LayerParams(sink=s, window=w, cap=C)
+    qd, kd, vd, md = q.cuda(), k.cuda(), v.cuda(), mask.cuda()
+    outs = []
+    for _ in range(3):
+        out = layer.prefill(qd, kd, vd, p, mask=md)
+        torch.cuda.synchronize()
+        outs.append((out.o.clone(), out.lse.clone()))
+    for o, lse in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
+    masks = fed_masks(mask, s)
+    rows = [0, w - 1, w, w + 5, 2 * w + 17, T // 2, T - 1]
+    for b, h in [(0, 0), (3, 2)]:
+        o_ref, lse_ref, _ = oracle_rows(q, k, v, masks, b, h, rows, s, w, C, scale_of(D))
+        G = Hq // Hkv
+        assert_attention_close(f64(outs[0][0][b, rows, h * G:(h + 1) * G]),
+                               f64(outs[0][1][b, h * G:(h + 1) * G][:, rows]).T, o_ref, lse_ref,
+                               torch.bfloat16, f"unit {b},{h}")
