@@ -35,6 +35,13 @@ gla_decode_kernel(int H, const TIn* __restrict__ q, const TIn* __restrict__ k,
                   float* __restrict__ state) {
   const int bh = blockIdx.x >> 1, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int row0 = (blockIdx.x & 1) * (DV / 2);       // this CTA's half of the value rows
+  // Programmatic dependent launch: wait until the previous kernel in the stream
+  // has completed (its outputs may be this step's inputs, and it may be the
+  // previous step on this state), then let the next kernel launch, so its CTAs
+  // are resident and through their prologue when this step ends.  Both are
+  // no-ops when the launch did not allow programmatic serialization.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long vb = (long long)bh * DK;
   float q4[4], k4[4], a4[4];
 #pragma unroll
@@ -102,14 +109,23 @@ cudaError_t gla_decode(int B, int H, int dk, int dv, int dtype, const void* q, c
                        const void* v, const float* a, void* o, float* state,
                        cudaStream_t stream) {
   if (dk != gla::DK || dv != gla::DV) return cudaErrorNotSupported;
+  // launched with programmatic stream serialization (see the kernel's first lines)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * H * 2);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (dtype == LTE_BF16)
-    gla::gla_decode_kernel<__nv_bfloat16><<<B * H * 2, 128, 0, stream>>>(
-        H, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, a,
-        (__nv_bfloat16*)o, state);
-  else
-    gla::gla_decode_kernel<float><<<B * H * 2, 128, 0, stream>>>(
-        H, (const float*)q, (const float*)k, (const float*)v, a, (float*)o, state);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, gla::gla_decode_kernel<__nv_bfloat16>, H,
+                              (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                              (const __nv_bfloat16*)v, a, (__nv_bfloat16*)o, state);
+  return cudaLaunchKernelEx(&cfg, gla::gla_decode_kernel<float>, H, (const float*)q,
+                            (const float*)k, (const float*)v, a, (float*)o, state);
 }
 
 }  // namespace lte

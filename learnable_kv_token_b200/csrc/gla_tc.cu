@@ -40,8 +40,8 @@
 // of 32 gates falls below 2^-100 (a gate near 0 -- or exactly 0 -- within a
 // chunk), that chunk instead runs the recurrence itself, token by token, in
 // fp32 on the state held in registers (the TMEM group: thread (row, half)
-// updates S[row, 64 half .. + 63] and the halves' partial o_t[row] are added
-// through shared memory).  So every gate in [0, 1] gives the recurrence's
+// updates S[row, 64 half .. + 63], reading the raw gates from global memory,
+// and the halves' partial o_t[row] are added through shared memory).  So every gate in [0, 1] gives the recurrence's
 // result; only the speed of such chunks differs.
 // Every mbarrier wait is bounded; a CTA that gives up writes NaN into its
 // final state, so the failure is visible to the caller.
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                       const __grid_constant__ CUtensorMap tm_o, int T, int H,
-                      float* __restrict__ state) {
+                      const float* __restrict__ a_raw, float* __restrict__ state) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const int bh = blockIdx.x, b = bh / H, hd = bh % H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -218,12 +218,12 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           in_range = pa >= 0x1p-100f;
           lam_r[j] = pa;                                   // e^{b_last - b_m}
         }
-        in_range = group_and(kBarGate, kGroup, in_range);
-        if (in_range) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) Xj[i * DK] = g[i];
-        }
+        for (int i = 0; i < 32; ++i) Xj[i * DK] = g[i];
       }
+      // one barrier both publishes the factors and takes the vote (the exact
+      // path reads the raw gates from global memory)
+      in_range = group_and(kBarGate, kGroup, in_range);
       if (!in_range) {                                     // chunk c runs the recurrence
         if (gt == 0) {
           exact[set] = 1;
@@ -232,7 +232,6 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         continue;
       }
       if (gt == 0) exact[set] = 0;
-      group_sync(kBarGate, kGroup);
       // ---- Q~ = q x and K~ = k / x in place, Khat = K~ e^{b_last - b_m} in its buffer
       {
         const float* X = reinterpret_cast<const float*>(sset + kSetA);
@@ -306,11 +305,15 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
       if (exact[set]) {
         // ---- the recurrence, token by token, on raw q, k, v and gates: this
-        // thread holds S[row, 64 hc .. + 63] in registers; the half hc = 1 hands
+        // thread holds S[row, 64 hc .. + 63] (in local memory: the loop over its
+        // 16-byte chunks is not unrolled, to keep the main path's registers
+        // free -- this path only runs for chunks with extreme gates); the half hc = 1 hands
         // its part of o_t[row] to hc = 0 through the set's (unused) Khat buffer,
         // which writes o_t as bf16 into the staging tile
         const uint8_t* sset = sm + set * kSet;
         float* xbuf = reinterpret_cast<float*>(sm + set * kSet + kSetKhat);   // [2][128]
+        // the raw gates of this chunk (the shared table holds the factors)
+        const float* a_chunk = a_raw + (((long long)b * T + (long long)c * L) * H + hd) * DK + hc * 64;
         float S[64];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
@@ -322,17 +325,17 @@ gla_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
 #pragma unroll 1
         for (int t = 0; t < L; ++t) {
-          const float* at = reinterpret_cast<const float*>(sset + kSetA) + t * DK + hc * 64;
+          const float* at = a_chunk + (long long)t * H * DK;
           const uint32_t vo = swz(L, t, row >> 3) + (row & 7) * 2;
           const float vt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sset + kSetV + vo));
           float o = 0.f;
-#pragma unroll
+#pragma unroll 1
           for (int e8 = 0; e8 < 8; ++e8) {                 // 16-byte chunk hc * 8 + e8 of row t
             const uint32_t off = swz(L, t, hc * 8 + e8);
             const uint4 kv = *reinterpret_cast<const uint4*>(sset + kSetK + off);
             const uint4 qv = *reinterpret_cast<const uint4*>(sset + kSetQ + off);
-            const float4 a0 = *reinterpret_cast<const float4*>(at + 8 * e8);
-            const float4 a1 = *reinterpret_cast<const float4*>(at + 8 * e8 + 4);
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(at + 8 * e8));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(at + 8 * e8 + 4));
             const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const uint32_t* kw = reinterpret_cast<const uint32_t*>(&kv);
             const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv);
@@ -565,7 +568,7 @@ cudaError_t gla_prefill_tc(int B, int T, int H, const void* q, const void* k, co
   cudaError_t e = cudaFuncSetAttribute(gla_prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  gla_prefill_tc_kernel<<<B * H, kThreads, kSmem, stream>>>(mq, mk, mv, ma, mo, T, H, state);
+  gla_prefill_tc_kernel<<<B * H, kThreads, kSmem, stream>>>(mq, mk, mv, ma, mo, T, H, a, state);
   return cudaGetLastError();
 }
 

@@ -332,3 +332,71 @@ def test_decode_scores_match_lte_score(layer):
                     assert abs(r[b, h, j] - ro[j]) <= R_TOL, (b, h, j)
                     checked += 1
     assert checked >= B * Hkv * 32
+
+
+def test_hybrid_pair_chain_in_graph(layer):
+    """The laLTE pair step -- a gated linear-attention decode step, then the LTE
+    decode step -- alternated over two layers inside one CUDA graph.  Both
+    kernels launch with programmatic dependent launch (each waits for its
+    predecessor before touching memory), so the chained graph must give
+    exactly what each layer gives run alone, step by step: the LTE outputs
+    and caches bit-identical to the plain decode, the GLA outputs and states
+    bit-identical to its own steps in a plain loop."""
+    from learnable_kv_token_b200 import lte as L
+    B, Hq, Hkv, D, sink, window, cap, T0, steps, n_layers = 2, 8, 2, 128, 4, 64, 32, 100, 24, 2
+    q, k, v, cnn = _inputs(B, Hq, Hkv, D, T0 + steps, 19, w_std=0.1)
+    o_ref, _, _, cache_ref, _ = _gpu_decode(layer, q, k, v, cnn, sink, window, cap, 0.5, T0, 8)
+    H_g = 4
+    gq, gk, gv, ga = (x.cuda() for x in LI.gla_inputs(B, steps, H_g, 128, 128, LI.generator(23)))
+    # GLA alone, plain loop
+    st_ref = torch.zeros(B, H_g, 128, 128, device="cuda")
+    go_ref = []
+    for i in range(steps):
+        o_t = torch.empty(B, H_g, 128, dtype=torch.bfloat16, device="cuda")
+        L.lte_gla_decode_step(gq[:, i].contiguous(), gk[:, i].contiguous(), gv[:, i].contiguous(),
+                              ga[:, i].contiguous(), o_t, st_ref)
+        go_ref.append(o_t)
+    # the pair, two layers with identical inputs, in one graph per step
+    p = layer.LayerParams(sink=sink, window=window, cap=cap, tau=0.5)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    cd = tuple(x.cuda() for x in cnn)
+    kp, vp = kd[:, :T0].contiguous(), vd[:, :T0].contiguous()
+    out = layer.prefill(qd[:, :T0].contiguous(), kp, vp, p, cnn=cd)
+    dims = p.dims(B, T0, Hq, Hkv, D, torch.bfloat16)
+    decs, states = [], []
+    for _ in range(n_layers):
+        c = layer.DecodeCache(B, Hkv, D, torch.bfloat16, sink, window, cap)
+        c.init_from_prefill(dims, kp, vp, out, T0)
+        decs.append(layer.Decoder(dims, cd, p.past1, p.past2, c, 8))
+        states.append(torch.zeros(B, H_g, 128, 128, device="cuda"))
+    q_in = torch.empty(B, Hq, D, dtype=torch.bfloat16, device="cuda")
+    k_in = torch.empty(B, Hkv, D, dtype=torch.bfloat16, device="cuda")
+    v_in = torch.empty_like(k_in)
+    g_in = [torch.empty(B, H_g, 128, dtype=dt, device="cuda")
+            for dt in (torch.bfloat16, torch.bfloat16, torch.bfloat16, torch.float32)]
+    g_out = [torch.empty(B, H_g, 128, dtype=torch.bfloat16, device="cuda") for _ in range(n_layers)]
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            for d_, st_, go_ in zip(decs, states, g_out):
+                L.lte_gla_decode_step(*g_in, go_, st_, s)
+                d_.step(q_in, k_in, v_in, stream=s)
+    outs = [[] for _ in range(n_layers)]
+    gouts = [[] for _ in range(n_layers)]
+    for i, t in enumerate(range(T0, T0 + steps)):
+        q_in.copy_(qd[:, t]); k_in.copy_(kd[:, t]); v_in.copy_(vd[:, t])
+        for dst, src in zip(g_in, (gq, gk, gv, ga)):
+            dst.copy_(src[:, i])
+        graph.replay()
+        for l in range(n_layers):
+            outs[l].append(decs[l].o.clone())
+            gouts[l].append(g_out[l].clone())
+    torch.cuda.synchronize()
+    for l in range(n_layers):
+        assert torch.equal(torch.stack(outs[l]), o_ref)
+        assert torch.equal(decs[l].cache.pos, cache_ref.pos)
+        assert torch.equal(torch.stack(gouts[l]), torch.stack(go_ref))
+        assert torch.equal(states[l], st_ref)
+        assert decs[l].device_error() == (0, 0)
