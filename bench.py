@@ -542,11 +542,6 @@ def sweep_bench(args, rank, world, device, only=None, reps=5):
             "launches": len(points) * (5 + reps + 2 + 1)}
 
 
-# fp32 FMA throughput of one B200 from its unit counts and clock (no measured
-# fp32 peak is recorded): 148 SMs x 128 lanes x 2 flops x 1.965 GHz
-FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-
-
 def rows_bench(args, rank, world, device, dec):
     """The hot-path rows outside the two headline steps, each launch timed alone
     with CUDA events after warm-up, on the hybrid workload (B=32, 4096-token
@@ -662,12 +657,11 @@ def rows_bench(args, rank, world, device, dec):
         "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
         "a3b_backward_ms": t_bwd, "a3b_roofline": tensor(bwd_flops, t_bwd),
         "a1b_score_backward_ms": t_sbwd,
-        "a1b_roofline": {"bound": "alu", "achieved": sbwd_flops / (t_sbwd / 1e3) / 1e12,
-                         "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
-                         "frac": sbwd_flops / (t_sbwd / 1e3) / 1e12 / FP32_FMA_TFLOPS,
-                         "flops": sbwd_flops,
-                         "note": "lte_score_backward, fp32 SIMT; peak = 148 SMs x 128 fp32 lanes "
-                                 "x 2 flops x 1.965 GHz"},
+        "a1b_roofline": dict(tensor(sbwd_flops, t_sbwd),
+                             note="lte_score_backward: layer-1 recompute, dx and dw1 on tcgen05 "
+                                  "(hi/lo bf16 operands: 2-3x the MMA work of these algorithmic "
+                                  "flops), the elementwise pass on CUDA cores; FLOPs = 3 x 2 x "
+                                  "c_hid x 2D x k1 per (b, KV head, position)"),
         "a3b_note": "lte_sparse_attn_backward (delta, dQ, dK/dV window, dK/dV column: 4 "
                     "launches, tcgen05) on the same scored mask; FLOPs = 2.5 x the forward's",
         "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),

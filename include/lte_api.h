@@ -132,10 +132,15 @@ lte_status lte_score(const lte_dims* d, const lte_cnn* cnn,
  *   dw1 [Hkv,c_hid,2D,k1], db1 [Hkv,c_hid], dw2 [Hkv,c_hid,k2], db2 [Hkv]
  *          (fp32): dL/dweights summed over the batch, OVERWRITTEN.
  * k, v as in lte_score (kv_strides may be NULL); dr: fp32 [B,Hkv,T], entries
- * j >= n_scored ignored; 0 <= n_scored <= T - F.  fp32 SIMT arithmetic; the
+ * j >= n_scored ignored; 0 <= n_scored <= T - F.  Arithmetic: fp32 throughout,
+ * except that for bf16 inputs with head dim 128 and c_hid 32 the three
+ * contractions (the layer-1 recompute, dx and dw1) run on tcgen05 tensor
+ * cores with fp32 operands split into bf16 hi + lo pairs (relative error
+ * about 2^-16) and fp32 accumulation; elsewhere fp32 CUDA-core kernels.  The
  * weight gradients add fp32 partial sums with atomics (last bits may vary).
- * Workspace: lte_score_backward_workspace_bytes(d, cnn) bytes (error word and
- * 2 x B x Hkv x c_hid x T floats).
+ * Workspace: lte_score_backward_workspace_bytes(d, cnn) bytes (error word,
+ * 2 x B x Hkv x c_hid x T floats, and on the tensor-core path the hidden
+ * gradient again as two bf16 planes).
  * ------------------------------------------------------------------------- */
 size_t lte_score_backward_workspace_bytes(const lte_dims* d, const lte_cnn* cnn);
 lte_status lte_score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,

@@ -158,6 +158,7 @@ lte_status lte_score_backward(const lte_dims* d, const lte_cnn* cnn, const void*
   if ((st = get_strides(d, kv_strides, d->Hkv, &s)) != LTE_OK) return st;
   return from_cuda(lte::score_backward(d, cnn, k, v, s, n_scored, dr, dk, dv, dw1, db1, dw2, db2,
                                        static_cast<char*>(workspace) + kErrBytes,
+                                       reinterpret_cast<lte::DevError*>(workspace),
                                        as_stream(stream)));
 }
 

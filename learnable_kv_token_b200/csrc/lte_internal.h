@@ -17,16 +17,26 @@ cudaError_t score_linear(const lte_dims* d, const lte_cnn* cnn, const void* k, c
 
 // score_tcgen05.cu
 bool score_tcgen05_supported(const lte_dims* d, const lte_cnn* cnn, Strides4 s);
+// z1 != NULL: write the first layer's pre-activation for tokens [j_begin, j_end)
+// (any j_end <= T) into z1 [B*Hkv][c_hid][T] instead of scores (r, mask unused)
 cudaError_t score_tcgen05(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
                           Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
-                          cudaStream_t stream);
+                          cudaStream_t stream, float* z1 = nullptr);
 
 // score_backward.cu
 size_t score_backward_scratch_bytes(const lte_dims* d, const lte_cnn* cnn);
 cudaError_t score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
                            Strides4 s, int n_scored, const float* dr, float* dk, float* dv,
                            float* dw1, float* db1, float* dw2, float* db2, void* scratch,
-                           cudaStream_t stream);
+                           DevError* err, cudaStream_t stream);
+// score_backward_tc.cu: dw1 on tcgen05 (bf16, head dim 128, c_hid 32, k1 <= 8)
+bool score_backward_tc_supported(const lte_dims* d, const lte_cnn* cnn);
+cudaError_t score_backward_dw1_tc(const lte_dims* d, const lte_cnn* cnn, const void* k,
+                                  const void* v, Strides4 s, const void* dz_planes, float* dw1,
+                                  DevError* err, cudaStream_t stream);
+bool score_backward_dx_tc_supported(const lte_dims* d, const lte_cnn* cnn);
+cudaError_t score_backward_dx_tc(const lte_dims* d, const lte_cnn* cnn, const void* dz_planes,
+                                 float* dk, float* dv, DevError* err, cudaStream_t stream);
 
 // evict_compact.cu
 cudaError_t evict_compact(const lte_dims* d, const float* r, const uint8_t* mask, int n_scored,

@@ -44,6 +44,8 @@ struct Args {
   const float *w1, *b1, *w2, *b2, *dr;
   float *dk, *dv, *dw1, *db1, *dw2, *db2;
   float *z1, *dz1;                  // scratch [B*Hkv][c_hid][T]
+  __nv_bfloat16* dzp;               // dz1 as bf16 hi, lo planes [2][B*Hkv][T][32] for the
+                                    // tensor-core dw1 pass, else NULL (then dw1 pass adds db1)
 };
 
 // x[ch][i] of unit (b, h): k channels first, then v; 0 outside [0, T)
@@ -120,7 +122,9 @@ __global__ void __launch_bounds__(kThreads) cnnb_dz_kernel(const Args a) {
   __shared__ float us[kMaxHid][kW];              // u over [p0 - (k2-1), p0 + 64 + k2 - 1)
   __shared__ float dz2s[kTile + kMaxK];          // dz2 over [p0 - (k2-1-past2), p0 + 64 + past2)
   __shared__ float w2s[kMaxHid * kMaxK];
+  __shared__ float db1s[kMaxHid];
   const int u = blockIdx.y, h = u % a.Hkv, tid = threadIdx.x;
+  if (tid < kMaxHid) db1s[tid] = 0.f;
   const int p0 = blockIdx.x * kTile;
   const int C = a.c_hid, K2 = a.k2, P2 = a.past2, F2 = K2 - 1 - P2;
   const int ulo = p0 - (K2 - 1), uw = kTile + 2 * (K2 - 1);
@@ -158,7 +162,20 @@ __global__ void __launch_bounds__(kThreads) cnnb_dz_kernel(const Args a) {
     for (int kk = 0; kk < K2; ++kk) du = fmaf(w2s[c * K2 + kk], dz2s[i - kk + P2 - jlo], du);
     const long long zi = ((long long)u * C + c) * a.T + i;
     const float z = a.z1[zi], sg = sigm(z);
-    a.dz1[zi] = du * sg * (1.f + z * (1.f - sg));
+    const float dz = du * sg * (1.f + z * (1.f - sg));
+    a.dz1[zi] = dz;
+    if (a.dzp != nullptr) {                          // bf16 hi + lo for the tensor-core dw1 pass
+      const __nv_bfloat16 hi = __float2bfloat16_rn(dz);
+      const long long pi = ((long long)u * a.T + i) * C + c;
+      const long long plane = (long long)a.B * a.Hkv * a.T * C;
+      a.dzp[pi] = hi;
+      a.dzp[plane + pi] = __float2bfloat16_rn(dz - __bfloat162float(hi));
+      atomicAdd_block(&db1s[c], dz);
+    }
+  }
+  if (a.dzp != nullptr) {
+    __syncthreads();
+    if (tid < C) atomicAdd(a.db1 + h * C + tid, db1s[tid]);
   }
   for (int t = tid; t < C * K2; t += kThreads) {
     const int c = t / K2, kk = t % K2;
@@ -294,13 +311,16 @@ __global__ void __launch_bounds__(kThreads) cnnb_dw1_kernel(const Args a) {
 }  // namespace cnnb
 
 size_t score_backward_scratch_bytes(const lte_dims* d, const lte_cnn* cnn) {
-  return 2 * (size_t)d->B * d->Hkv * cnn->c_hid * d->T * sizeof(float);
+  size_t n = 2 * (size_t)d->B * d->Hkv * cnn->c_hid * d->T * sizeof(float);
+  if (score_backward_tc_supported(d, cnn))                 // dz1 planes for the tensor-core dw1
+    n += 2 * (size_t)d->B * d->Hkv * d->T * cnn->c_hid * sizeof(__nv_bfloat16);
+  return n;
 }
 
 cudaError_t score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
                            Strides4 s, int n_scored, const float* dr, float* dk, float* dv,
                            float* dw1, float* db1, float* dw2, float* db2, void* scratch,
-                           cudaStream_t stream) {
+                           DevError* err, cudaStream_t stream) {
   cnnb::Args a{};
   a.B = d->B; a.T = d->T; a.Hkv = d->Hkv; a.D = d->D;
   a.c_hid = cnn->c_hid; a.k1 = cnn->k1; a.past1 = cnn->past1; a.k2 = cnn->k2; a.past2 = cnn->past2;
@@ -310,6 +330,9 @@ cudaError_t score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k,
   a.dk = dk; a.dv = dv; a.dw1 = dw1; a.db1 = db1; a.dw2 = dw2; a.db2 = db2;
   a.z1 = reinterpret_cast<float*>(scratch);
   a.dz1 = a.z1 + (size_t)d->B * d->Hkv * cnn->c_hid * d->T;
+  const bool tc = score_backward_tc_supported(d, cnn);
+  a.dzp = tc ? reinterpret_cast<__nv_bfloat16*>(a.dz1 + (size_t)d->B * d->Hkv * cnn->c_hid * d->T)
+             : nullptr;
   const size_t C = cnn->c_hid;
   cudaError_t e;
   if ((e = cudaMemsetAsync(dw1, 0, d->Hkv * C * 2 * d->D * cnn->k1 * sizeof(float), stream)) != cudaSuccess ||
@@ -327,12 +350,23 @@ cudaError_t score_backward(const lte_dims* d, const lte_cnn* cnn, const void* k,
                                 (int)dw_smem)) != cudaSuccess)
     return e;
   const dim3 grid((d->T + cnnb::kTile - 1) / cnnb::kTile, d->B * d->Hkv);
-  cnnb::cnnb_z1_kernel<<<grid, cnnb::kThreads, ws_smem, stream>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (tc && score_tcgen05_supported(d, cnn, s)) {
+    // the layer-1 recompute on tensor cores: the forward scorer writing z1
+    if ((e = score_tcgen05(d, cnn, k, v, s, 0, d->T, nullptr, nullptr, stream, a.z1)) != cudaSuccess)
+      return e;
+  } else {
+    cnnb::cnnb_z1_kernel<<<grid, cnnb::kThreads, ws_smem, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   cnnb::cnnb_dz_kernel<<<grid, cnnb::kThreads, 0, stream>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  cnnb::cnnb_dx_kernel<<<grid, cnnb::kThreads, ws_smem, stream>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (tc && score_backward_dx_tc_supported(d, cnn)) {
+    if ((e = score_backward_dx_tc(d, cnn, a.dzp, dk, dv, err, stream)) != cudaSuccess) return e;
+  } else {
+    cnnb::cnnb_dx_kernel<<<grid, cnnb::kThreads, ws_smem, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (tc) return score_backward_dw1_tc(d, cnn, k, v, s, a.dzp, dw1, err, stream);
   const int chunks = (d->T + cnnb::kDwChunk - 1) / cnnb::kDwChunk;
   const dim3 gw(d->B * chunks, d->Hkv, (2 * d->D) / cnnb::kChanChunk);
   cnnb::cnnb_dw1_kernel<<<gw, cnnb::kThreads, dw_smem, stream>>>(a);

@@ -82,6 +82,9 @@ struct Params {
   float tau;
   float* r;
   uint8_t* mask;
+  float* z1;      // non-NULL: write the first layer's pre-activation b1 + W1 * x as
+                  // z1[(b * Hkv + h) * c_hid + c][token] (the CNN backward's recompute)
+                  // instead of scores
 };
 
 __host__ __device__ inline uint32_t w_bytes(int D, int N) { return (uint32_t)(2 * D / 64) * N * 128; }
@@ -174,7 +177,7 @@ score_tcgen05_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
   const int P = p.past1 + p.past2;
 
   if ((sbase & 1023u) != 0) {                    // swizzle atoms need 1 KiB alignment
-    if (warp >= 4) write_nan_from(p, h, slot, n_slots, warp & 3, lane);
+    if (warp >= 4 && p.z1 == nullptr) write_nan_from(p, h, slot, n_slots, warp & 3, lane);
     return;
   }
   if (tid == 0) {
@@ -311,6 +314,15 @@ score_tcgen05_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_YE + eg));     // the accumulator may be overwritten
+        if (p.z1 != nullptr) {                          // the pre-activation, this lane's token
+          if (lane >= P && lane < P + p.NW && tok < min(j0 + p.NT, p.j_end)) {
+            float* zo = p.z1 + (long long)(b * p.Hkv + h) * p.c_hid * p.Trow + tok;
+#pragma unroll
+            for (int c = 0; c < kMaxC; ++c)
+              if (c < p.c_hid) zo[(long long)c * p.Trow] = b1s[c] + z[c];
+          }
+          continue;
+        }
         const bool in_seq = tok >= 0 && tok < p.T_avail;
 #pragma unroll
         for (int c = 0; c < kMaxC; c += 4) {
@@ -341,7 +353,7 @@ score_tcgen05_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_cons
           if (p.mask) p.mask[o] = (tok >= p.sink && r >= p.tau) ? 1 : 0;
         }
       }
-      if (!ok) write_nan_from(p, h, t, 2 * n_slots, q, lane);
+      if (!ok && p.z1 == nullptr) write_nan_from(p, h, t, 2 * n_slots, q, lane);
     }
   }
   tc_fence_before();
@@ -377,7 +389,7 @@ bool score_tcgen05_supported(const lte_dims* d, const lte_cnn* cnn, Strides4 s) 
 
 cudaError_t score_tcgen05(const lte_dims* d, const lte_cnn* cnn, const void* k, const void* v,
                           Strides4 s, int j_begin, int j_end, float* r, uint8_t* mask,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, float* z1) {
   using namespace sc5;
   Params p{};
   p.Hkv = d->Hkv; p.D = d->D; p.T_avail = d->T; p.Trow = d->T;
@@ -391,7 +403,7 @@ cudaError_t score_tcgen05(const lte_dims* d, const lte_cnn* cnn, const void* k, 
   p.tiles_per_unit = (j_end - j_begin + p.NT - 1) / p.NT;
   p.n_tiles = d->B * p.tiles_per_unit;
   p.w1 = cnn->w1; p.b1 = cnn->b1; p.w2 = cnn->w2; p.b2 = cnn->b2;
-  p.sink = d->sink; p.tau = d->tau; p.r = r; p.mask = mask;
+  p.sink = d->sink; p.tau = d->tau; p.r = r; p.mask = mask; p.z1 = z1;
   if (p.n_tiles == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   {
