@@ -83,16 +83,47 @@ __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Args a, DevError* err) {
+// Pipelined roles (256 threads, one CTA per SM):
+//   warp 0     TMA copies (one elected lane): Q and dO once, then K and V of key
+//              tile j into ring stage j % 3 (128-byte swizzled 64-column halves;
+//              rows past the tensor read as zero);
+//   warp 1     issues, per tile j: S(j), dP(j) into TMEM buffer j % 2, then
+//              dQ += dS(j-1) K(j-1) once dS(j-1) is in shared memory -- so the
+//              tensor core computes tile j's products while the rows of tile
+//              j - 1 are being formed;
+//   warps 4-11 two threads per query row (warps 4-7 the first 32 keys of a
+//              tile, 8-11 the last 32): P and dS of tile j from TMEM buffer
+//              j % 2 into the shared dS buffer j % 2; at the end, dQ out (64
+//              of the 128 columns each).  Two warps per sub-partition hide
+//              each other's TMEM and special-function latency.
+// TMEM: S[2] 0..127, dP[2] 128..255, dQ 256..383.
+constexpr int kThreadsP = 384;
+constexpr int kStagesP = 3;                             // K/V ring
+constexpr uint32_t kK2 = 65536;                         // stage s: K at + 32 KiB s, V at + 16 KiB
+constexpr uint32_t kDS2 = kK2 + kStagesP * 32768;       // dS buffers: 2 x [128][64] bf16
+constexpr uint32_t kBar2 = kDS2 + 2 * 16384;            // barriers
+constexpr int kSmemP = kBar2 + 256;
+constexpr uint32_t kColSP = 0, kColDPP = 128, kColDQP = 256;
+enum {
+  P_QF = 0, P_KVF = 1, P_KVE = P_KVF + kStagesP, P_SF = P_KVE + kStagesP, P_SE = P_SF + 2,
+  P_DSF = P_SE + 2, P_DSE = P_DSF + 2, P_DQ = P_DSE + 2, kNumBarsP = P_DQ + 1
+};
+static_assert(8 * kNumBarsP + 8 <= 256, "barriers fit");
+
+__global__ void __launch_bounds__(kThreadsP, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+                 const bwd::Args a, DevError* err) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sb = sa(sm);
   if ((sb & 1023u) != 0) {                      // swizzle atoms need 1 KiB alignment
     if (threadIdx.x == 0) record_error(err, LTE_ERR_DEVICE, 403);
     return;
   }
-  const uint32_t bar_s = sb + kBar, bar_q = sb + kBar + 8;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kBar + 16);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kBar + 20);
+  auto bar = [&](int i) { return sb + kBar2 + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kBar2 + 8 * kNumBarsP);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kBar2 + 8 * kNumBarsP + 4);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int G = a.G, TOK = kRowsTc / G;
   const int n_tiles = (a.T + TOK - 1) / TOK;
@@ -104,45 +135,32 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
   const bool lowest = a.death != nullptr;
 
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_q, 1);
+    mbar_init(bar(P_QF), 1);
+    for (int x = 0; x < kStagesP; ++x) {
+      mbar_init(bar(P_KVF + x), 1);
+      mbar_init(bar(P_KVE + x), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(P_SF + x), 1);
+      mbar_init(bar(P_SE + x), 256);
+      mbar_init(bar(P_DSF + x), 256);
+      mbar_init(bar(P_DSE + x), 1);
+    }
+    mbar_init(bar(P_DQ), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      sa(tmem_slot)),
-                 "r"(kTmemCols)
+                 "r"(512)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // Q and dO rows (row rho = token * G + head; rows past T zero)
-  for (int i = tid; i < kRowsTc * 16; i += kThreadsTc) {
-    const int r = i >> 4, c = i & 15;
-    const int tt = t0 + r / G, g = r % G;
-    const bool ok = tt < a.T;
-    const long long off = ok ? (((long long)b * a.T + tt) * a.Hq + h * G + g) * HD + c * 8 : 0;
-    cpa16(sb + kQ + sw(kRowsTc, r, c), a.q + off, ok);
-    cpa16(sb + kDO + sw(kRowsTc, r, c), a.dO + off, ok);
-  }
-  cpa_commit();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-
-  // this thread's row
-  const int tt = t0 + tid / G, gq = tid % G;
-  int lo_r, hi_r;
-  bwd::row_range(a, crow, tt, lo_r, hi_r);
-  if (lowest) lo_r = 0;
-  float lse2 = 0.f, dl = 0.f;
-  if (tt < a.T) {
-    const long long li = ((long long)b * a.Hq + h * G + gq) * a.T + tt;
-    lse2 = a.lse[li] * 1.4426950408889634f;
-    dl = a.delta[li];
-  }
 
   // key ranges of the tile: 0 sink slots, 1 retained slots, 2 window band
   int start[3], count[3];
@@ -161,10 +179,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
   }
   const int n0 = (count[0] + kKeysTc - 1) / kKeysTc, n1 = (count[1] + kKeysTc - 1) / kKeysTc;
   const int total = n0 + n1 + (count[2] + kKeysTc - 1) / kKeysTc;
-
-  const uint32_t id_s = idesc(kRowsTc, kKeysTc, false);     // S, dP: K-major A and B
-  const uint32_t id_q = idesc(kRowsTc, HD, true);           // dQ: K as an N-contiguous B
-  // tile j: range, first key, valid keys
   auto tile_of = [&](int j, int& rg, int& key0, int& nk) {
     int it = j;
     if (it < n0) rg = 0;
@@ -173,92 +187,151 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
     key0 = start[rg] + it * kKeysTc;
     nk = min(kKeysTc, count[rg] - it * kKeysTc);
   };
-  // K (which = 0) or V (which = 1) rows of tile j into their buffer, zero past nk
-  auto load_kv = [&](int j, int which) {
-    int rg, key0, nk;
-    tile_of(j, rg, key0, nk);
-    const __nv_bfloat16* base = which == 0 ? (rg == 2 ? a.k : a.k_col) : (rg == 2 ? a.v : a.v_col);
-    const uint32_t dst = sb + (which == 0 ? kK : kV);
-    for (int i = tid; i < kKeysTc * 16; i += kThreadsTc) {
-      const int r = i >> 4, c = i & 15;
-      const bool v_ok = r < nk;
-      long long e = 0;
-      if (v_ok) {
-        const int key = key0 + r;
-        e = rg == 2 ? (((long long)b * a.T + key) * a.Hkv + h) * HD + c * 8
-                    : (col_base + key) * HD + c * 8;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    bool ok = true;
+    if (elect_one()) {
+      mbar_expect_tx(bar(P_QF), 2 * kRowsTc * HD * 2);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_4d(sb + kQ + hf * (kRowsTc * 128), &tm_q, bar(P_QF), hf * 64, h * G, t0, b);
+        tma_load_4d(sb + kDO + hf * (kRowsTc * 128), &tm_do, bar(P_QF), hf * 64, h * G, t0, b);
       }
-      cpa16(dst + sw(kKeysTc, r, c), base + e, v_ok);
     }
-  };
-  bool ok = true;
-  int issued_q = 0;                                         // dQ products committed
-  if (total > 0) {
-    load_kv(0, 0);
-    load_kv(0, 1);
-  }
-  cpa_commit();
-  for (int j = 0; j < total && ok; ++j) {
-    int rg, key0, nk;
-    tile_of(j, rg, key0, nk);
-    // 1. K and V of tile j have landed (V was fetched while tile j - 1 was
-    //    being processed, K once tile j - 1's dQ product had completed)
-    cpa_wait_all();
-    fence_proxy_async();                                     // generic writes -> tensor core
-    __syncthreads();
-    // 2. S = Q K^T, dP = dO V^T
-    if (tid == 0) {
-      tc_fence_after();
-      const uint64_t dq_ = sdesc(sb + kQ, 16, 1024), ddo = sdesc(sb + kDO, 16, 1024);
-      const uint64_t dk = sdesc(sb + kK, 16, 1024), dv = sdesc(sb + kV, 16, 1024);
-#pragma unroll
-      for (int ks = 0; ks < HD / 16; ++ks) {
-        const uint32_t oa = ((ks >> 2) * (kRowsTc * 128) + (ks & 3) * 32) >> 4;
-        const uint32_t ob = ((ks >> 2) * (kKeysTc * 128) + (ks & 3) * 32) >> 4;
-        mma_f16(tmem + kColS, dq_ + oa, dk + ob, id_s, ks > 0 ? 1u : 0u);
-        mma_f16(tmem + kColDP, ddo + oa, dv + ob, id_s, ks > 0 ? 1u : 0u);
-      }
-      mma_commit(bar_s);
-    }
-    ok = mbar_wait(bar_s, j & 1, abort_flag, err, 401);
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    tc_fence_after();
-    if (j + 1 < total) load_kv(j + 1, 1);                  // V is free once dP is done
-    cpa_commit();
-    // 3. P and dS of this row.  The row's keys in the tile form at most two
-    //    intervals (sink slots, retained slots [lo, hi)) or one (window band)
-    uint64_t bits = 0ull;
-    if (tt < a.T) {
-      if (rg == 2) {
-        bits = span64(tt - a.window + 1 - key0, min(nk, tt - key0 + 1));
-      } else {
-        const int sink_end = min(a.sink, tt - a.window + 1);
-        uint64_t ret = span64(a.sink + lo_r - key0, min(nk, a.sink + hi_r - key0));
-        if (lowest && ret != 0ull) {                   // lifetimes: held at count hi_r
-#pragma unroll 4
-          for (int kk = 0; kk < kKeysTc; ++kk)
-            if (((ret >> kk) & 1ull) && __ldg(a.death + crow + key0 + kk - a.sink) <= hi_r)
-              ret &= ~(1ull << kk);
+    __syncwarp();
+    int issued = 0;
+    for (int j = 0; j < total && ok; ++j) {
+      const int st = j % kStagesP, use = j / kStagesP;
+      if (use >= 1 && !(ok = wwait(bar(P_KVE + st), (use - 1) & 1, abort_flag, err, 404))) break;
+      int rg, key0, nk;
+      tile_of(j, rg, key0, nk);
+      if (elect_one()) {
+        const uint32_t kd = sb + kK2 + st * 32768u, vd = kd + 16384u;
+        mbar_expect_tx(bar(P_KVF + st), 2 * kKeysTc * HD * 2);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (rg == 2) {
+            tma_load_4d(kd + hf * (kKeysTc * 128), &tm_k, bar(P_KVF + st), hf * 64, h, key0, b);
+            tma_load_4d(vd + hf * (kKeysTc * 128), &tm_v, bar(P_KVF + st), hf * 64, h, key0, b);
+          } else {
+            tma_load_3d(kd + hf * (kKeysTc * 128), &tm_kc, bar(P_KVF + st), hf * 64, key0, u);
+            tma_load_3d(vd + hf * (kKeysTc * 128), &tm_vc, bar(P_KVF + st), hf * 64, key0, u);
+          }
         }
-        bits = span64(-key0, min(nk, sink_end - key0)) | ret;
       }
+      __syncwarp();
+      issued = j + 1;
     }
-    // relaxed retention: the column slots' logit offsets (0 on sinks)
-    const float* brow = (a.bias != nullptr && rg != 2) ? a.bias + col_base + key0 : nullptr;
-    {
-      uint32_t rs[32], rp[32];
-      uint32_t pkd[32];
+    // every issued copy has landed before the CTA may exit
+    mbar_drain(bar(P_QF), 0);
+    for (int q = issued - kStagesP > 0 ? issued - kStagesP : 0; q < issued; ++q)
+      mbar_drain(bar(P_KVF + q % kStagesP), (q / kStagesP) & 1);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t id_s = idesc(kRowsTc, kKeysTc, false);     // S, dP: K-major A and B
+    const uint32_t id_q = idesc(kRowsTc, HD, true);           // dQ: K as an N-contiguous B
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QF), 0, abort_flag, err, 405));
+    auto issue_dq = [&](int jj) -> bool {                     // dQ += dS(jj) K(jj)
+      const int x = jj & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(P_DSF + x), (jj >> 1) & 1, abort_flag, err, 406)))
+        return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dds = sdesc(sb + kDS2 + x * 16384u, 16, 1024);
+        const uint64_t dkb = sdesc(sb + kK2 + (jj % kStagesP) * 32768u, kKeysTc * 128, 1024);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        tmem_ld32(lane_addr + kColS + half * 32, rs);
-        tmem_ld32(lane_addr + kColDP + half * 32, rp);
+        for (int ks = 0; ks < kKeysTc / 16; ++ks)
+          mma_f16(tmem + kColDQP, dds + ((ks * 32) >> 4), dkb + ((ks * 2048) >> 4), id_q,
+                  (jj > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(bar(P_DSE + x));                           // dS buffer x is free
+        mma_commit(bar(P_KVE + jj % kStagesP));               // K, V of tile jj are free
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int j = 0; j < total && ok; ++j) {
+      const int x = j & 1, use = j >> 1, st = j % kStagesP;
+      ok = mbar_wait(bar(P_KVF + st), (j / kStagesP) & 1, abort_flag, err, 407);
+      if (ok && use >= 1) ok = mbar_wait(bar(P_SE + x), (use - 1) & 1, abort_flag, err, 408);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dq_ = sdesc(sb + kQ, 16, 1024), ddo = sdesc(sb + kDO, 16, 1024);
+        const uint64_t dk = sdesc(sb + kK2 + st * 32768u, 16, 1024);
+        const uint64_t dv = sdesc(sb + kK2 + st * 32768u + 16384u, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t oa = ((ks >> 2) * (kRowsTc * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t ob = ((ks >> 2) * (kKeysTc * 128) + (ks & 3) * 32) >> 4;
+          mma_f16(tmem + kColSP + x * 64, dq_ + oa, dk + ob, id_s, ks > 0 ? 1u : 0u);
+          mma_f16(tmem + kColDPP + x * 64, ddo + oa, dv + ob, id_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(P_SF + x));
+      }
+      __syncwarp();
+      if (j >= 1 && !(ok = issue_dq(j - 1))) break;
+    }
+    if (ok && total > 0) ok = issue_dq(total - 1);
+    if (elect_one()) mma_commit(bar(P_DQ));                   // every product above has completed
+    __syncwarp();
+    mbar_drain(bar(P_DQ), 0);
+  } else {
+    // ---------------------------------------------------------------- rows (warps 4-11)
+    if (warp < 4) {
+      // warps 2-3 have no role
+    } else {
+    const int quad = warp & 3, kh = (warp - 4) >> 2;   // TMEM lane quadrant, key half of a tile
+    const int row = quad * 32 + (tid & 31);
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int tt = t0 + row / G, gq = row % G;
+    int lo_r, hi_r;
+    bwd::row_range(a, crow, tt, lo_r, hi_r);
+    if (lowest) lo_r = 0;
+    float lse2 = 0.f, dl = 0.f;
+    if (tt < a.T) {
+      const long long li = ((long long)b * a.Hq + h * G + gq) * a.T + tt;
+      lse2 = a.lse[li] * 1.4426950408889634f;
+      dl = a.delta[li];
+    }
+    bool ok = true;
+    for (int j = 0; j < total && ok; ++j) {
+      const int x = j & 1, use = j >> 1;
+      int rg, key0, nk;
+      tile_of(j, rg, key0, nk);
+      // this row's keys in the tile: at most two intervals (sink slots, retained
+      // slots [lo, hi)) or one (window band); this thread takes keys 32 kh ..
+      uint64_t bits = 0ull;
+      if (tt < a.T) {
+        if (rg == 2) {
+          bits = span64(tt - a.window + 1 - key0, min(nk, tt - key0 + 1));
+        } else {
+          const int sink_end = min(a.sink, tt - a.window + 1);
+          uint64_t ret = span64(a.sink + lo_r - key0, min(nk, a.sink + hi_r - key0));
+          if (lowest && ret != 0ull) {                 // lifetimes: held at count hi_r
+#pragma unroll 4
+            for (int kk = 32 * kh; kk < 32 * kh + 32; ++kk)
+              if (((ret >> kk) & 1ull) && __ldg(a.death + crow + key0 + kk - a.sink) <= hi_r)
+                ret &= ~(1ull << kk);
+          }
+          bits = span64(-key0, min(nk, sink_end - key0)) | ret;
+        }
+      }
+      const uint32_t hb = (uint32_t)(bits >> (32 * kh));
+      const float* brow = (a.bias != nullptr && rg != 2) ? a.bias + col_base + key0 + 32 * kh : nullptr;
+      ok = mbar_wait(bar(P_SF + x), use & 1, abort_flag, err, 409);
+      if (ok && use >= 1) ok = mbar_wait(bar(P_DSE + x), (use - 1) & 1, abort_flag, err, 410);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      uint32_t pkd[16];
+      {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(lane_addr + kColSP + x * 64 + 32 * kh, rs);
+        tmem_ld32(lane_addr + kColDPP + x * 64 + 32 * kh, rp);
         tmem_wait_ld();
-        const uint32_t hb = (uint32_t)(bits >> (half * 32));
         if (brow != nullptr) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if ((hb >> c) & 1u)
-              rs[c] = __float_as_uint(__uint_as_float(rs[c]) + __ldg(brow + half * 32 + c));
+            if ((hb >> c) & 1u) rs[c] = __float_as_uint(__uint_as_float(rs[c]) + __ldg(brow + c));
         }
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -270,70 +343,53 @@ __global__ void __launch_bounds__(kThreadsTc, 2) bwd_dq_tc_kernel(const bwd::Arg
                                 : 0.f;
             ds2[e] = p * (__uint_as_float(rp[c + e]) - dl);
           }
-          pkd[half * 16 + (c >> 1)] = pk2(ds2[0], ds2[1]);
+          pkd[c >> 1] = pk2(ds2[0], ds2[1]);
         }
       }
-      // the dS row (64 keys = 128 bytes) into the swizzled K-major A operand
-      uint8_t* row = sm + kDS + tid * 128;
+      tc_fence_before();
+      mbar_arrive(bar(P_SE + x));                      // this thread's part of S, dP x is read
+      // 64 bytes of the dS row (keys 32 kh ..) into the swizzled K-major A operand
+      uint8_t* drow = sm + kDS2 + x * 16384u + row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(row + ((c ^ (tid & 7)) << 4)) =
+      for (int c = 0; c < 4; ++c) {
+        const int ch = 4 * kh + c;
+        *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
             make_uint4(pkd[4 * c], pkd[4 * c + 1], pkd[4 * c + 2], pkd[4 * c + 3]);
+      }
+      fence_proxy_async();
+      mbar_arrive(bar(P_DSF + x));
     }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    // 4. dQ += dS K
-    if (tid == 0) {
+    // dQ row: scale, fp32 out, columns 64 kh .. (every lane loads: tcgen05.ld is warp-collective)
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(P_DQ), 0, abort_flag, err, 411));
+    if (ok) {
       tc_fence_after();
-      const uint64_t dds = sdesc(sb + kDS, 16, 1024);
-      const uint64_t dkb = sdesc(sb + kK, kKeysTc * 128, 1024);   // K: N-contiguous, halves 8 KiB apart
-#pragma unroll
-      for (int ks = 0; ks < kKeysTc / 16; ++ks)
-        mma_f16(tmem + kColDQ, dds + ((ks * 32) >> 4), dkb + ((ks * 2048) >> 4), id_q,
-                (j > 0 || ks > 0) ? 1u : 0u);
-      mma_commit(bar_q);
-    }
-    ++issued_q;
-    ok = mbar_wait(bar_q, j & 1, abort_flag, err, 402);
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    tc_fence_after();
-    if (j + 1 < total) load_kv(j + 1, 0);                  // K is free once dQ is done
-    cpa_commit();
-  }
-  cpa_wait_all();
-  if (ok) {
-    // dQ row: scale, fp32 out (every lane loads: tcgen05.ld is warp-collective)
-    float* out = a.dq + (((long long)b * a.T + min(tt, a.T - 1)) * a.Hq + h * G + gq) * HD;
+      float* out = a.dq + (((long long)b * a.T + min(tt, a.T - 1)) * a.Hq + h * G + gq) * HD;
 #pragma unroll 1
-    for (int c0 = 0; c0 < HD; c0 += 32) {
-      uint32_t r[32];
-      if (total > 0) {
-        tmem_ld32(lane_addr + kColDQ + c0, r);
-        tmem_wait_ld();
-      } else {
+      for (int c0 = 64 * kh; c0 < 64 * kh + 64; c0 += 32) {
+        uint32_t r[32];
+        if (total > 0) {
+          tmem_ld32(lane_addr + kColDQP + c0, r);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = 0u;
-      }
-      if (tt < a.T) {
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (tt < a.T) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(out + c0 + e) =
-              make_float4(__uint_as_float(r[e]) * a.scale, __uint_as_float(r[e + 1]) * a.scale,
-                          __uint_as_float(r[e + 2]) * a.scale, __uint_as_float(r[e + 3]) * a.scale);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(out + c0 + e) =
+                make_float4(__uint_as_float(r[e]) * a.scale, __uint_as_float(r[e + 1]) * a.scale,
+                            __uint_as_float(r[e + 2]) * a.scale, __uint_as_float(r[e + 3]) * a.scale);
+        }
       }
     }
-  } else if (tid == 0) {
-    // drain the products this CTA issued before its TMEM is freed
-    mbar_drain(bar_s, 0);
-    mbar_drain(bar_s, 1);
-    if (issued_q > 0) mbar_drain(bar_q, (issued_q - 1) & 1);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
                  : "memory");
 }
 
@@ -710,12 +766,38 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
 
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
   using namespace bwdtc;
-  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e != cudaSuccess) return e;
   const int TOK = kRowsTc / a.G;
+  // tensor maps (contiguous [B,T,H,128] bf16; 128-byte swizzle, 64-column boxes)
+  CUtensorMap mq, mdo, mk, mv, mkc, mvc;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
+    const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hq * HD * 2, (cuuint64_t)a.T * a.Hq * HD * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)a.G, (cuuint32_t)TOK, 1};
+    if (!encode(&mq, a.q, 4, dims, st, box) || !encode(&mdo, a.dO, 4, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hkv, (cuuint64_t)a.T, (cuuint64_t)B};
+    const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hkv * HD * 2,
+                              (cuuint64_t)a.T * a.Hkv * HD * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kKeysTc, 1};
+    if (!encode(&mk, a.k, 4, dims, st, box) || !encode(&mv, a.v, 4, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t rows = (cuuint64_t)a.sink + a.T;
+    const cuuint64_t dims[3] = {(cuuint64_t)HD, rows, (cuuint64_t)B * a.Hkv};
+    const cuuint64_t st[2] = {(cuuint64_t)HD * 2, rows * HD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kKeysTc, 1};
+    if (!encode(&mkc, a.k_col, 3, dims, st, box) || !encode(&mvc, a.v_col, 3, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemP);
+  if (e != cudaSuccess) return e;
   const int n_tiles = (a.T + TOK - 1) / TOK;
-  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsTc, kSmemBytes, stream>>>(a, err);
+  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsP, kSmemP, stream>>>(mq, mdo, mk, mv, mkc, mvc,
+                                                                          a, err);
   return cudaGetLastError();
 }
 

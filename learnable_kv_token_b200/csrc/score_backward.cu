@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kThreads) cnnb_dz_kernel(const Args a) {
   __shared__ float dz2s[kTile + kMaxK];          // dz2 over [p0 - (k2-1-past2), p0 + 64 + past2)
   __shared__ float w2s[kMaxHid * kMaxK];
   __shared__ float db1s[kMaxHid];
+  __shared__ float dzt[kTile][33];               // dz1 of the tile, [position][c] (32 channels)
   const int u = blockIdx.y, h = u % a.Hkv, tid = threadIdx.x;
   if (tid < kMaxHid) db1s[tid] = 0.f;
   const int p0 = blockIdx.x * kTile;
@@ -155,27 +156,52 @@ __global__ void __launch_bounds__(kThreads) cnnb_dz_kernel(const Args a) {
   }
   __syncthreads();
   // du, dz1 of the tile; dw2 / db2 partial sums over the tile's own j
-  for (int t = tid; t < C * kTile; t += kThreads) {
+  for (int t = tid; t < C * kTile; t += kThreads) {   // whole warps (C * kTile % 256 == 0)
     const int c = t / kTile, i = p0 + t % kTile;
-    if (i >= a.T) continue;
-    float du = 0.f;
-    for (int kk = 0; kk < K2; ++kk) du = fmaf(w2s[c * K2 + kk], dz2s[i - kk + P2 - jlo], du);
-    const long long zi = ((long long)u * C + c) * a.T + i;
-    const float z = a.z1[zi], sg = sigm(z);
-    const float dz = du * sg * (1.f + z * (1.f - sg));
-    a.dz1[zi] = dz;
-    if (a.dzp != nullptr) {                          // bf16 hi + lo for the tensor-core dw1 pass
-      const __nv_bfloat16 hi = __float2bfloat16_rn(dz);
-      const long long pi = ((long long)u * a.T + i) * C + c;
-      const long long plane = (long long)a.B * a.Hkv * a.T * C;
-      a.dzp[pi] = hi;
-      a.dzp[plane + pi] = __float2bfloat16_rn(dz - __bfloat162float(hi));
-      atomicAdd_block(&db1s[c], dz);
+    float dz = 0.f;                                    // 0 past the sequence
+    if (i < a.T) {
+      float du = 0.f;
+      for (int kk = 0; kk < K2; ++kk) du = fmaf(w2s[c * K2 + kk], dz2s[i - kk + P2 - jlo], du);
+      const long long zi = ((long long)u * C + c) * a.T + i;
+      const float z = a.z1[zi], sg = sigm(z);
+      dz = du * sg * (1.f + z * (1.f - sg));
+      a.dz1[zi] = dz;
+    }
+    if (a.dzp != nullptr) {
+      // the 32 lanes of a warp share c (kTile = 64): one shared atomic per warp for db1
+      float sum = dz;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if ((tid & 31) == 0) atomicAdd_block(&db1s[c], sum);
+      dzt[t % kTile][c] = dz;
     }
   }
   if (a.dzp != nullptr) {
+    // dz1 as bf16 hi and lo planes [unit][T][32], 16-byte chunks of 64-byte rows
+    // (the tensor-core dx and dw1 passes read them)
     __syncthreads();
     if (tid < C) atomicAdd(a.db1 + h * C + tid, db1s[tid]);
+    const long long plane = (long long)a.B * a.Hkv * a.T * C;
+    for (int e = tid; e < 2 * kTile * 4; e += kThreads) {
+      const int g = e & 3, r = (e >> 2) % kTile, pl = e / (kTile * 4);
+      const int i = p0 + r;
+      if (i >= a.T) continue;
+      uint32_t w[4];
+#pragma unroll
+      for (int f = 0; f < 4; ++f) {
+        float v2[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float x = dzt[r][g * 8 + 2 * f + q];
+          const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+          v2[q] = pl == 0 ? __bfloat162float(hi) : x - __bfloat162float(hi);
+        }
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v2[0], v2[1]);
+        w[f] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(a.dzp + pl * plane + ((long long)u * a.T + i) * C + g * 8) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
   for (int t = tid; t < C * K2; t += kThreads) {
     const int c = t / K2, kk = t % K2;
