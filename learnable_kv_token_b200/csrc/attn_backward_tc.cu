@@ -394,49 +394,57 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ---------------------------------------------------------------- dK, dV
-// One CTA of 256 threads per 128-key tile (keys of k for the window part,
-// kColumn = false; slots of the column segment, kColumn = true, for this
-// CTA's share of the attending rows).  Keys are the MMA rows: per 128-row
-// tile of attending query rows,
-//   S^T = K Q^T, dP^T = V dO^T            (M128 N128 K128)
-//   P^T, dS^T = P^T (dP^T - D)             (thread pair per key row, 64 rows each)
-//   dV += P^T dO, dK += dS^T Q             (M128 N128 K128; dO, Q as N-contiguous B)
-// with Q and dO of the next row tile loading (cp.async, double-buffered)
-// while the current one is processed.  P^T and dS^T are written over S^T and
-// dP^T in TMEM and read from there as A operands; the four accumulators fill
-// the 512 TMEM columns.
+// One CTA per 128-key tile (keys of k for the window part, kColumn = false;
+// slots of the column segment, kColumn = true, for this CTA's share of the
+// attending rows).  Keys are the MMA rows; the attending query rows come in
+// tiles of 64 (64/G tokens x the G heads), and per row tile i:
+//   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM buffer i % 2
+//   P^T, dS^T = P^T (dP^T - D)         (two threads per key row, 32 rows each)
+//   dV += P^T dO, dK += dS^T Q         (M128 N128 K64; P^T, dS^T read from TMEM)
+// Roles (384 threads, one CTA per SM):
+//   warp 0     TMA producer (one elected lane): K and V once; per row tile, Q
+//              and dO into a 3-stage ring, the rows' lse, D, token and retained
+//              range written by the warp's lanes into the stage;
+//   warp 1     MMA issuer: S^T(i), dP^T(i), then dV and dK of tile i - 1 once
+//              its P^T and dS^T are in TMEM -- the tensor core computes tile i
+//              while the rows of tile i - 1 are formed;
+//   warps 4-11 two threads per key row (warps 4-7 rows 0-31 of a tile, 8-11
+//              rows 32-63): P^T and dS^T, written as bf16 over their own
+//              columns of S^T and dP^T; at the end, dK and dV out.
+// TMEM: S^T[2] 0..127, dP^T[2] 128..255, dV 256..383, dK 384..511.
 constexpr int kKeysKV = 128;
-constexpr int kRowsKV = 128;
-constexpr int kThreadsKV = 256;
-constexpr int kSplitRowsKV = 16;                  // row tiles per CTA of the column pass
-constexpr uint32_t kvK = 0;                       // [128][128]: halves of 16 KiB
-constexpr uint32_t kvV = 32768;
-constexpr uint32_t kvQD = 65536;                  // [2 stages][Q, dO][128][128]: halves of 16 KiB
-constexpr uint32_t kvQBytes = kRowsKV * 128 * 2;  // one Q (or dO) tile
-constexpr uint32_t kvStage = 2 * kvQBytes;        // one stage: Q then dO
-constexpr uint32_t kvMeta = kvQD + 2 * kvStage;   // [2 stages][128] x {lse2, D, t, lo, hi}
-constexpr uint32_t kvBar = kvMeta + 2 * 5 * kRowsKV * 4;   // bar_s, bar_kv, abort, TMEM slot, range
-constexpr int kvSmemBytes = kvBar + 64;
-constexpr int kvTmemCols = 512;
-// S^T 0..127 (P^T over its first 64 as bf16 pairs), dP^T 128..255 (dS^T over its
-// first 64), dV 256..383, dK 384..511
-constexpr uint32_t kvColS = 0, kvColDP = 128, kvColDV = 256, kvColDK = 384;
+constexpr int kRowsK2 = 64;                       // attending query rows per tile
+constexpr int kStagesK2 = 3;
+constexpr int kThreadsK2 = 384;
+constexpr int kSplitRowsK2 = 32;                  // row tiles per CTA of the column pass
+constexpr uint32_t k2K = 0, k2V = 32768;          // [128][128] bf16: halves of 16 KiB
+constexpr uint32_t k2QD = 65536;                  // stage s: Q at + 32 KiB s, dO at + 16 KiB
+constexpr uint32_t k2Meta = k2QD + kStagesK2 * 32768;            // stage s: [5][64] words
+constexpr uint32_t k2Bar = k2Meta + kStagesK2 * 5 * kRowsK2 * 4;
+constexpr int k2Smem = k2Bar + 256;
+enum {
+  K2_KVF = 0, K2_F = 1, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_PF = K2_SF + 2,
+  K2_DONE = K2_PF + 2, kNumBarsK2 = K2_DONE + 1
+};
+static_assert(8 * kNumBarsK2 + 16 <= 256, "barriers, flags and the row range fit");
 
 template <bool kColumn>
-__global__ void __launch_bounds__(kThreadsKV, 1)
-bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
+__global__ void __launch_bounds__(kThreadsK2, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const bwd::Args a, int n_split, DevError* err) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sb = sa(sm);
   if ((sb & 1023u) != 0) {
     if (threadIdx.x == 0) record_error(err, LTE_ERR_DEVICE, 413);
     return;
   }
-  const uint32_t bar_s = sb + kvBar, bar_kv = sb + kvBar + 8;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kvBar + 16);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kvBar + 20);
-  int* range_sh = reinterpret_cast<int*>(sm + kvBar + 24);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int G = a.G, TOK = kRowsKV / G;
+  auto bar = [&](int i) { return sb + k2Bar + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + k2Bar + 8 * kNumBarsK2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + k2Bar + 8 * kNumBarsK2 + 4);
+  int* range_sh = reinterpret_cast<int*>(sm + k2Bar + 8 * kNumBarsK2 + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.G, TOK = kRowsK2 / G;
   const int h = blockIdx.y, b = blockIdx.z, u = b * a.Hkv + h;
   const long long crow = (long long)u * a.T;
   const long long col_base = (long long)u * (a.sink + a.T);
@@ -447,7 +455,7 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   const int nk = kColumn ? min(kKeysKV, a.sink + __ldg(a.nret + u) - k0) : min(kKeysKV, a.T - k0);
   if (nk <= 0) return;
 
-  // token range of the attending rows
+  // row tiles that attend some key of this tile (this CTA's share of them)
   if (tid == 0) {
     int lo_t, hi_t;
     bwd::attending_tokens(a, crow, kColumn, k0, nk, lo_t, hi_t);
@@ -455,8 +463,8 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
     if (lo_t > hi_t) rt0 = 1, rt1 = 0;
     if constexpr (kColumn) {
       if (rt0 <= rt1) {
-        const int first = rt0 + split * kSplitRowsKV;
-        rt1 = min(rt1, first + kSplitRowsKV - 1);
+        const int first = rt0 + split * kSplitRowsK2;
+        rt1 = min(rt1, first + kSplitRowsK2 - 1);
         rt0 = first;
       }
     }
@@ -468,144 +476,166 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
   if (n_rt <= 0) return;                               // nothing attends (uniform)
 
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_kv, 1);
+    mbar_init(bar(K2_KVF), 1);
+    for (int st = 0; st < kStagesK2; ++st) {
+      mbar_init(bar(K2_F + st), 1);
+      mbar_init(bar(K2_E + st), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(K2_SF + x), 1);
+      mbar_init(bar(K2_PF + x), 256);
+    }
+    mbar_init(bar(K2_DONE), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      sa(tmem_slot)),
-                 "r"(kvTmemCols)
+                 "r"(512)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // K, V of the tile (resident; rows past nk zero)
-  for (int i = tid; i < kKeysKV * 16; i += kThreadsKV) {
-    const int r = i >> 4, c = i & 15;
-    const bool ok = r < nk;
-    long long e = 0;
-    if (ok) {
-      if constexpr (kColumn) e = (col_base + k0 + r) * HD + c * 8;
-      else e = (((long long)b * a.T + k0 + r) * a.Hkv + h) * HD + c * 8;
-    }
-    cpa16(sb + kvK + sw(kKeysKV, r, c), (kColumn ? a.k_col : a.k) + e, ok);
-    cpa16(sb + kvV + sw(kKeysKV, r, c), (kColumn ? a.v_col : a.v) + e, ok);
-  }
-  // Q, dO of row tile `it` into stage it & 1 (cp.async), and its row data:
-  // issue_rows starts the loads of lse, D and the retained count into
-  // registers (threads < 64, one row each); put_rows, called after other
-  // work, stores them, so that their latency is off the critical path
-  float m_l2 = 0.f, m_dd = 0.f;
-  int m_cnt = 0;
-  auto issue_rows = [&](int it) {
-    const int st = it & 1, t0 = (rt0 + it) * TOK;
-    const uint32_t qs = sb + kvQD + st * kvStage;
-    for (int i = tid; i < kRowsKV * 16; i += kThreadsKV) {
-      const int r = i >> 4, c = i & 15;
-      const int tt = t0 + r / G, g = r % G;
-      const bool ok = tt < a.T;
-      const long long off = ok ? (((long long)b * a.T + tt) * a.Hq + h * G + g) * HD + c * 8 : 0;
-      cpa16(qs + sw(kRowsKV, r, c), a.q + off, ok);
-      cpa16(qs + kvQBytes + sw(kRowsKV, r, c), a.dO + off, ok);
-    }
-    if (tid < kRowsKV) {
-      const int r = tid, tt = t0 + r / G, g = r % G;
-      m_l2 = 0.f; m_dd = 0.f; m_cnt = 0;
-      if (tt < a.T) {
-        const long long li = ((long long)b * a.Hq + h * G + g) * a.T + tt;
-        m_l2 = __ldg(a.lse + li);
-        m_dd = __ldg(a.delta + li);
-        if (tt >= a.window) m_cnt = __ldg(a.cnt + crow + tt - a.window);
-      }
-    }
-  };
-  auto put_rows = [&](int it) {
-    if (tid < kRowsKV) {
-      const int st = it & 1, r = tid, tt = (rt0 + it) * TOK + r / G;
-      float* mf = reinterpret_cast<float*>(sm + kvMeta) + st * 5 * kRowsKV;
-      int* mi = reinterpret_cast<int*>(mf);
-      const int hi = (tt < a.T && tt >= a.window) ? held_retained(m_cnt, a.cap, a.cap_policy) : 0;
-      const int lo = (!lowest && a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
-      mf[r] = m_l2 * 1.4426950408889634f;
-      mf[kRowsKV + r] = m_dd;
-      mi[2 * kRowsKV + r] = tt;
-      mi[3 * kRowsKV + r] = lo;
-      mi[4 * kRowsKV + r] = hi;
-    }
-  };
-  issue_rows(0);
-  put_rows(0);
-  cpa_commit();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int key_row = tid & 127, half = tid >> 7;       // this thread: key row, column half
-  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-  // this key's identity for the masks
-  const int kpos = k0 + key_row;                         // position (window) or slot (column)
-  int kdeath = 0;
-  if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
-  // relaxed retention: log2 of this slot's weight r (0 for sinks and window keys),
-  // and the partial sum of dS over the rows this thread sees, for dL/dr
-  float bk2 = 0.f, dr_acc = 0.f;
-  if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
 
-  cpa_wait_all();
-  __syncthreads();
-
-  const uint32_t id_s = idesc(kKeysKV, kRowsKV, false);
-  const uint32_t id_o = idesc(kKeysKV, HD, true);
-  bool ok = true;
-  int kv_issued = 0;
-  for (int it = 0; it < n_rt && ok; ++it) {
-    const int st = it & 1;
-    const uint32_t qs = sb + kvQD + st * kvStage, ds_ = qs + kvQBytes;
-    // this stage's rows have landed
-    cpa_wait_all();
-    fence_proxy_async();
-    __syncthreads();
-    // S^T = K Q^T, dP^T = V dO^T (K, V from TMEM).  They overwrite P^T, dS^T of
-    // the previous tile, whose products were issued earlier: the tensor pipe
-    // runs them in issue order
-    if (tid == 0) {
-      tc_fence_after();
-      const uint64_t dk = sdesc(sb + kvK, 16, 1024), dv = sdesc(sb + kvV, 16, 1024);
-      const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(ds_, 16, 1024);
-#pragma unroll
-      for (int ks = 0; ks < HD / 16; ++ks) {
-        const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
-        const uint32_t ob = ((ks >> 2) * (kRowsKV * 128) + (ks & 3) * 32) >> 4;
-        mma_f16(tmem + kvColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
-        mma_f16(tmem + kvColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    bool ok = true;
+    if (elect_one()) {
+      mbar_expect_tx(bar(K2_KVF), 2 * kKeysKV * HD * 2);
+      for (int hf = 0; hf < 2; ++hf) {
+        if constexpr (kColumn) {
+          tma_load_3d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, k0, u);
+          tma_load_3d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, k0, u);
+        } else {
+          tma_load_4d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, h, k0, b);
+          tma_load_4d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, h, k0, b);
+        }
       }
-      mma_commit(bar_s);
     }
-    // the previous tile's dV, dK products are done: its Q / dO stage is free
-    if (it > 0) {
-      ok = mbar_wait(bar_kv, (it - 1) & 1, abort_flag, err, 411);
-      if (!__syncthreads_and(ok)) { ok = false; break; }
+    __syncwarp();
+    int issued = 0;
+    for (int i = 0; i < n_rt && ok; ++i) {
+      const int st = i % kStagesK2, use = i / kStagesK2;
+      if (use >= 1 && !(ok = wwait(bar(K2_E + st), (use - 1) & 1, abort_flag, err, 414))) break;
+      // the rows' data: lse (log2), D, token, retained range [lo, hi)
+      const int t0r = (rt0 + i) * TOK;
+      float* mf = reinterpret_cast<float*>(sm + k2Meta) + st * 5 * kRowsK2;
+      int* mi = reinterpret_cast<int*>(mf);
+      for (int r = lane; r < kRowsK2; r += 32) {
+        const int tt = t0r + r / G, g = r % G;
+        float l2 = 0.f, dd = 0.f;
+        int cv = 0;
+        if (tt < a.T) {
+          const long long li = ((long long)b * a.Hq + h * G + g) * a.T + tt;
+          l2 = __ldg(a.lse + li) * 1.4426950408889634f;
+          dd = __ldg(a.delta + li);
+          if (tt >= a.window) cv = __ldg(a.cnt + crow + tt - a.window);
+        }
+        const int hi = (tt < a.T && tt >= a.window) ? held_retained(cv, a.cap, a.cap_policy) : 0;
+        const int lo = (!lowest && a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
+        mf[r] = l2;
+        mf[kRowsK2 + r] = dd;
+        mi[2 * kRowsK2 + r] = tt;
+        mi[3 * kRowsK2 + r] = lo;
+        mi[4 * kRowsK2 + r] = hi;
+      }
+      __syncwarp();
+      if (elect_one()) {
+        const uint32_t qs = sb + k2QD + st * 32768u;
+        mbar_expect_tx(bar(K2_F + st), 2 * kRowsK2 * HD * 2);
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_4d(qs + hf * 8192u, &tm_q, bar(K2_F + st), hf * 64, h * G, t0r, b);
+          tma_load_4d(qs + 16384u + hf * 8192u, &tm_do, bar(K2_F + st), hf * 64, h * G, t0r, b);
+        }
+      }
+      __syncwarp();
+      issued = i + 1;
     }
-    if (it + 1 < n_rt) issue_rows(it + 1);
-    cpa_commit();
-    ok = mbar_wait(bar_s, it & 1, abort_flag, err, 412);
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    tc_fence_after();
-    // P^T and dS^T: 32 row-columns of this key row
-    {
-      uint32_t rs[64], rp[64];
-      tmem_ld32(lane_addr + kvColS + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&rs[0]));
-      tmem_ld32(lane_addr + kvColS + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rs[32]));
-      tmem_ld32(lane_addr + kvColDP + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&rp[0]));
-      tmem_ld32(lane_addr + kvColDP + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rp[32]));
-      tmem_wait_ld();
-      const float* mf = reinterpret_cast<const float*>(sm + kvMeta) + st * 5 * kRowsKV;
+    // every issued copy has landed before the CTA may exit
+    mbar_drain(bar(K2_KVF), 0);
+    for (int q = issued - kStagesK2 > 0 ? issued - kStagesK2 : 0; q < issued; ++q)
+      mbar_drain(bar(K2_F + q % kStagesK2), (q / kStagesK2) & 1);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t id_s = idesc(kKeysKV, kRowsK2, false);    // S^T, dP^T: K-major A and B
+    const uint32_t id_o = idesc(kKeysKV, HD, true);          // dV, dK: dO, Q as N-contiguous B
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_KVF), 0, abort_flag, err, 415));
+    auto issue_dvdk = [&](int i) -> bool {                   // dV, dK of row tile i
+      const int x = i & 1, st = i % kStagesK2;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(K2_PF + x), (i >> 1) & 1, abort_flag, err, 416)))
+        return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t qs = sb + k2QD + st * 32768u;
+        const uint64_t qb = sdesc(qs, kRowsK2 * 128, 1024), dob = sdesc(qs + 16384u, kRowsK2 * 128, 1024);
+#pragma unroll
+        for (int ks = 0; ks < kRowsK2 / 16; ++ks) {
+          // rows 16 ks .. of P^T, dS^T: the 32 rows of a thread pair's half sit in
+          // columns 32 half .. + 15 of the buffer
+          const uint32_t pc = (uint32_t)(x * 64 + 32 * (ks >> 1) + 8 * (ks & 1));
+          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
+          mma_f16_ts(tmem + 256, tmem + pc, dob + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + 384, tmem + 128 + pc, qb + ((ks * 2048) >> 4), id_o, acc);
+        }
+        mma_commit(bar(K2_E + st));                          // the row tile's stage is free
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int i = 0; i < n_rt && ok; ++i) {
+      const int x = i & 1, st = i % kStagesK2;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_F + st), (i / kStagesK2) & 1, abort_flag, err, 417));
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t qs = sb + k2QD + st * 32768u;
+        const uint64_t dk = sdesc(sb + k2K, 16, 1024), dv = sdesc(sb + k2V, 16, 1024);
+        const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
+          mma_f16(tmem + x * 64, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
+          mma_f16(tmem + 128 + x * 64, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(K2_SF + x));
+      }
+      __syncwarp();
+      if (i >= 1 && !(ok = issue_dvdk(i - 1))) break;
+    }
+    if (ok) ok = issue_dvdk(n_rt - 1);
+    if (elect_one()) mma_commit(bar(K2_DONE));             // every product above has completed
+    __syncwarp();
+    mbar_drain(bar(K2_DONE), 0);
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- key rows (warps 4-11)
+    const int quad = warp & 3, half = (warp - 4) >> 2;     // TMEM lane quadrant, row half
+    const int key_row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int kpos = k0 + key_row;                         // position (window) or slot (column)
+    int kdeath = 0;
+    if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
+    // relaxed retention: log2 of this slot's weight r (0 for sinks and window keys),
+    // and the partial sum of dS over the rows this thread sees, for dL/dr
+    float bk2 = 0.f, dr_acc = 0.f;
+    if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
+    bool ok = true;
+    for (int i = 0; i < n_rt && ok; ++i) {
+      const int x = i & 1, st = i % kStagesK2;
+      ok = mbar_wait(bar(K2_F + st), (i / kStagesK2) & 1, abort_flag, err, 418);   // row data
+      if (ok) ok = mbar_wait(bar(K2_SF + x), (i >> 1) & 1, abort_flag, err, 419);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float* mf = reinterpret_cast<const float*>(sm + k2Meta) + st * 5 * kRowsK2;
       const int* mi = reinterpret_cast<const int*>(mf);
-      // the rows of this tile that attend to this key: one interval of the
+      // the rows of this tile that attend this key: one interval [r_a, r_b) of the
       // (token-major) rows; tokens past T never attend
-      const int t0r = (rt0 + it) * TOK;
-      const int r_end = min(kRowsKV, (a.T - t0r) * G);
+      const int t0r = (rt0 + i) * TOK;
+      const int r_end = min(kRowsK2, (a.T - t0r) * G);
       int r_a = 0, r_b = 0;
       if (key_row < nk) {
         if constexpr (!kColumn) {
@@ -613,126 +643,102 @@ bwd_dkdv_tc_kernel(const bwd::Args a, int n_split, DevError* err) {
           r_b = (kpos + a.window - t0r) * G;
         } else if (kpos < a.sink) {
           r_a = (kpos + a.window - t0r) * G;               // tokens >= kpos + w
-          r_b = kRowsKV;
+          r_b = kRowsK2;
         } else {
-          // lo(t) <= i < hi(t) (and, lowest, hi(t) < death): hi and lo grow with
-          // t over the rows of tokens below T (the searches stop there)
-          const int i = kpos - a.sink, n = max(r_end, 0);
-          r_a = first_above(mi + 4 * kRowsKV, n, i);               // hi > i
-          r_b = first_above(mi + 3 * kRowsKV, n, i);               // lo > i
-          if (lowest) r_b = min(r_b, first_above(mi + 4 * kRowsKV, n, kdeath - 1));
+          // lo(t) <= i < hi(t) (and, lowest, hi(t) < death): hi and lo grow with t
+          const int ii = kpos - a.sink, n = max(r_end, 0);
+          r_a = first_above(mi + 4 * kRowsK2, n, ii);       // hi > i
+          r_b = first_above(mi + 3 * kRowsK2, n, ii);       // lo > i
+          if (lowest) r_b = min(r_b, first_above(mi + 4 * kRowsK2, n, kdeath - 1));
         }
         r_a = max(r_a, 0);
         r_b = min(r_b, r_end);
       }
-      const uint64_t hb = span64(r_a - half * 64, r_b - half * 64);   // this thread's 64 rows
-      uint32_t pp[32], pd[32];
+      const uint32_t hb = (uint32_t)span64(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
+      uint32_t rs[32], rp[32];
+      tmem_ld32(lane_addr + (uint32_t)(x * 64 + 32 * half), rs);
+      tmem_ld32(lane_addr + (uint32_t)(128 + x * 64 + 32 * half), rp);
+      tmem_wait_ld();
+      uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         float p2[2], d2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int rho = half * 64 + c + e;
-          const float p = ((hb >> (c + e)) & 1ull)
-                              ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, bk2 - mf[rho]))
-                              : 0.f;
+          const int rho = 32 * half + c + e;
+          const bool on = (hb >> (c + e)) & 1u;
+          const float p = on ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, bk2 - mf[rho])) : 0.f;
           p2[e] = p;
-          d2[e] = p * (__uint_as_float(rp[c + e]) - mf[kRowsKV + rho]);
+          d2[e] = on ? p * (__uint_as_float(rp[c + e]) - mf[kRowsK2 + rho]) : 0.f;
           if constexpr (kColumn) dr_acc += d2[e];
         }
         pp[c >> 1] = pk2(p2[0], p2[1]);
         pd[c >> 1] = pk2(d2[0], d2[1]);
       }
-      // P^T, dS^T over the first 64 columns of S^T, dP^T (32 per half), once
-      // both threads of the key row have read their columns
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      tmem_st32(lane_addr + kvColS + half * 32, pp);
-      tmem_st32(lane_addr + kvColDP + half * 32, pd);
+      // P^T, dS^T over the first 16 of this thread's 32 columns of S^T, dP^T
+      tmem_st16(lane_addr + (uint32_t)(x * 64 + 32 * half), pp);
+      tmem_st16(lane_addr + (uint32_t)(128 + x * 64 + 32 * half), pd);
       tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(K2_PF + x));
     }
-    if (it + 1 < n_rt) put_rows(it + 1);               // the next stage's row data
-    tc_fence_before();
-    __syncthreads();
-    // dV += P^T dO, dK += dS^T Q (P^T, dS^T from TMEM)
-    if (tid == 0) {
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(K2_DONE), 0, abort_flag, err, 420));
+    if (ok) {
       tc_fence_after();
-      const uint64_t dob = sdesc(ds_, kRowsKV * 128, 1024), qb = sdesc(qs, kRowsKV * 128, 1024);
-#pragma unroll
-      for (int ks = 0; ks < kRowsKV / 16; ++ks) {
-        const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
-        mma_f16_ts(tmem + kvColDV, tmem + kvColS + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
-        mma_f16_ts(tmem + kvColDK, tmem + kvColDP + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
+      // this thread: key row, dims [64 half, 64 half + 64) of dK and dV
+      int pos = kpos;
+      bool store = key_row < nk;
+      if constexpr (kColumn) {
+        if (store) {
+          pos = kpos < a.sink ? kpos : __ldg(a.idx + crow + kpos - a.sink);
+          store = pos < a.T;
+        }
       }
-      mma_commit(bar_kv);
-    }
-    ++kv_issued;
-  }
-  if (ok && kv_issued > 0) {
-    ok = mbar_wait(bar_kv, (kv_issued - 1) & 1, abort_flag, err, 414);
-    ok = __syncthreads_and(ok);
-  }
-  cpa_wait_all();
-  if (ok) {
-    tc_fence_after();
-    // this thread: key row, dims [64 half, 64 half + 64) of dK and dV
-    int pos = kpos;
-    bool store = key_row < nk;
-    if constexpr (kColumn) {
-      if (store) {
-        pos = kpos < a.sink ? kpos : __ldg(a.idx + crow + kpos - a.sink);
-        store = pos < a.T;
+      // dL/dr of a retained slot: sum of dS over its rows, over r (both halves add)
+      if constexpr (kColumn) {
+        if (store && a.dr != nullptr && kpos >= a.sink) atomicAdd(a.dr + crow + pos, dr_acc * ex2(-bk2));
       }
-    }
-    // dL/dr of a retained slot: sum of dS over its rows, over r (both halves add)
-    if constexpr (kColumn) {
-      if (store && a.dr != nullptr && kpos >= a.sink) atomicAdd(a.dr + crow + pos, dr_acc * ex2(-bk2));
-    }
-    const long long rowoff = (((long long)b * a.T + (store ? pos : 0)) * a.Hkv + h) * HD;
+      const long long rowoff = (((long long)b * a.T + (store ? pos : 0)) * a.Hkv + h) * HD;
 #pragma unroll 1
-    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-      uint32_t rk[32], rv[32];
-      tmem_ld32(lane_addr + kvColDK + c0, rk);
-      tmem_ld32(lane_addr + kvColDV + c0, rv);
-      tmem_wait_ld();
-      if (store) {
-        float* dkr = a.dk + rowoff + c0;
-        float* dvr = a.dv + rowoff + c0;
-        if constexpr (kColumn) {
-          // 16-byte vector atomics (rows are 512-byte aligned, c0 + e a multiple of 4)
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+        uint32_t rk[32], rv[32];
+        tmem_ld32(lane_addr + 384 + c0, rk);
+        tmem_ld32(lane_addr + 256 + c0, rv);
+        tmem_wait_ld();
+        if (store) {
+          float* dkr = a.dk + rowoff + c0;
+          float* dvr = a.dv + rowoff + c0;
+          if constexpr (kColumn) {
+            // 16-byte vector atomics (rows are 512-byte aligned, c0 + e a multiple of 4)
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            atomicAdd(reinterpret_cast<float4*>(dkr + e),
-                      make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
-                                  __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale));
-            atomicAdd(reinterpret_cast<float4*>(dvr + e),
-                      make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
-                                  __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3])));
-          }
-        } else {
+            for (int e = 0; e < 32; e += 4) {
+              atomicAdd(reinterpret_cast<float4*>(dkr + e),
+                        make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
+                                    __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale));
+              atomicAdd(reinterpret_cast<float4*>(dvr + e),
+                        make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
+                                    __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3])));
+            }
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            *reinterpret_cast<float4*>(dkr + e) =
-                make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
-                            __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale);
-            *reinterpret_cast<float4*>(dvr + e) =
-                make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
-                            __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3]));
+            for (int e = 0; e < 32; e += 4) {
+              *reinterpret_cast<float4*>(dkr + e) =
+                  make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
+                              __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale);
+              *reinterpret_cast<float4*>(dvr + e) =
+                  make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
+                              __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3]));
+            }
           }
         }
       }
     }
-  } else if (tid == 0) {
-    mbar_drain(bar_s, 0);
-    mbar_drain(bar_s, 1);
-    if (kv_issued > 0) mbar_drain(bar_kv, (kv_issued - 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kvTmemCols)
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
                  : "memory");
 }
 
@@ -745,22 +751,49 @@ bool attn_backward_dq_tc_supported(const lte_dims* d) {
 
 cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
   using namespace bwdtc;
+  const int TOK = kRowsK2 / a.G;
+  // tensor maps (contiguous bf16 rows of 128; 128-byte swizzle, 64-column boxes;
+  // rows past a tensor's end read as zero)
+  CUtensorMap mq, mdo, mk, mv, mkc, mvc;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
+    const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hq * HD * 2, (cuuint64_t)a.T * a.Hq * HD * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)a.G, (cuuint32_t)TOK, 1};
+    if (!encode(&mq, a.q, 4, dims, st, box) || !encode(&mdo, a.dO, 4, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hkv, (cuuint64_t)a.T, (cuuint64_t)B};
+    const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hkv * HD * 2,
+                              (cuuint64_t)a.T * a.Hkv * HD * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kKeysKV, 1};
+    if (!encode(&mk, a.k, 4, dims, st, box) || !encode(&mv, a.v, 4, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t rows = (cuuint64_t)a.sink + a.T;
+    const cuuint64_t dims[3] = {(cuuint64_t)HD, rows, (cuuint64_t)B * a.Hkv};
+    const cuuint64_t st[2] = {(cuuint64_t)HD * 2, rows * HD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kKeysKV, 1};
+    if (!encode(&mkc, a.k_col, 3, dims, st, box) || !encode(&mvc, a.v_col, 3, dims, st, box))
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kvSmemBytes);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kvSmemBytes);
+                           k2Smem);
   if (e != cudaSuccess) return e;
   const int n_ktiles = (a.T + kKeysKV - 1) / kKeysKV;
-  bwd_dkdv_tc_kernel<false><<<dim3(n_ktiles, a.Hkv, B), kThreadsKV, kvSmemBytes, stream>>>(a, 1, err);
+  bwd_dkdv_tc_kernel<false><<<dim3(n_ktiles, a.Hkv, B), kThreadsK2, k2Smem, stream>>>(mq, mdo, mk, mv, a,
+                                                                                     1, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int TOK = kRowsKV / a.G;
   const int n_ctiles = (a.sink + a.T + kKeysKV - 1) / kKeysKV;
-  const int n_split = ((a.T + TOK - 1) / TOK + kSplitRowsKV - 1) / kSplitRowsKV;
+  const int n_split = ((a.T + TOK - 1) / TOK + kSplitRowsK2 - 1) / kSplitRowsK2;
   const long long gx = (long long)n_ctiles * n_split;
   if (gx > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-  bwd_dkdv_tc_kernel<true><<<dim3((unsigned)gx, a.Hkv, B), kThreadsKV, kvSmemBytes, stream>>>(
-      a, n_split, err);
+  bwd_dkdv_tc_kernel<true><<<dim3((unsigned)gx, a.Hkv, B), kThreadsK2, k2Smem, stream>>>(
+      mq, mdo, mkc, mvc, a, n_split, err);
   return cudaGetLastError();
 }
 
