@@ -23,6 +23,9 @@ struct Args {
   // sinks) and dL/dr ([B,Hkv,T], accumulated with atomics onto zeros)
   const float* bias;
   float* dr;
+  // the tcgen05 column pass's work list: item count (int) at offset 0, items
+  // (16 bytes each) from offset 256
+  void* col_work;
 };
 
 // retained count a row sees and the start of its retained range

@@ -579,8 +579,12 @@ cudaError_t launch(const Args& a, int B, bool dq_tc, DevError* err, cudaStream_t
 
 }  // namespace bwd
 
+// D_t, then (256-aligned) the work list of the tcgen05 column pass
+static size_t delta_bytes_aligned(const lte_dims* d) {
+  return ((size_t)d->B * d->Hq * d->T * sizeof(float) + 255) / 256 * 256;
+}
 size_t attn_backward_scratch_bytes(const lte_dims* d) {
-  return (size_t)d->B * d->Hq * d->T * sizeof(float);        // D_t
+  return delta_bytes_aligned(d) + 256 + 16 * attn_backward_col_items_cap(d);
 }
 
 cudaError_t attn_backward(const BackwardArgs& g, cudaStream_t stream) {
@@ -595,6 +599,7 @@ cudaError_t attn_backward(const BackwardArgs& g, cudaStream_t stream) {
   a.v_col = (const __nv_bfloat16*)g.v_col;
   a.cnt = g.cnt; a.death = g.death; a.idx = g.idx; a.nret = g.nret; a.lse = g.lse;
   a.delta = reinterpret_cast<float*>(g.scratch);
+  a.col_work = static_cast<char*>(g.scratch) + delta_bytes_aligned(d);
   a.dq = g.dq; a.dk = g.dk; a.dv = g.dv;
   a.bias = g.bias; a.dr = g.dr;
   // tcgen05 kernels where they apply (head dim 128), else the warp-MMA kernels

@@ -69,15 +69,7 @@ __device__ __forceinline__ uint64_t span64(int a, int b) {
   const uint64_t ones = (b - a == 64) ? ~0ull : ((1ull << (b - a)) - 1ull);
   return ones << a;
 }
-// first index i in [0, n) with v[i] > x for a nondecreasing v (n if none)
-__device__ __forceinline__ int first_above(const int* v, int n, int x) {
-  int l = 0, r = n;
-  while (l < r) {
-    const int m = (l + r) >> 1;
-    if (v[m] > x) r = m; else l = m + 1;
-  }
-  return l;
-}
+
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -394,98 +386,222 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ---------------------------------------------------------------- dK, dV
-// One CTA per 128-key tile (keys of k for the window part, kColumn = false;
-// slots of the column segment, kColumn = true, for this CTA's share of the
-// attending rows).  Keys are the MMA rows; the attending query rows come in
-// tiles of 64 (64/G tokens x the G heads), and per row tile i:
-//   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM buffer i % 2
+// Persistent: one CTA per SM takes work items in a static stride.  An item is
+// a 128-key tile and a run of the query-row tiles that attend it: for the
+// window part (kColumn = false) the keys of k, item = (b, h, tile), all rows
+// t in [j, j + w); for the column part (kColumn = true) slots of the column
+// segment, items from the list bwd_col_items_kernel writes (a slot's rows are
+// split into runs of about kSplitRowsK2 row tiles, so several CTAs share a
+// busy tile and add into dK, dV with atomics).  Keys are the MMA rows; the
+// attending query rows come in tiles of 64 (64/G tokens x the G heads), and
+// per row tile:
+//   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM
 //   P^T, dS^T = P^T (dP^T - D)         (two threads per key row, 32 rows each)
+//                                      into TMEM, as bf16
 //   dV += P^T dO, dK += dS^T Q         (M128 N128 K64; P^T, dS^T read from TMEM)
-// Roles (384 threads, one CTA per SM):
-//   warp 0     TMA producer (one elected lane): K and V once; per row tile, Q
-//              and dO into a 3-stage ring, the rows' lse, D, token and retained
-//              range written by the warp's lanes into the stage;
-//   warp 1     MMA issuer: S^T(i), dP^T(i), then dV and dK of tile i - 1 once
-//              its P^T and dS^T are in TMEM -- the tensor core computes tile i
-//              while the rows of tile i - 1 are formed;
+// K sits in TMEM (bf16 pairs) as the A operand of S^T and V in shared memory,
+// so that the shared-memory operand reads of a row tile (Q and dO twice each,
+// V once) stay within what the tensor core's full rate needs.
+// Roles (384 threads):
+//   warp 0     TMA producer (one elected lane): V of each item into one of two
+//              buffers, once the products of the item before last are done; per
+//              row tile, Q and dO into
+//              a 4-stage ring, then the rows' lse, D, token and retained range,
+//              written by the warp's lanes while the copies fly;
+//   warp 1     MMA issuer: S^T and dP^T of a row tile as soon as the rows have
+//              read those of the tile before, then dV and dK of the tile before
+//              once its P^T and dS^T are written -- the tensor core computes
+//              S^T of the next tile while the rows of this one are formed;
 //   warps 4-11 two threads per key row (warps 4-7 rows 0-31 of a tile, 8-11
-//              rows 32-63): P^T and dS^T, written as bf16 over their own
-//              columns of S^T and dP^T; at the end, dK and dV out.
-// TMEM: S^T[2] 0..127, dP^T[2] 128..255, dV 256..383, dK 384..511.
+//              rows 32-63): K of each item into TMEM (loaded while the item
+//              before finishes); P^T and dS^T, written once dV and dK of the
+//              tile before have read theirs; at the end of an item, dK and dV
+//              out through a shared-memory stage in 32-column chunks, so that
+//              each warp store (or add) covers four whole 128-byte rows.
+// TMEM: S^T 0..63, dP^T 64..127, P^T 128..159 and dS^T 160..191 (64 bf16 rows
+// packed in pairs), K 192..255, dV 256..383, dK 384..511.  Barrier phases run
+// on a row-tile counter that continues across items (ring stages, S, P) or on
+// the item counter (V buffers and the items' completion: one barrier each per
+// buffer, K).
 constexpr int kKeysKV = 128;
 constexpr int kRowsK2 = 64;                       // attending query rows per tile
-constexpr int kStagesK2 = 3;
+constexpr int kStagesK2 = 4;
 constexpr int kThreadsK2 = 384;
-constexpr int kSplitRowsK2 = 32;                  // row tiles per CTA of the column pass
-constexpr uint32_t k2K = 0, k2V = 32768;          // [128][128] bf16: halves of 16 KiB
+constexpr int kSplitRowsK2 = 32;                  // row tiles per column item, at most
+constexpr uint32_t k2V = 0;                       // 2 x [128][128] bf16: halves of 16 KiB
 constexpr uint32_t k2QD = 65536;                  // stage s: Q at + 32 KiB s, dO at + 16 KiB
 constexpr uint32_t k2Meta = k2QD + kStagesK2 * 32768;            // stage s: [5][64] words
-constexpr uint32_t k2Bar = k2Meta + kStagesK2 * 5 * kRowsK2 * 4;
+constexpr uint32_t k2Stage = k2Meta + kStagesK2 * 5 * kRowsK2 * 4;   // [128][32] fp32, swizzled
+constexpr uint32_t k2Pos = k2Stage + kKeysKV * 128;                  // [128] output row per key
+constexpr uint32_t k2Bar = k2Pos + kKeysKV * 4;
 constexpr int k2Smem = k2Bar + 256;
+constexpr uint32_t k2ColS = 0, k2ColDP = 64, k2ColP = 128, k2ColDS = 160, k2ColK = 192, k2ColDV = 256,
+                   k2ColDK = 384;
 enum {
-  K2_KVF = 0, K2_F = 1, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_PF = K2_SF + 2,
-  K2_DONE = K2_PF + 2, kNumBarsK2 = K2_DONE + 1
+  K2_KVF = 0, K2_F = 2, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_SE = K2_SF + 1,
+  K2_PF = K2_SE + 1, K2_PE = K2_PF + 1, K2_KT = K2_PE + 1, K2_DONE = K2_KT + 1, kNumBarsK2 = K2_DONE + 2
 };
-static_assert(8 * kNumBarsK2 + 16 <= 256, "barriers, flags and the row range fit");
+static_assert(8 * kNumBarsK2 + 16 <= 256, "barriers and flags fit");
+static_assert(k2Smem <= 227 * 1024, "shared memory fits one CTA");
+
+// One work item: KV unit u = b Hkv + h, key tile, first row tile, row tiles.
+struct K2Item {
+  int u, tile, rt0, n_rt;
+};
+
+// Warp-wide: first m in [l, r) with pred(m) true for a predicate that is false
+// then true over [l, r) (r if none); every lane returns it.  Rounds of 32 probes.
+template <class Pred>
+__device__ __forceinline__ int warp_first_true(int l, int r, int lane, Pred pred) {
+  while (r - l > 32) {
+    const int step = (r - l + 31) / 32;
+    const int p = l + lane * step;
+    const unsigned hit = __ballot_sync(0xffffffffu, p < r && pred(p));
+    const unsigned probed = __ballot_sync(0xffffffffu, p < r);
+    if (hit == 0u) {
+      l = l + (31 - __clz(probed)) * step + 1;           // past the last probe
+    } else {
+      const int f = __ffs(hit) - 1;
+      if (f == 0) return l;
+      r = l + f * step;                                   // true there
+      l = l + (f - 1) * step + 1;
+    }
+  }
+  const int p = l + lane;
+  const unsigned hit = __ballot_sync(0xffffffffu, p < r && pred(p));
+  return hit ? l + __ffs(hit) - 1 : r;
+}
+
+// The column part's work list: one CTA per KV unit, one warp per slot tile
+// (32 tiles per round); the query tokens [lo_t, hi_t] that attend some slot of
+// the tile (the same bounds the row masks use: a sink slot j is attended by
+// rows t >= j + w, a retained slot i by the rows whose retained count n_t,
+// nondecreasing in t, holds it), cut into runs of at most kSplitRowsK2 row
+// tiles of near-equal length.  Each round's items are written in tile order
+// at a block reserved with one atomic, so a unit's items sit together: CTAs
+// that take neighbouring items work on the same unit's Q and dO, which then
+// stay in L2.
+constexpr int kColItemsThreads = 1024;
+__global__ void __launch_bounds__(kColItemsThreads)
+bwd_col_items_kernel(const bwd::Args a, int n_ctiles, K2Item* items, int* n_items) {
+  __shared__ int rt0_sh[32], n_sh[32], runs_sh[32], off_sh[33];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int u = blockIdx.x;
+  const long long crow = (long long)u * a.T;
+  const int nret = __ldg(a.nret + u);
+  const int TOK = kRowsK2 / a.G;
+  for (int base_tile = 0; base_tile < n_ctiles; base_tile += 32) {
+    const int tile = base_tile + wid;
+    const int k0 = tile * kKeysKV;
+    const int nk = tile < n_ctiles ? min(kKeysKV, a.sink + nret - k0) : 0;
+    int lo_t = a.T, hi_t = -1;
+    if (nk > 0) {
+      const int s_end = min(min(a.sink, k0 + nk), a.T);
+      if (k0 < s_end) {
+        lo_t = k0 + a.window;
+        hi_t = a.T - 1;
+      }
+      const int i0 = max(k0, a.sink) - a.sink, i1 = k0 + nk - a.sink;
+      if (i1 > i0 && a.cap > 0 && (a.cap_policy != LTE_CAP_FIRST || i0 < a.cap) && a.window < a.T) {
+        auto cnt = [&](int t) { return __ldg(a.cnt + crow + t - a.window); };   // rows t >= w
+        const int l = warp_first_true(a.window, a.T, lane, [&](int m) { return cnt(m) > i0; });
+        if (l < a.T) {
+          long long bound;                                 // rows need cnt < bound
+          if (a.cap_policy == LTE_CAP_RECENT) bound = (long long)i1 + a.cap;
+          else if (a.cap_policy == LTE_CAP_FIRST) bound = 1ll << 40;
+          else {
+            int md = 0;
+            for (int i = i0 + lane; i < i1; i += 32) md = max(md, __ldg(a.death + crow + i));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) md = max(md, __shfl_xor_sync(0xffffffffu, md, o));
+            bound = md;
+          }
+          const int l2 = warp_first_true(l, a.T, lane, [&](int m) { return (long long)cnt(m) >= bound; });
+          if (l2 > l) {
+            lo_t = min(lo_t, l);
+            hi_t = max(hi_t, l2 - 1);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      int r0 = 0, n = 0, runs = 0;
+      if (lo_t <= hi_t) {
+        r0 = lo_t / TOK;
+        n = hi_t / TOK - r0 + 1;
+        runs = (n + kSplitRowsK2 - 1) / kSplitRowsK2;
+      }
+      rt0_sh[wid] = r0, n_sh[wid] = n, runs_sh[wid] = runs;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0;
+      for (int w = 0; w < 32; ++w) off_sh[w] = acc, acc += runs_sh[w];
+      off_sh[32] = acc > 0 ? atomicAdd(n_items, acc) : 0;
+    }
+    __syncthreads();
+    if (lane == 0 && runs_sh[wid] > 0) {
+      const int n = n_sh[wid], runs = runs_sh[wid], len = (n + runs - 1) / runs;
+      K2Item* dst = items + off_sh[32] + off_sh[wid];
+      for (int c = 0; c < runs; ++c) dst[c] = K2Item{u, tile, rt0_sh[wid] + c * len, min(len, n - c * len)};
+    }
+    __syncthreads();                                       // the round's arrays may be reused
+  }
+}
 
 template <bool kColumn>
 __global__ void __launch_bounds__(kThreadsK2, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const bwd::Args a, int n_split, DevError* err) {
+                   const __grid_constant__ CUtensorMap tm_v, const bwd::Args a, const K2Item* items,
+                   const int* n_items_p, int n_items_win, DevError* err) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sb = sa(sm);
   if ((sb & 1023u) != 0) {
     if (threadIdx.x == 0) record_error(err, LTE_ERR_DEVICE, 413);
     return;
   }
+  const int n_items = kColumn ? __ldg(n_items_p) : n_items_win;
+  if ((int)blockIdx.x >= n_items) return;              // no work (uniform)
   auto bar = [&](int i) { return sb + k2Bar + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + k2Bar + 8 * kNumBarsK2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + k2Bar + 8 * kNumBarsK2 + 4);
-  int* range_sh = reinterpret_cast<int*>(sm + k2Bar + 8 * kNumBarsK2 + 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G, TOK = kRowsK2 / G;
-  const int h = blockIdx.y, b = blockIdx.z, u = b * a.Hkv + h;
-  const long long crow = (long long)u * a.T;
-  const long long col_base = (long long)u * (a.sink + a.T);
   const bool lowest = a.death != nullptr;
-  const int tile = kColumn ? (int)blockIdx.x / n_split : (int)blockIdx.x;
-  const int split = kColumn ? (int)blockIdx.x % n_split : 0;
-  const int k0 = tile * kKeysKV;
-  const int nk = kColumn ? min(kKeysKV, a.sink + __ldg(a.nret + u) - k0) : min(kKeysKV, a.T - k0);
-  if (nk <= 0) return;
-
-  // row tiles that attend some key of this tile (this CTA's share of them)
-  if (tid == 0) {
-    int lo_t, hi_t;
-    bwd::attending_tokens(a, crow, kColumn, k0, nk, lo_t, hi_t);
-    int rt0 = lo_t / TOK, rt1 = hi_t / TOK;
-    if (lo_t > hi_t) rt0 = 1, rt1 = 0;
+  const int n_ktiles = (a.T + kKeysKV - 1) / kKeysKV;
+  // item `it` -> KV unit, key tile, its row tiles [rt0, rt0 + n_rt) and keys
+  auto item_at = [&](int it) {
+    K2Item w;
     if constexpr (kColumn) {
-      if (rt0 <= rt1) {
-        const int first = rt0 + split * kSplitRowsK2;
-        rt1 = min(rt1, first + kSplitRowsK2 - 1);
-        rt0 = first;
-      }
+      w = items[it];
+    } else {
+      w.tile = it % n_ktiles;
+      w.u = it / n_ktiles;
+      const int k0 = w.tile * kKeysKV, nk = min(kKeysKV, a.T - k0);
+      w.rt0 = k0 / TOK;                                  // rows t in [k0, k0 + nk - 1 + w - 1]
+      w.n_rt = min(a.T - 1, k0 + nk - 1 + a.window - 1) / TOK - w.rt0 + 1;
     }
-    range_sh[0] = rt0;
-    range_sh[1] = rt1;
-  }
-  __syncthreads();
-  const int rt0 = range_sh[0], n_rt = range_sh[1] - range_sh[0] + 1;
-  if (n_rt <= 0) return;                               // nothing attends (uniform)
+    return w;
+  };
+  auto keys_of = [&](const K2Item& w) {
+    const int k0 = w.tile * kKeysKV;
+    return kColumn ? min(kKeysKV, a.sink + __ldg(a.nret + w.u) - k0) : min(kKeysKV, a.T - k0);
+  };
 
   if (tid == 0) {
     mbar_init(bar(K2_KVF), 1);
+    mbar_init(bar(K2_KVF + 1), 1);
     for (int st = 0; st < kStagesK2; ++st) {
       mbar_init(bar(K2_F + st), 1);
       mbar_init(bar(K2_E + st), 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(bar(K2_SF + x), 1);
-      mbar_init(bar(K2_PF + x), 256);
-    }
+    mbar_init(bar(K2_SF), 1);
+    mbar_init(bar(K2_SE), 256);
+    mbar_init(bar(K2_PF), 256);
+    mbar_init(bar(K2_PE), 1);
+    mbar_init(bar(K2_KT), 256);
     mbar_init(bar(K2_DONE), 1);
+    mbar_init(bar(K2_DONE + 1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -504,188 +620,272 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     bool ok = true;
-    if (elect_one()) {
-      mbar_expect_tx(bar(K2_KVF), 2 * kKeysKV * HD * 2);
-      for (int hf = 0; hf < 2; ++hf) {
-        if constexpr (kColumn) {
-          tma_load_3d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, k0, u);
-          tma_load_3d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, k0, u);
-        } else {
-          tma_load_4d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, h, k0, b);
-          tma_load_4d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, h, k0, b);
-        }
-      }
-    }
-    __syncwarp();
-    int issued = 0;
-    for (int i = 0; i < n_rt && ok; ++i) {
-      const int st = i % kStagesK2, use = i / kStagesK2;
-      if (use >= 1 && !(ok = wwait(bar(K2_E + st), (use - 1) & 1, abort_flag, err, 414))) break;
-      // the rows' data: lse (log2), D, token, retained range [lo, hi)
-      const int t0r = (rt0 + i) * TOK;
-      float* mf = reinterpret_cast<float*>(sm + k2Meta) + st * 5 * kRowsK2;
-      int* mi = reinterpret_cast<int*>(mf);
-      for (int r = lane; r < kRowsK2; r += 32) {
-        const int tt = t0r + r / G, g = r % G;
-        float l2 = 0.f, dd = 0.f;
-        int cv = 0;
-        if (tt < a.T) {
-          const long long li = ((long long)b * a.Hq + h * G + g) * a.T + tt;
-          l2 = __ldg(a.lse + li) * 1.4426950408889634f;
-          dd = __ldg(a.delta + li);
-          if (tt >= a.window) cv = __ldg(a.cnt + crow + tt - a.window);
-        }
-        const int hi = (tt < a.T && tt >= a.window) ? held_retained(cv, a.cap, a.cap_policy) : 0;
-        const int lo = (!lowest && a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
-        mf[r] = l2;
-        mf[kRowsK2 + r] = dd;
-        mi[2 * kRowsK2 + r] = tt;
-        mi[3 * kRowsK2 + r] = lo;
-        mi[4 * kRowsK2 + r] = hi;
-      }
-      __syncwarp();
+    int g = 0, k = 0;                                      // row tiles, items issued
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      const K2Item w = item_at(it);
+      const int h = w.u % a.Hkv, b = w.u / a.Hkv, k0 = w.tile * kKeysKV;
+      const long long crow = (long long)w.u * a.T;
+      // V into buffer k % 2: the products of item k - 2 have all completed
+      const int vb = k & 1;
+      if (k >= 2 && !(ok = wwait(bar(K2_DONE + vb), ((k - 2) >> 1) & 1, abort_flag, err, 424))) break;
       if (elect_one()) {
-        const uint32_t qs = sb + k2QD + st * 32768u;
-        mbar_expect_tx(bar(K2_F + st), 2 * kRowsK2 * HD * 2);
+        const uint32_t vs = sb + k2V + (uint32_t)vb * 32768u;
+        mbar_expect_tx(bar(K2_KVF + vb), kKeysKV * HD * 2);
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_4d(qs + hf * 8192u, &tm_q, bar(K2_F + st), hf * 64, h * G, t0r, b);
-          tma_load_4d(qs + 16384u + hf * 8192u, &tm_do, bar(K2_F + st), hf * 64, h * G, t0r, b);
+          if constexpr (kColumn) tma_load_3d(vs + hf * 16384u, &tm_v, bar(K2_KVF + vb), hf * 64, k0, w.u);
+          else tma_load_4d(vs + hf * 16384u, &tm_v, bar(K2_KVF + vb), hf * 64, h, k0, b);
         }
       }
       __syncwarp();
-      issued = i + 1;
+      for (int i = 0; i < w.n_rt; ++i, ++g) {
+        const int st = g % kStagesK2, use = g / kStagesK2;
+        if (use >= 1 && !(ok = wwait(bar(K2_E + st), (use - 1) & 1, abort_flag, err, 414))) break;
+        const int t0r = (w.rt0 + i) * TOK;
+        // the copies first (the phase also waits for the arrive below) ...
+        if (elect_one()) {
+          const uint32_t qs = sb + k2QD + st * 32768u;
+          mbar_add_tx(bar(K2_F + st), 2 * kRowsK2 * HD * 2);
+          for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(qs + hf * 8192u, &tm_q, bar(K2_F + st), hf * 64, h * G, t0r, b);
+            tma_load_4d(qs + 16384u + hf * 8192u, &tm_do, bar(K2_F + st), hf * 64, h * G, t0r, b);
+          }
+        }
+        // ... then the rows' data: lse (log2) and D per row; the retained range
+        // [lo, hi) per token (j < 64/G), INT_MAX for tokens past T
+        float* mf = reinterpret_cast<float*>(sm + k2Meta) + st * 5 * kRowsK2;
+        int* mi = reinterpret_cast<int*>(mf);
+        float l2[2], dd[2];
+        int cv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = lane + 32 * e, tt = t0r + r / G, gg = r % G, tj = t0r + r;
+          l2[e] = 0.f, dd[e] = 0.f, cv[e] = 0;
+          if (tt < a.T) {
+            const long long li = ((long long)b * a.Hq + h * G + gg) * a.T + tt;
+            l2[e] = __ldg(a.lse + li);
+            dd[e] = __ldg(a.delta + li);
+          }
+          if (kColumn && r < TOK && tj < a.T && tj >= a.window) cv[e] = __ldg(a.cnt + crow + tj - a.window);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = lane + 32 * e, tj = t0r + r;
+          mf[r] = l2[e] * 1.4426950408889634f;
+          mf[kRowsK2 + r] = dd[e];
+          if (kColumn && r < TOK) {
+            int hi = INT_MAX, lo = INT_MAX;
+            if (tj < a.T) {
+              hi = tj >= a.window ? held_retained(cv[e], a.cap, a.cap_policy) : 0;
+              lo = (!lowest && a.cap_policy == LTE_CAP_RECENT && hi - a.cap > 0) ? hi - a.cap : 0;
+            }
+            mi[3 * kRowsK2 + r] = lo;
+            mi[4 * kRowsK2 + r] = hi;
+          }
+        }
+        __syncwarp();
+        if (elect_one()) mbar_arrive(bar(K2_F + st));
+        __syncwarp();
+      }
     }
     // every issued copy has landed before the CTA may exit
-    mbar_drain(bar(K2_KVF), 0);
-    for (int q = issued - kStagesK2 > 0 ? issued - kStagesK2 : 0; q < issued; ++q)
+    for (int q = k - 2 > 0 ? k - 2 : 0; q < k; ++q) mbar_drain(bar(K2_KVF + (q & 1)), (q >> 1) & 1);
+    for (int q = g - kStagesK2 > 0 ? g - kStagesK2 : 0; q < g; ++q)
       mbar_drain(bar(K2_F + q % kStagesK2), (q / kStagesK2) & 1);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t id_s = idesc(kKeysKV, kRowsK2, false);    // S^T, dP^T: K-major A and B
     const uint32_t id_o = idesc(kKeysKV, HD, true);          // dV, dK: dO, Q as N-contiguous B
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_KVF), 0, abort_flag, err, 415));
-    auto issue_dvdk = [&](int i) -> bool {                   // dV, dK of row tile i
-      const int x = i & 1, st = i % kStagesK2;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(K2_PF + x), (i >> 1) & 1, abort_flag, err, 416)))
-        return false;
+    bool ok = true;
+    auto issue_dvdk = [&](int gg, bool first) -> bool {      // dV, dK of row tile gg
+      const int st = gg % kStagesK2;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(K2_PF), gg & 1, abort_flag, err, 416))) return false;
       tc_fence_after();
       if (elect_one()) {
         const uint32_t qs = sb + k2QD + st * 32768u;
         const uint64_t qb = sdesc(qs, kRowsK2 * 128, 1024), dob = sdesc(qs + 16384u, kRowsK2 * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < kRowsK2 / 16; ++ks) {
-          // rows 16 ks .. of P^T, dS^T: the 32 rows of a thread pair's half sit in
-          // columns 32 half .. + 15 of the buffer
-          const uint32_t pc = (uint32_t)(x * 64 + 32 * (ks >> 1) + 8 * (ks & 1));
-          const uint32_t acc = (i > 0 || ks > 0) ? 1u : 0u;
-          mma_f16_ts(tmem + 256, tmem + pc, dob + ((ks * 2048) >> 4), id_o, acc);
-          mma_f16_ts(tmem + 384, tmem + 128 + pc, qb + ((ks * 2048) >> 4), id_o, acc);
+          const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
+          mma_f16_ts(tmem + k2ColDV, tmem + k2ColP + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + k2ColDK, tmem + k2ColDS + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
         }
         mma_commit(bar(K2_E + st));                          // the row tile's stage is free
+        mma_commit(bar(K2_PE));                              // P^T, dS^T may be overwritten
       }
       __syncwarp();
       return true;
     };
-    for (int i = 0; i < n_rt && ok; ++i) {
-      const int x = i & 1, st = i % kStagesK2;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_F + st), (i / kStagesK2) & 1, abort_flag, err, 417));
-      if (!ok) break;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint32_t qs = sb + k2QD + st * 32768u;
-        const uint64_t dk = sdesc(sb + k2K, 16, 1024), dv = sdesc(sb + k2V, 16, 1024);
-        const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
+    int g = 0, k = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      const int n_rt = item_at(it).n_rt, vb = k & 1;
+      // V landed; K in TMEM (and the previous item's dK, dV read out)
+      ok = mbar_wait(bar(K2_KVF + vb), (k >> 1) & 1, abort_flag, err, 415);
+      if (ok) ok = mbar_wait(bar(K2_KT), k & 1, abort_flag, err, 422);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      for (int i = 0; i < n_rt; ++i, ++g) {
+        const int st = g % kStagesK2;
+        ok = mbar_wait(bar(K2_F + st), (g / kStagesK2) & 1, abort_flag, err, 417);
+        // S^T, dP^T of the tile before have been read by the rows
+        if (ok && g >= 1) ok = mbar_wait(bar(K2_SE), (g - 1) & 1, abort_flag, err, 421);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t qs = sb + k2QD + st * 32768u;
+          const uint64_t dv = sdesc(sb + k2V + (uint32_t)vb * 32768u, 16, 1024);
+          const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
-          const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
-          mma_f16(tmem + x * 64, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
-          mma_f16(tmem + 128 + x * 64, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < HD / 16; ++ks) {
+            const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
+            const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
+            mma_f16_ts(tmem + k2ColS, tmem + k2ColK + 8 * ks, dq + ob, id_s, ks > 0 ? 1u : 0u);
+            mma_f16(tmem + k2ColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(K2_SF));
         }
-        mma_commit(bar(K2_SF + x));
+        __syncwarp();
+        if (i >= 1 && !(ok = issue_dvdk(g - 1, i == 1))) break;
       }
+      if (ok) ok = issue_dvdk(g - 1, n_rt == 1);
+      if (elect_one()) mma_commit(bar(K2_DONE + vb));      // every product of the item has completed
       __syncwarp();
-      if (i >= 1 && !(ok = issue_dvdk(i - 1))) break;
     }
-    if (ok) ok = issue_dvdk(n_rt - 1);
-    if (elect_one()) mma_commit(bar(K2_DONE));             // every product above has completed
-    __syncwarp();
-    mbar_drain(bar(K2_DONE), 0);
+    if (k >= 1) mbar_drain(bar(K2_DONE + ((k - 1) & 1)), ((k - 1) >> 1) & 1);
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- key rows (warps 4-11)
     const int quad = warp & 3, half = (warp - 4) >> 2;     // TMEM lane quadrant, row half
     const int key_row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const int kpos = k0 + key_row;                         // position (window) or slot (column)
-    int kdeath = 0;
-    if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
-    // relaxed retention: log2 of this slot's weight r (0 for sinks and window keys),
-    // and the partial sum of dS over the rows this thread sees, for dL/dr
-    float bk2 = 0.f, dr_acc = 0.f;
-    if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
+    // K of item `it`: this thread's key row, dims [64 half, 64 half + 64) as bf16
+    // pairs (zeros past the tile's keys)
+    uint32_t kr[32];
+    auto load_k = [&](int it) {
+      const K2Item w = item_at(it);
+      const int kpos = w.tile * kKeysKV + key_row;
+      if (key_row < keys_of(w)) {
+        const __nv_bfloat16* src =
+            kColumn ? a.k_col + ((long long)w.u * (a.sink + a.T) + kpos) * HD
+                    : a.k + (((long long)(w.u / a.Hkv) * a.T + kpos) * a.Hkv + w.u % a.Hkv) * HD;
+        const uint4* s4 = reinterpret_cast<const uint4*>(src + 64 * half);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v4 = __ldg(s4 + c);
+          kr[4 * c] = v4.x, kr[4 * c + 1] = v4.y, kr[4 * c + 2] = v4.z, kr[4 * c + 3] = v4.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) kr[c] = 0u;
+      }
+    };
+    load_k(blockIdx.x);
     bool ok = true;
-    for (int i = 0; i < n_rt && ok; ++i) {
-      const int x = i & 1, st = i % kStagesK2;
-      ok = mbar_wait(bar(K2_F + st), (i / kStagesK2) & 1, abort_flag, err, 418);   // row data
-      if (ok) ok = mbar_wait(bar(K2_SF + x), (i >> 1) & 1, abort_flag, err, 419);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      tc_fence_after();
-      const float* mf = reinterpret_cast<const float*>(sm + k2Meta) + st * 5 * kRowsK2;
-      const int* mi = reinterpret_cast<const int*>(mf);
-      // the rows of this tile that attend this key: one interval [r_a, r_b) of the
-      // (token-major) rows; tokens past T never attend
-      const int t0r = (rt0 + i) * TOK;
-      const int r_end = min(kRowsK2, (a.T - t0r) * G);
-      int r_a = 0, r_b = 0;
-      if (key_row < nk) {
-        if constexpr (!kColumn) {
-          r_a = (kpos - t0r) * G;                          // tokens [kpos, kpos + w)
-          r_b = (kpos + a.window - t0r) * G;
-        } else if (kpos < a.sink) {
-          r_a = (kpos + a.window - t0r) * G;               // tokens >= kpos + w
-          r_b = kRowsK2;
-        } else {
-          // lo(t) <= i < hi(t) (and, lowest, hi(t) < death): hi and lo grow with t
-          const int ii = kpos - a.sink, n = max(r_end, 0);
-          r_a = first_above(mi + 4 * kRowsK2, n, ii);       // hi > i
-          r_b = first_above(mi + 3 * kRowsK2, n, ii);       // lo > i
-          if (lowest) r_b = min(r_b, first_above(mi + 4 * kRowsK2, n, kdeath - 1));
-        }
-        r_a = max(r_a, 0);
-        r_b = min(r_b, r_end);
-      }
-      const uint32_t hb = (uint32_t)span64(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
-      uint32_t rs[32], rp[32];
-      tmem_ld32(lane_addr + (uint32_t)(x * 64 + 32 * half), rs);
-      tmem_ld32(lane_addr + (uint32_t)(128 + x * 64 + 32 * half), rp);
-      tmem_wait_ld();
-      uint32_t pp[16], pd[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float p2[2], d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int rho = 32 * half + c + e;
-          const bool on = (hb >> (c + e)) & 1u;
-          const float p = on ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, bk2 - mf[rho])) : 0.f;
-          p2[e] = p;
-          d2[e] = on ? p * (__uint_as_float(rp[c + e]) - mf[kRowsK2 + rho]) : 0.f;
-          if constexpr (kColumn) dr_acc += d2[e];
-        }
-        pp[c >> 1] = pk2(p2[0], p2[1]);
-        pd[c >> 1] = pk2(d2[0], d2[1]);
-      }
-      // P^T, dS^T over the first 16 of this thread's 32 columns of S^T, dP^T
-      tmem_st16(lane_addr + (uint32_t)(x * 64 + 32 * half), pp);
-      tmem_st16(lane_addr + (uint32_t)(128 + x * 64 + 32 * half), pd);
+    int g = 0, k = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      const K2Item w = item_at(it);
+      const int h = w.u % a.Hkv, b = w.u / a.Hkv, k0 = w.tile * kKeysKV, nk = keys_of(w);
+      const long long crow = (long long)w.u * a.T;
+      const long long col_base = (long long)w.u * (a.sink + a.T);
+      const int kpos = k0 + key_row;                       // position (window) or slot (column)
+      int kdeath = 0;
+      if (kColumn && lowest && kpos >= a.sink && key_row < nk) kdeath = __ldg(a.death + crow + kpos - a.sink);
+      // relaxed retention: log2 of this slot's weight r (0 for sinks and window keys),
+      // and the partial sum of dS over the rows this thread sees, for dL/dr
+      float bk2 = 0.f, dr_acc = 0.f;
+      if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
+      // K (loaded into registers before) into TMEM.  The previous item's S^T
+      // products are done (its last tile's S^T was read) and its dK, dV read out.
+      tmem_st32(lane_addr + k2ColK + 32 * half, kr);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(K2_PF + x));
-    }
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(K2_DONE), 0, abort_flag, err, 420));
-    if (ok) {
+      mbar_arrive(bar(K2_KT));
+      for (int i = 0; i < w.n_rt; ++i, ++g) {
+        const int st = g % kStagesK2;
+        // the row data first: the rows' range is found while S^T is computed
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_F + st), (g / kStagesK2) & 1, abort_flag, err, 418))))
+          break;
+        const float* mf = reinterpret_cast<const float*>(sm + k2Meta) + st * 5 * kRowsK2;
+        const int* mi = reinterpret_cast<const int*>(mf);
+        // the rows of this tile that attend this key: one interval [r_a, r_b) of the
+        // (token-major) rows; tokens past T never attend
+        const int t0r = (w.rt0 + i) * TOK;
+        const int r_end = min(kRowsK2, (a.T - t0r) * G);
+        int r_a = 0, r_b = 0;
+        if (key_row < nk) {
+          if constexpr (!kColumn) {
+            r_a = (kpos - t0r) * G;                        // tokens [kpos, kpos + w)
+            r_b = (kpos + a.window - t0r) * G;
+          } else if (kpos < a.sink) {
+            r_a = (kpos + a.window - t0r) * G;             // tokens >= kpos + w
+            r_b = kRowsK2;
+          } else {
+            // lo(t) <= i < hi(t) (and, lowest, hi(t) < death): hi and lo grow with t
+            // (INT_MAX past T), so the first token above a bound is the count of
+            // tokens at or below it -- counted over broadcast reads
+            const int ii = kpos - a.sink, hd = lowest ? kdeath - 1 : INT_MAX - 1;
+            int ca = 0, cb = 0, cd = 0;
+            for (int j = 0; j < TOK; j += 4) {
+              const int4 hv = *reinterpret_cast<const int4*>(mi + 4 * kRowsK2 + j);
+              const int4 lv = *reinterpret_cast<const int4*>(mi + 3 * kRowsK2 + j);
+              ca += (hv.x <= ii) + (hv.y <= ii) + (hv.z <= ii) + (hv.w <= ii);
+              cb += (lv.x <= ii) + (lv.y <= ii) + (lv.z <= ii) + (lv.w <= ii);
+              cd += (hv.x <= hd) + (hv.y <= hd) + (hv.z <= hd) + (hv.w <= hd);
+            }
+            r_a = G * ca;                                  // first row with hi > i
+            r_b = G * min(cb, cd);                         // first row with lo > i (or hi >= death)
+          }
+          r_a = max(r_a, 0);
+          r_b = min(r_b, r_end);
+        }
+        const uint32_t hb = (uint32_t)span64(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_SF), g & 1, abort_flag, err, 419)))) break;
+        tc_fence_after();
+        uint32_t rs[32], rp[32];
+        tmem_ld32(lane_addr + k2ColS + 32 * half, rs);
+        tmem_ld32(lane_addr + k2ColDP + 32 * half, rp);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(K2_SE));                           // S^T, dP^T may be overwritten
+        const float4* ml = reinterpret_cast<const float4*>(mf + 32 * half);
+        const float4* md = reinterpret_cast<const float4*>(mf + kRowsK2 + 32 * half);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = ml[c4], d4 = md[c4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p4[4], q4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const bool on = (hb >> c) & 1u;
+            const float p = on ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, bk2 - lv[e])) : 0.f;
+            p4[e] = p;
+            q4[e] = on ? p * (__uint_as_float(rp[c]) - dv4[e]) : 0.f;
+            if constexpr (kColumn) dr_acc += q4[e];
+          }
+          pp[2 * c4] = pk2(p4[0], p4[1]);
+          pp[2 * c4 + 1] = pk2(p4[2], p4[3]);
+          pd[2 * c4] = pk2(q4[0], q4[1]);
+          pd[2 * c4 + 1] = pk2(q4[2], q4[3]);
+        }
+        // dV, dK of the tile before have read its P^T, dS^T
+        if (g >= 1 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_PE), (g - 1) & 1, abort_flag, err, 423))))
+          break;
+        tc_fence_after();
+        // rows 32 half .. + 31 of P^T, dS^T: columns 16 half .. + 15
+        tmem_st16(lane_addr + k2ColP + (uint32_t)(16 * half), pp);
+        tmem_st16(lane_addr + k2ColDS + (uint32_t)(16 * half), pd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(K2_PF));
+      }
+      // the next item's K into registers while this item's products finish
+      if (ok && it + (int)gridDim.x < n_items) load_k(it + gridDim.x);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_DONE + (k & 1)), (k >> 1) & 1, abort_flag, err, 420));
+      // the eight row warps go on together or stop together (the stage below
+      // synchronises them with a named barrier)
+      if (!(ok = bar_and(1, 256, ok))) break;
       tc_fence_after();
-      // this thread: key row, dims [64 half, 64 half + 64) of dK and dV
+      // this thread's key row: output row (-1: none), and dL/dr of a retained slot
+      // (sum of dS over its rows, over r; both halves add)
       int pos = kpos;
       bool store = key_row < nk;
       if constexpr (kColumn) {
@@ -693,45 +893,43 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           pos = kpos < a.sink ? kpos : __ldg(a.idx + crow + kpos - a.sink);
           store = pos < a.T;
         }
-      }
-      // dL/dr of a retained slot: sum of dS over its rows, over r (both halves add)
-      if constexpr (kColumn) {
         if (store && a.dr != nullptr && kpos >= a.sink) atomicAdd(a.dr + crow + pos, dr_acc * ex2(-bk2));
       }
-      const long long rowoff = (((long long)b * a.T + (store ? pos : 0)) * a.Hkv + h) * HD;
-#pragma unroll 1
-      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-        uint32_t rk[32], rv[32];
-        tmem_ld32(lane_addr + 384 + c0, rk);
-        tmem_ld32(lane_addr + 256 + c0, rv);
+      int* pos_sh = reinterpret_cast<int*>(sm + k2Pos);
+      if (half == 0) pos_sh[key_row] = store ? pos : -1;
+      // dK (x scale) then dV, 32 columns per round: each thread stages 16 columns
+      // of its key row (16-byte chunks XOR-swizzled by row), then the 256 threads
+      // write rows out, eight threads per 128-byte row
+      const int t2 = tid - 128, c16 = t2 & 7;
+      for (int r = 0; r < 8; ++r) {
+        const int c = r & 3;
+        const bool is_v = r >= 4;
+        uint32_t v16[16];
+        tmem_ld16(lane_addr + (is_v ? k2ColDV : k2ColDK) + (uint32_t)(32 * c + 16 * half), v16);
         tmem_wait_ld();
-        if (store) {
-          float* dkr = a.dk + rowoff + c0;
-          float* dvr = a.dv + rowoff + c0;
-          if constexpr (kColumn) {
-            // 16-byte vector atomics (rows are 512-byte aligned, c0 + e a multiple of 4)
+        const float sc = is_v ? 1.f : a.scale;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              atomicAdd(reinterpret_cast<float4*>(dkr + e),
-                        make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
-                                    __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale));
-              atomicAdd(reinterpret_cast<float4*>(dvr + e),
-                        make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
-                                    __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3])));
-            }
-          } else {
+        for (int j = 0; j < 4; ++j) {
+          const int ch = (4 * half + j) ^ (key_row & 7);
+          *reinterpret_cast<float4*>(sm + k2Stage + key_row * 128 + ch * 16) =
+              make_float4(__uint_as_float(v16[4 * j]) * sc, __uint_as_float(v16[4 * j + 1]) * sc,
+                          __uint_as_float(v16[4 * j + 2]) * sc, __uint_as_float(v16[4 * j + 3]) * sc);
+        }
+        bar_sync(1, 256);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              *reinterpret_cast<float4*>(dkr + e) =
-                  make_float4(__uint_as_float(rk[e]) * a.scale, __uint_as_float(rk[e + 1]) * a.scale,
-                              __uint_as_float(rk[e + 2]) * a.scale, __uint_as_float(rk[e + 3]) * a.scale);
-              *reinterpret_cast<float4*>(dvr + e) =
-                  make_float4(__uint_as_float(rv[e]), __uint_as_float(rv[e + 1]),
-                              __uint_as_float(rv[e + 2]), __uint_as_float(rv[e + 3]));
-            }
+        for (int q = 0; q < 4; ++q) {
+          const int row = q * 32 + (t2 >> 3), p = pos_sh[row];
+          const float4 val =
+              *reinterpret_cast<const float4*>(sm + k2Stage + row * 128 + ((c16 ^ (row & 7)) * 16));
+          if (p >= 0) {
+            float* dst = (is_v ? a.dv : a.dk) + (((long long)b * a.T + p) * a.Hkv + h) * HD + 32 * c + 4 * c16;
+            if constexpr (kColumn) atomicAdd(reinterpret_cast<float4*>(dst), val);
+            else *reinterpret_cast<float4*>(dst) = val;
           }
         }
+        bar_sync(1, 256);                                  // the stage may be overwritten
       }
+      tc_fence_before();                                   // dK, dV read before the next item's K
     }
   }
   tc_fence_before();
@@ -749,12 +947,19 @@ bool attn_backward_dq_tc_supported(const lte_dims* d) {
   return d->D == bwdtc::HD && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
+size_t attn_backward_col_items_cap(const lte_dims* d) {
+  const int G = d->Hq / d->Hkv, TOK = G > 0 && G <= bwdtc::kRowsK2 ? bwdtc::kRowsK2 / G : 1;
+  const long long n_ctiles = ((long long)d->sink + d->T + bwdtc::kKeysKV - 1) / bwdtc::kKeysKV;
+  const long long runs = (((long long)d->T + TOK - 1) / TOK + bwdtc::kSplitRowsK2 - 1) / bwdtc::kSplitRowsK2;
+  return (size_t)d->B * d->Hkv * n_ctiles * runs;
+}
+
 cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
   using namespace bwdtc;
   const int TOK = kRowsK2 / a.G;
   // tensor maps (contiguous bf16 rows of 128; 128-byte swizzle, 64-column boxes;
   // rows past a tensor's end read as zero)
-  CUtensorMap mq, mdo, mk, mv, mkc, mvc;
+  CUtensorMap mq, mdo, mv, mvc;
   {
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
     const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hq * HD * 2, (cuuint64_t)a.T * a.Hq * HD * 2};
@@ -767,16 +972,14 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
     const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hkv * HD * 2,
                               (cuuint64_t)a.T * a.Hkv * HD * 2};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)kKeysKV, 1};
-    if (!encode(&mk, a.k, 4, dims, st, box) || !encode(&mv, a.v, 4, dims, st, box))
-      return cudaErrorInvalidValue;
+    if (!encode(&mv, a.v, 4, dims, st, box)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t rows = (cuuint64_t)a.sink + a.T;
     const cuuint64_t dims[3] = {(cuuint64_t)HD, rows, (cuuint64_t)B * a.Hkv};
     const cuuint64_t st[2] = {(cuuint64_t)HD * 2, rows * HD * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)kKeysKV, 1};
-    if (!encode(&mkc, a.k_col, 3, dims, st, box) || !encode(&mvc, a.v_col, 3, dims, st, box))
-      return cudaErrorInvalidValue;
+    if (!encode(&mvc, a.v_col, 3, dims, st, box)) return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
@@ -784,16 +987,28 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
   e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            k2Smem);
   if (e != cudaSuccess) return e;
-  const int n_ktiles = (a.T + kKeysKV - 1) / kKeysKV;
-  bwd_dkdv_tc_kernel<false><<<dim3(n_ktiles, a.Hkv, B), kThreadsK2, k2Smem, stream>>>(mq, mdo, mk, mv, a,
-                                                                                     1, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  // window part: item = (b, h, key tile)
+  const long long n_win = (long long)((a.T + kKeysKV - 1) / kKeysKV) * a.Hkv * B;
+  if (n_win > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  if (n_win > 0) {
+    const int grid = (int)(n_win < n_sm ? n_win : n_sm);
+    bwd_dkdv_tc_kernel<false><<<grid, kThreadsK2, k2Smem, stream>>>(mq, mdo, mv, a, nullptr, nullptr,
+                                                                   (int)n_win, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // column part: the work list, then one CTA per SM over it
   const int n_ctiles = (a.sink + a.T + kKeysKV - 1) / kKeysKV;
-  const int n_split = ((a.T + TOK - 1) / TOK + kSplitRowsK2 - 1) / kSplitRowsK2;
-  const long long gx = (long long)n_ctiles * n_split;
-  if (gx > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-  bwd_dkdv_tc_kernel<true><<<dim3((unsigned)gx, a.Hkv, B), kThreadsK2, k2Smem, stream>>>(
-      mq, mdo, mkc, mvc, a, n_split, err);
+  const long long units = (long long)B * a.Hkv;
+  if (units == 0 || n_ctiles == 0) return cudaSuccess;
+  if (units > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  int* n_items = reinterpret_cast<int*>(a.col_work);
+  K2Item* items = reinterpret_cast<K2Item*>(static_cast<char*>(a.col_work) + 256);
+  if ((e = cudaMemsetAsync(n_items, 0, sizeof(int), stream)) != cudaSuccess) return e;
+  bwd_col_items_kernel<<<(unsigned)units, kColItemsThreads, 0, stream>>>(a, n_ctiles, items, n_items);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_dkdv_tc_kernel<true><<<n_sm, kThreadsK2, k2Smem, stream>>>(mq, mdo, mvc, a, items, n_items, 0, err);
   return cudaGetLastError();
 }
 

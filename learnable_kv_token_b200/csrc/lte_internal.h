@@ -97,6 +97,7 @@ namespace bwd { struct Args; }
 bool attn_backward_dq_tc_supported(const lte_dims* d);
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream);
 cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream);
+size_t attn_backward_col_items_cap(const lte_dims* d);   // work items the column pass may list
 
 // decode.cu
 size_t decode_scratch_bytes(const lte_dims* d);
