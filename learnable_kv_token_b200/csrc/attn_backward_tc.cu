@@ -397,49 +397,45 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // per row tile:
 //   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM
 //   P^T, dS^T = P^T (dP^T - D)         (two threads per key row, 32 rows each)
-//                                      into TMEM, as bf16
+//                                      into TMEM buffer (tile % 2), as bf16
 //   dV += P^T dO, dK += dS^T Q         (M128 N128 K64; P^T, dS^T read from TMEM)
-// K sits in TMEM (bf16 pairs) as the A operand of S^T and V in shared memory,
-// so that the shared-memory operand reads of a row tile (Q and dO twice each,
-// V once) stay within what the tensor core's full rate needs.
+// The tensor core runs its products in issue order, so the schedule keeps any
+// product from waiting behind one that waits for the rows: S^T of a tile is
+// issued as soon as the rows have read the S^T before it (one S^T buffer), dV
+// and dK of the tile before once its P^T and dS^T are written, and those have
+// two buffers, so the rows never wait for dV and dK.
 // Roles (384 threads):
-//   warp 0     TMA producer (one elected lane): V of each item into one of two
-//              buffers, once the products of the item before last are done; per
-//              row tile, Q and dO into
-//              a 4-stage ring, then the rows' lse, D, token and retained range,
-//              written by the warp's lanes while the copies fly;
-//   warp 1     MMA issuer: S^T and dP^T of a row tile as soon as the rows have
-//              read those of the tile before, then dV and dK of the tile before
-//              once its P^T and dS^T are written -- the tensor core computes
-//              S^T of the next tile while the rows of this one are formed;
+//   warp 0     TMA producer (one elected lane): K and V of each item, once the
+//              item before has issued its last S^T and that has completed; per
+//              row tile, Q and dO into a 4-stage ring, then the rows' lse and D
+//              and the tokens' retained range, written by the warp's lanes
+//              while the copies fly;
+//   warp 1     MMA issuer, as above;
 //   warps 4-11 two threads per key row (warps 4-7 rows 0-31 of a tile, 8-11
-//              rows 32-63): K of each item into TMEM (loaded while the item
-//              before finishes); P^T and dS^T, written once dV and dK of the
-//              tile before have read theirs; at the end of an item, dK and dV
-//              out through a shared-memory stage in 32-column chunks, so that
-//              each warp store (or add) covers four whole 128-byte rows.
-// TMEM: S^T 0..63, dP^T 64..127, P^T 128..159 and dS^T 160..191 (64 bf16 rows
-// packed in pairs), K 192..255, dV 256..383, dK 384..511.  Barrier phases run
-// on a row-tile counter that continues across items (ring stages, S, P) or on
-// the item counter (V buffers and the items' completion: one barrier each per
-// buffer, K).
+//              rows 32-63): P^T and dS^T; at the end of an item, dK and dV out
+//              through a shared-memory stage in 32-column chunks, so that each
+//              warp store (or add) covers four whole 128-byte rows, while the
+//              tensor core already computes the next item's first S^T.
+// TMEM: S^T 0..63, dP^T 64..127, P^T and dS^T of buffer x at 128 + 64 x and
+// 160 + 64 x (64 bf16 rows packed in pairs), dV 256..383, dK 384..511.
+// Barrier phases run on a row-tile counter that continues across items (ring
+// stages, S^T, P^T buffers) or on the item counter (K and V, items' completion).
 constexpr int kKeysKV = 128;
 constexpr int kRowsK2 = 64;                       // attending query rows per tile
 constexpr int kStagesK2 = 4;
 constexpr int kThreadsK2 = 384;
 constexpr int kSplitRowsK2 = 32;                  // row tiles per column item, at most
-constexpr uint32_t k2V = 0;                       // 2 x [128][128] bf16: halves of 16 KiB
+constexpr uint32_t k2K = 0, k2V = 32768;          // [128][128] bf16 each: halves of 16 KiB
 constexpr uint32_t k2QD = 65536;                  // stage s: Q at + 32 KiB s, dO at + 16 KiB
 constexpr uint32_t k2Meta = k2QD + kStagesK2 * 32768;            // stage s: [5][64] words
 constexpr uint32_t k2Stage = k2Meta + kStagesK2 * 5 * kRowsK2 * 4;   // [128][32] fp32, swizzled
 constexpr uint32_t k2Pos = k2Stage + kKeysKV * 128;                  // [128] output row per key
 constexpr uint32_t k2Bar = k2Pos + kKeysKV * 4;
 constexpr int k2Smem = k2Bar + 256;
-constexpr uint32_t k2ColS = 0, k2ColDP = 64, k2ColP = 128, k2ColDS = 160, k2ColK = 192, k2ColDV = 256,
-                   k2ColDK = 384;
+constexpr uint32_t k2ColS = 0, k2ColDP = 64, k2ColP = 128, k2ColDV = 256, k2ColDK = 384;
 enum {
-  K2_KVF = 0, K2_F = 2, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_SE = K2_SF + 1,
-  K2_PF = K2_SE + 1, K2_PE = K2_PF + 1, K2_KT = K2_PE + 1, K2_DONE = K2_KT + 1, kNumBarsK2 = K2_DONE + 2
+  K2_KVF = 0, K2_KVE = 1, K2_F = 2, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_SE = K2_SF + 1,
+  K2_PF = K2_SE + 1, K2_PE = K2_PF + 2, K2_DONE = K2_PE + 2, kNumBarsK2 = K2_DONE + 1
 };
 static_assert(8 * kNumBarsK2 + 16 <= 256, "barriers and flags fit");
 static_assert(k2Smem <= 227 * 1024, "shared memory fits one CTA");
@@ -552,7 +548,8 @@ bwd_col_items_kernel(const bwd::Args a, int n_ctiles, K2Item* items, int* n_item
 template <bool kColumn>
 __global__ void __launch_bounds__(kThreadsK2, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_v, const bwd::Args a, const K2Item* items,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const bwd::Args a, const K2Item* items,
                    const int* n_items_p, int n_items_win, DevError* err) {
   extern __shared__ __align__(1024) uint8_t sm[];
   const uint32_t sb = sa(sm);
@@ -590,18 +587,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (tid == 0) {
     mbar_init(bar(K2_KVF), 1);
-    mbar_init(bar(K2_KVF + 1), 1);
+    mbar_init(bar(K2_KVE), 1);
     for (int st = 0; st < kStagesK2; ++st) {
       mbar_init(bar(K2_F + st), 1);
       mbar_init(bar(K2_E + st), 1);
     }
     mbar_init(bar(K2_SF), 1);
     mbar_init(bar(K2_SE), 256);
-    mbar_init(bar(K2_PF), 256);
-    mbar_init(bar(K2_PE), 1);
-    mbar_init(bar(K2_KT), 256);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(K2_PF + x), 256);
+      mbar_init(bar(K2_PE + x), 1);
+    }
     mbar_init(bar(K2_DONE), 1);
-    mbar_init(bar(K2_DONE + 1), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -625,15 +622,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const K2Item w = item_at(it);
       const int h = w.u % a.Hkv, b = w.u / a.Hkv, k0 = w.tile * kKeysKV;
       const long long crow = (long long)w.u * a.T;
-      // V into buffer k % 2: the products of item k - 2 have all completed
-      const int vb = k & 1;
-      if (k >= 2 && !(ok = wwait(bar(K2_DONE + vb), ((k - 2) >> 1) & 1, abort_flag, err, 424))) break;
+      // K and V: the previous item's last S^T, dP^T have completed
+      if (k >= 1 && !(ok = wwait(bar(K2_KVE), (k - 1) & 1, abort_flag, err, 424))) break;
       if (elect_one()) {
-        const uint32_t vs = sb + k2V + (uint32_t)vb * 32768u;
-        mbar_expect_tx(bar(K2_KVF + vb), kKeysKV * HD * 2);
+        mbar_expect_tx(bar(K2_KVF), 2 * kKeysKV * HD * 2);
         for (int hf = 0; hf < 2; ++hf) {
-          if constexpr (kColumn) tma_load_3d(vs + hf * 16384u, &tm_v, bar(K2_KVF + vb), hf * 64, k0, w.u);
-          else tma_load_4d(vs + hf * 16384u, &tm_v, bar(K2_KVF + vb), hf * 64, h, k0, b);
+          if constexpr (kColumn) {
+            tma_load_3d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, k0, w.u);
+            tma_load_3d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, k0, w.u);
+          } else {
+            tma_load_4d(sb + k2K + hf * 16384u, &tm_k, bar(K2_KVF), hf * 64, h, k0, b);
+            tma_load_4d(sb + k2V + hf * 16384u, &tm_v, bar(K2_KVF), hf * 64, h, k0, b);
+          }
         }
       }
       __syncwarp();
@@ -688,7 +688,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
     }
     // every issued copy has landed before the CTA may exit
-    for (int q = k - 2 > 0 ? k - 2 : 0; q < k; ++q) mbar_drain(bar(K2_KVF + (q & 1)), (q >> 1) & 1);
+    if (k >= 1) mbar_drain(bar(K2_KVF), (k - 1) & 1);
     for (int q = g - kStagesK2 > 0 ? g - kStagesK2 : 0; q < g; ++q)
       mbar_drain(bar(K2_F + q % kStagesK2), (q / kStagesK2) & 1);
   } else if (warp == 1) {
@@ -697,31 +697,29 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t id_o = idesc(kKeysKV, HD, true);          // dV, dK: dO, Q as N-contiguous B
     bool ok = true;
     auto issue_dvdk = [&](int gg, bool first) -> bool {      // dV, dK of row tile gg
-      const int st = gg % kStagesK2;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(K2_PF), gg & 1, abort_flag, err, 416))) return false;
+      const int st = gg % kStagesK2, x = gg & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(K2_PF + x), (gg >> 1) & 1, abort_flag, err, 416))) return false;
       tc_fence_after();
       if (elect_one()) {
         const uint32_t qs = sb + k2QD + st * 32768u;
         const uint64_t qb = sdesc(qs, kRowsK2 * 128, 1024), dob = sdesc(qs + 16384u, kRowsK2 * 128, 1024);
+        const uint32_t pb = tmem + k2ColP + (uint32_t)(64 * x);
 #pragma unroll
         for (int ks = 0; ks < kRowsK2 / 16; ++ks) {
           const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
-          mma_f16_ts(tmem + k2ColDV, tmem + k2ColP + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
-          mma_f16_ts(tmem + k2ColDK, tmem + k2ColDS + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + k2ColDV, pb + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + k2ColDK, pb + 32 + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
         }
         mma_commit(bar(K2_E + st));                          // the row tile's stage is free
-        mma_commit(bar(K2_PE));                              // P^T, dS^T may be overwritten
+        mma_commit(bar(K2_PE + x));                          // P^T, dS^T buffer x is free
       }
       __syncwarp();
       return true;
     };
     int g = 0, k = 0;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
-      const int n_rt = item_at(it).n_rt, vb = k & 1;
-      // V landed; K in TMEM (and the previous item's dK, dV read out)
-      ok = mbar_wait(bar(K2_KVF + vb), (k >> 1) & 1, abort_flag, err, 415);
-      if (ok) ok = mbar_wait(bar(K2_KT), k & 1, abort_flag, err, 422);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      const int n_rt = item_at(it).n_rt;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_KVF), k & 1, abort_flag, err, 415)))) break;
       for (int i = 0; i < n_rt; ++i, ++g) {
         const int st = g % kStagesK2;
         ok = mbar_wait(bar(K2_F + st), (g / kStagesK2) & 1, abort_flag, err, 417);
@@ -731,52 +729,31 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tc_fence_after();
         if (elect_one()) {
           const uint32_t qs = sb + k2QD + st * 32768u;
-          const uint64_t dv = sdesc(sb + k2V + (uint32_t)vb * 32768u, 16, 1024);
+          const uint64_t dk = sdesc(sb + k2K, 16, 1024), dv = sdesc(sb + k2V, 16, 1024);
           const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
 #pragma unroll
           for (int ks = 0; ks < HD / 16; ++ks) {
             const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
             const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
-            mma_f16_ts(tmem + k2ColS, tmem + k2ColK + 8 * ks, dq + ob, id_s, ks > 0 ? 1u : 0u);
+            mma_f16(tmem + k2ColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
             mma_f16(tmem + k2ColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
           }
           mma_commit(bar(K2_SF));
+          if (i == n_rt - 1) mma_commit(bar(K2_KVE));        // K, V no longer read
         }
         __syncwarp();
         if (i >= 1 && !(ok = issue_dvdk(g - 1, i == 1))) break;
       }
       if (ok) ok = issue_dvdk(g - 1, n_rt == 1);
-      if (elect_one()) mma_commit(bar(K2_DONE + vb));      // every product of the item has completed
+      if (elect_one()) mma_commit(bar(K2_DONE));           // every product of the item has completed
       __syncwarp();
     }
-    if (k >= 1) mbar_drain(bar(K2_DONE + ((k - 1) & 1)), ((k - 1) >> 1) & 1);
+    if (k >= 1) mbar_drain(bar(K2_DONE), (k - 1) & 1);
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- key rows (warps 4-11)
     const int quad = warp & 3, half = (warp - 4) >> 2;     // TMEM lane quadrant, row half
     const int key_row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    // K of item `it`: this thread's key row, dims [64 half, 64 half + 64) as bf16
-    // pairs (zeros past the tile's keys)
-    uint32_t kr[32];
-    auto load_k = [&](int it) {
-      const K2Item w = item_at(it);
-      const int kpos = w.tile * kKeysKV + key_row;
-      if (key_row < keys_of(w)) {
-        const __nv_bfloat16* src =
-            kColumn ? a.k_col + ((long long)w.u * (a.sink + a.T) + kpos) * HD
-                    : a.k + (((long long)(w.u / a.Hkv) * a.T + kpos) * a.Hkv + w.u % a.Hkv) * HD;
-        const uint4* s4 = reinterpret_cast<const uint4*>(src + 64 * half);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v4 = __ldg(s4 + c);
-          kr[4 * c] = v4.x, kr[4 * c + 1] = v4.y, kr[4 * c + 2] = v4.z, kr[4 * c + 3] = v4.w;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) kr[c] = 0u;
-      }
-    };
-    load_k(blockIdx.x);
     bool ok = true;
     int g = 0, k = 0;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
@@ -791,12 +768,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       // and the partial sum of dS over the rows this thread sees, for dL/dr
       float bk2 = 0.f, dr_acc = 0.f;
       if (kColumn && a.bias != nullptr && key_row < nk) bk2 = __ldg(a.bias + col_base + kpos) * a.scale_log2;
-      // K (loaded into registers before) into TMEM.  The previous item's S^T
-      // products are done (its last tile's S^T was read) and its dK, dV read out.
-      tmem_st32(lane_addr + k2ColK + 32 * half, kr);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(K2_KT));
       for (int i = 0; i < w.n_rt; ++i, ++g) {
         const int st = g % kStagesK2;
         // the row data first: the rows' range is found while S^T is computed
@@ -866,20 +837,20 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           pd[2 * c4] = pk2(q4[0], q4[1]);
           pd[2 * c4 + 1] = pk2(q4[2], q4[3]);
         }
-        // dV, dK of the tile before have read its P^T, dS^T
-        if (g >= 1 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_PE), (g - 1) & 1, abort_flag, err, 423))))
+        // dV, dK of tile g - 2 have read P^T, dS^T buffer g % 2
+        const int x = g & 1;
+        if (g >= 2 &&
+            !(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_PE + x), ((g - 2) >> 1) & 1, abort_flag, err, 423))))
           break;
         tc_fence_after();
-        // rows 32 half .. + 31 of P^T, dS^T: columns 16 half .. + 15
-        tmem_st16(lane_addr + k2ColP + (uint32_t)(16 * half), pp);
-        tmem_st16(lane_addr + k2ColDS + (uint32_t)(16 * half), pd);
+        // rows 32 half .. + 31 of P^T, dS^T: columns 16 half .. + 15 of the buffer
+        tmem_st16(lane_addr + k2ColP + (uint32_t)(64 * x + 16 * half), pp);
+        tmem_st16(lane_addr + k2ColP + (uint32_t)(64 * x + 32 + 16 * half), pd);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(K2_PF));
+        mbar_arrive(bar(K2_PF + x));
       }
-      // the next item's K into registers while this item's products finish
-      if (ok && it + (int)gridDim.x < n_items) load_k(it + gridDim.x);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_DONE + (k & 1)), (k >> 1) & 1, abort_flag, err, 420));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_DONE), k & 1, abort_flag, err, 420));
       // the eight row warps go on together or stop together (the stage below
       // synchronises them with a named barrier)
       if (!(ok = bar_and(1, 256, ok))) break;
@@ -929,7 +900,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         bar_sync(1, 256);                                  // the stage may be overwritten
       }
-      tc_fence_before();                                   // dK, dV read before the next item's K
+      tc_fence_before();                                   // dK, dV read before the next item's products
     }
   }
   tc_fence_before();
@@ -959,7 +930,7 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
   const int TOK = kRowsK2 / a.G;
   // tensor maps (contiguous bf16 rows of 128; 128-byte swizzle, 64-column boxes;
   // rows past a tensor's end read as zero)
-  CUtensorMap mq, mdo, mv, mvc;
+  CUtensorMap mq, mdo, mk, mv, mkc, mvc;
   {
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
     const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hq * HD * 2, (cuuint64_t)a.T * a.Hq * HD * 2};
@@ -972,14 +943,15 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
     const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hkv * HD * 2,
                               (cuuint64_t)a.T * a.Hkv * HD * 2};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)kKeysKV, 1};
-    if (!encode(&mv, a.v, 4, dims, st, box)) return cudaErrorInvalidValue;
+    if (!encode(&mk, a.k, 4, dims, st, box) || !encode(&mv, a.v, 4, dims, st, box)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t rows = (cuuint64_t)a.sink + a.T;
     const cuuint64_t dims[3] = {(cuuint64_t)HD, rows, (cuuint64_t)B * a.Hkv};
     const cuuint64_t st[2] = {(cuuint64_t)HD * 2, rows * HD * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)kKeysKV, 1};
-    if (!encode(&mvc, a.v_col, 3, dims, st, box)) return cudaErrorInvalidValue;
+    if (!encode(&mkc, a.k_col, 3, dims, st, box) || !encode(&mvc, a.v_col, 3, dims, st, box))
+      return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
@@ -994,7 +966,7 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
   if (n_win > 0x7fffffffll) return cudaErrorInvalidConfiguration;
   if (n_win > 0) {
     const int grid = (int)(n_win < n_sm ? n_win : n_sm);
-    bwd_dkdv_tc_kernel<false><<<grid, kThreadsK2, k2Smem, stream>>>(mq, mdo, mv, a, nullptr, nullptr,
+    bwd_dkdv_tc_kernel<false><<<grid, kThreadsK2, k2Smem, stream>>>(mq, mdo, mk, mv, a, nullptr, nullptr,
                                                                    (int)n_win, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1008,7 +980,7 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
   if ((e = cudaMemsetAsync(n_items, 0, sizeof(int), stream)) != cudaSuccess) return e;
   bwd_col_items_kernel<<<(unsigned)units, kColItemsThreads, 0, stream>>>(a, n_ctiles, items, n_items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_dkdv_tc_kernel<true><<<n_sm, kThreadsK2, k2Smem, stream>>>(mq, mdo, mvc, a, items, n_items, 0, err);
+  bwd_dkdv_tc_kernel<true><<<n_sm, kThreadsK2, k2Smem, stream>>>(mq, mdo, mkc, mvc, a, items, n_items, 0, err);
   return cudaGetLastError();
 }
 
