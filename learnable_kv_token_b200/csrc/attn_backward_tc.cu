@@ -26,6 +26,8 @@
 // what it issued, frees its TMEM and leaves.
 #include <math.h>
 
+#include <type_traits>
+
 #include "attn_backward.cuh"
 #include "lte_common.cuh"
 #include "lte_internal.h"
@@ -40,8 +42,6 @@ constexpr int HD = 128;
 constexpr int kRowsTc = 128;                    // query rows per CTA
 constexpr int kKeysTc = 64;                     // keys per tile
 constexpr int kThreadsTc = 128;
-constexpr uint32_t kQ = 0;                      // [128][128] bf16: two 64-column halves of 16 KiB
-constexpr uint32_t kDO = 32768;                 // same for dO
 constexpr uint32_t kK = 65536;                  // [64][128]: two halves of 8 KiB
 constexpr uint32_t kV = 81920;
 constexpr uint32_t kDS = 98304;                 // [128][64] bf16 (one half)
@@ -75,32 +75,43 @@ __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Pipelined roles (256 threads, one CTA per SM):
-//   warp 0     TMA copies (one elected lane): Q and dO once, then K and V of key
-//              tile j into ring stage j % 3 (128-byte swizzled 64-column halves;
-//              rows past the tensor read as zero);
-//   warp 1     issues, per tile j: S(j), dP(j) into TMEM buffer j % 2, then
-//              dQ += dS(j-1) K(j-1) once dS(j-1) is in shared memory -- so the
-//              tensor core computes tile j's products while the rows of tile
-//              j - 1 are being formed;
+// Roles (384 threads, one CTA per SM), per key tile j of the CTA's rows:
+//   warp 0     TMA copies (one elected lane): K of tile j into a 7-stage ring
+//              and V into a 4-stage ring (128-byte swizzled 64-column halves;
+//              rows past the tensor read as zero) -- V is free once S(j), dP(j)
+//              have completed, K only once dQ += dS(j) K(j) has;
+//   warp 1     MMA issuer: S(j), dP(j) into TMEM buffer j % 2 (Q and dO are A
+//              operands from TMEM), issued two tiles ahead of the rows, and
+//              dQ += dS(j) K(j) once dS(j) is in shared memory: per rows' tile
+//              r it issues dQ(r - 1) and then S(r + 2), so no S waits in the
+//              tensor core's in-order queue behind a product that waits for
+//              the rows;
 //   warps 4-11 two threads per query row (warps 4-7 the first 32 keys of a
-//              tile, 8-11 the last 32): P and dS of tile j from TMEM buffer
-//              j % 2 into the shared dS buffer j % 2; at the end, dQ out (64
-//              of the 128 columns each).  Two warps per sub-partition hide
-//              each other's TMEM and special-function latency.
-// TMEM: S[2] 0..127, dP[2] 128..255, dQ 256..383.
+//              tile, 8-11 the last 32): Q and dO into TMEM at the start; P and
+//              dS of tile j from TMEM buffer j % 2 (released as soon as read)
+//              into the shared dS buffer j % 2; at the end, dQ out through a
+//              shared-memory stage, whole 512-byte rows per warp store.
+// TMEM: S[2] 0..127, dP[2] 128..255, dQ 256..383, Q 384..447, dO 448..511
+// (bf16 pairs).
 constexpr int kThreadsP = 384;
-constexpr int kStagesP = 3;                             // K/V ring
-constexpr uint32_t kK2 = 65536;                         // stage s: K at + 32 KiB s, V at + 16 KiB
-constexpr uint32_t kDS2 = kK2 + kStagesP * 32768;       // dS buffers: 2 x [128][64] bf16
+constexpr int kStagesKP = 7, kStagesVP = 4;            // K and V rings
+constexpr uint32_t kKR = 0;                             // K stage s at 16 KiB s
+constexpr uint32_t kVR = kKR + kStagesKP * 16384;       // V stage s at 16 KiB s
+constexpr uint32_t kDS2 = kVR + kStagesVP * 16384;      // dS buffers: 2 x [128][64] bf16
 constexpr uint32_t kBar2 = kDS2 + 2 * 16384;            // barriers
-constexpr int kSmemP = kBar2 + 256;
-constexpr uint32_t kColSP = 0, kColDPP = 128, kColDQP = 256;
+constexpr int kSmemP = kBar2 + 512;
+constexpr uint32_t kColSP = 0, kColDPP = 128, kColDQP = 256, kColQP = 384, kColDOP = 448;
+constexpr int kQStage = 3;                              // Q, dO arrive in K stages 3..6
+constexpr uint32_t kQS = kKR + kQStage * 16384;         // Q [128][128] bf16 (32 KiB), then dO
+static_assert(kQStage * 16384 + 65536 <= kStagesKP * 16384, "Q and dO fit the K ring's tail");
 enum {
-  P_QF = 0, P_KVF = 1, P_KVE = P_KVF + kStagesP, P_SF = P_KVE + kStagesP, P_SE = P_SF + 2,
-  P_DSF = P_SE + 2, P_DSE = P_DSF + 2, P_DQ = P_DSE + 2, kNumBarsP = P_DQ + 1
+  P_QF = 0, P_QT = 1, P_KF = 2, P_KE = P_KF + kStagesKP, P_VF = P_KE + kStagesKP, P_VE = P_VF + kStagesVP,
+  P_SF = P_VE + kStagesVP, P_SE = P_SF + 2, P_DSF = P_SE + 2, P_DSE = P_DSF + 2, P_DQ = P_DSE + 2,
+  kNumBarsP = P_DQ + 1
 };
-static_assert(8 * kNumBarsP + 8 <= 256, "barriers fit");
+static_assert(8 * kNumBarsP + 8 <= 512, "barriers fit");
+static_assert(kSmemP <= 227 * 1024, "shared memory fits one CTA");
+static_assert(kStagesKP * 16384 >= kRowsTc * HD * 4, "the K ring holds the dQ stage");
 
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -128,9 +139,14 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   if (tid == 0) {
     mbar_init(bar(P_QF), 1);
-    for (int x = 0; x < kStagesP; ++x) {
-      mbar_init(bar(P_KVF + x), 1);
-      mbar_init(bar(P_KVE + x), 1);
+    mbar_init(bar(P_QT), 256);
+    for (int x = 0; x < kStagesKP; ++x) {
+      mbar_init(bar(P_KF + x), 1);
+      mbar_init(bar(P_KE + x), 1);
+    }
+    for (int x = 0; x < kStagesVP; ++x) {
+      mbar_init(bar(P_VF + x), 1);
+      mbar_init(bar(P_VE + x), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(P_SF + x), 1);
@@ -155,7 +171,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t tmem = *tmem_slot;
 
   // key ranges of the tile: 0 sink slots, 1 retained slots, 2 window band
-  int start[3], count[3];
+  int start0, count0, start1, count1, start2, count2;
   {
     int lo_f, n_first, lo_l, n_last;
     bwd::row_range(a, crow, t0, lo_f, n_first);
@@ -165,48 +181,53 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     nsink = nsink < 0 ? 0 : (nsink > a.sink ? a.sink : nsink);
     nsink = nsink > a.T ? a.T : nsink;
     const int w_lo = t0 - a.window + 1 > 0 ? t0 - a.window + 1 : 0;
-    start[0] = 0; count[0] = nsink;
-    start[1] = a.sink + lo_min; count[1] = (a.cap > 0 && n_last > lo_min) ? n_last - lo_min : 0;
-    start[2] = w_lo; count[2] = t_last - w_lo + 1;
+    start0 = 0; count0 = nsink;
+    start1 = a.sink + lo_min; count1 = (a.cap > 0 && n_last > lo_min) ? n_last - lo_min : 0;
+    start2 = w_lo; count2 = t_last - w_lo + 1;
   }
-  const int n0 = (count[0] + kKeysTc - 1) / kKeysTc, n1 = (count[1] + kKeysTc - 1) / kKeysTc;
-  const int total = n0 + n1 + (count[2] + kKeysTc - 1) / kKeysTc;
-  auto tile_of = [&](int j, int& rg, int& key0, int& nk) {
-    int it = j;
-    if (it < n0) rg = 0;
-    else if (it < n0 + n1) { rg = 1; it -= n0; }
-    else { rg = 2; it -= n0 + n1; }
-    key0 = start[rg] + it * kKeysTc;
-    nk = min(kKeysTc, count[rg] - it * kKeysTc);
+  const int n0 = (count0 + kKeysTc - 1) / kKeysTc, n1 = (count1 + kKeysTc - 1) / kKeysTc;
+  const int total = n0 + n1 + (count2 + kKeysTc - 1) / kKeysTc;
+  auto tile_of = [&](int j, int& rg, int& key0, int& nk) {   // (registers only)
+    rg = j < n0 ? 0 : (j < n0 + n1 ? 1 : 2);
+    const int it = j - (rg == 0 ? 0 : (rg == 1 ? n0 : n0 + n1));
+    const int st_ = rg == 0 ? start0 : (rg == 1 ? start1 : start2);
+    const int ct_ = rg == 0 ? count0 : (rg == 1 ? count1 : count2);
+    key0 = st_ + it * kKeysTc;
+    nk = min(kKeysTc, ct_ - it * kKeysTc);
   };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     bool ok = true;
+    // Q and dO into K-ring stages kQStage .. (free until the rows have moved them
+    // into TMEM)
     if (elect_one()) {
       mbar_expect_tx(bar(P_QF), 2 * kRowsTc * HD * 2);
       for (int hf = 0; hf < 2; ++hf) {
-        tma_load_4d(sb + kQ + hf * (kRowsTc * 128), &tm_q, bar(P_QF), hf * 64, h * G, t0, b);
-        tma_load_4d(sb + kDO + hf * (kRowsTc * 128), &tm_do, bar(P_QF), hf * 64, h * G, t0, b);
+        tma_load_4d(sb + kQS + hf * (kRowsTc * 128), &tm_q, bar(P_QF), hf * 64, h * G, t0, b);
+        tma_load_4d(sb + kQS + 32768u + hf * (kRowsTc * 128), &tm_do, bar(P_QF), hf * 64, h * G, t0, b);
       }
     }
     __syncwarp();
     int issued = 0;
     for (int j = 0; j < total && ok; ++j) {
-      const int st = j % kStagesP, use = j / kStagesP;
-      if (use >= 1 && !(ok = wwait(bar(P_KVE + st), (use - 1) & 1, abort_flag, err, 404))) break;
+      const int sk = j % kStagesKP, sv = j % kStagesVP;
+      if (j >= kStagesKP && !(ok = wwait(bar(P_KE + sk), (j / kStagesKP - 1) & 1, abort_flag, err, 404))) break;
+      if (j >= kQStage && j < kStagesKP && !(ok = wwait(bar(P_QT), 0, abort_flag, err, 414))) break;
+      if (j >= kStagesVP && !(ok = wwait(bar(P_VE + sv), (j / kStagesVP - 1) & 1, abort_flag, err, 412))) break;
       int rg, key0, nk;
       tile_of(j, rg, key0, nk);
       if (elect_one()) {
-        const uint32_t kd = sb + kK2 + st * 32768u, vd = kd + 16384u;
-        mbar_expect_tx(bar(P_KVF + st), 2 * kKeysTc * HD * 2);
+        const uint32_t kd = sb + kKR + sk * 16384u, vd = sb + kVR + sv * 16384u;
+        mbar_expect_tx(bar(P_KF + sk), kKeysTc * HD * 2);
+        mbar_expect_tx(bar(P_VF + sv), kKeysTc * HD * 2);
         for (int hf = 0; hf < 2; ++hf) {
           if (rg == 2) {
-            tma_load_4d(kd + hf * (kKeysTc * 128), &tm_k, bar(P_KVF + st), hf * 64, h, key0, b);
-            tma_load_4d(vd + hf * (kKeysTc * 128), &tm_v, bar(P_KVF + st), hf * 64, h, key0, b);
+            tma_load_4d(kd + hf * (kKeysTc * 128), &tm_k, bar(P_KF + sk), hf * 64, h, key0, b);
+            tma_load_4d(vd + hf * (kKeysTc * 128), &tm_v, bar(P_VF + sv), hf * 64, h, key0, b);
           } else {
-            tma_load_3d(kd + hf * (kKeysTc * 128), &tm_kc, bar(P_KVF + st), hf * 64, key0, u);
-            tma_load_3d(vd + hf * (kKeysTc * 128), &tm_vc, bar(P_KVF + st), hf * 64, key0, u);
+            tma_load_3d(kd + hf * (kKeysTc * 128), &tm_kc, bar(P_KF + sk), hf * 64, key0, u);
+            tma_load_3d(vd + hf * (kKeysTc * 128), &tm_vc, bar(P_VF + sv), hf * 64, key0, u);
           }
         }
       }
@@ -215,53 +236,61 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     // every issued copy has landed before the CTA may exit
     mbar_drain(bar(P_QF), 0);
-    for (int q = issued - kStagesP > 0 ? issued - kStagesP : 0; q < issued; ++q)
-      mbar_drain(bar(P_KVF + q % kStagesP), (q / kStagesP) & 1);
+    for (int q = issued - kStagesKP > 0 ? issued - kStagesKP : 0; q < issued; ++q)
+      mbar_drain(bar(P_KF + q % kStagesKP), (q / kStagesKP) & 1);
+    for (int q = issued - kStagesVP > 0 ? issued - kStagesVP : 0; q < issued; ++q)
+      mbar_drain(bar(P_VF + q % kStagesVP), (q / kStagesVP) & 1);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t id_s = idesc(kRowsTc, kKeysTc, false);     // S, dP: K-major A and B
     const uint32_t id_q = idesc(kRowsTc, HD, true);           // dQ: K as an N-contiguous B
-    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QF), 0, abort_flag, err, 405));
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QT), 0, abort_flag, err, 405));
+    auto issue_s = [&](int j) -> bool {                       // S(j), dP(j) into buffer j % 2
+      const int x = j & 1, sk = j % kStagesKP, sv = j % kStagesVP;
+      bool w = mbar_wait(bar(P_KF + sk), (j / kStagesKP) & 1, abort_flag, err, 407);
+      if (w) w = mbar_wait(bar(P_VF + sv), (j / kStagesVP) & 1, abort_flag, err, 413);
+      // the rows have read S, dP of tile j - 2
+      if (w && j >= 2) w = mbar_wait(bar(P_SE + x), ((j - 2) >> 1) & 1, abort_flag, err, 408);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dk = sdesc(sb + kKR + sk * 16384u, 16, 1024);
+        const uint64_t dv = sdesc(sb + kVR + sv * 16384u, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t ob = ((ks >> 2) * (kKeysTc * 128) + (ks & 3) * 32) >> 4;
+          mma_f16_ts(tmem + kColSP + x * 64, tmem + kColQP + 8 * ks, dk + ob, id_s, ks > 0 ? 1u : 0u);
+          mma_f16_ts(tmem + kColDPP + x * 64, tmem + kColDOP + 8 * ks, dv + ob, id_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(P_SF + x));
+        mma_commit(bar(P_VE + sv));                           // V of tile j is free
+      }
+      __syncwarp();
+      return true;
+    };
     auto issue_dq = [&](int jj) -> bool {                     // dQ += dS(jj) K(jj)
-      const int x = jj & 1;
+      const int x = jj & 1, sk = jj % kStagesKP;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(P_DSF + x), (jj >> 1) & 1, abort_flag, err, 406)))
         return false;
       tc_fence_after();
       if (elect_one()) {
         const uint64_t dds = sdesc(sb + kDS2 + x * 16384u, 16, 1024);
-        const uint64_t dkb = sdesc(sb + kK2 + (jj % kStagesP) * 32768u, kKeysTc * 128, 1024);
+        const uint64_t dkb = sdesc(sb + kKR + sk * 16384u, kKeysTc * 128, 1024);
 #pragma unroll
         for (int ks = 0; ks < kKeysTc / 16; ++ks)
           mma_f16(tmem + kColDQP, dds + ((ks * 32) >> 4), dkb + ((ks * 2048) >> 4), id_q,
                   (jj > 0 || ks > 0) ? 1u : 0u);
         mma_commit(bar(P_DSE + x));                           // dS buffer x is free
-        mma_commit(bar(P_KVE + jj % kStagesP));               // K, V of tile jj are free
+        mma_commit(bar(P_KE + sk));                           // K of tile jj is free
       }
       __syncwarp();
       return true;
     };
-    for (int j = 0; j < total && ok; ++j) {
-      const int x = j & 1, use = j >> 1, st = j % kStagesP;
-      ok = mbar_wait(bar(P_KVF + st), (j / kStagesP) & 1, abort_flag, err, 407);
-      if (ok && use >= 1) ok = mbar_wait(bar(P_SE + x), (use - 1) & 1, abort_flag, err, 408);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t dq_ = sdesc(sb + kQ, 16, 1024), ddo = sdesc(sb + kDO, 16, 1024);
-        const uint64_t dk = sdesc(sb + kK2 + st * 32768u, 16, 1024);
-        const uint64_t dv = sdesc(sb + kK2 + st * 32768u + 16384u, 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < HD / 16; ++ks) {
-          const uint32_t oa = ((ks >> 2) * (kRowsTc * 128) + (ks & 3) * 32) >> 4;
-          const uint32_t ob = ((ks >> 2) * (kKeysTc * 128) + (ks & 3) * 32) >> 4;
-          mma_f16(tmem + kColSP + x * 64, dq_ + oa, dk + ob, id_s, ks > 0 ? 1u : 0u);
-          mma_f16(tmem + kColDPP + x * 64, ddo + oa, dv + ob, id_s, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(P_SF + x));
-      }
-      __syncwarp();
-      if (j >= 1 && !(ok = issue_dq(j - 1))) break;
+    if (ok && total > 0) ok = issue_s(0);
+    if (ok && total > 1) ok = issue_s(1);
+    for (int r = 0; r < total && ok; ++r) {
+      if (r >= 1) ok = issue_dq(r - 1);
+      if (ok && r + 2 < total) ok = issue_s(r + 2);
     }
     if (ok && total > 0) ok = issue_dq(total - 1);
     if (elect_one()) mma_commit(bar(P_DQ));                   // every product above has completed
@@ -276,6 +305,26 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int row = quad * 32 + (tid & 31);
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int tt = t0 + row / G, gq = row % G;
+    // Q and dO of this row, dims [64 kh, 64 kh + 64), from their 128-byte swizzled
+    // halves in shared memory (zeros past T, as the copy fills them) into TMEM
+    bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QF), 0, abort_flag, err, 415));
+    if (ok) {
+      uint32_t rq[32], rd[32];
+      const uint8_t* qrow = sm + kQS + kh * (kRowsTc * 128) + row * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int off = (c ^ (row & 7)) << 4;
+        const uint4 vq = *reinterpret_cast<const uint4*>(qrow + off);
+        const uint4 vd = *reinterpret_cast<const uint4*>(qrow + 32768 + off);
+        rq[4 * c] = vq.x, rq[4 * c + 1] = vq.y, rq[4 * c + 2] = vq.z, rq[4 * c + 3] = vq.w;
+        rd[4 * c] = vd.x, rd[4 * c + 1] = vd.y, rd[4 * c + 2] = vd.z, rd[4 * c + 3] = vd.w;
+      }
+      tmem_st32(lane_addr + kColQP + 32 * kh, rq);
+      tmem_st32(lane_addr + kColDOP + 32 * kh, rd);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(bar(P_QT));                            // (also on a failed wait: never blocks the others)
     int lo_r, hi_r;
     bwd::row_range(a, crow, tt, lo_r, hi_r);
     if (lowest) lo_r = 0;
@@ -285,9 +334,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       lse2 = a.lse[li] * 1.4426950408889634f;
       dl = a.delta[li];
     }
-    bool ok = true;
     for (int j = 0; j < total && ok; ++j) {
-      const int x = j & 1, use = j >> 1;
+      const int x = j & 1;
       int rg, key0, nk;
       tile_of(j, rg, key0, nk);
       // this row's keys in the tile: at most two intervals (sink slots, retained
@@ -310,9 +358,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       const uint32_t hb = (uint32_t)(bits >> (32 * kh));
       const float* brow = (a.bias != nullptr && rg != 2) ? a.bias + col_base + key0 + 32 * kh : nullptr;
-      ok = mbar_wait(bar(P_SF + x), use & 1, abort_flag, err, 409);
-      if (ok && use >= 1) ok = mbar_wait(bar(P_DSE + x), (use - 1) & 1, abort_flag, err, 410);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(P_SF + x), (j >> 1) & 1, abort_flag, err, 409))))
+        break;
       tc_fence_after();
       uint32_t pkd[16];
       {
@@ -320,26 +367,35 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_ld32(lane_addr + kColSP + x * 64 + 32 * kh, rs);
         tmem_ld32(lane_addr + kColDPP + x * 64 + 32 * kh, rp);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(P_SE + x));                    // this thread's part of S, dP x is read
         if (brow != nullptr) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if ((hb >> c) & 1u) rs[c] = __float_as_uint(__uint_as_float(rs[c]) + __ldg(brow + c));
         }
+        // dS = P (dP - D); a row that attends all 32 keys (the common case) takes
+        // the unmasked form
+        auto form = [&](auto all_on) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float ds2[2];
+          for (int c = 0; c < 32; c += 2) {
+            float ds2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float p = ((hb >> (c + e)) & 1u)
-                                ? ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -lse2))
-                                : 0.f;
-            ds2[e] = p * (__uint_as_float(rp[c + e]) - dl);
+            for (int e = 0; e < 2; ++e) {
+              float p = ex2(fmaf(__uint_as_float(rs[c + e]), a.scale_log2, -lse2));
+              if constexpr (!decltype(all_on)::value) p = ((hb >> (c + e)) & 1u) ? p : 0.f;
+              ds2[e] = p * (__uint_as_float(rp[c + e]) - dl);
+            }
+            pkd[c >> 1] = pk2(ds2[0], ds2[1]);
           }
-          pkd[c >> 1] = pk2(ds2[0], ds2[1]);
-        }
+        };
+        if (hb == 0xffffffffu) form(std::true_type{});
+        else form(std::false_type{});
       }
-      tc_fence_before();
-      mbar_arrive(bar(P_SE + x));                      // this thread's part of S, dP x is read
+      // dQ += dS(j - 2) K(j - 2) has read dS buffer x
+      if (j >= 2 &&
+          !(ok = __all_sync(0xffffffffu, mbar_wait(bar(P_DSE + x), ((j - 2) >> 1) & 1, abort_flag, err, 410))))
+        break;
       // 64 bytes of the dS row (keys 32 kh ..) into the swizzled K-major A operand
       uint8_t* drow = sm + kDS2 + x * 16384u + row * 128;
 #pragma unroll
@@ -351,11 +407,16 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       fence_proxy_async();
       mbar_arrive(bar(P_DSF + x));
     }
-    // dQ row: scale, fp32 out, columns 64 kh .. (every lane loads: tcgen05.ld is warp-collective)
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(P_DQ), 0, abort_flag, err, 411));
+    // dQ out.  Once every product has completed (and so every K, V copy has
+    // landed and been read), each thread stages its row's 64 columns (x scale) in
+    // the K ring, 16-byte chunks XOR-swizzled by row, then each warp writes
+    // whole 512-byte rows.  The eight row warps go on together or stop together
+    // (named barrier 1).
+    ok = ok && mbar_wait(bar(P_DQ), 0, abort_flag, err, 411);
+    ok = bar_and(1, 256, __all_sync(0xffffffffu, ok));
     if (ok) {
       tc_fence_after();
-      float* out = a.dq + (((long long)b * a.T + min(tt, a.T - 1)) * a.Hq + h * G + gq) * HD;
+      uint8_t* stage = sm + kKR;                         // [128][128] fp32
 #pragma unroll 1
       for (int c0 = 64 * kh; c0 < 64 * kh + 64; c0 += 32) {
         uint32_t r[32];
@@ -366,12 +427,23 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
           for (int e = 0; e < 32; ++e) r[e] = 0u;
         }
-        if (tt < a.T) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(out + c0 + e) =
-                make_float4(__uint_as_float(r[e]) * a.scale, __uint_as_float(r[e + 1]) * a.scale,
-                            __uint_as_float(r[e + 2]) * a.scale, __uint_as_float(r[e + 3]) * a.scale);
+        for (int e = 0; e < 32; e += 4) {
+          const int ch = (c0 + e) >> 2;                  // 16-byte chunk of the 512-byte row
+          *reinterpret_cast<float4*>(stage + row * 512 + ((ch ^ (row & 31)) << 4)) =
+              make_float4(__uint_as_float(r[e]) * a.scale, __uint_as_float(r[e + 1]) * a.scale,
+                          __uint_as_float(r[e + 2]) * a.scale, __uint_as_float(r[e + 3]) * a.scale);
+        }
+      }
+      bar_sync(1, 256);
+      const int lane = tid & 31, w8 = warp - 4;
+#pragma unroll 4
+      for (int rr = w8; rr < kRowsTc; rr += 8) {
+        const int t_r = t0 + rr / G;
+        if (t_r < a.T) {
+          const float4 v = *reinterpret_cast<const float4*>(stage + rr * 512 + ((lane ^ (rr & 31)) << 4));
+          float* out = a.dq + (((long long)b * a.T + t_r) * a.Hq + h * G + rr % G) * HD;
+          *reinterpret_cast<float4*>(out + 4 * lane) = v;
         }
       }
     }
@@ -818,25 +890,36 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const float4* ml = reinterpret_cast<const float4*>(mf + 32 * half);
         const float4* md = reinterpret_cast<const float4*>(mf + kRowsK2 + 32 * half);
         uint32_t pp[16], pd[16];
+        // P^T, dS^T; a key that all 32 rows attend (the common case) takes the
+        // unmasked form
+        auto form = [&](auto all_on) {
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = ml[c4], d4 = md[c4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p4[4], q4[4];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l4 = ml[c4], d4 = md[c4];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float p4[4], q4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            const bool on = (hb >> c) & 1u;
-            const float p = on ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, bk2 - lv[e])) : 0.f;
-            p4[e] = p;
-            q4[e] = on ? p * (__uint_as_float(rp[c]) - dv4[e]) : 0.f;
-            if constexpr (kColumn) dr_acc += q4[e];
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * c4 + e;
+              float p = ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, bk2 - lv[e]));
+              float q = p * (__uint_as_float(rp[c]) - dv4[e]);
+              if constexpr (!decltype(all_on)::value) {
+                const bool on = (hb >> c) & 1u;
+                p = on ? p : 0.f;
+                q = on ? q : 0.f;
+              }
+              p4[e] = p;
+              q4[e] = q;
+              if constexpr (kColumn) dr_acc += q;
+            }
+            pp[2 * c4] = pk2(p4[0], p4[1]);
+            pp[2 * c4 + 1] = pk2(p4[2], p4[3]);
+            pd[2 * c4] = pk2(q4[0], q4[1]);
+            pd[2 * c4 + 1] = pk2(q4[2], q4[3]);
           }
-          pp[2 * c4] = pk2(p4[0], p4[1]);
-          pp[2 * c4 + 1] = pk2(p4[2], p4[3]);
-          pd[2 * c4] = pk2(q4[0], q4[1]);
-          pd[2 * c4 + 1] = pk2(q4[2], q4[3]);
-        }
+        };
+        if (hb == 0xffffffffu) form(std::true_type{});
+        else form(std::false_type{});
         // dV, dK of tile g - 2 have read P^T, dS^T buffer g % 2
         const int x = g & 1;
         if (g >= 2 &&
@@ -987,7 +1070,8 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
   using namespace bwdtc;
   const int TOK = kRowsTc / a.G;
-  // tensor maps (contiguous [B,T,H,128] bf16; 128-byte swizzle, 64-column boxes)
+  // tensor maps of Q, dO, K, V and of the column segment (contiguous rows of 128
+  // bf16; 128-byte swizzle, 64-column boxes)
   CUtensorMap mq, mdo, mk, mv, mkc, mvc;
   {
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
@@ -1016,8 +1100,7 @@ cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaSt
                                        kSmemP);
   if (e != cudaSuccess) return e;
   const int n_tiles = (a.T + TOK - 1) / TOK;
-  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsP, kSmemP, stream>>>(mq, mdo, mk, mv, mkc, mvc,
-                                                                          a, err);
+  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsP, kSmemP, stream>>>(mq, mdo, mk, mv, mkc, mvc, a, err);
   return cudaGetLastError();
 }
 
