@@ -1,29 +1,22 @@
-// dQ of the prefill sparse attention's backward on 5th-generation tensor
-// cores (tcgen05 + TMEM), head dim 128, bf16 operands, fp32 accumulation.
+// Backward of the prefill sparse attention on 5th-generation tensor cores
+// (tcgen05 + TMEM), head dim 128, bf16 operands, fp32 accumulation.
 //
 // "Alleviating Forgetfulness of Linear Attention by Hybrid Sparse Attention
 // and Contextualized Learnable Token Eviction", Abstract (trained end to end)
-// and Fig. 2 caption (right): the attended sets S_t, held fixed.  Per query
-// row, with P recomputed from the forward's lse and D_t = <dO_t, o_t>:
-//   dS = P * (dO V^T - D_t),   dQ = scale dS K.
+// and Fig. 2 caption (right): the attended sets S_t, held fixed.  With P
+// recomputed from the forward's lse and D_t = <dO_t, o_t>:
+//   dS = P * (dO V^T - D_t),   dQ = scale dS K,   dV = P^T dO,   dK = scale dS^T Q.
 //
-// One CTA of 128 threads per 128 query rows (128/G tokens x the G heads of a
-// KV head, token-major), one row per thread; two CTAs share an SM (112 KiB of
-// shared memory and 256 TMEM columns each).  Q and dO stay in shared memory;
-// per 64-key tile of the forward's key ranges (sink slots and retained slots
-// of the column segment, window band of k):
-//   1. K and V of the tile arrive by cp.async (zero-filled past the tile's
-//      valid rows) in the 128-byte-swizzled K-major layout;
-//   2. one thread issues S = Q K^T and dP = dO V^T (M128 N64 K128, both
-//      operands in shared memory) into TMEM and commits;
-//   3. each thread reads its row of S and dP, forms P (masked keys 0) and
-//      dS = P (dP - D_t), and writes dS as bf16 into shared memory (the A
-//      operand of the next product);
-//   4. one thread issues dQ += dS K (M128 N128 K64; K as an N-contiguous B
-//      operand) into the TMEM accumulator and commits; the tile's buffers are
-//      reused once that product has completed.
-// Every wait is bounded; on expiry the CTA records LTE_ERR_TIMEOUT, drains
-// what it issued, frees its TMEM and leaves.
+// bwd_dq_tc_kernel: one CTA per 128 query rows (128/G tokens x the G heads of
+// a KV head), over 64-key tiles of the rows' key ranges (sink slots and
+// retained slots of the column segment, window band of k).
+// bwd_dkdv_tc_kernel: persistent, one CTA per SM over work items of one
+// 128-key tile (keys of k, or slots of the column segment) and a run of the
+// 64-row query tiles that attend it.
+// Both are warp-specialised: a TMA producer warp, a single-thread MMA issuer
+// and eight row warps that form P and dS between the products; the roles are
+// described above each kernel.  Every wait is bounded; on expiry the CTA
+// records LTE_ERR_TIMEOUT, drains what it issued, frees its TMEM and leaves.
 #include <math.h>
 
 #include <type_traits>
@@ -41,14 +34,6 @@ using namespace tc;
 constexpr int HD = 128;
 constexpr int kRowsTc = 128;                    // query rows per CTA
 constexpr int kKeysTc = 64;                     // keys per tile
-constexpr int kThreadsTc = 128;
-constexpr uint32_t kK = 65536;                  // [64][128]: two halves of 8 KiB
-constexpr uint32_t kV = 81920;
-constexpr uint32_t kDS = 98304;                 // [128][64] bf16 (one half)
-constexpr uint32_t kBar = 114688;               // bar_s, bar_q, abort flag, TMEM slot
-constexpr int kSmemBytes = kBar + 64;
-constexpr int kTmemCols = 256;                  // S 0..63, dP 64..127, dQ 128..255
-constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128;
 
 // byte offset of 16-byte chunk c16 (0..15) of row r in a K-major [rows][128]
 // bf16 tile stored as two 64-column halves, 128-byte swizzle
