@@ -35,26 +35,13 @@ constexpr int HD = 128;
 constexpr int kRowsTc = 128;                    // query rows per CTA
 constexpr int kKeysTc = 64;                     // keys per tile
 
-// byte offset of 16-byte chunk c16 (0..15) of row r in a K-major [rows][128]
-// bf16 tile stored as two 64-column halves, 128-byte swizzle
-__device__ __forceinline__ uint32_t sw(int rows, int r, int c16) {
-  return (uint32_t)((c16 >> 3) * rows * 128 + r * 128 + ((((c16 & 7) ^ (r & 7))) << 4));
-}
-__device__ __forceinline__ void cpa16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0));
-}
-__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-__device__ __forceinline__ void cpa_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::); }
-// bits [a, b) of a 64-bit set (empty when b <= a), clipped to [0, 64)
-__device__ __forceinline__ uint64_t span64(int a, int b) {
+// bits [a, b) of a 32-bit set (empty when b <= a), clipped to [0, 32)
+__device__ __forceinline__ uint32_t span32(int a, int b) {
   a = a > 0 ? a : 0;
-  b = b < 64 ? b : 64;
-  if (b <= a) return 0ull;
-  const uint64_t ones = (b - a == 64) ? ~0ull : ((1ull << (b - a)) - 1ull);
-  return ones << a;
+  b = b < 32 ? b : 32;
+  if (b <= a) return 0u;
+  return (0xffffffffu >> (32 - (b - a))) << a;
 }
-
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -323,25 +310,26 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int x = j & 1;
       int rg, key0, nk;
       tile_of(j, rg, key0, nk);
-      // this row's keys in the tile: at most two intervals (sink slots, retained
-      // slots [lo, hi)) or one (window band); this thread takes keys 32 kh ..
-      uint64_t bits = 0ull;
+      // this row's keys among this thread's 32 (keys kb .. kb + 31 of the tile's
+      // positions or slots): at most two intervals (sink slots, retained slots
+      // [lo, hi)) or one (window band)
+      const int kb = key0 + 32 * kh, nkh = nk - 32 * kh;
+      uint32_t hb = 0u;
       if (tt < a.T) {
         if (rg == 2) {
-          bits = span64(tt - a.window + 1 - key0, min(nk, tt - key0 + 1));
+          hb = span32(tt - a.window + 1 - kb, min(nkh, tt - kb + 1));
         } else {
           const int sink_end = min(a.sink, tt - a.window + 1);
-          uint64_t ret = span64(a.sink + lo_r - key0, min(nk, a.sink + hi_r - key0));
-          if (lowest && ret != 0ull) {                 // lifetimes: held at count hi_r
+          uint32_t ret = span32(a.sink + lo_r - kb, min(nkh, a.sink + hi_r - kb));
+          if (lowest && ret != 0u) {                   // lifetimes: held at count hi_r
 #pragma unroll 4
-            for (int kk = 32 * kh; kk < 32 * kh + 32; ++kk)
-              if (((ret >> kk) & 1ull) && __ldg(a.death + crow + key0 + kk - a.sink) <= hi_r)
-                ret &= ~(1ull << kk);
+            for (int kk = 0; kk < 32; ++kk)
+              if (((ret >> kk) & 1u) && __ldg(a.death + crow + kb + kk - a.sink) <= hi_r)
+                ret &= ~(1u << kk);
           }
-          bits = span64(-key0, min(nk, sink_end - key0)) | ret;
+          hb = span32(-kb, min(nkh, sink_end - kb)) | ret;
         }
       }
-      const uint32_t hb = (uint32_t)(bits >> (32 * kh));
       const float* brow = (a.bias != nullptr && rg != 2) ? a.bias + col_base + key0 + 32 * kh : nullptr;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(P_SF + x), (j >> 1) & 1, abort_flag, err, 409))))
         break;
@@ -863,7 +851,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           r_a = max(r_a, 0);
           r_b = min(r_b, r_end);
         }
-        const uint32_t hb = (uint32_t)span64(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
+        const uint32_t hb = span32(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_SF), g & 1, abort_flag, err, 419)))) break;
         tc_fence_after();
         uint32_t rs[32], rp[32];
