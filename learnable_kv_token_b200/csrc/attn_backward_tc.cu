@@ -54,23 +54,24 @@ __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
 //              have completed, K only once dQ += dS(j) K(j) has;
 //   warp 1     MMA issuer: S(j), dP(j) into TMEM buffer j % 2 (Q and dO are A
 //              operands from TMEM), issued two tiles ahead of the rows, and
-//              dQ += dS(j) K(j) once dS(j) is in shared memory: per rows' tile
-//              r it issues dQ(r - 1) and then S(r + 2), so no S waits in the
-//              tensor core's in-order queue behind a product that waits for
-//              the rows;
+//              dQ += dS(j) K(j) once dS(j) is written: per rows' tile r it
+//              issues dQ(r) and then S(r + 2), which reuses buffer r % 2 -- the
+//              tensor core runs its products in issue order, so dQ(r) has read
+//              dS(r) before S(r + 2) overwrites it;
 //   warps 4-11 two threads per query row (warps 4-7 the first 32 keys of a
 //              tile, 8-11 the last 32): Q and dO into TMEM at the start; P and
-//              dS of tile j from TMEM buffer j % 2 (released as soon as read)
-//              into the shared dS buffer j % 2; at the end, dQ out through a
-//              shared-memory stage, whole 512-byte rows per warp store.
-// TMEM: S[2] 0..127, dP[2] 128..255, dQ 256..383, Q 384..447, dO 448..511
-// (bf16 pairs).
+//              dS of tile j from TMEM buffer j % 2, dS written back as bf16
+//              pairs over the first 16 of the 32 S columns each thread read
+//              (no thread writes a column another still reads); at the end, dQ
+//              out through a shared-memory stage, whole 512-byte rows per warp
+//              store.
+// TMEM: S[2] 0..127 (dS over them), dP[2] 128..255, dQ 256..383, Q 384..447,
+// dO 448..511 (bf16 pairs).
 constexpr int kThreadsP = 384;
 constexpr int kStagesKP = 7, kStagesVP = 4;            // K and V rings
 constexpr uint32_t kKR = 0;                             // K stage s at 16 KiB s
 constexpr uint32_t kVR = kKR + kStagesKP * 16384;       // V stage s at 16 KiB s
-constexpr uint32_t kDS2 = kVR + kStagesVP * 16384;      // dS buffers: 2 x [128][64] bf16
-constexpr uint32_t kBar2 = kDS2 + 2 * 16384;            // barriers
+constexpr uint32_t kBar2 = kVR + kStagesVP * 16384;     // barriers
 constexpr int kSmemP = kBar2 + 512;
 constexpr uint32_t kColSP = 0, kColDPP = 128, kColDQP = 256, kColQP = 384, kColDOP = 448;
 constexpr int kQStage = 3;                              // Q, dO arrive in K stages 3..6
@@ -78,7 +79,7 @@ constexpr uint32_t kQS = kKR + kQStage * 16384;         // Q [128][128] bf16 (32
 static_assert(kQStage * 16384 + 65536 <= kStagesKP * 16384, "Q and dO fit the K ring's tail");
 enum {
   P_QF = 0, P_QT = 1, P_KF = 2, P_KE = P_KF + kStagesKP, P_VF = P_KE + kStagesKP, P_VE = P_VF + kStagesVP,
-  P_SF = P_VE + kStagesVP, P_SE = P_SF + 2, P_DSF = P_SE + 2, P_DSE = P_DSF + 2, P_DQ = P_DSE + 2,
+  P_SF = P_VE + kStagesVP, P_DSF = P_SF + 2, P_DQ = P_DSF + 2,
   kNumBarsP = P_DQ + 1
 };
 static_assert(8 * kNumBarsP + 8 <= 512, "barriers fit");
@@ -122,9 +123,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(P_SF + x), 1);
-      mbar_init(bar(P_SE + x), 256);
       mbar_init(bar(P_DSF + x), 256);
-      mbar_init(bar(P_DSE + x), 1);
     }
     mbar_init(bar(P_DQ), 1);
     *abort_flag = 0;
@@ -219,10 +218,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QT), 0, abort_flag, err, 405));
     auto issue_s = [&](int j) -> bool {                       // S(j), dP(j) into buffer j % 2
       const int x = j & 1, sk = j % kStagesKP, sv = j % kStagesVP;
+      // (for j >= 2, dQ(j - 2) was issued just before: the rows have read S, dP
+      // of tile j - 2, and the tensor core reads their dS before this overwrites it)
       bool w = mbar_wait(bar(P_KF + sk), (j / kStagesKP) & 1, abort_flag, err, 407);
       if (w) w = mbar_wait(bar(P_VF + sv), (j / kStagesVP) & 1, abort_flag, err, 413);
-      // the rows have read S, dP of tile j - 2
-      if (w && j >= 2) w = mbar_wait(bar(P_SE + x), ((j - 2) >> 1) & 1, abort_flag, err, 408);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       if (elect_one()) {
@@ -246,13 +245,15 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return false;
       tc_fence_after();
       if (elect_one()) {
-        const uint64_t dds = sdesc(sb + kDS2 + x * 16384u, 16, 1024);
         const uint64_t dkb = sdesc(sb + kKR + sk * 16384u, kKeysTc * 128, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kKeysTc / 16; ++ks)
-          mma_f16(tmem + kColDQP, dds + ((ks * 32) >> 4), dkb + ((ks * 2048) >> 4), id_q,
-                  (jj > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(bar(P_DSE + x));                           // dS buffer x is free
+        for (int ks = 0; ks < kKeysTc / 16; ++ks) {
+          // keys 16 ks ..: the packed dS a row's thread (ks >> 1) wrote over the first
+          // 16 of its 32 columns of S buffer x
+          const uint32_t pc = (uint32_t)(x * 64 + 32 * (ks >> 1) + 8 * (ks & 1));
+          mma_f16_ts(tmem + kColDQP, tmem + kColSP + pc, dkb + ((ks * 2048) >> 4), id_q,
+                     (jj > 0 || ks > 0) ? 1u : 0u);
+        }
         mma_commit(bar(P_KE + sk));                           // K of tile jj is free
       }
       __syncwarp();
@@ -261,10 +262,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (ok && total > 0) ok = issue_s(0);
     if (ok && total > 1) ok = issue_s(1);
     for (int r = 0; r < total && ok; ++r) {
-      if (r >= 1) ok = issue_dq(r - 1);
+      ok = issue_dq(r);
       if (ok && r + 2 < total) ok = issue_s(r + 2);
     }
-    if (ok && total > 0) ok = issue_dq(total - 1);
     if (elect_one()) mma_commit(bar(P_DQ));                   // every product above has completed
     __syncwarp();
     mbar_drain(bar(P_DQ), 0);
@@ -340,8 +340,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_ld32(lane_addr + kColSP + x * 64 + 32 * kh, rs);
         tmem_ld32(lane_addr + kColDPP + x * 64 + 32 * kh, rp);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(P_SE + x));                    // this thread's part of S, dP x is read
         if (brow != nullptr) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
@@ -365,19 +363,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (hb == 0xffffffffu) form(std::true_type{});
         else form(std::false_type{});
       }
-      // dQ += dS(j - 2) K(j - 2) has read dS buffer x
-      if (j >= 2 &&
-          !(ok = __all_sync(0xffffffffu, mbar_wait(bar(P_DSE + x), ((j - 2) >> 1) & 1, abort_flag, err, 410))))
-        break;
-      // 64 bytes of the dS row (keys 32 kh ..) into the swizzled K-major A operand
-      uint8_t* drow = sm + kDS2 + x * 16384u + row * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int ch = 4 * kh + c;
-        *reinterpret_cast<uint4*>(drow + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(pkd[4 * c], pkd[4 * c + 1], pkd[4 * c + 2], pkd[4 * c + 3]);
-      }
-      fence_proxy_async();
+      // dS of keys 32 kh .. as bf16 pairs over the first 16 of the 32 S columns this
+      // thread has read: the A operand of dQ += dS K
+      tmem_st16(lane_addr + kColSP + x * 64 + 32 * kh, pkd);
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(bar(P_DSF + x));
     }
     // dQ out.  Once every product has completed (and so every K, V copy has
