@@ -430,15 +430,17 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // busy tile and add into dK, dV with atomics).  Keys are the MMA rows; the
 // attending query rows come in tiles of 64 (64/G tokens x the G heads), and
 // per row tile:
-//   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM
-//   P^T, dS^T = P^T (dP^T - D)         (two threads per key row, 32 rows each)
-//                                      into TMEM buffer (tile % 2), as bf16
+//   S^T = K Q^T, dP^T = V dO^T        (M128 N64 K128) into TMEM buffer g % 2
+//   P^T, dS^T = P^T (dP^T - D)         (two threads per key row, 32 rows each),
+//                                      as bf16 over the columns of S^T and dP^T
+//                                      each thread read
 //   dV += P^T dO, dK += dS^T Q         (M128 N128 K64; P^T, dS^T read from TMEM)
-// The tensor core runs its products in issue order, so the schedule keeps any
-// product from waiting behind one that waits for the rows: S^T of a tile is
-// issued as soon as the rows have read the S^T before it (one S^T buffer), dV
-// and dK of the tile before once its P^T and dS^T are written, and those have
-// two buffers, so the rows never wait for dV and dK.
+// The tensor core runs its products in issue order.  The MMA thread issues
+// S^T two row tiles ahead of the rows (across items: K and V of the next item
+// arrive once the current item's last S^T has completed) and, per row tile g,
+// dV and dK of g once its P^T and dS^T are written, then S^T of g + 2 into the
+// same buffer -- so S^T of a tile never waits behind a product that waits for
+// the rows, and the rows never wait for S^T.
 // Roles (384 threads):
 //   warp 0     TMA producer (one elected lane): K and V of each item, once the
 //              item before has issued its last S^T and that has completed; per
@@ -447,14 +449,16 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 //              while the copies fly;
 //   warp 1     MMA issuer, as above;
 //   warps 4-11 two threads per key row (warps 4-7 rows 0-31 of a tile, 8-11
-//              rows 32-63): P^T and dS^T; at the end of an item, dK and dV out
+//              rows 32-63): P^T and dS^T, each written over the first 16 of the
+//              32 columns of S^T (dP^T) the thread read, so no thread writes a
+//              column another still reads; at the end of an item, dK and dV out
 //              through a shared-memory stage in 32-column chunks, so that each
 //              warp store (or add) covers four whole 128-byte rows, while the
 //              tensor core already computes the next item's first S^T.
-// TMEM: S^T 0..63, dP^T 64..127, P^T and dS^T of buffer x at 128 + 64 x and
-// 160 + 64 x (64 bf16 rows packed in pairs), dV 256..383, dK 384..511.
-// Barrier phases run on a row-tile counter that continues across items (ring
-// stages, S^T, P^T buffers) or on the item counter (K and V, items' completion).
+// TMEM: S^T of buffer x at 64 x (P^T over it), dP^T at 128 + 64 x (dS^T over
+// it), dV 256..383, dK 384..511.  Barrier phases run on a row-tile counter that
+// continues across items (ring stages, S^T buffers) or on the item counter (K
+// and V, items' completion).
 constexpr int kKeysKV = 128;
 constexpr int kRowsK2 = 64;                       // attending query rows per tile
 constexpr int kStagesK2 = 4;
@@ -467,10 +471,10 @@ constexpr uint32_t k2Stage = k2Meta + kStagesK2 * 5 * kRowsK2 * 4;   // [128][32
 constexpr uint32_t k2Pos = k2Stage + kKeysKV * 128;                  // [128] output row per key
 constexpr uint32_t k2Bar = k2Pos + kKeysKV * 4;
 constexpr int k2Smem = k2Bar + 256;
-constexpr uint32_t k2ColS = 0, k2ColDP = 64, k2ColP = 128, k2ColDV = 256, k2ColDK = 384;
+constexpr uint32_t k2ColS = 0, k2ColDP = 128, k2ColDV = 256, k2ColDK = 384;
 enum {
-  K2_KVF = 0, K2_KVE = 1, K2_F = 2, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_SE = K2_SF + 1,
-  K2_PF = K2_SE + 1, K2_PE = K2_PF + 2, K2_DONE = K2_PE + 2, kNumBarsK2 = K2_DONE + 1
+  K2_KVF = 0, K2_KVE = 1, K2_F = 2, K2_E = K2_F + kStagesK2, K2_SF = K2_E + kStagesK2, K2_PF = K2_SF + 2,
+  K2_DONE = K2_PF + 2, kNumBarsK2 = K2_DONE + 1
 };
 static_assert(8 * kNumBarsK2 + 16 <= 256, "barriers and flags fit");
 static_assert(k2Smem <= 227 * 1024, "shared memory fits one CTA");
@@ -627,11 +631,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(bar(K2_F + st), 1);
       mbar_init(bar(K2_E + st), 1);
     }
-    mbar_init(bar(K2_SF), 1);
-    mbar_init(bar(K2_SE), 256);
     for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(K2_SF + x), 1);
       mbar_init(bar(K2_PF + x), 256);
-      mbar_init(bar(K2_PE + x), 1);
     }
     mbar_init(bar(K2_DONE), 1);
     *abort_flag = 0;
@@ -738,50 +740,77 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (elect_one()) {
         const uint32_t qs = sb + k2QD + st * 32768u;
         const uint64_t qb = sdesc(qs, kRowsK2 * 128, 1024), dob = sdesc(qs + 16384u, kRowsK2 * 128, 1024);
-        const uint32_t pb = tmem + k2ColP + (uint32_t)(64 * x);
 #pragma unroll
         for (int ks = 0; ks < kRowsK2 / 16; ++ks) {
+          // rows 16 ks ..: packed by the thread of row half ks >> 1 over the first 16
+          // of its 32 columns of buffer x
+          const uint32_t pc = (uint32_t)(x * 64 + 32 * (ks >> 1) + 8 * (ks & 1));
           const uint32_t acc = (!first || ks > 0) ? 1u : 0u;
-          mma_f16_ts(tmem + k2ColDV, pb + 8 * ks, dob + ((ks * 2048) >> 4), id_o, acc);
-          mma_f16_ts(tmem + k2ColDK, pb + 32 + 8 * ks, qb + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + k2ColDV, tmem + k2ColS + pc, dob + ((ks * 2048) >> 4), id_o, acc);
+          mma_f16_ts(tmem + k2ColDK, tmem + k2ColDP + pc, qb + ((ks * 2048) >> 4), id_o, acc);
         }
         mma_commit(bar(K2_E + st));                          // the row tile's stage is free
-        mma_commit(bar(K2_PE + x));                          // P^T, dS^T buffer x is free
       }
       __syncwarp();
       return true;
     };
+    // S^T stream: a cursor over (item, row tile) that runs two tiles ahead
+    int s_item = blockIdx.x, s_k = 0, s_i = 0, s_n = item_at(s_item).n_rt, gs = 0;
+    auto issue_next_s = [&]() -> bool {
+      if (s_item >= n_items) return true;                     // nothing left to start
+      const int st = gs % kStagesK2, x = gs & 1;
+      // (for gs >= 2, dV and dK of gs - 2 were issued just before: they read
+      // P^T, dS^T from this buffer before S^T of gs overwrites it)
+      bool w = true;
+      if (s_i == 0) w = mbar_wait(bar(K2_KVF), s_k & 1, abort_flag, err, 415);   // K, V of the item
+      if (w) w = mbar_wait(bar(K2_F + st), (gs / kStagesK2) & 1, abort_flag, err, 417);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t qs = sb + k2QD + st * 32768u;
+        const uint64_t dk = sdesc(sb + k2K, 16, 1024), dv = sdesc(sb + k2V, 16, 1024);
+        const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
+          mma_f16(tmem + k2ColS + x * 64, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
+          mma_f16(tmem + k2ColDP + x * 64, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(K2_SF + x));
+        if (s_i == s_n - 1) mma_commit(bar(K2_KVE));         // K, V of the item no longer read
+      }
+      __syncwarp();
+      ++gs;
+      if (++s_i == s_n) {
+        s_i = 0;
+        ++s_k;
+        s_item += gridDim.x;
+        if (s_item < n_items) s_n = item_at(s_item).n_rt;
+      }
+      return true;
+    };
+    ok = issue_next_s();
+    if (ok) ok = issue_next_s();
     int g = 0, k = 0;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
       const int n_rt = item_at(it).n_rt;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_KVF), k & 1, abort_flag, err, 415)))) break;
-      for (int i = 0; i < n_rt; ++i, ++g) {
-        const int st = g % kStagesK2;
-        ok = mbar_wait(bar(K2_F + st), (g / kStagesK2) & 1, abort_flag, err, 417);
-        // S^T, dP^T of the tile before have been read by the rows
-        if (ok && g >= 1) ok = mbar_wait(bar(K2_SE), (g - 1) & 1, abort_flag, err, 421);
-        if (!(ok = __all_sync(0xffffffffu, ok))) break;
-        tc_fence_after();
-        if (elect_one()) {
-          const uint32_t qs = sb + k2QD + st * 32768u;
-          const uint64_t dk = sdesc(sb + k2K, 16, 1024), dv = sdesc(sb + k2V, 16, 1024);
-          const uint64_t dq = sdesc(qs, 16, 1024), ddo = sdesc(qs + 16384u, 16, 1024);
-#pragma unroll
-          for (int ks = 0; ks < HD / 16; ++ks) {
-            const uint32_t oa = ((ks >> 2) * (kKeysKV * 128) + (ks & 3) * 32) >> 4;
-            const uint32_t ob = ((ks >> 2) * (kRowsK2 * 128) + (ks & 3) * 32) >> 4;
-            mma_f16(tmem + k2ColS, dk + oa, dq + ob, id_s, ks > 0 ? 1u : 0u);
-            mma_f16(tmem + k2ColDP, dv + oa, ddo + ob, id_s, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(K2_SF));
-          if (i == n_rt - 1) mma_commit(bar(K2_KVE));        // K, V no longer read
+      bool done = false;
+      for (int i = 0; i < n_rt && ok; ++i, ++g) {
+        ok = issue_dvdk(g, i == 0);
+        if (ok && i == n_rt - 1) {
+          // every product of the item has completed (before S^T of the next
+          // item's tiles that follow in the queue)
+          if (elect_one()) mma_commit(bar(K2_DONE));
+          __syncwarp();
+          done = true;
         }
-        __syncwarp();
-        if (i >= 1 && !(ok = issue_dvdk(g - 1, i == 1))) break;
+        if (ok) ok = issue_next_s();
       }
-      if (ok) ok = issue_dvdk(g - 1, n_rt == 1);
-      if (elect_one()) mma_commit(bar(K2_DONE));           // every product of the item has completed
-      __syncwarp();
+      if (!done) {
+        if (elect_one()) mma_commit(bar(K2_DONE));
+        __syncwarp();
+      }
     }
     if (k >= 1) mbar_drain(bar(K2_DONE), (k - 1) & 1);
   } else if (warp >= 4) {
@@ -842,14 +871,14 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           r_b = min(r_b, r_end);
         }
         const uint32_t hb = span32(r_a - 32 * half, r_b - 32 * half);   // this thread's 32 rows
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_SF), g & 1, abort_flag, err, 419)))) break;
+        const int x = g & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_SF + x), (g >> 1) & 1, abort_flag, err, 419))))
+          break;
         tc_fence_after();
         uint32_t rs[32], rp[32];
-        tmem_ld32(lane_addr + k2ColS + 32 * half, rs);
-        tmem_ld32(lane_addr + k2ColDP + 32 * half, rp);
+        tmem_ld32(lane_addr + k2ColS + x * 64 + 32 * half, rs);
+        tmem_ld32(lane_addr + k2ColDP + x * 64 + 32 * half, rp);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(K2_SE));                           // S^T, dP^T may be overwritten
         const float4* ml = reinterpret_cast<const float4*>(mf + 32 * half);
         const float4* md = reinterpret_cast<const float4*>(mf + kRowsK2 + 32 * half);
         uint32_t pp[16], pd[16];
@@ -883,15 +912,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         };
         if (hb == 0xffffffffu) form(std::true_type{});
         else form(std::false_type{});
-        // dV, dK of tile g - 2 have read P^T, dS^T buffer g % 2
-        const int x = g & 1;
-        if (g >= 2 &&
-            !(ok = __all_sync(0xffffffffu, mbar_wait(bar(K2_PE + x), ((g - 2) >> 1) & 1, abort_flag, err, 423))))
-          break;
-        tc_fence_after();
-        // rows 32 half .. + 31 of P^T, dS^T: columns 16 half .. + 15 of the buffer
-        tmem_st16(lane_addr + k2ColP + (uint32_t)(64 * x + 16 * half), pp);
-        tmem_st16(lane_addr + k2ColP + (uint32_t)(64 * x + 32 + 16 * half), pd);
+        // rows 32 half .. + 31 of P^T, dS^T over the first 16 of the 32 columns of
+        // S^T, dP^T this thread read
+        tmem_st16(lane_addr + k2ColS + (uint32_t)(64 * x + 32 * half), pp);
+        tmem_st16(lane_addr + k2ColDP + (uint32_t)(64 * x + 32 * half), pd);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(K2_PF + x));
