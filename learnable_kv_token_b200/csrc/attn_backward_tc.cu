@@ -463,7 +463,7 @@ constexpr int kKeysKV = 128;
 constexpr int kRowsK2 = 64;                       // attending query rows per tile
 constexpr int kStagesK2 = 4;
 constexpr int kThreadsK2 = 384;
-constexpr int kSplitRowsK2 = 32;                  // row tiles per column item, at most
+constexpr int kSplitRowsK2 = 64;                  // row tiles per column item, at most
 constexpr uint32_t k2K = 0, k2V = 32768;          // [128][128] bf16 each: halves of 16 KiB
 constexpr uint32_t k2QD = 65536;                  // stage s: Q at + 32 KiB s, dO at + 16 KiB
 constexpr uint32_t k2Meta = k2QD + kStagesK2 * 32768;            // stage s: [5][64] words
