@@ -662,8 +662,9 @@ def rows_bench(args, rank, world, device, dec):
                                   "(hi/lo bf16 operands: 2-3x the MMA work of these algorithmic "
                                   "flops), the elementwise pass on CUDA cores; FLOPs = 3 x 2 x "
                                   "c_hid x 2D x k1 per (b, KV head, position)"),
-        "a3b_note": "lte_sparse_attn_backward (delta, dQ, dK/dV window, dK/dV column: 4 "
-                    "launches, tcgen05) on the same scored mask; FLOPs = 2.5 x the forward's",
+        "a3b_note": "lte_sparse_attn_backward (dQ with D_t, column work list, dK/dV window, "
+                    "dK/dV column: 4 launches, tcgen05) on the same scored mask; FLOPs = 2.5 x "
+                    "the forward's",
         "a7_gla_prefill_ms": t_gla, "a7_prefill_roofline": hbm(gla_bytes, t_gla),
         "a7_gla_decode_us": 1e3 * t_gla_dec, "a7_decode_roofline": hbm(gla_dec_bytes, t_gla_dec),
         "pair_prefill": {"value": DI.job_throughput(B * T, world, (t_gla + lte_prefill_ms) / 1e3),

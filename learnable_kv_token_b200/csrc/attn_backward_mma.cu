@@ -541,14 +541,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const Args a, int
 
 template <int D>
 cudaError_t launch(const Args& a, int B, bool dq_tc, DevError* err, cudaStream_t stream) {
-  const long long rows = (long long)B * a.T * a.Hq;
-  bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(rows, a.o, a.dO, a.T, a.Hq,
-                                                                       a.delta);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   if (dq_tc) {
+    // the tcgen05 dQ kernel forms D_t itself (it holds each row's dO and o) and
+    // writes it for the dK/dV passes
     if ((e = attn_backward_dq_tc(a, B, err, stream)) != cudaSuccess) return e;
   } else {
+    const long long rows = (long long)B * a.T * a.Hq;
+    bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(rows, a.o, a.dO, a.T, a.Hq,
+                                                                         a.delta);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t smem_dq = 2 * (size_t)kRows * D * 2 + 2 * 2 * (size_t)kKeys * D * 2;
     e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_dq);

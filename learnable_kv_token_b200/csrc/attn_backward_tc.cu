@@ -71,7 +71,9 @@ constexpr int kThreadsP = 384;
 constexpr int kStagesKP = 7, kStagesVP = 4;            // K and V rings
 constexpr uint32_t kKR = 0;                             // K stage s at 16 KiB s
 constexpr uint32_t kVR = kKR + kStagesKP * 16384;       // V stage s at 16 KiB s
-constexpr uint32_t kBar2 = kVR + kStagesVP * 16384;     // barriers
+constexpr uint32_t kOS = kVR + kStagesVP * 16384;       // o [128][128] bf16 (32 KiB), for D_t
+constexpr uint32_t kDP = kOS + 32768;                   // [2][128] fp32 partial sums of D_t
+constexpr uint32_t kBar2 = kDP + 2 * kRowsTc * 4;       // barriers
 constexpr int kSmemP = kBar2 + 512;
 constexpr uint32_t kColSP = 0, kColDPP = 128, kColDQP = 256, kColQP = 384, kColDOP = 448;
 constexpr int kQStage = 3;                              // Q, dO arrive in K stages 3..6
@@ -88,6 +90,7 @@ static_assert(kStagesKP * 16384 >= kRowsTc * HD * 4, "the K ring holds the dQ st
 
 __global__ void __launch_bounds__(kThreadsP, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_o,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
                  const bwd::Args a, DevError* err) {
@@ -173,10 +176,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // Q and dO into K-ring stages kQStage .. (free until the rows have moved them
     // into TMEM)
     if (elect_one()) {
-      mbar_expect_tx(bar(P_QF), 2 * kRowsTc * HD * 2);
+      mbar_expect_tx(bar(P_QF), 3 * kRowsTc * HD * 2);
       for (int hf = 0; hf < 2; ++hf) {
         tma_load_4d(sb + kQS + hf * (kRowsTc * 128), &tm_q, bar(P_QF), hf * 64, h * G, t0, b);
         tma_load_4d(sb + kQS + 32768u + hf * (kRowsTc * 128), &tm_do, bar(P_QF), hf * 64, h * G, t0, b);
+        tma_load_4d(sb + kOS + hf * (kRowsTc * 128), &tm_o, bar(P_QF), hf * 64, h * G, t0, b);
       }
     }
     __syncwarp();
@@ -278,33 +282,52 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int tt = t0 + row / G, gq = row % G;
     // Q and dO of this row, dims [64 kh, 64 kh + 64), from their 128-byte swizzled
-    // halves in shared memory (zeros past T, as the copy fills them) into TMEM
+    // halves in shared memory (zeros past T, as the copy fills them) into TMEM;
+    // with o, this half's part of D_t = <dO_t, o_t>
+    float* dpart = reinterpret_cast<float*>(sm + kDP);
     bool ok = __all_sync(0xffffffffu, mbar_wait(bar(P_QF), 0, abort_flag, err, 415));
-    if (ok) {
-      uint32_t rq[32], rd[32];
-      const uint8_t* qrow = sm + kQS + kh * (kRowsTc * 128) + row * 128;
+    {
+      float dsum = 0.f;
+      if (ok) {
+        uint32_t rq[32], rd[32];
+        const uint8_t* qrow = sm + kQS + kh * (kRowsTc * 128) + row * 128;
+        const uint8_t* orow = sm + kOS + kh * (kRowsTc * 128) + row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int off = (c ^ (row & 7)) << 4;
-        const uint4 vq = *reinterpret_cast<const uint4*>(qrow + off);
-        const uint4 vd = *reinterpret_cast<const uint4*>(qrow + 32768 + off);
-        rq[4 * c] = vq.x, rq[4 * c + 1] = vq.y, rq[4 * c + 2] = vq.z, rq[4 * c + 3] = vq.w;
-        rd[4 * c] = vd.x, rd[4 * c + 1] = vd.y, rd[4 * c + 2] = vd.z, rd[4 * c + 3] = vd.w;
+        for (int c = 0; c < 8; ++c) {
+          const int off = (c ^ (row & 7)) << 4;
+          const uint4 vq = *reinterpret_cast<const uint4*>(qrow + off);
+          const uint4 vd = *reinterpret_cast<const uint4*>(qrow + 32768 + off);
+          const uint4 vo = *reinterpret_cast<const uint4*>(orow + off);
+          rq[4 * c] = vq.x, rq[4 * c + 1] = vq.y, rq[4 * c + 2] = vq.z, rq[4 * c + 3] = vq.w;
+          rd[4 * c] = vd.x, rd[4 * c + 1] = vd.y, rd[4 * c + 2] = vd.z, rd[4 * c + 3] = vd.w;
+          const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 xo = *reinterpret_cast<const __nv_bfloat162*>(&ow[e]);
+            const __nv_bfloat162 xd = *reinterpret_cast<const __nv_bfloat162*>(&rd[4 * c + e]);
+            dsum = fmaf(__low2float(xo), __low2float(xd), dsum);
+            dsum = fmaf(__high2float(xo), __high2float(xd), dsum);
+          }
+        }
+        tmem_st32(lane_addr + kColQP + 32 * kh, rq);
+        tmem_st32(lane_addr + kColDOP + 32 * kh, rd);
+        tmem_wait_st();
       }
-      tmem_st32(lane_addr + kColQP + 32 * kh, rq);
-      tmem_st32(lane_addr + kColDOP + 32 * kh, rd);
-      tmem_wait_st();
+      dpart[kh * kRowsTc + row] = dsum;
     }
     tc_fence_before();
     mbar_arrive(bar(P_QT));                            // (also on a failed wait: never blocks the others)
+    bar_sync(1, 256);                                  // both halves of every D_t are in dpart
     int lo_r, hi_r;
     bwd::row_range(a, crow, tt, lo_r, hi_r);
     if (lowest) lo_r = 0;
+    // D_t for this row (written out once for the dK/dV passes) and the row's lse
     float lse2 = 0.f, dl = 0.f;
     if (tt < a.T) {
       const long long li = ((long long)b * a.Hq + h * G + gq) * a.T + tt;
       lse2 = a.lse[li] * 1.4426950408889634f;
-      dl = a.delta[li];
+      dl = dpart[row] + dpart[kRowsTc + row];
+      if (kh == 0) a.delta[li] = dl;
     }
     for (int j = 0; j < total && ok; ++j) {
       const int x = j & 1;
@@ -1057,14 +1080,15 @@ cudaError_t attn_backward_dkdv_tc(const bwd::Args& a, int B, DevError* err, cuda
 cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaStream_t stream) {
   using namespace bwdtc;
   const int TOK = kRowsTc / a.G;
-  // tensor maps of Q, dO, K, V and of the column segment (contiguous rows of 128
-  // bf16; 128-byte swizzle, 64-column boxes)
-  CUtensorMap mq, mdo, mk, mv, mkc, mvc;
+  // tensor maps of Q, dO, o, K, V and of the column segment (contiguous rows of
+  // 128 bf16; 128-byte swizzle, 64-column boxes)
+  CUtensorMap mq, mdo, mo, mk, mv, mkc, mvc;
   {
     const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)a.Hq, (cuuint64_t)a.T, (cuuint64_t)B};
     const cuuint64_t st[3] = {(cuuint64_t)HD * 2, (cuuint64_t)a.Hq * HD * 2, (cuuint64_t)a.T * a.Hq * HD * 2};
     const cuuint32_t box[4] = {64, (cuuint32_t)a.G, (cuuint32_t)TOK, 1};
-    if (!encode(&mq, a.q, 4, dims, st, box) || !encode(&mdo, a.dO, 4, dims, st, box))
+    if (!encode(&mq, a.q, 4, dims, st, box) || !encode(&mdo, a.dO, 4, dims, st, box) ||
+        !encode(&mo, a.o, 4, dims, st, box))
       return cudaErrorInvalidValue;
   }
   {
@@ -1087,7 +1111,7 @@ cudaError_t attn_backward_dq_tc(const bwd::Args& a, int B, DevError* err, cudaSt
                                        kSmemP);
   if (e != cudaSuccess) return e;
   const int n_tiles = (a.T + TOK - 1) / TOK;
-  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsP, kSmemP, stream>>>(mq, mdo, mk, mv, mkc, mvc, a, err);
+  bwd_dq_tc_kernel<<<dim3(n_tiles, a.Hkv, B), kThreadsP, kSmemP, stream>>>(mq, mdo, mo, mk, mv, mkc, mvc, a, err);
   return cudaGetLastError();
 }
 
