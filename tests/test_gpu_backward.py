@@ -54,6 +54,10 @@ CASES = [
     (1, 300, 16, 1, 128, 4, 48, 12, "recent", 0.5),     # G = 16 on the tcgen05 kernels
     (1, 260, 16, 2, 128, 2, 40, 9, "first", 0.4),       # G = 8
     (2, 190, 4, 2, 128, 1, 30, 6, "lowest", 16),        # G = 2, lowest-score policy
+    # long enough that a column tile's attending rows exceed one work item of the
+    # tcgen05 column pass (several CTAs add into the same slots) under each policy
+    (1, 2048, 8, 2, 128, 4, 256, 48, "first", 0.5),
+    (1, 2048, 8, 2, 128, 4, 256, 48, "lowest", 8),
 ]
 POLICY = {"recent": (0, O.CAP_RECENT), "first": (1, O.CAP_FIRST), "lowest": (2, O.CAP_LOWEST)}
 
