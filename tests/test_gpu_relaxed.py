@@ -31,6 +31,9 @@ CASES = [
     (1, 500, 16, 4, 4, 64, 40, "lowest", 8),
     (1, 300, 8, 8, 0, 16, 3, "first", 0),
     (1, 260, 16, 1, 2, 40, 9, "recent", 16),
+    # the first C retained slots are attended by every later row: their rows span
+    # several column work items, whose dK, dV and dL/dr adds meet in the same slots
+    (1, 2048, 8, 2, 4, 256, 48, "first", 0),
 ]
 
 
