@@ -223,3 +223,20 @@ def test_golden_fig2_setting():
     for t, S in enumerate(gold["sets"]):
         assert O.attended_set(t, m, s, w, C) == S
         assert S == [j for j in range(len(m)) if brute_member(j, t, m, s, w, C)]
+
+
+def test_worked_example_sets_by_hand():
+    """A hand-derived example (tests/golden/worked_example_sets.json, with its
+    derivation): s = 1, w = 3, C = 2 over ten tokens, for all three cap
+    policies.  The expected sets were worked out from the LTE paper's Fig. 2
+    caption (sinks, window, at most C retained KVs per head), not by the oracle,
+    so this pins the oracle's set logic independently of its own code."""
+    with open(os.path.join(GOLDEN, "worked_example_sets.json")) as f:
+        gold = json.load(f)
+    s, w, C = gold["sink"], gold["window"], gold["cap"]
+    m = O.fed_mask(np.array(gold["mask"], np.uint8), s)
+    r = np.array(gold["scores"], np.float64)
+    for policy, sets in gold["sets"].items():
+        for t, expect in enumerate(sets):
+            got = O.attended_set(t, m, s, w, C, policy, r if policy == O.CAP_LOWEST else None)
+            assert got == expect, f"{policy} t={t}: {got} != {expect}"
