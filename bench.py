@@ -13,8 +13,8 @@ Also reported on the same JSON line:
   e2e          the same step from pinned host buffers (H2D of q, k, v, mask
                and D2H of o inside the timed region);
   decode       the decode workload (4096-token prompt, B=32, CNN scored live,
-               deferred batch 64): per-layer decode steps rotating over 4
-               layer caches (> L2), captured in a CUDA graph;
+               deferred batch 64): its 512 generated tokens, each fed once
+               to each of 4 layer caches (> L2), in one CUDA graph;
   cpu_baseline the CPU oracle on a bounded sample of the same workload.
 `--impl reference` times the CPU oracle alone (the reference arm).
 """
@@ -349,12 +349,19 @@ def prefill_bench(args, rank, world, device):
     }
 
 
-def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
+def decode_bench(args, rank, world, device, n_layers=4):
+    """Decode after the 4096-token prompt: each of `n_layers` layer caches (together
+    larger than L2) is initialised from the prompt's prefill, then fed the
+    workload's generated tokens, one per step, rotating over the layers, in one
+    CUDA graph.  The graph is replayed once to warm up; the caches are then put
+    back to their post-prompt state and the timed replay feeds every generated
+    token exactly once per layer cache, at positions T0 .. T0 + S - 1."""
     from learnable_kv_token_b200 import layer
     wl = LI.WORKLOADS["decode"]
     inp = LI.lte_inputs(wl.with_(seed=DI.shard_seed(wl.seed, rank)))
     q, k, v, cnn = inp["q"], inp["k"], inp["v"], inp["cnn"]
     B, T0, Hq, Hkv, D = wl.B, wl.T, wl.Hq, wl.Hkv, wl.D
+    S = wl.decode_steps
     p = layer.LayerParams(sink=wl.sink, window=wl.window, cap=wl.cap, tau=wl.tau)
     qd, kd, vd = (x.to(device) for x in (q, k, v))
     cd = tuple(x.to(device) for x in cnn)
@@ -370,29 +377,37 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
         cache = layer.DecodeCache(B, Hkv, D, torch.bfloat16, wl.sink, wl.window, wl.cap, device)
         cache.init_from_prefill(dims, kp, vp, out, T0)
         decs.append(layer.Decoder(dims, cd, p.past1, p.past2, cache, wl.score_batch, device))
-    del out
+    del out, qp, kp, vp
+    torch.cuda.synchronize()
+    snaps = [d.cache.snapshot() for d in decs]
+
+    def rewind():
+        torch.cuda.synchronize()
+        for d, sn in zip(decs, snaps):
+            d.cache.restore(sn)
+        torch.cuda.synchronize()
+
     qs = qd[:, T0:].permute(1, 0, 2, 3).contiguous()
     ks = kd[:, T0:].permute(1, 0, 2, 3).contiguous()
     vs = vd[:, T0:].permute(1, 0, 2, 3).contiguous()
+    del qd, kd, vd
+    assert qs.shape[0] == S
     stream = torch.cuda.Stream(device)
     # warm-up: a few eager steps per layer
     with torch.cuda.stream(stream):
         for i in range(3):
             for d in decs:
                 d.step(qs[i], ks[i], vs[i], stream=stream)
-    stream.synchronize()
+    rewind()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
-            for i in range(steps_per_layer):
+            for t in range(S):
                 for d in decs:
-                    t = 3 + i
                     d.step(qs[t], ks[t], vs[t], stream=stream)
     with torch.cuda.stream(stream):    # replay() launches on the current stream
         graph.replay()                 # warm replay
-    torch.cuda.synchronize()
-    ret = decs[0].cache.ret_total.clone()
-    t_meta = int(decs[0].cache.meta[0])
+    rewind()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     DI.barrier(world)
     torch.cuda.synchronize()
@@ -401,37 +416,51 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
         graph.replay()
         e1.record(stream)
     torch.cuda.synchronize()
-    n_steps = steps_per_layer * n_layers
+    n_steps = S * n_layers
     ms_step = DI.max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
+    assert all(d_.device_error() == (0, 0) for d_ in decs)
+    ret = decs[0].cache.ret_total.clone()
+    t_meta = int(decs[0].cache.meta[0])
+    assert t_meta == T0 + S
     del graph
     # the laLTE pair step: one gated linear-attention layer step (16 heads,
     # dk = dv = 128, its own fp32 state per layer) followed by the LTE layer
-    # step, over the same 4 layers, in one CUDA graph.  The GLA step is
-    # launched with programmatic dependent launch, so each kernel's CTAs are
-    # resident and through their prologue when its predecessor ends.
+    # step, over the same 4 layers, in one CUDA graph, for the hybrid
+    # workload's generated tokens (each fed once per layer in the timed
+    # replay, the caches rewound to the prompt and the states zeroed before it).
+    # The GLA step is launched with programmatic dependent launch, so each
+    # kernel's CTAs are resident and through their prologue when its
+    # predecessor ends.
     from learnable_kv_token_b200 import lte as L
+    S_pair = LI.WORKLOADS["hybrid"].decode_steps
     H_g, dk_g = 16, 128
-    gq, gk, gv, ga = (x[:, 0].contiguous().to(device) for x in
-                      LI.gla_inputs(B, 1, H_g, dk_g, dk_g, LI.generator(wl.seed + 2000)))
-    go = torch.empty_like(gv)
+    gq, gk, gv, ga = (x.transpose(0, 1).contiguous().to(device) for x in
+                      LI.gla_inputs(B, S_pair, H_g, dk_g, dk_g, LI.generator(wl.seed + 2000)))
+    go = torch.empty_like(gv[0])
     states = [torch.zeros(B, H_g, dk_g, dk_g, dtype=torch.float32, device=device)
               for _ in range(n_layers)]
+
+    def rewind_pair():
+        rewind()
+        for st_ in states:
+            st_.zero_()
+        torch.cuda.synchronize()
+
     with torch.cuda.stream(stream):
         for d_, st_ in zip(decs, states):
-            L.lte_gla_decode_step(gq, gk, gv, ga, go, st_, stream)
+            L.lte_gla_decode_step(gq[0], gk[0], gv[0], ga[0], go, st_, stream)
             d_.step(qs[0], ks[0], vs[0], stream=stream)
-    stream.synchronize()
+    rewind_pair()
     pgraph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(pgraph, stream=stream):
-            for i in range(steps_per_layer):
+            for t in range(S_pair):
                 for d_, st_ in zip(decs, states):
-                    t = 3 + i
-                    L.lte_gla_decode_step(gq, gk, gv, ga, go, st_, stream)
+                    L.lte_gla_decode_step(gq[t], gk[t], gv[t], ga[t], go, st_, stream)
                     d_.step(qs[t], ks[t], vs[t], stream=stream)
     with torch.cuda.stream(stream):
         pgraph.replay()
-    torch.cuda.synchronize()
+    rewind_pair()
     DI.barrier(world)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -439,9 +468,9 @@ def decode_bench(args, rank, world, device, n_layers=4, steps_per_layer=64):
         pgraph.replay()
         e1.record(stream)
     torch.cuda.synchronize()
-    pair_ms = DI.max_over_ranks(e0.elapsed_time(e1) / n_steps, world, device)
+    pair_ms = DI.max_over_ranks(e0.elapsed_time(e1) / (S_pair * n_layers), world, device)
     assert all(d_.device_error() == (0, 0) for d_ in decs)
-    del pgraph, states
+    del pgraph, states, snaps
     gla_bytes = 2 * B * H_g * dk_g * dk_g * 4 + B * H_g * dk_g * (4 * 2 + 4)
     # algorithmic bytes of one layer step (steady state)
     n_keys = (min(wl.window, t_meta) + wl.sink + torch.clamp(ret, max=wl.cap)).sum().item()
@@ -675,7 +704,8 @@ def rows_bench(args, rank, world, device, dec):
                          "roofline": hbm(dec["pair_bytes"], dec["pair_ms"]),
                          "sum_of_separate_steps_us": 1e3 * (t_gla_dec + dec["ms_step"]),
                          "note": "GLA step then LTE step per layer, 4 layers rotated, one CUDA "
-                                 "graph of 256 pair steps, programmatic dependent launch"}),
+                                 "graph of 256 generated tokens x 4 layers, each token fed once, "
+                                 "programmatic dependent launch"}),
         "launches": 2 + 5 * 3 + 5 + 50 + 4 * 7 + 4 * 7,
     }
 
@@ -764,8 +794,9 @@ def main():
             gbs = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
             line["decode"] = {
                 "workload": "decode B=32, 4096-token prompt, Hq=16 Hkv=4 D=128 bf16 s=4 w=512 "
-                            "C=512, CNN scored live (tau 0.5, deferred batch 64); per-layer steps "
-                            "over 4 layer caches (> L2) in one CUDA graph",
+                            "C=512, CNN scored live (tau 0.5, deferred batch 64); the 512 "
+                            "generated tokens, each fed once to each of 4 layer caches (> L2), "
+                            "2048 steps in one CUDA graph",
                 "value": DI.job_throughput(dec["B"], world, dec["ms_step"] / 1e3), "unit": "tokens/s",
                 "us_per_layer_step": 1e3 * dec["ms_step"],
                 "roofline": {"bound": "hbm",

@@ -201,6 +201,21 @@ class DecodeCache:
         L.lte_cache_init_from_prefill(dims, self.struct, k, v, out.r, out.idx, out.cnt, T_prompt,
                                       out.n_scored, stream, death=out.death)
 
+    def _state(self):
+        return (self.k, self.v, self.pos, self.win_r, self.ret_total, self.meta, self.ret_r)
+
+    def snapshot(self):
+        """Device copies of every tensor the decode step reads or writes (the
+        step index and its ticket live in `meta`), for `restore`."""
+        return tuple(t.clone() for t in self._state())
+
+    def restore(self, snap):
+        """Put the cache back to a `snapshot` in place, on the current stream
+        (same buffers, so a CUDA graph captured over this cache stays valid).
+        No decode step of this cache may be in flight."""
+        for t, s in zip(self._state(), snap):
+            t.copy_(s)
+
     def retained_positions(self):
         """Sorted retained positions per unit (host copy, for checks)."""
         w, s = self.window, self.sink
