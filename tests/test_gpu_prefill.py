@@ -86,26 +86,28 @@ def test_score_causal_variant(L):
             np.testing.assert_allclose(f64(r[b, h]), ro, atol=R_TOL, rtol=0)
 
 
-@pytest.mark.parametrize("B,T,Hkv,D,c_hid,past1,past2", [
-    (3, 1500, 2, 64, 32, 2, 1),       # head dim 64, several sequences and heads
-    (2, 1000, 4, 128, 20, 4, 2),      # fewer hidden channels than columns per tap; causal taps
-    (1, 40, 1, 128, 32, 2, 1),        # a sequence shorter than one tile
+@pytest.mark.parametrize("B,T,Hkv,D,c_hid,past1,past2,k1,k2", [
+    (3, 1500, 2, 64, 32, 2, 1, 5, 3),     # head dim 64, several sequences and heads
+    (2, 1000, 4, 128, 20, 4, 2, 5, 3),    # fewer hidden channels than columns per tap; causal taps
+    (1, 40, 1, 128, 32, 2, 1, 5, 3),      # a sequence shorter than one tile (one CTA of the pair idle)
+    (2, 700, 2, 128, 32, 4, 1, 8, 3),     # the widest first layer: 256 output columns
+    (3, 900, 3, 64, 16, 1, 2, 3, 5),      # a narrow first layer, a wide second, an odd tile count
 ])
-def test_score_tensor_core_shapes(L, B, T, Hkv, D, c_hid, past1, past2):
+def test_score_tensor_core_shapes(L, B, T, Hkv, D, c_hid, past1, past2, k1, k2):
     """bf16 scores from the tcgen05 scorer, with k and v strided views into one
     packed [B, T, Hkv, 2, D] tensor, against the oracle; a split launch gives
     the same values bit for bit."""
     g = LI.generator(23)
     kv = (torch.randn(B, T, Hkv, 2, D, generator=g) / math.sqrt(D)).to(torch.bfloat16)
     k, v = kv[:, :, :, 0], kv[:, :, :, 1]
-    w1, _, w2, _ = LI.cnn_weights(Hkv, D, c_hid, 5, 3, g, 0.05)
+    w1, _, w2, _ = LI.cnn_weights(Hkv, D, c_hid, k1, k2, g, 0.05)
     cnn = (w1, 0.1 * torch.randn(Hkv, c_hid, generator=g), w2, 0.1 * torch.randn(Hkv, generator=g))
     kvd = kv.cuda()
     kd, vd = kvd[:, :, :, 0], kvd[:, :, :, 1]
     cd = _dev(*cnn)
     dims = L.make_dims(B, T, Hkv, Hkv, D, 4, 64, 32, 0.5, 1.0 / math.sqrt(D), torch.bfloat16)
     c, _keep = L.make_cnn(*cd, past1, past2)
-    F = (5 - 1 - past1) + (3 - 1 - past2)
+    F = (k1 - 1 - past1) + (k2 - 1 - past2)
     n = T - F
     r = torch.full((B, Hkv, T), float("nan"), device="cuda")
     m = torch.zeros(B, Hkv, T, dtype=torch.uint8, device="cuda")
