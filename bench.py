@@ -680,7 +680,8 @@ def rows_bench(args, rank, world, device, dec):
         "workload": f"hybrid B={B} T=4096 (prompt) Hq=16 Hkv=4 D=128 bf16 s=4 w=512 C=512, CNN "
                     "32ch k5/k3 scored live, tau 0.5; GLA 16 heads dk=dv=128, chunk 64",
         "a1_score_ms": t_score, "a1_roofline": tensor(score_flops, t_score),
-        "a1_bytes_rate": hbm(score_bytes, t_score),
+        "a1_bytes_rate": dict(hbm(score_bytes, t_score), traffic=traffic_from_profiles(
+            "learnable_kv_token_b200/csrc/score_tcgen05.cu", B * Hkv * n_scored)),
         "a2_compact_ms": t_compact, "a2_roofline": hbm(compact_bytes, t_compact),
         "a3_attn_ms": t_attn, "a3_roofline": tensor(attn_flops, t_attn),
         "a3_retention_rate": float(mask[..., wl.sink:n_scored].mean()),
