@@ -159,3 +159,32 @@ def test_kernel_choice_is_reported(lib):
     assert f.lte_noalloc_read_device_error(None, None, None) == 1
     assert f.lte_sparse_attn_prefill_kernel(C.byref(mk(128, L.LTE_BF16)), None, None, None,
                                             None) == 1
+
+
+def test_decode_cache_snapshot_restore_on_host(lib):
+    """DecodeCache.snapshot / restore copy every tensor the decode step reads or
+    writes and put them back in place (same buffers, so the cache struct a
+    captured graph holds stays valid).  Host tensors, no GPU needed."""
+    import torch
+    from learnable_kv_token_b200 import layer
+    c = layer.DecodeCache(2, 3, 16, torch.float32, sink=2, window=8, cap=4, device="cpu")
+    g = torch.Generator().manual_seed(3)
+    for t in c._state():
+        if t.dtype.is_floating_point:
+            t.copy_(torch.randn(t.shape, generator=g))
+        else:
+            t.copy_(torch.randint(-5, 50, t.shape, generator=g, dtype=t.dtype))
+    ptrs = [t.data_ptr() for t in c._state()]
+    snap = c.snapshot()
+    before = [t.clone() for t in c._state()]
+    assert all(s.data_ptr() != p for s, p in zip(snap, ptrs))      # copies, not views
+    for t in c._state():
+        t.fill_(7)
+    c.restore(snap)
+    assert [t.data_ptr() for t in c._state()] == ptrs
+    for t, b in zip(c._state(), before):
+        assert torch.equal(t, b)
+    # the state covers the struct the library sees: every pointer it holds is one of them
+    held = {c.struct.k, c.struct.v, c.struct.pos, c.struct.win_r, c.struct.ret_total,
+            c.struct.meta, c.struct.ret_r}
+    assert held == set(ptrs)
