@@ -31,22 +31,25 @@
 // x rows as A and holds half of the weight rows (output columns) as B, and
 // each CTA's TMEM receives its own rows.  So each SM keeps only half of the
 // head's bf16 hi/lo weights resident (converted once), which leaves room for
-// an x ring two tiles deep.  Roles per CTA (384 threads):
+// an x ring two tiles deep.  Roles per CTA (448 threads):
 //   warp 0     TMA producer: one 64-channel chunk of this CTA's tile's x rows
 //              (four boxes of 32 rows x 128 B, 128-byte swizzle; rows outside
 //              the tokens read as zero) per stage; the bytes of both CTAs'
 //              copies of a stage complete on the leader's barrier;
 //   warp 1     TMEM owner in both CTAs; in the leader, the MMA issuer (one
 //              elected lane): per chunk, four K-steps of 16 channels, each an
-//              (hi, lo) pair of M256 x N x K16 MMAs into one of two TMEM
-//              accumulators (N = 32 * k1), with every commit signalled to both
-//              CTAs;
-//   warps 1-11 convert this CTA's half of the head's weights first (warp 0 is
+//              (hi, lo) pair of M256 x N x K16 MMAs into one of the TMEM
+//              accumulators (N = 32 * k1; three of them, N columns apart, when
+//              they fit in 512 columns, else two), with every commit signalled
+//              to both CTAs;
+//   warps 1-13 convert this CTA's half of the head's weights first (warp 0 is
 //              already loading);
-//   warps 4-7, 8-11  two epilogue groups, one per accumulator (even and odd
-//              pair-tiles), one lane quadrant per warp: tap sums by shuffles,
-//              SiLU, layer 2, sigmoid, r and the mask.  The accumulator is
-//              released to the leader as soon as its columns are in registers.
+//   warps 2-5, 6-9, 10-13  the epilogue groups, one per accumulator (pair-
+//              tiles i with i mod 3, or mod 2, equal to the group), one lane
+//              quadrant per warp (warp w reads quadrant w mod 4): tap sums by
+//              shuffles, SiLU, layer 2, sigmoid, r and the mask.  The
+//              accumulator goes back to the leader as soon as its columns are
+//              in registers.
 // Every mbarrier wait is bounded.  A CTA that gives up writes NaN scores
 // (mask 0) for the tokens it did not score, so a failure is visible in r.
 // The two CTAs meet at a cluster barrier after setting up their barriers and
