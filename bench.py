@@ -65,7 +65,8 @@ def attended_pairs(mask: np.ndarray, sink: int, window: int, cap: int) -> np.nda
     win = np.minimum(t + 1, window)
     sinks = np.clip(t - window + 1, 0, sink)
     n = np.zeros_like(cnt)
-    n[..., window:] = cnt[..., :T - window]
+    if window < T:                       # retained tokens that have left the window
+        n[..., window:] = cnt[..., :T - window]
     return win[None, None] + sinks[None, None] + np.minimum(n, cap)
 
 
