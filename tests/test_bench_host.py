@@ -50,3 +50,20 @@ def test_attended_pairs_full_causal_when_everything_is_kept(bench):
     mask = np.ones((1, 2, T), np.uint8)
     got = bench.attended_pairs(mask, 4, 16, T)
     np.testing.assert_array_equal(got[0, 0], np.arange(1, T + 1))
+
+
+def test_clock_summary_reads_nvidia_smi_rows(bench):
+    """The clocks object of the bench line: median SM clock under load, the
+    highest max clock seen, and only reasons reported Active."""
+    c = bench.Clocks(0)
+    c.out = "\n".join([
+        "0, 1965, 1965, 701.2, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 998.0, Not Active, Not Active, Not Active, Active",
+        "0, 1900, 1965, 900.5, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 0, Not Active, Not Active, Not Active, Not Active",
+    ])
+    s = c.summary()
+    assert s == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c.out = ""
+    assert c.summary()["samples"] == 0
